@@ -1,0 +1,303 @@
+/*
+ * rodref.c -- plain, slow, obviously-correct CPU oracle for the Rodimus+ token mixers.
+ *
+ * TEST INFRASTRUCTURE ONLY. Nothing on the product path may link, load or call this
+ * library: only the tests, the smoke check and the benchmark's CPU-baseline leg use it.
+ * It shares no code, header, table or helper with the CUDA library.
+ *
+ * Everything is computed in IEEE double precision with plain loops, in the order the
+ * definitions are written. Inputs arrive as float arrays: the GPU path receives bf16 or
+ * fp32 values, and every bf16 and fp32 value is exactly representable as a float, so the
+ * oracle sees exactly the numbers the kernels see and widens them to double on use.
+ * Work is split only across independent units ((batch, head) pairs for the recurrence,
+ * output rows for attention) with POSIX threads; each unit is computed sequentially.
+ *
+ * Sources (web pages; cited by title and section):
+ *  [CodeFuse]  "ICLR 2025 | Rodimus*: a hybrid attention mechanism balancing performance and
+ *              efficiency" (CodeFuse article): the Rodimus block compresses the history into a
+ *              fixed-size hidden state, updated recurrently at inference (O(1) space); SKA shares
+ *              one key matrix across all heads and keeps per-head values (Fig. 4 and the SKA
+ *              paragraph); Rodimus+ uses SKA inside sliding-window attention (SW-SKA).
+ *  [Setup]     "Rodimus* ... what problem does it solve" setup/benchmark blog, §3 (module
+ *              config): the sliding window only looks at the most recent 4096 tokens; keys are
+ *              shared across heads and values are kept per head.
+ *  [SALA]      sparse + linear attention blog: §2.1 sliding-window attention (each query looks
+ *              only at recent keys), §2.2 linear attention state O_i = phi(q_i) * sum_j phi(k_j)^T v_j
+ *              with a d x d state, §3.3 ring-buffer window cache and in-place state update at
+ *              decode, §4.3 third tip (a decay factor makes old state weights fall exponentially).
+ *
+ * Readings taken where the pages are silent or garbled (the DDTS gate equation in [CodeFuse]
+ * is stripped from the extracted text):
+ *  - the gates g_t are inputs, one per key channel, and decay the ROWS of the d_k x d_v state:
+ *        S_t = diag(g_t) S_{t-1} + k_t^T v_t,   o_t = q_t S_t   (readout after the update);
+ *    no scale and no normaliser are applied to the recurrence output.
+ *  - the window of query t holds W keys including t itself: j in [t-W+1, t], clipped at 0.
+ *    W = 1 then gives o_t = v_t and W >= T gives full causal attention.
+ *  - softmax attention uses o = sum_j p_j v_j / sum_j p_j with p_j = exp(s_j - max s).
+ */
+#include <math.h>
+#include <pthread.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+
+#define RODREF_OK 0
+#define RODREF_EINVAL (-1)
+#define RODREF_ENOMEM (-2)
+
+/* ------------------------------------------------------------------------------------------
+ * tiny work-splitting helper: run fn(arg, unit) for unit in [0, n_units) on nthreads threads
+ * ---------------------------------------------------------------------------------------- */
+typedef void (*unit_fn)(const void* arg, int64_t unit);
+
+typedef struct {
+    unit_fn fn;
+    const void* arg;
+    int64_t n_units;
+    int tid;
+    int nthreads;
+} worker_t;
+
+static void* worker_main(void* p) {
+    worker_t* w = (worker_t*)p;
+    for (int64_t u = w->tid; u < w->n_units; u += w->nthreads) w->fn(w->arg, u);
+    return NULL;
+}
+
+static int run_units(unit_fn fn, const void* arg, int64_t n_units, int nthreads) {
+    if (nthreads < 1) nthreads = 1;
+    if (nthreads > 256) nthreads = 256;
+    if (n_units < nthreads) nthreads = (int)(n_units > 0 ? n_units : 1);
+    if (nthreads == 1) {
+        for (int64_t u = 0; u < n_units; ++u) fn(arg, u);
+        return RODREF_OK;
+    }
+    pthread_t th[256];
+    worker_t w[256];
+    int started = 0;
+    for (int i = 0; i < nthreads; ++i) {
+        w[i].fn = fn; w[i].arg = arg; w[i].n_units = n_units; w[i].tid = i; w[i].nthreads = nthreads;
+        if (pthread_create(&th[i], NULL, worker_main, &w[i]) != 0) break;
+        ++started;
+    }
+    for (int i = 0; i < started; ++i) pthread_join(th[i], NULL);
+    /* units a failed thread would have taken are done here, sequentially */
+    for (int i = started; i < nthreads; ++i) worker_main(&w[i]);
+    return RODREF_OK;
+}
+
+/* ------------------------------------------------------------------------------------------
+ * Gated linear recurrence (the Rodimus semantic-compression state) -- [CodeFuse] Rodimus block
+ * (recurrent inference form keeps only a fixed-size state); [SALA] §2.2 (state = sum of k^T v,
+ * readout q * state) and §4.3 tip 3 (per-step decay of the old state).
+ *
+ * One step for one (batch, head):
+ *     S[c][j] <- g[c] * S[c][j] + k[c] * v[j]        c < dk, j < dv
+ *     o[j]     = sum_c q[c] * S[c][j]                 (S after the update)
+ * ---------------------------------------------------------------------------------------- */
+static void gla_step(const float* q, const float* k, const float* v, const float* g,
+                     double* S, double* o, int64_t dk, int64_t dv) {
+    for (int64_t c = 0; c < dk; ++c) {
+        const double gc = (double)g[c];
+        const double kc = (double)k[c];
+        double* row = S + c * dv;
+        for (int64_t j = 0; j < dv; ++j) row[j] = gc * row[j] + kc * (double)v[j];
+    }
+    for (int64_t j = 0; j < dv; ++j) {
+        double acc = 0.0;
+        for (int64_t c = 0; c < dk; ++c) acc += (double)q[c] * S[c * dv + j];
+        o[j] = acc;
+    }
+}
+
+typedef struct {
+    const float *q, *k, *v, *g;
+    double *state, *o;
+    int64_t T, dk, dv;
+} gla_args_t;
+
+/* one unit = one (batch, head) pair, walked sequentially in t */
+static void gla_unit(const void* p, int64_t bh) {
+    const gla_args_t* a = (const gla_args_t*)p;
+    const int64_t T = a->T, dk = a->dk, dv = a->dv;
+    double* S = a->state + bh * dk * dv;
+    for (int64_t t = 0; t < T; ++t) {
+        const int64_t tk = (bh * T + t) * dk, tv = (bh * T + t) * dv;
+        gla_step(a->q + tk, a->k + tk, a->v + tv, a->g + tk, S, a->o + tv, dk, dv);
+    }
+}
+
+/*
+ * q, k, g: [B,H,T,dk]; v: [B,H,T,dv] (row-major, contiguous).
+ * state: [B,H,dk,dv], read as the initial state and overwritten with the final state.
+ * o: [B,H,T,dv].
+ */
+int rodref_gla_prefill(const float* q, const float* k, const float* v, const float* g,
+                       double* state, double* o, int64_t B, int64_t H, int64_t T,
+                       int64_t dk, int64_t dv, int nthreads) {
+    if (!q || !k || !v || !g || !state || !o) return RODREF_EINVAL;
+    if (B < 0 || H < 0 || T < 0 || dk < 1 || dv < 1) return RODREF_EINVAL;
+    gla_args_t a = {q, k, v, g, state, o, T, dk, dv};
+    return run_units(gla_unit, &a, B * H, nthreads);
+}
+
+/*
+ * One decode step for N sequences: q, k, g: [N,H,dk]; v: [N,H,dv];
+ * state [N,H,dk,dv] updated in place; o: [N,H,dv]. Identical to a prefill with T = 1.
+ */
+int rodref_gla_decode_step(const float* q, const float* k, const float* v, const float* g,
+                           double* state, double* o, int64_t N, int64_t H, int64_t dk,
+                           int64_t dv, int nthreads) {
+    return rodref_gla_prefill(q, k, v, g, state, o, N, H, 1, dk, dv, nthreads);
+}
+
+/* ------------------------------------------------------------------------------------------
+ * Sliding-window shared-key softmax attention (SW-SKA) -- [CodeFuse] Fig. 4 / SKA paragraph
+ * (one K for all heads, per-head V), [Setup] §3 (window = most recent W tokens), [SALA] §2.1.
+ *
+ * For query t of head h in batch b, with window J_t = [max(0, t-W+1), t]:
+ *     s_j = scale * sum_c q[b,h,t,c] * k[b,j,c]
+ *     p_j = exp(s_j - max_{j' in J_t} s_j')
+ *     o[b,h,t,:] = sum_j p_j v[b,h,j,:] / sum_j p_j
+ * ---------------------------------------------------------------------------------------- */
+static void softmax_row(const float* qrow, const float* kbase, const float* vbase,
+                        int64_t j0, int64_t j1, int64_t dk, int64_t dv, double scale,
+                        double* s, double* out) {
+    /* kbase row j is kbase + j*dk; vbase row j is vbase + j*dv; keys j0..j1 inclusive */
+    double m = -INFINITY;
+    for (int64_t j = j0; j <= j1; ++j) {
+        double acc = 0.0;
+        const float* kr = kbase + j * dk;
+        for (int64_t c = 0; c < dk; ++c) acc += (double)qrow[c] * (double)kr[c];
+        s[j - j0] = scale * acc;
+        if (s[j - j0] > m) m = s[j - j0];
+    }
+    double l = 0.0;
+    for (int64_t i = 0; i < dv; ++i) out[i] = 0.0;
+    for (int64_t j = j0; j <= j1; ++j) {
+        const double p = exp(s[j - j0] - m);
+        l += p;
+        const float* vr = vbase + j * dv;
+        for (int64_t i = 0; i < dv; ++i) out[i] += p * (double)vr[i];
+    }
+    for (int64_t i = 0; i < dv; ++i) out[i] /= l;
+}
+
+typedef struct {
+    const float *q, *k, *v;
+    double* o;
+    int64_t B, H, T, dk, dv, W;
+    double scale;
+    const int64_t* rows;
+} ska_args_t;
+
+static void ska_unit(const void* p, int64_t r) {
+    const ska_args_t* a = (const ska_args_t*)p;
+    const int64_t flat = a->rows ? a->rows[r] : r; /* ((b*H + h)*T + t) */
+    const int64_t t = flat % a->T;
+    const int64_t bh = flat / a->T;
+    const int64_t b = bh / a->H;
+    int64_t j0 = t - a->W + 1;
+    if (j0 < 0) j0 = 0;
+    double* s = (double*)malloc((size_t)(t - j0 + 1) * sizeof(double));
+    if (!s) { for (int64_t i = 0; i < a->dv; ++i) a->o[r * a->dv + i] = NAN; return; }
+    softmax_row(a->q + flat * a->dk, a->k + b * a->T * a->dk, a->v + bh * a->T * a->dv,
+                j0, t, a->dk, a->dv, a->scale, s, a->o + r * a->dv);
+    free(s);
+}
+
+/*
+ * q: [B,H,T,dk]; k: [B,T,dk] (shared by the H heads); v: [B,H,T,dv].
+ * rows == NULL: o is [B,H,T,dv] (every output row).
+ * rows != NULL: o is [n_rows, dv]; row r is output row rows[r] = (b*H + h)*T + t.
+ */
+int rodref_swska_prefill(const float* q, const float* k, const float* v, double* o,
+                         int64_t B, int64_t H, int64_t T, int64_t dk, int64_t dv, int64_t W,
+                         double scale, const int64_t* rows, int64_t n_rows, int nthreads) {
+    if (!q || !k || !v || !o) return RODREF_EINVAL;
+    if (B < 0 || H < 0 || T < 0 || dk < 1 || dv < 1 || W < 1) return RODREF_EINVAL;
+    const int64_t total = B * H * T;
+    if (rows) {
+        for (int64_t r = 0; r < n_rows; ++r)
+            if (rows[r] < 0 || rows[r] >= total) return RODREF_EINVAL;
+    } else {
+        n_rows = total;
+    }
+    ska_args_t a = {q, k, v, o, B, H, T, dk, dv, W, scale, rows};
+    return run_units(ska_unit, &a, n_rows, nthreads);
+}
+
+/*
+ * SW-SKA decode with a ring-buffer window cache -- [SALA] §3.3 (self-made circular buffer,
+ * window rolls at every decode step), [CodeFuse] SKA (one shared K cache per sequence).
+ *
+ * For each sequence n with new position P = pos[n]:
+ *   1. write the new token into slot P mod W:  k_cache[n, P mod W, :] = k_new[n, :],
+ *      v_cache[n, h, P mod W, :] = v_new[n, h, :] for every head h;
+ *   2. attend over the tokens at positions p = max(0, P-W+1) .. P, whose keys sit in
+ *      slot p mod W, with the same softmax as above.
+ * q: [N,H,dk]; k_new: [N,dk]; v_new: [N,H,dv]; k_cache: [N,W,dk]; v_cache: [N,H,W,dv];
+ * o: [N,H,dv]. The caches are updated in place.
+ */
+typedef struct {
+    const float *q, *k_new, *v_new;
+    float *k_cache, *v_cache;
+    const int64_t* pos;
+    double* o;
+    int64_t H, dk, dv, W;
+    double scale;
+} ska_dec_args_t;
+
+static void ska_dec_unit(const void* p, int64_t nh) {
+    const ska_dec_args_t* a = (const ska_dec_args_t*)p;
+    const int64_t n = nh / a->H, h = nh % a->H;
+    const int64_t P = a->pos[n];
+    const int64_t p0 = P - a->W + 1 > 0 ? P - a->W + 1 : 0;
+    const int64_t cnt = P - p0 + 1;
+    const float* kc = a->k_cache + n * a->W * a->dk;
+    const float* vc = a->v_cache + (n * a->H + h) * a->W * a->dv;
+    const float* qr = a->q + nh * a->dk;
+    double* out = a->o + nh * a->dv;
+    double* s = (double*)malloc((size_t)cnt * sizeof(double));
+    if (!s) { for (int64_t i = 0; i < a->dv; ++i) out[i] = NAN; return; }
+    double m = -INFINITY;
+    for (int64_t pp = p0; pp <= P; ++pp) {
+        const float* kr = kc + (pp % a->W) * a->dk;
+        double acc = 0.0;
+        for (int64_t c = 0; c < a->dk; ++c) acc += (double)qr[c] * (double)kr[c];
+        s[pp - p0] = a->scale * acc;
+        if (s[pp - p0] > m) m = s[pp - p0];
+    }
+    double l = 0.0;
+    for (int64_t i = 0; i < a->dv; ++i) out[i] = 0.0;
+    for (int64_t pp = p0; pp <= P; ++pp) {
+        const double pr = exp(s[pp - p0] - m);
+        l += pr;
+        const float* vr = vc + (pp % a->W) * a->dv;
+        for (int64_t i = 0; i < a->dv; ++i) out[i] += pr * (double)vr[i];
+    }
+    for (int64_t i = 0; i < a->dv; ++i) out[i] /= l;
+    free(s);
+}
+
+int rodref_swska_decode(const float* q, const float* k_new, const float* v_new, float* k_cache,
+                        float* v_cache, const int64_t* pos, double* o, int64_t N, int64_t H,
+                        int64_t dk, int64_t dv, int64_t W, double scale, int nthreads) {
+    if (!q || !k_new || !v_new || !k_cache || !v_cache || !pos || !o) return RODREF_EINVAL;
+    if (N < 0 || H < 1 || dk < 1 || dv < 1 || W < 1) return RODREF_EINVAL;
+    for (int64_t n = 0; n < N; ++n)
+        if (pos[n] < 0) return RODREF_EINVAL;
+    /* step 1: ring-buffer write of the new token */
+    for (int64_t n = 0; n < N; ++n) {
+        const int64_t slot = pos[n] % W;
+        memcpy(k_cache + (n * W + slot) * dk, k_new + n * dk, (size_t)dk * sizeof(float));
+        for (int64_t h = 0; h < H; ++h)
+            memcpy(v_cache + ((n * H + h) * W + slot) * dv, v_new + (n * H + h) * dv,
+                   (size_t)dv * sizeof(float));
+    }
+    /* step 2: attention over the window */
+    ska_dec_args_t a = {q, k_new, v_new, k_cache, v_cache, pos, o, H, dk, dv, W, scale};
+    return run_units(ska_dec_unit, &a, N * H, nthreads);
+}
+
+int rodref_abi_version(void) { return 1; }

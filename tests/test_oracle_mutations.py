@@ -1,0 +1,88 @@
+"""Planted-mistake check for the oracle's pins (CPU only).
+
+Each case copies oracle/rodref.c to a temporary directory, plants one plausible mistake by a
+textual substitution (a gate applied to the wrong channel, a decay that also hits the new
+term, the readout using k, an off-by-one window, a dropped scale or normaliser, a wrong
+ring-buffer slot), builds the copy with gcc and runs every pin against it. Each planted
+mistake must make at least one pin fail; otherwise the pins are too weak to trust.
+"""
+import inspect
+import os
+import subprocess
+
+import numpy as np
+import pytest
+
+import oracle
+from oracle import build as obuild
+
+from . import test_oracle_pins as pins
+
+MUTATIONS = {
+    "gate_on_wrong_channel": ("const double gc = (double)g[c];",
+                              "const double gc = (double)g[(c + 1) % dk];"),
+    "decay_hits_new_term": ("row[j] = gc * row[j] + kc * (double)v[j];",
+                            "row[j] = gc * (row[j] + kc * (double)v[j]);"),
+    "readout_uses_key": ("acc += (double)q[c] * S[c * dv + j];",
+                         "acc += (double)k[c] * S[c * dv + j];"),
+    "window_one_too_wide": ("int64_t j0 = t - a->W + 1;", "int64_t j0 = t - a->W;"),
+    "scale_dropped": ("s[j - j0] = scale * acc;", "s[j - j0] = acc;"),
+    "normaliser_dropped": ("for (int64_t i = 0; i < dv; ++i) out[i] /= l;\n}",
+                           "for (int64_t i = 0; i < dv; ++i) out[i] /= 1.0;\n}"),
+    "ring_slot_off_by_one": ("const int64_t slot = pos[n] % W;",
+                             "const int64_t slot = (pos[n] + 1) % W;"),
+    "decode_window_too_wide": ("const int64_t p0 = P - a->W + 1 > 0 ? P - a->W + 1 : 0;",
+                               "const int64_t p0 = P - a->W > 0 ? P - a->W : 0;"),
+}
+
+
+def _pin_calls():
+    """Every pin test with each of its parametrizations, as zero-argument callables."""
+    calls = []
+    for name, fn in inspect.getmembers(pins, inspect.isfunction):
+        if not name.startswith("test_"):
+            continue
+        marks = getattr(fn, "pytestmark", [])
+        params = [m for m in marks if m.name == "parametrize"]
+        if not params:
+            calls.append((name, fn, {}))
+            continue
+        argnames, values = params[0].args[0], params[0].args[1]
+        names = [a.strip() for a in argnames.split(",")]
+        for val in values:
+            val = val if len(names) > 1 else (val,)
+            calls.append((name, fn, dict(zip(names, val))))
+    return calls
+
+
+def _build_mutant(tmp_path, old, new):
+    src = open(obuild.SRC).read()
+    assert src.count(old) == 1, f"mutation anchor not unique/found: {old!r}"
+    path = tmp_path / "rodref_mut.c"
+    path.write_text(src.replace(old, new))
+    so = tmp_path / "librodref_mut.so"
+    subprocess.run(["gcc", "-std=c11", "-O2", "-fPIC", "-shared", "-o", str(so), str(path),
+                    "-lm", "-lpthread"], check=True)
+    return oracle.OracleLib(str(so))
+
+
+@pytest.mark.parametrize("mutation", sorted(MUTATIONS))
+def test_pins_catch_planted_mistake(mutation, tmp_path):
+    old, new = MUTATIONS[mutation]
+    lib = _build_mutant(tmp_path, old, new)
+    caught = []
+    with oracle.using(lib):
+        for name, fn, kw in _pin_calls():
+            try:
+                fn(**kw)
+            except AssertionError:
+                caught.append(name)
+    assert caught, f"no pin caught the planted mistake '{mutation}'"
+
+
+def test_unmutated_copy_passes_every_pin(tmp_path):
+    lib = _build_mutant(tmp_path, "int rodref_abi_version(void) { return 1; }",
+                        "int rodref_abi_version(void) { return 1; }")
+    with oracle.using(lib):
+        for name, fn, kw in _pin_calls():
+            fn(**kw)

@@ -1,0 +1,276 @@
+"""Pins for the fp64 CPU oracle: it is checked against things other than itself.
+
+Each test compares the oracle with an independent statement of what the pages and the
+mathematics fix: hand-worked examples (tests/golden), the O(T^2) unrolled form of the
+recurrence, closed forms for special gates (g = 1: causal linear attention, SALA blog §2.2
+with phi = identity; g = 0: state reset; scalar g: geometric decay, SALA blog §4.3 tip 3),
+PyTorch's fp64 CPU softmax attention as a library routine (window >= T is full causal
+attention; SKA equals multi-head attention with the shared K replicated per head, CodeFuse
+Rodimus* article Fig. 4), window edge cases (W = 1, uniform softmax), and decode/prefill and
+split-prefill consistency (SALA blog §3.3 chunked prefill, §3.4 train/infer consistency).
+Inputs use dk != dv and per-channel gates so that a transposed operand, a row/column mix-up,
+an off-by-one window or a dropped term fails at least one test (tests/test_oracle_mutations.py
+plants such mistakes and checks that they are caught).
+"""
+import json
+import math
+import os
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+
+GOLD = os.path.join(os.path.dirname(__file__), "golden")
+RTOL = 1e-12
+
+
+def _rng(seed):
+    return np.random.default_rng(seed)
+
+
+def _gla_case(B=2, H=3, T=23, dk=5, dv=7, seed=0, gate="rand"):
+    r = _rng(seed)
+    q = r.standard_normal((B, H, T, dk)).astype(np.float32)
+    k = r.standard_normal((B, H, T, dk)).astype(np.float32)
+    v = r.standard_normal((B, H, T, dv)).astype(np.float32)
+    if gate == "rand":
+        g = r.uniform(0.05, 1.0, (B, H, T, dk)).astype(np.float32)
+    elif gate == "one":
+        g = np.ones((B, H, T, dk), np.float32)
+    elif gate == "zero":
+        g = np.zeros((B, H, T, dk), np.float32)
+    else:
+        g = np.full((B, H, T, dk), float(gate), np.float32)
+    S0 = r.standard_normal((B, H, dk, dv))
+    return q, k, v, g, S0
+
+
+def _close(a, b, tol=RTOL):
+    a, b = np.asarray(a, np.float64), np.asarray(b, np.float64)
+    scale = max(1.0, float(np.max(np.abs(b))) if b.size else 1.0)
+    err = float(np.max(np.abs(a - b))) if a.size else 0.0
+    assert err <= tol * scale, f"max abs err {err:.3e} > {tol * scale:.3e}"
+
+
+# ------------------------------------------------------------------------------------------
+# gated linear recurrence
+# ------------------------------------------------------------------------------------------
+
+
+def test_gla_hand_worked_example():
+    gd = json.load(open(os.path.join(GOLD, "gla_hand_t3.json")))
+    f = lambda x: np.asarray(x, np.float32)[None, None]
+    o, S = oracle.gla_prefill(f(gd["q"]), f(gd["k"]), f(gd["v"]), f(gd["g"]),
+                              np.asarray(gd["state0"], np.float64)[None, None])
+    np.testing.assert_array_equal(o[0, 0], np.asarray(gd["o"], np.float64))
+    np.testing.assert_array_equal(S[0, 0], np.asarray(gd["state"], np.float64))
+
+
+def _unrolled(q, k, v, g, S0):
+    """o_t = sum_{s<=t} sum_c q_tc k_sc (prod_{r=s+1..t} g_rc) v_s + sum_c q_tc (prod_{r<=t} g_rc) S0[c,:]
+    and the final state, written as explicit products of gates (no recurrence)."""
+    B, H, T, dk = q.shape
+    dv = v.shape[-1]
+    q, k, v, g = (x.astype(np.float64) for x in (q, k, v, g))
+    o = np.zeros((B, H, T, dv))
+    S = np.zeros((B, H, dk, dv))
+    for b in range(B):
+        for h in range(H):
+            for t in range(T):
+                acc = np.zeros(dv)
+                for s in range(t + 1):
+                    dec = np.prod(g[b, h, s + 1:t + 1], axis=0)          # [dk]
+                    acc += np.sum(q[b, h, t] * k[b, h, s] * dec) * v[b, h, s]
+                dec0 = np.prod(g[b, h, :t + 1], axis=0)
+                acc += (q[b, h, t] * dec0) @ S0[b, h]
+                o[b, h, t] = acc
+            for s in range(T):
+                dec = np.prod(g[b, h, s + 1:T], axis=0)
+                S[b, h] += np.outer(k[b, h, s] * dec, v[b, h, s])
+            S[b, h] += np.prod(g[b, h, :T], axis=0)[:, None] * S0[b, h]
+    return o, S
+
+
+@pytest.mark.parametrize("seed", [0, 1])
+def test_gla_recurrence_equals_unrolled_masked_form(seed):
+    q, k, v, g, S0 = _gla_case(seed=seed)
+    o, S = oracle.gla_prefill(q, k, v, g, S0)
+    o_ref, S_ref = _unrolled(q, k, v, g, S0)
+    _close(o, o_ref)
+    _close(S, S_ref)
+
+
+def test_gla_g1_is_causal_linear_attention():
+    q, k, v, g, S0 = _gla_case(gate="one", seed=3)
+    o, S = oracle.gla_prefill(q, k, v, g, S0)
+    q64, k64, v64 = (x.astype(np.float64) for x in (q, k, v))
+    T = q.shape[2]
+    mask = np.tril(np.ones((T, T)))
+    o_ref = (q64 @ np.swapaxes(k64, -1, -2) * mask) @ v64 + q64 @ S0
+    S_ref = S0 + np.swapaxes(k64, -1, -2) @ v64
+    _close(o, o_ref)
+    _close(S, S_ref)
+
+
+def test_gla_g0_resets_state():
+    q, k, v, g, S0 = _gla_case(gate="zero", seed=4)
+    o, S = oracle.gla_prefill(q, k, v, g, S0)
+    q64, k64, v64 = (x.astype(np.float64) for x in (q, k, v))
+    o_ref = np.sum(q64 * k64, axis=-1, keepdims=True) * v64
+    S_ref = k64[:, :, -1, :, None] * v64[:, :, -1, None, :]
+    _close(o, o_ref)
+    _close(S, S_ref)
+
+
+def test_gla_scalar_gate_is_geometric_decay():
+    gamma = 0.75
+    q, k, v, g, S0 = _gla_case(gate=gamma, seed=5, T=17)
+    o, S = oracle.gla_prefill(q, k, v, g, S0)
+    q64, k64, v64 = (x.astype(np.float64) for x in (q, k, v))
+    T = q.shape[2]
+    t = np.arange(T)
+    D = np.where(t[:, None] >= t[None, :], gamma ** (t[:, None] - t[None, :]), 0.0)
+    o_ref = (q64 @ np.swapaxes(k64, -1, -2) * D) @ v64 + (gamma ** (t + 1))[:, None] * (q64 @ S0)
+    _close(o, o_ref)
+
+
+def test_gla_decode_steps_equal_prefill():
+    q, k, v, g, S0 = _gla_case(seed=6, T=11)
+    o, S = oracle.gla_prefill(q, k, v, g, S0)
+    St = S0.copy()
+    for t in range(q.shape[2]):
+        ot, St = oracle.gla_decode_step(q[:, :, t], k[:, :, t], v[:, :, t], g[:, :, t], St)
+        np.testing.assert_array_equal(ot, o[:, :, t])
+    np.testing.assert_array_equal(St, S)
+
+
+@pytest.mark.parametrize("t1", [1, 9, 22])
+def test_gla_split_prefill_hands_off_state(t1):
+    q, k, v, g, S0 = _gla_case(seed=7)
+    o, S = oracle.gla_prefill(q, k, v, g, S0)
+    o1, S1 = oracle.gla_prefill(q[:, :, :t1], k[:, :, :t1], v[:, :, :t1], g[:, :, :t1], S0)
+    o2, S2 = oracle.gla_prefill(q[:, :, t1:], k[:, :, t1:], v[:, :, t1:], g[:, :, t1:], S1)
+    np.testing.assert_array_equal(np.concatenate([o1, o2], axis=2), o)
+    np.testing.assert_array_equal(S2, S)
+
+
+def test_gla_empty_sequence_keeps_state():
+    q, k, v, g, S0 = _gla_case(T=0, seed=8)
+    o, S = oracle.gla_prefill(q, k, v, g, S0)
+    assert o.shape == (2, 3, 0, 7)
+    np.testing.assert_array_equal(S, S0)
+
+
+# ------------------------------------------------------------------------------------------
+# sliding-window shared-key attention
+# ------------------------------------------------------------------------------------------
+
+
+def _ska_case(B=2, H=3, T=29, dk=6, dv=5, seed=0):
+    r = _rng(100 + seed)
+    q = r.standard_normal((B, H, T, dk)).astype(np.float32)
+    k = r.standard_normal((B, T, dk)).astype(np.float32)
+    v = r.standard_normal((B, H, T, dv)).astype(np.float32)
+    return q, k, v
+
+
+def _sdpa(q, k_rep, v, mask=None, causal=False, scale=None):
+    t = lambda x: torch.from_numpy(np.asarray(x, np.float64))
+    return torch.nn.functional.scaled_dot_product_attention(
+        t(q), t(k_rep), t(v), attn_mask=None if mask is None else torch.from_numpy(mask),
+        is_causal=causal, scale=scale).numpy()
+
+
+def test_swska_hand_worked_example():
+    gd = json.load(open(os.path.join(GOLD, "swska_hand_t4.json")))
+    q = np.asarray(gd["q"], np.float32)[None, None, :, None]
+    k = np.asarray(gd["k"], np.float32)[None, :, None]
+    v = np.asarray(gd["v"], np.float32)[None, None, :, None]
+    o = oracle.swska_prefill(q, k, v, gd["window"], scale=1.0)
+    _close(o[0, 0, :, 0], gd["o"], 1e-15)
+    o3 = oracle.swska_prefill(q, k, v, 3, scale=1.0)
+    _close(o3[0, 0, :, 0], gd["o_window3"], 1e-15)
+
+
+def test_swska_two_key_closed_form():
+    # one query against two keys: o = (v0 + e^{s1-s0} v1) / (1 + e^{s1-s0})
+    q = np.array([0.0, 1.5], np.float32)[None, None, :, None]
+    k = np.array([0.5, 2.0], np.float32)[None, :, None]
+    v = np.array([2.0, -4.0], np.float32)[None, None, :, None]
+    o = oracle.swska_prefill(q, k, v, 2, scale=1.0)
+    e = math.exp(1.5 * 2.0 - 1.5 * 0.5)
+    _close(o[0, 0, 1, 0], (2.0 - 4.0 * e) / (1.0 + e), 1e-15)
+
+
+@pytest.mark.parametrize("W", [29, 64])
+def test_swska_window_ge_T_is_full_causal_attention(W):
+    q, k, v = _ska_case(seed=1)
+    H = q.shape[1]
+    o = oracle.swska_prefill(q, k, v, W)
+    k_rep = np.repeat(k[:, None], H, axis=1)
+    _close(o, _sdpa(q, k_rep, v, causal=True), 1e-12)
+
+
+@pytest.mark.parametrize("W", [1, 2, 5, 17])
+def test_swska_shared_key_equals_mha_with_replicated_key(W):
+    q, k, v = _ska_case(seed=2)
+    B, H, T, _ = q.shape
+    o = oracle.swska_prefill(q, k, v, W, scale=0.3)
+    k_rep = np.repeat(k[:, None], H, axis=1)
+    # boolean "may attend" mask built from the window as a set of positions
+    allowed = np.zeros((T, T), bool)
+    for t in range(T):
+        allowed[t, list(range(max(0, t - W + 1), t + 1))] = True
+    _close(o, _sdpa(q, k_rep, v, mask=allowed, scale=0.3), 1e-12)
+
+
+def test_swska_window_one_is_identity_on_v():
+    q, k, v = _ska_case(seed=3)
+    o = oracle.swska_prefill(q, k, v, 1)
+    np.testing.assert_array_equal(o, v.astype(np.float64))
+
+
+@pytest.mark.parametrize("W", [3, 8])
+def test_swska_zero_query_averages_the_window(W):
+    q, k, v = _ska_case(seed=4)
+    q[:] = 0
+    o = oracle.swska_prefill(q, k, v, W)
+    T = q.shape[2]
+    ref = np.stack([v[:, :, max(0, t - W + 1):t + 1].astype(np.float64).mean(axis=2)
+                    for t in range(T)], axis=2)
+    _close(o, ref, 1e-14)
+
+
+def test_swska_row_sampling_matches_full_output():
+    q, k, v = _ska_case(seed=5)
+    B, H, T, _ = q.shape
+    o = oracle.swska_prefill(q, k, v, 7)
+    rows = np.array([0, 5, T - 1, T, 2 * T + 3, B * H * T - 1])
+    osub = oracle.swska_prefill(q, k, v, 7, rows=rows)
+    np.testing.assert_array_equal(osub, o.reshape(-1, o.shape[-1])[rows])
+
+
+@pytest.mark.parametrize("W,positions", [(8, [0, 3, 7, 8, 13, 30]), (5, [4, 5, 6, 9, 24])])
+def test_swska_ring_buffer_decode_equals_prefill_row(W, positions):
+    """Fill a ring buffer from a sequence, then decode position P: the output must equal the
+    prefill output row P (SALA blog §3.3 rolling window; §3.4 consistency)."""
+    H, dk, dv = 3, 6, 5
+    T = max(positions) + 1
+    q, k, v = _ska_case(B=1, H=H, T=T, dk=dk, dv=dv, seed=6)
+    o_pre = oracle.swska_prefill(q, k, v, W)
+    N = len(positions)
+    kc = np.zeros((N, W, dk), np.float32)
+    vc = np.zeros((N, H, W, dv), np.float32)
+    for n, P in enumerate(positions):           # tokens before P sit in slot p mod W
+        for p in range(max(0, P - W + 1), P):
+            kc[n, p % W] = k[0, p]
+            vc[n, :, p % W] = v[0, :, p]
+    P = np.asarray(positions)
+    o, kc2, vc2 = oracle.swska_decode(q[0][:, P].transpose(1, 0, 2), k[0, P], v[0][:, P].transpose(1, 0, 2),
+                                      kc, vc, P, W)
+    _close(o, o_pre[0][:, P].transpose(1, 0, 2), 1e-13)
+    for n, p in enumerate(positions):
+        np.testing.assert_array_equal(kc2[n, p % W], k[0, p])
+        np.testing.assert_array_equal(vc2[n, :, p % W], v[0, :, p])
