@@ -1,0 +1,485 @@
+#!/usr/bin/env python3
+"""Benchmark of the Rodimus+ token-mixing hot path on B200.
+
+One step = one prefill pass of the long-context Rodimus+ mixer stack (B=1, T=131072,
+hidden 2048 = 16 heads x 128, 24 layers alternating the gated linear recurrence and SW-SKA
+with window 4096), every layer through the library's C ABI. value = prefill tokens/s over all
+ranks (each rank runs its own replica on its own seeded inputs: weak scaling, no collective
+in the data path). The same line carries the batched decode step (256 sequences x 1 token:
+recurrence update + readout over 16 heads of 128x128 fp32 state, and SW-SKA over a
+4096-slot ring buffer) as "decode", the roofline of the dominant kernel, the oracle's CPU
+baseline, an end-to-end number through host buffers, clocks and the launch count.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "Rodimus+ mixer prefill tokens/s & decode tok/s on 1 B200; % of HBM/TC roofline"
+WORKLOAD = "stack_t131072"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+# ------------------------------------------------------------------------------------------
+# helpers
+# ------------------------------------------------------------------------------------------
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            p = json.load(f)
+        return p, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+def swska_pairs(T, W):
+    """Number of (query, key) pairs inside the causal window, per (batch, head)."""
+    if W >= T:
+        return T * (T + 1) // 2
+    return W * T - W * (W - 1) // 2
+
+
+class ClockSampler:
+    """nvidia-smi sampled every 200 ms while the timed region runs."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index):
+        self.gpu = gpu_index
+        self.proc = None
+        self.file = None
+
+    def __enter__(self):
+        try:
+            self.file = tempfile.NamedTemporaryFile("w+", suffix=".csv", delete=False)
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=self.file, stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+        return self
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+        return False
+
+    def summary(self):
+        if self.proc is None or self.file is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.file.flush()
+        with open(self.file.name) as f:
+            rows = [r.strip().split(", ") for r in f if r.strip()]
+        os.unlink(self.file.name)
+        sm, mx, reasons, power = [], None, set(), []
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for r in rows:
+            if len(r) < 9:
+                continue
+            try:
+                sm.append(float(r[1]))
+                mx = float(r[2])
+                power.append(float(r[3]))
+            except ValueError:
+                continue
+            for n, val in zip(names, r[5:9]):
+                if val.strip().lower() == "active":
+                    reasons.add(n)
+        loaded = [s for s, p in zip(sm, power) if p > 300] or sm
+        return {"sm_mhz": statistics.median(loaded) if loaded else None, "sm_max_mhz": mx,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+def kernel_source_hash(*names):
+    h = hashlib.sha256()
+    for n in names:
+        with open(os.path.join(ROOT, "sliding_window_attention_chunked_b200", "csrc", n), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def recorded_traffic(kernel_key, sources):
+    """DRAM bytes per launch from a committed ncu capture, if the kernel is unchanged since."""
+    path = os.path.join(ROOT, "profiles", "ncu_traffic.json")
+    if not os.path.exists(path):
+        return None
+    with open(path) as f:
+        rec = json.load(f).get(kernel_key)
+    if not rec or rec.get("source_hash") != kernel_source_hash(*sources):
+        return None
+    return rec.get("dram_bytes_per_launch")
+
+
+# ------------------------------------------------------------------------------------------
+# CPU baseline: the oracle, timed on a bounded sample of the same workload
+# ------------------------------------------------------------------------------------------
+
+
+def oracle_stack_sample(dims):
+    """Time the fp64 oracle on a sample of the stack and scale to stack tokens/s.
+
+    Recurrence layer: all 16 heads over the first n tokens (sequential in t, one thread per
+    (b,h) unit). SW-SKA layer: full-window rows (t >= W) of random (head, t) pairs. The stack
+    time per token is 12 x (recurrence per token + SW-SKA per token)."""
+    import numpy as np
+
+    import oracle
+    from sliding_window_attention_chunked_b200 import workloads as wl
+
+    H, dk, dv, W, T = dims["H"], dims["dk"], dims["dv"], dims["window"], dims["T"]
+    n_gla = 32768
+    q, k, v, g = wl.gla_inputs(1, H, n_gla, dk, dv, dist="l2", seed=0)
+    t0 = time.perf_counter()
+    oracle.gla_prefill(q, k, v, g)
+    t_gla = time.perf_counter() - t0
+    gla_per_tok = t_gla / n_gla                   # all H heads for one token
+    # SW-SKA: rows with a full window
+    Ts = W + 64
+    qs, ks, vs = wl.swska_inputs(1, H, Ts, dk, dv, dist="l2", seed=1)
+    n_rows = 32768
+    rng = np.random.default_rng(0)
+    hs = rng.integers(0, H, n_rows)
+    ts = rng.integers(W - 1, Ts, n_rows)
+    rows = hs * Ts + ts
+    t0 = time.perf_counter()
+    oracle.swska_prefill(qs, ks, vs, W, rows=rows)
+    t_ska = time.perf_counter() - t0
+    ska_per_tok = t_ska / n_rows * H               # all H heads for one token
+    layers = dims["layers"]
+    per_tok = (layers // 2) * (gla_per_tok + ska_per_tok)
+    cores = oracle.default_threads()
+    sample = (f"oracle fp64 on {cores} threads: recurrence {H} heads x {n_gla} tokens "
+              f"({t_gla:.2f} s) + SW-SKA {n_rows} full-window rows ({t_ska:.2f} s), scaled to "
+              f"the {layers}-layer stack per token")
+    return {"value": 1.0 / per_tok, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+            "sample": sample, "seconds": t_gla + t_ska}
+
+
+# ------------------------------------------------------------------------------------------
+# the GPU arm
+# ------------------------------------------------------------------------------------------
+
+
+def run_gpu(args):
+    import torch
+    import torch.distributed as dist
+
+    import sliding_window_attention_chunked_b200 as rod
+    from sliding_window_attention_chunked_b200 import build as rbuild
+    from sliding_window_attention_chunked_b200 import workloads as wl
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    else:
+        torch.cuda.set_device(0)
+    dev = torch.device("cuda", torch.cuda.current_device())
+    if rank == 0:
+        rbuild.build()
+    if world > 1:
+        dist.barrier()
+    rod.load_library()
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize()
+
+    def max_over_ranks(x):
+        if world == 1:
+            return x
+        t = torch.tensor([x], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        return float(t.item())
+
+    d = wl.WORKLOADS[WORKLOAD].dims
+    B, H, T, dk, dv, L, W, C = d["B"], d["H"], d["T"], d["dk"], d["dv"], d["layers"], d["window"], d["chunk"]
+    seed_base = 1000 * rank
+    layers = []
+    for l in range(L):
+        ins = wl.stack_layer_inputs(l, B, H, T, dk, dv, seed_base=seed_base, device=dev)
+        out = torch.empty(B, H, T, dv, dtype=torch.bfloat16, device=dev)
+        st = torch.zeros(B, H, dk, dv, device=dev) if wl.stack_layer_kind(l) == "gla" else None
+        layers.append((wl.stack_layer_kind(l), ins, out, st))
+    ws_bytes = rod.gla_prefill_workspace_size(B, H, T, dk, dv, C)
+    ws = torch.empty(max(ws_bytes, 16), dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream()
+    ska_events = []
+
+    def step(record=False):
+        for kind, ins, out, st in layers:
+            if kind == "gla":
+                q, k, v, g = ins
+                st.zero_()
+                rod.gla_prefill(q, k, v, g, st, o=out, chunk=C, workspace=ws)
+            else:
+                q, k, v = ins
+                if record:
+                    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                    e0.record(stream)
+                rod.swska_prefill(q, k, v, W, o=out)
+                if record:
+                    e1.record(stream)
+                    ska_events.append((e0, e1))
+
+    for _ in range(args.warmup):
+        step()
+    rod.check()
+    barrier()
+    n0 = rod.launch_count()
+    with ClockSampler(dev.index) as clk:
+        ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        barrier()
+        ev0.record(stream)
+        for _ in range(args.steps):
+            step(record=True)
+        ev1.record(stream)
+        barrier()
+    launches = rod.launch_count() - n0
+    rod.check()
+    ms_local = ev0.elapsed_time(ev1)
+    ms = max_over_ranks(ms_local)
+    ms_per_step = ms / args.steps
+    tokens = B * T * world * args.steps
+    value = tokens / (ms / 1e3)
+    ska_ms = [a.elapsed_time(b) for a, b in ska_events]
+    ska_avg_ms = max_over_ranks(sum(ska_ms) / len(ska_ms))
+    clocks = clk.summary()
+
+    peaks, peaks_src = load_peaks()
+    ska_flop = 4.0 * (dk + dv) / 2 * swska_pairs(T, W) * B * H  # 2*dk (QK^T) + 2*dv (PV) per pair
+    achieved_tflops = ska_flop / (ska_avg_ms / 1e3) / 1e12
+    peak_tf = peaks.get("bf16_tflops_sustained") or peaks.get("bf16_tflops")
+    roofline = {"bound": "tensor", "kernel": "rod_swska_prefill", "achieved": round(achieved_tflops, 2),
+                "peak": peak_tf, "unit": "TFLOP/s", "frac": round(achieved_tflops / peak_tf, 4),
+                "peak_source": f"{peaks_src} (bf16_tflops_sustained: kernel timed inside a long step)",
+                "flop_per_launch": ska_flop, "avg_launch_ms": round(ska_avg_ms, 4),
+                "traffic": recorded_traffic("swska_prefill_stack", ["swska_prefill_simt.cu"])}
+
+    # ---- batched decode step (recurrence + SW-SKA), 256 sequences ----
+    dd_dims = wl.WORKLOADS["decode_n256"].dims
+    N, Wd = dd_dims["N"], dd_dims["window"]
+    dd = wl.decode_inputs(N, H, dk, dv, Wd, seed=seed_base + 77, device=dev)
+    o1 = torch.empty(N, H, dv, dtype=torch.bfloat16, device=dev)
+    o2 = torch.empty_like(o1)
+
+    def dec_step():
+        rod.gla_decode_step(dd["q"], dd["k"], dd["v"], dd["g"], dd["state"], o=o1)
+        rod.swska_decode(dd["sq"], dd["k_new"], dd["v_new"], dd["k_cache"], dd["v_cache"],
+                         dd["pos"], Wd, o=o2)
+
+    for _ in range(max(3, args.warmup)):
+        dec_step()
+    rod.check()
+    dsteps = max(20, args.steps * 4)
+    ge = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(dsteps)]
+    se = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(dsteps)]
+    barrier()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for i in range(dsteps):
+        ge[i][0].record(stream)
+        rod.gla_decode_step(dd["q"], dd["k"], dd["v"], dd["g"], dd["state"], o=o1)
+        ge[i][1].record(stream)
+        se[i][0].record(stream)
+        rod.swska_decode(dd["sq"], dd["k_new"], dd["v_new"], dd["k_cache"], dd["v_cache"],
+                         dd["pos"], Wd, o=o2)
+        se[i][1].record(stream)
+    e1.record(stream)
+    barrier()
+    rod.check()
+    dec_ms = max_over_ranks(e0.elapsed_time(e1) / dsteps)
+    gla_dec_ms = max_over_ranks(sum(a.elapsed_time(b) for a, b in ge) / dsteps)
+    ska_dec_ms = max_over_ranks(sum(a.elapsed_time(b) for a, b in se) / dsteps)
+    gla_dec_bytes = 2.0 * N * H * dk * dv * 4 + N * H * (2 * dk * 2 + dk * 4 + dv * 2 + dv * 2)
+    ska_dec_bytes = 1.0 * N * Wd * dk * 2 + N * H * Wd * dv * 2 + N * H * (dk + dv + dv) * 2 + N * dk * 2
+    hbm = peaks.get("hbm_gbs")
+    decode = {
+        "workload": "decode_n256 (N=256 sequences x 1 token, H=16, 128x128 fp32 state, "
+                    "SW-SKA ring window 4096)",
+        "value": round(N * world / (dec_ms / 1e3), 1), "unit": "tokens/s",
+        "ms_per_step": round(dec_ms, 4),
+        "kernels": {
+            "rod_gla_decode_step": {"bound": "hbm", "avg_launch_ms": round(gla_dec_ms, 4),
+                                    "algorithmic_bytes": gla_dec_bytes,
+                                    "achieved": round(gla_dec_bytes / (gla_dec_ms / 1e3) / 1e9, 1),
+                                    "peak": hbm, "unit": "GB/s",
+                                    "frac": round(gla_dec_bytes / (gla_dec_ms / 1e3) / 1e9 / hbm, 4)},
+            "rod_swska_decode": {"bound": "hbm", "avg_launch_ms": round(ska_dec_ms, 4),
+                                 "algorithmic_bytes": ska_dec_bytes,
+                                 "achieved": round(ska_dec_bytes / (ska_dec_ms / 1e3) / 1e9, 1),
+                                 "peak": hbm, "unit": "GB/s",
+                                 "frac": round(ska_dec_bytes / (ska_dec_ms / 1e3) / 1e9 / hbm, 4)},
+        },
+    }
+
+    # ---- per-layer-type breakdown of the prefill step (GLA layers by difference) ----
+    gla_ms_per_layer = (ms_per_step - (L // 2) * ska_avg_ms) / (L // 2)
+    gla_bytes = B * H * T * (3 * dk * 2 + dk * 4 + dv * 2) + B * H * dk * dv * 4 * 2
+    kernels = {
+        "rod_swska_prefill": {"bound": "tensor", "avg_launch_ms": round(ska_avg_ms, 4),
+                              "achieved_tflops": round(achieved_tflops, 2)},
+        "rod_gla_prefill": {"bound": "hbm", "avg_layer_ms": round(gla_ms_per_layer, 4),
+                            "algorithmic_bytes": gla_bytes,
+                            "achieved_gbs": round(gla_bytes / (gla_ms_per_layer / 1e3) / 1e9, 1),
+                            "frac_hbm": round(gla_bytes / (gla_ms_per_layer / 1e3) / 1e9 / hbm, 4)},
+    }
+
+    # ---- end to end through the public API with host buffers ----
+    e2e = None
+    if not args.no_e2e:
+        e2e = run_e2e(args, rod, torch, layers, d, ws, stream, barrier, max_over_ranks, world)
+
+    del layers, dd
+    torch.cuda.empty_cache()
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu = oracle_stack_sample(d)
+        cpu.pop("seconds", None)
+
+    line = {
+        "metric": METRIC, "value": round(value, 1), "unit": "tokens/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_per_step, 3),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic (seeded; per-layer inputs drawn on the device, seed = 1000*rank + layer)",
+        "config": {"workload": f"{WORKLOAD}: Rodimus+ mixer stack prefill, B=1, T=131072, "
+                               "H=16, d=128, 24 layers alternating recurrence (chunk 64) / "
+                               "SW-SKA (window 4096)",
+                   "global_batch": B * world, "seq_len": T, "layers": L,
+                   "parallelism": f"replicas x{world} (independent sequences, no collective)",
+                   "l2": "inputs > L2 (55 GB per step), no flush needed"},
+        "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": launches,
+        "clocks": clocks, "decode": decode, "kernels": kernels,
+    }
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.destroy_process_group()
+
+
+def run_e2e(args, rod, torch, layers, d, ws, stream, barrier, max_over_ranks, world):
+    """Same stack, but every step copies each layer's inputs from pinned host memory into the
+    device buffers and reads each layer's output back to pinned host memory."""
+    B, T, C, W = d["B"], d["T"], d["chunk"], d["window"]
+    host = {}
+    for kind, ins, out, st in layers:
+        if kind not in host:
+            host[kind] = ([t.to("cpu").pin_memory() for t in ins],
+                          torch.empty(out.shape, dtype=out.dtype).pin_memory())
+    h2d = d2h = 0
+
+    def step():
+        nonlocal h2d, d2h
+        h2d = d2h = 0
+        for kind, ins, out, st in layers:
+            hin, hout = host[kind]
+            for dst, src in zip(ins, hin):
+                dst.copy_(src, non_blocking=True)
+                h2d += src.numel() * src.element_size()
+            if kind == "gla":
+                st.zero_()
+                rod.gla_prefill(ins[0], ins[1], ins[2], ins[3], st, o=out, chunk=C, workspace=ws)
+            else:
+                rod.swska_prefill(ins[0], ins[1], ins[2], W, o=out)
+            hout.copy_(out, non_blocking=True)
+            d2h += out.numel() * out.element_size()
+
+    step()
+    barrier()
+    n = args.e2e_steps
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(n):
+        step()
+    e1.record(stream)
+    barrier()
+    ms = max_over_ranks(e0.elapsed_time(e1))
+    return {"value": round(B * T * world * n / (ms / 1e3), 1), "unit": "tokens/s",
+            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": n,
+            "note": "pinned host buffers per layer kind reused for every layer; copies and "
+                    "kernels serialised on one stream"}
+
+
+# ------------------------------------------------------------------------------------------
+# the reference arm: the oracle, timed on the host cores
+# ------------------------------------------------------------------------------------------
+
+
+def run_reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    if rank != 0:
+        return
+    from sliding_window_attention_chunked_b200 import workloads as wl
+    d = wl.WORKLOADS[WORKLOAD].dims
+    for _ in range(args.warmup):
+        oracle_stack_sample(d)
+    vals, secs = [], 0.0
+    for _ in range(args.steps):
+        r = oracle_stack_sample(d)
+        vals.append(r["value"])
+        secs += r.pop("seconds")
+    value = statistics.mean(vals)
+    r["value"] = value
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s",
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": 1e3 * secs / args.steps, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic (seeded)",
+        "config": {"workload": f"{WORKLOAD}: Rodimus+ mixer stack prefill (bounded sample, "
+                               "scaled per token)", "seq_len": d["T"], "layers": d["layers"]},
+        "cpu_baseline": r,
+        "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=5)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", default="rod", choices=["rod", "reference"])
+    ap.add_argument("--e2e-steps", type=int, default=1)
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    args.warmup = max(3, args.warmup)  # timing rule: at least 3 untimed warm-up steps
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_gpu(args)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,163 @@
+/*
+ * rod.h -- C ABI of librod.so: the Rodimus+ token-mixing hot path on one NVIDIA B200 (sm_100a).
+ *
+ * Two mixers, as the source pages describe them:
+ *  - the Rodimus gated linear recurrence, which compresses the history into a fixed-size
+ *    per-head state ("Rodimus block" paragraph of the CodeFuse article "ICLR 2025 | Rodimus*:
+ *    a hybrid attention mechanism balancing performance and efficiency": a chunkwise-parallel
+ *    algorithm for training/prefill, a fixed-size recurrent state at inference):
+ *        S_t = diag(g_t) S_{t-1} + k_t^T v_t,      o_t = q_t S_t
+ *    with the per-key-channel gates g_t in (0, 1] supplied by the caller;
+ *  - SW-SKA, causal sliding-window softmax attention whose key matrix is shared by all heads
+ *    while every head keeps its own values (same article, Fig. 4 and the SKA paragraph; window
+ *    of the most recent W tokens: setup blog "Rodimus* ... what problem does it solve", §3):
+ *        o[h,t] = sum_{j=max(0,t-W+1)}^{t} softmax_j(scale * q[h,t] . k[j]) v[h,j].
+ *
+ * Conventions shared by every call
+ *  - Every tensor pointer is caller-owned DEVICE memory (e.g. from PyTorch), row-major and
+ *    contiguous in the layout given per argument, 16-byte aligned. The library never frees or
+ *    keeps caller memory and allocates no device memory of its own on these calls.
+ *  - Every call is asynchronous on the given CUDA stream (a cudaStream_t passed as void*;
+ *    NULL = the legacy default stream) and returns a status: ROD_OK (0) or a negative ROD_ERR_*.
+ *    Argument errors are detected on the host before anything is launched; nothing is
+ *    written in that case. No exception crosses this ABI.
+ *  - dtype ROD_BF16: q, k, v, o (and the attention caches) are bf16; gates g and recurrent
+ *    states are fp32; all arithmetic accumulates in fp32.
+ *    dtype ROD_FP32: every tensor is fp32 and every product is an fp32 FMA (no tensor cores).
+ *  - Supported head dimensions dk, dv: 16, 32, 64, 128.
+ *  - A device-side wait that exceeds its bound (it never should) makes the kernel give up,
+ *    leave its outputs unspecified and raise a flag that rod_check() reports as
+ *    ROD_ERR_TIMEOUT.
+ */
+#ifndef ROD_H
+#define ROD_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define ROD_API __attribute__((visibility("default")))
+#else
+#define ROD_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* ---- status codes ----------------------------------------------------------------------- */
+#define ROD_OK 0
+#define ROD_ERR_NULL (-1)        /* a required pointer is NULL                                 */
+#define ROD_ERR_SHAPE (-2)       /* a size is out of range or unsupported                      */
+#define ROD_ERR_ALIGN (-3)       /* a pointer is not 16-byte aligned                           */
+#define ROD_ERR_DTYPE (-4)       /* dtype is neither ROD_BF16 nor ROD_FP32                     */
+#define ROD_ERR_WORKSPACE (-5)   /* workspace missing or smaller than the size query returns   */
+#define ROD_ERR_CUDA (-6)        /* a CUDA launch/runtime error; see rod_last_cuda_error()     */
+#define ROD_ERR_TIMEOUT (-7)     /* a bounded device-side wait expired (reported by rod_check) */
+
+/* ---- dtypes ------------------------------------------------------------------------------ */
+#define ROD_BF16 1
+#define ROD_FP32 2
+
+/* Human-readable name of a status code (static string, never NULL). */
+ROD_API const char* rod_status_string(int status);
+
+/* The cudaError_t value behind the most recent ROD_ERR_CUDA returned on this host thread
+ * (0 if none). */
+ROD_API int rod_last_cuda_error(void);
+
+/* Synchronise `stream`, then report ROD_ERR_TIMEOUT if any kernel of this library gave up on
+ * a bounded device wait since the last rod_check (and clear that flag), ROD_ERR_CUDA on a
+ * CUDA error, else ROD_OK. */
+ROD_API int rod_check(void* stream);
+
+/* Version of this ABI (incremented on any incompatible change). */
+ROD_API int rod_abi_version(void);
+
+/* Number of kernels this library has launched in this process so far (every entry point
+ * counts each kernel it enqueues; host-side counter, no synchronisation). */
+ROD_API uint64_t rod_launch_count(void);
+
+/* ---- gated linear recurrence: chunkwise prefill ------------------------------------------ */
+/*
+ * Bytes of device workspace rod_gla_prefill needs for these sizes (0 if none). The caller
+ * allocates it; its content on entry is irrelevant. Returns 0 for invalid sizes as well.
+ */
+ROD_API size_t rod_gla_prefill_workspace_size(int B, int H, int T, int dk, int dv, int chunk, int dtype);
+
+/*
+ * Prefill of T tokens for B sequences x H heads (CodeFuse article, Rodimus block: the
+ * chunkwise-parallel form used for training/prefill; it reaches the same result as the
+ * recurrence above up to rounding).
+ *   q, k  [B,H,T,dk]   dtype          queries and keys (any input gate pre-multiplied into k)
+ *   v     [B,H,T,dv]   dtype          values
+ *   g     [B,H,T,dk]   fp32           per-channel decay gates, expected in [0, 1]
+ *   state [B,H,dk,dv]  fp32, in/out   initial state on entry (zeros for a fresh sequence),
+ *                                     final state S_{T-1} on return
+ *   o     [B,H,T,dv]   dtype          outputs o_t = q_t S_t (no scale, no normaliser)
+ *   chunk              tokens per chunk: a multiple of 16 in [16, 128]. It changes rounding
+ *                      only, never the mathematical result; a T that is not a multiple of
+ *                      chunk is handled by masking the tail chunk.
+ *   workspace, ws_bytes  at least rod_gla_prefill_workspace_size(...) bytes (may be NULL
+ *                      when that size is 0).
+ * Calling it twice, on tokens [0,T1) and then [T1,T) with the returned state, equals one
+ * call on [0,T) up to rounding (chunked prefill: SALA blog §3.3).
+ * Errors: ROD_ERR_NULL, ROD_ERR_SHAPE (B,H < 0, T < 0, dk/dv unsupported, bad chunk),
+ * ROD_ERR_ALIGN, ROD_ERR_DTYPE, ROD_ERR_WORKSPACE, ROD_ERR_CUDA. T = 0 or B*H = 0 is a
+ * no-op (state unchanged).
+ */
+ROD_API int rod_gla_prefill(const void* q, const void* k, const void* v, const float* g, float* state,
+                    void* o, int B, int H, int T, int dk, int dv, int chunk, int dtype,
+                    void* workspace, size_t ws_bytes, void* stream);
+
+/* ---- gated linear recurrence: one decode step --------------------------------------------- */
+/*
+ * One token for each of N sequences x H heads, with the fixed-size state updated in place
+ * (CodeFuse article, Rodimus block: O(1)-space recurrent inference; SALA blog §3.3: the state
+ * stays resident on the GPU and is accumulated in place every step):
+ *   S <- diag(g) S + k^T v ;  o = q S   (S after the update)
+ *   q, k  [N,H,dk]  dtype;  v [N,H,dv] dtype;  g [N,H,dk] fp32;
+ *   state [N,H,dk,dv] fp32, read and overwritten;  o [N,H,dv] dtype.
+ * Errors: ROD_ERR_NULL, ROD_ERR_SHAPE, ROD_ERR_ALIGN, ROD_ERR_DTYPE, ROD_ERR_CUDA.
+ * N*H = 0 is a no-op.
+ */
+ROD_API int rod_gla_decode_step(const void* q, const void* k, const void* v, const float* g,
+                        float* state, void* o, int N, int H, int dk, int dv, int dtype,
+                        void* stream);
+
+/* ---- SW-SKA: prefill ----------------------------------------------------------------------- */
+/*
+ * Causal sliding-window attention with one key matrix shared by the H heads:
+ *   q [B,H,T,dk] dtype;  k [B,T,dk] dtype (shared);  v [B,H,T,dv] dtype;  o [B,H,T,dv] dtype.
+ *   window W >= 1: query t sees keys max(0, t-W+1) .. t (W keys including itself);
+ *   scale: multiplies q.k before the softmax; scale <= 0 selects 1/sqrt(dk).
+ * Errors: ROD_ERR_NULL, ROD_ERR_SHAPE (window < 1, dims unsupported, H > 64), ROD_ERR_ALIGN,
+ * ROD_ERR_DTYPE, ROD_ERR_CUDA. T = 0 or B*H = 0 is a no-op.
+ */
+ROD_API int rod_swska_prefill(const void* q, const void* k, const void* v, void* o, int B, int H,
+                      int T, int dk, int dv, int window, float scale, int dtype, void* stream);
+
+/* ---- SW-SKA: decode with a ring-buffer window cache --------------------------------------- */
+/*
+ * One new token per sequence (SALA blog §3.3: a self-made circular buffer holds the rolling
+ * window; CodeFuse article: the SKA cache holds one K and per-head V):
+ *   1. writes k_new[n] to k_cache[n, pos[n] mod W] and v_new[n,h] to v_cache[n,h,pos[n] mod W];
+ *   2. attends q[n,h] over the tokens at positions max(0, pos[n]-W+1) .. pos[n], whose
+ *      entries sit in slots p mod W (the caller keeps the cache filled by this same rule).
+ *   q [N,H,dk], k_new [N,dk], v_new [N,H,dv]: dtype;  k_cache [N,W,dk], v_cache [N,H,W,dv]:
+ *   dtype, updated in place;  pos [N] int64 on the device, read only (the caller advances
+ *   it);  o [N,H,dv] dtype.  window W >= 1, scale as for the prefill.
+ * A negative pos[n] is not detected on the host (it lives on the device): that sequence's
+ * output is set to NaN and its caches are left untouched.
+ * Errors: ROD_ERR_NULL, ROD_ERR_SHAPE (H > 64, dims unsupported, window < 1), ROD_ERR_ALIGN,
+ * ROD_ERR_DTYPE, ROD_ERR_CUDA. N = 0 is a no-op.
+ */
+ROD_API int rod_swska_decode(const void* q, const void* k_new, const void* v_new, void* k_cache,
+                     void* v_cache, const int64_t* pos, void* o, int N, int H, int dk, int dv,
+                     int window, float scale, int dtype, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* ROD_H */

@@ -1,0 +1,27 @@
+"""Rodimus+ token-mixing hot path on one NVIDIA B200 (sm_100a).
+
+A thin ctypes binding over ``librod.so`` (C ABI in ``include/rod.h``): every call here only
+checks and marshals torch CUDA tensors into the library, which runs every step of the path in
+its own CUDA kernels. There is no CPU fallback: without the built library (or without a GPU)
+the calls raise.
+
+    gla_prefill(q, k, v, g, state, chunk=64)       chunkwise prefill of the gated recurrence
+    gla_decode_step(q, k, v, g, state)              one fused recurrent decode step
+    swska_prefill(q, k, v, window, scale=None)      sliding-window shared-key attention
+    swska_decode(q, k_new, v_new, k_cache, v_cache, pos, window)   ring-buffer decode
+"""
+from ._binding import (  # noqa: F401
+    ROD_BF16,
+    ROD_FP32,
+    RodError,
+    abi_version,
+    check,
+    gla_decode_step,
+    gla_prefill,
+    gla_prefill_workspace_size,
+    launch_count,
+    library_path,
+    load_library,
+    swska_decode,
+    swska_prefill,
+)

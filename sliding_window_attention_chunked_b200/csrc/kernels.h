@@ -1,0 +1,38 @@
+// kernels.h -- internal launch interface between the C ABI (rod_api.cu) and the kernels.
+// Every launcher validates nothing (rod_api.cu has done it), enqueues on `stream` and
+// returns the launch status.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+namespace rod {
+
+// host-side count of kernel launches enqueued by this library (reported by rod_launch_count)
+void note_launches(unsigned n);
+
+// gated linear recurrence, one decode step (fused, HBM-bound)
+cudaError_t gla_decode_launch(const void* q, const void* k, const void* v, const float* g,
+                              float* state, void* o, int N, int H, int dk, int dv, bool bf16,
+                              cudaStream_t stream);
+
+// gated linear recurrence prefill, sequential-in-time form on CUDA cores (exact fp32 FMA)
+cudaError_t gla_prefill_recurrent_launch(const void* q, const void* k, const void* v,
+                                         const float* g, float* state, void* o, int B, int H,
+                                         int T, int dk, int dv, bool bf16, cudaStream_t stream);
+
+// SW-SKA prefill on CUDA cores (fp32 FMA, online softmax)
+cudaError_t swska_prefill_simt_launch(const void* q, const void* k, const void* v, void* o,
+                                      int B, int H, int T, int dk, int dv, int window,
+                                      float scale, bool bf16, cudaStream_t stream);
+
+// SW-SKA decode: ring-buffer write + split-window attention combined across a cluster
+cudaError_t swska_decode_launch(const void* q, const void* k_new, const void* v_new,
+                                void* k_cache, void* v_cache, const int64_t* pos, void* o,
+                                int N, int H, int dk, int dv, int window, float scale, bool bf16,
+                                cudaStream_t stream);
+// read and clear the "bounded wait expired" flag of the decode attention kernel
+unsigned swska_decode_take_timeout_flag();
+
+}  // namespace rod

@@ -1,0 +1,136 @@
+// rod_api.cu -- the C ABI of librod.so (declared in include/rod.h): host-side argument
+// validation, then dispatch to the kernels. Nothing here computes on the data.
+#include <math.h>
+#include <stdint.h>
+
+#include <atomic>
+
+#include "../../include/rod.h"
+#include "kernels.h"
+
+namespace rod {
+static std::atomic<uint64_t> g_launches{0};
+void note_launches(unsigned n) { g_launches.fetch_add(n, std::memory_order_relaxed); }
+}  // namespace rod
+
+namespace {
+
+thread_local int t_last_cuda_error = 0;
+
+bool dim_ok(int d) { return d == 16 || d == 32 || d == 64 || d == 128; }
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+bool dtype_ok(int dt) { return dt == ROD_BF16 || dt == ROD_FP32; }
+
+int from_cuda(cudaError_t e) {
+    if (e == cudaSuccess) return ROD_OK;
+    t_last_cuda_error = (int)e;
+    return ROD_ERR_CUDA;
+}
+
+float resolve_scale(float scale, int dk) { return scale > 0.f ? scale : 1.0f / sqrtf((float)dk); }
+
+}  // namespace
+
+extern "C" {
+
+const char* rod_status_string(int status) {
+    switch (status) {
+        case ROD_OK: return "ok";
+        case ROD_ERR_NULL: return "null pointer argument";
+        case ROD_ERR_SHAPE: return "unsupported or out-of-range size";
+        case ROD_ERR_ALIGN: return "pointer not 16-byte aligned";
+        case ROD_ERR_DTYPE: return "unsupported dtype";
+        case ROD_ERR_WORKSPACE: return "workspace missing or too small";
+        case ROD_ERR_CUDA: return "CUDA error";
+        case ROD_ERR_TIMEOUT: return "a bounded device wait expired";
+    }
+    return "unknown status";
+}
+
+int rod_last_cuda_error(void) { return t_last_cuda_error; }
+
+int rod_abi_version(void) { return 1; }
+
+uint64_t rod_launch_count(void) { return rod::g_launches.load(std::memory_order_relaxed); }
+
+int rod_check(void* stream) {
+    cudaError_t e = cudaStreamSynchronize(static_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return from_cuda(e);
+    const unsigned flags = rod::swska_decode_take_timeout_flag();
+    if (flags) return ROD_ERR_TIMEOUT;
+    return from_cuda(cudaGetLastError());
+}
+
+size_t rod_gla_prefill_workspace_size(int B, int H, int T, int dk, int dv, int chunk, int dtype) {
+    if (B < 0 || H < 0 || T < 0 || !dim_ok(dk) || !dim_ok(dv) || !dtype_ok(dtype)) return 0;
+    if (chunk < 16 || chunk > 128 || chunk % 16 != 0) return 0;
+    return 0;
+}
+
+int rod_gla_prefill(const void* q, const void* k, const void* v, const float* g, float* state,
+                    void* o, int B, int H, int T, int dk, int dv, int chunk, int dtype,
+                    void* workspace, size_t ws_bytes, void* stream) {
+    if (!dtype_ok(dtype)) return ROD_ERR_DTYPE;
+    if (B < 0 || H < 0 || T < 0 || !dim_ok(dk) || !dim_ok(dv)) return ROD_ERR_SHAPE;
+    if (chunk < 16 || chunk > 128 || chunk % 16 != 0) return ROD_ERR_SHAPE;
+    if ((int64_t)B * H == 0 || T == 0) return ROD_OK;
+    if (!q || !k || !v || !g || !state || !o) return ROD_ERR_NULL;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(g) || !aligned16(state) ||
+        !aligned16(o))
+        return ROD_ERR_ALIGN;
+    const size_t need = rod_gla_prefill_workspace_size(B, H, T, dk, dv, chunk, dtype);
+    if (need > 0 && (!workspace || ws_bytes < need)) return ROD_ERR_WORKSPACE;
+    (void)workspace;
+    (void)ws_bytes;
+    return from_cuda(rod::gla_prefill_recurrent_launch(q, k, v, g, state, o, B, H, T, dk, dv,
+                                                       dtype == ROD_BF16,
+                                                       static_cast<cudaStream_t>(stream)));
+}
+
+int rod_gla_decode_step(const void* q, const void* k, const void* v, const float* g,
+                        float* state, void* o, int N, int H, int dk, int dv, int dtype,
+                        void* stream) {
+    if (!dtype_ok(dtype)) return ROD_ERR_DTYPE;
+    if (N < 0 || H < 0 || !dim_ok(dk) || !dim_ok(dv)) return ROD_ERR_SHAPE;
+    if ((int64_t)N * H == 0) return ROD_OK;
+    if (!q || !k || !v || !g || !state || !o) return ROD_ERR_NULL;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(g) || !aligned16(state) ||
+        !aligned16(o))
+        return ROD_ERR_ALIGN;
+    return from_cuda(rod::gla_decode_launch(q, k, v, g, state, o, N, H, dk, dv,
+                                            dtype == ROD_BF16, static_cast<cudaStream_t>(stream)));
+}
+
+int rod_swska_prefill(const void* q, const void* k, const void* v, void* o, int B, int H,
+                      int T, int dk, int dv, int window, float scale, int dtype, void* stream) {
+    if (!dtype_ok(dtype)) return ROD_ERR_DTYPE;
+    if (B < 0 || H < 0 || T < 0 || H > 64 || window < 1 || !dim_ok(dk) || !dim_ok(dv))
+        return ROD_ERR_SHAPE;
+    if (!(scale == scale) || isinf(scale)) return ROD_ERR_SHAPE;
+    if ((int64_t)B * H == 0 || T == 0) return ROD_OK;
+    if (!q || !k || !v || !o) return ROD_ERR_NULL;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o)) return ROD_ERR_ALIGN;
+    return from_cuda(rod::swska_prefill_simt_launch(q, k, v, o, B, H, T, dk, dv, window,
+                                                    resolve_scale(scale, dk), dtype == ROD_BF16,
+                                                    static_cast<cudaStream_t>(stream)));
+}
+
+int rod_swska_decode(const void* q, const void* k_new, const void* v_new, void* k_cache,
+                     void* v_cache, const int64_t* pos, void* o, int N, int H, int dk, int dv,
+                     int window, float scale, int dtype, void* stream) {
+    if (!dtype_ok(dtype)) return ROD_ERR_DTYPE;
+    if (N < 0 || H < 1 || H > 64 || window < 1 || !dim_ok(dk) || !dim_ok(dv))
+        return ROD_ERR_SHAPE;
+    if (!(scale == scale) || isinf(scale)) return ROD_ERR_SHAPE;
+    if (N == 0) return ROD_OK;
+    if (!q || !k_new || !v_new || !k_cache || !v_cache || !pos || !o) return ROD_ERR_NULL;
+    if (!aligned16(q) || !aligned16(k_new) || !aligned16(v_new) || !aligned16(k_cache) ||
+        !aligned16(v_cache) || !aligned16(pos) || !aligned16(o))
+        return ROD_ERR_ALIGN;
+    return from_cuda(rod::swska_decode_launch(q, k_new, v_new, k_cache, v_cache, pos, o, N, H, dk,
+                                              dv, window, resolve_scale(scale, dk),
+                                              dtype == ROD_BF16,
+                                              static_cast<cudaStream_t>(stream)));
+}
+
+}  // extern "C"

@@ -1,0 +1,134 @@
+"""C-ABI checks that need no GPU: librod.so loads, exports every entry point include/rod.h
+declares, and rejects bad arguments on the host with the documented status codes before
+anything is launched (no call below reaches a kernel)."""
+import ctypes
+import os
+import re
+import subprocess
+
+import pytest
+
+import sliding_window_attention_chunked_b200 as rod
+from sliding_window_attention_chunked_b200 import build as rbuild
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "rod.h")
+
+OK, NULL, SHAPE, ALIGN, DTYPE, WS, CUDA, TIMEOUT = 0, -1, -2, -3, -4, -5, -6, -7
+
+
+@pytest.fixture(scope="module")
+def lib():
+    rbuild.build()
+    return rod.load_library()
+
+
+def declared_symbols():
+    src = open(HEADER).read()
+    return re.findall(r"ROD_API\s+[\w\s\*]+?\b(rod_\w+)\s*\(", src)
+
+
+def test_header_declares_the_four_entry_points():
+    names = set(declared_symbols())
+    for n in ("rod_gla_prefill", "rod_gla_decode_step", "rod_swska_prefill", "rod_swska_decode",
+              "rod_gla_prefill_workspace_size", "rod_check", "rod_status_string"):
+        assert n in names
+
+
+def test_library_exports_every_declared_symbol(lib):
+    names = declared_symbols()
+    assert names
+    out = subprocess.run(["nm", "-D", "--defined-only", rod.library_path()], check=True,
+                         capture_output=True, text=True).stdout
+    exported = {line.split()[-1] for line in out.splitlines() if line.strip()}
+    for n in names:
+        assert n in exported, f"{n} declared in rod.h but not exported"
+        assert getattr(lib, n) is not None
+    # the library exports exactly the declared ABI (no C++ or CUDA-runtime internals)
+    assert exported == set(names), sorted(exported ^ set(names))
+
+
+def test_status_strings_and_version(lib):
+    for st in (OK, NULL, SHAPE, ALIGN, DTYPE, WS, CUDA, TIMEOUT):
+        assert lib.rod_status_string(st)
+    assert lib.rod_status_string(12345) == b"unknown status"
+    assert lib.rod_abi_version() == 1
+
+
+P = ctypes.c_void_p(0x10000)   # aligned, never dereferenced (every call below fails first)
+MIS = ctypes.c_void_p(0x10008)  # 8-byte aligned only
+
+
+def gla(lib, **kw):
+    a = dict(q=P, k=P, v=P, g=P, s=P, o=P, B=1, H=2, T=8, dk=16, dv=32, chunk=32, dtype=2,
+             ws=None, wsb=0)
+    a.update(kw)
+    return lib.rod_gla_prefill(a["q"], a["k"], a["v"], a["g"], a["s"], a["o"], a["B"], a["H"],
+                               a["T"], a["dk"], a["dv"], a["chunk"], a["dtype"], a["ws"],
+                               a["wsb"], None)
+
+
+def test_gla_prefill_validation(lib):
+    assert gla(lib, dtype=3) == DTYPE
+    assert gla(lib, dk=24) == SHAPE
+    assert gla(lib, dv=256) == SHAPE
+    assert gla(lib, chunk=24) == SHAPE
+    assert gla(lib, chunk=144) == SHAPE
+    assert gla(lib, T=-1) == SHAPE
+    assert gla(lib, q=None) == NULL
+    assert gla(lib, g=None) == NULL
+    assert gla(lib, o=MIS) == ALIGN
+    assert gla(lib, T=0, q=None) == OK          # empty: a no-op that touches nothing
+    assert gla(lib, B=0, q=None) == OK
+
+
+def test_gla_prefill_workspace_size_is_deterministic(lib):
+    a = lib.rod_gla_prefill_workspace_size(4, 16, 4096, 128, 128, 64, 1)
+    b = lib.rod_gla_prefill_workspace_size(4, 16, 4096, 128, 128, 64, 1)
+    assert a == b
+    assert lib.rod_gla_prefill_workspace_size(4, 16, 4096, 100, 128, 64, 1) == 0
+
+
+def test_gla_decode_validation(lib):
+    f = lib.rod_gla_decode_step
+    assert f(P, P, P, P, P, P, 4, 2, 16, 32, 7, None) == DTYPE
+    assert f(P, P, P, P, P, P, 4, 2, 48, 32, 2, None) == SHAPE
+    assert f(None, P, P, P, P, P, 4, 2, 16, 32, 2, None) == NULL
+    assert f(P, P, P, P, MIS, P, 4, 2, 16, 32, 2, None) == ALIGN
+    assert f(None, None, None, None, None, None, 0, 2, 16, 32, 2, None) == OK
+
+
+def test_swska_prefill_validation(lib):
+    f = lib.rod_swska_prefill
+    assert f(P, P, P, P, 1, 2, 8, 16, 32, 0, 0.0, 2, None) == SHAPE      # window < 1
+    assert f(P, P, P, P, 1, 65, 8, 16, 32, 4, 0.0, 2, None) == SHAPE     # too many heads
+    assert f(P, P, P, P, 1, 2, 8, 16, 32, 4, float("nan"), 2, None) == SHAPE
+    assert f(P, P, P, P, 1, 2, 8, 16, 32, 4, 0.0, 0, None) == DTYPE
+    assert f(P, None, P, P, 1, 2, 8, 16, 32, 4, 0.0, 2, None) == NULL
+    assert f(P, P, MIS, P, 1, 2, 8, 16, 32, 4, 0.0, 2, None) == ALIGN
+    assert f(None, None, None, None, 1, 2, 0, 16, 32, 4, 0.0, 2, None) == OK
+
+
+def test_swska_decode_validation(lib):
+    f = lib.rod_swska_decode
+    assert f(P, P, P, P, P, P, P, 4, 2, 16, 32, 0, 0.0, 2, None) == SHAPE
+    assert f(P, P, P, P, P, P, P, 4, 0, 16, 32, 8, 0.0, 2, None) == SHAPE
+    assert f(P, P, P, P, P, None, P, 4, 2, 16, 32, 8, 0.0, 2, None) == NULL
+    assert f(P, P, P, P, MIS, P, P, 4, 2, 16, 32, 8, 0.0, 2, None) == ALIGN
+    assert f(P, P, P, P, P, P, P, 4, 2, 16, 32, 8, 0.0, 9, None) == DTYPE
+    assert f(None, None, None, None, None, None, None, 0, 2, 16, 32, 8, 0.0, 2, None) == OK
+
+
+def test_binding_refuses_cpu_tensors():
+    import torch
+    q = torch.zeros(1, 2, 8, 16)
+    with pytest.raises(ValueError, match="CUDA"):
+        rod.swska_prefill(q, torch.zeros(1, 8, 16), torch.zeros(1, 2, 8, 32), 4)
+
+
+def test_binding_fails_loudly_without_library(monkeypatch, tmp_path):
+    from sliding_window_attention_chunked_b200 import _binding
+    monkeypatch.setattr(_binding, "_lib", None)
+    monkeypatch.setattr(_binding, "_PKG", str(tmp_path))
+    with pytest.raises(RuntimeError, match="not built"):
+        _binding.load_library()

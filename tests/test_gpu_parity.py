@@ -1,0 +1,289 @@
+"""GPU parity: every entry point of librod.so against the fp64 CPU oracle on the same seeded
+inputs, through the C ABI (via the ctypes binding), with the tolerances in tests/parity.py.
+
+Sizes: small cases the oracle finishes in seconds that still span several tiles and a ragged
+tail, the edge cases of the method (T = 1, T < chunk, W = 1, W >= T, g = 0, g = 1, partially
+filled decode windows, a negative decode position), and the full workload sizes in the launch
+configuration the benchmark times, checked on sampled outputs the oracle computes one by one.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import sliding_window_attention_chunked_b200 as rod
+from sliding_window_attention_chunked_b200 import workloads as wl
+
+from .parity import compare
+
+pytestmark = pytest.mark.gpu
+DEV = "cuda"
+
+
+def _cuda(*ts):
+    return [t.to(DEV) for t in ts]
+
+
+# ------------------------------------------------------------------------------------------
+# gated linear recurrence: prefill
+# ------------------------------------------------------------------------------------------
+
+
+def _gla_check(B, H, T, dk, dv, chunk, dtype, dist, seed=0, state0_scale=0.0, gate=None):
+    q, k, v, g = wl.gla_inputs(B, H, T, dk, dv, dist=dist, seed=seed, dtype=dtype)
+    if gate is not None:
+        g = torch.full_like(g, float(gate))
+    S0 = torch.randn(B, H, dk, dv, generator=torch.Generator().manual_seed(seed + 7)) * state0_scale
+    o_ref, S_ref = oracle.gla_prefill(q, k, v, g, S0)
+    qd, kd, vd, gd = _cuda(q, k, v, g)
+    S = S0.to(DEV).contiguous()
+    o = rod.gla_prefill(qd, kd, vd, gd, S, chunk=chunk)
+    rod.check()
+    compare(o, o_ref, dtype, "o")
+    compare(S, S_ref, dtype, "state")
+    return o, S
+
+
+def test_gla_prefill_tiny_fp32():
+    d = wl.WORKLOADS["tiny_fp32"].dims
+    _gla_check(d["B"], d["H"], d["T"], d["dk"], d["dv"], d["chunk"], "fp32", "tiny")
+
+
+@pytest.mark.parametrize("dk,dv", [(16, 32), (32, 16), (64, 64), (128, 128), (16, 128)])
+def test_gla_prefill_fp32_dims(dk, dv):
+    _gla_check(2, 2, 77, dk, dv, 32, "fp32", "tiny", seed=dk + dv, state0_scale=0.5)
+
+
+def test_gla_prefill_bf16_ragged_with_initial_state():
+    _gla_check(2, 3, 1000, 128, 128, 64, "bf16", "l2", seed=1, state0_scale=0.3)
+
+
+@pytest.mark.parametrize("T", [1, 17, 64, 65])
+def test_gla_prefill_bf16_short(T):
+    _gla_check(1, 2, T, 128, 128, 64, "bf16", "l2", seed=T)
+
+
+@pytest.mark.parametrize("chunk", [16, 32, 128])
+def test_gla_prefill_bf16_chunk_sizes(chunk):
+    _gla_check(1, 2, 300, 128, 128, chunk, "bf16", "l2", seed=chunk)
+
+
+def test_gla_prefill_gate_zero_resets():
+    _gla_check(1, 2, 130, 128, 64, 64, "bf16", "l2", seed=3, gate=0.0)
+
+
+def test_gla_prefill_gate_one_linear_attention():
+    _gla_check(1, 2, 130, 64, 128, 64, "bf16", "l2", seed=4, gate=1.0)
+
+
+def test_gla_prefill_split_hands_off_state():
+    B, H, T, d = 1, 2, 500, 128
+    q, k, v, g = [t.to(DEV) for t in wl.gla_inputs(B, H, T, d, d, dist="l2", seed=5)]
+    S = torch.zeros(B, H, d, d, device=DEV)
+    o = rod.gla_prefill(q, k, v, g, S)
+    S2 = torch.zeros_like(S)
+    o1 = rod.gla_prefill(q[:, :, :211].contiguous(), k[:, :, :211].contiguous(),
+                         v[:, :, :211].contiguous(), g[:, :, :211].contiguous(), S2)
+    o2 = rod.gla_prefill(q[:, :, 211:].contiguous(), k[:, :, 211:].contiguous(),
+                         v[:, :, 211:].contiguous(), g[:, :, 211:].contiguous(), S2)
+    rod.check()
+    compare(torch.cat([o1, o2], dim=2), o.float(), "bf16", "split o")
+    compare(S2, S, "bf16", "split state")
+
+
+def test_gla_prefill_full_workload():
+    """B=4, T=4096, H=16, d=128, chunk 64, bf16 in / fp32 state: every output vs the oracle."""
+    d = wl.WORKLOADS["gla_prefill_b4_t4096"].dims
+    _gla_check(d["B"], d["H"], d["T"], d["dk"], d["dv"], d["chunk"], "bf16", "l2")
+
+
+# ------------------------------------------------------------------------------------------
+# gated linear recurrence: decode
+# ------------------------------------------------------------------------------------------
+
+
+@pytest.mark.parametrize("dtype,N,H,dk,dv", [("fp32", 3, 2, 16, 32), ("fp32", 5, 3, 128, 64),
+                                             ("bf16", 256, 16, 128, 128)])
+def test_gla_decode_step(dtype, N, H, dk, dv):
+    dd = wl.decode_inputs(N, H, dk, dv, 8, seed=N + dk, dtype=dtype)
+    o_ref, S_ref = oracle.gla_decode_step(dd["q"], dd["k"], dd["v"], dd["g"], dd["state"])
+    q, k, v, g, S = _cuda(dd["q"], dd["k"], dd["v"], dd["g"], dd["state"])
+    o = rod.gla_decode_step(q, k, v, g, S)
+    rod.check()
+    compare(o, o_ref, dtype, "o")
+    compare(S, S_ref, dtype, "state")
+
+
+def test_gla_decode_steps_equal_prefill_fp32():
+    B, H, T, dk, dv = 2, 2, 40, 32, 16
+    q, k, v, g = [t.to(DEV) for t in wl.gla_inputs(B, H, T, dk, dv, dist="tiny", seed=9,
+                                                   dtype="fp32")]
+    S_pre = torch.zeros(B, H, dk, dv, device=DEV)
+    o_pre = rod.gla_prefill(q, k, v, g, S_pre, chunk=16)
+    S = torch.zeros_like(S_pre)
+    outs = [rod.gla_decode_step(q[:, :, t].contiguous(), k[:, :, t].contiguous(),
+                                v[:, :, t].contiguous(), g[:, :, t].contiguous(), S)
+            for t in range(T)]
+    rod.check()
+    compare(torch.stack(outs, dim=2), o_pre, "fp32", "decode vs prefill o")
+    compare(S, S_pre, "fp32", "decode vs prefill state")
+
+
+# ------------------------------------------------------------------------------------------
+# SW-SKA prefill
+# ------------------------------------------------------------------------------------------
+
+
+def _ska_check(B, H, T, dk, dv, W, dtype, dist, seed=0, rows=None, scale=None):
+    q, k, v = wl.swska_inputs(B, H, T, dk, dv, dist=dist, seed=seed, dtype=dtype)
+    qd, kd, vd = _cuda(q, k, v)
+    o = rod.swska_prefill(qd, kd, vd, W, scale=scale)
+    rod.check()
+    if rows is None:
+        ref = oracle.swska_prefill(q, k, v, W, scale=scale)
+        compare(o, ref, dtype, "o")
+    else:
+        ref = oracle.swska_prefill(q, k, v, W, scale=scale, rows=rows)
+        compare(o.reshape(-1, dv)[torch.as_tensor(rows, device=DEV)], ref, dtype, "o rows")
+    return o
+
+
+def test_swska_prefill_tiny_fp32():
+    d = wl.WORKLOADS["tiny_fp32"].dims
+    _ska_check(d["B"], d["H"], d["T"], d["dk"], d["dv"], d["window"], "fp32", "tiny")
+
+
+@pytest.mark.parametrize("dk,dv,W", [(16, 32, 1), (32, 16, 7), (64, 64, 100), (128, 128, 300),
+                                     (16, 128, 1000)])
+def test_swska_prefill_fp32_dims(dk, dv, W):
+    _ska_check(2, 2, 333, dk, dv, W, "fp32", "tiny", seed=dk + W)
+
+
+def test_swska_prefill_bf16_ragged():
+    _ska_check(2, 3, 1500, 128, 128, 300, "bf16", "normal", seed=2)
+
+
+@pytest.mark.parametrize("T,W", [(1, 4096), (130, 1), (200, 4096), (700, 129), (700, 128)])
+def test_swska_prefill_bf16_edges(T, W):
+    _ska_check(1, 2, T, 128, 128, W, "bf16", "normal", seed=T + W)
+
+
+def test_swska_prefill_window_one_is_v():
+    q, k, v = [t.to(DEV) for t in wl.swska_inputs(1, 2, 257, 128, 128, seed=3)]
+    o = rod.swska_prefill(q, k, v, 1)
+    rod.check()
+    assert torch.equal(o, v)
+
+
+def test_swska_prefill_full_workload_sampled():
+    """B=2, T=32768, H=16, d=128, W=4096, scale 1/sqrt(128): the whole launch runs; the first
+    W rows of (b=0, h=0) (sub-sampled) and random rows elsewhere are checked one by one."""
+    d = wl.WORKLOADS["swska_prefill_b2_t32768"].dims
+    B, H, T, W = d["B"], d["H"], d["T"], d["window"]
+    r = np.random.default_rng(0)
+    rows = np.concatenate([np.arange(0, W + 256, 37),
+                           r.integers(0, B * H * T, 512),
+                           [B * H * T - 1, T - 1, T, (B * H - 1) * T]])
+    _ska_check(B, H, T, d["dk"], d["dv"], W, "bf16", "normal", rows=np.unique(rows))
+
+
+# ------------------------------------------------------------------------------------------
+# SW-SKA decode (ring buffer)
+# ------------------------------------------------------------------------------------------
+
+
+def _ska_decode_check(N, H, dk, dv, W, dtype, full, seed=0, check_n=None):
+    dd = wl.decode_inputs(N, H, dk, dv, W, seed=seed, dtype=dtype, full=full)
+    sq, kn, vn, kc, vc, pos = _cuda(dd["sq"], dd["k_new"], dd["v_new"], dd["k_cache"],
+                                    dd["v_cache"], dd["pos"])
+    o = rod.swska_decode(sq, kn, vn, kc, vc, pos, W)
+    rod.check()
+    sel = np.arange(N) if check_n is None else np.unique(
+        np.concatenate([np.arange(min(4, N)), np.random.default_rng(seed).integers(0, N, check_n)]))
+    ref, kc_ref, vc_ref = oracle.swska_decode(dd["sq"][sel], dd["k_new"][sel], dd["v_new"][sel],
+                                              dd["k_cache"][sel], dd["v_cache"][sel],
+                                              dd["pos"][sel], W)
+    compare(o[torch.as_tensor(sel, device=DEV)], ref, dtype, "o")
+    # the ring-buffer write is a copy: bit-exact
+    s = torch.as_tensor(sel, device=DEV)
+    np.testing.assert_array_equal(kc[s].float().cpu().numpy(), kc_ref)
+    np.testing.assert_array_equal(vc[s].float().cpu().numpy(), vc_ref)
+
+
+def test_swska_decode_tiny_fp32():
+    _ska_decode_check(5, 2, 16, 32, 64, "fp32", full=False, seed=1)
+
+
+@pytest.mark.parametrize("W", [600, 1030])
+def test_swska_decode_bf16_cluster_split(W):
+    _ska_decode_check(7, 4, 128, 128, W, "bf16", full=False, seed=W)
+    _ska_decode_check(7, 4, 128, 128, W, "bf16", full=True, seed=W + 1)
+
+
+def test_swska_decode_full_workload_sampled():
+    d = wl.WORKLOADS["decode_n256"].dims
+    _ska_decode_check(d["N"], d["H"], d["dk"], d["dv"], d["window"], "bf16", full=True,
+                      check_n=20)
+
+
+def test_swska_decode_negative_position_gives_nan_and_keeps_cache():
+    N, H, d, W = 3, 2, 64, 32
+    dd = wl.decode_inputs(N, H, d, d, W, seed=5, dtype="bf16", full=False)
+    pos = dd["pos"].clone()
+    pos[1] = -5
+    sq, kn, vn, kc, vc, p = _cuda(dd["sq"], dd["k_new"], dd["v_new"], dd["k_cache"],
+                                  dd["v_cache"], pos)
+    kc0, vc0 = kc.clone(), vc.clone()
+    o = rod.swska_decode(sq, kn, vn, kc, vc, p, W)
+    rod.check()
+    assert torch.isnan(o[1].float()).all()
+    assert torch.isfinite(o[0].float()).all() and torch.isfinite(o[2].float()).all()
+    assert torch.equal(kc[1], kc0[1]) and torch.equal(vc[1], vc0[1])
+
+
+def test_swska_decode_equals_prefill_rows():
+    """Fill the ring from a prefix of one sequence and decode position P: equals prefill row P."""
+    H, d, W, T = 4, 128, 96, 400
+    q, k, v = [t.to(DEV) for t in wl.swska_inputs(1, H, T, d, d, seed=8)]
+    o_pre = rod.swska_prefill(q, k, v, W)
+    positions = [0, 5, 95, 96, 97, 250, 399]
+    N = len(positions)
+    kc = torch.zeros(N, W, d, device=DEV, dtype=q.dtype)
+    vc = torch.zeros(N, H, W, d, device=DEV, dtype=q.dtype)
+    for n, P in enumerate(positions):
+        for p in range(max(0, P - W + 1), P):
+            kc[n, p % W] = k[0, p]
+            vc[n, :, p % W] = v[0, :, p]
+    P = torch.tensor(positions, device=DEV)
+    o = rod.swska_decode(q[0][:, P].transpose(0, 1).contiguous(), k[0, P].contiguous(),
+                         v[0][:, P].transpose(0, 1).contiguous(), kc, vc, P, W)
+    rod.check()
+    compare(o, o_pre[0][:, P].transpose(0, 1).float(), "bf16", "decode vs prefill")
+
+
+# ------------------------------------------------------------------------------------------
+# long-context stack: one layer of each kind at full length, sampled
+# ------------------------------------------------------------------------------------------
+
+
+def test_stack_layers_full_length_sampled():
+    d = wl.WORKLOADS["stack_t131072"].dims
+    B, H, T, dk, dv, W = d["B"], d["H"], d["T"], d["dk"], d["dv"], d["window"]
+    # layer 0: recurrence, every head on the GPU; head 0 and head H-1 vs the oracle in full
+    q, k, v, g = wl.stack_layer_inputs(0, B, H, T, dk, dv, device=DEV)
+    S = torch.zeros(B, H, dk, dv, device=DEV)
+    o = rod.gla_prefill(q, k, v, g, S, chunk=d["chunk"])
+    rod.check()
+    for h in (0, H - 1):
+        o_ref, S_ref = oracle.gla_prefill(q[:, h:h + 1], k[:, h:h + 1], v[:, h:h + 1], g[:, h:h + 1])
+        compare(o[:, h:h + 1], o_ref, "bf16", f"stack gla head {h}")
+        compare(S[:, h:h + 1], S_ref, "bf16", f"stack gla state head {h}")
+    del q, k, v, g, o
+    # layer 1: SW-SKA, sampled rows
+    q, k, v = wl.stack_layer_inputs(1, B, H, T, dk, dv, device=DEV)
+    o = rod.swska_prefill(q, k, v, W)
+    rod.check()
+    rows = np.unique(np.concatenate([np.arange(0, 300, 7),
+                                     np.random.default_rng(1).integers(0, B * H * T, 400)]))
+    ref = oracle.swska_prefill(q, k, v, W, rows=rows)
+    compare(o.reshape(-1, dv)[torch.as_tensor(rows, device=DEV)], ref, "bf16", "stack swska")
