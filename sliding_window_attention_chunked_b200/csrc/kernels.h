@@ -3,6 +3,7 @@
 // returns the launch status.
 #pragma once
 
+#include <cuda.h>
 #include <cuda_runtime.h>
 #include <stddef.h>
 #include <stdint.h>
@@ -26,6 +27,16 @@ cudaError_t gla_prefill_recurrent_launch(const void* q, const void* k, const voi
 cudaError_t swska_prefill_simt_launch(const void* q, const void* k, const void* v, void* o,
                                       int B, int H, int T, int dk, int dv, int window,
                                       float scale, bool bf16, cudaStream_t stream);
+
+// SW-SKA prefill on tcgen05 tensor cores (bf16, dk = dv = 128, T >= 128)
+bool swska_prefill_tc_supported(int H, int T, int dk, int dv);
+cudaError_t swska_prefill_tc_launch(const void* q, const void* k, const void* v, void* o, int B,
+                                    int H, int T, int window, float scale, cudaStream_t stream);
+unsigned swska_prefill_tc_take_timeout_flag();
+
+// TMA descriptor for a 3-D bf16 tensor [d2][d1][d0], boxes of box1 x box0, 128-byte swizzle
+cudaError_t make_tmap_bf16_3d(CUtensorMap* map, const void* base, uint64_t d0, uint64_t d1,
+                              uint64_t d2, uint32_t box0, uint32_t box1);
 
 // SW-SKA decode: ring-buffer write + split-window attention combined across a cluster
 cudaError_t swska_decode_launch(const void* q, const void* k_new, const void* v_new,

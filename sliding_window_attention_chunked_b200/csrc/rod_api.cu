@@ -56,7 +56,8 @@ uint64_t rod_launch_count(void) { return rod::g_launches.load(std::memory_order_
 int rod_check(void* stream) {
     cudaError_t e = cudaStreamSynchronize(static_cast<cudaStream_t>(stream));
     if (e != cudaSuccess) return from_cuda(e);
-    const unsigned flags = rod::swska_decode_take_timeout_flag();
+    const unsigned flags = rod::swska_decode_take_timeout_flag() |
+                           rod::swska_prefill_tc_take_timeout_flag();
     if (flags) return ROD_ERR_TIMEOUT;
     return from_cuda(cudaGetLastError());
 }
@@ -110,9 +111,14 @@ int rod_swska_prefill(const void* q, const void* k, const void* v, void* o, int 
     if ((int64_t)B * H == 0 || T == 0) return ROD_OK;
     if (!q || !k || !v || !o) return ROD_ERR_NULL;
     if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o)) return ROD_ERR_ALIGN;
+    const cudaStream_t s = static_cast<cudaStream_t>(stream);
+    // bf16 with 128-wide heads runs on the tensor cores; fp32 (exact FMA) and the small head
+    // dims run on the CUDA-core kernel
+    if (dtype == ROD_BF16 && rod::swska_prefill_tc_supported(H, T, dk, dv))
+        return from_cuda(rod::swska_prefill_tc_launch(q, k, v, o, B, H, T, window,
+                                                      resolve_scale(scale, dk), s));
     return from_cuda(rod::swska_prefill_simt_launch(q, k, v, o, B, H, T, dk, dv, window,
-                                                    resolve_scale(scale, dk), dtype == ROD_BF16,
-                                                    static_cast<cudaStream_t>(stream)));
+                                                    resolve_scale(scale, dk), dtype == ROD_BF16, s));
 }
 
 int rod_swska_decode(const void* q, const void* k_new, const void* v_new, void* k_cache,

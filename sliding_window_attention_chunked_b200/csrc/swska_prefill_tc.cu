@@ -1,0 +1,350 @@
+// swska_prefill_tc.cu -- SW-SKA prefill on the 5th-generation tensor cores (tcgen05, TMEM,
+// TMA), bf16 in / fp32 accumulate, head dim 128.
+//
+//   o[b,h,t] = sum_{j=max(0,t-W+1)}^{t} softmax_j(scale * q[b,h,t] . k[b,j]) v[b,h,j]
+// (CodeFuse Rodimus* article, Fig. 4 / SKA paragraph: one key matrix shared by all heads,
+// per-head values; setup blog §3: the window holds the most recent W tokens; SALA blog §2.1
+// and §3.2: block-wise windowed attention, each query block visiting only the key blocks of its
+// window -- here with a per-element causal/window mask on the two edge blocks.)
+//
+// One CTA computes a 128-query tile for a PAIR of heads of one sequence (with an odd head
+// count the last pair computes its single head twice and stores it once). Each shared key tile
+// is brought into shared memory once by TMA and feeds both heads' score MMAs (the pair's
+// remaining reuse of K across the other heads goes through L2). Warp roles (320 threads):
+//   warps 0-3   softmax warpgroup of head 0 (thread i owns query row i = TMEM lane i)
+//   warps 4-7   softmax warpgroup of head 1
+//   warp  8     TMA producer: Q once, then K_j, V0_j, V1_j into a ring of 32 KB slots
+//   warp  9     TMEM allocator and the single MMA-issuing thread
+// TMEM (512 columns): S0 | O0 | S1 | O1, 128 columns each. S_h = Q_h K_j^T is read by the
+// softmax warps, which write P_h (bf16, packed two per column) over the first 64 columns of
+// S_h; O_h += P_h V_h,j then reads P_h straight from TMEM (A operand in TMEM). The issue order
+//   S0(0) S1(0) | PV0(j) S0(j+1) PV1(j) S1(j+1) | ...
+// lets each head's softmax run while the tensor core works on the other head. Softmax is in
+// base 2 on scores pre-scaled by scale*log2(e), with lazy rescaling: the running maximum used
+// for the exponent only moves when a row's maximum grows by more than 8 (so P <= 256), and
+// then the O row is rescaled in TMEM by its owning thread. Every wait is bounded; a timeout
+// makes all roles stop, drain their in-flight copies and MMAs, and raise a flag.
+#include <cuda.h>
+#include <math.h>
+
+#include "common.cuh"
+#include "kernels.h"
+#include "tc.cuh"
+
+namespace rod {
+namespace {
+
+__device__ unsigned int g_swska_tc_timeout = 0;
+
+constexpr int BM = 128;                    // queries per tile
+constexpr int BN = 128;                    // keys per tile
+constexpr int HD = 128;                    // head dim (dk = dv)
+constexpr int NSLOT = 4;                   // ring slots
+constexpr int TILE_BYTES = BM * HD * 2;    // 32 KB: one 128 x 128 bf16 tile
+constexpr int HALF_BYTES = TILE_BYTES / 2; // one 128-row x 64-column TMA box
+constexpr int NTHREADS = 320;
+constexpr float kRescaleThreshold = 8.0f;  // log2 units
+
+constexpr int OFF_Q = 0;
+constexpr int OFF_RING = 2 * TILE_BYTES;
+constexpr int OFF_BAR = OFF_RING + NSLOT * TILE_BYTES;
+constexpr int NBAR = 2 * NSLOT + 8;        // full, empty, qfull, sfull[2], pfull[2], odone[2], drain
+constexpr int OFF_MISC = OFF_BAR + 8 * NBAR;
+constexpr int SMEM_BYTES = OFF_MISC + 16 + 1024;  // + slack for 1024-byte alignment
+
+__device__ __forceinline__ bool wait_bar(uint64_t* bar, uint32_t parity, volatile int* abort_flag) {
+    for (uint32_t i = 1;; ++i) {
+        if (mbar_try_wait(bar, parity)) return true;
+        if ((i & 255u) == 0) {
+            if (*abort_flag) return false;
+            if (i >= kWaitLimit) {
+                *abort_flag = 1;
+                atomicExch(&g_swska_tc_timeout, 1u);
+                return false;
+            }
+        }
+    }
+}
+
+__global__ void __maxnreg__(200)
+swska_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                const __grid_constant__ CUtensorMap tm_v, __nv_bfloat16* __restrict__ o, int T,
+                int H, int W, float scale_log2, int n_qtiles) {
+    extern __shared__ unsigned char smem_raw[];
+    unsigned char* smem = reinterpret_cast<unsigned char*>(
+        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+    const int qt = n_qtiles - 1 - (int)blockIdx.x;  // full-window tiles first, short ones last
+    const int hp = blockIdx.y;
+    const int b = blockIdx.z;
+    const int t0 = qt * BM;
+    const int kt_lo = (t0 - W + 1 > 0 ? t0 - W + 1 : 0) / BN;
+    const int kt_hi = t0 / BN;
+    const int n_it = kt_hi - kt_lo + 1;
+
+    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + OFF_BAR);
+    uint64_t* full = bars;
+    uint64_t* empty = bars + NSLOT;
+    uint64_t* qfull = bars + 2 * NSLOT;
+    uint64_t* sfull = qfull + 1;
+    uint64_t* pfull = sfull + 2;
+    uint64_t* odone = pfull + 2;
+    uint64_t* drain = odone + 2;
+    uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + OFF_MISC);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + OFF_MISC + 4);
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < NSLOT; ++s) {
+            mbar_init(&full[s], 1);
+            mbar_init(&empty[s], 1);
+        }
+        mbar_init(qfull, 1);
+        for (int h = 0; h < 2; ++h) {
+            mbar_init(&sfull[h], 1);
+            mbar_init(&pfull[h], 128);
+            mbar_init(&odone[h], 1);
+        }
+        mbar_init(drain, 1);
+        *abort_flag = 0;
+        fence_mbar_init();
+    }
+    if (warp == 9) {
+        tc::tmem_alloc(tmem_holder, 512);
+        tc::tmem_relinquish();
+    }
+    tc::fence_before_sync();
+    __syncthreads();
+    tc::fence_after_sync();
+    const uint32_t tmem = *tmem_holder;
+
+    if (warp == 8) {
+        // ------------------------------- TMA producer -------------------------------
+        if (lane == 0) {
+            tc::tma_prefetch_desc(&tm_q);
+            tc::tma_prefetch_desc(&tm_k);
+            tc::tma_prefetch_desc(&tm_v);
+            mbar_arrive_expect_tx(qfull, 2 * TILE_BYTES);
+            for (int h = 0; h < 2; ++h)
+                for (int half = 0; half < 2; ++half)
+                    tc::tma_load_3d(smem + OFF_Q + h * TILE_BYTES + half * HALF_BYTES, &tm_q,
+                                    half * 64, t0, b * H + min(2 * hp + h, H - 1), qfull);
+            int L = 0;
+            for (; L < 3 * n_it; ++L) {
+                const int slot = L % NSLOT, use = L / NSLOT;
+                if (use > 0 && !wait_bar(&empty[slot], (uint32_t)((use - 1) & 1), abort_flag)) break;
+                const int j = L / 3, which = L % 3, key0 = (kt_lo + j) * BN;
+                unsigned char* dst = smem + OFF_RING + slot * TILE_BYTES;
+                mbar_arrive_expect_tx(&full[slot], TILE_BYTES);
+                for (int half = 0; half < 2; ++half) {
+                    if (which == 0)
+                        tc::tma_load_3d(dst + half * HALF_BYTES, &tm_k, half * 64, key0, b, &full[slot]);
+                    else
+                        tc::tma_load_3d(dst + half * HALF_BYTES, &tm_v, half * 64, key0,
+                                        b * H + min(2 * hp + which - 1, H - 1), &full[slot]);
+                }
+            }
+            // every copy this thread started (loads 0 .. L-1) has landed before the CTA can
+            // leave: the last NSLOT of them are the latest phase of each slot
+            mbar_wait_bounded(qfull, 0, kWaitLimit);
+            for (int Li = (L > NSLOT ? L - NSLOT : 0); Li < L; ++Li)
+                mbar_wait_bounded(&full[Li % NSLOT], (uint32_t)((Li / NSLOT) & 1), kWaitLimit);
+        }
+    } else if (warp == 9) {
+        // ------------------------------- MMA issuer -------------------------------
+        if (lane == 0) {
+            const uint32_t idesc_s = tc::idesc_bf16_f32(BM, BN, 0, 0);  // Q K^T, both K-major
+            const uint32_t idesc_o = tc::idesc_bf16_f32(BM, HD, 0, 1);  // P V, V is MN-major
+            const uint32_t q_base = smem_u32(smem + OFF_Q);
+            // TMEM columns: S_h at 256 h, O_h at 256 h + 128; Q_h at q_base + h * TILE_BYTES
+            auto ring = [&](int L) { return smem_u32(smem + OFF_RING + (L % NSLOT) * TILE_BYTES); };
+            auto acquire = [&](int L) {
+                const bool ok = wait_bar(&full[L % NSLOT], (uint32_t)((L / NSLOT) & 1), abort_flag);
+                tc::fence_after_sync();
+                return ok;
+            };
+            auto issue_s = [&](int h, int L) {
+                const uint32_t bb = ring(L);
+#pragma unroll
+                for (int k = 0; k < HD / 16; ++k) {
+                    const uint32_t koff = (uint32_t)((k / 4) * HALF_BYTES + (k % 4) * 32);
+                    tc::mma_ss(tmem + 256u * h, tc::sdesc_sw128(q_base + h * TILE_BYTES + koff, 16, 1024),
+                               tc::sdesc_sw128(bb + koff, 16, 1024), idesc_s, k > 0);
+                }
+            };
+            auto issue_pv = [&](int h, int L, bool acc) {
+                const uint32_t bb = ring(L);
+#pragma unroll
+                for (int k = 0; k < BN / 16; ++k)
+                    tc::mma_ts(tmem + 256u * h + 128u, tmem + 256u * h + 8u * k,
+                               tc::sdesc_sw128(bb + 2048u * k, HALF_BYTES, 1024),
+                               idesc_o, (acc || k > 0) ? 1u : 0u);
+            };
+            bool ok = wait_bar(qfull, 0, abort_flag);
+            tc::fence_after_sync();
+            if (ok && acquire(0)) {
+                issue_s(0, 0);
+                tc::mma_commit(&sfull[0]);
+                issue_s(1, 0);
+                tc::mma_commit(&sfull[1]);
+                tc::mma_commit(&empty[0]);
+                for (int j = 0; j < n_it; ++j) {
+                    const bool more = j + 1 < n_it;
+                    if (!wait_bar(&pfull[0], (uint32_t)(j & 1), abort_flag)) break;
+                    tc::fence_after_sync();
+                    if (!acquire(3 * j + 1)) break;
+                    issue_pv(0, 3 * j + 1, j > 0);
+                    tc::mma_commit(&empty[(3 * j + 1) % NSLOT]);
+                    if (more) {
+                        if (!acquire(3 * j + 3)) break;
+                        issue_s(0, 3 * j + 3);
+                        tc::mma_commit(&sfull[0]);
+                    } else {
+                        tc::mma_commit(&odone[0]);
+                    }
+                    if (!wait_bar(&pfull[1], (uint32_t)(j & 1), abort_flag)) break;
+                    tc::fence_after_sync();
+                    if (!acquire(3 * j + 2)) break;
+                    issue_pv(1, 3 * j + 2, j > 0);
+                    tc::mma_commit(&empty[(3 * j + 2) % NSLOT]);
+                    if (more) {
+                        issue_s(1, 3 * j + 3);
+                        tc::mma_commit(&sfull[1]);
+                        tc::mma_commit(&empty[(3 * j + 3) % NSLOT]);
+                    } else {
+                        tc::mma_commit(&odone[1]);
+                    }
+                }
+            }
+            // every MMA this thread issued has completed before TMEM is released
+            tc::mma_commit(drain);
+            mbar_wait_bounded(drain, 0, kWaitLimit);
+        }
+    } else {
+        // ------------------------------- softmax warpgroups -------------------------------
+        const int h = warp / 4;                     // head within the pair
+        const int row = threadIdx.x % 128;          // query row == TMEM lane
+        const uint32_t lane_base = (uint32_t)(32 * (warp % 4)) << 16;
+        const uint32_t tS = tmem + 256u * h + lane_base;
+        const uint32_t tO = tS + 128u;
+        const int t = t0 + row;
+        float m_run = -INFINITY, l_run = 0.f;
+        bool ok = true;
+        for (int j = 0; j < n_it; ++j) {
+            if (!wait_bar(&sfull[h], (uint32_t)(j & 1), abort_flag)) { ok = false; break; }
+            tc::fence_after_sync();
+            uint32_t s[BN];  // raw fp32 bits of the score row
+            tc::tmem_ld32(tS + 0, s);
+            tc::tmem_ld32(tS + 32, s + 32);
+            tc::tmem_ld32(tS + 64, s + 64);
+            tc::tmem_ld32(tS + 96, s + 96);
+            tc::tmem_wait_ld();
+            const int key0 = (kt_lo + j) * BN;
+            const bool full_tile = key0 >= t0 + BM - W && key0 + BN - 1 <= t0;
+            if (!full_tile) {
+                const int lo = t - W + 1 - key0, hi = t - key0;  // valid key columns [lo, hi]
+#pragma unroll
+                for (int c = 0; c < BN; ++c)
+                    if (c < lo || c > hi) s[c] = 0xff800000u;  // -inf
+            }
+            float mx = __uint_as_float(s[0]);
+#pragma unroll
+            for (int c = 1; c < BN; ++c) mx = fmaxf(mx, __uint_as_float(s[c]));
+            const float m_tile = mx * scale_log2;
+            const bool need = m_tile > m_run + kRescaleThreshold;
+            if (j > 0 && __any_sync(0xffffffffu, need)) {
+                const float alpha = need ? tc::ex2(m_run - m_tile) : 1.f;
+#pragma unroll
+                for (int cb = 0; cb < HD; cb += 32) {
+                    uint32_t r[32];
+                    tc::tmem_ld32(tO + cb, r);
+                    tc::tmem_wait_ld();
+#pragma unroll
+                    for (int i = 0; i < 32; ++i) r[i] = __float_as_uint(__uint_as_float(r[i]) * alpha);
+                    tc::tmem_st32(tO + cb, r);
+                }
+                tc::tmem_wait_st();
+                l_run *= alpha;
+            }
+            if (need) m_run = m_tile;
+            const float m_use = m_run == -INFINITY ? 0.f : m_run;
+#pragma unroll
+            for (int half = 0; half < 2; ++half) {
+                uint32_t pk[32];
+#pragma unroll
+                for (int i = 0; i < 32; ++i) {
+                    const int c = 64 * half + 2 * i;
+                    const float p0 = tc::ex2(fmaf(__uint_as_float(s[c]), scale_log2, -m_use));
+                    const float p1 = tc::ex2(fmaf(__uint_as_float(s[c + 1]), scale_log2, -m_use));
+                    l_run += p0 + p1;
+                    pk[i] = pack_bf16x2(p0, p1);
+                }
+                tc::tmem_st32(tS + 32u * half, pk);
+            }
+            tc::tmem_wait_st();
+            tc::fence_before_sync();
+            mbar_arrive(&pfull[h]);
+        }
+        // epilogue: O / l -> bf16 rows
+        if (ok && wait_bar(&odone[h], 0, abort_flag)) {
+            tc::fence_after_sync();
+            const float inv = 1.f / l_run;
+            __nv_bfloat16* orow = o + ((int64_t)(b * H + 2 * hp + h) * T + t) * HD;
+#pragma unroll
+            for (int cb = 0; cb < HD; cb += 32) {
+                uint32_t r[32];
+                tc::tmem_ld32(tO + cb, r);
+                tc::tmem_wait_ld();
+                if (t < T && 2 * hp + h < H) {  // an odd H's last pair computes one head twice
+#pragma unroll
+                    for (int i = 0; i < 32; i += 8) {
+                        uint4 u;
+                        u.x = pack_bf16x2(__uint_as_float(r[i + 0]) * inv, __uint_as_float(r[i + 1]) * inv);
+                        u.y = pack_bf16x2(__uint_as_float(r[i + 2]) * inv, __uint_as_float(r[i + 3]) * inv);
+                        u.z = pack_bf16x2(__uint_as_float(r[i + 4]) * inv, __uint_as_float(r[i + 5]) * inv);
+                        u.w = pack_bf16x2(__uint_as_float(r[i + 6]) * inv, __uint_as_float(r[i + 7]) * inv);
+                        *reinterpret_cast<uint4*>(orow + cb + i) = u;
+                    }
+                }
+            }
+        }
+    }
+
+    tc::fence_before_sync();
+    __syncthreads();
+    tc::fence_after_sync();
+    if (warp == 9) tc::tmem_dealloc(tmem, 512);
+}
+
+}  // namespace
+
+bool swska_prefill_tc_supported(int H, int T, int dk, int dv) {
+    return dk == HD && dv == HD && H >= 1 && T >= BM;
+}
+
+cudaError_t swska_prefill_tc_launch(const void* q, const void* k, const void* v, void* o, int B,
+                                    int H, int T, int window, float scale, cudaStream_t stream) {
+    CUtensorMap mq, mk, mv;
+    cudaError_t e;
+    if ((e = make_tmap_bf16_3d(&mq, q, HD, (uint64_t)T, (uint64_t)B * H, 64, BM)) != cudaSuccess) return e;
+    if ((e = make_tmap_bf16_3d(&mk, k, HD, (uint64_t)T, (uint64_t)B, 64, BN)) != cudaSuccess) return e;
+    if ((e = make_tmap_bf16_3d(&mv, v, HD, (uint64_t)T, (uint64_t)B * H, 64, BN)) != cudaSuccess) return e;
+    e = cudaFuncSetAttribute(swska_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
+    if (e != cudaSuccess) return e;
+    const int n_qtiles = (T + BM - 1) / BM;
+    if (B > 65535 || (H + 1) / 2 > 65535) return cudaErrorInvalidConfiguration;
+    dim3 grid((unsigned)n_qtiles, (unsigned)((H + 1) / 2), (unsigned)B);
+    swska_tc_kernel<<<grid, NTHREADS, SMEM_BYTES, stream>>>(
+        mq, mk, mv, static_cast<__nv_bfloat16*>(o), T, H, window, scale * 1.4426950408889634f,
+        n_qtiles);
+    note_launches(1);
+    return cudaGetLastError();
+}
+
+unsigned swska_prefill_tc_take_timeout_flag() {
+    unsigned v = 0, zero = 0;
+    if (cudaMemcpyFromSymbol(&v, g_swska_tc_timeout, sizeof(v)) != cudaSuccess) return 0;
+    cudaMemcpyToSymbol(g_swska_tc_timeout, &zero, sizeof(zero));
+    return v;
+}
+
+}  // namespace rod

@@ -287,3 +287,33 @@ def test_stack_layers_full_length_sampled():
                                      np.random.default_rng(1).integers(0, B * H * T, 400)]))
     ref = oracle.swska_prefill(q, k, v, W, rows=rows)
     compare(o.reshape(-1, dv)[torch.as_tensor(rows, device=DEV)], ref, "bf16", "stack swska")
+
+
+# ------------------------------------------------------------------------------------------
+# tensor-core SW-SKA specifics: lazy rescaling, odd head counts, tile edges, determinism
+# ------------------------------------------------------------------------------------------
+
+
+@pytest.mark.parametrize("qscale", [4.0, 16.0])
+def test_swska_prefill_large_logits_exercise_rescaling(qscale):
+    """Scores with a spread of many units of log2 force the running-maximum rescale path."""
+    B, H, T, d, W = 1, 2, 1100, 128, 700
+    q, k, v = wl.swska_inputs(B, H, T, d, d, seed=21)
+    q = (q.float() * qscale).to(torch.bfloat16)
+    o = rod.swska_prefill(q.to(DEV), k.to(DEV), v.to(DEV), W)
+    rod.check()
+    compare(o, oracle.swska_prefill(q, k, v, W), "bf16", "large logits")
+
+
+@pytest.mark.parametrize("B,H,T,W", [(2, 1, 128, 64), (1, 3, 129, 128), (1, 5, 385, 257),
+                                     (3, 2, 640, 4096)])
+def test_swska_prefill_tile_edges(B, H, T, W):
+    _ska_check(B, H, T, 128, 128, W, "bf16", "normal", seed=B * 1000 + H * 100 + W)
+
+
+def test_swska_prefill_deterministic():
+    q, k, v = [t.to(DEV) for t in wl.swska_inputs(1, 4, 2000, 128, 128, seed=22)]
+    a = rod.swska_prefill(q, k, v, 512)
+    b = rod.swska_prefill(q, k, v, 512)
+    rod.check()
+    assert torch.equal(a, b)
