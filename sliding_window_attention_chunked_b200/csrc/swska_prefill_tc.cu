@@ -15,6 +15,7 @@
 //   warps 4-7   softmax warpgroup of head 1
 //   warp  8     TMA producer: Q once, then K_j, V0_j, V1_j into a ring of 32 KB slots
 //   warp  9     TMEM allocator and the single MMA-issuing thread
+//   warps 10-11 idle (they complete the third warpgroup, which gives its registers away)
 // TMEM (512 columns): S0 | O0 | S1 | O1, 128 columns each. S_h = Q_h K_j^T is read by the
 // softmax warps, which write P_h (bf16, packed two per column) over the first 64 columns of
 // S_h; O_h += P_h V_h,j then reads P_h straight from TMEM (A operand in TMEM). The issue order
@@ -42,7 +43,14 @@ constexpr int HD = 128;                    // head dim (dk = dv)
 constexpr int NSLOT = 4;                   // ring slots
 constexpr int TILE_BYTES = BM * HD * 2;    // 32 KB: one 128 x 128 bf16 tile
 constexpr int HALF_BYTES = TILE_BYTES / 2; // one 128-row x 64-column TMA box
-constexpr int NTHREADS = 320;
+constexpr int NTHREADS = 384;               // 3 warpgroups
+// Register split (setmaxnreg). The register file is divided among the SM's four sub-partitions
+// and each holds one warp of every warpgroup here, so per sub-partition the launch provides
+// 3 x 168 = 504 registers per lane; the split below uses 216 + 216 + 72 = 504 exactly.
+constexpr int kLaunchRegs = 168;
+constexpr int kSoftmaxRegs = 216;
+constexpr int kControlRegs = 72;
+static_assert(2 * kSoftmaxRegs + kControlRegs <= 3 * kLaunchRegs, "register split exceeds launch");
 constexpr float kRescaleThreshold = 8.0f;  // log2 units
 
 constexpr int OFF_Q = 0;
@@ -66,7 +74,7 @@ __device__ __forceinline__ bool wait_bar(uint64_t* bar, uint32_t parity, volatil
     }
 }
 
-__global__ void __maxnreg__(200)
+__global__ void __launch_bounds__(NTHREADS, 1)
 swska_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                 const __grid_constant__ CUtensorMap tm_v, __nv_bfloat16* __restrict__ o, int T,
                 int H, int W, float scale_log2, int n_qtiles) {
@@ -117,6 +125,9 @@ swska_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     tc::fence_after_sync();
     const uint32_t tmem = *tmem_holder;
 
+    if (warp >= 8) {
+        asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kControlRegs));
+    }
     if (warp == 8) {
         // ------------------------------- TMA producer -------------------------------
         if (lane == 0) {
@@ -219,8 +230,9 @@ swska_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             tc::mma_commit(drain);
             mbar_wait_bounded(drain, 0, kWaitLimit);
         }
-    } else {
+    } else if (warp < 8) {
         // ------------------------------- softmax warpgroups -------------------------------
+        asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kSoftmaxRegs));
         const int h = warp / 4;                     // head within the pair
         const int row = threadIdx.x % 128;          // query row == TMEM lane
         const uint32_t lane_base = (uint32_t)(32 * (warp % 4)) << 16;
@@ -251,22 +263,11 @@ swska_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             for (int c = 1; c < BN; ++c) mx = fmaxf(mx, __uint_as_float(s[c]));
             const float m_tile = mx * scale_log2;
             const bool need = m_tile > m_run + kRescaleThreshold;
-            if (j > 0 && __any_sync(0xffffffffu, need)) {
-                const float alpha = need ? tc::ex2(m_run - m_tile) : 1.f;
-#pragma unroll
-                for (int cb = 0; cb < HD; cb += 32) {
-                    uint32_t r[32];
-                    tc::tmem_ld32(tO + cb, r);
-                    tc::tmem_wait_ld();
-#pragma unroll
-                    for (int i = 0; i < 32; ++i) r[i] = __float_as_uint(__uint_as_float(r[i]) * alpha);
-                    tc::tmem_st32(tO + cb, r);
-                }
-                tc::tmem_wait_st();
-                l_run *= alpha;
-            }
+            const float alpha = need ? tc::ex2(m_run - m_tile) : 1.f;  // 0 when m_run = -inf
+            l_run *= alpha;
             if (need) m_run = m_tile;
             const float m_use = m_run == -INFINITY ? 0.f : m_run;
+            // P = 2^(s * scale * log2 e - m) as bf16 pairs over the first 64 columns of S
 #pragma unroll
             for (int half = 0; half < 2; ++half) {
                 uint32_t pk[32];
@@ -279,6 +280,19 @@ swska_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                     pk[i] = pack_bf16x2(p0, p1);
                 }
                 tc::tmem_st32(tS + 32u * half, pk);
+            }
+            // a row whose maximum moved rescales its O row (PV of the previous tile is done:
+            // this tile's S was committed after it)
+            if (j > 0 && __any_sync(0xffffffffu, need)) {
+#pragma unroll
+                for (int cb = 0; cb < HD; cb += 32) {
+                    uint32_t r[32];
+                    tc::tmem_ld32(tO + cb, r);
+                    tc::tmem_wait_ld();
+#pragma unroll
+                    for (int i = 0; i < 32; ++i) r[i] = __float_as_uint(__uint_as_float(r[i]) * alpha);
+                    tc::tmem_st32(tO + cb, r);
+                }
             }
             tc::tmem_wait_st();
             tc::fence_before_sync();
