@@ -23,6 +23,14 @@ cudaError_t gla_prefill_recurrent_launch(const void* q, const void* k, const voi
                                          const float* g, float* state, void* o, int B, int H,
                                          int T, int dk, int dv, bool bf16, cudaStream_t stream);
 
+// chunkwise gated-recurrence prefill on tcgen05 tensor cores (bf16, dk = dv = 128, chunk 64)
+bool gla_prefill_tc_supported(int dk, int dv, int chunk);
+size_t gla_prefill_tc_workspace_size(int B, int H, int T);
+cudaError_t gla_prefill_tc_launch(const void* q, const void* k, const void* v, const float* g,
+                                  float* state, void* o, int B, int H, int T, void* workspace,
+                                  cudaStream_t stream);
+unsigned gla_prefill_tc_take_timeout_flag();
+
 // SW-SKA prefill on CUDA cores (fp32 FMA, online softmax)
 cudaError_t swska_prefill_simt_launch(const void* q, const void* k, const void* v, void* o,
                                       int B, int H, int T, int dk, int dv, int window,
@@ -34,7 +42,9 @@ cudaError_t swska_prefill_tc_launch(const void* q, const void* k, const void* v,
                                     int H, int T, int window, float scale, cudaStream_t stream);
 unsigned swska_prefill_tc_take_timeout_flag();
 
-// TMA descriptor for a 3-D bf16 tensor [d2][d1][d0], boxes of box1 x box0, 128-byte swizzle
+// TMA descriptors for a 3-D tensor [d2][d1][d0] loaded as boxes of box1 x box0 elements
+cudaError_t make_tmap_3d(CUtensorMap* map, const void* base, bool fp32, uint64_t d0, uint64_t d1,
+                         uint64_t d2, uint32_t box0, uint32_t box1, bool swizzle128);
 cudaError_t make_tmap_bf16_3d(CUtensorMap* map, const void* base, uint64_t d0, uint64_t d1,
                               uint64_t d2, uint32_t box0, uint32_t box1);
 

@@ -57,7 +57,8 @@ int rod_check(void* stream) {
     cudaError_t e = cudaStreamSynchronize(static_cast<cudaStream_t>(stream));
     if (e != cudaSuccess) return from_cuda(e);
     const unsigned flags = rod::swska_decode_take_timeout_flag() |
-                           rod::swska_prefill_tc_take_timeout_flag();
+                           rod::swska_prefill_tc_take_timeout_flag() |
+                           rod::gla_prefill_tc_take_timeout_flag();
     if (flags) return ROD_ERR_TIMEOUT;
     return from_cuda(cudaGetLastError());
 }
@@ -65,6 +66,8 @@ int rod_check(void* stream) {
 size_t rod_gla_prefill_workspace_size(int B, int H, int T, int dk, int dv, int chunk, int dtype) {
     if (B < 0 || H < 0 || T < 0 || !dim_ok(dk) || !dim_ok(dv) || !dtype_ok(dtype)) return 0;
     if (chunk < 16 || chunk > 128 || chunk % 16 != 0) return 0;
+    if (dtype == ROD_BF16 && rod::gla_prefill_tc_supported(dk, dv, chunk))
+        return rod::gla_prefill_tc_workspace_size(B, H, T);
     return 0;
 }
 
@@ -81,11 +84,14 @@ int rod_gla_prefill(const void* q, const void* k, const void* v, const float* g,
         return ROD_ERR_ALIGN;
     const size_t need = rod_gla_prefill_workspace_size(B, H, T, dk, dv, chunk, dtype);
     if (need > 0 && (!workspace || ws_bytes < need)) return ROD_ERR_WORKSPACE;
-    (void)workspace;
-    (void)ws_bytes;
+    if (need > 0 && !aligned16(workspace)) return ROD_ERR_ALIGN;
+    const cudaStream_t s = static_cast<cudaStream_t>(stream);
+    // bf16 with 128-wide heads and 64-token chunks runs the chunkwise tensor-core kernels;
+    // fp32 (exact FMA) and the other shapes run the sequential-in-time CUDA-core kernel
+    if (dtype == ROD_BF16 && rod::gla_prefill_tc_supported(dk, dv, chunk))
+        return from_cuda(rod::gla_prefill_tc_launch(q, k, v, g, state, o, B, H, T, workspace, s));
     return from_cuda(rod::gla_prefill_recurrent_launch(q, k, v, g, state, o, B, H, T, dk, dv,
-                                                       dtype == ROD_BF16,
-                                                       static_cast<cudaStream_t>(stream)));
+                                                       dtype == ROD_BF16, s));
 }
 
 int rod_gla_decode_step(const void* q, const void* k, const void* v, const float* g,

@@ -68,12 +68,46 @@ def test_gla_prefill_bf16_chunk_sizes(chunk):
     _gla_check(1, 2, 300, 128, 128, chunk, "bf16", "l2", seed=chunk)
 
 
-def test_gla_prefill_gate_zero_resets():
-    _gla_check(1, 2, 130, 128, 64, 64, "bf16", "l2", seed=3, gate=0.0)
+@pytest.mark.parametrize("dk,dv", [(128, 128), (128, 64)])
+def test_gla_prefill_gate_zero_resets(dk, dv):
+    _gla_check(1, 2, 130, dk, dv, 64, "bf16", "l2", seed=3, gate=0.0)
 
 
-def test_gla_prefill_gate_one_linear_attention():
-    _gla_check(1, 2, 130, 64, 128, 64, "bf16", "l2", seed=4, gate=1.0)
+@pytest.mark.parametrize("dk,dv", [(128, 128), (64, 128)])
+def test_gla_prefill_gate_one_linear_attention(dk, dv):
+    _gla_check(1, 2, 130, dk, dv, 64, "bf16", "l2", seed=4, gate=1.0)
+
+
+def test_gla_prefill_mixed_strong_and_mild_decay():
+    """Chunks where a channel decays below 2^-60 take the exact CUDA-core path for the
+    intra-chunk scores; the others use the tensor cores. Both must agree with the oracle."""
+    B, H, T, d = 1, 2, 700, 128
+    q, k, v, g = wl.gla_inputs(B, H, T, d, d, dist="l2", seed=31)
+    g[:, :, 100:110, 5] = 1e-9     # chunk 1: strong decay in one channel
+    g[:, 1, 400:464, :] = 0.3      # chunk 6 of head 1: every channel decays hard
+    g[:, 0, 650, 77] = 0.0         # an exact zero gate in the tail chunk
+    o_ref, S_ref = oracle.gla_prefill(q, k, v, g)
+    S = torch.zeros(B, H, d, d, device=DEV)
+    o = rod.gla_prefill(q.to(DEV), k.to(DEV), v.to(DEV), g.to(DEV), S, chunk=64)
+    rod.check()
+    compare(o, o_ref, "bf16", "o")
+    compare(S, S_ref, "bf16", "state")
+
+
+@pytest.mark.parametrize("B,H,T", [(1, 2, 5000), (1, 1, 64 * 40 + 3), (3, 5, 777)])
+def test_gla_prefill_many_segments(B, H, T):
+    """Small B*H spreads the sequence over many segments (segment pass + state scan)."""
+    _gla_check(B, H, T, 128, 128, 64, "bf16", "l2", seed=T, state0_scale=0.2)
+
+
+def test_gla_prefill_deterministic():
+    q, k, v, g = [t.to(DEV) for t in wl.gla_inputs(1, 4, 3000, 128, 128, dist="l2", seed=32)]
+    S1 = torch.zeros(1, 4, 128, 128, device=DEV)
+    S2 = torch.zeros_like(S1)
+    o1 = rod.gla_prefill(q, k, v, g, S1)
+    o2 = rod.gla_prefill(q, k, v, g, S2)
+    rod.check()
+    assert torch.equal(o1, o2) and torch.equal(S1, S2)
 
 
 def test_gla_prefill_split_hands_off_state():
