@@ -110,6 +110,31 @@ ROD_API int rod_gla_prefill(const void* q, const void* k, const void* v, const f
                     void* o, int B, int H, int T, int dk, int dv, int chunk, int dtype,
                     void* workspace, size_t ws_bytes, void* stream);
 
+/* ---- gated linear recurrence: prefill for callers that cannot allocate ----------------------- */
+/*
+ * Not a step of the method (the source pages have no counterpart): the same computation as
+ * rod_gla_prefill, for callers that cannot allocate device memory per call -- code embedded in
+ * a host program that owns the GPU memory pool, plug-ins forbidden to call cudaMalloc or a
+ * framework allocator (an allocation may synchronise the device or fail under memory
+ * pressure), or paths that must not allocate after start-up. The scratch rod_gla_prefill takes
+ * as `workspace` lives instead in one fixed device array inside the library,
+ * ROD_GLA_PREFILL_NOALLOC_MAX_SCRATCH bytes, held on every GPU that uses it until the process
+ * exits. The call allocates nothing; the caller still passes all inputs and outputs, with the
+ * layouts and meaning of rod_gla_prefill.
+ *  - The first call made with a given device current looks up the array's device address on
+ *    that device; make that first call before any stream capture begins.
+ *  - A problem whose rod_gla_prefill_workspace_size exceeds the maximum returns
+ *    ROD_ERR_WORKSPACE before anything is launched.
+ *  - Every call shares the one array and it keeps the last call's contents; nothing in it needs
+ *    to start at zero. Calls that overlap on the GPU (unordered streams, concurrent host
+ *    threads) race on it and produce wrong results: serialise them.
+ * Other errors: as rod_gla_prefill.
+ */
+#define ROD_GLA_PREFILL_NOALLOC_MAX_SCRATCH ((size_t)48 << 20)
+ROD_API int rod_gla_prefill_noalloc(const void* q, const void* k, const void* v, const float* g,
+                                    float* state, void* o, int B, int H, int T, int dk, int dv,
+                                    int chunk, int dtype, void* stream);
+
 /* ---- gated linear recurrence: one decode step --------------------------------------------- */
 /*
  * One token for each of N sequences x H heads, with the fixed-size state updated in place

@@ -18,6 +18,7 @@ from ._binding import (  # noqa: F401
     check,
     gla_decode_step,
     gla_prefill,
+    gla_prefill_noalloc,
     gla_prefill_workspace_size,
     launch_count,
     library_path,

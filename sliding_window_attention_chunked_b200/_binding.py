@@ -57,6 +57,8 @@ def load_library() -> ctypes.CDLL:
     lib.rod_gla_prefill_workspace_size.restype = sz
     lib.rod_gla_prefill.argtypes = [vp, vp, vp, vp, vp, vp, i, i, i, i, i, i, i, vp, sz, vp]
     lib.rod_gla_prefill.restype = i
+    lib.rod_gla_prefill_noalloc.argtypes = [vp, vp, vp, vp, vp, vp, i, i, i, i, i, i, i, vp]
+    lib.rod_gla_prefill_noalloc.restype = i
     lib.rod_gla_decode_step.argtypes = [vp, vp, vp, vp, vp, vp, i, i, i, i, i, vp]
     lib.rod_gla_decode_step.restype = i
     lib.rod_swska_prefill.argtypes = [vp, vp, vp, vp, i, i, i, i, i, i, f, i, vp]
@@ -147,6 +149,31 @@ def gla_prefill(q, k, v, g, state, o=None, chunk=64, workspace=None, stream=None
                              B, H, T, dk, dv, chunk, _dtype_code(q), _ptr(workspace), ws_bytes,
                              _stream(stream))
     _raise_on("rod_gla_prefill", st)
+    return o
+
+
+def gla_prefill_noalloc(q, k, v, g, state, o=None, chunk=64, stream=None):
+    """rod_gla_prefill_noalloc: the same prefill as gla_prefill, but the library uses its own
+    fixed device scratch instead of a caller-provided workspace (for callers that cannot
+    allocate per call). ``o`` must be supplied by such callers; when omitted it is allocated
+    here for convenience. Returns o."""
+    for n, t in (("q", q), ("k", k), ("v", v)):
+        _need(t, n, q.dtype, 4)
+    _need(g, "g", torch.float32, 4)
+    _need(state, "state", torch.float32, 4)
+    B, H, T, dk = q.shape
+    dv = v.shape[-1]
+    if k.shape != q.shape or g.shape != q.shape or tuple(v.shape[:3]) != (B, H, T):
+        raise ValueError("q, k, g must be [B,H,T,dk] and v [B,H,T,dv]")
+    if tuple(state.shape) != (B, H, dk, dv):
+        raise ValueError("state must be [B,H,dk,dv]")
+    if o is None:
+        o = torch.empty((B, H, T, dv), dtype=q.dtype, device=q.device)
+    _need(o, "o", q.dtype, 4)
+    st = load_library().rod_gla_prefill_noalloc(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(state),
+                                                _ptr(o), B, H, T, dk, dv, chunk, _dtype_code(q),
+                                                _stream(stream))
+    _raise_on("rod_gla_prefill_noalloc", st)
     return o
 
 
