@@ -133,6 +133,28 @@ def recorded_traffic(kernel_key, sources):
     return rec.get("dram_bytes_per_launch")
 
 
+def replica_seed_base(rank):
+    """Each rank runs its own replica of the workload on its own seeded inputs."""
+    return 1000 * rank
+
+
+def max_over_ranks(x, device="cpu"):
+    """Max of a per-rank scalar over the default process group (identity on one rank)."""
+    import torch
+    import torch.distributed as dist
+
+    if not dist.is_available() or not dist.is_initialized() or dist.get_world_size() == 1:
+        return float(x)
+    t = torch.tensor([float(x)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_throughput(units_per_rank_step, steps, world, ms_max):
+    """Whole-job throughput: every rank's units over the slowest rank's time."""
+    return units_per_rank_step * world * steps / (ms_max / 1e3)
+
+
 # ------------------------------------------------------------------------------------------
 # CPU baseline: the oracle, timed on a bounded sample of the same workload
 # ------------------------------------------------------------------------------------------
@@ -213,16 +235,12 @@ def run_gpu(args):
             dist.barrier()
         torch.cuda.synchronize()
 
-    def max_over_ranks(x):
-        if world == 1:
-            return x
-        t = torch.tensor([x], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        return float(t.item())
+    def ranks_max(x):
+        return max_over_ranks(x, device=dev)
 
     d = wl.WORKLOADS[WORKLOAD].dims
     B, H, T, dk, dv, L, W, C = d["B"], d["H"], d["T"], d["dk"], d["dv"], d["layers"], d["window"], d["chunk"]
-    seed_base = 1000 * rank
+    seed_base = replica_seed_base(rank)
     layers = []
     for l in range(L):
         ins = wl.stack_layer_inputs(l, B, H, T, dk, dv, seed_base=seed_base, device=dev)
@@ -266,12 +284,11 @@ def run_gpu(args):
     launches = rod.launch_count() - n0
     rod.check()
     ms_local = ev0.elapsed_time(ev1)
-    ms = max_over_ranks(ms_local)
+    ms = ranks_max(ms_local)
     ms_per_step = ms / args.steps
-    tokens = B * T * world * args.steps
-    value = tokens / (ms / 1e3)
+    value = job_throughput(B * T, args.steps, world, ms)
     ska_ms = [a.elapsed_time(b) for a, b in ska_events]
-    ska_avg_ms = max_over_ranks(sum(ska_ms) / len(ska_ms))
+    ska_avg_ms = ranks_max(sum(ska_ms) / len(ska_ms))
     clocks = clk.summary()
 
     peaks, peaks_src = load_peaks()
@@ -317,9 +334,9 @@ def run_gpu(args):
     e1.record(stream)
     barrier()
     rod.check()
-    dec_ms = max_over_ranks(e0.elapsed_time(e1) / dsteps)
-    gla_dec_ms = max_over_ranks(sum(a.elapsed_time(b) for a, b in ge) / dsteps)
-    ska_dec_ms = max_over_ranks(sum(a.elapsed_time(b) for a, b in se) / dsteps)
+    dec_ms = ranks_max(e0.elapsed_time(e1) / dsteps)
+    gla_dec_ms = ranks_max(sum(a.elapsed_time(b) for a, b in ge) / dsteps)
+    ska_dec_ms = ranks_max(sum(a.elapsed_time(b) for a, b in se) / dsteps)
     gla_dec_bytes = 2.0 * N * H * dk * dv * 4 + N * H * (2 * dk * 2 + dk * 4 + dv * 2 + dv * 2)
     ska_dec_bytes = 1.0 * N * Wd * dk * 2 + N * H * Wd * dv * 2 + N * H * (dk + dv + dv) * 2 + N * dk * 2
     hbm = peaks.get("hbm_gbs")
@@ -357,7 +374,7 @@ def run_gpu(args):
     # ---- end to end through the public API with host buffers ----
     e2e = None
     if not args.no_e2e:
-        e2e = run_e2e(args, rod, torch, layers, d, ws, stream, barrier, max_over_ranks, world)
+        e2e = run_e2e(args, rod, torch, layers, d, ws, stream, barrier, ranks_max, world)
 
     del layers, dd
     torch.cuda.empty_cache()
@@ -386,7 +403,7 @@ def run_gpu(args):
         dist.destroy_process_group()
 
 
-def run_e2e(args, rod, torch, layers, d, ws, stream, barrier, max_over_ranks, world):
+def run_e2e(args, rod, torch, layers, d, ws, stream, barrier, reduce_max, world):
     """Same stack, but every step copies each layer's inputs from pinned host memory into the
     device buffers and reads each layer's output back to pinned host memory."""
     B, T, C, W = d["B"], d["T"], d["chunk"], d["window"]
@@ -422,8 +439,8 @@ def run_e2e(args, rod, torch, layers, d, ws, stream, barrier, max_over_ranks, wo
         step()
     e1.record(stream)
     barrier()
-    ms = max_over_ranks(e0.elapsed_time(e1))
-    return {"value": round(B * T * world * n / (ms / 1e3), 1), "unit": "tokens/s",
+    ms = reduce_max(e0.elapsed_time(e1))
+    return {"value": round(job_throughput(B * T, n, world, ms), 1), "unit": "tokens/s",
             "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": n,
             "note": "pinned host buffers per layer kind reused for every layer; copies and "
                     "kernels serialised on one stream"}
