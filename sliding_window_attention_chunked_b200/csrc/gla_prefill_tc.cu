@@ -6,27 +6,37 @@
 //     S_t = diag(g_t) S_{t-1} + k_t^T v_t,     o_t = q_t S_t.
 // Chunk form (the chunkwise-parallel algorithm the Rodimus block paragraph names for training
 // and prefill). For a chunk of C tokens with incoming state S_in, per key channel c let
-//     G_t = prod_{r<=t} g_r     (prefix product inside the chunk),
-//     F_t = prod_{t<r<=C-1} g_r (suffix product),  a = G_{C-1}.
+//     G_t = prod_{r<=t} g_r     (prefix product inside the chunk),   a = G_{C-1},
+//     F_t = prod_{t<r<=C-1} g_r = a / G_t   (suffix product).
 // Then, exactly,
 //     o_t   = sum_{s<=t} (sum_c q_tc k_sc G_tc / G_sc) v_s + (q_t . G_t) S_in
 //     S_out = diag(a) S_in + sum_s (k_s . F_s)^T v_s.
 // With q~ = q.G, k~ = k/G, k^ = k.F the chunk is four dense contractions on the tensor cores:
 //     A = q~ k~^T (masked to s <= t, rounded to bf16 as P),  O = P V + q~ S_in,  S += k^^T V
-// while the fp32 state lives in tensor memory for the whole segment. k~ needs 1/G, so a chunk
-// in which some channel decays below 2^-60 computes A on the CUDA cores from log2-gate sums
-// (exact in the limit, g = 0 included) instead; everything else is unchanged.
+// while the fp32 state lives in tensor memory for the whole segment. k~ = k/G needs G well
+// inside the fp32/bf16 exponent range, so a chunk in which some channel's product a falls below
+// 2^-100 takes the exact route instead: the scores are summed on the CUDA cores from log2-gate
+// prefix sums L (log2 g clamped at -126, so g = 0 contributes below fp32 resolution),
+// A_ts = sum_c q_tc k_sc 2^(L_tc - L_sc), and written straight into tensor memory, where the
+// tensor-core route would have put them; q~ = q.2^L and k^ = k.2^(L_last - L).
 //
 // Parallelism over the sequence: the T tokens are cut into segments of L_seg tokens. Pass A
 // (per segment but the last) computes the segment's state contribution U and decay a_seg
-// from k, v, g; a scan kernel chains S_in(m+1) = diag(a_seg,m) S_in(m) + U_m per (b, h) with
-// each thread walking its state elements through the segments; pass C recomputes every
-// segment from its S_in and writes o (and the final state). One segment means pass C alone.
+// from k, v, g; a scan kernel chains S_in(m+1) = diag(a_seg,m) S_in(m) + U_m per (b, h);
+// pass C recomputes every segment from its S_in and writes o (and the final state). One
+// segment means pass C alone.
 //
-// CTA layout (160 threads): warps 0-3 = compute warpgroup, thread c <-> key channel c <->
-// TMEM lane c of the state accumulator; warp 4 = TMA producer and TMEM allocator. Thread 0
-// issues the MMAs. TMEM: S (128 cols, M=128), O (128 cols) and A (64 cols), both M=64 (rows
-// 0-15 of each 32-lane quarter). Every wait is bounded; a timeout stops all roles, drains
+// CTA (288 threads), a three-stage pipeline over the chunks of a segment:
+//   warp 8        TMA producer (q, k, v, g of chunk n into stage n % 2) and TMEM allocator;
+//   warpgroup 0   operands of chunk n: gate prefix products (8 rows x 8 channels per thread,
+//                 block products combined through shared memory), q~ and k^ in place over q
+//                 and k, k~ over the gates; thread 0 issues A = q~ k~^T into TMEM buffer n % 2;
+//   warpgroup 1   state work of chunk n-1 ... n: output rows of the previous chunk, the state
+//                 row c (thread c = TMEM lane c) copied to bf16 for the readout and scaled by a,
+//                 P = mask(A), and thread 128 issues S += k^^T V and O = P V + q~ S_in.
+// So the operands of chunk n+1 are built while chunk n's state work and MMAs run.
+// TMEM: S (cols 0-127, M=128), O (128-255, M=64: rows in lanes 0-15 of each 32-lane quarter),
+// A0 / A1 (256-319 / 320-383, M=64). Every wait is bounded; a timeout stops all roles, drains
 // in-flight copies and MMAs, and raises a flag.
 #include <cuda.h>
 #include <math.h>
@@ -42,21 +52,23 @@ __device__ unsigned int g_gla_tc_timeout = 0;
 
 constexpr int C = 64;                    // tokens per chunk
 constexpr int D = 128;                   // d_k = d_v
-constexpr int NTHREADS = 160;
+constexpr int NTHREADS = 288;            // 2 warpgroups + producer warp
 constexpr int BOX_BYTES = C * 128;       // one 64-row x 64-col bf16 box (128 B rows) = 8 KB
 constexpr int OP_BYTES = 2 * BOX_BYTES;  // one 64 x 128 bf16 operand = 16 KB
 constexpr int G_BYTES = C * D * 4;       // 64 x 128 fp32 gates = 32 KB
-// stage: q | k | v | g
+// stage: q | k | v | g      (after warpgroup 0: q~ | k^ | v | k~ (first 16 KB) ...)
 constexpr int ST_Q = 0, ST_K = OP_BYTES, ST_V = 2 * OP_BYTES, ST_G = 3 * OP_BYTES;
 constexpr int STAGE_BYTES = 3 * OP_BYTES + G_BYTES;          // 80 KB
-constexpr int OFF_KHAT = 2 * STAGE_BYTES;                    // 16 KB
-constexpr int OFF_P = OFF_KHAT + OP_BYTES;                   // 8 KB
-constexpr int OFF_SBF = OFF_P + BOX_BYTES;                   // 32 KB (128 rows x 128 bf16)
-constexpr int OFF_BAR = OFF_SBF + 2 * D * 128;
-constexpr int NBAR = 8;                                      // full[2] empty[2] A O drain +1
+constexpr int OFF_P = 2 * STAGE_BYTES;                       // 8 KB   P (64 x 64 bf16)
+constexpr int OFF_SBF = OFF_P + BOX_BYTES;                   // 32 KB  S_in in bf16
+constexpr int OFF_SCAN = OFF_SBF + 2 * D * 128;              // 4 KB   block products [8][128]
+constexpr int OFF_ABUF = OFF_SCAN + 8 * D * 4;               // 1 KB   a of stage 0 / 1
+constexpr int OFF_FLAG = OFF_ABUF + 2 * D * 4;               // 16 B   exact-route flag per stage
+constexpr int OFF_BAR = OFF_FLAG + 16;
+constexpr int NBAR = 12;
 constexpr int OFF_MISC = OFF_BAR + 8 * NBAR;
 constexpr int SMEM_BYTES = OFF_MISC + 32 + 1024;
-constexpr float kFastMin = 8.673617e-19f;                    // 2^-60
+constexpr float kFastMin = 7.888609e-31f;                    // 2^-100
 constexpr float kLog2Floor = -126.0f;                        // log2 of the smallest gate used
 
 // TMEM columns
@@ -74,11 +86,15 @@ struct GlaArgs {
     int T, L_seg, n_seg;
 };
 
-// byte offset of element (row, col) of a K-major 128-byte-swizzled bf16 tile whose 64-column
-// boxes hold `rows` rows each
+// byte offset of the 16-byte chunk holding columns [col, col + 8) of row `row` in a K-major
+// 128-byte-swizzled bf16 tile whose 64-column boxes hold `rows` rows each (col % 8 == 0)
 __device__ __forceinline__ uint32_t sw_off(int row, int col, int rows) {
     const int box = col >> 6, cc = col & 63;
-    return (uint32_t)(box * rows * 128 + row * 128 + ((((cc >> 3) ^ (row & 7))) << 4) + ((cc & 7) << 1));
+    return (uint32_t)(box * rows * 128 + row * 128 + ((((cc >> 3) ^ (row & 7))) << 4));
+}
+// byte offset of one bf16 element (row, col) of such a tile
+__device__ __forceinline__ uint32_t sw_off_elem(int row, int col, int rows) {
+    return sw_off(row, col & ~7, rows) + ((col & 7) << 1);
 }
 
 __device__ __forceinline__ bool wait_bar(uint64_t* bar, uint32_t parity, volatile int* abort_flag) {
@@ -95,22 +111,37 @@ __device__ __forceinline__ bool wait_bar(uint64_t* bar, uint32_t parity, volatil
     }
 }
 
-// barrier 1 over the 128 threads of the compute warpgroup (the producer warp never joins)
-__device__ __forceinline__ void wg_sync() { asm volatile("bar.sync 1, 128;" ::: "memory"); }
-__device__ __forceinline__ bool wg_all(bool pred) {
+// named barriers: id 1 = warpgroup 0, id 2 = warpgroup 1 (128 threads each); the producer warp
+// and the other warpgroup never join them
+__device__ __forceinline__ void grp_sync(int id) {
+    asm volatile("bar.sync %0, 128;" ::"r"(id) : "memory");
+}
+__device__ __forceinline__ bool grp_all(int id, bool pred) {
     uint32_t out;
     asm volatile(
-        "{\n\t.reg .pred p, q;\n\tsetp.ne.u32 p, %1, 0;\n\t"
-        "bar.red.and.pred q, 1, 128, p;\n\tselp.u32 %0, 1, 0, q;\n\t}"
-        : "=r"(out) : "r"((uint32_t)pred) : "memory");
+        "{\n\t.reg .pred p, q;\n\tsetp.ne.u32 p, %2, 0;\n\t"
+        "bar.red.and.pred q, %1, 128, p;\n\tselp.u32 %0, 1, 0, q;\n\t}"
+        : "=r"(out) : "r"(id), "r"((uint32_t)pred) : "memory");
     return out != 0;
 }
 
-__device__ __forceinline__ float bf(const unsigned char* base, uint32_t off) {
-    return __bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(base + off));
+__device__ __forceinline__ void unpack8(const uint4& u, float* f) {
+    f[0] = bf16lo(u.x); f[1] = bf16hi(u.x); f[2] = bf16lo(u.y); f[3] = bf16hi(u.y);
+    f[4] = bf16lo(u.z); f[5] = bf16hi(u.z); f[6] = bf16lo(u.w); f[7] = bf16hi(u.w);
 }
-__device__ __forceinline__ void put_bf(unsigned char* base, uint32_t off, float x) {
-    *reinterpret_cast<__nv_bfloat16*>(base + off) = __float2bfloat16_rn(x);
+__device__ __forceinline__ uint4 pack8(const float* f) {
+    uint4 u;
+    u.x = pack_bf16x2(f[0], f[1]); u.y = pack_bf16x2(f[2], f[3]);
+    u.z = pack_bf16x2(f[4], f[5]); u.w = pack_bf16x2(f[6], f[7]);
+    return u;
+}
+__device__ __forceinline__ float ldbf(const unsigned char* p) {
+    return __bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(p));
+}
+__device__ __forceinline__ float lg2(float x) {  // log2 on the SFU (0 gives -inf)
+    float y;
+    asm("lg2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
 }
 
 template <int MODE>
@@ -131,11 +162,15 @@ gla_chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
     constexpr uint32_t kStageTx = MODE == PASS_C ? STAGE_BYTES : STAGE_BYTES - OP_BYTES;
 
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + OFF_BAR);
-    uint64_t* full = bars;         // [2]
-    uint64_t* empty = bars + 2;    // [2]
-    uint64_t* barA = bars + 4;
-    uint64_t* barO = bars + 5;     // all MMAs of a chunk done
-    uint64_t* drain = bars + 6;
+    uint64_t* full = bars;         // [2] TMA -> warpgroup 0
+    uint64_t* empty = bars + 2;    // [2] chunk MMAs done -> producer
+    uint64_t* ops = bars + 4;      // [2] operands ready -> warpgroup 1
+    uint64_t* barA = bars + 6;     // [2] A = q~ k~^T done
+    uint64_t* barO = bars + 8;     // all MMAs of warpgroup 1 for a chunk done
+    uint64_t* drain0 = bars + 9;
+    uint64_t* drain1 = bars + 10;
+    float* abuf = reinterpret_cast<float*>(smem + OFF_ABUF);
+    volatile int* flag = reinterpret_cast<volatile int*>(smem + OFF_FLAG);
     uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + OFF_MISC);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + OFF_MISC + 4);
 
@@ -143,14 +178,16 @@ gla_chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
         for (int s = 0; s < 2; ++s) {
             mbar_init(&full[s], 1);
             mbar_init(&empty[s], 1);
+            mbar_init(&ops[s], 1);
+            mbar_init(&barA[s], 1);
         }
-        mbar_init(barA, 1);
         mbar_init(barO, 1);
-        mbar_init(drain, 1);
+        mbar_init(drain0, 1);
+        mbar_init(drain1, 1);
         *abort_flag = 0;
         fence_mbar_init();
     }
-    if (warp == 4) {
+    if (warp == 8) {
         tc::tmem_alloc(tmem_holder, 512);
         tc::tmem_relinquish();
     }
@@ -158,8 +195,9 @@ gla_chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
     __syncthreads();
     tc::fence_after_sync();
     const uint32_t tmem = *tmem_holder;
+    bool ok = true;
 
-    if (warp == 4) {
+    if (warp == 8) {
         // ------------------------------- TMA producer -------------------------------
         if (lane == 0) {
             int n = 0;
@@ -180,20 +218,207 @@ gla_chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
             for (int ni = (n > 2 ? n - 2 : 0); ni < n; ++ni)  // copies still in flight land first
                 mbar_wait_bounded(&full[ni & 1], (uint32_t)((ni >> 1) & 1), kWaitLimit);
         }
-    } else {
-        // ------------------------------- compute warpgroup -------------------------------
-        const int c = tid;                                 // key channel / state row / TMEM lane
-        const uint32_t lane_base = (uint32_t)(32 * warp) << 16;
-        const uint32_t tS = tmem + TM_S + lane_base;
-        const int orow = 16 * warp + lane;                 // row of the M=64 accumulators
-        const bool orow_ok = lane < 16;
-        float a_seg = 1.f;                                 // PASS_A: decay over the segment
-        uint32_t nA = 0;                                   // completed MMA_A phases
-        bool ok = true;
-
+    } else if (warp < 4) {
+        // ------------------------------- warpgroup 0: operands -------------------------------
+        // thread = (channel group cg: channels 8cg..8cg+7, row block rb: rows 8rb..8rb+7)
+        const int cg = tid & 15, rb = tid >> 4;
+        const int c0 = 8 * cg, r0 = 8 * rb;
+        const bool rot = ((cg >> 2) & 1) != 0;  // alternate float4 halves: no bank conflicts
+        float* scan = reinterpret_cast<float*>(smem + OFF_SCAN);
         const uint32_t idesc_A = tc::idesc_bf16_f32(64, 64, 0, 0);
+        for (int n = 0; n < n_ch; ++n) {
+            const int st = n & 1;
+            unsigned char* base = smem + st * STAGE_BYTES;
+            float* gsm = reinterpret_cast<float*>(base + ST_G);
+            const int nvalid = min(C, t_end - (t_begin + n * C));
+            if (!grp_all(1, wait_bar(&full[st], (uint32_t)((n >> 1) & 1), abort_flag))) { ok = false; break; }
+
+            auto load_gates = [&](int i, float* g8) {  // gates of row r0+i, my 8 channels
+                const float4* p = reinterpret_cast<const float4*>(gsm + (r0 + i) * D + c0);
+                const float4 x0 = p[rot ? 1 : 0], x1 = p[rot ? 0 : 1];
+                const float4 lo = rot ? x1 : x0, hi = rot ? x0 : x1;
+                g8[0] = lo.x; g8[1] = lo.y; g8[2] = lo.z; g8[3] = lo.w;
+                g8[4] = hi.x; g8[5] = hi.y; g8[6] = hi.z; g8[7] = hi.w;
+            };
+            // prefix products of the gates: inside my row block, then across row blocks
+            float G[8][8];
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+                float g8[8];
+                load_gates(i, g8);
+                const bool valid = r0 + i < nvalid;  // rows past the sequence end: g = 1
+#pragma unroll
+                for (int j = 0; j < 8; ++j) G[i][j] = (valid ? g8[j] : 1.f) * (i > 0 ? G[i - 1][j] : 1.f);
+            }
+            *reinterpret_cast<float4*>(scan + rb * D + c0) = make_float4(G[7][0], G[7][1], G[7][2], G[7][3]);
+            *reinterpret_cast<float4*>(scan + rb * D + c0 + 4) = make_float4(G[7][4], G[7][5], G[7][6], G[7][7]);
+            grp_sync(1);
+            float pre[8], a[8];
+#pragma unroll
+            for (int j = 0; j < 8; ++j) { pre[j] = 1.f; a[j] = 1.f; }
+#pragma unroll
+            for (int b2 = 0; b2 < 8; ++b2) {
+                const float4 lo = *reinterpret_cast<const float4*>(scan + b2 * D + c0);
+                const float4 hi = *reinterpret_cast<const float4*>(scan + b2 * D + c0 + 4);
+                const float v[8] = {lo.x, lo.y, lo.z, lo.w, hi.x, hi.y, hi.z, hi.w};
+#pragma unroll
+                for (int j = 0; j < 8; ++j) {
+                    if (b2 < rb) pre[j] *= v[j];
+                    a[j] *= v[j];
+                }
+            }
+            bool mine = true;
+#pragma unroll
+            for (int j = 0; j < 8; ++j) mine = mine && a[j] >= kFastMin;
+            // vote (also a barrier: every gate and block product has been read past here)
+            const bool fast = grp_all(1, mine);
+
+            if (fast) {
+                // q~ = q.G over q, k^ = k.a/G over k, k~ = k/G over the (consumed) gates
+#pragma unroll
+                for (int i = 0; i < 8; ++i) {
+                    const uint32_t off = sw_off(r0 + i, c0, C);
+                    float qf[8], kf[8], qt[8], kt[8], kh[8];
+                    unpack8(*reinterpret_cast<const uint4*>(base + ST_K + off), kf);
+                    if (MODE == PASS_C) unpack8(*reinterpret_cast<const uint4*>(base + ST_Q + off), qf);
+#pragma unroll
+                    for (int j = 0; j < 8; ++j) {
+                        const float Gt = G[i][j] * pre[j];
+                        const float r = __frcp_rn(Gt);
+                        kh[j] = kf[j] * (a[j] * r);
+                        if (MODE == PASS_C) {
+                            qt[j] = qf[j] * Gt;
+                            kt[j] = kf[j] * r;
+                        }
+                    }
+                    *reinterpret_cast<uint4*>(base + ST_K + off) = pack8(kh);
+                    if (MODE == PASS_C) {
+                        *reinterpret_cast<uint4*>(base + ST_Q + off) = pack8(qt);
+                        *reinterpret_cast<uint4*>(base + ST_G + off) = pack8(kt);
+                    }
+                }
+            } else {
+                // exact route: L = prefix sums of clamped log2 gates, block sums through shared memory
+                float L[8][8];
+#pragma unroll
+                for (int i = 0; i < 8; ++i) {
+                    float g8[8];
+                    load_gates(i, g8);
+                    const bool valid = r0 + i < nvalid;
+#pragma unroll
+                    for (int j = 0; j < 8; ++j)
+                        L[i][j] = (valid ? fmaxf(lg2(g8[j]), kLog2Floor) : 0.f) + (i > 0 ? L[i - 1][j] : 0.f);
+                }
+                *reinterpret_cast<float4*>(scan + rb * D + c0) = make_float4(L[7][0], L[7][1], L[7][2], L[7][3]);
+                *reinterpret_cast<float4*>(scan + rb * D + c0 + 4) = make_float4(L[7][4], L[7][5], L[7][6], L[7][7]);
+                grp_sync(1);
+                float preL[8], Ltot[8];
+#pragma unroll
+                for (int j = 0; j < 8; ++j) { preL[j] = 0.f; Ltot[j] = 0.f; }
+#pragma unroll
+                for (int b2 = 0; b2 < 8; ++b2) {
+                    const float4 lo = *reinterpret_cast<const float4*>(scan + b2 * D + c0);
+                    const float4 hi = *reinterpret_cast<const float4*>(scan + b2 * D + c0 + 4);
+                    const float v[8] = {lo.x, lo.y, lo.z, lo.w, hi.x, hi.y, hi.z, hi.w};
+#pragma unroll
+                    for (int j = 0; j < 8; ++j) {
+                        if (b2 < rb) preL[j] += v[j];
+                        Ltot[j] += v[j];
+                    }
+                }
+                grp_sync(1);  // block sums and gates read before either is overwritten
+#pragma unroll
+                for (int j = 0; j < 8; ++j) a[j] = tc::ex2(Ltot[j]);
+#pragma unroll
+                for (int i = 0; i < 8; ++i)
+#pragma unroll
+                    for (int j = 0; j < 8; ++j) L[i][j] += preL[j];
+                if (MODE == PASS_C) {
+                    // L over the gates, then the exact scores of row t = 16 w + l into TMEM A[st]
+#pragma unroll
+                    for (int i = 0; i < 8; ++i) {
+                        *reinterpret_cast<float4*>(gsm + (r0 + i) * D + c0) = make_float4(L[i][0], L[i][1], L[i][2], L[i][3]);
+                        *reinterpret_cast<float4*>(gsm + (r0 + i) * D + c0 + 4) = make_float4(L[i][4], L[i][5], L[i][6], L[i][7]);
+                    }
+                    grp_sync(1);
+                    const int w = tid >> 5, l = tid & 31, trow = 16 * w + l;
+                    const uint32_t tA = tmem + TM_A + 64u * st + ((uint32_t)(32 * w) << 16);
+#pragma unroll
+                    for (int half = 0; half < 2; ++half) {
+                        uint32_t ar[32];
+#pragma unroll
+                        for (int jj = 0; jj < 32; ++jj) {
+                            const int s = 32 * half + jj;
+                            float acc = 0.f;
+                            if (l < 16 && s <= trow) {
+                                for (int cc = 0; cc < D; ++cc) {
+                                    const float wgt = tc::ex2(gsm[trow * D + cc] - gsm[s * D + cc]);
+                                    acc = fmaf(ldbf(base + ST_Q + sw_off_elem(trow, cc, C)) *
+                                                   ldbf(base + ST_K + sw_off_elem(s, cc, C)), wgt, acc);
+                                }
+                            }
+                            ar[jj] = __float_as_uint(acc);
+                        }
+                        tc::tmem_st32(tA + 32u * half, ar);
+                    }
+                    tc::tmem_wait_st();
+                    grp_sync(1);  // q, k and L read by every thread before they are overwritten
+                }
+                // q~ = q.2^L over q, k^ = k.2^(Ltot - L) over k
+#pragma unroll
+                for (int i = 0; i < 8; ++i) {
+                    const uint32_t off = sw_off(r0 + i, c0, C);
+                    float qf[8], kf[8], qt[8], kh[8];
+                    unpack8(*reinterpret_cast<const uint4*>(base + ST_K + off), kf);
+                    if (MODE == PASS_C) unpack8(*reinterpret_cast<const uint4*>(base + ST_Q + off), qf);
+#pragma unroll
+                    for (int j = 0; j < 8; ++j) {
+                        kh[j] = kf[j] * tc::ex2(Ltot[j] - L[i][j]);
+                        if (MODE == PASS_C) qt[j] = qf[j] * tc::ex2(L[i][j]);
+                    }
+                    *reinterpret_cast<uint4*>(base + ST_K + off) = pack8(kh);
+                    if (MODE == PASS_C) *reinterpret_cast<uint4*>(base + ST_Q + off) = pack8(qt);
+                }
+            }
+            if (rb == 0) {
+#pragma unroll
+                for (int j = 0; j < 8; ++j) abuf[st * D + c0 + j] = a[j];
+            }
+            if (tid == 0) flag[st] = fast ? 0 : 1;
+            asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+            tc::fence_before_sync();
+            grp_sync(1);
+            if (tid == 0) {
+                tc::fence_after_sync();
+                if (MODE == PASS_C && fast) {
+                    const uint32_t qa = smem_u32(base + ST_Q), ka = smem_u32(base + ST_G);
+#pragma unroll
+                    for (int k = 0; k < D / 16; ++k) {
+                        const uint32_t koff = (uint32_t)((k / 4) * BOX_BYTES + (k % 4) * 32);
+                        tc::mma_ss(tmem + TM_A + 64u * st, tc::sdesc_sw128(qa + koff, 16, 1024),
+                                   tc::sdesc_sw128(ka + koff, 16, 1024), idesc_A, k > 0);
+                    }
+                    tc::mma_commit(&barA[st]);
+                }
+                mbar_arrive(&ops[st]);
+            }
+        }
+        if (tid == 0) {  // every MMA this thread issued has completed before TMEM is released
+            tc::mma_commit(drain0);
+            mbar_wait_bounded(drain0, 0, kWaitLimit);
+        }
+    } else {
+        // ------------------------- warpgroup 1: state, P, outputs, MMAs -------------------------
+        const int c = tid - 128;                           // state row == TMEM lane
+        const int wq = warp - 4;                           // TMEM lane quarter of this warp
+        const uint32_t lane_base = (uint32_t)(32 * wq) << 16;
+        const uint32_t tS = tmem + TM_S + lane_base;
+        const int orow = 16 * wq + lane;                   // row of the M=64 accumulators
+        const bool orow_ok = lane < 16;
         const uint32_t idesc_U = tc::idesc_bf16_f32(128, 128, 1, 1);
         const uint32_t idesc_O = tc::idesc_bf16_f32(64, 128, 0, 1);
+        float a_seg = 1.f;                                 // PASS_A: decay over the segment
+        uint32_t nA0 = 0, nA1 = 0;                         // completed A phases per TMEM buffer
 
         auto epilogue = [&](int n) {  // O rows of chunk n -> bf16 global rows
             const int t0 = t_begin + n * C;
@@ -207,12 +432,10 @@ gla_chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                     __nv_bfloat16* dst = args.o + ((int64_t)bh * T + t) * D + cb;
 #pragma unroll
                     for (int i = 0; i < 32; i += 8) {
-                        uint4 u;
-                        u.x = pack_bf16x2(__uint_as_float(r[i + 0]), __uint_as_float(r[i + 1]));
-                        u.y = pack_bf16x2(__uint_as_float(r[i + 2]), __uint_as_float(r[i + 3]));
-                        u.z = pack_bf16x2(__uint_as_float(r[i + 4]), __uint_as_float(r[i + 5]));
-                        u.w = pack_bf16x2(__uint_as_float(r[i + 6]), __uint_as_float(r[i + 7]));
-                        *reinterpret_cast<uint4*>(dst + i) = u;
+                        float f[8];
+#pragma unroll
+                        for (int e = 0; e < 8; ++e) f[e] = __uint_as_float(r[i + e]);
+                        *reinterpret_cast<uint4*>(dst + i) = pack8(f);
                     }
                 }
             }
@@ -221,168 +444,91 @@ gla_chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
         for (int n = 0; n < n_ch; ++n) {
             const int st = n & 1;
             unsigned char* base = smem + st * STAGE_BYTES;
-            const int t0 = t_begin + n * C;
-            const int nvalid = min(C, t_end - t0);
-            // every wait of the warpgroup ends in a vote, so all 128 threads leave together
-            if (!wg_all(wait_bar(&full[st], (uint32_t)((n >> 1) & 1), abort_flag))) { ok = false; break; }
-
-            // ---- gates: prefix products G_t, suffix products F_t of channel c (rows >= nvalid: g = 1)
-            const float* gcol = reinterpret_cast<const float*>(base + ST_G) + c;
-            float G[C], F[C];
-            float run = 1.f;
-#pragma unroll
-            for (int t = 0; t < C; ++t) {
-                const float gt = t < nvalid ? gcol[t * D] : 1.f;
-                run *= gt;
-                G[t] = run;
-            }
-            const float a = run;  // decay of the whole chunk for channel c
-            run = 1.f;
-#pragma unroll
-            for (int t = C - 1; t >= 0; --t) {
-                F[t] = run;
-                run *= t < nvalid ? gcol[t * D] : 1.f;
-            }
-            const bool fast = wg_all(a >= kFastMin);
-
-            // ---- the previous chunk's MMAs are complete: its output rows, then its buffers are free
+            if (!grp_all(2, wait_bar(&ops[st], (uint32_t)((n >> 1) & 1), abort_flag))) { ok = false; break; }
+            tc::fence_after_sync();
+            const bool exact = flag[st] != 0;
+            const float a = abuf[st * D + c];
+            // the previous chunk's MMAs are done: its outputs, then S, S_bf and P are free
             if (n > 0) {
-                if (!wg_all(wait_bar(barO, (uint32_t)((n - 1) & 1), abort_flag))) { ok = false; break; }
+                if (!grp_all(2, wait_bar(barO, (uint32_t)((n - 1) & 1), abort_flag))) { ok = false; break; }
                 tc::fence_after_sync();
                 if (MODE == PASS_C) epilogue(n - 1);
             }
-
-            if (MODE == PASS_C && !fast) {
-                // A on the CUDA cores: A[t][s] = sum_c q_tc k_sc 2^(L_tc - L_sc), L = sum log2 g
-                float* Lbuf = reinterpret_cast<float*>(smem + OFF_SBF);  // [C][D] fp32, free now
-                float L = 0.f;
-#pragma unroll 4
-                for (int t = 0; t < C; ++t) {
-                    const float gt = t < nvalid ? gcol[t * D] : 1.f;
-                    L += fmaxf(__log2f(gt), kLog2Floor);
-                    Lbuf[t * D + c] = L;
-                }
-                wg_sync();
-                for (int pr = tid; pr < C * C; pr += 128) {
-                    const int t = pr / C, s = pr % C;
-                    float acc = 0.f;
-                    if (s <= t) {
-                        for (int cc = 0; cc < D; ++cc) {
-                            const float w = exp2f(Lbuf[t * D + cc] - Lbuf[s * D + cc]);
-                            acc = fmaf(bf(base + ST_Q, sw_off(t, cc, C)) * bf(base + ST_K, sw_off(s, cc, C)), w, acc);
-                        }
-                    }
-                    put_bf(smem + OFF_P, sw_off(t, s, C), acc);
-                }
-                wg_sync();
-            }
-
-            // ---- operands: q~ = q.G (in place), k~ = k/G (in place), k^ = k.F
+            // state row c: bf16 copy of S_in for the readout, then S <- diag(a) S, 32 columns at a time
 #pragma unroll
-            for (int t = 0; t < C; ++t) {
-                const uint32_t off = sw_off(t, c, C);
-                const float kv = bf(base + ST_K, off);
-                put_bf(smem + OFF_KHAT, off, kv * F[t]);
-                if (MODE == PASS_C) {
-                    put_bf(base + ST_Q, off, bf(base + ST_Q, off) * G[t]);
-                    if (fast) put_bf(base + ST_K, off, kv * __frcp_rn(G[t]));
-                }
-            }
-            asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-            tc::fence_before_sync();
-            wg_sync();
-            tc::fence_after_sync();
-            if (MODE == PASS_C && fast && tid == 0) {
-                const uint32_t qa = smem_u32(base + ST_Q), ka = smem_u32(base + ST_K);
-#pragma unroll
-                for (int k = 0; k < D / 16; ++k) {
-                    const uint32_t koff = (uint32_t)((k / 4) * BOX_BYTES + (k % 4) * 32);
-                    tc::mma_ss(tmem + TM_A, tc::sdesc_sw128(qa + koff, 16, 1024),
-                               tc::sdesc_sw128(ka + koff, 16, 1024), idesc_A, k > 0);
-                }
-                tc::mma_commit(barA);
-            }
-
-            // ---- state row c: bf16 copy of S_in for the readout, then S <- diag(a) S in TMEM
-            {
-                uint32_t srow[D];  // fp32 bits of state row c
+            for (int jb = 0; jb < D; jb += 32) {
+                uint32_t r[32];
                 if (n == 0) {
                     if (MODE == PASS_C) {
                         const int slot = args.s_in_slots == 1 ? 0 : seg;
-                        const float* src = args.s_in + (((int64_t)bh * args.s_in_slots + slot) * D + c) * D;
+                        const uint4* src = reinterpret_cast<const uint4*>(
+                            args.s_in + (((int64_t)bh * args.s_in_slots + slot) * D + c) * D + jb);
 #pragma unroll
-                        for (int j = 0; j < D; j += 4) {
-                            const uint4 v4 = *reinterpret_cast<const uint4*>(src + j);
-                            srow[j] = v4.x; srow[j + 1] = v4.y; srow[j + 2] = v4.z; srow[j + 3] = v4.w;
+                        for (int e = 0; e < 8; ++e) {
+                            const uint4 v4 = src[e];
+                            r[4 * e] = v4.x; r[4 * e + 1] = v4.y; r[4 * e + 2] = v4.z; r[4 * e + 3] = v4.w;
                         }
                     } else {
 #pragma unroll
-                        for (int j = 0; j < D; ++j) srow[j] = 0u;
+                        for (int e = 0; e < 32; ++e) r[e] = 0u;
                     }
                 } else {
-#pragma unroll
-                    for (int j = 0; j < D; j += 32) tc::tmem_ld32(tS + j, srow + j);
+                    tc::tmem_ld32(tS + jb, r);
                     tc::tmem_wait_ld();
                 }
                 if (MODE == PASS_C) {
-                    unsigned char* sb = smem + OFF_SBF;
 #pragma unroll
-                    for (int j = 0; j < D; j += 8) {
-                        uint4 u;
-                        u.x = pack_bf16x2(__uint_as_float(srow[j]), __uint_as_float(srow[j + 1]));
-                        u.y = pack_bf16x2(__uint_as_float(srow[j + 2]), __uint_as_float(srow[j + 3]));
-                        u.z = pack_bf16x2(__uint_as_float(srow[j + 4]), __uint_as_float(srow[j + 5]));
-                        u.w = pack_bf16x2(__uint_as_float(srow[j + 6]), __uint_as_float(srow[j + 7]));
-                        *reinterpret_cast<uint4*>(sb + sw_off(c, j, D)) = u;
+                    for (int e = 0; e < 32; e += 8) {
+                        float f[8];
+#pragma unroll
+                        for (int x = 0; x < 8; ++x) f[x] = __uint_as_float(r[e + x]);
+                        *reinterpret_cast<uint4*>(smem + OFF_SBF + sw_off(c, jb + e, D)) = pack8(f);
                     }
                 }
 #pragma unroll
-                for (int j = 0; j < D; ++j) srow[j] = __float_as_uint(__uint_as_float(srow[j]) * a);
-#pragma unroll
-                for (int j = 0; j < D; j += 32) tc::tmem_st32(tS + j, srow + j);
-                tc::tmem_wait_st();
+                for (int e = 0; e < 32; ++e) r[e] = __float_as_uint(__uint_as_float(r[e]) * a);
+                tc::tmem_st32(tS + jb, r);
             }
+            tc::tmem_wait_st();
             a_seg *= a;
             asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
             tc::fence_before_sync();
-            wg_sync();
-            tc::fence_after_sync();
-            if (tid == 0) {  // S += k^^T V
-                const uint32_t kh = smem_u32(smem + OFF_KHAT), va = smem_u32(base + ST_V);
+            grp_sync(2);
+            if (tid == 128) {  // S += k^^T V
+                tc::fence_after_sync();
+                const uint32_t kh = smem_u32(base + ST_K), va = smem_u32(base + ST_V);
 #pragma unroll
                 for (int k = 0; k < C / 16; ++k)
                     tc::mma_ss(tmem + TM_S, tc::sdesc_sw128(kh + 2048u * k, BOX_BYTES, 1024),
                                tc::sdesc_sw128(va + 2048u * k, BOX_BYTES, 1024), idesc_U, 1u);
             }
-
             if (MODE == PASS_C) {
-                // ---- P = mask(A) in bf16 (fast path; the slow path wrote P above)
-                if (fast) {
-                    if (!wg_all(wait_bar(barA, nA & 1, abort_flag))) { ok = false; break; }
-                    ++nA;
-                    tc::fence_after_sync();
-                    uint32_t r[64];
-                    tc::tmem_ld32(tmem + TM_A + lane_base, r);
-                    tc::tmem_ld32(tmem + TM_A + lane_base + 32, r + 32);
-                    tc::tmem_wait_ld();
-                    if (orow_ok) {
-#pragma unroll
-                        for (int s = 0; s < C; s += 8) {
-                            uint4 u;
-                            float f[8];
-#pragma unroll
-                            for (int i = 0; i < 8; ++i) f[i] = s + i <= orow ? __uint_as_float(r[s + i]) : 0.f;
-                            u.x = pack_bf16x2(f[0], f[1]); u.y = pack_bf16x2(f[2], f[3]);
-                            u.z = pack_bf16x2(f[4], f[5]); u.w = pack_bf16x2(f[6], f[7]);
-                            *reinterpret_cast<uint4*>(smem + OFF_P + sw_off(orow, s, C)) = u;
-                        }
-                    }
-                    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-                    tc::fence_before_sync();
-                    wg_sync();
+                // P = mask(A) in bf16; A came from the tensor cores or, on the exact route, was
+                // stored into TMEM by warpgroup 0 before it signalled the operands
+                if (!exact) {
+                    const uint32_t ph = st == 0 ? nA0 : nA1;
+                    if (!grp_all(2, wait_bar(&barA[st], ph & 1, abort_flag))) { ok = false; break; }
+                    if (st == 0) ++nA0; else ++nA1;
                     tc::fence_after_sync();
                 }
-                if (tid == 0) {  // O = P V + q~ S_in
+                uint32_t r[64];
+                tc::tmem_ld32(tmem + TM_A + 64u * st + lane_base, r);
+                tc::tmem_ld32(tmem + TM_A + 64u * st + lane_base + 32, r + 32);
+                tc::tmem_wait_ld();
+                if (orow_ok) {
+#pragma unroll
+                    for (int s = 0; s < C; s += 8) {
+                        float f[8];
+#pragma unroll
+                        for (int i = 0; i < 8; ++i) f[i] = s + i <= orow ? __uint_as_float(r[s + i]) : 0.f;
+                        *reinterpret_cast<uint4*>(smem + OFF_P + sw_off(orow, s, C)) = pack8(f);
+                    }
+                }
+                asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+                tc::fence_before_sync();
+                grp_sync(2);
+                if (tid == 128) {  // O = P V + q~ S_in
+                    tc::fence_after_sync();
                     const uint32_t pa = smem_u32(smem + OFF_P), va = smem_u32(base + ST_V);
                     const uint32_t qa = smem_u32(base + ST_Q), sb = smem_u32(smem + OFF_SBF);
 #pragma unroll
@@ -396,14 +542,14 @@ gla_chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                                    tc::sdesc_sw128(sb + 2048u * k, D * 128, 1024), idesc_O, 1u);
                 }
             }
-            if (tid == 0) {
+            if (tid == 128) {
                 tc::mma_commit(barO);
                 tc::mma_commit(&empty[st]);
             }
         }
 
         // ---- tail: last chunk's outputs and the segment's state
-        if (ok && n_ch > 0 && wg_all(wait_bar(barO, (uint32_t)((n_ch - 1) & 1), abort_flag))) {
+        if (ok && n_ch > 0 && grp_all(2, wait_bar(barO, (uint32_t)((n_ch - 1) & 1), abort_flag))) {
             tc::fence_after_sync();
             if (MODE == PASS_C) epilogue(n_ch - 1);
             float* dst = nullptr;
@@ -412,6 +558,7 @@ gla_chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                 dst = args.u_out + (((int64_t)bh * args.n_seg + seg + 1) * D + c) * D;
                 args.a_out[((int64_t)bh * args.n_seg + seg) * D + c] = a_seg;
             }
+#pragma unroll
             for (int j = 0; j < D; j += 32) {
                 uint32_t r[32];
                 tc::tmem_ld32(tS + j, r);
@@ -419,24 +566,21 @@ gla_chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                 if (dst) {
 #pragma unroll
                     for (int i = 0; i < 32; i += 4)
-                        *reinterpret_cast<float4*>(dst + j + i) =
-                            make_float4(__uint_as_float(r[i]), __uint_as_float(r[i + 1]),
-                                        __uint_as_float(r[i + 2]), __uint_as_float(r[i + 3]));
+                        *reinterpret_cast<uint4*>(dst + j + i) = make_uint4(r[i], r[i + 1], r[i + 2], r[i + 3]);
                 }
             }
         }
-        if (tid == 0) {  // every MMA issued has completed before TMEM is released
-            tc::mma_commit(drain);
-            mbar_wait_bounded(drain, 0, kWaitLimit);
+        if (tid == 128) {  // every MMA this thread issued has completed before TMEM is released
+            tc::mma_commit(drain1);
+            mbar_wait_bounded(drain1, 0, kWaitLimit);
         }
     }
 
     tc::fence_before_sync();
     __syncthreads();
     tc::fence_after_sync();
-    if (warp == 4) tc::tmem_dealloc(tmem, 512);
+    if (warp == 8) tc::tmem_dealloc(tmem, 512);
 }
-
 // S_in(0) = state; S_in(m+1) = diag(a_m) S_in(m) + U_m in place of U_m, for every (b, h) and
 // state element; each thread owns 4 consecutive elements of one state row and walks the
 // segments in order, with the next segment's U loaded ahead of the dependent update.
