@@ -70,6 +70,7 @@ constexpr int OFF_MISC = OFF_BAR + 8 * NBAR;
 constexpr int SMEM_BYTES = OFF_MISC + 32 + 1024;
 constexpr float kFastMin = 7.888609e-31f;                    // 2^-100
 constexpr float kLog2Floor = -126.0f;                        // log2 of the smallest gate used
+constexpr int kPrefetchChunks = 3;                           // L2 prefetch distance in chunks
 
 // TMEM columns
 constexpr uint32_t TM_S = 0, TM_O = 128, TM_A = 256;
@@ -83,6 +84,8 @@ struct GlaArgs {
     __nv_bfloat16* o;       // PASS_C: [BH][T][D]
     float* u_out;           // PASS_A: [BH][n_seg][D][D] (segment m writes slot m+1)
     float* a_out;           // PASS_A: [BH][n_seg][D]    (segment m writes slot m)
+    const __nv_bfloat16 *q, *k, *v;  // the inputs again, for L2 prefetches ahead of TMA
+    const float* g;
     int T, L_seg, n_seg;
 };
 
@@ -214,6 +217,17 @@ gla_chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                     tc::tma_load_3d(base + ST_V + half * BOX_BYTES, &tm_v, half * 64, y, bh, &full[st]);
                 }
                 tc::tma_load_3d(base + ST_G, &tm_g, 0, y, bh, &full[st]);
+                // keep later chunks of the segment streaming into L2 while the two stages turn over
+                const int pf = n + kPrefetchChunks;
+                if (pf < n_ch) {
+                    const int yp = t_begin + pf * C;
+                    const uint32_t rows = (uint32_t)min(C, t_end - yp);
+                    const int64_t row0 = (int64_t)bh * T + yp;
+                    if (MODE == PASS_C) tc::prefetch_l2(args.q + row0 * D, rows * D * 2);
+                    tc::prefetch_l2(args.k + row0 * D, rows * D * 2);
+                    tc::prefetch_l2(args.v + row0 * D, rows * D * 2);
+                    tc::prefetch_l2(args.g + row0 * D, rows * D * 4);
+                }
             }
             for (int ni = (n > 2 ? n - 2 : 0); ni < n; ++ni)  // copies still in flight land first
                 mbar_wait_bounded(&full[ni & 1], (uint32_t)((ni >> 1) & 1), kWaitLimit);
@@ -653,6 +667,10 @@ cudaError_t gla_prefill_tc_launch(const void* q, const void* k, const void* v, c
         if (e != cudaSuccess) return e;
     }
     GlaArgs a{};
+    a.q = static_cast<const __nv_bfloat16*>(q);
+    a.k = static_cast<const __nv_bfloat16*>(k);
+    a.v = static_cast<const __nv_bfloat16*>(v);
+    a.g = g;
     a.T = T;
     a.L_seg = p.L_seg;
     a.n_seg = p.n_seg;

@@ -130,6 +130,10 @@ __device__ __forceinline__ void tma_load_3d(void* dst_smem, const CUtensorMap* m
           "r"(smem_u32(bar))
         : "memory");
 }
+// bring `bytes` of global memory into L2 ahead of use (16-byte aligned address and size)
+__device__ __forceinline__ void prefetch_l2(const void* gmem, uint32_t bytes) {
+    asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(gmem), "r"(bytes) : "memory");
+}
 __device__ __forceinline__ void tma_prefetch_desc(const CUtensorMap* map) {
     asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
 }
