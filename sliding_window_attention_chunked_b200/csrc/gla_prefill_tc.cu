@@ -59,16 +59,18 @@ constexpr int G_BYTES = C * D * 4;       // 64 x 128 fp32 gates = 32 KB
 // stage: q | k | v | g      (after warpgroup 0: q~ | k^ | v | k~ (first 16 KB) ...)
 constexpr int ST_Q = 0, ST_K = OP_BYTES, ST_V = 2 * OP_BYTES, ST_G = 3 * OP_BYTES;
 constexpr int STAGE_BYTES = 3 * OP_BYTES + G_BYTES;          // 80 KB
-constexpr int OFF_P = 2 * STAGE_BYTES;                       // 8 KB   P (64 x 64 bf16)
-constexpr int OFF_SBF = OFF_P + BOX_BYTES;                   // 32 KB  S_in in bf16
+constexpr int ST_P = ST_G + OP_BYTES;                        // P (64 x 64 bf16) after k~
+constexpr int OFF_SBF = 2 * STAGE_BYTES;                     // 32 KB  R in bf16 for the readout
 constexpr int OFF_SCAN = OFF_SBF + 2 * D * 128;              // 4 KB   block products [8][128]
-constexpr int OFF_ABUF = OFF_SCAN + 8 * D * 4;               // 1 KB   a of stage 0 / 1
-constexpr int OFF_FLAG = OFF_ABUF + 2 * D * 4;               // 16 B   exact-route flag per stage
+constexpr int OFF_ABUF = OFF_SCAN + 8 * D * 4;               // 2 KB   a and D.a per stage
+constexpr int OFF_FLAG = OFF_ABUF + 4 * D * 4;               // 16 B   route / rescale flags
 constexpr int OFF_BAR = OFF_FLAG + 16;
 constexpr int NBAR = 12;
 constexpr int OFF_MISC = OFF_BAR + 8 * NBAR;
 constexpr int SMEM_BYTES = OFF_MISC + 32 + 1024;
-constexpr float kFastMin = 7.888609e-31f;                    // 2^-100
+constexpr float kFastMin = 8.673617e-19f;                    // 2^-60: chunk decay for q~ k~^T
+constexpr float kRescaleMin = 9.094947e-13f;                 // 2^-40: smallest running decay D
+constexpr int kFlagExact = 1, kFlagRescale = 2;
 constexpr float kLog2Floor = -126.0f;                        // log2 of the smallest gate used
 constexpr int kPrefetchChunks = 3;                           // L2 prefetch distance in chunks
 
@@ -138,8 +140,21 @@ __device__ __forceinline__ uint4 pack8(const float* f) {
     u.z = pack_bf16x2(f[4], f[5]); u.w = pack_bf16x2(f[6], f[7]);
     return u;
 }
+// true when no channel's running decay D * a would fall below 2^-40 (no rescale of R needed)
+__device__ __forceinline__ bool rescale_vote(const float* Dc, const float* a) {
+    bool ok = true;
+#pragma unroll
+    for (int j = 0; j < 8; ++j) ok = ok && Dc[j] * a[j] >= kRescaleMin;
+    return ok;
+}
+
 __device__ __forceinline__ float ldbf(const unsigned char* p) {
     return __bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(p));
+}
+__device__ __forceinline__ float rcp(float x) {  // 1/x on the SFU (about 1 ulp)
+    float y;
+    asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
 }
 __device__ __forceinline__ float lg2(float x) {  // log2 on the SFU (0 gives -inf)
     float y;
@@ -240,6 +255,12 @@ gla_chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
         const bool rot = ((cg >> 2) & 1) != 0;  // alternate float4 halves: no bank conflicts
         float* scan = reinterpret_cast<float*>(smem + OFF_SCAN);
         const uint32_t idesc_A = tc::idesc_bf16_f32(64, 64, 0, 0);
+        // The state is kept as S = diag(D) R with a running per-channel decay D (reset to 1 by a
+        // rescale of R when it would drop below 2^-40), so that chunk contributions enter R as
+        // k^/D without touching R: D of my 8 channels (same in every row-block thread)
+        float Dc[8];
+#pragma unroll
+        for (int j = 0; j < 8; ++j) Dc[j] = 1.f;
         for (int n = 0; n < n_ch; ++n) {
             const int st = n & 1;
             unsigned char* base = smem + st * STAGE_BYTES;
@@ -286,9 +307,30 @@ gla_chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
             for (int j = 0; j < 8; ++j) mine = mine && a[j] >= kFastMin;
             // vote (also a barrier: every gate and block product has been read past here)
             const bool fast = grp_all(1, mine);
+            // hand a, the rescale factor D.a and the route to warpgroup 1; advance D
+            auto publish = [&](bool rmw, const float* dn) {
+                if (rb == 0) {
+#pragma unroll
+                    for (int j = 0; j < 8; ++j) {
+                        abuf[(st * 2 + 0) * D + c0 + j] = a[j];
+                        abuf[(st * 2 + 1) * D + c0 + j] = Dc[j] * a[j];
+                    }
+                }
+                if (tid == 0) flag[st] = (fast ? 0 : kFlagExact) | (rmw ? kFlagRescale : 0);
+#pragma unroll
+                for (int j = 0; j < 8; ++j) Dc[j] = dn[j];
+            };
 
             if (fast) {
-                // q~ = q.G over q, k^ = k.a/G over k, k~ = k/G over the (consumed) gates
+                // q~ = q.G.D over q, k^ = k.(a/G)/D' over k, k~ = k/(G.D) over the (consumed) gates
+                const bool rmw = !grp_all(1, rescale_vote(Dc, a));
+                float dn[8], a_dn[8], inv_d[8];  // per-channel factors, hoisted out of the rows
+#pragma unroll
+                for (int j = 0; j < 8; ++j) {
+                    dn[j] = rmw ? 1.f : Dc[j] * a[j];
+                    a_dn[j] = a[j] * rcp(dn[j]);
+                    inv_d[j] = rcp(Dc[j]);
+                }
 #pragma unroll
                 for (int i = 0; i < 8; ++i) {
                     const uint32_t off = sw_off(r0 + i, c0, C);
@@ -298,11 +340,11 @@ gla_chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
 #pragma unroll
                     for (int j = 0; j < 8; ++j) {
                         const float Gt = G[i][j] * pre[j];
-                        const float r = __frcp_rn(Gt);
-                        kh[j] = kf[j] * (a[j] * r);
+                        const float r = rcp(Gt);
+                        kh[j] = kf[j] * (r * a_dn[j]);
                         if (MODE == PASS_C) {
-                            qt[j] = qf[j] * Gt;
-                            kt[j] = kf[j] * r;
+                            qt[j] = qf[j] * (Gt * Dc[j]);
+                            kt[j] = kf[j] * (r * inv_d[j]);
                         }
                     }
                     *reinterpret_cast<uint4*>(base + ST_K + off) = pack8(kh);
@@ -311,6 +353,7 @@ gla_chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                         *reinterpret_cast<uint4*>(base + ST_G + off) = pack8(kt);
                     }
                 }
+                publish(rmw, dn);
             } else {
                 // exact route: L = prefix sums of clamped log2 gates, block sums through shared memory
                 float L[8][8];
@@ -378,7 +421,11 @@ gla_chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                     tc::tmem_wait_st();
                     grp_sync(1);  // q, k and L read by every thread before they are overwritten
                 }
-                // q~ = q.2^L over q, k^ = k.2^(Ltot - L) over k
+                // q~ = q.2^L.D over q, k^ = k.2^(Ltot - L)/D' over k
+                const bool rmw = !grp_all(1, rescale_vote(Dc, a));
+                float dn[8];
+#pragma unroll
+                for (int j = 0; j < 8; ++j) dn[j] = rmw ? 1.f : Dc[j] * a[j];
 #pragma unroll
                 for (int i = 0; i < 8; ++i) {
                     const uint32_t off = sw_off(r0 + i, c0, C);
@@ -387,18 +434,14 @@ gla_chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                     if (MODE == PASS_C) unpack8(*reinterpret_cast<const uint4*>(base + ST_Q + off), qf);
 #pragma unroll
                     for (int j = 0; j < 8; ++j) {
-                        kh[j] = kf[j] * tc::ex2(Ltot[j] - L[i][j]);
-                        if (MODE == PASS_C) qt[j] = qf[j] * tc::ex2(L[i][j]);
+                        kh[j] = kf[j] * tc::ex2(Ltot[j] - L[i][j]) * rcp(dn[j]);
+                        if (MODE == PASS_C) qt[j] = qf[j] * (tc::ex2(L[i][j]) * Dc[j]);
                     }
                     *reinterpret_cast<uint4*>(base + ST_K + off) = pack8(kh);
                     if (MODE == PASS_C) *reinterpret_cast<uint4*>(base + ST_Q + off) = pack8(qt);
                 }
+                publish(rmw, dn);
             }
-            if (rb == 0) {
-#pragma unroll
-                for (int j = 0; j < 8; ++j) abuf[st * D + c0 + j] = a[j];
-            }
-            if (tid == 0) flag[st] = fast ? 0 : 1;
             asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
             tc::fence_before_sync();
             grp_sync(1);
@@ -432,25 +475,24 @@ gla_chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
         const uint32_t idesc_U = tc::idesc_bf16_f32(128, 128, 1, 1);
         const uint32_t idesc_O = tc::idesc_bf16_f32(64, 128, 0, 1);
         float a_seg = 1.f;                                 // PASS_A: decay over the segment
+        float Drow = 1.f;                                  // running decay D of state row c
         uint32_t nA0 = 0, nA1 = 0;                         // completed A phases per TMEM buffer
 
         auto epilogue = [&](int n) {  // O rows of chunk n -> bf16 global rows
             const int t0 = t_begin + n * C;
+            uint32_t r[D];
 #pragma unroll
-            for (int cb = 0; cb < D; cb += 32) {
-                uint32_t r[32];
-                tc::tmem_ld32(tmem + TM_O + lane_base + cb, r);
-                tc::tmem_wait_ld();
-                const int t = t0 + orow;
-                if (orow_ok && t < t_end) {
-                    __nv_bfloat16* dst = args.o + ((int64_t)bh * T + t) * D + cb;
+            for (int cb = 0; cb < D; cb += 32) tc::tmem_ld32(tmem + TM_O + lane_base + cb, r + cb);
+            tc::tmem_wait_ld();
+            const int t = t0 + orow;
+            if (orow_ok && t < t_end) {
+                __nv_bfloat16* dst = args.o + ((int64_t)bh * T + t) * D;
 #pragma unroll
-                    for (int i = 0; i < 32; i += 8) {
-                        float f[8];
+                for (int i = 0; i < D; i += 8) {
+                    float f[8];
 #pragma unroll
-                        for (int e = 0; e < 8; ++e) f[e] = __uint_as_float(r[i + e]);
-                        *reinterpret_cast<uint4*>(dst + i) = pack8(f);
-                    }
+                    for (int e = 0; e < 8; ++e) f[e] = __uint_as_float(r[i + e]);
+                    *reinterpret_cast<uint4*>(dst + i) = pack8(f);
                 }
             }
         };
@@ -460,65 +502,13 @@ gla_chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
             unsigned char* base = smem + st * STAGE_BYTES;
             if (!grp_all(2, wait_bar(&ops[st], (uint32_t)((n >> 1) & 1), abort_flag))) { ok = false; break; }
             tc::fence_after_sync();
-            const bool exact = flag[st] != 0;
-            const float a = abuf[st * D + c];
-            // the previous chunk's MMAs are done: its outputs, then S, S_bf and P are free
-            if (n > 0) {
-                if (!grp_all(2, wait_bar(barO, (uint32_t)((n - 1) & 1), abort_flag))) { ok = false; break; }
-                tc::fence_after_sync();
-                if (MODE == PASS_C) epilogue(n - 1);
-            }
-            // state row c: bf16 copy of S_in for the readout, then S <- diag(a) S, 32 columns at a time
-#pragma unroll
-            for (int jb = 0; jb < D; jb += 32) {
-                uint32_t r[32];
-                if (n == 0) {
-                    if (MODE == PASS_C) {
-                        const int slot = args.s_in_slots == 1 ? 0 : seg;
-                        const uint4* src = reinterpret_cast<const uint4*>(
-                            args.s_in + (((int64_t)bh * args.s_in_slots + slot) * D + c) * D + jb);
-#pragma unroll
-                        for (int e = 0; e < 8; ++e) {
-                            const uint4 v4 = src[e];
-                            r[4 * e] = v4.x; r[4 * e + 1] = v4.y; r[4 * e + 2] = v4.z; r[4 * e + 3] = v4.w;
-                        }
-                    } else {
-#pragma unroll
-                        for (int e = 0; e < 32; ++e) r[e] = 0u;
-                    }
-                } else {
-                    tc::tmem_ld32(tS + jb, r);
-                    tc::tmem_wait_ld();
-                }
-                if (MODE == PASS_C) {
-#pragma unroll
-                    for (int e = 0; e < 32; e += 8) {
-                        float f[8];
-#pragma unroll
-                        for (int x = 0; x < 8; ++x) f[x] = __uint_as_float(r[e + x]);
-                        *reinterpret_cast<uint4*>(smem + OFF_SBF + sw_off(c, jb + e, D)) = pack8(f);
-                    }
-                }
-#pragma unroll
-                for (int e = 0; e < 32; ++e) r[e] = __float_as_uint(__uint_as_float(r[e]) * a);
-                tc::tmem_st32(tS + jb, r);
-            }
-            tc::tmem_wait_st();
-            a_seg *= a;
-            asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-            tc::fence_before_sync();
-            grp_sync(2);
-            if (tid == 128) {  // S += k^^T V
-                tc::fence_after_sync();
-                const uint32_t kh = smem_u32(base + ST_K), va = smem_u32(base + ST_V);
-#pragma unroll
-                for (int k = 0; k < C / 16; ++k)
-                    tc::mma_ss(tmem + TM_S, tc::sdesc_sw128(kh + 2048u * k, BOX_BYTES, 1024),
-                               tc::sdesc_sw128(va + 2048u * k, BOX_BYTES, 1024), idesc_U, 1u);
-            }
+            const int fl = flag[st];
+            const bool exact = (fl & kFlagExact) != 0, rmw = (fl & kFlagRescale) != 0;
+            const float a_n = abuf[(st * 2 + 0) * D + c];
+            const float sig = abuf[(st * 2 + 1) * D + c];  // D_prev * a: R's rescale factor
             if (MODE == PASS_C) {
-                // P = mask(A) in bf16; A came from the tensor cores or, on the exact route, was
-                // stored into TMEM by warpgroup 0 before it signalled the operands
+                // P = mask(A) in bf16 into this stage (A came from the tensor cores or, on the
+                // exact route, was stored into TMEM by warpgroup 0 before the operands signal)
                 if (!exact) {
                     const uint32_t ph = st == 0 ? nA0 : nA1;
                     if (!grp_all(2, wait_bar(&barA[st], ph & 1, abort_flag))) { ok = false; break; }
@@ -535,16 +525,71 @@ gla_chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                         float f[8];
 #pragma unroll
                         for (int i = 0; i < 8; ++i) f[i] = s + i <= orow ? __uint_as_float(r[s + i]) : 0.f;
-                        *reinterpret_cast<uint4*>(smem + OFF_P + sw_off(orow, s, C)) = pack8(f);
+                        *reinterpret_cast<uint4*>(base + ST_P + sw_off(orow, s, C)) = pack8(f);
                     }
                 }
-                asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-                tc::fence_before_sync();
-                grp_sync(2);
-                if (tid == 128) {  // O = P V + q~ S_in
-                    tc::fence_after_sync();
-                    const uint32_t pa = smem_u32(smem + OFF_P), va = smem_u32(base + ST_V);
-                    const uint32_t qa = smem_u32(base + ST_Q), sb = smem_u32(smem + OFF_SBF);
+            }
+            // pass C needs the previous chunk's MMAs done every chunk (its outputs, S_bf reuse);
+            // pass A only when R is rescaled (S = diag(D) R takes new terms without touching R)
+            const bool need_prev = n > 0 && (MODE == PASS_C || rmw);
+            if (need_prev) {
+                if (!grp_all(2, wait_bar(barO, (uint32_t)((n - 1) & 1), abort_flag))) { ok = false; break; }
+                tc::fence_after_sync();
+                if (MODE == PASS_C) epilogue(n - 1);
+            }
+            // state row c: bf16 copy of R for the readout (S_in = diag(D) R, D folded into q~),
+            // and R <- sig R when the running decay is reset; R starts as S_in (pass C) or 0
+            if (MODE == PASS_C || (rmw && n > 0)) {
+                uint32_t r[D];
+                if (n == 0) {
+                    const int slot = args.s_in_slots == 1 ? 0 : seg;
+                    const uint4* src = reinterpret_cast<const uint4*>(
+                        args.s_in + (((int64_t)bh * args.s_in_slots + slot) * D + c) * D);
+#pragma unroll
+                    for (int e = 0; e < D / 4; ++e) {
+                        const uint4 v4 = src[e];
+                        r[4 * e] = v4.x; r[4 * e + 1] = v4.y; r[4 * e + 2] = v4.z; r[4 * e + 3] = v4.w;
+                    }
+                } else {
+#pragma unroll
+                    for (int jb = 0; jb < D; jb += 32) tc::tmem_ld32(tS + jb, r + jb);
+                    tc::tmem_wait_ld();
+                }
+                if (MODE == PASS_C) {
+#pragma unroll
+                    for (int e = 0; e < D; e += 8) {
+                        float f[8];
+#pragma unroll
+                        for (int x = 0; x < 8; ++x) f[x] = __uint_as_float(r[e + x]);
+                        *reinterpret_cast<uint4*>(smem + OFF_SBF + sw_off(c, e, D)) = pack8(f);
+                    }
+                }
+                if (n == 0 || rmw) {
+                    const float sc = rmw ? sig : 1.f;
+#pragma unroll
+                    for (int e = 0; e < D; ++e) r[e] = __float_as_uint(__uint_as_float(r[e]) * sc);
+#pragma unroll
+                    for (int jb = 0; jb < D; jb += 32) tc::tmem_st32(tS + jb, r + jb);
+                    tc::tmem_wait_st();
+                }
+            }
+            a_seg *= a_n;
+            Drow = rmw ? 1.f : sig;
+            asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+            tc::fence_before_sync();
+            grp_sync(2);
+            if (tid == 128) {
+                tc::fence_after_sync();
+                // R += k^'^T V (pass A starts from an empty R: the first MMA overwrites)
+                const uint32_t kh = smem_u32(base + ST_K), va = smem_u32(base + ST_V);
+#pragma unroll
+                for (int k = 0; k < C / 16; ++k)
+                    tc::mma_ss(tmem + TM_S, tc::sdesc_sw128(kh + 2048u * k, BOX_BYTES, 1024),
+                               tc::sdesc_sw128(va + 2048u * k, BOX_BYTES, 1024), idesc_U,
+                               (MODE == PASS_A && n == 0 && k == 0) ? 0u : 1u);
+                if (MODE == PASS_C) {  // O = P V + q~' R_bf16
+                    const uint32_t pa = smem_u32(base + ST_P), qa = smem_u32(base + ST_Q);
+                    const uint32_t sb = smem_u32(smem + OFF_SBF);
 #pragma unroll
                     for (int k = 0; k < C / 16; ++k)
                         tc::mma_ss(tmem + TM_O, tc::sdesc_sw128(pa + 32u * k, 16, 1024),
@@ -555,14 +600,12 @@ gla_chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                                    tc::sdesc_sw128(qa + (uint32_t)((k / 4) * BOX_BYTES + (k % 4) * 32), 16, 1024),
                                    tc::sdesc_sw128(sb + 2048u * k, D * 128, 1024), idesc_O, 1u);
                 }
-            }
-            if (tid == 128) {
                 tc::mma_commit(barO);
                 tc::mma_commit(&empty[st]);
             }
         }
 
-        // ---- tail: last chunk's outputs and the segment's state
+        // ---- tail: last chunk's outputs and the segment's state S = diag(D) R
         if (ok && n_ch > 0 && grp_all(2, wait_bar(barO, (uint32_t)((n_ch - 1) & 1), abort_flag))) {
             tc::fence_after_sync();
             if (MODE == PASS_C) epilogue(n_ch - 1);
@@ -580,7 +623,9 @@ gla_chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                 if (dst) {
 #pragma unroll
                     for (int i = 0; i < 32; i += 4)
-                        *reinterpret_cast<uint4*>(dst + j + i) = make_uint4(r[i], r[i + 1], r[i + 2], r[i + 3]);
+                        *reinterpret_cast<float4*>(dst + j + i) =
+                            make_float4(__uint_as_float(r[i]) * Drow, __uint_as_float(r[i + 1]) * Drow,
+                                        __uint_as_float(r[i + 2]) * Drow, __uint_as_float(r[i + 3]) * Drow);
                 }
             }
         }
@@ -595,6 +640,7 @@ gla_chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
     tc::fence_after_sync();
     if (warp == 8) tc::tmem_dealloc(tmem, 512);
 }
+
 // S_in(0) = state; S_in(m+1) = diag(a_m) S_in(m) + U_m in place of U_m, for every (b, h) and
 // state element; each thread owns 4 consecutive elements of one state row and walks the
 // segments in order, with the next segment's U loaded ahead of the dependent update.
