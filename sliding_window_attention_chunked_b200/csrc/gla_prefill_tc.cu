@@ -26,8 +26,9 @@
 // pass C recomputes every segment from its S_in and writes o (and the final state). One
 // segment means pass C alone.
 //
-// CTA (288 threads), a three-stage pipeline over the chunks of a segment:
-//   warp 8        TMA producer (q, k, v, g of chunk n into stage n % 2) and TMEM allocator;
+// CTA (384 threads = 3 warpgroups), a three-stage pipeline over the chunks of a segment:
+//   warp 8        TMA producer (q, k, v, g of chunk n into stage n % 2) and TMEM allocator
+//                 (warps 9-11 idle: they complete the warpgroup that gives its registers away);
 //   warpgroup 0   operands of chunk n: gate prefix products (8 rows x 8 channels per thread,
 //                 block products combined through shared memory), q~ and k^ in place over q
 //                 and k, k~ over the gates; thread 0 issues A = q~ k~^T into TMEM buffer n % 2;
@@ -52,7 +53,15 @@ __device__ unsigned int g_gla_tc_timeout = 0;
 
 constexpr int C = 64;                    // tokens per chunk
 constexpr int D = 128;                   // d_k = d_v
-constexpr int NTHREADS = 288;            // 2 warpgroups + producer warp
+constexpr int NTHREADS = 384;            // 3 warpgroups: operands, state, producer (+3 idle)
+// Register split (setmaxnreg). Each of the SM's four sub-partitions holds one warp of every
+// warpgroup, so per sub-partition the launch provides 3 x 168 = 504 registers per lane; the split
+// 232 (operands) + 216 (state) + 56 (producer warpgroup) = 504 uses exactly that.
+constexpr int kLaunchRegs = 168;
+constexpr int kOperandRegs = 232;
+constexpr int kStateRegs = 216;
+constexpr int kControlRegs = 56;
+static_assert(kOperandRegs + kStateRegs + kControlRegs <= 3 * kLaunchRegs, "register split exceeds launch");
 constexpr int BOX_BYTES = C * 128;       // one 64-row x 64-col bf16 box (128 B rows) = 8 KB
 constexpr int OP_BYTES = 2 * BOX_BYTES;  // one 64 x 128 bf16 operand = 16 KB
 constexpr int G_BYTES = C * D * 4;       // 64 x 128 fp32 gates = 32 KB
@@ -215,6 +224,9 @@ gla_chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
     const uint32_t tmem = *tmem_holder;
     bool ok = true;
 
+    if (warp >= 8) {
+        asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kControlRegs));
+    }
     if (warp == 8) {
         // ------------------------------- TMA producer -------------------------------
         if (lane == 0) {
@@ -248,6 +260,7 @@ gla_chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                 mbar_wait_bounded(&full[ni & 1], (uint32_t)((ni >> 1) & 1), kWaitLimit);
         }
     } else if (warp < 4) {
+        asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kOperandRegs));
         // ------------------------------- warpgroup 0: operands -------------------------------
         // thread = (channel group cg: channels 8cg..8cg+7, row block rb: rows 8rb..8rb+7)
         const int cg = tid & 15, rb = tid >> 4;
@@ -464,7 +477,8 @@ gla_chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
             tc::mma_commit(drain0);
             mbar_wait_bounded(drain0, 0, kWaitLimit);
         }
-    } else {
+    } else if (warp < 8) {
+        asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kStateRegs));
         // ------------------------- warpgroup 1: state, P, outputs, MMAs -------------------------
         const int c = tid - 128;                           // state row == TMEM lane
         const int wq = warp - 4;                           // TMEM lane quarter of this warp
