@@ -55,5 +55,11 @@ cudaError_t swska_decode_launch(const void* q, const void* k_new, const void* v_
                                 cudaStream_t stream);
 // read and clear the "bounded wait expired" flag of the decode attention kernel
 unsigned swska_decode_take_timeout_flag();
+// bf16, d_k = d_v = 128, H <= 16: one warp per head, producer warp, mbarrier ring
+bool swska_decode_warp_supported(int H, int dk, int dv);
+cudaError_t swska_decode_warp_launch(const void* q, const void* k_new, const void* v_new,
+                                     void* k_cache, void* v_cache, const int64_t* pos, void* o,
+                                     int N, int H, int window, float scale, cudaStream_t stream);
+unsigned swska_decode_warp_take_timeout_flag();
 
 }  // namespace rod

@@ -57,6 +57,7 @@ int rod_check(void* stream) {
     cudaError_t e = cudaStreamSynchronize(static_cast<cudaStream_t>(stream));
     if (e != cudaSuccess) return from_cuda(e);
     const unsigned flags = rod::swska_decode_take_timeout_flag() |
+                           rod::swska_decode_warp_take_timeout_flag() |
                            rod::swska_prefill_tc_take_timeout_flag() |
                            rod::gla_prefill_tc_take_timeout_flag();
     if (flags) return ROD_ERR_TIMEOUT;

@@ -314,6 +314,9 @@ cudaError_t swska_decode_launch(const void* q, const void* k_new, const void* v_
                                 int N, int H, int dk, int dv, int window, float scale, bool bf16,
                                 cudaStream_t stream) {
     if (N == 0) return cudaSuccess;
+    if (bf16 && swska_decode_warp_supported(H, dk, dv))
+        return swska_decode_warp_launch(q, k_new, v_new, k_cache, v_cache, pos, o, N, H, window,
+                                        scale, stream);
     return bf16 ? launch_t<__nv_bfloat16>(q, k_new, v_new, k_cache, v_cache, pos, o, N, H, dk, dv,
                                           window, scale, stream)
                 : launch_t<float>(q, k_new, v_new, k_cache, v_cache, pos, o, N, H, dk, dv,

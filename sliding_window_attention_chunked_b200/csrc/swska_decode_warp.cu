@@ -1,0 +1,429 @@
+// swska_decode_warp.cu -- SW-SKA decode for bf16 caches with d_k = d_v = 128 and up to 16 heads:
+// one warp per head, one producer warp, an mbarrier ring with no block-wide barrier per stage.
+//
+// Semantics as in swska_decode.cu (SALA blog §3.3: the rolling window is a circular buffer,
+// slot(p) = p mod W; CodeFuse Rodimus* article, Fig. 4 / SKA paragraph: one K row per position
+// shared by every head, one V row per head):
+//   o[n,h] = softmax over p in [max(0, P-W+1), P] of scale * q[n,h] . K[slot(p)], applied to
+//            V[h, slot(p)],  with P = pos[n] and the new token stored at slot(P) first.
+//
+// Bound by HBM: per sequence and slot one 256-byte K row and H 256-byte V rows are read once.
+//  * A thread-block cluster of SP CTAs serves one sequence; CTA r streams a contiguous run of
+//    the valid slots. SP is chosen on the host from the number of clusters that fit at once.
+//  * Warp H (the producer) moves KT-slot stages into a ring in shared memory with bulk async
+//    copies: one for the K rows and one per head for its V rows (each contiguous in the cache).
+//    The slot the new token overwrites is never read from the cache: its rows are written into
+//    the stage (and into the cache) from k_new / v_new, and the copies skip it.
+//  * Warp h (head h), lane l owns channels 4l .. 4l+3. Scores: each lane forms partial dots of
+//    q_h with the stage's K rows over its channels; a reduce-scatter across the warp leaves the
+//    score of slot j in lanes 4j .. 4j+3. The products are bf16 x bf16 FMAs into fp32
+//    (fma.rn.f32.bf16), so the rows are used without unpacking. The online softmax runs in base
+//    2 (scores times scale * log2 e); p_j, rounded to bf16 like the probabilities of the
+//    tensor-core prefill, is broadcast by shuffle and accumulated into the lane's 4 output
+//    columns from V_h. Shared-memory reads are 8 bytes per lane over a 256-byte row: no bank
+//    conflicts.
+//  * Stage hand-off: full[b] completes when the copies land (transaction bytes), empty[b] when
+//    all H head warps have read the stage.
+//  * The SP partial (max, sum, accumulator) triples meet in distributed shared memory; CTA r
+//    finalises the heads h with h mod SP == r.
+// Every wait is bounded. On expiry the waiting warp raises the CTA's abort flag, every role stops
+// at its next wait, the producer waits (bounded) for the copies it issued, the timeout flag is
+// raised, the affected outputs are NaN, and all threads still meet at the cluster barriers.
+#include <cooperative_groups.h>
+
+#include <math.h>
+
+#include <mutex>
+
+#include "common.cuh"
+#include "kernels.h"
+
+namespace cg = cooperative_groups;
+
+namespace rod {
+namespace {
+
+__device__ unsigned int g_swska_decode_warp_timeout = 0;
+
+constexpr int KT = 8;            // slots per stage
+constexpr int STAGES = 3;        // ring depth
+constexpr int DH = 128;          // d_k = d_v
+constexpr int ROW = DH * 2;      // bytes of one bf16 row
+constexpr int MAX_H = 16;
+constexpr int OFF_FLAG = 64;     // after 2 * STAGES mbarriers
+constexpr int OFF_PM = 128;      // per-head max   [16] f32
+constexpr int OFF_PL = 192;      // per-head sum   [16] f32
+constexpr int OFF_PACC = 256;    // per-head accumulator [H][128] f32
+
+__host__ __device__ constexpr uint32_t stage_bytes(int H) { return (uint32_t)(KT * ROW * (1 + H)); }
+__host__ __device__ constexpr uint32_t ring_offset(int H) { return (uint32_t)(OFF_PACC + H * DH * 4); }
+__host__ __device__ constexpr uint32_t smem_total(int H) { return ring_offset(H) + STAGES * stage_bytes(H); }
+
+__device__ __forceinline__ bool wait_stage(uint64_t* bar, uint32_t parity, volatile int* abort_flag) {
+    for (uint32_t i = 1;; ++i) {
+        if (mbar_try_wait(bar, parity)) return true;
+        if ((i & 255u) == 0) {
+            if (*abort_flag) return false;
+            if (i >= kWaitLimit) {
+                *abort_flag = 1;
+                atomicExch(&g_swska_decode_warp_timeout, 1u);
+                return false;
+            }
+        }
+    }
+}
+
+__device__ __forceinline__ float ex2_approx(float x) {  // 2^x on the SFU (x = -inf gives 0)
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+
+
+
+// c + a.lo * b.lo + a.hi * b.hi for two packed bf16 pairs: bf16 operands, fp32 products and sum
+__device__ __forceinline__ float dot2_bf16(uint32_t a, uint32_t b, float c) {
+    asm("{\n\t.reg .b16 al, ah, bl, bh;\n\tmov.b32 {al, ah}, %1;\n\tmov.b32 {bl, bh}, %2;\n\t"
+        "fma.rn.f32.bf16 %0, al, bl, %0;\n\tfma.rn.f32.bf16 %0, ah, bh, %0;\n\t}"
+        : "+f"(c) : "r"(a), "r"(b));
+    return c;
+}
+// acc[i] += p * v[i] for the 4 bf16 of w, p a bf16 in the low half of pw; fp32 accumulation
+__device__ __forceinline__ void axpy4_bf16(uint32_t pw, uint2 w, float* acc) {
+    asm("{\n\t.reg .b16 p, ph, v0, v1, v2, v3;\n\tmov.b32 {p, ph}, %4;\n\tmov.b32 {v0, v1}, %5;\n\t"
+        "mov.b32 {v2, v3}, %6;\n\tfma.rn.f32.bf16 %0, p, v0, %0;\n\tfma.rn.f32.bf16 %1, p, v1, %1;\n\t"
+        "fma.rn.f32.bf16 %2, p, v2, %2;\n\tfma.rn.f32.bf16 %3, p, v3, %3;\n\t}"
+        : "+f"(acc[0]), "+f"(acc[1]), "+f"(acc[2]), "+f"(acc[3]) : "r"(pw), "r"(w.x), "r"(w.y));
+}
+
+struct HeadState {
+    float acc[4] = {0.f, 0.f, 0.f, 0.f};  // output columns 4 lane .. 4 lane + 3, unnormalised
+    float m_run = -INFINITY;               // running max of the base-2 scores (warp-uniform)
+    float l_part = 0.f;                    // this lane's share of the running sum
+};
+
+// One stage of KT slots for one head. kb / vb point at this lane's 8 bytes of the stage's first
+// K row and first V row of the head (rows ROW bytes apart). FULL: all KT rows are valid.
+template <bool FULL>
+__device__ __forceinline__ void head_stage(const unsigned char* kb, const unsigned char* vb, uint2 qw,
+                                           float scale_log2, int rows, int lane, HeadState& hs) {
+    // partial dots over this lane's 4 channels, one per slot
+    float part[KT];
+#pragma unroll
+    for (int j = 0; j < KT; ++j) {
+        const uint2 kw = *reinterpret_cast<const uint2*>(kb + j * ROW);
+        part[j] = dot2_bf16(kw.y, qw.y, dot2_bf16(kw.x, qw.x, 0.f));
+    }
+    // reduce-scatter over the warp: halves of the slot set cross lane bit 4, then bit 3, then
+    // bit 2; bits 1 and 0 finish the sums. Lane l ends with the score of slot (l >> 2) & 7.
+    const bool b4 = (lane & 16) != 0, b3 = (lane & 8) != 0, b2 = (lane & 4) != 0;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const float send = b4 ? part[i] : part[i + 4];
+        const float keep = b4 ? part[i + 4] : part[i];
+        part[i] = keep + __shfl_xor_sync(0xffffffffu, send, 16);
+    }
+#pragma unroll
+    for (int i = 0; i < 2; ++i) {
+        const float send = b3 ? part[i] : part[i + 2];
+        const float keep = b3 ? part[i + 2] : part[i];
+        part[i] = keep + __shfl_xor_sync(0xffffffffu, send, 8);
+    }
+    float dot;
+    {
+        const float send = b2 ? part[0] : part[1];
+        const float keep = b2 ? part[1] : part[0];
+        dot = keep + __shfl_xor_sync(0xffffffffu, send, 4);
+    }
+    dot += __shfl_xor_sync(0xffffffffu, dot, 2);
+    dot += __shfl_xor_sync(0xffffffffu, dot, 1);
+    float s = dot * scale_log2;  // base-2 softmax
+    if (!FULL && ((lane >> 2) & (KT - 1)) >= rows) s = -INFINITY;
+    float mx = fmaxf(s, __shfl_xor_sync(0xffffffffu, s, 4));
+    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 8));
+    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 16));
+    if (mx > hs.m_run) {  // uniform branch
+        const float alpha = ex2_approx(hs.m_run - mx);  // m_run = -inf gives 0
+        hs.l_part *= alpha;
+#pragma unroll
+        for (int i = 0; i < 4; ++i) hs.acc[i] *= alpha;
+        hs.m_run = mx;
+    }
+    // p in bf16 (as the weights of V); the sum takes the same rounded value
+    const __nv_bfloat16 pb = __float2bfloat16_rn(ex2_approx(s - hs.m_run));  // past the end: 0
+    if ((lane & 3) == 0) hs.l_part += __bfloat162float(pb);
+    const uint32_t pw = (uint32_t)__bfloat16_as_ushort(pb);
+#pragma unroll
+    for (int j = 0; j < KT; ++j) {
+        const uint32_t pj = __shfl_sync(0xffffffffu, pw, 4 * j);
+        if (FULL || j < rows) {  // rows past the end hold stale bytes
+            const uint2 vw = *reinterpret_cast<const uint2*>(vb + j * ROW);
+            axpy4_bf16(pj, vw, hs.acc);
+        }
+    }
+}
+
+__global__ void __launch_bounds__(32 * (MAX_H + 1), 2)
+swska_decode_warp_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ k_new,
+                         const __nv_bfloat16* __restrict__ v_new, __nv_bfloat16* __restrict__ k_cache,
+                         __nv_bfloat16* __restrict__ v_cache, const int64_t* __restrict__ pos,
+                         __nv_bfloat16* __restrict__ o, int H, int W, float scale_log2) {
+    extern __shared__ __align__(128) unsigned char smem[];
+    cg::cluster_group cluster = cg::this_cluster();
+    const int SP = (int)cluster.num_blocks();
+    const int rank = (int)cluster.block_rank();
+    const int64_t n = blockIdx.x / SP;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const uint32_t SB = stage_bytes(H);
+    uint64_t* full = reinterpret_cast<uint64_t*>(smem);
+    uint64_t* empty = full + STAGES;
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + OFF_FLAG);
+    float* s_pm = reinterpret_cast<float*>(smem + OFF_PM);
+    float* s_pl = reinterpret_cast<float*>(smem + OFF_PL);
+    float* s_pacc = reinterpret_cast<float*>(smem + OFF_PACC);
+    unsigned char* ring = smem + ring_offset(H);
+
+    const int64_t P = pos[n];
+    const bool bad = P < 0;
+    const int64_t cnt = bad ? 0 : (P + 1 < W ? P + 1 : W);  // valid slots 0 .. cnt-1
+    const int64_t s_new = bad ? -1 : P % W;
+    const int64_t per = (cnt + SP - 1) / SP;
+    const int64_t s_begin = (int64_t)rank * per < cnt ? (int64_t)rank * per : cnt;
+    const int64_t s_end = s_begin + per < cnt ? s_begin + per : cnt;
+    const int nst = (int)((s_end - s_begin + KT - 1) / KT);
+    const __nv_bfloat16* Kc = k_cache + n * (int64_t)W * DH;
+    const __nv_bfloat16* Vc = v_cache + n * (int64_t)H * W * DH;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < STAGES; ++s) {
+            mbar_init(&full[s], 1);
+            mbar_init(&empty[s], (uint32_t)H);
+        }
+        *abort_flag = 0;
+        fence_mbar_init();
+    }
+    __syncthreads();
+
+    if (warp == H) {
+        // ---------------------------------- producer warp ----------------------------------
+        int issued = 0;
+        for (int st = 0; st < nst; ++st) {
+            const int buf = st % STAGES;
+            if (st >= STAGES) {
+                const bool ok = wait_stage(&empty[buf], (uint32_t)(((st / STAGES) - 1) & 1), abort_flag);
+                if (!__all_sync(0xffffffffu, ok)) break;
+            }
+            const int64_t s0 = s_begin + (int64_t)st * KT;
+            const int rows = (int)((s_end - s0) < KT ? (s_end - s0) : KT);
+            unsigned char* dst = ring + (size_t)buf * SB;
+            const int r_new = (s_new >= s0 && s_new < s0 + rows) ? (int)(s_new - s0) : -1;
+            if (r_new >= 0) {
+                // the evicted slot takes the new token: into the stage and into the cache
+                // (its old content lies outside the window, so it is never copied in)
+                for (int i = lane; i < (1 + H) * (ROW / 16); i += 32) {
+                    const int row = i / (ROW / 16), c16 = i % (ROW / 16);
+                    const uint4* src = row == 0
+                        ? reinterpret_cast<const uint4*>(k_new + n * DH)
+                        : reinterpret_cast<const uint4*>(v_new + (n * H + (row - 1)) * (int64_t)DH);
+                    const uint4 val = src[c16];
+                    reinterpret_cast<uint4*>(dst + (size_t)row * KT * ROW + (size_t)r_new * ROW)[c16] = val;
+                    uint4* gdst = row == 0
+                        ? reinterpret_cast<uint4*>(k_cache + (n * (int64_t)W + s_new) * DH)
+                        : reinterpret_cast<uint4*>(v_cache + ((n * H + (row - 1)) * (int64_t)W + s_new) * DH);
+                    gdst[c16] = val;
+                }
+                // the generic stores precede later bulk copies into the same bytes
+                asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+            }
+            __syncwarp();
+            const int copied = rows - (r_new >= 0 ? 1 : 0);
+            if (lane == 0) mbar_arrive_expect_tx(&full[buf], (uint32_t)(copied * ROW * (1 + H)));
+            __syncwarp();
+            if (lane <= H) {  // lane 0: the K rows; lane 1 + h: head h's V rows
+                unsigned char* d = dst + (size_t)lane * KT * ROW;
+                const __nv_bfloat16* src = lane == 0 ? Kc + s0 * DH : Vc + ((int64_t)(lane - 1) * W + s0) * DH;
+                const int a0 = 0, a1 = r_new >= 0 ? r_new : rows;   // rows [a0, a1)
+                const int b0 = r_new >= 0 ? r_new + 1 : rows, b1 = rows;  // rows [b0, b1)
+                if (a1 > a0) bulk_g2s(d + (size_t)a0 * ROW, src + (int64_t)a0 * DH, (uint32_t)((a1 - a0) * ROW), &full[buf]);
+                if (b1 > b0) bulk_g2s(d + (size_t)b0 * ROW, src + (int64_t)b0 * DH, (uint32_t)((b1 - b0) * ROW), &full[buf]);
+            }
+            ++issued;
+        }
+        // every copy issued has landed before the CTA's shared memory can go away (in the normal
+        // course the head warps waited for these phases already)
+        if (lane == 0) {
+            for (int s2 = issued > STAGES ? issued - STAGES : 0; s2 < issued; ++s2)
+                if (!mbar_wait_bounded(&full[s2 % STAGES], (uint32_t)((s2 / STAGES) & 1), kWaitLimit))
+                    atomicExch(&g_swska_decode_warp_timeout, 1u);
+        }
+        __syncwarp();
+    }
+    else {
+        // ------------------------------- head warp h = warp --------------------------------
+        const int h = warp;
+        const uint2 qw = *reinterpret_cast<const uint2*>(q + (n * H + h) * (int64_t)DH + 4 * lane);
+        HeadState hs;
+        bool ok = true;
+        for (int st = 0; st < nst; ++st) {
+            const int buf = st % STAGES;
+            if (!__all_sync(0xffffffffu, wait_stage(&full[buf], (uint32_t)((st / STAGES) & 1), abort_flag))) {
+                ok = false;
+                break;
+            }
+            const int64_t s0 = s_begin + (int64_t)st * KT;
+            const int rows = (int)((s_end - s0) < KT ? (s_end - s0) : KT);
+            const unsigned char* kb = ring + (size_t)buf * SB + 8 * lane;
+            const unsigned char* vb = kb + (size_t)(1 + h) * KT * ROW;
+            if (rows == KT) head_stage<true>(kb, vb, qw, scale_log2, KT, lane, hs);
+            else head_stage<false>(kb, vb, qw, scale_log2, rows, lane, hs);
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&empty[buf]);
+        }
+        float l = hs.l_part;
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) l += __shfl_xor_sync(0xffffffffu, l, off);
+        if (lane == 0) { s_pm[h] = ok ? hs.m_run : NAN; s_pl[h] = l; }
+        *reinterpret_cast<float4*>(s_pacc + h * DH + 4 * lane) =
+            make_float4(hs.acc[0], hs.acc[1], hs.acc[2], hs.acc[3]);
+    }
+    cluster.sync();
+    // ---- combine: CTA `rank` finalises the heads h with h mod SP == rank (warp h, 4 columns a lane)
+    if (warp < H && warp % SP == rank) {
+        const int h = warp;
+        float out[4];
+        if (bad) {
+#pragma unroll
+            for (int i = 0; i < 4; ++i) out[i] = NAN;
+        } else {
+            float M = -INFINITY;
+            for (int r = 0; r < SP; ++r) M = fmaxf(M, cluster.map_shared_rank(s_pm, r)[h]);
+            float L = 0.f, a[4] = {0.f, 0.f, 0.f, 0.f};
+            for (int r = 0; r < SP; ++r) {
+                const float mr = cluster.map_shared_rank(s_pm, r)[h];
+                const float lr = cluster.map_shared_rank(s_pl, r)[h];
+                if (!(lr > 0.f) && !isnan(mr)) continue;  // a CTA without slots
+                const float w = ex2_approx(mr - M);
+                L = fmaf(w, lr, L);
+                const float4 pa = *reinterpret_cast<const float4*>(cluster.map_shared_rank(s_pacc, r) + h * DH + 4 * lane);
+                a[0] = fmaf(w, pa.x, a[0]); a[1] = fmaf(w, pa.y, a[1]);
+                a[2] = fmaf(w, pa.z, a[2]); a[3] = fmaf(w, pa.w, a[3]);
+            }
+            const float inv = 1.f / L;
+#pragma unroll
+            for (int i = 0; i < 4; ++i) out[i] = a[i] * inv;
+        }
+        store4(o + (n * H + h) * (int64_t)DH + 4 * lane, make_float4(out[0], out[1], out[2], out[3]));
+    }
+    cluster.sync();  // this CTA's shared memory stays alive until every peer has read it
+}
+
+
+// Clusters of each size that the GPU holds at once for this kernel (queried once per device and
+// head count; 0 if the size cannot be launched).
+int clusters_that_fit(int H, int sp) {
+    static std::mutex mu;
+    static int cache[64][MAX_H + 1][4];
+    static bool init = false;
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 0;
+    const int si = sp == 1 ? 0 : sp == 2 ? 1 : sp == 4 ? 2 : 3;
+    std::lock_guard<std::mutex> lock(mu);
+    if (!init) {
+        for (auto& a : cache)
+            for (auto& b : a)
+                for (int& c : b) c = -1;
+        init = true;
+    }
+    int& slot = cache[dev][H][si];
+    if (slot < 0) {
+        cudaLaunchConfig_t cfg = {};
+        cfg.gridDim = dim3((unsigned)sp, 1, 1);
+        cfg.blockDim = dim3((unsigned)(32 * (H + 1)), 1, 1);
+        cfg.dynamicSmemBytes = smem_total(H);
+        cudaLaunchAttribute attr[1];
+        attr[0].id = cudaLaunchAttributeClusterDimension;
+        attr[0].val.clusterDim.x = (unsigned)sp;
+        attr[0].val.clusterDim.y = 1;
+        attr[0].val.clusterDim.z = 1;
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+        int num = 0;
+        if (cudaOccupancyMaxActiveClusters(&num, swska_decode_warp_kernel, &cfg) != cudaSuccess) {
+            cudaGetLastError();
+            num = 0;
+        }
+        slot = num;
+    }
+    return slot;
+}
+
+// Split of the window over a cluster. One CTA streams its slots at about 1/200 of the GPU's HBM
+// bandwidth (31-32 GB/s a CTA against 6.4 TB/s, measured with this kernel on B200), so about 200
+// CTAs in flight saturate HBM; a larger split past that adds cluster waves and combine work and
+// no bandwidth. Estimated time in slot-steps: the larger of the HBM bound N W / 200 and
+// (waves of CTAs) x (slots per CTA), over SP in {1, 2, 4, 8}; ties go to the smaller split.
+constexpr double kCtasToSaturate = 200.0;
+
+int pick_split(int N, int H, int W) {
+    int best = 1;
+    double best_cost = -1.0;
+    const double t_hbm = (double)N * (double)W / kCtasToSaturate;
+    for (int sp = 1; sp <= 8; sp *= 2) {
+        const int64_t cap = (int64_t)clusters_that_fit(H, sp) * sp;  // CTAs resident at once
+        if (cap <= 0) continue;
+        const int64_t ctas = (int64_t)N * sp;
+        const double waves = (double)((ctas + cap - 1) / cap);
+        const double t = waves * (double)((W + sp - 1) / sp);
+        const double cost = t > t_hbm ? t : t_hbm;
+        if (best_cost < 0.0 || cost < best_cost) {
+            best_cost = cost;
+            best = sp;
+        }
+    }
+    return best;
+}
+
+}  // namespace
+
+bool swska_decode_warp_supported(int H, int dk, int dv) {
+    return dk == DH && dv == DH && H >= 1 && H <= MAX_H;
+}
+
+cudaError_t swska_decode_warp_launch(const void* q, const void* k_new, const void* v_new,
+                                     void* k_cache, void* v_cache, const int64_t* pos, void* o,
+                                     int N, int H, int window, float scale, cudaStream_t stream) {
+    if (N == 0) return cudaSuccess;
+    const size_t smem = smem_total(H);
+    cudaError_t e = cudaFuncSetAttribute(swska_decode_warp_kernel,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    const int SP = pick_split(N, H, window);
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)((int64_t)N * SP), 1, 1);
+    cfg.blockDim = dim3((unsigned)(32 * (H + 1)), 1, 1);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = (unsigned)SP;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    const float scale_log2 = scale * 1.4426950408889634f;
+    note_launches(1);
+    return cudaLaunchKernelEx(&cfg, swska_decode_warp_kernel,
+                              static_cast<const __nv_bfloat16*>(q), static_cast<const __nv_bfloat16*>(k_new),
+                              static_cast<const __nv_bfloat16*>(v_new), static_cast<__nv_bfloat16*>(k_cache),
+                              static_cast<__nv_bfloat16*>(v_cache), pos, static_cast<__nv_bfloat16*>(o), H,
+                              window, scale_log2);
+}
+
+unsigned swska_decode_warp_take_timeout_flag() {
+    unsigned v = 0, zero = 0;
+    if (cudaMemcpyFromSymbol(&v, g_swska_decode_warp_timeout, sizeof(v)) != cudaSuccess) return 0;
+    cudaMemcpyToSymbol(g_swska_decode_warp_timeout, &zero, sizeof(zero));
+    return v;
+}
+
+}  // namespace rod

@@ -254,14 +254,29 @@ def test_swska_decode_bf16_cluster_split(W):
     _ska_decode_check(7, 4, 128, 128, W, "bf16", full=True, seed=W + 1)
 
 
+@pytest.mark.parametrize("H", [1, 3, 16, 20])
+def test_swska_decode_bf16_heads(H):
+    """H <= 16 runs one warp per head, H = 20 the general kernel: both against the oracle."""
+    _ska_decode_check(6, H, 128, 128, 300, "bf16", full=False, seed=40 + H)
+    _ska_decode_check(6, H, 128, 128, 300, "bf16", full=True, seed=50 + H)
+
+
+@pytest.mark.parametrize("W", [1, 2, 7, 8, 9, 17])
+def test_swska_decode_bf16_small_windows(W):
+    """Windows shorter than, equal to and just past one stage of slots; W = 1 gives o = v_new."""
+    _ska_decode_check(9, 2, 128, 128, W, "bf16", full=False, seed=60 + W)
+    _ska_decode_check(9, 2, 128, 128, W, "bf16", full=True, seed=70 + W)
+
+
 def test_swska_decode_full_workload_sampled():
     d = wl.WORKLOADS["decode_n256"].dims
     _ska_decode_check(d["N"], d["H"], d["dk"], d["dv"], d["window"], "bf16", full=True,
                       check_n=20)
 
 
-def test_swska_decode_negative_position_gives_nan_and_keeps_cache():
-    N, H, d, W = 3, 2, 64, 32
+@pytest.mark.parametrize("d", [64, 128])
+def test_swska_decode_negative_position_gives_nan_and_keeps_cache(d):
+    N, H, W = 3, 2, 32
     dd = wl.decode_inputs(N, H, d, d, W, seed=5, dtype="bf16", full=False)
     pos = dd["pos"].clone()
     pos[1] = -5
