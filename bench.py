@@ -299,7 +299,7 @@ def run_gpu(args):
                 "peak": peak_tf, "unit": "TFLOP/s", "frac": round(achieved_tflops / peak_tf, 4),
                 "peak_source": f"{peaks_src} (bf16_tflops_sustained: kernel timed inside a long step)",
                 "flop_per_launch": ska_flop, "avg_launch_ms": round(ska_avg_ms, 4),
-                "traffic": recorded_traffic("swska_prefill_stack", ["swska_prefill_simt.cu"])}
+                "traffic": recorded_traffic("swska_prefill_stack", ["swska_prefill_tc.cu", "tc.cuh", "common.cuh"])}
 
     # ---- batched decode step (recurrence + SW-SKA), 256 sequences ----
     dd_dims = wl.WORKLOADS["decode_n256"].dims
@@ -350,12 +350,16 @@ def run_gpu(args):
                                     "algorithmic_bytes": gla_dec_bytes,
                                     "achieved": round(gla_dec_bytes / (gla_dec_ms / 1e3) / 1e9, 1),
                                     "peak": hbm, "unit": "GB/s",
-                                    "frac": round(gla_dec_bytes / (gla_dec_ms / 1e3) / 1e9 / hbm, 4)},
+                                    "frac": round(gla_dec_bytes / (gla_dec_ms / 1e3) / 1e9 / hbm, 4),
+                                    "traffic": recorded_traffic("gla_decode_n256",
+                                                                ["gla_decode.cu", "common.cuh"])},
             "rod_swska_decode": {"bound": "hbm", "avg_launch_ms": round(ska_dec_ms, 4),
                                  "algorithmic_bytes": ska_dec_bytes,
                                  "achieved": round(ska_dec_bytes / (ska_dec_ms / 1e3) / 1e9, 1),
                                  "peak": hbm, "unit": "GB/s",
-                                 "frac": round(ska_dec_bytes / (ska_dec_ms / 1e3) / 1e9 / hbm, 4)},
+                                 "frac": round(ska_dec_bytes / (ska_dec_ms / 1e3) / 1e9 / hbm, 4),
+                                 "traffic": recorded_traffic("swska_decode_n256",
+                                                             ["swska_decode_warp.cu", "common.cuh"])},
         },
     }
 
@@ -368,7 +372,9 @@ def run_gpu(args):
         "rod_gla_prefill": {"bound": "hbm", "avg_layer_ms": round(gla_ms_per_layer, 4),
                             "algorithmic_bytes": gla_bytes,
                             "achieved_gbs": round(gla_bytes / (gla_ms_per_layer / 1e3) / 1e9, 1),
-                            "frac_hbm": round(gla_bytes / (gla_ms_per_layer / 1e3) / 1e9 / hbm, 4)},
+                            "frac_hbm": round(gla_bytes / (gla_ms_per_layer / 1e3) / 1e9 / hbm, 4),
+                            "traffic": recorded_traffic("gla_prefill_stack",
+                                                        ["gla_prefill_tc.cu", "tc.cuh", "common.cuh"])},
     }
 
     # ---- end to end through the public API with host buffers ----
@@ -481,6 +487,62 @@ def run_reference(args):
     print(json.dumps(line), flush=True)
 
 
+def run_profile_case(args):
+    """One kernel family on one layer of the stack workload (or one decode batch), for ncu:
+    warm-up + steps launches, each timed with CUDA events; no stack, no e2e, no oracle. The
+    device holds one layer's inputs (about 1.6 GB for SW-SKA, 3 GB for the recurrence) or the
+    decode caches of --profile-n sequences (17 MiB each)."""
+    import torch
+
+    import sliding_window_attention_chunked_b200 as rod
+    from sliding_window_attention_chunked_b200 import build as rbuild
+    from sliding_window_attention_chunked_b200 import workloads as wl
+
+    torch.cuda.set_device(0)
+    dev = torch.device("cuda", 0)
+    rbuild.build()
+    rod.load_library()
+    d = wl.WORKLOADS[WORKLOAD].dims
+    B, H, T, dk, dv, W, C = d["B"], d["H"], d["T"], d["dk"], d["dv"], d["window"], d["chunk"]
+    case = args.profile_case
+    if case in ("ska_prefill", "gla_prefill"):
+        layer = 1 if case == "ska_prefill" else 0
+        ins = wl.stack_layer_inputs(layer, B, H, T, dk, dv, device=dev)
+        out = torch.empty(B, H, T, dv, dtype=torch.bfloat16, device=dev)
+        if case == "ska_prefill":
+            q, k, v = ins
+            fn = lambda: rod.swska_prefill(q, k, v, W, o=out)
+        else:
+            q, k, v, g = ins
+            st = torch.zeros(B, H, dk, dv, device=dev)
+            ws = torch.empty(max(rod.gla_prefill_workspace_size(B, H, T, dk, dv, C), 16),
+                             dtype=torch.uint8, device=dev)
+            fn = lambda: rod.gla_prefill(q, k, v, g, st.zero_(), o=out, chunk=C, workspace=ws)
+    else:
+        N, Wd = args.profile_n, wl.WORKLOADS["decode_n256"].dims["window"]
+        dd = wl.decode_inputs(N, H, dk, dv, Wd, seed=77, device=dev)
+        o = torch.empty(N, H, dv, dtype=torch.bfloat16, device=dev)
+        if case == "ska_decode":
+            fn = lambda: rod.swska_decode(dd["sq"], dd["k_new"], dd["v_new"], dd["k_cache"],
+                                          dd["v_cache"], dd["pos"], Wd, o=o)
+        else:
+            fn = lambda: rod.gla_decode_step(dd["q"], dd["k"], dd["v"], dd["g"], dd["state"], o=o)
+    for _ in range(args.warmup):
+        fn()
+    rod.check()
+    times = []
+    for _ in range(args.steps):
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        fn()
+        e1.record()
+        torch.cuda.synchronize()
+        times.append(e0.elapsed_time(e1))
+    rod.check()
+    print(json.dumps({"profile_case": case, "launch_ms": [round(t, 4) for t in times],
+                      "n": args.profile_n if case.endswith("decode") else None}), flush=True)
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -490,9 +552,14 @@ def main():
     ap.add_argument("--e2e-steps", type=int, default=1)
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--profile-case", choices=["ska_prefill", "gla_prefill", "ska_decode", "gla_decode"],
+                    help="run one kernel family alone (for ncu captures) and exit")
+    ap.add_argument("--profile-n", type=int, default=128, help="sequences for the decode cases")
     args = ap.parse_args()
     args.warmup = max(3, args.warmup)  # timing rule: at least 3 untimed warm-up steps
-    if args.impl == "reference":
+    if args.profile_case:
+        run_profile_case(args)
+    elif args.impl == "reference":
         run_reference(args)
     else:
         run_gpu(args)

@@ -10,7 +10,7 @@
 // One CTA computes a 128-query tile for a PAIR of heads of one sequence (with an odd head
 // count the last pair computes its single head twice and stores it once). Each shared key tile
 // is brought into shared memory once by TMA and feeds both heads' score MMAs (the pair's
-// remaining reuse of K across the other heads goes through L2). Warp roles (320 threads):
+// remaining reuse of K across the other heads goes through L2). Warp roles (384 threads):
 //   warps 0-3   softmax warpgroup of head 0 (thread i owns query row i = TMEM lane i)
 //   warps 4-7   softmax warpgroup of head 1
 //   warp  8     TMA producer: Q once, then K_j, V0_j, V1_j into a ring of 32 KB slots
@@ -23,7 +23,9 @@
 // lets each head's softmax run while the tensor core works on the other head. Softmax is in
 // base 2 on scores pre-scaled by scale*log2(e), with lazy rescaling: the running maximum used
 // for the exponent only moves when a row's maximum grows by more than 8 (so P <= 256), and
-// then the O row is rescaled in TMEM by its owning thread. Every wait is bounded; a timeout
+// then the O row is rescaled in TMEM by its owning thread. The row maximum runs as eight
+// independent chains of three-input maxima, and the exponent arguments and the row sum use the
+// two-wide fp32 instructions (fma.rn.f32x2 / add.rn.f32x2). Every wait is bounded; a timeout
 // makes all roles stop, drain their in-flight copies and MMAs, and raise a flag.
 #include <cuda.h>
 #include <math.h>
@@ -72,6 +74,27 @@ __device__ __forceinline__ bool wait_bar(uint64_t* bar, uint32_t parity, volatil
             }
         }
     }
+}
+
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+    float d;
+    asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+    return d;
+}
+// two-wide fp32 fma / add (one instruction for both lanes of the pair)
+__device__ __forceinline__ float2 ffma2(float2 a, float2 b, float2 c) {
+    float2 d;
+    asm("{\n\t.reg .b64 ra, rb, rc, rd;\n\tmov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\t"
+        "mov.b64 rc, {%6, %7};\n\tfma.rn.f32x2 rd, ra, rb, rc;\n\tmov.b64 {%0, %1}, rd;\n\t}"
+        : "=f"(d.x), "=f"(d.y) : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y), "f"(c.x), "f"(c.y));
+    return d;
+}
+__device__ __forceinline__ float2 fadd2(float2 a, float2 b) {
+    float2 d;
+    asm("{\n\t.reg .b64 ra, rb, rd;\n\tmov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\t"
+        "add.rn.f32x2 rd, ra, rb;\n\tmov.b64 {%0, %1}, rd;\n\t}"
+        : "=f"(d.x), "=f"(d.y) : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
+    return d;
 }
 
 __global__ void __launch_bounds__(NTHREADS, 1)
@@ -258,28 +281,44 @@ swska_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                 for (int c = 0; c < BN; ++c)
                     if (c < lo || c > hi) s[c] = 0xff800000u;  // -inf
             }
-            float mx = __uint_as_float(s[0]);
+            // row maximum: 8 independent chains of 3-input maxima over the columns c = 8k + i
+            float m8[8];
 #pragma unroll
-            for (int c = 1; c < BN; ++c) mx = fmaxf(mx, __uint_as_float(s[c]));
+            for (int i = 0; i < 8; ++i) {
+                float m = __uint_as_float(s[i]);
+#pragma unroll
+                for (int k = 1; k < 15; k += 2)
+                    m = fmax3(m, __uint_as_float(s[8 * k + i]), __uint_as_float(s[8 * k + 8 + i]));
+                m8[i] = fmaxf(m, __uint_as_float(s[120 + i]));
+            }
+            const float mx = fmax3(fmax3(m8[0], m8[1], m8[2]), fmax3(m8[3], m8[4], m8[5]), fmaxf(m8[6], m8[7]));
             const float m_tile = mx * scale_log2;
             const bool need = m_tile > m_run + kRescaleThreshold;
             const float alpha = need ? tc::ex2(m_run - m_tile) : 1.f;  // 0 when m_run = -inf
             l_run *= alpha;
             if (need) m_run = m_tile;
             const float m_use = m_run == -INFINITY ? 0.f : m_run;
-            // P = 2^(s * scale * log2 e - m) as bf16 pairs over the first 64 columns of S
+            // P = 2^(s * scale * log2 e - m) as bf16 pairs over the first 64 columns of S; the
+            // exponent arguments and the row sum use packed two-wide fp32 arithmetic, the sum in
+            // four independent accumulators
+            const float2 sc2 = make_float2(scale_log2, scale_log2), nm2 = make_float2(-m_use, -m_use);
+            float2 l4[4] = {{0.f, 0.f}, {0.f, 0.f}, {0.f, 0.f}, {0.f, 0.f}};
 #pragma unroll
             for (int half = 0; half < 2; ++half) {
                 uint32_t pk[32];
 #pragma unroll
                 for (int i = 0; i < 32; ++i) {
                     const int c = 64 * half + 2 * i;
-                    const float p0 = tc::ex2(fmaf(__uint_as_float(s[c]), scale_log2, -m_use));
-                    const float p1 = tc::ex2(fmaf(__uint_as_float(s[c + 1]), scale_log2, -m_use));
-                    l_run += p0 + p1;
-                    pk[i] = pack_bf16x2(p0, p1);
+                    const float2 x = ffma2(make_float2(__uint_as_float(s[c]), __uint_as_float(s[c + 1])), sc2, nm2);
+                    const float2 p = make_float2(tc::ex2(x.x), tc::ex2(x.y));
+                    l4[i & 3] = fadd2(l4[i & 3], p);
+                    pk[i] = pack_bf16x2(p.x, p.y);
                 }
                 tc::tmem_st32(tS + 32u * half, pk);
+            }
+            {
+                const float2 a = fadd2(l4[0], l4[1]), b2 = fadd2(l4[2], l4[3]), t2 = fadd2(a, b2);
+                l_run += t2.x + t2.y;
             }
             // a row whose maximum moved rescales its O row (PV of the previous tile is done:
             // this tile's S was committed after it)
