@@ -196,22 +196,26 @@ swska_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                 tc::fence_after_sync();
                 return ok;
             };
+            // descriptors built once; a K step adds its offset (bytes >> 4) to the low word
+            const uint64_t dq0 = tc::sdesc_sw128(q_base, 16, 1024);
+            const uint64_t dq1 = tc::sdesc_sw128(q_base + TILE_BYTES, 16, 1024);
+            const uint32_t dk_hi = tc::desc_hi(tc::sdesc_sw128(q_base, 16, 1024));  // LBO 16, SBO 1024
+            const uint32_t dv_hi = tc::desc_hi(tc::sdesc_sw128(q_base, HALF_BYTES, 1024));
             auto issue_s = [&](int h, int L) {
-                const uint32_t bb = ring(L);
+                const uint32_t a_lo = tc::desc_lo(h ? dq1 : dq0), a_hi = tc::desc_hi(h ? dq1 : dq0);
+                const uint32_t b_lo = tc::desc_lo(tc::sdesc_sw128(ring(L), 16, 1024));
 #pragma unroll
                 for (int k = 0; k < HD / 16; ++k) {
-                    const uint32_t koff = (uint32_t)((k / 4) * HALF_BYTES + (k % 4) * 32);
-                    tc::mma_ss(tmem + 256u * h, tc::sdesc_sw128(q_base + h * TILE_BYTES + koff, 16, 1024),
-                               tc::sdesc_sw128(bb + koff, 16, 1024), idesc_s, k > 0);
+                    const uint32_t koff = (uint32_t)(((k / 4) * HALF_BYTES + (k % 4) * 32) >> 4);
+                    tc::mma_ss_lh(tmem + 256u * h, a_lo + koff, a_hi, b_lo + koff, dk_hi, idesc_s, k > 0);
                 }
             };
             auto issue_pv = [&](int h, int L, bool acc) {
-                const uint32_t bb = ring(L);
+                const uint32_t b_lo = tc::desc_lo(tc::sdesc_sw128(ring(L), HALF_BYTES, 1024));
 #pragma unroll
                 for (int k = 0; k < BN / 16; ++k)
-                    tc::mma_ts(tmem + 256u * h + 128u, tmem + 256u * h + 8u * k,
-                               tc::sdesc_sw128(bb + 2048u * k, HALF_BYTES, 1024),
-                               idesc_o, (acc || k > 0) ? 1u : 0u);
+                    tc::mma_ts_lh(tmem + 256u * h + 128u, tmem + 256u * h + 8u * k, b_lo + (uint32_t)((2048 * k) >> 4),
+                                  dv_hi, idesc_o, (acc || k > 0) ? 1u : 0u);
             };
             bool ok = wait_bar(qfull, 0, abort_flag);
             tc::fence_after_sync();
@@ -223,21 +227,27 @@ swska_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                 tc::mma_commit(&empty[0]);
                 for (int j = 0; j < n_it; ++j) {
                     const bool more = j + 1 < n_it;
-                    if (!wait_bar(&pfull[0], (uint32_t)(j & 1), abort_flag)) break;
-                    tc::fence_after_sync();
+                    // V0_j first (it landed long ago), then the softmax hand-off; the next key
+                    // tile is only tested, so PV0 is never delayed by it, and when it is there
+                    // PV0 and S0 go to the tensor core back to back (an empty issue queue costs
+                    // the pipe's start latency again)
                     if (!acquire(3 * j + 1)) break;
+                    if (!wait_bar(&pfull[0], (uint32_t)(j & 1), abort_flag)) break;
+                    const bool k_ready =
+                        more && mbar_test_wait(&full[(3 * j + 3) % NSLOT], (uint32_t)(((3 * j + 3) / NSLOT) & 1));
+                    tc::fence_after_sync();
                     issue_pv(0, 3 * j + 1, j > 0);
                     tc::mma_commit(&empty[(3 * j + 1) % NSLOT]);
                     if (more) {
-                        if (!acquire(3 * j + 3)) break;
+                        if (!k_ready && !acquire(3 * j + 3)) break;
                         issue_s(0, 3 * j + 3);
                         tc::mma_commit(&sfull[0]);
                     } else {
                         tc::mma_commit(&odone[0]);
                     }
+                    if (!acquire(3 * j + 2)) break;
                     if (!wait_bar(&pfull[1], (uint32_t)(j & 1), abort_flag)) break;
                     tc::fence_after_sync();
-                    if (!acquire(3 * j + 2)) break;
                     issue_pv(1, 3 * j + 2, j > 0);
                     tc::mma_commit(&empty[(3 * j + 2) % NSLOT]);
                     if (more) {
