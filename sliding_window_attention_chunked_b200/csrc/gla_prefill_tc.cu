@@ -15,10 +15,13 @@
 //     A = q~ k~^T (masked to s <= t, rounded to bf16 as P),  O = P V + q~ S_in,  S += k^^T V
 // while the fp32 state lives in tensor memory for the whole segment. k~ = k/G needs G well
 // inside the fp32/bf16 exponent range, so a chunk in which some channel's product a falls below
-// 2^-100 takes the exact route instead: the scores are summed on the CUDA cores from log2-gate
+// 2^-60 takes the exact route instead: the scores are summed on the CUDA cores from log2-gate
 // prefix sums L (log2 g clamped at -126, so g = 0 contributes below fp32 resolution),
 // A_ts = sum_c q_tc k_sc 2^(L_tc - L_sc), and written straight into tensor memory, where the
 // tensor-core route would have put them; q~ = q.2^L and k^ = k.2^(L_last - L).
+// The state is held as S = diag(D) R with a running per-channel decay D: a chunk multiplies D
+// by a and adds (k^/D)^T V to R, so R is never read and rewritten per chunk; D is folded into
+// q~ for the readout, and R is rescaled (D reset to 1) only when D would fall below 2^-40.
 //
 // Parallelism over the sequence: the T tokens are cut into segments of L_seg tokens. Pass A
 // (per segment but the last) computes the segment's state contribution U and decay a_seg
@@ -26,15 +29,17 @@
 // pass C recomputes every segment from its S_in and writes o (and the final state). One
 // segment means pass C alone.
 //
-// CTA (384 threads = 3 warpgroups), a three-stage pipeline over the chunks of a segment:
-//   warp 8        TMA producer (q, k, v, g of chunk n into stage n % 2) and TMEM allocator
-//                 (warps 9-11 idle: they complete the warpgroup that gives its registers away);
+// CTA (384 threads = 3 warpgroups, setmaxnreg 232 / 216 / 56), a pipeline over the chunks of
+// a segment through two 80 KB stages:
+//   warp 8        TMA producer (q, k, v, g of chunk n into stage n % 2, L2 prefetch of later
+//                 chunks) and TMEM allocator (warps 9-11 idle: they complete the warpgroup
+//                 that gives its registers away);
 //   warpgroup 0   operands of chunk n: gate prefix products (8 rows x 8 channels per thread,
 //                 block products combined through shared memory), q~ and k^ in place over q
 //                 and k, k~ over the gates; thread 0 issues A = q~ k~^T into TMEM buffer n % 2;
-//   warpgroup 1   state work of chunk n-1 ... n: output rows of the previous chunk, the state
-//                 row c (thread c = TMEM lane c) copied to bf16 for the readout and scaled by a,
-//                 P = mask(A), and thread 128 issues S += k^^T V and O = P V + q~ S_in.
+//   warpgroup 1   state work: P = mask(A) of chunk n into the stage, output rows of chunk n-1,
+//                 the state row c (thread c = TMEM lane c) copied to bf16 for the readout, and
+//                 thread 128 issues R += k^'^T V and O = P V + q~' R_bf16.
 // So the operands of chunk n+1 are built while chunk n's state work and MMAs run.
 // TMEM: S (cols 0-127, M=128), O (128-255, M=64: rows in lanes 0-15 of each 32-lane quarter),
 // A0 / A1 (256-319 / 320-383, M=64). Every wait is bounded; a timeout stops all roles, drains
@@ -687,10 +692,21 @@ struct Plan {
     int L_seg, n_seg;
 };
 
+// Segments per (b, h): one wave of the output pass (one CTA per SM), i.e. floor(SMs / (B H)),
+// at least 1. Measured on B200 (recurrence layer, d = 128): at B4 H16 T4096 two segments per
+// head take 240 us against 271 us for a single segment (the sequential schedule) and 284 us for
+// four waves; at B1 H16 T131072 nine segments take 1330 us against 1374 us for four waves.
+// Fewer segments also mean fewer k, v, g bytes read twice (segment pass and output pass).
 Plan plan(int B, int H, int T) {
     const int64_t BH = (int64_t)B * H;
     const int chunks = (T + C - 1) / C;
-    int64_t want = (4 * 148 + BH - 1) / BH;  // about four waves of one-CTA-per-SM units
+    int dev = 0, sms = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || sms < 1) {
+        cudaGetLastError();
+        sms = 148;
+    }
+    int64_t want = BH > 0 ? sms / BH : 1;
     if (want < 1) want = 1;
     if (want > chunks) want = chunks;
     const int per = (int)((chunks + want - 1) / want);
