@@ -181,6 +181,22 @@ ROD_API int rod_swska_decode(const void* q, const void* k_new, const void* v_new
                      void* v_cache, const int64_t* pos, void* o, int N, int H, int dk, int dv,
                      int window, float scale, int dtype, void* stream);
 
+/* ---- SW-SKA: prefill -> decode hand-off ----------------------------------------------------- */
+/*
+ * Fills the decode ring buffers from a prefill's keys and values (SALA blog §3.3: chunked
+ * prefill, then decode over a self-managed circular window buffer; CodeFuse article, SKA
+ * paragraph: one shared K, per-head V). After a prefill of T tokens every position
+ * p in [max(0, T-W), T) is copied to slot p mod W:
+ *   k_cache[b, p mod W, :] = k[b, p, :];   v_cache[b, h, p mod W, :] = v[b, h, p, :]
+ * so that rod_swska_decode with pos = T attends over exactly the window prefill row T would.
+ *   k [B,T,dk], v [B,H,T,dv]: dtype, read;  k_cache [B,W,dk], v_cache [B,H,W,dv]: dtype,
+ *   written (slots not named above are left untouched).  window W >= 1.
+ * Errors: ROD_ERR_NULL, ROD_ERR_SHAPE (H > 64, dims unsupported, window < 1), ROD_ERR_ALIGN,
+ * ROD_ERR_DTYPE, ROD_ERR_CUDA. B = 0 or T = 0 is a no-op.
+ */
+ROD_API int rod_swska_cache_fill(const void* k, const void* v, void* k_cache, void* v_cache, int B,
+                                 int H, int T, int dk, int dv, int window, int dtype, void* stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -41,8 +41,10 @@ class OracleLib:
         lib.rodref_swska_decode.argtypes = [f32p, f32p, f32p, f32p, f32p, i64p, f64p,
                                             i64, i64, i64, i64, i64, ctypes.c_double,
                                             ctypes.c_int]
+        lib.rodref_swska_cache_fill.argtypes = [f32p, f32p, f32p, f32p, i64, i64, i64, i64, i64,
+                                                i64]
         for name in ("rodref_gla_prefill", "rodref_gla_decode_step", "rodref_swska_prefill",
-                     "rodref_swska_decode"):
+                     "rodref_swska_decode", "rodref_swska_cache_fill"):
             getattr(lib, name).restype = ctypes.c_int
         self.lib = lib
         self.path = path
@@ -194,3 +196,17 @@ def swska_decode(q, k_new, v_new, k_cache, v_cache, pos, window, scale=None, nth
                                   nthreads or default_threads())
     _check(rc, "swska_decode")
     return o, kc, vc
+
+
+def swska_cache_fill(k, v, k_cache, v_cache, window):
+    """Prefill -> decode hand-off (rodref_swska_cache_fill). Returns float32 copies of the
+    caches with positions max(0, T-W) .. T-1 of k [B,T,dk] and v [B,H,T,dv] in slots p mod W."""
+    k, v = _f32(k), _f32(v)
+    kc, vc = _f32(k_cache).copy(), _f32(v_cache).copy()
+    B, T, dk = k.shape
+    H, dv = v.shape[1], v.shape[-1]
+    W = int(window)
+    assert v.shape == (B, H, T, dv) and kc.shape == (B, W, dk) and vc.shape == (B, H, W, dv)
+    rc = _L().rodref_swska_cache_fill(_p32(k), _p32(v), _p32(kc), _p32(vc), B, H, T, dk, dv, W)
+    _check(rc, "swska_cache_fill")
+    return kc, vc

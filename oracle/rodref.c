@@ -300,4 +300,24 @@ int rodref_swska_decode(const float* q, const float* k_new, const float* v_new, 
     return run_units(ska_dec_unit, &a, N * H, nthreads);
 }
 
+/* Prefill -> decode hand-off (SALA blog §3.3: decode keeps the most recent W tokens in a
+ * circular buffer; the ring rule is the one rodref_swska_decode writes by): every position p in
+ * [max(0, T-W), T) of the prefill's shared keys k [B,T,dk] and per-head values v [B,H,T,dv] is
+ * copied to slot p mod W of k_cache [B,W,dk] and v_cache [B,H,W,dv]. Other slots are untouched. */
+int rodref_swska_cache_fill(const float* k, const float* v, float* k_cache, float* v_cache,
+                            int64_t B, int64_t H, int64_t T, int64_t dk, int64_t dv, int64_t W) {
+    if (!k || !v || !k_cache || !v_cache) return RODREF_EINVAL;
+    if (B < 0 || H < 1 || T < 0 || dk < 1 || dv < 1 || W < 1) return RODREF_EINVAL;
+    const int64_t p0 = T > W ? T - W : 0;
+    for (int64_t b = 0; b < B; ++b)
+        for (int64_t p = p0; p < T; ++p) {
+            const int64_t slot = p % W;
+            memcpy(k_cache + (b * W + slot) * dk, k + (b * T + p) * dk, (size_t)dk * sizeof(float));
+            for (int64_t h = 0; h < H; ++h)
+                memcpy(v_cache + ((b * H + h) * W + slot) * dv, v + ((b * H + h) * T + p) * dv,
+                       (size_t)dv * sizeof(float));
+        }
+    return 0;
+}
+
 int rodref_abi_version(void) { return 1; }

@@ -9,6 +9,7 @@ the calls raise.
     gla_decode_step(q, k, v, g, state)              one fused recurrent decode step
     swska_prefill(q, k, v, window, scale=None)      sliding-window shared-key attention
     swska_decode(q, k_new, v_new, k_cache, v_cache, pos, window)   ring-buffer decode
+    swska_cache_fill(k, v, k_cache, v_cache, window)   prefill -> decode ring-buffer hand-off
 """
 from ._binding import (  # noqa: F401
     ROD_BF16,
@@ -23,6 +24,7 @@ from ._binding import (  # noqa: F401
     launch_count,
     library_path,
     load_library,
+    swska_cache_fill,
     swska_decode,
     swska_prefill,
 )

@@ -65,6 +65,8 @@ def load_library() -> ctypes.CDLL:
     lib.rod_swska_prefill.restype = i
     lib.rod_swska_decode.argtypes = [vp, vp, vp, vp, vp, vp, vp, i, i, i, i, i, f, i, vp]
     lib.rod_swska_decode.restype = i
+    lib.rod_swska_cache_fill.argtypes = [vp, vp, vp, vp, i, i, i, i, i, i, i, vp]
+    lib.rod_swska_cache_fill.restype = i
     _lib = lib
     return lib
 
@@ -240,3 +242,22 @@ def swska_decode(q, k_new, v_new, k_cache, v_cache, pos, window, scale=None, o=N
                                          float(scale or 0.0), _dtype_code(q), _stream(stream))
     _raise_on("rod_swska_decode", st)
     return o
+
+
+def swska_cache_fill(k, v, k_cache, v_cache, window, stream=None):
+    """Prefill -> decode hand-off: k [B,T,dk], v [B,H,T,dv] into the ring buffers k_cache
+    [B,W,dk], v_cache [B,H,W,dv] (position p of the last W goes to slot p mod W)."""
+    _need(k, "k", None, 3)
+    _need(v, "v", k.dtype, 4)
+    _need(k_cache, "k_cache", k.dtype, 3)
+    _need(v_cache, "v_cache", k.dtype, 4)
+    B, T, dk = k.shape
+    H, dv = v.shape[1], v.shape[-1]
+    W = int(window)
+    if (tuple(v.shape) != (B, H, T, dv) or tuple(k_cache.shape) != (B, W, dk)
+            or tuple(v_cache.shape) != (B, H, W, dv)):
+        raise ValueError("shape mismatch")
+    st = load_library().rod_swska_cache_fill(_ptr(k), _ptr(v), _ptr(k_cache), _ptr(v_cache), B, H, T,
+                                             dk, dv, W, _dtype_code(k), _stream(stream))
+    _raise_on("rod_swska_cache_fill", st)
+    return k_cache, v_cache

@@ -62,4 +62,9 @@ cudaError_t swska_decode_warp_launch(const void* q, const void* k_new, const voi
                                      int N, int H, int window, float scale, cudaStream_t stream);
 unsigned swska_decode_warp_take_timeout_flag();
 
+// SW-SKA prefill -> decode hand-off: the last W tokens' K / V rows into the ring buffers
+cudaError_t swska_cache_fill_launch(const void* k, const void* v, void* k_cache, void* v_cache, int B,
+                                    int H, int T, int dk, int dv, int window, size_t elem_bytes,
+                                    cudaStream_t stream);
+
 }  // namespace rod

@@ -146,4 +146,18 @@ int rod_swska_decode(const void* q, const void* k_new, const void* v_new, void* 
                                               static_cast<cudaStream_t>(stream)));
 }
 
+int rod_swska_cache_fill(const void* k, const void* v, void* k_cache, void* v_cache, int B, int H,
+                         int T, int dk, int dv, int window, int dtype, void* stream) {
+    if (!dtype_ok(dtype)) return ROD_ERR_DTYPE;
+    if (B < 0 || H < 1 || H > 64 || T < 0 || window < 1 || !dim_ok(dk) || !dim_ok(dv))
+        return ROD_ERR_SHAPE;
+    if (B == 0 || T == 0) return ROD_OK;
+    if (!k || !v || !k_cache || !v_cache) return ROD_ERR_NULL;
+    if (!aligned16(k) || !aligned16(v) || !aligned16(k_cache) || !aligned16(v_cache))
+        return ROD_ERR_ALIGN;
+    return from_cuda(rod::swska_cache_fill_launch(k, v, k_cache, v_cache, B, H, T, dk, dv, window,
+                                                  dtype == ROD_BF16 ? 2 : 4,
+                                                  static_cast<cudaStream_t>(stream)));
+}
+
 }  // extern "C"

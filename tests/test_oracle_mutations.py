@@ -3,7 +3,7 @@
 Each case copies oracle/rodref.c to a temporary directory, plants one plausible mistake by a
 textual substitution (a gate applied to the wrong channel, a decay that also hits the new
 term, the readout using k, an off-by-one window, a dropped scale or normaliser, a wrong
-ring-buffer slot), builds the copy with gcc and runs every pin against it. Each planted
+ring-buffer slot, a hand-off that drops a token or numbers slots from the window start), builds the copy with gcc and runs every pin against it. Each planted
 mistake must make at least one pin fail; otherwise the pins are too weak to trust.
 """
 import inspect
@@ -33,6 +33,10 @@ MUTATIONS = {
                              "const int64_t slot = (pos[n] + 1) % W;"),
     "decode_window_too_wide": ("const int64_t p0 = P - a->W + 1 > 0 ? P - a->W + 1 : 0;",
                                "const int64_t p0 = P - a->W > 0 ? P - a->W : 0;"),
+    "cache_fill_drops_oldest": ("const int64_t p0 = T > W ? T - W : 0;",
+                                "const int64_t p0 = T > W ? T - W + 1 : 0;"),
+    "cache_fill_slot_from_start": ("const int64_t slot = p % W;",
+                                   "const int64_t slot = (p - p0) % W;"),
 }
 
 

@@ -274,3 +274,42 @@ def test_swska_ring_buffer_decode_equals_prefill_row(W, positions):
     for n, p in enumerate(positions):
         np.testing.assert_array_equal(kc2[n, p % W], k[0, p])
         np.testing.assert_array_equal(vc2[n, :, p % W], v[0, :, p])
+
+
+@pytest.mark.parametrize("W,T,steps", [(8, 5, 6), (8, 8, 4), (5, 23, 7), (1, 4, 3)])
+def test_swska_cache_fill_then_decode_continues_the_prefill(W, T, steps):
+    """Prefill -> decode hand-off (SALA blog §3.3): fill the ring buffers from a T-token prefill,
+    then decode positions T .. T+steps-1 one at a time; each decode output equals the prefill
+    output row of the whole sequence at that position, and slots the fill does not name keep
+    their previous contents."""
+    H, dk, dv, B = 3, 6, 5, 2
+    total = T + steps
+    q, k, v = _ska_case(B=B, H=H, T=total, dk=dk, dv=dv, seed=11)
+    o_pre = oracle.swska_prefill(q, k, v, W)
+    kc = np.full((B, W, dk), 9.0, np.float32)
+    vc = np.full((B, H, W, dv), 9.0, np.float32)
+    kc, vc = oracle.swska_cache_fill(k[:, :T], v[:, :, :T], kc, vc, W)
+    if T < W:
+        assert (kc[:, T:] == 9.0).all() and (vc[:, :, T:] == 9.0).all()
+    for P in range(T, total):
+        o, kc, vc = oracle.swska_decode(q[:, :, P], k[:, P], v[:, :, P], kc, vc,
+                                        np.full(B, P, np.int64), W)
+        _close(o, o_pre[:, :, P], 1e-13)
+
+
+@pytest.mark.parametrize("W,T", [(8, 5), (8, 8), (5, 23), (1, 4), (6, 13)])
+def test_swska_cache_fill_equals_decode_writes(W, T):
+    """The hand-off fill leaves the caches exactly as T decode steps at positions 0 .. T-1
+    would (each writes its token at slot p mod W; the ring rule of the decode is pinned by the
+    decode tests above): the last W tokens, each in its slot, other slots untouched."""
+    H, dk, dv, B = 2, 4, 3, 2
+    q, k, v = _ska_case(B=B, H=H, T=T, dk=dk, dv=dv, seed=12)
+    kc0 = np.full((B, W, dk), 9.0, np.float32)
+    vc0 = np.full((B, H, W, dv), 9.0, np.float32)
+    kf, vf = oracle.swska_cache_fill(k, v, kc0, vc0, W)
+    kd, vd = kc0, vc0
+    for p in range(T):
+        _, kd, vd = oracle.swska_decode(q[:, :, p], k[:, p], v[:, :, p], kd, vd,
+                                        np.full(B, p, np.int64), W)
+    np.testing.assert_array_equal(kf, kd)
+    np.testing.assert_array_equal(vf, vd)
