@@ -384,6 +384,12 @@ def run_gpu(args):
 
     del layers, dd
     torch.cuda.empty_cache()
+
+    # ---- generation loop: one token through all 24 layers' decode kernels, eager vs graph ----
+    generate = None
+    if not args.no_generate:
+        generate = run_generate(rod, torch, wl, dev, L, H, dk, W, seed_base, barrier, ranks_max,
+                                world)
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         cpu = oracle_stack_sample(d)
@@ -401,12 +407,62 @@ def run_gpu(args):
                    "parallelism": f"replicas x{world} (independent sequences, no collective)",
                    "l2": "inputs > L2 (55 GB per step), no flush needed"},
         "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": launches,
-        "clocks": clocks, "decode": decode, "kernels": kernels,
+        "clocks": clocks, "decode": decode, "generate": generate, "kernels": kernels,
     }
     if rank == 0:
         print(json.dumps(line), flush=True)
     if world > 1:
         dist.destroy_process_group()
+
+
+def run_generate(rod, torch, wl, dev, L, H, d, W, seed_base, barrier, reduce_max, world):
+    """Per-token decode step of the whole L-layer stack (every layer's decode kernel, then the
+    position advance) for N sequences with full windows: eager launches against one CUDA-graph
+    replay per token. Caches, states and per-step inputs are seeded random, resident in HBM."""
+    from sliding_window_attention_chunked_b200.generate import MixerStack
+
+    out = {"workload": f"{L}-layer Rodimus+ decode step (alternating recurrence / SW-SKA, H={H}, "
+                       f"d={d}, window {W}, full windows), one token per sequence",
+           "unit": "ms per token step", "runs": []}
+    for N in (1, 256):
+        stack = MixerStack(L, N, H, d, W, device=dev)
+        gen = torch.Generator(device=dev)
+        gen.manual_seed(seed_base + 9000 + N)
+        for lay in stack.layers:
+            for key, t in lay.items():
+                if key == "g":
+                    t.uniform_(0.9, 1.0, generator=gen)
+                else:
+                    t.normal_(generator=gen)
+        pos = wl.decode_positions(N, W, full=True, device=dev)
+        stack.pos.copy_(pos)
+        for _ in range(3):
+            stack.step_eager()
+        rod.check()
+        steps = 50 if N == 1 else 20
+
+        def timed(fn):
+            barrier()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            for _ in range(steps):
+                fn()
+            e1.record()
+            barrier()
+            return reduce_max(e0.elapsed_time(e1) / steps)
+
+        eager_ms = timed(stack.step_eager)
+        stack.capture()
+        for _ in range(3):
+            stack.step()
+        graph_ms = timed(stack.step)
+        rod.check()
+        out["runs"].append({"N": N, "eager_ms": round(eager_ms, 4), "graph_ms": round(graph_ms, 4),
+                            "graph_tokens_per_s": round(N * world / (graph_ms / 1e3), 1),
+                            "kernels_per_step": stack.kernels_per_step()})
+        del stack
+        torch.cuda.empty_cache()
+    return out
 
 
 def run_e2e(args, rod, torch, layers, d, ws, stream, barrier, reduce_max, world):
@@ -552,6 +608,7 @@ def main():
     ap.add_argument("--e2e-steps", type=int, default=1)
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-generate", action="store_true")
     ap.add_argument("--profile-case", choices=["ska_prefill", "gla_prefill", "ska_decode", "gla_decode"],
                     help="run one kernel family alone (for ncu captures) and exit")
     ap.add_argument("--profile-n", type=int, default=128, help="sequences for the decode cases")

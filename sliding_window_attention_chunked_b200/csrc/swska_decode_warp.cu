@@ -8,12 +8,16 @@
 //            V[h, slot(p)],  with P = pos[n] and the new token stored at slot(P) first.
 //
 // Bound by HBM: per sequence and slot one 256-byte K row and H 256-byte V rows are read once.
-//  * A thread-block cluster of SP CTAs serves one sequence; CTA r streams a contiguous run of
-//    the valid slots. SP is chosen on the host from the number of clusters that fit at once.
-//  * Warp H (the producer) moves KT-slot stages into a ring in shared memory with bulk async
+//  * The grid is (N x SP) x (H / HG): a thread-block cluster of SP CTAs (up to 16) splits one
+//    sequence's window into contiguous runs of valid slots, and each CTA serves a group of HG
+//    heads (the shared K rows are then read once per head group). The host picks SP and HG
+//    from the batch: large batches keep all heads in one CTA (K read once), small ones split
+//    heads and window so that enough CTAs stream at once.
+//  * Warp HG (the producer) moves KT-slot stages into a ring in shared memory with bulk async
 //    copies: one for the K rows and one per head for its V rows (each contiguous in the cache).
-//    The slot the new token overwrites is never read from the cache: its rows are written into
-//    the stage (and into the cache) from k_new / v_new, and the copies skip it.
+//    The ring depth is a launch parameter (about 64 KB in flight per CTA). The slot the new
+//    token overwrites is never read from the cache: its rows are written into the stage (and
+//    into the cache) from k_new / v_new, and the copies skip it.
 //  * Warp h (head h), lane l owns channels 4l .. 4l+3. Scores: each lane forms partial dots of
 //    q_h with the stage's K rows over its channels; a reduce-scatter across the warp leaves the
 //    score of slot j in lanes 4j .. 4j+3. The products are bf16 x bf16 FMAs into fp32
@@ -23,7 +27,7 @@
 //    columns from V_h. Shared-memory reads are 8 bytes per lane over a 256-byte row: no bank
 //    conflicts.
 //  * Stage hand-off: full[b] completes when the copies land (transaction bytes), empty[b] when
-//    all H head warps have read the stage.
+//    all HG head warps have read the stage.
 //  * The SP partial (max, sum, accumulator) triples meet in distributed shared memory; CTA r
 //    finalises the heads h with h mod SP == r.
 // Every wait is bounded. On expiry the waiting warp raises the CTA's abort flag, every role stops
@@ -46,18 +50,21 @@ namespace {
 __device__ unsigned int g_swska_decode_warp_timeout = 0;
 
 constexpr int KT = 8;            // slots per stage
-constexpr int STAGES = 3;        // ring depth
+constexpr int MAX_STAGES = 16;   // ring depth limit (the depth is a launch parameter)
 constexpr int DH = 128;          // d_k = d_v
 constexpr int ROW = DH * 2;      // bytes of one bf16 row
-constexpr int MAX_H = 16;
-constexpr int OFF_FLAG = 64;     // after 2 * STAGES mbarriers
-constexpr int OFF_PM = 128;      // per-head max   [16] f32
-constexpr int OFF_PL = 192;      // per-head sum   [16] f32
-constexpr int OFF_PACC = 256;    // per-head accumulator [H][128] f32
+constexpr int MAX_H = 16;        // heads per CTA (one warp each)
+constexpr int OFF_FLAG = 256;    // after full[MAX_STAGES] and empty[MAX_STAGES]
+constexpr int OFF_PM = 320;      // per-head max   [MAX_H] f32
+constexpr int OFF_PL = 384;      // per-head sum   [MAX_H] f32
+constexpr int OFF_PACC = 512;    // per-head accumulator [HG][128] f32
 
-__host__ __device__ constexpr uint32_t stage_bytes(int H) { return (uint32_t)(KT * ROW * (1 + H)); }
-__host__ __device__ constexpr uint32_t ring_offset(int H) { return (uint32_t)(OFF_PACC + H * DH * 4); }
-__host__ __device__ constexpr uint32_t smem_total(int H) { return ring_offset(H) + STAGES * stage_bytes(H); }
+// HG: heads served by one CTA (warps 0 .. HG-1) next to the producer warp HG
+__host__ __device__ constexpr uint32_t stage_bytes(int HG) { return (uint32_t)(KT * ROW * (1 + HG)); }
+__host__ __device__ constexpr uint32_t ring_offset(int HG) { return (uint32_t)(OFF_PACC + HG * DH * 4); }
+__host__ __device__ constexpr uint32_t smem_total(int HG, int stages) {
+    return ring_offset(HG) + (uint32_t)stages * stage_bytes(HG);
+}
 
 __device__ __forceinline__ bool wait_stage(uint64_t* bar, uint32_t parity, volatile int* abort_flag) {
     for (uint32_t i = 1;; ++i) {
@@ -167,21 +174,22 @@ __global__ void __launch_bounds__(32 * (MAX_H + 1), 2)
 swska_decode_warp_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ k_new,
                          const __nv_bfloat16* __restrict__ v_new, __nv_bfloat16* __restrict__ k_cache,
                          __nv_bfloat16* __restrict__ v_cache, const int64_t* __restrict__ pos,
-                         __nv_bfloat16* __restrict__ o, int H, int W, float scale_log2) {
+                         __nv_bfloat16* __restrict__ o, int H, int HG, int W, int stages, float scale_log2) {
     extern __shared__ __align__(128) unsigned char smem[];
     cg::cluster_group cluster = cg::this_cluster();
     const int SP = (int)cluster.num_blocks();
     const int rank = (int)cluster.block_rank();
     const int64_t n = blockIdx.x / SP;
+    const int hg0 = (int)blockIdx.y * HG;  // this CTA serves heads hg0 .. hg0 + HG - 1
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const uint32_t SB = stage_bytes(H);
+    const uint32_t SB = stage_bytes(HG);
     uint64_t* full = reinterpret_cast<uint64_t*>(smem);
-    uint64_t* empty = full + STAGES;
+    uint64_t* empty = full + MAX_STAGES;
     volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + OFF_FLAG);
     float* s_pm = reinterpret_cast<float*>(smem + OFF_PM);
     float* s_pl = reinterpret_cast<float*>(smem + OFF_PL);
     float* s_pacc = reinterpret_cast<float*>(smem + OFF_PACC);
-    unsigned char* ring = smem + ring_offset(H);
+    unsigned char* ring = smem + ring_offset(HG);
 
     const int64_t P = pos[n];
     const bool bad = P < 0;
@@ -192,25 +200,26 @@ swska_decode_warp_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat1
     const int64_t s_end = s_begin + per < cnt ? s_begin + per : cnt;
     const int nst = (int)((s_end - s_begin + KT - 1) / KT);
     const __nv_bfloat16* Kc = k_cache + n * (int64_t)W * DH;
-    const __nv_bfloat16* Vc = v_cache + n * (int64_t)H * W * DH;
+    const __nv_bfloat16* Vc = v_cache + (n * H + hg0) * (int64_t)W * DH;
 
     if (threadIdx.x == 0) {
-        for (int s = 0; s < STAGES; ++s) {
+        for (int s = 0; s < stages; ++s) {
             mbar_init(&full[s], 1);
-            mbar_init(&empty[s], (uint32_t)H);
+            mbar_init(&empty[s], (uint32_t)HG);
         }
         *abort_flag = 0;
         fence_mbar_init();
     }
     __syncthreads();
 
-    if (warp == H) {
+    if (warp == HG) {
         // ---------------------------------- producer warp ----------------------------------
         int issued = 0;
+        int buf = 0;
+        uint32_t par = 0;  // parity of this use of buffer buf (uses counted from 0)
         for (int st = 0; st < nst; ++st) {
-            const int buf = st % STAGES;
-            if (st >= STAGES) {
-                const bool ok = wait_stage(&empty[buf], (uint32_t)(((st / STAGES) - 1) & 1), abort_flag);
+            if (st >= stages) {
+                const bool ok = wait_stage(&empty[buf], par ^ 1u, abort_flag);
                 if (!__all_sync(0xffffffffu, ok)) break;
             }
             const int64_t s0 = s_begin + (int64_t)st * KT;
@@ -218,28 +227,31 @@ swska_decode_warp_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat1
             unsigned char* dst = ring + (size_t)buf * SB;
             const int r_new = (s_new >= s0 && s_new < s0 + rows) ? (int)(s_new - s0) : -1;
             if (r_new >= 0) {
-                // the evicted slot takes the new token: into the stage and into the cache
-                // (its old content lies outside the window, so it is never copied in)
-                for (int i = lane; i < (1 + H) * (ROW / 16); i += 32) {
+                // the evicted slot takes the new token: into the stage and into the cache (its
+                // old content lies outside the window, so it is never copied in); the shared K
+                // row goes to the cache from head group 0 only
+                for (int i = lane; i < (1 + HG) * (ROW / 16); i += 32) {
                     const int row = i / (ROW / 16), c16 = i % (ROW / 16);
-                    const uint4* src = row == 0
-                        ? reinterpret_cast<const uint4*>(k_new + n * DH)
-                        : reinterpret_cast<const uint4*>(v_new + (n * H + (row - 1)) * (int64_t)DH);
+                    const int64_t hv = n * H + hg0 + (row - 1);  // (sequence, head) of a V row
+                    const uint4* src = row == 0 ? reinterpret_cast<const uint4*>(k_new + n * DH)
+                                                : reinterpret_cast<const uint4*>(v_new + hv * DH);
                     const uint4 val = src[c16];
                     reinterpret_cast<uint4*>(dst + (size_t)row * KT * ROW + (size_t)r_new * ROW)[c16] = val;
-                    uint4* gdst = row == 0
-                        ? reinterpret_cast<uint4*>(k_cache + (n * (int64_t)W + s_new) * DH)
-                        : reinterpret_cast<uint4*>(v_cache + ((n * H + (row - 1)) * (int64_t)W + s_new) * DH);
-                    gdst[c16] = val;
+                    if (row == 0) {
+                        if (blockIdx.y == 0)
+                            reinterpret_cast<uint4*>(k_cache + (n * (int64_t)W + s_new) * DH)[c16] = val;
+                    } else {
+                        reinterpret_cast<uint4*>(v_cache + (hv * W + s_new) * DH)[c16] = val;
+                    }
                 }
                 // the generic stores precede later bulk copies into the same bytes
                 asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
             }
             __syncwarp();
             const int copied = rows - (r_new >= 0 ? 1 : 0);
-            if (lane == 0) mbar_arrive_expect_tx(&full[buf], (uint32_t)(copied * ROW * (1 + H)));
+            if (lane == 0) mbar_arrive_expect_tx(&full[buf], (uint32_t)(copied * ROW * (1 + HG)));
             __syncwarp();
-            if (lane <= H) {  // lane 0: the K rows; lane 1 + h: head h's V rows
+            if (lane <= HG) {  // lane 0: the K rows; lane 1 + h: head hg0 + h's V rows
                 unsigned char* d = dst + (size_t)lane * KT * ROW;
                 const __nv_bfloat16* src = lane == 0 ? Kc + s0 * DH : Vc + ((int64_t)(lane - 1) * W + s0) * DH;
                 const int a0 = 0, a1 = r_new >= 0 ? r_new : rows;   // rows [a0, a1)
@@ -248,25 +260,27 @@ swska_decode_warp_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat1
                 if (b1 > b0) bulk_g2s(d + (size_t)b0 * ROW, src + (int64_t)b0 * DH, (uint32_t)((b1 - b0) * ROW), &full[buf]);
             }
             ++issued;
+            if (++buf == stages) { buf = 0; par ^= 1u; }
         }
         // every copy issued has landed before the CTA's shared memory can go away (in the normal
         // course the head warps waited for these phases already)
         if (lane == 0) {
-            for (int s2 = issued > STAGES ? issued - STAGES : 0; s2 < issued; ++s2)
-                if (!mbar_wait_bounded(&full[s2 % STAGES], (uint32_t)((s2 / STAGES) & 1), kWaitLimit))
+            for (int s2 = issued > stages ? issued - stages : 0; s2 < issued; ++s2)
+                if (!mbar_wait_bounded(&full[s2 % stages], (uint32_t)((s2 / stages) & 1), kWaitLimit))
                     atomicExch(&g_swska_decode_warp_timeout, 1u);
         }
         __syncwarp();
     }
     else {
-        // ------------------------------- head warp h = warp --------------------------------
+        // -------------------------- head warp h: head hg0 + h --------------------------
         const int h = warp;
-        const uint2 qw = *reinterpret_cast<const uint2*>(q + (n * H + h) * (int64_t)DH + 4 * lane);
+        const uint2 qw = *reinterpret_cast<const uint2*>(q + (n * H + hg0 + h) * (int64_t)DH + 4 * lane);
         HeadState hs;
         bool ok = true;
+        int buf = 0;
+        uint32_t par = 0;
         for (int st = 0; st < nst; ++st) {
-            const int buf = st % STAGES;
-            if (!__all_sync(0xffffffffu, wait_stage(&full[buf], (uint32_t)((st / STAGES) & 1), abort_flag))) {
+            if (!__all_sync(0xffffffffu, wait_stage(&full[buf], par, abort_flag))) {
                 ok = false;
                 break;
             }
@@ -278,6 +292,7 @@ swska_decode_warp_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat1
             else head_stage<false>(kb, vb, qw, scale_log2, rows, lane, hs);
             __syncwarp();
             if (lane == 0) mbar_arrive(&empty[buf]);
+            if (++buf == stages) { buf = 0; par ^= 1u; }
         }
         float l = hs.l_part;
 #pragma unroll
@@ -288,7 +303,7 @@ swska_decode_warp_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat1
     }
     cluster.sync();
     // ---- combine: CTA `rank` finalises the heads h with h mod SP == rank (warp h, 4 columns a lane)
-    if (warp < H && warp % SP == rank) {
+    if (warp < HG && warp % SP == rank) {
         const int h = warp;
         float out[4];
         if (bad) {
@@ -312,21 +327,42 @@ swska_decode_warp_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat1
 #pragma unroll
             for (int i = 0; i < 4; ++i) out[i] = a[i] * inv;
         }
-        store4(o + (n * H + h) * (int64_t)DH + 4 * lane, make_float4(out[0], out[1], out[2], out[3]));
+        store4(o + (n * H + hg0 + h) * (int64_t)DH + 4 * lane, make_float4(out[0], out[1], out[2], out[3]));
     }
     cluster.sync();  // this CTA's shared memory stays alive until every peer has read it
 }
 
 
-// Clusters of each size that the GPU holds at once for this kernel (queried once per device and
-// head count; 0 if the size cannot be launched).
-int clusters_that_fit(int H, int sp) {
+struct DecodeConfig {
+    int SP;      // CTAs per cluster: the window split
+    int HG;      // heads per CTA
+    int stages;  // ring depth
+};
+
+// ring depth: about 64 KB of copies in flight per CTA, at least 3 stages
+int stages_for(int HG) {
+    int st = (int)(65536u / stage_bytes(HG));
+    return st < 3 ? 3 : (st > MAX_STAGES ? MAX_STAGES : st);
+}
+
+cudaError_t set_attributes(size_t smem) {
+    cudaError_t e = cudaFuncSetAttribute(swska_decode_warp_kernel,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e == cudaSuccess)
+        e = cudaFuncSetAttribute(swska_decode_warp_kernel, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+    return e;
+}
+
+// Clusters of the given shape that the GPU holds at once (queried once per device and shape;
+// 0 if the shape cannot be launched).
+int clusters_that_fit(int HG, int sp) {
     static std::mutex mu;
-    static int cache[64][MAX_H + 1][4];
+    static int cache[64][MAX_H + 1][5];
     static bool init = false;
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 0;
-    const int si = sp == 1 ? 0 : sp == 2 ? 1 : sp == 4 ? 2 : 3;
+    int si = 0;
+    while ((1 << si) < sp) ++si;
     std::lock_guard<std::mutex> lock(mu);
     if (!init) {
         for (auto& a : cache)
@@ -334,50 +370,59 @@ int clusters_that_fit(int H, int sp) {
                 for (int& c : b) c = -1;
         init = true;
     }
-    int& slot = cache[dev][H][si];
+    int& slot = cache[dev][HG][si];
     if (slot < 0) {
-        cudaLaunchConfig_t cfg = {};
-        cfg.gridDim = dim3((unsigned)sp, 1, 1);
-        cfg.blockDim = dim3((unsigned)(32 * (H + 1)), 1, 1);
-        cfg.dynamicSmemBytes = smem_total(H);
-        cudaLaunchAttribute attr[1];
-        attr[0].id = cudaLaunchAttributeClusterDimension;
-        attr[0].val.clusterDim.x = (unsigned)sp;
-        attr[0].val.clusterDim.y = 1;
-        attr[0].val.clusterDim.z = 1;
-        cfg.attrs = attr;
-        cfg.numAttrs = 1;
+        const size_t smem = smem_total(HG, stages_for(HG));
         int num = 0;
-        if (cudaOccupancyMaxActiveClusters(&num, swska_decode_warp_kernel, &cfg) != cudaSuccess) {
-            cudaGetLastError();
-            num = 0;
+        if (set_attributes(smem) == cudaSuccess) {
+            cudaLaunchConfig_t cfg = {};
+            cfg.gridDim = dim3((unsigned)sp, 1, 1);
+            cfg.blockDim = dim3((unsigned)(32 * (HG + 1)), 1, 1);
+            cfg.dynamicSmemBytes = smem;
+            cudaLaunchAttribute attr[1];
+            attr[0].id = cudaLaunchAttributeClusterDimension;
+            attr[0].val.clusterDim.x = (unsigned)sp;
+            attr[0].val.clusterDim.y = 1;
+            attr[0].val.clusterDim.z = 1;
+            cfg.attrs = attr;
+            cfg.numAttrs = 1;
+            if (cudaOccupancyMaxActiveClusters(&num, swska_decode_warp_kernel, &cfg) != cudaSuccess) num = 0;
         }
+        cudaGetLastError();
         slot = num;
     }
     return slot;
 }
 
-// Split of the window over a cluster. One CTA streams its slots at about 1/200 of the GPU's HBM
-// bandwidth (31-32 GB/s a CTA against 6.4 TB/s, measured with this kernel on B200), so about 200
-// CTAs in flight saturate HBM; a larger split past that adds cluster waves and combine work and
-// no bandwidth. Estimated time in slot-steps: the larger of the HBM bound N W / 200 and
-// (waves of CTAs) x (slots per CTA), over SP in {1, 2, 4, 8}; ties go to the smaller split.
+// Launch shape. The work is HBM-bound: per sequence W shared-K rows (read once per head group)
+// and H x W V rows. Estimated time, in bytes-at-full-bandwidth units, is the larger of
+//   - the total bytes, and
+//   - (waves of CTAs) x (bytes one CTA streams) x (SMs-worth of CTAs that saturate HBM),
+// where one CTA streams about 1/200 of the GPU's bandwidth (measured: ~31 GB/s against
+// 6.4 TB/s with 16 heads per CTA). Splitting the heads (fewer per CTA) and the window (bigger
+// clusters, up to 16) multiplies the CTAs for small batches at the price of reading K once per
+// head group. Among equal estimates the smaller split wins.
 constexpr double kCtasToSaturate = 200.0;
 
-int pick_split(int N, int H, int W) {
-    int best = 1;
+DecodeConfig pick_config(int N, int H, int W) {
+    DecodeConfig best{1, H, stages_for(H)};
     double best_cost = -1.0;
-    const double t_hbm = (double)N * (double)W / kCtasToSaturate;
-    for (int sp = 1; sp <= 8; sp *= 2) {
-        const int64_t cap = (int64_t)clusters_that_fit(H, sp) * sp;  // CTAs resident at once
-        if (cap <= 0) continue;
-        const int64_t ctas = (int64_t)N * sp;
-        const double waves = (double)((ctas + cap - 1) / cap);
-        const double t = waves * (double)((W + sp - 1) / sp);
-        const double cost = t > t_hbm ? t : t_hbm;
-        if (best_cost < 0.0 || cost < best_cost) {
-            best_cost = cost;
-            best = sp;
+    for (int HG = H; HG >= 1; --HG) {
+        if (H % HG) continue;
+        const int groups = H / HG;
+        const double bytes = (double)N * W * (double)(groups + H);
+        for (int sp = 1; sp <= 16; sp *= 2) {
+            const int64_t cap = (int64_t)clusters_that_fit(HG, sp) * sp;  // CTAs resident at once
+            if (cap <= 0) continue;
+            const int64_t ctas = (int64_t)N * sp * groups;
+            const double waves = (double)((ctas + cap - 1) / cap);
+            const double per_cta = (double)((W + sp - 1) / sp) * (1 + HG);
+            const double t = waves * per_cta * kCtasToSaturate;
+            const double cost = t > bytes ? t : bytes;
+            if (best_cost < 0.0 || cost < best_cost * 0.98) {
+                best_cost = cost;
+                best = DecodeConfig{sp, HG, stages_for(HG)};
+            }
         }
     }
     return best;
@@ -393,19 +438,18 @@ cudaError_t swska_decode_warp_launch(const void* q, const void* k_new, const voi
                                      void* k_cache, void* v_cache, const int64_t* pos, void* o,
                                      int N, int H, int window, float scale, cudaStream_t stream) {
     if (N == 0) return cudaSuccess;
-    const size_t smem = smem_total(H);
-    cudaError_t e = cudaFuncSetAttribute(swska_decode_warp_kernel,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    const DecodeConfig c = pick_config(N, H, window);
+    const size_t smem = smem_total(c.HG, c.stages);
+    cudaError_t e = set_attributes(smem);
     if (e != cudaSuccess) return e;
-    const int SP = pick_split(N, H, window);
     cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3((unsigned)((int64_t)N * SP), 1, 1);
-    cfg.blockDim = dim3((unsigned)(32 * (H + 1)), 1, 1);
+    cfg.gridDim = dim3((unsigned)((int64_t)N * c.SP), (unsigned)(H / c.HG), 1);
+    cfg.blockDim = dim3((unsigned)(32 * (c.HG + 1)), 1, 1);
     cfg.dynamicSmemBytes = smem;
     cfg.stream = stream;
     cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeClusterDimension;
-    attr[0].val.clusterDim.x = (unsigned)SP;
+    attr[0].val.clusterDim.x = (unsigned)c.SP;
     attr[0].val.clusterDim.y = 1;
     attr[0].val.clusterDim.z = 1;
     cfg.attrs = attr;
@@ -416,7 +460,7 @@ cudaError_t swska_decode_warp_launch(const void* q, const void* k_new, const voi
                               static_cast<const __nv_bfloat16*>(q), static_cast<const __nv_bfloat16*>(k_new),
                               static_cast<const __nv_bfloat16*>(v_new), static_cast<__nv_bfloat16*>(k_cache),
                               static_cast<__nv_bfloat16*>(v_cache), pos, static_cast<__nv_bfloat16*>(o), H,
-                              window, scale_log2);
+                              c.HG, window, c.stages, scale_log2);
 }
 
 unsigned swska_decode_warp_take_timeout_flag() {

@@ -268,6 +268,15 @@ def test_swska_decode_bf16_small_windows(W):
     _ska_decode_check(9, 2, 128, 128, W, "bf16", full=True, seed=70 + W)
 
 
+@pytest.mark.parametrize("N,H,W", [(1, 16, 4096), (2, 16, 4096), (3, 12, 1000), (1, 3, 4096),
+                                   (5, 16, 2048), (12, 16, 4096)])
+def test_swska_decode_bf16_small_batches(N, H, W):
+    """Small batches split the heads over CTAs (K read once per head group) and the window over
+    clusters of up to 16 CTAs: full and partially filled windows against the oracle."""
+    _ska_decode_check(N, H, 128, 128, W, "bf16", full=True, seed=80 + N + H)
+    _ska_decode_check(N, H, 128, 128, W, "bf16", full=False, seed=90 + N + H)
+
+
 def test_swska_decode_full_workload_sampled():
     d = wl.WORKLOADS["decode_n256"].dims
     _ska_decode_check(d["N"], d["H"], d["dk"], d["dv"], d["window"], "bf16", full=True,
