@@ -181,6 +181,30 @@ ROD_API int rod_swska_decode(const void* q, const void* k_new, const void* v_new
                      void* v_cache, const int64_t* pos, void* o, int N, int H, int dk, int dv,
                      int window, float scale, int dtype, void* stream);
 
+/* ---- SW-SKA: decode over a paged window cache ---------------------------------------------- */
+/*
+ * rod_swska_decode with the ring buffer kept in pages (SALA blog §3.3: a paged KV cache split
+ * into small blocks that are allocated on demand and evicted by window). The ring's W slots
+ * are cut into pages_per_seq pages of page_size slots (W = pages_per_seq * page_size); logical
+ * page i of sequence n is physical page block_table[n * pages_per_seq + i] of the pools:
+ *   k_pool [P][page_size][dk],  v_pool [P][H][page_size][dv]   (P physical pages), bf16;
+ *   ring slot s of sequence n:  K row  k_pool[t][s mod page_size],
+ *                               V rows v_pool[t][h][s mod page_size],  t = table entry of s / page_size.
+ * The new token is written at slot pos[n] mod W through the same mapping, then attended as in
+ * rod_swska_decode (same q, k_new, v_new, pos, o, window, scale).
+ *   block_table [N * pages_per_seq] int32 on the device: each entry must name a page inside the
+ *   pools, and sequences must not share a page (both are the caller's to keep; they are not
+ *   checked, on the host or the device).
+ * Supported: dtype ROD_BF16, dk = dv = 128, 1 <= H <= 16, page_size a positive multiple of 8.
+ * Errors: ROD_ERR_NULL, ROD_ERR_SHAPE (unsupported shape, window != pages_per_seq *
+ * page_size), ROD_ERR_ALIGN (pools, q, k_new, v_new, o, pos: 16 bytes; table: 4 bytes),
+ * ROD_ERR_DTYPE, ROD_ERR_CUDA. N = 0 is a no-op.
+ */
+ROD_API int rod_swska_decode_paged(const void* q, const void* k_new, const void* v_new, void* k_pool,
+                                   void* v_pool, const int32_t* block_table, int page_size,
+                                   int pages_per_seq, const int64_t* pos, void* o, int N, int H,
+                                   int dk, int dv, int window, float scale, int dtype, void* stream);
+
 /* ---- SW-SKA: prefill -> decode hand-off ----------------------------------------------------- */
 /*
  * Fills the decode ring buffers from a prefill's keys and values (SALA blog §3.3: chunked

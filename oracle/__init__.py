@@ -43,8 +43,12 @@ class OracleLib:
                                             ctypes.c_int]
         lib.rodref_swska_cache_fill.argtypes = [f32p, f32p, f32p, f32p, i64, i64, i64, i64, i64,
                                                 i64]
+        lib.rodref_swska_decode_paged.argtypes = [f32p, f32p, f32p, f32p, f32p,
+                                                  ctypes.POINTER(ctypes.c_int32), i64, i64, i64p,
+                                                  f64p, i64, i64, i64, i64, i64, ctypes.c_double,
+                                                  ctypes.c_int]
         for name in ("rodref_gla_prefill", "rodref_gla_decode_step", "rodref_swska_prefill",
-                     "rodref_swska_decode", "rodref_swska_cache_fill"):
+                     "rodref_swska_decode", "rodref_swska_cache_fill", "rodref_swska_decode_paged"):
             getattr(lib, name).restype = ctypes.c_int
         self.lib = lib
         self.path = path
@@ -210,3 +214,31 @@ def swska_cache_fill(k, v, k_cache, v_cache, window):
     rc = _L().rodref_swska_cache_fill(_p32(k), _p32(v), _p32(kc), _p32(vc), B, H, T, dk, dv, W)
     _check(rc, "swska_cache_fill")
     return kc, vc
+
+
+def swska_decode_paged(q, k_new, v_new, k_pool, v_pool, block_table, page_size, pos, window,
+                       scale=None, nthreads=None):
+    """Decode over a paged window cache (rodref_swska_decode_paged). Returns (o [N,H,dv] float64,
+    k_pool', v_pool') with float32 copies of the pools, the new tokens written to their pages."""
+    q, k_new, v_new = _f32(q), _f32(k_new), _f32(v_new)
+    kp, vp = _f32(k_pool).copy(), _f32(v_pool).copy()
+    N, H, dk = q.shape
+    dv = v_new.shape[-1]
+    W, page = int(window), int(page_size)
+    if hasattr(block_table, "detach"):
+        block_table = block_table.detach().cpu().numpy()
+    table = np.ascontiguousarray(np.asarray(block_table, dtype=np.int32)).reshape(-1)
+    pps = W // page
+    assert table.size == N * pps and kp.shape[1:] == (page, dk) and vp.shape[1:] == (H, page, dv)
+    if hasattr(pos, "detach"):
+        pos = pos.detach().cpu().numpy()
+    pos = np.ascontiguousarray(np.asarray(pos, dtype=np.int64))
+    if scale is None or scale <= 0:
+        scale = 1.0 / np.sqrt(dk)
+    o = np.empty((N, H, dv))
+    rc = _L().rodref_swska_decode_paged(_p32(q), _p32(k_new), _p32(v_new), _p32(kp), _p32(vp),
+                                        table.ctypes.data_as(ctypes.POINTER(ctypes.c_int32)), page,
+                                        pps, _pi64(pos), _p64(o), N, H, dk, dv, W, float(scale),
+                                        nthreads or default_threads())
+    _check(rc, "swska_decode_paged")
+    return o, kp, vp

@@ -300,6 +300,43 @@ int rodref_swska_decode(const float* q, const float* k_new, const float* v_new, 
     return run_units(ska_dec_unit, &a, N * H, nthreads);
 }
 
+/* Decode over a paged window cache (SALA blog §3.3: paged KV cache in small blocks): the ring's
+ * W slots are cut into pps pages of `page` slots; slot s of sequence n lives in physical page
+ * t = table[n*pps + s/page] at row s mod page of the pools k_pool [P][page][dk] and
+ * v_pool [P][H][page][dv]. The step is the ring-buffer decode on the logical cache: gather the
+ * window from the pages, run rodref_swska_decode, and write the new token's rows back to its
+ * page. */
+int rodref_swska_decode_paged(const float* q, const float* k_new, const float* v_new, float* k_pool,
+                              float* v_pool, const int32_t* table, int64_t page, int64_t pps,
+                              const int64_t* pos, double* o, int64_t N, int64_t H, int64_t dk,
+                              int64_t dv, int64_t W, double scale, int nthreads) {
+    if (!table || !k_pool || !v_pool || !pos || page < 1 || pps < 1 || page * pps != W || N < 0 || H < 1)
+        return RODREF_EINVAL;
+    float* kc = malloc((size_t)(N * W * dk + 1) * sizeof(float));
+    float* vc = malloc((size_t)(N * H * W * dv + 1) * sizeof(float));
+    if (!kc || !vc) { free(kc); free(vc); return RODREF_EINVAL; }
+    for (int64_t n = 0; n < N; ++n)
+        for (int64_t s = 0; s < W; ++s) {
+            const int64_t t = table[n * pps + s / page], r = s % page;
+            memcpy(kc + (n * W + s) * dk, k_pool + (t * page + r) * dk, (size_t)dk * sizeof(float));
+            for (int64_t h = 0; h < H; ++h)
+                memcpy(vc + ((n * H + h) * W + s) * dv, v_pool + ((t * H + h) * page + r) * dv,
+                       (size_t)dv * sizeof(float));
+        }
+    const int rc = rodref_swska_decode(q, k_new, v_new, kc, vc, pos, o, N, H, dk, dv, W, scale, nthreads);
+    if (rc == 0)
+        for (int64_t n = 0; n < N; ++n) {
+            const int64_t s = pos[n] % W, t = table[n * pps + s / page], r = s % page;
+            memcpy(k_pool + (t * page + r) * dk, kc + (n * W + s) * dk, (size_t)dk * sizeof(float));
+            for (int64_t h = 0; h < H; ++h)
+                memcpy(v_pool + ((t * H + h) * page + r) * dv, vc + ((n * H + h) * W + s) * dv,
+                       (size_t)dv * sizeof(float));
+        }
+    free(kc);
+    free(vc);
+    return rc;
+}
+
 /* Prefill -> decode hand-off (SALA blog §3.3: decode keeps the most recent W tokens in a
  * circular buffer; the ring rule is the one rodref_swska_decode writes by): every position p in
  * [max(0, T-W), T) of the prefill's shared keys k [B,T,dk] and per-head values v [B,H,T,dv] is

@@ -10,6 +10,8 @@ the calls raise.
     swska_prefill(q, k, v, window, scale=None)      sliding-window shared-key attention
     swska_decode(q, k_new, v_new, k_cache, v_cache, pos, window)   ring-buffer decode
     swska_cache_fill(k, v, k_cache, v_cache, window)   prefill -> decode ring-buffer hand-off
+    swska_decode_paged(q, k_new, v_new, k_pool, v_pool, block_table, page_size, pos, window)
+                                                    decode over a paged window cache
 """
 from ._binding import (  # noqa: F401
     ROD_BF16,
@@ -26,5 +28,6 @@ from ._binding import (  # noqa: F401
     load_library,
     swska_cache_fill,
     swska_decode,
+    swska_decode_paged,
     swska_prefill,
 )

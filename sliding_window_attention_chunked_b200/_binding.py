@@ -66,6 +66,9 @@ def load_library() -> ctypes.CDLL:
     lib.rod_swska_decode.argtypes = [vp, vp, vp, vp, vp, vp, vp, i, i, i, i, i, f, i, vp]
     lib.rod_swska_decode.restype = i
     lib.rod_swska_cache_fill.argtypes = [vp, vp, vp, vp, i, i, i, i, i, i, i, vp]
+    lib.rod_swska_decode_paged.argtypes = [vp, vp, vp, vp, vp, vp, i, i, vp, vp, i, i, i, i, i, f,
+                                           i, vp]
+    lib.rod_swska_decode_paged.restype = i
     lib.rod_swska_cache_fill.restype = i
     _lib = lib
     return lib
@@ -261,3 +264,32 @@ def swska_cache_fill(k, v, k_cache, v_cache, window, stream=None):
                                              dk, dv, W, _dtype_code(k), _stream(stream))
     _raise_on("rod_swska_cache_fill", st)
     return k_cache, v_cache
+
+
+def swska_decode_paged(q, k_new, v_new, k_pool, v_pool, block_table, page_size, pos, window,
+                       scale=None, o=None, stream=None):
+    """Ring-buffer decode over a paged window cache: k_pool [P,page,dk], v_pool [P,H,page,dv]
+    (bf16), block_table [N, W/page] int32 (logical page -> physical page). Returns o [N,H,dv]."""
+    _need(q, "q", None, 3)
+    for n, t, nd in (("k_new", k_new, 2), ("v_new", v_new, 3), ("k_pool", k_pool, 3),
+                     ("v_pool", v_pool, 4)):
+        _need(t, n, q.dtype, nd)
+    _need(pos, "pos", torch.int64, 1)
+    _need(block_table, "block_table", torch.int32, 2)
+    N, H, dk = q.shape
+    dv = v_new.shape[-1]
+    W, page = int(window), int(page_size)
+    pps = W // page if page > 0 else 0
+    if (tuple(k_new.shape) != (N, dk) or tuple(block_table.shape) != (N, pps)
+            or tuple(k_pool.shape[1:]) != (page, dk) or tuple(v_pool.shape[1:]) != (H, page, dv)
+            or v_pool.shape[0] != k_pool.shape[0] or pos.shape[0] != N):
+        raise ValueError("shape mismatch")
+    if o is None:
+        o = torch.empty((N, H, dv), dtype=q.dtype, device=q.device)
+    _need(o, "o", q.dtype, 3)
+    st = load_library().rod_swska_decode_paged(_ptr(q), _ptr(k_new), _ptr(v_new), _ptr(k_pool),
+                                               _ptr(v_pool), _ptr(block_table), page, pps, _ptr(pos),
+                                               _ptr(o), N, H, dk, dv, W, float(scale or 0.0),
+                                               _dtype_code(q), _stream(stream))
+    _raise_on("rod_swska_decode_paged", st)
+    return o

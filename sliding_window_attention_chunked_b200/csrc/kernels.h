@@ -61,6 +61,11 @@ cudaError_t swska_decode_warp_launch(const void* q, const void* k_new, const voi
                                      void* k_cache, void* v_cache, const int64_t* pos, void* o,
                                      int N, int H, int window, float scale, cudaStream_t stream);
 unsigned swska_decode_warp_take_timeout_flag();
+// the same decode over a paged window cache (pools + block table)
+cudaError_t swska_decode_paged_launch(const void* q, const void* k_new, const void* v_new, void* k_pool,
+                                      void* v_pool, const int32_t* block_table, int page_size,
+                                      int pages_per_seq, const int64_t* pos, void* o, int N, int H,
+                                      int window, float scale, cudaStream_t stream);
 
 // SW-SKA prefill -> decode hand-off: the last W tokens' K / V rows into the ring buffers
 cudaError_t swska_cache_fill_launch(const void* k, const void* v, void* k_cache, void* v_cache, int B,

@@ -146,6 +146,28 @@ int rod_swska_decode(const void* q, const void* k_new, const void* v_new, void* 
                                               static_cast<cudaStream_t>(stream)));
 }
 
+int rod_swska_decode_paged(const void* q, const void* k_new, const void* v_new, void* k_pool,
+                           void* v_pool, const int32_t* block_table, int page_size, int pages_per_seq,
+                           const int64_t* pos, void* o, int N, int H, int dk, int dv, int window,
+                           float scale, int dtype, void* stream) {
+    if (!dtype_ok(dtype)) return ROD_ERR_DTYPE;
+    if (dtype != ROD_BF16) return ROD_ERR_DTYPE;
+    if (N < 0 || !rod::swska_decode_warp_supported(H, dk, dv) || page_size < 8 || page_size % 8 != 0 ||
+        pages_per_seq < 1 || window < 1 || (int64_t)page_size * pages_per_seq != window)
+        return ROD_ERR_SHAPE;
+    if (!(scale == scale) || isinf(scale)) return ROD_ERR_SHAPE;
+    if (N == 0) return ROD_OK;
+    if (!q || !k_new || !v_new || !k_pool || !v_pool || !block_table || !pos || !o) return ROD_ERR_NULL;
+    if (!aligned16(q) || !aligned16(k_new) || !aligned16(v_new) || !aligned16(k_pool) ||
+        !aligned16(v_pool) || !aligned16(pos) || !aligned16(o) ||
+        (reinterpret_cast<uintptr_t>(block_table) & 3u) != 0)
+        return ROD_ERR_ALIGN;
+    return from_cuda(rod::swska_decode_paged_launch(q, k_new, v_new, k_pool, v_pool, block_table,
+                                                    page_size, pages_per_seq, pos, o, N, H, window,
+                                                    resolve_scale(scale, dk),
+                                                    static_cast<cudaStream_t>(stream)));
+}
+
 int rod_swska_cache_fill(const void* k, const void* v, void* k_cache, void* v_cache, int B, int H,
                          int T, int dk, int dv, int window, int dtype, void* stream) {
     if (!dtype_ok(dtype)) return ROD_ERR_DTYPE;

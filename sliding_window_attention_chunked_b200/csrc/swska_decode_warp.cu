@@ -170,11 +170,33 @@ __device__ __forceinline__ void head_stage(const unsigned char* kb, const unsign
     }
 }
 
+// Where the window cache lives. Contiguous: k [N][W][DH], v [N][H][W][DH], ring slot s of
+// sequence n at row s. Paged (SALA blog §3.3: paged KV cache, allocated in blocks and evicted by
+// window): the ring's slots are cut into pages of `page` slots; logical page i of sequence n is
+// physical page table[n * pps + i] of the pools k [pages][page][DH] and v [pages][H][page][DH].
+struct CacheRef {
+    __nv_bfloat16* k;
+    __nv_bfloat16* v;
+    const int32_t* table;  // paged only
+    int page, pps;         // slots per page, pages per sequence (paged only)
+};
+template <bool PAGED>
+__device__ __forceinline__ int64_t k_row(const CacheRef& c, int64_t n, int W, int64_t slot) {
+    if (!PAGED) return n * W + slot;
+    return (int64_t)c.table[n * c.pps + slot / c.page] * c.page + slot % c.page;
+}
+template <bool PAGED>
+__device__ __forceinline__ int64_t v_row(const CacheRef& c, int64_t n, int H, int W, int64_t h, int64_t slot) {
+    if (!PAGED) return (n * H + h) * W + slot;
+    return ((int64_t)c.table[n * c.pps + slot / c.page] * H + h) * c.page + slot % c.page;
+}
+
+template <bool PAGED>
 __global__ void __launch_bounds__(32 * (MAX_H + 1), 2)
 swska_decode_warp_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ k_new,
-                         const __nv_bfloat16* __restrict__ v_new, __nv_bfloat16* __restrict__ k_cache,
-                         __nv_bfloat16* __restrict__ v_cache, const int64_t* __restrict__ pos,
-                         __nv_bfloat16* __restrict__ o, int H, int HG, int W, int stages, float scale_log2) {
+                         const __nv_bfloat16* __restrict__ v_new, CacheRef cache,
+                         const int64_t* __restrict__ pos, __nv_bfloat16* __restrict__ o, int H, int HG,
+                         int W, int stages, float scale_log2) {
     extern __shared__ __align__(128) unsigned char smem[];
     cg::cluster_group cluster = cg::this_cluster();
     const int SP = (int)cluster.num_blocks();
@@ -195,12 +217,11 @@ swska_decode_warp_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat1
     const bool bad = P < 0;
     const int64_t cnt = bad ? 0 : (P + 1 < W ? P + 1 : W);  // valid slots 0 .. cnt-1
     const int64_t s_new = bad ? -1 : P % W;
-    const int64_t per = (cnt + SP - 1) / SP;
+    // slots per CTA, a multiple of the stage length so that no stage crosses a page
+    const int64_t per = ((cnt + SP - 1) / SP + KT - 1) / KT * KT;
     const int64_t s_begin = (int64_t)rank * per < cnt ? (int64_t)rank * per : cnt;
     const int64_t s_end = s_begin + per < cnt ? s_begin + per : cnt;
     const int nst = (int)((s_end - s_begin + KT - 1) / KT);
-    const __nv_bfloat16* Kc = k_cache + n * (int64_t)W * DH;
-    const __nv_bfloat16* Vc = v_cache + (n * H + hg0) * (int64_t)W * DH;
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < stages; ++s) {
@@ -239,9 +260,9 @@ swska_decode_warp_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat1
                     reinterpret_cast<uint4*>(dst + (size_t)row * KT * ROW + (size_t)r_new * ROW)[c16] = val;
                     if (row == 0) {
                         if (blockIdx.y == 0)
-                            reinterpret_cast<uint4*>(k_cache + (n * (int64_t)W + s_new) * DH)[c16] = val;
+                            reinterpret_cast<uint4*>(cache.k + k_row<PAGED>(cache, n, W, s_new) * DH)[c16] = val;
                     } else {
-                        reinterpret_cast<uint4*>(v_cache + (hv * W + s_new) * DH)[c16] = val;
+                        reinterpret_cast<uint4*>(cache.v + v_row<PAGED>(cache, n, H, W, hg0 + row - 1, s_new) * DH)[c16] = val;
                     }
                 }
                 // the generic stores precede later bulk copies into the same bytes
@@ -253,7 +274,9 @@ swska_decode_warp_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat1
             __syncwarp();
             if (lane <= HG) {  // lane 0: the K rows; lane 1 + h: head hg0 + h's V rows
                 unsigned char* d = dst + (size_t)lane * KT * ROW;
-                const __nv_bfloat16* src = lane == 0 ? Kc + s0 * DH : Vc + ((int64_t)(lane - 1) * W + s0) * DH;
+                // rows s0 .. s0 + rows - 1 are contiguous (one page holds a whole stage)
+                const __nv_bfloat16* src = lane == 0 ? cache.k + k_row<PAGED>(cache, n, W, s0) * DH
+                                                     : cache.v + v_row<PAGED>(cache, n, H, W, hg0 + lane - 1, s0) * DH;
                 const int a0 = 0, a1 = r_new >= 0 ? r_new : rows;   // rows [a0, a1)
                 const int b0 = r_new >= 0 ? r_new + 1 : rows, b1 = rows;  // rows [b0, b1)
                 if (a1 > a0) bulk_g2s(d + (size_t)a0 * ROW, src + (int64_t)a0 * DH, (uint32_t)((a1 - a0) * ROW), &full[buf]);
@@ -345,11 +368,13 @@ int stages_for(int HG) {
     return st < 3 ? 3 : (st > MAX_STAGES ? MAX_STAGES : st);
 }
 
+template <bool PAGED>
 cudaError_t set_attributes(size_t smem) {
-    cudaError_t e = cudaFuncSetAttribute(swska_decode_warp_kernel,
+    cudaError_t e = cudaFuncSetAttribute(swska_decode_warp_kernel<PAGED>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e == cudaSuccess)
-        e = cudaFuncSetAttribute(swska_decode_warp_kernel, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+        e = cudaFuncSetAttribute(swska_decode_warp_kernel<PAGED>,
+                                 cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
     return e;
 }
 
@@ -374,7 +399,7 @@ int clusters_that_fit(int HG, int sp) {
     if (slot < 0) {
         const size_t smem = smem_total(HG, stages_for(HG));
         int num = 0;
-        if (set_attributes(smem) == cudaSuccess) {
+        if (set_attributes<false>(smem) == cudaSuccess) {
             cudaLaunchConfig_t cfg = {};
             cfg.gridDim = dim3((unsigned)sp, 1, 1);
             cfg.blockDim = dim3((unsigned)(32 * (HG + 1)), 1, 1);
@@ -386,7 +411,8 @@ int clusters_that_fit(int HG, int sp) {
             attr[0].val.clusterDim.z = 1;
             cfg.attrs = attr;
             cfg.numAttrs = 1;
-            if (cudaOccupancyMaxActiveClusters(&num, swska_decode_warp_kernel, &cfg) != cudaSuccess) num = 0;
+            // the paged instance has the same resources
+            if (cudaOccupancyMaxActiveClusters(&num, swska_decode_warp_kernel<false>, &cfg) != cudaSuccess) num = 0;
         }
         cudaGetLastError();
         slot = num;
@@ -434,13 +460,15 @@ bool swska_decode_warp_supported(int H, int dk, int dv) {
     return dk == DH && dv == DH && H >= 1 && H <= MAX_H;
 }
 
-cudaError_t swska_decode_warp_launch(const void* q, const void* k_new, const void* v_new,
-                                     void* k_cache, void* v_cache, const int64_t* pos, void* o,
-                                     int N, int H, int window, float scale, cudaStream_t stream) {
+namespace {
+
+template <bool PAGED>
+cudaError_t launch(const void* q, const void* k_new, const void* v_new, CacheRef cache, const int64_t* pos,
+                   void* o, int N, int H, int window, float scale, cudaStream_t stream) {
     if (N == 0) return cudaSuccess;
     const DecodeConfig c = pick_config(N, H, window);
     const size_t smem = smem_total(c.HG, c.stages);
-    cudaError_t e = set_attributes(smem);
+    cudaError_t e = set_attributes<PAGED>(smem);
     if (e != cudaSuccess) return e;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3((unsigned)((int64_t)N * c.SP), (unsigned)(H / c.HG), 1);
@@ -456,11 +484,28 @@ cudaError_t swska_decode_warp_launch(const void* q, const void* k_new, const voi
     cfg.numAttrs = 1;
     const float scale_log2 = scale * 1.4426950408889634f;
     note_launches(1);
-    return cudaLaunchKernelEx(&cfg, swska_decode_warp_kernel,
+    return cudaLaunchKernelEx(&cfg, swska_decode_warp_kernel<PAGED>,
                               static_cast<const __nv_bfloat16*>(q), static_cast<const __nv_bfloat16*>(k_new),
-                              static_cast<const __nv_bfloat16*>(v_new), static_cast<__nv_bfloat16*>(k_cache),
-                              static_cast<__nv_bfloat16*>(v_cache), pos, static_cast<__nv_bfloat16*>(o), H,
-                              c.HG, window, c.stages, scale_log2);
+                              static_cast<const __nv_bfloat16*>(v_new), cache, pos,
+                              static_cast<__nv_bfloat16*>(o), H, c.HG, window, c.stages, scale_log2);
+}
+
+}  // namespace
+
+cudaError_t swska_decode_warp_launch(const void* q, const void* k_new, const void* v_new,
+                                     void* k_cache, void* v_cache, const int64_t* pos, void* o,
+                                     int N, int H, int window, float scale, cudaStream_t stream) {
+    const CacheRef c{static_cast<__nv_bfloat16*>(k_cache), static_cast<__nv_bfloat16*>(v_cache), nullptr, 0, 0};
+    return launch<false>(q, k_new, v_new, c, pos, o, N, H, window, scale, stream);
+}
+
+cudaError_t swska_decode_paged_launch(const void* q, const void* k_new, const void* v_new, void* k_pool,
+                                      void* v_pool, const int32_t* block_table, int page_size,
+                                      int pages_per_seq, const int64_t* pos, void* o, int N, int H,
+                                      int window, float scale, cudaStream_t stream) {
+    const CacheRef c{static_cast<__nv_bfloat16*>(k_pool), static_cast<__nv_bfloat16*>(v_pool), block_table,
+                     page_size, pages_per_seq};
+    return launch<true>(q, k_new, v_new, c, pos, o, N, H, window, scale, stream);
 }
 
 unsigned swska_decode_warp_take_timeout_flag() {

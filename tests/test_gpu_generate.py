@@ -133,3 +133,52 @@ def test_graph_replay_equals_eager_step():
         for key in la:
             assert torch.equal(la[key], lb[key]), key
     assert torch.equal(eager.pos, graphed.pos)
+
+
+# ------------------------------------------------------------------------------------------
+# paged window cache
+# ------------------------------------------------------------------------------------------
+
+
+@pytest.mark.parametrize("N,H,W,page,full", [(3, 16, 4096, 64, True), (2, 16, 4096, 8, False),
+                                             (5, 4, 512, 128, True), (1, 16, 2048, 2048, True),
+                                             (7, 3, 96, 16, False)])
+def test_swska_decode_paged_matches_oracle(N, H, W, page, full):
+    """Random pool contents, a shuffled block table with spare pages, full and partial windows:
+    outputs within the bf16 tolerance, pools bit-exact after the new tokens are written."""
+    d = 128
+    dd = wl.decode_inputs(N, H, d, d, W, seed=N + W + page, dtype="bf16", full=full)
+    pps = W // page
+    P = N * pps + 5
+    g = torch.Generator().manual_seed(W + page)
+    k_pool = torch.randn(P, page, d, generator=g).to(torch.bfloat16)
+    v_pool = torch.randn(P, H, page, d, generator=g).to(torch.bfloat16)
+    table = torch.randperm(P, generator=g)[:N * pps].to(torch.int32).reshape(N, pps)
+    ref, kp_ref, vp_ref = oracle.swska_decode_paged(dd["sq"], dd["k_new"], dd["v_new"], k_pool,
+                                                    v_pool, table, page, dd["pos"], W)
+    kp, vp = k_pool.to(DEV), v_pool.to(DEV)
+    o = rod.swska_decode_paged(dd["sq"].to(DEV), dd["k_new"].to(DEV), dd["v_new"].to(DEV), kp, vp,
+                               table.to(DEV), page, dd["pos"].to(DEV), W)
+    rod.check()
+    compare(o, ref, "bf16", "paged o")
+    np.testing.assert_array_equal(kp.float().cpu().numpy(), kp_ref)
+    np.testing.assert_array_equal(vp.float().cpu().numpy(), vp_ref)
+
+
+def test_swska_decode_paged_identity_table_equals_ring():
+    """With the pool laid out as [N*pages][page] and the identity table, the K pool is the ring
+    buffer itself: paged and ring decode give the same outputs bit for bit."""
+    N, H, d, W, page = 4, 16, 128, 1024, 128
+    dd = wl.decode_inputs(N, H, d, d, W, seed=9, dtype="bf16", full=True)
+    pps = W // page
+    kc, vc = dd["k_cache"].to(DEV), dd["v_cache"].to(DEV)
+    k_pool = kc.reshape(N * pps, page, d).clone()
+    v_pool = vc.reshape(N, H, pps, page, d).permute(0, 2, 1, 3, 4).reshape(N * pps, H, page, d).contiguous()
+    table = torch.arange(N * pps, dtype=torch.int32, device=DEV).reshape(N, pps)
+    args = (dd["sq"].to(DEV), dd["k_new"].to(DEV), dd["v_new"].to(DEV))
+    pos = dd["pos"].to(DEV)
+    o_ring = rod.swska_decode(*args, kc, vc, pos, W)
+    o_paged = rod.swska_decode_paged(*args, k_pool, v_pool, table, page, pos, W)
+    rod.check()
+    assert torch.equal(o_ring, o_paged)
+    assert torch.equal(kc.reshape(N * pps, page, d), k_pool)

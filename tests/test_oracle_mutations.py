@@ -3,7 +3,8 @@
 Each case copies oracle/rodref.c to a temporary directory, plants one plausible mistake by a
 textual substitution (a gate applied to the wrong channel, a decay that also hits the new
 term, the readout using k, an off-by-one window, a dropped scale or normaliser, a wrong
-ring-buffer slot, a hand-off that drops a token or numbers slots from the window start), builds the copy with gcc and runs every pin against it. Each planted
+ring-buffer slot, a hand-off that drops a token or numbers slots from the window start, a paged cache read
+without its table or written at the wrong row), builds the copy with gcc and runs every pin against it. Each planted
 mistake must make at least one pin fail; otherwise the pins are too weak to trust.
 """
 import inspect
@@ -37,6 +38,10 @@ MUTATIONS = {
                                 "const int64_t p0 = T > W ? T - W + 1 : 0;"),
     "cache_fill_slot_from_start": ("const int64_t slot = p % W;",
                                    "const int64_t slot = (p - p0) % W;"),
+    "paged_read_ignores_table": ("const int64_t t = table[n * pps + s / page], r = s % page;",
+                                 "const int64_t t = n * pps + s / page, r = s % page;"),
+    "paged_write_wrong_row": ("t = table[n * pps + s / page], r = s % page;\n            memcpy(k_pool",
+                              "t = table[n * pps + s / page], r = (s + 1) % page;\n            memcpy(k_pool"),
 }
 
 

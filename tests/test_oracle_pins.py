@@ -313,3 +313,52 @@ def test_swska_cache_fill_equals_decode_writes(W, T):
                                         np.full(B, p, np.int64), W)
     np.testing.assert_array_equal(kf, kd)
     np.testing.assert_array_equal(vf, vd)
+
+
+def test_swska_paged_decode_hand_worked_layout():
+    """W = 16 slots in pages of 8, table [3, 1] over a pool of 4 pages: position 9 (slot 9,
+    logical page 1) lands in physical page 1 at row 1; position 2 (slot 2, logical page 0) in
+    physical page 3 at row 2; nothing else in the pools changes."""
+    H, dk, dv, W, page = 2, 4, 3, 16, 8
+    r = _rng(77)
+    kp = np.full((4, page, dk), 5.0, np.float32)
+    vp = np.full((4, H, page, dv), 5.0, np.float32)
+    table = np.array([3, 1], np.int32)
+    for P, (pg, row) in ((9, (1, 1)), (2, (3, 2))):
+        q = r.standard_normal((1, H, dk)).astype(np.float32)
+        kn = r.standard_normal((1, dk)).astype(np.float32)
+        vn = r.standard_normal((1, H, dv)).astype(np.float32)
+        before_k, before_v = kp.copy(), vp.copy()
+        _, kp, vp = oracle.swska_decode_paged(q, kn, vn, kp, vp, table, page, np.array([P]), W)
+        np.testing.assert_array_equal(kp[pg, row], kn[0])
+        np.testing.assert_array_equal(vp[pg, :, row], vn[0])
+        before_k[pg, row] = kn[0]
+        before_v[pg, :, row] = vn[0]
+        np.testing.assert_array_equal(kp, before_k)
+        np.testing.assert_array_equal(vp, before_v)
+
+
+@pytest.mark.parametrize("W,page", [(16, 8), (24, 8), (32, 16)])
+def test_swska_paged_decode_continues_prefill_and_writes_only_its_pages(W, page):
+    """Three sequences share a pool through a shuffled table with spare pages. Decoding every
+    position of each sequence from an empty cache (each step writes its token through the table)
+    reproduces the prefill rows of that sequence; afterwards exactly the pages the table names
+    have been written and the spare pages still hold their fill value."""
+    H, dk, dv, N = 2, 5, 4, 3
+    pps = W // page
+    T = W + 9
+    q, k, v = _ska_case(B=N, H=H, T=T, dk=dk, dv=dv, seed=21)
+    o_pre = oracle.swska_prefill(q, k, v, W)
+    P_pages = N * pps + 3
+    perm = _rng(5).permutation(P_pages).astype(np.int32)
+    table = perm[:N * pps]
+    kp = np.full((P_pages, page, dk), 7.0, np.float32)
+    vp = np.full((P_pages, H, page, dv), 7.0, np.float32)
+    for t in range(T):
+        o, kp, vp = oracle.swska_decode_paged(q[:, :, t], k[:, t], v[:, :, t], kp, vp, table, page,
+                                              np.full(N, t, np.int64), W)
+        _close(o, o_pre[:, :, t], 1e-13)
+    used = set(table.tolist())
+    for pg in range(P_pages):
+        untouched = bool((kp[pg] == 7.0).all() and (vp[pg] == 7.0).all())
+        assert untouched == (pg not in used), pg
