@@ -195,11 +195,13 @@ ROD_API int rod_swska_decode(const void* q, const void* k_new, const void* v_new
  *   block_table [N * pages_per_seq] int32 on the device: each entry must name a page inside the
  *   pools, and sequences must not share a page (both are the caller's to keep; they are not
  *   checked, on the host or the device).
- * Supported: dtype ROD_BF16, dk = dv = 128, 1 <= H <= 16, page_size a positive multiple of 8.
+ * Supported: dtype ROD_BF16, dk = dv = 128, 1 <= H <= 16, page_size a positive multiple of 8,
+ * pages_per_seq <= ROD_MAX_PAGES_PER_SEQ.
  * Errors: ROD_ERR_NULL, ROD_ERR_SHAPE (unsupported shape, window != pages_per_seq *
  * page_size), ROD_ERR_ALIGN (pools, q, k_new, v_new, o, pos: 16 bytes; table: 4 bytes),
  * ROD_ERR_DTYPE, ROD_ERR_CUDA. N = 0 is a no-op.
  */
+#define ROD_MAX_PAGES_PER_SEQ 512
 ROD_API int rod_swska_decode_paged(const void* q, const void* k_new, const void* v_new, void* k_pool,
                                    void* v_pool, const int32_t* block_table, int page_size,
                                    int pages_per_seq, const int64_t* pos, void* o, int N, int H,

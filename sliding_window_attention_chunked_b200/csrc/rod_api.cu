@@ -153,7 +153,8 @@ int rod_swska_decode_paged(const void* q, const void* k_new, const void* v_new, 
     if (!dtype_ok(dtype)) return ROD_ERR_DTYPE;
     if (dtype != ROD_BF16) return ROD_ERR_DTYPE;
     if (N < 0 || !rod::swska_decode_warp_supported(H, dk, dv) || page_size < 8 || page_size % 8 != 0 ||
-        pages_per_seq < 1 || window < 1 || (int64_t)page_size * pages_per_seq != window)
+        pages_per_seq < 1 || pages_per_seq > ROD_MAX_PAGES_PER_SEQ || window < 1 ||
+        (int64_t)page_size * pages_per_seq != window)
         return ROD_ERR_SHAPE;
     if (!(scale == scale) || isinf(scale)) return ROD_ERR_SHAPE;
     if (N == 0) return ROD_OK;

@@ -62,8 +62,10 @@ constexpr int OFF_PACC = 512;    // per-head accumulator [HG][128] f32
 // HG: heads served by one CTA (warps 0 .. HG-1) next to the producer warp HG
 __host__ __device__ constexpr uint32_t stage_bytes(int HG) { return (uint32_t)(KT * ROW * (1 + HG)); }
 __host__ __device__ constexpr uint32_t ring_offset(int HG) { return (uint32_t)(OFF_PACC + HG * DH * 4); }
+// a CTA's slice of a paged block table: at most pages_per_seq + 1 entries (ROD_MAX_PAGES_PER_SEQ)
+constexpr uint32_t kPageSlice = 520;
 __host__ __device__ constexpr uint32_t smem_total(int HG, int stages) {
-    return ring_offset(HG) + (uint32_t)stages * stage_bytes(HG);
+    return ring_offset(HG) + (uint32_t)stages * stage_bytes(HG) + 4u * kPageSlice;
 }
 
 __device__ __forceinline__ bool wait_stage(uint64_t* bar, uint32_t parity, volatile int* abort_flag) {
@@ -180,15 +182,19 @@ struct CacheRef {
     const int32_t* table;  // paged only
     int page, pps;         // slots per page, pages per sequence (paged only)
 };
+// Paged lookups read the CTA's slice of the block table, staged in shared memory at kernel start
+// (pages[i] = table entry of logical page pg0 + i).
 template <bool PAGED>
-__device__ __forceinline__ int64_t k_row(const CacheRef& c, int64_t n, int W, int64_t slot) {
+__device__ __forceinline__ int64_t k_row(const CacheRef& c, int64_t n, int W, int slot,
+                                         const int32_t* pages, int pg0) {
     if (!PAGED) return n * W + slot;
-    return (int64_t)c.table[n * c.pps + slot / c.page] * c.page + slot % c.page;
+    return (int64_t)pages[slot / c.page - pg0] * c.page + slot % c.page;
 }
 template <bool PAGED>
-__device__ __forceinline__ int64_t v_row(const CacheRef& c, int64_t n, int H, int W, int64_t h, int64_t slot) {
+__device__ __forceinline__ int64_t v_row(const CacheRef& c, int64_t n, int H, int W, int64_t h, int slot,
+                                         const int32_t* pages, int pg0) {
     if (!PAGED) return (n * H + h) * W + slot;
-    return ((int64_t)c.table[n * c.pps + slot / c.page] * H + h) * c.page + slot % c.page;
+    return ((int64_t)pages[slot / c.page - pg0] * H + h) * c.page + slot % c.page;
 }
 
 template <bool PAGED>
@@ -215,12 +221,13 @@ swska_decode_warp_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat1
 
     const int64_t P = pos[n];
     const bool bad = P < 0;
-    const int64_t cnt = bad ? 0 : (P + 1 < W ? P + 1 : W);  // valid slots 0 .. cnt-1
-    const int64_t s_new = bad ? -1 : P % W;
+    // slot indices are below W (an int): 32-bit arithmetic keeps registers free
+    const int cnt = bad ? 0 : (P + 1 < W ? (int)P + 1 : W);  // valid slots 0 .. cnt-1
+    const int s_new = bad ? -1 : (int)(P % W);
     // slots per CTA, a multiple of the stage length so that no stage crosses a page
-    const int64_t per = ((cnt + SP - 1) / SP + KT - 1) / KT * KT;
-    const int64_t s_begin = (int64_t)rank * per < cnt ? (int64_t)rank * per : cnt;
-    const int64_t s_end = s_begin + per < cnt ? s_begin + per : cnt;
+    const int per = ((cnt + SP - 1) / SP + KT - 1) / KT * KT;
+    const int s_begin = rank * per < cnt ? rank * per : cnt;
+    const int s_end = s_begin + per < cnt ? s_begin + per : cnt;
     const int nst = (int)((s_end - s_begin + KT - 1) / KT);
 
     if (threadIdx.x == 0) {
@@ -235,16 +242,24 @@ swska_decode_warp_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat1
 
     if (warp == HG) {
         // ---------------------------------- producer warp ----------------------------------
+        int32_t* pages = reinterpret_cast<int32_t*>(ring + (size_t)stages * SB);
+        const int pg0 = PAGED ? s_begin / cache.page : 0;
+        if (PAGED) {
+            const int npg = s_end > s_begin ? (s_end - 1) / cache.page - pg0 + 1 : 0;
+            for (int i = lane; i < npg; i += 32) pages[i] = cache.table[n * cache.pps + pg0 + i];
+            __syncwarp();
+        }
         int issued = 0;
         int buf = 0;
         uint32_t par = 0;  // parity of this use of buffer buf (uses counted from 0)
+        int pi = 0, off = PAGED ? (int)(s_begin % cache.page) : 0;  // page slot of s0 (paged)
         for (int st = 0; st < nst; ++st) {
             if (st >= stages) {
                 const bool ok = wait_stage(&empty[buf], par ^ 1u, abort_flag);
                 if (!__all_sync(0xffffffffu, ok)) break;
             }
-            const int64_t s0 = s_begin + (int64_t)st * KT;
-            const int rows = (int)((s_end - s0) < KT ? (s_end - s0) : KT);
+            const int s0 = s_begin + st * KT;
+            const int rows = s_end - s0 < KT ? s_end - s0 : KT;
             unsigned char* dst = ring + (size_t)buf * SB;
             const int r_new = (s_new >= s0 && s_new < s0 + rows) ? (int)(s_new - s0) : -1;
             if (r_new >= 0) {
@@ -260,9 +275,9 @@ swska_decode_warp_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat1
                     reinterpret_cast<uint4*>(dst + (size_t)row * KT * ROW + (size_t)r_new * ROW)[c16] = val;
                     if (row == 0) {
                         if (blockIdx.y == 0)
-                            reinterpret_cast<uint4*>(cache.k + k_row<PAGED>(cache, n, W, s_new) * DH)[c16] = val;
+                            reinterpret_cast<uint4*>(cache.k + k_row<PAGED>(cache, n, W, s_new, pages, pg0) * DH)[c16] = val;
                     } else {
-                        reinterpret_cast<uint4*>(cache.v + v_row<PAGED>(cache, n, H, W, hg0 + row - 1, s_new) * DH)[c16] = val;
+                        reinterpret_cast<uint4*>(cache.v + v_row<PAGED>(cache, n, H, W, hg0 + row - 1, s_new, pages, pg0) * DH)[c16] = val;
                     }
                 }
                 // the generic stores precede later bulk copies into the same bytes
@@ -275,8 +290,14 @@ swska_decode_warp_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat1
             if (lane <= HG) {  // lane 0: the K rows; lane 1 + h: head hg0 + h's V rows
                 unsigned char* d = dst + (size_t)lane * KT * ROW;
                 // rows s0 .. s0 + rows - 1 are contiguous (one page holds a whole stage)
-                const __nv_bfloat16* src = lane == 0 ? cache.k + k_row<PAGED>(cache, n, W, s0) * DH
-                                                     : cache.v + v_row<PAGED>(cache, n, H, W, hg0 + lane - 1, s0) * DH;
+                int64_t row0;
+                if (PAGED) {
+                    const int64_t t = pages[pi];
+                    row0 = lane == 0 ? t * cache.page + off : (t * H + hg0 + lane - 1) * cache.page + off;
+                } else {
+                    row0 = lane == 0 ? n * W + s0 : (n * H + hg0 + lane - 1) * W + s0;
+                }
+                const __nv_bfloat16* src = (lane == 0 ? cache.k : cache.v) + row0 * DH;
                 const int a0 = 0, a1 = r_new >= 0 ? r_new : rows;   // rows [a0, a1)
                 const int b0 = r_new >= 0 ? r_new + 1 : rows, b1 = rows;  // rows [b0, b1)
                 if (a1 > a0) bulk_g2s(d + (size_t)a0 * ROW, src + (int64_t)a0 * DH, (uint32_t)((a1 - a0) * ROW), &full[buf]);
@@ -284,6 +305,7 @@ swska_decode_warp_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat1
             }
             ++issued;
             if (++buf == stages) { buf = 0; par ^= 1u; }
+            if (PAGED && (off += KT) == cache.page) { off = 0; ++pi; }
         }
         // every copy issued has landed before the CTA's shared memory can go away (in the normal
         // course the head warps waited for these phases already)
@@ -307,8 +329,8 @@ swska_decode_warp_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat1
                 ok = false;
                 break;
             }
-            const int64_t s0 = s_begin + (int64_t)st * KT;
-            const int rows = (int)((s_end - s0) < KT ? (s_end - s0) : KT);
+            const int s0 = s_begin + st * KT;
+            const int rows = s_end - s0 < KT ? s_end - s0 : KT;
             const unsigned char* kb = ring + (size_t)buf * SB + 8 * lane;
             const unsigned char* vb = kb + (size_t)(1 + h) * KT * ROW;
             if (rows == KT) head_stage<true>(kb, vb, qw, scale_log2, KT, lane, hs);

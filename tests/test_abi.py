@@ -119,6 +119,34 @@ def test_swska_decode_validation(lib):
     assert f(None, None, None, None, None, None, None, 0, 2, 16, 32, 8, 0.0, 2, None) == OK
 
 
+def test_swska_decode_paged_validation(lib):
+    f = lib.rod_swska_decode_paged
+    # (q, k_new, v_new, k_pool, v_pool, table, page, pps, pos, o, N, H, dk, dv, W, scale, dtype, s)
+    ok = (P, P, P, P, P, P, 64, 4, P, P, 2, 16, 128, 128, 256, 0.0, 1, None)
+    args = lambda **kw: tuple(kw.get(k, v) for k, v in zip(
+        ("q", "kn", "vn", "kp", "vp", "t", "page", "pps", "pos", "o", "N", "H", "dk", "dv", "W",
+         "scale", "dt", "s"), ok))
+    assert f(*args(W=255)) == SHAPE                   # window != pages x page size
+    assert f(*args(page=12, W=48)) == SHAPE            # page size not a multiple of 8
+    assert f(*args(pps=513, W=64 * 513)) == SHAPE      # more pages than a CTA's table slice holds
+    assert f(*args(H=17)) == SHAPE
+    assert f(*args(dk=64, dv=64)) == SHAPE             # only 128-wide heads
+    assert f(*args(dt=2)) == DTYPE                     # bf16 only
+    assert f(*args(t=None)) == NULL
+    assert f(*args(kp=MIS)) == ALIGN
+    assert f(*args(N=0, q=None, kn=None, vn=None, kp=None, vp=None, t=None, pos=None, o=None)) == OK
+
+
+def test_swska_cache_fill_validation(lib):
+    f = lib.rod_swska_cache_fill
+    assert f(P, P, P, P, 1, 2, 8, 16, 32, 0, 2, None) == SHAPE    # window < 1
+    assert f(P, P, P, P, 1, 0, 8, 16, 32, 4, 2, None) == SHAPE    # no heads
+    assert f(P, P, P, P, 1, 2, 8, 16, 32, 4, 0, None) == DTYPE
+    assert f(P, None, P, P, 1, 2, 8, 16, 32, 4, 2, None) == NULL
+    assert f(P, P, MIS, P, 1, 2, 8, 16, 32, 4, 2, None) == ALIGN
+    assert f(None, None, None, None, 1, 2, 0, 16, 32, 4, 2, None) == OK   # T = 0
+
+
 def test_binding_refuses_cpu_tensors():
     import torch
     q = torch.zeros(1, 2, 8, 16)
