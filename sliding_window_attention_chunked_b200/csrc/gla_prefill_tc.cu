@@ -466,12 +466,14 @@ gla_chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
             if (tid == 0) {
                 tc::fence_after_sync();
                 if (MODE == PASS_C && fast) {
-                    const uint32_t qa = smem_u32(base + ST_Q), ka = smem_u32(base + ST_G);
+                    // descriptors built once; a K step adds its offset (bytes >> 4) to the low word
+                    const uint64_t dq = tc::sdesc_sw128(smem_u32(base + ST_Q), 16, 1024);
+                    const uint32_t q_lo = tc::desc_lo(dq), hi = tc::desc_hi(dq);
+                    const uint32_t k_lo = tc::desc_lo(tc::sdesc_sw128(smem_u32(base + ST_G), 16, 1024));
 #pragma unroll
                     for (int k = 0; k < D / 16; ++k) {
-                        const uint32_t koff = (uint32_t)((k / 4) * BOX_BYTES + (k % 4) * 32);
-                        tc::mma_ss(tmem + TM_A + 64u * st, tc::sdesc_sw128(qa + koff, 16, 1024),
-                                   tc::sdesc_sw128(ka + koff, 16, 1024), idesc_A, k > 0);
+                        const uint32_t koff = (uint32_t)(((k / 4) * BOX_BYTES + (k % 4) * 32) >> 4);
+                        tc::mma_ss_lh(tmem + TM_A + 64u * st, q_lo + koff, hi, k_lo + koff, hi, idesc_A, k > 0);
                     }
                     tc::mma_commit(&barA[st]);
                 }
@@ -600,24 +602,26 @@ gla_chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
             if (tid == 128) {
                 tc::fence_after_sync();
                 // R += k^'^T V (pass A starts from an empty R: the first MMA overwrites)
-                const uint32_t kh = smem_u32(base + ST_K), va = smem_u32(base + ST_V);
+                // descriptors built once (all share the high word: SBO 1024, SW128); a K step adds
+                // its offset (bytes >> 4) to the low word
+                const uint64_t dkh = tc::sdesc_sw128(smem_u32(base + ST_K), BOX_BYTES, 1024);
+                const uint32_t kh_lo = tc::desc_lo(dkh), hi = tc::desc_hi(dkh);
+                const uint32_t va_lo = tc::desc_lo(tc::sdesc_sw128(smem_u32(base + ST_V), BOX_BYTES, 1024));
 #pragma unroll
                 for (int k = 0; k < C / 16; ++k)
-                    tc::mma_ss(tmem + TM_S, tc::sdesc_sw128(kh + 2048u * k, BOX_BYTES, 1024),
-                               tc::sdesc_sw128(va + 2048u * k, BOX_BYTES, 1024), idesc_U,
-                               (MODE == PASS_A && n == 0 && k == 0) ? 0u : 1u);
+                    tc::mma_ss_lh(tmem + TM_S, kh_lo + 128u * k, hi, va_lo + 128u * k, hi, idesc_U,
+                                  (MODE == PASS_A && n == 0 && k == 0) ? 0u : 1u);
                 if (MODE == PASS_C) {  // O = P V + q~' R_bf16
-                    const uint32_t pa = smem_u32(base + ST_P), qa = smem_u32(base + ST_Q);
-                    const uint32_t sb = smem_u32(smem + OFF_SBF);
+                    const uint32_t pa_lo = tc::desc_lo(tc::sdesc_sw128(smem_u32(base + ST_P), 16, 1024));
+                    const uint32_t qa_lo = tc::desc_lo(tc::sdesc_sw128(smem_u32(base + ST_Q), 16, 1024));
+                    const uint32_t sb_lo = tc::desc_lo(tc::sdesc_sw128(smem_u32(smem + OFF_SBF), D * 128, 1024));
 #pragma unroll
                     for (int k = 0; k < C / 16; ++k)
-                        tc::mma_ss(tmem + TM_O, tc::sdesc_sw128(pa + 32u * k, 16, 1024),
-                                   tc::sdesc_sw128(va + 2048u * k, BOX_BYTES, 1024), idesc_O, k > 0);
+                        tc::mma_ss_lh(tmem + TM_O, pa_lo + 2u * k, hi, va_lo + 128u * k, hi, idesc_O, k > 0);
 #pragma unroll
                     for (int k = 0; k < D / 16; ++k)
-                        tc::mma_ss(tmem + TM_O,
-                                   tc::sdesc_sw128(qa + (uint32_t)((k / 4) * BOX_BYTES + (k % 4) * 32), 16, 1024),
-                                   tc::sdesc_sw128(sb + 2048u * k, D * 128, 1024), idesc_O, 1u);
+                        tc::mma_ss_lh(tmem + TM_O, qa_lo + (uint32_t)(((k / 4) * BOX_BYTES + (k % 4) * 32) >> 4), hi,
+                                      sb_lo + 128u * k, hi, idesc_O, 1u);
                 }
                 tc::mma_commit(barO);
                 tc::mma_commit(&empty[st]);
