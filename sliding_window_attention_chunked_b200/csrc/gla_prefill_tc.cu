@@ -116,6 +116,23 @@ __device__ __forceinline__ uint32_t sw_off_elem(int row, int col, int rows) {
     return sw_off(row, col & ~7, rows) + ((col & 7) << 1);
 }
 
+// fp32 pairs in one 64-bit register for the two-wide instructions
+__device__ __forceinline__ uint64_t pk2(float a, float b) {
+    uint64_t r;
+    asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(a), "f"(b));
+    return r;
+}
+__device__ __forceinline__ float2 upk2(uint64_t r) {
+    float2 d;
+    asm("mov.b64 {%0, %1}, %2;" : "=f"(d.x), "=f"(d.y) : "l"(r));
+    return d;
+}
+__device__ __forceinline__ uint64_t mul2(uint64_t a, uint64_t b) {
+    uint64_t d;
+    asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+    return d;
+}
+
 __device__ __forceinline__ bool wait_bar(uint64_t* bar, uint32_t parity, volatile int* abort_flag) {
     for (uint32_t i = 1;; ++i) {
         if (mbar_try_wait(bar, parity)) return true;
@@ -349,26 +366,42 @@ gla_chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                     a_dn[j] = a[j] * rcp(dn[j]);
                     inv_d[j] = rcp(Dc[j]);
                 }
+                // channel pairs in two-wide fp32 registers (mul.rn.f32x2: one instruction per pair)
+                uint64_t pre2[4], adn2[4], dc2[4], invd2[4];
+#pragma unroll
+                for (int p = 0; p < 4; ++p) {
+                    pre2[p] = pk2(pre[2 * p], pre[2 * p + 1]);
+                    adn2[p] = pk2(a_dn[2 * p], a_dn[2 * p + 1]);
+                    dc2[p] = pk2(Dc[2 * p], Dc[2 * p + 1]);
+                    invd2[p] = pk2(inv_d[2 * p], inv_d[2 * p + 1]);
+                }
 #pragma unroll
                 for (int i = 0; i < 8; ++i) {
                     const uint32_t off = sw_off(r0 + i, c0, C);
-                    float qf[8], kf[8], qt[8], kt[8], kh[8];
-                    unpack8(*reinterpret_cast<const uint4*>(base + ST_K + off), kf);
-                    if (MODE == PASS_C) unpack8(*reinterpret_cast<const uint4*>(base + ST_Q + off), qf);
+                    const uint4 kw = *reinterpret_cast<const uint4*>(base + ST_K + off);
+                    uint4 qw = make_uint4(0u, 0u, 0u, 0u);
+                    if (MODE == PASS_C) qw = *reinterpret_cast<const uint4*>(base + ST_Q + off);
+                    const uint32_t kws[4] = {kw.x, kw.y, kw.z, kw.w}, qws[4] = {qw.x, qw.y, qw.z, qw.w};
+                    uint32_t khp[4], qtp[4], ktp[4];
 #pragma unroll
-                    for (int j = 0; j < 8; ++j) {
-                        const float Gt = G[i][j] * pre[j];
-                        const float r = rcp(Gt);
-                        kh[j] = kf[j] * (r * a_dn[j]);
+                    for (int p = 0; p < 4; ++p) {
+                        const uint64_t kf2 = pk2(bf16lo(kws[p]), bf16hi(kws[p]));
+                        const uint64_t Gt2 = mul2(pk2(G[i][2 * p], G[i][2 * p + 1]), pre2[p]);
+                        const float2 gt = upk2(Gt2);
+                        const uint64_t r2 = pk2(rcp(gt.x), rcp(gt.y));
+                        const float2 kh = upk2(mul2(kf2, mul2(r2, adn2[p])));
+                        khp[p] = pack_bf16x2(kh.x, kh.y);
                         if (MODE == PASS_C) {
-                            qt[j] = qf[j] * (Gt * Dc[j]);
-                            kt[j] = kf[j] * (r * inv_d[j]);
+                            const float2 qt = upk2(mul2(pk2(bf16lo(qws[p]), bf16hi(qws[p])), mul2(Gt2, dc2[p])));
+                            const float2 kt = upk2(mul2(kf2, mul2(r2, invd2[p])));
+                            qtp[p] = pack_bf16x2(qt.x, qt.y);
+                            ktp[p] = pack_bf16x2(kt.x, kt.y);
                         }
                     }
-                    *reinterpret_cast<uint4*>(base + ST_K + off) = pack8(kh);
+                    *reinterpret_cast<uint4*>(base + ST_K + off) = make_uint4(khp[0], khp[1], khp[2], khp[3]);
                     if (MODE == PASS_C) {
-                        *reinterpret_cast<uint4*>(base + ST_Q + off) = pack8(qt);
-                        *reinterpret_cast<uint4*>(base + ST_G + off) = pack8(kt);
+                        *reinterpret_cast<uint4*>(base + ST_Q + off) = make_uint4(qtp[0], qtp[1], qtp[2], qtp[3]);
+                        *reinterpret_cast<uint4*>(base + ST_G + off) = make_uint4(ktp[0], ktp[1], ktp[2], ktp[3]);
                     }
                 }
                 publish(rmw, dn);
