@@ -135,6 +135,31 @@ ROD_API int rod_gla_prefill_noalloc(const void* q, const void* k, const void* v,
                                     float* state, void* o, int B, int H, int T, int dk, int dv,
                                     int chunk, int dtype, void* stream);
 
+/* ---- gated linear recurrence: backward (training path) -------------------------------------- */
+/*
+ * Gradients of the recurrence of rod_gla_prefill (CodeFuse article, Rodimus block: the
+ * chunkwise-parallel algorithm serves training as well as prefill). For the loss gradients
+ * dO_t of every output o_t and dstate_final of the final state:
+ *   dq_t = S_t dO_t;  dS_t = q_t^T dO_t + diag(g_{t+1}) dS_{t+1} (dS_T from dstate_final);
+ *   dk_t = dS_t v_t;  dv_t = dS_t^T k_t;  dg_t[c] = sum_j dS_t[c][j] S_{t-1}[c][j];
+ *   dstate0 = diag(g_1) dS_1  (the gradient of the initial state; dstate_final when T = 0).
+ *   q, k [B,H,T,dk], v [B,H,T,dv], dO [B,H,T,dv]: dtype;  g [B,H,T,dk] fp32;
+ *   state0 [B,H,dk,dv] fp32: the initial state the forward started from;
+ *   dstate_final [B,H,dk,dv] fp32, or NULL for no loss on the final state;
+ *   outputs dq, dk [B,H,T,dk] and dv [B,H,T,dv] in dtype; dg [B,H,T,dk] and dstate0
+ *   [B,H,dk,dv] fp32; workspace of rod_gla_backward_workspace_size bytes (caller-owned).
+ * Runs on CUDA cores with every product an fp32 FMA (three sweeps over the sequence per
+ * (batch, head), states in registers).
+ * Errors: ROD_ERR_NULL, ROD_ERR_SHAPE, ROD_ERR_ALIGN, ROD_ERR_DTYPE, ROD_ERR_WORKSPACE,
+ * ROD_ERR_CUDA. B*H = 0 is a no-op.
+ */
+ROD_API size_t rod_gla_backward_workspace_size(int B, int H, int T, int dk, int dv);
+ROD_API int rod_gla_backward(const void* q, const void* k, const void* v, const float* g,
+                             const float* state0, const void* dO, const float* dstate_final,
+                             void* dq, void* dk, void* dv, float* dg, float* dstate0, int B,
+                             int H, int T, int dk_dim, int dv_dim, int dtype, void* workspace,
+                             size_t ws_bytes, void* stream);
+
 /* ---- gated linear recurrence: one decode step --------------------------------------------- */
 /*
  * One token for each of N sequences x H heads, with the fixed-size state updated in place

@@ -47,7 +47,10 @@ class OracleLib:
                                                   ctypes.POINTER(ctypes.c_int32), i64, i64, i64p,
                                                   f64p, i64, i64, i64, i64, i64, ctypes.c_double,
                                                   ctypes.c_int]
-        for name in ("rodref_gla_prefill", "rodref_gla_decode_step", "rodref_swska_prefill",
+        lib.rodref_gla_backward.argtypes = [f32p, f32p, f32p, f32p, f64p, f32p, f32p, f64p, f64p,
+                                            f64p, f64p, f64p, i64, i64, i64, i64, i64, ctypes.c_int]
+        for name in ("rodref_gla_backward", "rodref_gla_prefill", "rodref_gla_decode_step",
+                     "rodref_swska_prefill",
                      "rodref_swska_decode", "rodref_swska_cache_fill", "rodref_swska_decode_paged"):
             getattr(lib, name).restype = ctypes.c_int
         self.lib = lib
@@ -242,3 +245,23 @@ def swska_decode_paged(q, k_new, v_new, k_pool, v_pool, block_table, page_size, 
                                         nthreads or default_threads())
     _check(rc, "swska_decode_paged")
     return o, kp, vp
+
+
+def gla_backward(q, k, v, g, dO, state0=None, dS_final=None, nthreads=None):
+    """Gradients of the recurrence (rodref_gla_backward) for loss gradients dO [B,H,T,dv] and
+    dS_final [B,H,dk,dv] (None: no loss on the final state). Returns float64
+    (dq, dk, dv, dg, dstate0)."""
+    q, k, v, g, dO = _f32(q), _f32(k), _f32(v), _f32(g), _f32(dO)
+    B, H, T, dk = q.shape
+    dv = v.shape[-1]
+    S0 = np.zeros((B, H, dk, dv)) if state0 is None else np.ascontiguousarray(_f64(state0))
+    dSf = None if dS_final is None else _f32(dS_final)
+    outs = [np.empty((B, H, T, dk)), np.empty((B, H, T, dk)), np.empty((B, H, T, dv)),
+            np.empty((B, H, T, dk)), np.empty((B, H, dk, dv))]
+    dq, dk_, dv_, dg, dS0 = outs
+    rc = _L().rodref_gla_backward(_p32(q), _p32(k), _p32(v), _p32(g), _p64(S0), _p32(dO),
+                                  None if dSf is None else _p32(dSf), _p64(dq), _p64(dk_),
+                                  _p64(dv_), _p64(dg), _p64(dS0), B, H, T, dk, dv,
+                                  nthreads or default_threads())
+    _check(rc, "gla_backward")
+    return dq, dk_, dv_, dg, dS0

@@ -141,6 +141,107 @@ int rodref_gla_prefill(const float* q, const float* k, const float* v, const flo
     return run_units(gla_unit, &a, B * H, nthreads);
 }
 
+/* ------------------------------------------------------------------------------------------
+ * Backward of the recurrence (the chunkwise-parallel algorithm is stated for training too,
+ * [CodeFuse] Rodimus block): reverse-mode differentiation of gla_step, written out.
+ * Loss gradients dO_t (of every o_t) and dS_final (of the final state S_T, may be absent).
+ *   dq_t[c]  = sum_j dO_t[j] S_t[c][j]                       (S_t after step t)
+ *   dS_t     = q_t^T dO_t + diag(g_{t+1}) dS_{t+1},  dS_T starting from dS_final
+ *   dk_t[c]  = sum_j dS_t[c][j] v_t[j];   dv_t[j] = sum_c dS_t[c][j] k_t[c]
+ *   dg_t[c]  = sum_j dS_t[c][j] S_{t-1}[c][j]
+ *   dS_0     = diag(g_1) dS_1  (gradient of the initial state)
+ * The states S_{t-1} the reverse sweep needs are recomputed per block of 64 steps from
+ * checkpoints saved by the forward sweep.
+ * ---------------------------------------------------------------------------------------- */
+typedef struct {
+    const float *q, *k, *v, *g, *dO, *dSf;
+    const double* state0;
+    double *dq, *dk, *dv, *dg, *dstate0;
+    int64_t T, dk_, dv_;
+} gla_bwd_args_t;
+
+#define GLA_BWD_BLOCK 64
+
+static void gla_bwd_unit(const void* p, int64_t bh) {
+    const gla_bwd_args_t* a = (const gla_bwd_args_t*)p;
+    const int64_t T = a->T, dk = a->dk_, dv = a->dv_, DD = dk * dv;
+    const int64_t nblk = (T + GLA_BWD_BLOCK - 1) / GLA_BWD_BLOCK;
+    double* ckpt = malloc((size_t)((nblk + 1) * DD) * sizeof(double));
+    double* Sb = malloc((size_t)((GLA_BWD_BLOCK + 1) * DD) * sizeof(double));
+    double* dS = malloc((size_t)DD * sizeof(double));
+    if (!ckpt || !Sb || !dS) { free(ckpt); free(Sb); free(dS); return; }
+    /* forward sweep: checkpoints (state before each block) and dq */
+    double* S = Sb;
+    memcpy(S, a->state0 + bh * DD, (size_t)DD * sizeof(double));
+    for (int64_t t = 0; t < T; ++t) {
+        if (t % GLA_BWD_BLOCK == 0) memcpy(ckpt + (t / GLA_BWD_BLOCK) * DD, S, (size_t)DD * sizeof(double));
+        const int64_t tk = (bh * T + t) * dk, tv = (bh * T + t) * dv;
+        for (int64_t c = 0; c < dk; ++c)
+            for (int64_t j = 0; j < dv; ++j)
+                S[c * dv + j] = (double)a->g[tk + c] * S[c * dv + j] + (double)a->k[tk + c] * (double)a->v[tv + j];
+        for (int64_t c = 0; c < dk; ++c) {
+            double acc = 0.0;
+            for (int64_t j = 0; j < dv; ++j) acc += (double)a->dO[tv + j] * S[c * dv + j];
+            a->dq[tk + c] = acc;
+        }
+    }
+    /* reverse sweep */
+    for (int64_t i = 0; i < DD; ++i) dS[i] = a->dSf ? (double)a->dSf[bh * DD + i] : 0.0;
+    for (int64_t blk = nblk - 1; blk >= 0; --blk) {
+        const int64_t t0 = blk * GLA_BWD_BLOCK, t1 = t0 + GLA_BWD_BLOCK < T ? t0 + GLA_BWD_BLOCK : T;
+        memcpy(Sb, ckpt + blk * DD, (size_t)DD * sizeof(double));   /* Sb[i] = S before step t0+i */
+        for (int64_t t = t0; t < t1; ++t) {
+            const double* Sp = Sb + (t - t0) * DD;
+            double* Sn = Sb + (t - t0 + 1) * DD;
+            const int64_t tk = (bh * T + t) * dk, tv = (bh * T + t) * dv;
+            for (int64_t c = 0; c < dk; ++c)
+                for (int64_t j = 0; j < dv; ++j)
+                    Sn[c * dv + j] = (double)a->g[tk + c] * Sp[c * dv + j] + (double)a->k[tk + c] * (double)a->v[tv + j];
+        }
+        for (int64_t t = t1 - 1; t >= t0; --t) {
+            const double* Sprev = Sb + (t - t0) * DD;
+            const int64_t tk = (bh * T + t) * dk, tv = (bh * T + t) * dv;
+            for (int64_t c = 0; c < dk; ++c)
+                for (int64_t j = 0; j < dv; ++j) dS[c * dv + j] += (double)a->q[tk + c] * (double)a->dO[tv + j];
+            for (int64_t c = 0; c < dk; ++c) {
+                double acck = 0.0, accg = 0.0;
+                for (int64_t j = 0; j < dv; ++j) {
+                    acck += dS[c * dv + j] * (double)a->v[tv + j];
+                    accg += dS[c * dv + j] * Sprev[c * dv + j];
+                }
+                a->dk[tk + c] = acck;
+                a->dg[tk + c] = accg;
+            }
+            for (int64_t j = 0; j < dv; ++j) {
+                double acc = 0.0;
+                for (int64_t c = 0; c < dk; ++c) acc += dS[c * dv + j] * (double)a->k[tk + c];
+                a->dv[tv + j] = acc;
+            }
+            for (int64_t c = 0; c < dk; ++c)
+                for (int64_t j = 0; j < dv; ++j) dS[c * dv + j] *= (double)a->g[tk + c];
+        }
+    }
+    memcpy(a->dstate0 + bh * DD, dS, (size_t)DD * sizeof(double));
+    free(ckpt);
+    free(Sb);
+    free(dS);
+}
+
+/*
+ * q, k, g, dq, dk, dg: [B,H,T,dk]; v, dO, dv: [B,H,T,dv]; state0, dstate0: [B,H,dk,dv];
+ * dS_final: [B,H,dk,dv] or NULL (no loss on the final state).
+ */
+int rodref_gla_backward(const float* q, const float* k, const float* v, const float* g,
+                        const double* state0, const float* dO, const float* dS_final, double* dq,
+                        double* dk_out, double* dv_out, double* dg, double* dstate0, int64_t B,
+                        int64_t H, int64_t T, int64_t dk, int64_t dv, int nthreads) {
+    if (!q || !k || !v || !g || !state0 || !dO || !dq || !dk_out || !dv_out || !dg || !dstate0)
+        return RODREF_EINVAL;
+    if (B < 0 || H < 0 || T < 0 || dk < 1 || dv < 1) return RODREF_EINVAL;
+    gla_bwd_args_t a = {q, k, v, g, dO, dS_final, state0, dq, dk_out, dv_out, dg, dstate0, T, dk, dv};
+    return run_units(gla_bwd_unit, &a, B * H, nthreads);
+}
+
 /*
  * One decode step for N sequences: q, k, g: [N,H,dk]; v: [N,H,dv];
  * state [N,H,dk,dv] updated in place; o: [N,H,dv]. Identical to a prefill with T = 1.

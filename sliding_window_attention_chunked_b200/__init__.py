@@ -7,6 +7,7 @@ the calls raise.
 
     gla_prefill(q, k, v, g, state, chunk=64)       chunkwise prefill of the gated recurrence
     gla_decode_step(q, k, v, g, state)              one fused recurrent decode step
+    gla_backward(q, k, v, g, dO, state0, dstate_final)   gradients of the recurrence
     swska_prefill(q, k, v, window, scale=None)      sliding-window shared-key attention
     swska_decode(q, k_new, v_new, k_cache, v_cache, pos, window)   ring-buffer decode
     swska_cache_fill(k, v, k_cache, v_cache, window)   prefill -> decode ring-buffer hand-off
@@ -19,6 +20,7 @@ from ._binding import (  # noqa: F401
     RodError,
     abi_version,
     check,
+    gla_backward,
     gla_decode_step,
     gla_prefill,
     gla_prefill_noalloc,

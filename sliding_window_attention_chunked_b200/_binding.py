@@ -69,6 +69,10 @@ def load_library() -> ctypes.CDLL:
     lib.rod_swska_decode_paged.argtypes = [vp, vp, vp, vp, vp, vp, i, i, vp, vp, i, i, i, i, i, f,
                                            i, vp]
     lib.rod_swska_decode_paged.restype = i
+    lib.rod_gla_backward_workspace_size.argtypes = [i, i, i, i, i]
+    lib.rod_gla_backward_workspace_size.restype = sz
+    lib.rod_gla_backward.argtypes = [vp] * 12 + [i] * 6 + [vp, sz, vp]
+    lib.rod_gla_backward.restype = i
     lib.rod_swska_cache_fill.restype = i
     _lib = lib
     return lib
@@ -293,3 +297,34 @@ def swska_decode_paged(q, k_new, v_new, k_pool, v_pool, block_table, page_size, 
                                                _dtype_code(q), _stream(stream))
     _raise_on("rod_swska_decode_paged", st)
     return o
+
+
+def gla_backward(q, k, v, g, dO, state0=None, dstate_final=None, workspace=None, stream=None):
+    """Gradients of gla_prefill: q, k, v, dO [B,H,T,*] (dtype), g fp32, state0 [B,H,dk,dv] fp32
+    (None: zeros), dstate_final [B,H,dk,dv] fp32 or None. Returns (dq, dk, dv, dg, dstate0)."""
+    _need(q, "q", None, 4)
+    for n, t in (("k", k), ("v", v), ("dO", dO)):
+        _need(t, n, q.dtype, 4)
+    _need(g, "g", torch.float32, 4)
+    B, H, T, dk = q.shape
+    dv = v.shape[-1]
+    if tuple(k.shape) != (B, H, T, dk) or tuple(g.shape) != (B, H, T, dk) or tuple(dO.shape) != (B, H, T, dv):
+        raise ValueError("shape mismatch")
+    if state0 is None:
+        state0 = torch.zeros(B, H, dk, dv, dtype=torch.float32, device=q.device)
+    _need(state0, "state0", torch.float32, 4)
+    if dstate_final is not None:
+        _need(dstate_final, "dstate_final", torch.float32, 4)
+    lib = load_library()
+    need = lib.rod_gla_backward_workspace_size(B, H, T, dk, dv)
+    if workspace is None:
+        workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=q.device)
+    dq, dk_, dv_ = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    dg = torch.empty_like(g)
+    dS0 = torch.empty_like(state0)
+    st = lib.rod_gla_backward(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(state0), _ptr(dO),
+                              None if dstate_final is None else _ptr(dstate_final), _ptr(dq),
+                              _ptr(dk_), _ptr(dv_), _ptr(dg), _ptr(dS0), B, H, T, dk, dv,
+                              _dtype_code(q), _ptr(workspace), workspace.numel(), _stream(stream))
+    _raise_on("rod_gla_backward", st)
+    return dq, dk_, dv_, dg, dS0

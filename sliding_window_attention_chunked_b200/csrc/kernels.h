@@ -67,6 +67,22 @@ cudaError_t swska_decode_paged_launch(const void* q, const void* k_new, const vo
                                       int pages_per_seq, const int64_t* pos, void* o, int N, int H,
                                       int window, float scale, cudaStream_t stream);
 
+// backward of the recurrence (CUDA cores): gradients of q, k, v, g and of the initial state
+struct GlaBackwardArgs {
+    const void *q, *k, *v;
+    const float* g;
+    const float* state0;        // [B,H,dk,dv]
+    const void* dO;             // [B,H,T,dv]
+    const float* dstate_final;  // [B,H,dk,dv] or nullptr
+    void *dq, *dk, *dv;         // dtype
+    float* dg;                  // [B,H,T,dk]
+    float* dstate0;             // [B,H,dk,dv]
+    int B, H, T, d_k, d_v;
+    void* workspace;
+};
+size_t gla_backward_workspace_size(int B, int H, int T, int dk, int dv);
+cudaError_t gla_backward_launch(const GlaBackwardArgs& a, bool bf16, cudaStream_t stream);
+
 // SW-SKA prefill -> decode hand-off: the last W tokens' K / V rows into the ring buffers
 cudaError_t swska_cache_fill_launch(const void* k, const void* v, void* k_cache, void* v_cache, int B,
                                     int H, int T, int dk, int dv, int window, size_t elem_bytes,

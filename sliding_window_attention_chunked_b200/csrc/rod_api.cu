@@ -146,6 +146,40 @@ int rod_swska_decode(const void* q, const void* k_new, const void* v_new, void* 
                                               static_cast<cudaStream_t>(stream)));
 }
 
+size_t rod_gla_backward_workspace_size(int B, int H, int T, int dk, int dv) {
+    if (B < 0 || H < 0 || T < 0 || !dim_ok(dk) || !dim_ok(dv)) return 0;
+    return rod::gla_backward_workspace_size(B, H, T, dk, dv);
+}
+
+int rod_gla_backward(const void* q, const void* k, const void* v, const float* g, const float* state0,
+                     const void* dO, const float* dstate_final, void* dq, void* dk, void* dv, float* dg,
+                     float* dstate0, int B, int H, int T, int dk_dim, int dv_dim, int dtype,
+                     void* workspace, size_t ws_bytes, void* stream) {
+    if (!dtype_ok(dtype)) return ROD_ERR_DTYPE;
+    if (B < 0 || H < 0 || T < 0 || !dim_ok(dk_dim) || !dim_ok(dv_dim)) return ROD_ERR_SHAPE;
+    if ((int64_t)B * H == 0) return ROD_OK;
+    if (!state0 || !dstate0) return ROD_ERR_NULL;
+    if (!aligned16(state0) || !aligned16(dstate0) || (dstate_final && !aligned16(dstate_final)))
+        return ROD_ERR_ALIGN;
+    const cudaStream_t s = static_cast<cudaStream_t>(stream);
+    const size_t state_bytes = (size_t)B * H * dk_dim * dv_dim * sizeof(float);
+    if (T == 0) {  // nothing in between: the initial state's gradient is the final state's
+        return from_cuda(dstate_final
+                             ? cudaMemcpyAsync(dstate0, dstate_final, state_bytes, cudaMemcpyDeviceToDevice, s)
+                             : cudaMemsetAsync(dstate0, 0, state_bytes, s));
+    }
+    if (!q || !k || !v || !g || !dO || !dq || !dk || !dv || !dg) return ROD_ERR_NULL;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(g) || !aligned16(dO) ||
+        !aligned16(dq) || !aligned16(dk) || !aligned16(dv) || !aligned16(dg))
+        return ROD_ERR_ALIGN;
+    const size_t need = rod::gla_backward_workspace_size(B, H, T, dk_dim, dv_dim);
+    if (!workspace || ws_bytes < need) return ROD_ERR_WORKSPACE;
+    if (!aligned16(workspace)) return ROD_ERR_ALIGN;
+    rod::GlaBackwardArgs a{q, k, v, g, state0, dO, dstate_final, dq, dk, dv, dg, dstate0,
+                           B, H, T, dk_dim, dv_dim, workspace};
+    return from_cuda(rod::gla_backward_launch(a, dtype == ROD_BF16, s));
+}
+
 int rod_swska_decode_paged(const void* q, const void* k_new, const void* v_new, void* k_pool,
                            void* v_pool, const int32_t* block_table, int page_size, int pages_per_seq,
                            const int64_t* pos, void* o, int N, int H, int dk, int dv, int window,

@@ -1,0 +1,77 @@
+"""Backward of the gated linear recurrence on the GPU against the oracle's reverse-mode sweep.
+
+The oracle's gradients are pinned on the CPU (central differences, PyTorch autograd through a
+float64 loop, and the gate identity); here every gradient the library returns (dq, dk, dv in the
+input dtype; dg and the initial-state gradient in fp32) is compared with them element by
+element: fp32 inputs within the fp32 tolerance, bf16 inputs within the bf16 tolerance for the
+bf16 outputs and the fp32 tolerance for the fp32 ones (their arithmetic is fp32 throughout).
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import sliding_window_attention_chunked_b200 as rod
+from sliding_window_attention_chunked_b200 import workloads as wl
+
+from .parity import compare
+
+pytestmark = pytest.mark.gpu
+DEV = "cuda"
+
+
+def _case(B, H, T, dk, dv, dtype, seed, gate=None, final=True):
+    q, k, v, g = wl.gla_inputs(B, H, T, dk, dv, dist="l2", seed=seed, dtype=dtype)
+    if gate is not None:
+        g = torch.full_like(g, float(gate))
+    # loss gradients and initial state scaled so the gradients are O(1): the bf16 bound (2e-2
+    # absolute) is stated for outputs of that size (bf16 rounding alone is |x| 2^-9)
+    gen = torch.Generator().manual_seed(seed + 1)
+    S0 = torch.randn(B, H, dk, dv, generator=gen) * 0.1
+    dO = (torch.randn(B, H, T, dv, generator=gen) * 0.2).to(q.dtype)
+    dSf = torch.randn(B, H, dk, dv, generator=gen) * 0.1 if final else None
+    return q, k, v, g, S0, dO, dSf
+
+
+def _check(B, H, T, dk, dv, dtype, seed, gate=None, final=True):
+    q, k, v, g, S0, dO, dSf = _case(B, H, T, dk, dv, dtype, seed, gate, final)
+    ref = oracle.gla_backward(q, k, v, g, dO, S0.double(), dSf)
+    got = rod.gla_backward(q.to(DEV), k.to(DEV), v.to(DEV), g.to(DEV), dO.to(DEV), S0.to(DEV),
+                           None if dSf is None else dSf.to(DEV))
+    rod.check()
+    names = ("dq", "dk", "dv", "dg", "dstate0")
+    for name, a, b in zip(names, got, ref):
+        tol = dtype if name in ("dq", "dk", "dv") else "fp32"
+        compare(a, b, tol, f"{name} B{B} H{H} T{T} dk{dk} dv{dv} {dtype}")
+
+
+@pytest.mark.parametrize("dk,dv", [(16, 32), (32, 16), (64, 64), (128, 128), (16, 128)])
+def test_gla_backward_fp32(dk, dv):
+    _check(2, 3, 200, dk, dv, "fp32", seed=dk + dv)
+
+
+@pytest.mark.parametrize("T", [1, 63, 64, 65, 300])
+def test_gla_backward_bf16_lengths_across_checkpoints(T):
+    _check(1, 2, T, 128, 128, "bf16", seed=T)
+
+
+@pytest.mark.parametrize("gate", [0.0, 1.0])
+def test_gla_backward_gate_edges(gate):
+    """g = 0 (the state resets every step: no gradient flows back through it) and g = 1."""
+    _check(1, 2, 130, 64, 32, "fp32", seed=7, gate=gate)
+
+
+def test_gla_backward_without_final_state_loss():
+    _check(2, 2, 150, 32, 64, "fp32", seed=9, final=False)
+
+
+def test_gla_backward_empty_sequence_passes_the_final_gradient_through():
+    B, H, d = 2, 3, 32
+    dSf = torch.randn(B, H, d, d, device=DEV)
+    z = torch.zeros(B, H, 0, d, device=DEV)
+    _, _, _, _, dS0 = rod.gla_backward(z, z, z, z, z, torch.zeros(B, H, d, d, device=DEV), dSf)
+    rod.check()
+    assert torch.equal(dS0, dSf)
+    _, _, _, _, dS0 = rod.gla_backward(z, z, z, z, z, torch.zeros(B, H, d, d, device=DEV), None)
+    rod.check()
+    assert torch.equal(dS0, torch.zeros_like(dSf))

@@ -4,7 +4,8 @@ Each case copies oracle/rodref.c to a temporary directory, plants one plausible 
 textual substitution (a gate applied to the wrong channel, a decay that also hits the new
 term, the readout using k, an off-by-one window, a dropped scale or normaliser, a wrong
 ring-buffer slot, a hand-off that drops a token or numbers slots from the window start, a paged cache read
-without its table or written at the wrong row), builds the copy with gcc and runs every pin against it. Each planted
+without its table or written at the wrong row, a backward that weights the gate gradient
+with the updated state or decays the gradient state on the wrong channel), builds the copy with gcc and runs every pin against it. Each planted
 mistake must make at least one pin fail; otherwise the pins are too weak to trust.
 """
 import inspect
@@ -40,6 +41,10 @@ MUTATIONS = {
                                    "const int64_t slot = (p - p0) % W;"),
     "paged_read_ignores_table": ("const int64_t t = table[n * pps + s / page], r = s % page;",
                                  "const int64_t t = n * pps + s / page, r = s % page;"),
+    "bwd_dg_with_new_state": ("accg += dS[c * dv + j] * Sprev[c * dv + j];",
+                              "accg += dS[c * dv + j] * Sprev[DD + c * dv + j];"),
+    "bwd_decay_wrong_channel": ("for (int64_t j = 0; j < dv; ++j) dS[c * dv + j] *= (double)a->g[tk + c];",
+                                "for (int64_t j = 0; j < dv; ++j) dS[c * dv + j] *= (double)a->g[tk + (c + 1) % dk];"),
     "paged_write_wrong_row": ("t = table[n * pps + s / page], r = s % page;\n            memcpy(k_pool",
                               "t = table[n * pps + s / page], r = (s + 1) % page;\n            memcpy(k_pool"),
 }

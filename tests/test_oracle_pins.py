@@ -362,3 +362,92 @@ def test_swska_paged_decode_continues_prefill_and_writes_only_its_pages(W, page)
     for pg in range(P_pages):
         untouched = bool((kp[pg] == 7.0).all() and (vp[pg] == 7.0).all())
         assert untouched == (pg not in used), pg
+
+
+# ------------------------------------------------------------------------------------------
+# backward of the recurrence
+# ------------------------------------------------------------------------------------------
+
+
+def _gla_loss(q, k, v, g, S0, dO, dSf):
+    o, ST = oracle.gla_prefill(q, k, v, g, S0)
+    return float(np.sum(o * dO) + np.sum(ST * dSf))
+
+
+def test_gla_backward_finite_differences():
+    """Central differences of L = sum(o . dO) + sum(S_T . dS_final) on a tiny case. Inputs are
+    multiples of 2^-8 and the step is 2^-8, so every perturbed input is exact in fp32; L is
+    linear in q, k, v, S_0 (central differences exact up to rounding) and a degree-T polynomial
+    in the gates (truncation ~h^2)."""
+    B, H, T, dk, dv = 1, 1, 7, 3, 2
+    r = _rng(31)
+    grid = lambda shape, lo, hi: (np.round(r.uniform(lo, hi, shape) * 256) / 256).astype(np.float32)
+    q, k = grid((B, H, T, dk), -1, 1), grid((B, H, T, dk), -1, 1)
+    v, g = grid((B, H, T, dv), -1, 1), grid((B, H, T, dk), 0.3, 0.95)
+    S0 = r.standard_normal((B, H, dk, dv))
+    dO = r.standard_normal((B, H, T, dv)).astype(np.float32)
+    dSf = r.standard_normal((B, H, dk, dv)).astype(np.float32)
+    dq, dk_, dv_, dg, dS0 = oracle.gla_backward(q, k, v, g, dO, S0, dSf)
+    h = 2.0 ** -8
+    for name, x, grad, tol in (("q", q, dq, 1e-9), ("k", k, dk_, 1e-9), ("v", v, dv_, 1e-9),
+                               ("g", g, dg, 2e-4)):
+        for idx in np.ndindex(x.shape):
+            xp, xm = x.copy(), x.copy()
+            xp[idx] += h
+            xm[idx] -= h
+            args = {"q": q, "k": k, "v": v, "g": g}
+            fp = _gla_loss(*[xp if n == name else args[n] for n in "qkvg"], S0, dO, dSf)
+            fm = _gla_loss(*[xm if n == name else args[n] for n in "qkvg"], S0, dO, dSf)
+            fd = (fp - fm) / (2 * h)
+            assert abs(fd - grad[idx]) <= tol * max(1.0, abs(fd)), (name, idx, fd, grad[idx])
+    for idx in np.ndindex(S0.shape):
+        Sp, Sm = S0.copy(), S0.copy()
+        Sp[idx] += h
+        Sm[idx] -= h
+        fd = (_gla_loss(q, k, v, g, Sp, dO, dSf) - _gla_loss(q, k, v, g, Sm, dO, dSf)) / (2 * h)
+        assert abs(fd - dS0[idx]) <= 1e-9 * max(1.0, abs(fd))
+
+
+def test_gla_backward_matches_torch_autograd():
+    """The same gradients from PyTorch autograd through a float64 loop of the recurrence."""
+    torch = pytest.importorskip("torch")
+    B, H, T, dk, dv = 2, 2, 70, 5, 4
+    r = _rng(32)
+    q, k = [r.standard_normal((B, H, T, dk)).astype(np.float32) for _ in range(2)]
+    v = r.standard_normal((B, H, T, dv)).astype(np.float32)
+    g = r.uniform(0.2, 1.0, (B, H, T, dk)).astype(np.float32)
+    S0 = r.standard_normal((B, H, dk, dv))
+    dO = r.standard_normal((B, H, T, dv)).astype(np.float32)
+    dSf = r.standard_normal((B, H, dk, dv)).astype(np.float32)
+    tq, tk, tv, tg = [torch.tensor(x, dtype=torch.float64, requires_grad=True) for x in (q, k, v, g)]
+    tS0 = torch.tensor(S0, requires_grad=True)
+    S, outs = tS0, []
+    for t in range(T):
+        S = tg[:, :, t, :, None] * S + tk[:, :, t, :, None] * tv[:, :, t, None, :]
+        outs.append(torch.einsum("bhc,bhcj->bhj", tq[:, :, t], S))
+    o = torch.stack(outs, dim=2)
+    loss = (o * torch.tensor(dO, dtype=torch.float64)).sum() + (S * torch.tensor(dSf, dtype=torch.float64)).sum()
+    loss.backward()
+    got = oracle.gla_backward(q, k, v, g, dO, S0, dSf)
+    for name, ref, val in zip(("dq", "dk", "dv", "dg", "dS0"), (tq, tk, tv, tg, tS0), got):
+        np.testing.assert_allclose(val, ref.grad.numpy(), rtol=1e-10, atol=1e-10, err_msg=name)
+
+
+def test_gla_backward_gate_identity():
+    """d(log g_r) = g_r dg_r equals the reverse cumulative sum over t >= r of q_t dq_t - k_t dk_t,
+    plus the final-state term sum_j dS_final[c, j] S_T[c, j] (pairs s < r <= t of the unrolled
+    form), an identity independent of how dg was computed."""
+    B, H, T, dk, dv = 2, 3, 130, 6, 5
+    r = _rng(33)
+    q, k = [r.standard_normal((B, H, T, dk)).astype(np.float32) for _ in range(2)]
+    v = r.standard_normal((B, H, T, dv)).astype(np.float32)
+    g = r.uniform(0.5, 1.0, (B, H, T, dk)).astype(np.float32)
+    S0 = r.standard_normal((B, H, dk, dv))
+    dO = r.standard_normal((B, H, T, dv)).astype(np.float32)
+    dSf = r.standard_normal((B, H, dk, dv)).astype(np.float32)
+    dq, dk_, _, dg, _ = oracle.gla_backward(q, k, v, g, dO, S0, dSf)
+    _, ST = oracle.gla_prefill(q, k, v, g, S0)
+    F = np.sum(dSf.astype(np.float64) * ST, axis=-1)              # [B,H,dk]
+    terms = q.astype(np.float64) * dq - k.astype(np.float64) * dk_  # [B,H,T,dk]
+    rev = np.flip(np.cumsum(np.flip(terms, axis=2), axis=2), axis=2) + F[:, :, None, :]
+    _close(g.astype(np.float64) * dg, rev, 1e-10)
