@@ -187,6 +187,25 @@ ROD_API int rod_gla_decode_step(const void* q, const void* k, const void* v, con
 ROD_API int rod_swska_prefill(const void* q, const void* k, const void* v, void* o, int B, int H,
                       int T, int dk, int dv, int window, float scale, int dtype, void* stream);
 
+/* ---- SW-SKA: backward (training path) -------------------------------------------------------- */
+/*
+ * Gradients of rod_swska_prefill for the loss gradient dO of every output row (same window
+ * and scale rules; CodeFuse article, SKA paragraph: the shared K gathers every head's part):
+ *   D_t = dO_t . o_t;  dS_tj = p_tj (dO_t . v_j - D_t);  dq_t = scale sum_j dS_tj k_j;
+ *   dk_j = scale sum_h sum_t dS_tj q_t;  dv_j = sum_t p_tj dO_t (per head).
+ *   q [B,H,T,dk], k [B,T,dk], v [B,H,T,dv], dO [B,H,T,dv]: dtype;  outputs dq, dk, dv in the
+ *   layouts of q, k, v and dtype;  workspace of rod_swska_backward_workspace_size bytes
+ *   (the row log-sum-exp and D_t, recomputed here from the inputs).
+ * Runs on CUDA cores with fp32 dot products (one warp per query row, then one per key).
+ * Errors: ROD_ERR_NULL, ROD_ERR_SHAPE (window < 1, dims unsupported, H > 64), ROD_ERR_ALIGN,
+ * ROD_ERR_DTYPE, ROD_ERR_WORKSPACE, ROD_ERR_CUDA. T = 0 or B*H = 0 is a no-op.
+ */
+ROD_API size_t rod_swska_backward_workspace_size(int B, int H, int T);
+ROD_API int rod_swska_backward(const void* q, const void* k, const void* v, const void* dO,
+                               void* dq, void* dk, void* dv, int B, int H, int T, int dk_dim,
+                               int dv_dim, int window, float scale, int dtype, void* workspace,
+                               size_t ws_bytes, void* stream);
+
 /* ---- SW-SKA: decode with a ring-buffer window cache --------------------------------------- */
 /*
  * One new token per sequence (SALA blog §3.3: a self-made circular buffer holds the rolling

@@ -47,9 +47,11 @@ class OracleLib:
                                                   ctypes.POINTER(ctypes.c_int32), i64, i64, i64p,
                                                   f64p, i64, i64, i64, i64, i64, ctypes.c_double,
                                                   ctypes.c_int]
+        lib.rodref_swska_backward.argtypes = [f32p, f32p, f32p, f32p, f64p, f64p, f64p, i64, i64,
+                                              i64, i64, i64, i64, ctypes.c_double, ctypes.c_int]
         lib.rodref_gla_backward.argtypes = [f32p, f32p, f32p, f32p, f64p, f32p, f32p, f64p, f64p,
                                             f64p, f64p, f64p, i64, i64, i64, i64, i64, ctypes.c_int]
-        for name in ("rodref_gla_backward", "rodref_gla_prefill", "rodref_gla_decode_step",
+        for name in ("rodref_gla_backward", "rodref_swska_backward", "rodref_gla_prefill", "rodref_gla_decode_step",
                      "rodref_swska_prefill",
                      "rodref_swska_decode", "rodref_swska_cache_fill", "rodref_swska_decode_paged"):
             getattr(lib, name).restype = ctypes.c_int
@@ -265,3 +267,19 @@ def gla_backward(q, k, v, g, dO, state0=None, dS_final=None, nthreads=None):
                                   nthreads or default_threads())
     _check(rc, "gla_backward")
     return dq, dk_, dv_, dg, dS0
+
+
+def swska_backward(q, k, v, dO, window, scale=None, nthreads=None):
+    """Gradients of SW-SKA prefill (rodref_swska_backward) for the loss gradient dO [B,H,T,dv].
+    Returns float64 (dq [B,H,T,dk], dk [B,T,dk] summed over heads, dv [B,H,T,dv])."""
+    q, k, v, dO = _f32(q), _f32(k), _f32(v), _f32(dO)
+    B, H, T, dk = q.shape
+    dv = v.shape[-1]
+    if scale is None or scale <= 0:
+        scale = 1.0 / np.sqrt(dk)
+    dq, dk_, dv_ = np.empty((B, H, T, dk)), np.empty((B, T, dk)), np.empty((B, H, T, dv))
+    rc = _L().rodref_swska_backward(_p32(q), _p32(k), _p32(v), _p32(dO), _p64(dq), _p64(dk_),
+                                    _p64(dv_), B, H, T, dk, dv, int(window), float(scale),
+                                    nthreads or default_threads())
+    _check(rc, "swska_backward")
+    return dq, dk_, dv_

@@ -401,6 +401,89 @@ int rodref_swska_decode(const float* q, const float* k_new, const float* v_new, 
     return run_units(ska_dec_unit, &a, N * H, nthreads);
 }
 
+/* Backward of SW-SKA prefill (training path; same attention as rodref_swska_prefill). For the
+ * loss gradient dO of every output row, per (b, h, t) with window J_t and p = softmax(s):
+ *   D_t = sum_j p_tj (dO_t . v_j)  (= dO_t . o_t),   dS_tj = p_tj (dO_t . v_j - D_t)
+ *   dq_t  = scale sum_j dS_tj k_j
+ *   dk_j  = scale sum_h sum_t dS_tj q_t      (one K shared by the heads: summed over them)
+ *   dv_j  = sum_t p_tj dO_t                  (per head)
+ * Units are (b, h) pairs; each writes its dq and dv and a private dk partial, and the partials
+ * are summed over heads afterwards. */
+typedef struct {
+    const float *q, *k, *v, *dO;
+    double *dq, *dkp, *dv;
+    int64_t H, T, dk, dv_, W;
+    double scale;
+} ska_bwd_args_t;
+
+static void ska_bwd_unit(const void* p, int64_t bh) {
+    const ska_bwd_args_t* a = (const ska_bwd_args_t*)p;
+    const int64_t H = a->H, T = a->T, dk = a->dk, dv = a->dv_, W = a->W, b = bh / H;
+    double* s = malloc((size_t)(W + 1) * sizeof(double));
+    double* pr = malloc((size_t)(W + 1) * sizeof(double));
+    double* dp = malloc((size_t)(W + 1) * sizeof(double));
+    double* dkp = a->dkp + bh * T * dk;
+    if (!s || !pr || !dp) { free(s); free(pr); free(dp); return; }
+    for (int64_t i = 0; i < T * dk; ++i) dkp[i] = 0.0;
+    for (int64_t i = 0; i < T * dv; ++i) a->dv[bh * T * dv + i] = 0.0;
+    for (int64_t t = 0; t < T; ++t) {
+        const int64_t j0 = t - W + 1 > 0 ? t - W + 1 : 0;
+        const float* qt = a->q + (bh * T + t) * dk;
+        const float* dot = a->dO + (bh * T + t) * dv;
+        double m = -INFINITY;
+        for (int64_t j = j0; j <= t; ++j) {
+            double acc = 0.0;
+            for (int64_t c = 0; c < dk; ++c) acc += (double)qt[c] * (double)a->k[(b * T + j) * dk + c];
+            s[j - j0] = a->scale * acc;
+            if (s[j - j0] > m) m = s[j - j0];
+        }
+        double l = 0.0;
+        for (int64_t j = j0; j <= t; ++j) { pr[j - j0] = exp(s[j - j0] - m); l += pr[j - j0]; }
+        double D = 0.0;
+        for (int64_t j = j0; j <= t; ++j) {
+            pr[j - j0] /= l;
+            double acc = 0.0;
+            for (int64_t i = 0; i < dv; ++i) acc += (double)dot[i] * (double)a->v[(bh * T + j) * dv + i];
+            dp[j - j0] = acc;
+            D += pr[j - j0] * acc;
+        }
+        double* dqt = a->dq + (bh * T + t) * dk;
+        for (int64_t c = 0; c < dk; ++c) dqt[c] = 0.0;
+        for (int64_t j = j0; j <= t; ++j) {
+            const double dS = pr[j - j0] * (dp[j - j0] - D);
+            for (int64_t c = 0; c < dk; ++c) {
+                dqt[c] += a->scale * dS * (double)a->k[(b * T + j) * dk + c];
+                dkp[j * dk + c] += a->scale * dS * (double)qt[c];
+            }
+            for (int64_t i = 0; i < dv; ++i) a->dv[(bh * T + j) * dv + i] += pr[j - j0] * (double)dot[i];
+        }
+    }
+    free(s);
+    free(pr);
+    free(dp);
+}
+
+/* q [B,H,T,dk], k [B,T,dk], v [B,H,T,dv], dO [B,H,T,dv] -> dq [B,H,T,dk], dk [B,T,dk],
+ * dv [B,H,T,dv] (float64). */
+int rodref_swska_backward(const float* q, const float* k, const float* v, const float* dO,
+                          double* dq, double* dk_out, double* dv_out, int64_t B, int64_t H,
+                          int64_t T, int64_t dk, int64_t dv, int64_t W, double scale, int nthreads) {
+    if (!q || !k || !v || !dO || !dq || !dk_out || !dv_out) return RODREF_EINVAL;
+    if (B < 0 || H < 1 || T < 0 || dk < 1 || dv < 1 || W < 1) return RODREF_EINVAL;
+    double* dkp = malloc((size_t)(B * H * T * dk + 1) * sizeof(double));
+    if (!dkp) return RODREF_EINVAL;
+    ska_bwd_args_t a = {q, k, v, dO, dq, dkp, dv_out, H, T, dk, dv, W, scale};
+    run_units(ska_bwd_unit, &a, B * H, nthreads);
+    for (int64_t b = 0; b < B; ++b)
+        for (int64_t i = 0; i < T * dk; ++i) {
+            double acc = 0.0;
+            for (int64_t h = 0; h < H; ++h) acc += dkp[(b * H + h) * T * dk + i];
+            dk_out[b * T * dk + i] = acc;
+        }
+    free(dkp);
+    return 0;
+}
+
 /* Decode over a paged window cache (SALA blog §3.3: paged KV cache in small blocks): the ring's
  * W slots are cut into pps pages of `page` slots; slot s of sequence n lives in physical page
  * t = table[n*pps + s/page] at row s mod page of the pools k_pool [P][page][dk] and

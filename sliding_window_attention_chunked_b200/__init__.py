@@ -9,6 +9,7 @@ the calls raise.
     gla_decode_step(q, k, v, g, state)              one fused recurrent decode step
     gla_backward(q, k, v, g, dO, state0, dstate_final)   gradients of the recurrence
     swska_prefill(q, k, v, window, scale=None)      sliding-window shared-key attention
+    swska_backward(q, k, v, dO, window)             gradients of the attention
     swska_decode(q, k_new, v_new, k_cache, v_cache, pos, window)   ring-buffer decode
     swska_cache_fill(k, v, k_cache, v_cache, window)   prefill -> decode ring-buffer hand-off
     swska_decode_paged(q, k_new, v_new, k_pool, v_pool, block_table, page_size, pos, window)
@@ -28,6 +29,7 @@ from ._binding import (  # noqa: F401
     launch_count,
     library_path,
     load_library,
+    swska_backward,
     swska_cache_fill,
     swska_decode,
     swska_decode_paged,

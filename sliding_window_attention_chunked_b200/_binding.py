@@ -73,6 +73,10 @@ def load_library() -> ctypes.CDLL:
     lib.rod_gla_backward_workspace_size.restype = sz
     lib.rod_gla_backward.argtypes = [vp] * 12 + [i] * 6 + [vp, sz, vp]
     lib.rod_gla_backward.restype = i
+    lib.rod_swska_backward_workspace_size.argtypes = [i, i, i]
+    lib.rod_swska_backward_workspace_size.restype = sz
+    lib.rod_swska_backward.argtypes = [vp] * 7 + [i] * 6 + [f, i, vp, sz, vp]
+    lib.rod_swska_backward.restype = i
     lib.rod_swska_cache_fill.restype = i
     _lib = lib
     return lib
@@ -328,3 +332,26 @@ def gla_backward(q, k, v, g, dO, state0=None, dstate_final=None, workspace=None,
                               _dtype_code(q), _ptr(workspace), workspace.numel(), _stream(stream))
     _raise_on("rod_gla_backward", st)
     return dq, dk_, dv_, dg, dS0
+
+
+def swska_backward(q, k, v, dO, window, scale=None, workspace=None, stream=None):
+    """Gradients of swska_prefill: q [B,H,T,dk], shared k [B,T,dk], v and dO [B,H,T,dv].
+    Returns (dq, dk, dv) in the layouts and dtype of q, k, v."""
+    _need(q, "q", None, 4)
+    _need(k, "k", q.dtype, 3)
+    _need(v, "v", q.dtype, 4)
+    _need(dO, "dO", q.dtype, 4)
+    B, H, T, dk = q.shape
+    dv = v.shape[-1]
+    if tuple(k.shape) != (B, T, dk) or tuple(v.shape[:3]) != (B, H, T) or tuple(dO.shape) != tuple(v.shape):
+        raise ValueError("shape mismatch")
+    lib = load_library()
+    need = lib.rod_swska_backward_workspace_size(B, H, T)
+    if workspace is None:
+        workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=q.device)
+    dq, dk_, dv_ = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    st = lib.rod_swska_backward(_ptr(q), _ptr(k), _ptr(v), _ptr(dO), _ptr(dq), _ptr(dk_), _ptr(dv_),
+                                B, H, T, dk, dv, int(window), float(scale or 0.0), _dtype_code(q),
+                                _ptr(workspace), workspace.numel(), _stream(stream))
+    _raise_on("rod_swska_backward", st)
+    return dq, dk_, dv_

@@ -81,6 +81,17 @@ struct GlaBackwardArgs {
     void* workspace;
 };
 size_t gla_backward_workspace_size(int B, int H, int T, int dk, int dv);
+
+// backward of SW-SKA prefill (CUDA cores): gradients of q, the shared k, and v
+struct SkaBackwardArgs {
+    const void *q, *k, *v, *dO;  // [B,H,T,dk], [B,T,dk], [B,H,T,dv], [B,H,T,dv]
+    void *dq, *dk, *dv;          // same layouts as q, k, v
+    int B, H, T, d_k, d_v, W;
+    float scale;                 // resolved (> 0)
+    void* workspace;             // 2 B H T floats: base-2 log-sum-exp and D per row
+};
+size_t swska_backward_workspace_size(int B, int H, int T);
+cudaError_t swska_backward_launch(const SkaBackwardArgs& a, bool bf16, cudaStream_t stream);
 cudaError_t gla_backward_launch(const GlaBackwardArgs& a, bool bf16, cudaStream_t stream);
 
 // SW-SKA prefill -> decode hand-off: the last W tokens' K / V rows into the ring buffers

@@ -180,6 +180,30 @@ int rod_gla_backward(const void* q, const void* k, const void* v, const float* g
     return from_cuda(rod::gla_backward_launch(a, dtype == ROD_BF16, s));
 }
 
+size_t rod_swska_backward_workspace_size(int B, int H, int T) {
+    if (B < 0 || H < 0 || T < 0) return 0;
+    return rod::swska_backward_workspace_size(B, H, T);
+}
+
+int rod_swska_backward(const void* q, const void* k, const void* v, const void* dO, void* dq, void* dk,
+                       void* dv, int B, int H, int T, int dk_dim, int dv_dim, int window, float scale,
+                       int dtype, void* workspace, size_t ws_bytes, void* stream) {
+    if (!dtype_ok(dtype)) return ROD_ERR_DTYPE;
+    if (B < 0 || H < 0 || T < 0 || H > 64 || window < 1 || !dim_ok(dk_dim) || !dim_ok(dv_dim))
+        return ROD_ERR_SHAPE;
+    if (!(scale == scale) || isinf(scale)) return ROD_ERR_SHAPE;
+    if ((int64_t)B * H == 0 || T == 0) return ROD_OK;
+    if (!q || !k || !v || !dO || !dq || !dk || !dv) return ROD_ERR_NULL;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(dO) || !aligned16(dq) ||
+        !aligned16(dk) || !aligned16(dv))
+        return ROD_ERR_ALIGN;
+    if (!workspace || ws_bytes < rod::swska_backward_workspace_size(B, H, T)) return ROD_ERR_WORKSPACE;
+    if (!aligned16(workspace)) return ROD_ERR_ALIGN;
+    rod::SkaBackwardArgs a{q, k, v, dO, dq, dk, dv, B, H, T, dk_dim, dv_dim, window,
+                           resolve_scale(scale, dk_dim), workspace};
+    return from_cuda(rod::swska_backward_launch(a, dtype == ROD_BF16, static_cast<cudaStream_t>(stream)));
+}
+
 int rod_swska_decode_paged(const void* q, const void* k_new, const void* v_new, void* k_pool,
                            void* v_pool, const int32_t* block_table, int page_size, int pages_per_seq,
                            const int64_t* pos, void* o, int N, int H, int dk, int dv, int window,

@@ -75,3 +75,28 @@ def test_gla_backward_empty_sequence_passes_the_final_gradient_through():
     _, _, _, _, dS0 = rod.gla_backward(z, z, z, z, z, torch.zeros(B, H, d, d, device=DEV), None)
     rod.check()
     assert torch.equal(dS0, torch.zeros_like(dSf))
+
+
+# ------------------------------------------------------------------------------------------
+# SW-SKA
+# ------------------------------------------------------------------------------------------
+
+
+def _ska_check(B, H, T, dk, dv, W, dtype, seed):
+    q, k, v = wl.swska_inputs(B, H, T, dk, dv, seed=seed, dtype=dtype)
+    dO = (torch.randn(B, H, T, dv, generator=torch.Generator().manual_seed(seed + 5)) * 0.5).to(q.dtype)
+    ref = oracle.swska_backward(q, k, v, dO, W)
+    got = rod.swska_backward(q.to(DEV), k.to(DEV), v.to(DEV), dO.to(DEV), W)
+    rod.check()
+    for name, a, b in zip(("dq", "dk", "dv"), got, ref):
+        compare(a, b, dtype, f"{name} B{B} H{H} T{T} dk{dk} dv{dv} W{W} {dtype}")
+
+
+@pytest.mark.parametrize("dk,dv,W", [(16, 32, 7), (32, 16, 64), (64, 64, 1), (128, 128, 40)])
+def test_swska_backward_fp32(dk, dv, W):
+    _ska_check(2, 3, 150, dk, dv, W, "fp32", seed=dk + dv + W)
+
+
+@pytest.mark.parametrize("T,W", [(1, 64), (200, 64), (300, 300), (257, 128)])
+def test_swska_backward_bf16(T, W):
+    _ska_check(1, 4, T, 128, 128, W, "bf16", seed=T + W)

@@ -5,7 +5,8 @@ textual substitution (a gate applied to the wrong channel, a decay that also hit
 term, the readout using k, an off-by-one window, a dropped scale or normaliser, a wrong
 ring-buffer slot, a hand-off that drops a token or numbers slots from the window start, a paged cache read
 without its table or written at the wrong row, a backward that weights the gate gradient
-with the updated state or decays the gradient state on the wrong channel), builds the copy with gcc and runs every pin against it. Each planted
+with the updated state or decays the gradient state on the wrong channel, an attention backward
+without the softmax row term or with the shared key's gradient from one head), builds the copy with gcc and runs every pin against it. Each planted
 mistake must make at least one pin fail; otherwise the pins are too weak to trust.
 """
 import inspect
@@ -45,6 +46,10 @@ MUTATIONS = {
                               "accg += dS[c * dv + j] * Sprev[DD + c * dv + j];"),
     "bwd_decay_wrong_channel": ("for (int64_t j = 0; j < dv; ++j) dS[c * dv + j] *= (double)a->g[tk + c];",
                                 "for (int64_t j = 0; j < dv; ++j) dS[c * dv + j] *= (double)a->g[tk + (c + 1) % dk];"),
+    "ska_bwd_drops_row_term": ("const double dS = pr[j - j0] * (dp[j - j0] - D);",
+                               "const double dS = pr[j - j0] * dp[j - j0];"),
+    "ska_bwd_shared_key_one_head": ("for (int64_t h = 0; h < H; ++h) acc += dkp[(b * H + h) * T * dk + i];",
+                                    "for (int64_t h = 0; h < 1; ++h) acc += dkp[(b * H + h) * T * dk + i];"),
     "paged_write_wrong_row": ("t = table[n * pps + s / page], r = s % page;\n            memcpy(k_pool",
                               "t = table[n * pps + s / page], r = (s + 1) % page;\n            memcpy(k_pool"),
 }

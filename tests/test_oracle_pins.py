@@ -451,3 +451,51 @@ def test_gla_backward_gate_identity():
     terms = q.astype(np.float64) * dq - k.astype(np.float64) * dk_  # [B,H,T,dk]
     rev = np.flip(np.cumsum(np.flip(terms, axis=2), axis=2), axis=2) + F[:, :, None, :]
     _close(g.astype(np.float64) * dg, rev, 1e-10)
+
+
+# ------------------------------------------------------------------------------------------
+# backward of SW-SKA
+# ------------------------------------------------------------------------------------------
+
+
+def test_swska_backward_finite_differences():
+    """Central differences of L = sum(o . dO) on a tiny case (step 2^-8 on inputs that are
+    multiples of 2^-8, so perturbed inputs are exact in fp32)."""
+    B, H, T, dk, dv, W = 1, 2, 6, 3, 2, 4
+    r = _rng(41)
+    grid = lambda shape: (np.round(r.uniform(-1, 1, shape) * 256) / 256).astype(np.float32)
+    q, k, v = grid((B, H, T, dk)), grid((B, T, dk)), grid((B, H, T, dv))
+    dO = r.standard_normal((B, H, T, dv)).astype(np.float32)
+    dq, dk_, dv_ = oracle.swska_backward(q, k, v, dO, W)
+    loss = lambda q_, k_, v_: float(np.sum(oracle.swska_prefill(q_, k_, v_, W) * dO))
+    h = 2.0 ** -8
+    for name, x, grad in (("q", q, dq), ("k", k, dk_), ("v", v, dv_)):
+        for idx in np.ndindex(x.shape):
+            xp, xm = x.copy(), x.copy()
+            xp[idx] += h
+            xm[idx] -= h
+            args = lambda xx: [xx if n == name else a for n, a in (("q", q), ("k", k), ("v", v))]
+            fd = (loss(*args(xp)) - loss(*args(xm))) / (2 * h)
+            assert abs(fd - grad[idx]) <= 2e-5 * max(1.0, abs(fd)), (name, idx, fd, grad[idx])
+
+
+@pytest.mark.parametrize("W", [1, 5, 40])
+def test_swska_backward_matches_torch_autograd(W):
+    """The same gradients from PyTorch autograd through float64 attention with the key
+    replicated over heads (its gradient is the sum of the replicas') and an explicit window
+    mask."""
+    torch = pytest.importorskip("torch")
+    B, H, T, dk, dv = 2, 3, 33, 6, 5
+    q, k, v = _ska_case(B=B, H=H, T=T, dk=dk, dv=dv, seed=42)
+    dO = _rng(43).standard_normal((B, H, T, dv)).astype(np.float32)
+    tq, tk, tv = [torch.tensor(x, dtype=torch.float64, requires_grad=True) for x in (q, k, v)]
+    t = torch.arange(T)
+    mask = (t[None, :] <= t[:, None]) & (t[None, :] > t[:, None] - W)
+    s = torch.einsum("bhtc,bjc->bhtj", tq, tk) / np.sqrt(dk)
+    s = s.masked_fill(~mask, float("-inf"))
+    o = torch.einsum("bhtj,bhjd->bhtd", torch.softmax(s, dim=-1), tv)
+    (o * torch.tensor(dO, dtype=torch.float64)).sum().backward()
+    dq, dk_, dv_ = oracle.swska_backward(q, k, v, dO, W)
+    np.testing.assert_allclose(dq, tq.grad.numpy(), rtol=1e-10, atol=1e-12)
+    np.testing.assert_allclose(dk_, tk.grad.numpy(), rtol=1e-10, atol=1e-12)
+    np.testing.assert_allclose(dv_, tv.grad.numpy(), rtol=1e-10, atol=1e-12)
