@@ -423,6 +423,9 @@ def run_gpu(args):
     if not args.no_generate:
         generate = run_generate(rod, torch, wl, dev, L, H, dk, W, seed_base, barrier, ranks_max,
                                 world)
+    backward = None
+    if not args.no_backward:
+        backward = run_backward(rod, torch, wl, dev, H, dk, W, seed_base, barrier, ranks_max, world)
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         cpu = oracle_stack_sample(d)
@@ -440,12 +443,67 @@ def run_gpu(args):
                    "parallelism": f"replicas x{world} (independent sequences, no collective)",
                    "l2": "inputs > L2 (55 GB per step), no flush needed"},
         "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": launches,
-        "clocks": clocks, "decode": decode, "generate": generate, "kernels": kernels,
+        "clocks": clocks, "decode": decode, "generate": generate, "backward": backward,
+        "kernels": kernels,
     }
     if rank == 0:
         print(json.dumps(line), flush=True)
     if world > 1:
         dist.destroy_process_group()
+
+
+def run_backward(rod, torch, wl, dev, H, d, W, seed_base, barrier, reduce_max, world):
+    """Training path: the backward of each mixer on its own configuration (CUDA cores, fp32
+    dot products), timed with CUDA events after a warm-up call. Roofline: fp32 FMA issue,
+    148 SMs x 128 FMA/clk x 2 FLOP x the max SM clock."""
+    peak = 148 * 128 * 2 * 1.965e9 / 1e12  # TFLOP/s
+    out = {"bound": "alu", "peak": round(peak, 1), "unit": "TFLOP/s",
+           "peak_source": "148 SMs x 128 fp32 FMA/clk x 2 x 1965 MHz (nominal, CUDA cores)"}
+
+    def timed(fn, iters):
+        fn()
+        barrier()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for _ in range(iters):
+            fn()
+        e1.record()
+        barrier()
+        rod.check()
+        return reduce_max(e0.elapsed_time(e1) / iters)
+
+    # recurrence: B4 H16 T4096, d 128 (the chunked-prefill workload); 13 dk dv FLOP per
+    # head-token (S_t, dq, dS, dk, dv, dg)
+    B, T = 4, 4096
+    q, k, v, g = wl.gla_inputs(B, H, T, d, d, dist="l2", seed=seed_base + 300, device=dev)
+    gen = torch.Generator(device=dev)
+    gen.manual_seed(seed_base + 301)
+    dO = (torch.randn(B, H, T, d, generator=gen, device=dev) * 0.2).to(q.dtype)
+    S0 = torch.zeros(B, H, d, d, device=dev)
+    dSf = torch.randn(B, H, d, d, generator=gen, device=dev) * 0.1
+    ws = torch.empty(rod.load_library().rod_gla_backward_workspace_size(B, H, T, d, d), dtype=torch.uint8,
+                     device=dev)
+    ms = timed(lambda: rod.gla_backward(q, k, v, g, dO, S0, dSf, workspace=ws), 3)
+    flop = 13.0 * d * d * B * H * T
+    out["gla_backward"] = {"workload": f"B{B} H{H} T{T} d{d} bf16", "ms": round(ms, 3),
+                           "tokens_per_s": round(B * T * world / (ms / 1e3), 1),
+                           "achieved": round(flop / (ms / 1e3) / 1e12, 3),
+                           "frac": round(flop / (ms / 1e3) / 1e12 / peak, 4)}
+    del q, k, v, g, dO, S0, dSf, ws
+    # SW-SKA: B1 H16 T8192, window W, d 128; 10 d FLOP per (query, key) pair (scores, dP, dq,
+    # dk, dv)
+    B, T = 1, 8192
+    q, k, v = wl.swska_inputs(B, H, T, d, d, seed=seed_base + 302, device=dev)
+    dO = (torch.randn(B, H, T, d, generator=gen, device=dev) * 0.5).to(q.dtype)
+    ms = timed(lambda: rod.swska_backward(q, k, v, dO, W), 2)
+    flop = 10.0 * d * swska_pairs(T, W) * B * H
+    out["swska_backward"] = {"workload": f"B{B} H{H} T{T} d{d} window {W} bf16", "ms": round(ms, 3),
+                             "tokens_per_s": round(B * T * world / (ms / 1e3), 1),
+                             "achieved": round(flop / (ms / 1e3) / 1e12, 3),
+                             "frac": round(flop / (ms / 1e3) / 1e12 / peak, 4)}
+    del q, k, v, dO
+    torch.cuda.empty_cache()
+    return out
 
 
 def run_generate(rod, torch, wl, dev, L, H, d, W, seed_base, barrier, reduce_max, world):
@@ -642,6 +700,7 @@ def main():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-generate", action="store_true")
+    ap.add_argument("--no-backward", action="store_true")
     ap.add_argument("--profile-case", choices=["ska_prefill", "gla_prefill", "ska_decode", "gla_decode"],
                     help="run one kernel family alone (for ncu captures) and exit")
     ap.add_argument("--profile-n", type=int, default=128, help="sequences for the decode cases")
