@@ -665,6 +665,15 @@ def run_profile_case(args):
             ws = torch.empty(max(rod.gla_prefill_workspace_size(B, H, T, dk, dv, C), 16),
                              dtype=torch.uint8, device=dev)
             fn = lambda: rod.gla_prefill(q, k, v, g, st.zero_(), o=out, chunk=C, workspace=ws)
+    elif case == "gla_backward":  # B4 H16 T4096 (the backward line of the bench)
+        q, k, v, g = wl.gla_inputs(4, H, 4096, dk, dv, dist="l2", seed=300, device=dev)
+        dO = (torch.randn(4, H, 4096, dv, device=dev) * 0.2).to(q.dtype)
+        S0 = torch.zeros(4, H, dk, dv, device=dev)
+        fn = lambda: rod.gla_backward(q, k, v, g, dO, S0, None)
+    elif case == "ska_backward":  # B1 H16 T8192, window W
+        q, k, v = wl.swska_inputs(1, H, 8192, dk, dv, seed=302, device=dev)
+        dO = (torch.randn(1, H, 8192, dv, device=dev) * 0.5).to(q.dtype)
+        fn = lambda: rod.swska_backward(q, k, v, dO, W)
     else:
         N, Wd = args.profile_n, wl.WORKLOADS["decode_n256"].dims["window"]
         dd = wl.decode_inputs(N, H, dk, dv, Wd, seed=77, device=dev)
@@ -672,6 +681,14 @@ def run_profile_case(args):
         if case == "ska_decode":
             fn = lambda: rod.swska_decode(dd["sq"], dd["k_new"], dd["v_new"], dd["k_cache"],
                                           dd["v_cache"], dd["pos"], Wd, o=o)
+        elif case == "ska_decode_paged":  # pages of 64 slots, shuffled table
+            page, pps = 64, Wd // 64
+            k_pool = dd["k_cache"].reshape(N * pps, page, dk)
+            v_pool = (dd["v_cache"].reshape(N, H, pps, page, dv).permute(0, 2, 1, 3, 4)
+                      .reshape(N * pps, H, page, dv).contiguous())
+            table = torch.randperm(N * pps, device=dev).to(torch.int32).reshape(N, pps)
+            fn = lambda: rod.swska_decode_paged(dd["sq"], dd["k_new"], dd["v_new"], k_pool, v_pool,
+                                                table, page, dd["pos"], Wd, o=o)
         else:
             fn = lambda: rod.gla_decode_step(dd["q"], dd["k"], dd["v"], dd["g"], dd["state"], o=o)
     for _ in range(args.warmup):
@@ -687,7 +704,7 @@ def run_profile_case(args):
         times.append(e0.elapsed_time(e1))
     rod.check()
     print(json.dumps({"profile_case": case, "launch_ms": [round(t, 4) for t in times],
-                      "n": args.profile_n if case.endswith("decode") else None}), flush=True)
+                      "n": args.profile_n if "decode" in case else None}), flush=True)
 
 
 def main():
@@ -701,7 +718,8 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-generate", action="store_true")
     ap.add_argument("--no-backward", action="store_true")
-    ap.add_argument("--profile-case", choices=["ska_prefill", "gla_prefill", "ska_decode", "gla_decode"],
+    ap.add_argument("--profile-case", choices=["ska_prefill", "gla_prefill", "ska_decode", "gla_decode",
+                                               "ska_decode_paged", "gla_backward", "ska_backward"],
                     help="run one kernel family alone (for ncu captures) and exit")
     ap.add_argument("--profile-n", type=int, default=128, help="sequences for the decode cases")
     args = ap.parse_args()
