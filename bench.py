@@ -453,12 +453,14 @@ def run_gpu(args):
 
 
 def run_backward(rod, torch, wl, dev, H, d, W, seed_base, barrier, reduce_max, world):
-    """Training path: the backward of each mixer on its own configuration (CUDA cores, fp32
-    dot products), timed with CUDA events after a warm-up call. Roofline: fp32 FMA issue,
-    148 SMs x 128 FMA/clk x 2 FLOP x the max SM clock."""
-    peak = 148 * 128 * 2 * 1.965e9 / 1e12  # TFLOP/s
-    out = {"bound": "alu", "peak": round(peak, 1), "unit": "TFLOP/s",
-           "peak_source": "148 SMs x 128 fp32 FMA/clk x 2 x 1965 MHz (nominal, CUDA cores)"}
+    """Training path: the backward of each mixer on its own configuration, timed with CUDA
+    events after a warm-up call. The recurrence's backward runs on CUDA cores (roofline: fp32
+    FMA issue, 148 SMs x 128 FMA/clk x 2 FLOP x the max SM clock); the SW-SKA backward runs on
+    the tensor cores (roofline: the measured dense bf16 peak, burst figure: timed alone)."""
+    alu_peak = 148 * 128 * 2 * 1.965e9 / 1e12  # TFLOP/s
+    peaks, peaks_src = load_peaks()
+    tc_peak = peaks.get("bf16_tflops")
+    out = {}
 
     def timed(fn, iters):
         fn()
@@ -487,20 +489,28 @@ def run_backward(rod, torch, wl, dev, H, d, W, seed_base, barrier, reduce_max, w
     flop = 13.0 * d * d * B * H * T
     out["gla_backward"] = {"workload": f"B{B} H{H} T{T} d{d} bf16", "ms": round(ms, 3),
                            "tokens_per_s": round(B * T * world / (ms / 1e3), 1),
-                           "achieved": round(flop / (ms / 1e3) / 1e12, 3),
-                           "frac": round(flop / (ms / 1e3) / 1e12 / peak, 4)}
+                           "bound": "alu", "achieved": round(flop / (ms / 1e3) / 1e12, 3),
+                           "peak": round(alu_peak, 1), "unit": "TFLOP/s",
+                           "frac": round(flop / (ms / 1e3) / 1e12 / alu_peak, 4),
+                           "peak_source": "148 SMs x 128 fp32 FMA/clk x 2 x 1965 MHz (nominal, CUDA cores)"}
     del q, k, v, g, dO, S0, dSf, ws
-    # SW-SKA: B1 H16 T8192, window W, d 128; 10 d FLOP per (query, key) pair (scores, dP, dq,
-    # dk, dv)
+    # SW-SKA: B1 H16 T8192, window W, d 128; algorithmic work 10 d FLOP per (query, key, head)
+    # pair inside the window: the five products S = Q K^T, dP = dO V^T, dV = P^T dO,
+    # dK = dS^T Q, dQ = dS K (the kernels recompute S and dP, 18 d FLOP per pair in all)
     B, T = 1, 8192
     q, k, v = wl.swska_inputs(B, H, T, d, d, seed=seed_base + 302, device=dev)
     dO = (torch.randn(B, H, T, d, generator=gen, device=dev) * 0.5).to(q.dtype)
-    ms = timed(lambda: rod.swska_backward(q, k, v, dO, W), 2)
+    ws = torch.empty(rod.load_library().rod_swska_backward_workspace_size(B, H, T), dtype=torch.uint8,
+                     device=dev)
+    ms = timed(lambda: rod.swska_backward(q, k, v, dO, W, workspace=ws), 10)
     flop = 10.0 * d * swska_pairs(T, W) * B * H
     out["swska_backward"] = {"workload": f"B{B} H{H} T{T} d{d} window {W} bf16", "ms": round(ms, 3),
                              "tokens_per_s": round(B * T * world / (ms / 1e3), 1),
-                             "achieved": round(flop / (ms / 1e3) / 1e12, 3),
-                             "frac": round(flop / (ms / 1e3) / 1e12 / peak, 4)}
+                             "bound": "tensor", "achieved": round(flop / (ms / 1e3) / 1e12, 1),
+                             "peak": tc_peak, "unit": "TFLOP/s",
+                             "frac": round(flop / (ms / 1e3) / 1e12 / tc_peak, 4),
+                             "peak_source": f"{peaks_src} bf16_tflops (burst: timed alone)",
+                             "executed_flop_per_pair": 18 * d}
     del q, k, v, dO
     torch.cuda.empty_cache()
     return out

@@ -82,16 +82,22 @@ struct GlaBackwardArgs {
 };
 size_t gla_backward_workspace_size(int B, int H, int T, int dk, int dv);
 
-// backward of SW-SKA prefill (CUDA cores): gradients of q, the shared k, and v
+// backward of SW-SKA prefill: gradients of q, the shared k, and v (tensor cores for bf16 with
+// head dim 128 and T >= 128, CUDA cores otherwise)
 struct SkaBackwardArgs {
     const void *q, *k, *v, *dO;  // [B,H,T,dk], [B,T,dk], [B,H,T,dv], [B,H,T,dv]
     void *dq, *dk, *dv;          // same layouts as q, k, v
     int B, H, T, d_k, d_v, W;
     float scale;                 // resolved (> 0)
-    void* workspace;             // 2 B H T floats: base-2 log-sum-exp and D per row
+    void* workspace;             // swska_backward_workspace_size bytes, 16-byte aligned
 };
 size_t swska_backward_workspace_size(int B, int H, int T);
 cudaError_t swska_backward_launch(const SkaBackwardArgs& a, bool bf16, cudaStream_t stream);
+size_t swska_backward_tc_workspace_size(int B, int H, int T);
+bool swska_backward_tc_supported(int H, int T, int dk, int dv);
+int swska_backward_tc_groups(int B, int H, int T);
+cudaError_t swska_backward_tc_launch(const SkaBackwardArgs& a, cudaStream_t stream);
+unsigned swska_backward_tc_take_timeout_flag();
 cudaError_t gla_backward_launch(const GlaBackwardArgs& a, bool bf16, cudaStream_t stream);
 
 // SW-SKA prefill -> decode hand-off: the last W tokens' K / V rows into the ring buffers

@@ -59,7 +59,8 @@ int rod_check(void* stream) {
     const unsigned flags = rod::swska_decode_take_timeout_flag() |
                            rod::swska_decode_warp_take_timeout_flag() |
                            rod::swska_prefill_tc_take_timeout_flag() |
-                           rod::gla_prefill_tc_take_timeout_flag();
+                           rod::gla_prefill_tc_take_timeout_flag() |
+                           rod::swska_backward_tc_take_timeout_flag();
     if (flags) return ROD_ERR_TIMEOUT;
     return from_cuda(cudaGetLastError());
 }

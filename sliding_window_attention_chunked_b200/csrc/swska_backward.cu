@@ -13,7 +13,8 @@
 //   2. one warp per key position (b, j): for every head, the queries t in [j, j+W-1] that see
 //      it give dv_j of that head and their share of dk_j, which is complete when the warp has
 //      gone through all heads (no atomics).
-// This is the correctness-first form of the training path (every dot product in fp32).
+// These kernels serve fp32 inputs and head dims other than 128 (every dot product in fp32);
+// bf16 with head dim 128 runs on the tensor cores (swska_backward_tc.cu).
 #include <math.h>
 
 #include "common.cuh"
@@ -198,11 +199,13 @@ cudaError_t launch_nk(const SkaBackwardArgs& a, cudaStream_t s) {
 }  // namespace
 
 size_t swska_backward_workspace_size(int B, int H, int T) {
-    return (size_t)2 * B * H * T * sizeof(float);
+    // the tensor-core path's need covers the 2 B H T floats used here
+    return swska_backward_tc_workspace_size(B, H, T);
 }
 
 cudaError_t swska_backward_launch(const SkaBackwardArgs& a, bool bf16, cudaStream_t stream) {
     if ((int64_t)a.B * a.H == 0 || a.T == 0) return cudaSuccess;
+    if (bf16 && swska_backward_tc_supported(a.H, a.T, a.d_k, a.d_v)) return swska_backward_tc_launch(a, stream);
     return bf16 ? launch_nk<__nv_bfloat16>(a, stream) : launch_nk<float>(a, stream);
 }
 

@@ -1,0 +1,838 @@
+// swska_backward_tc.cu -- backward of SW-SKA prefill on the 5th-generation tensor cores
+// (tcgen05 MMAs with bf16 operands and fp32 accumulators in tensor memory), head dim 128.
+//
+// Forward (CodeFuse Rodimus* article, Fig. 4 / SKA paragraph: one K shared by all heads,
+// per-head V; setup blog §3: a window of the most recent W tokens):
+//   s_tj = scale q_t . k_j for j in [t-W+1, t],  p_t = softmax(s_t),  o_t = sum_j p_tj v_j.
+// For the loss gradient dO of every output row, with dP_tj = dO_t . v_j:
+//   D_t = sum_j p_tj dP_tj (= dO_t . o_t),   dS_tj = p_tj (dP_tj - D_t),
+//   dq_t = scale sum_j dS_tj k_j,   dv_j = sum_t p_tj dO_t (per head),
+//   dk_j = scale sum_h sum_t dS_tj q_t   (the shared key gathers every head's share).
+//
+// Three launches:
+//  1. Query tiles: one CTA per 128 queries of one head. A first sweep over the window's key
+//     tiles computes S = Q K^T and dP = dO V^T and keeps, per query row, the running maximum,
+//     the normaliser and D (online, base 2). The row's negated base-2 log-sum-exp and D are
+//     stored for launch 2 (-inf and 0 for rows past the end of the sequence). A second sweep recomputes S
+//     and dP, forms dS in bf16 in tensor memory and accumulates dQ += dS K there.
+//  2. Key tiles: one CTA per 128 keys and group of heads. For every head of the group and every
+//     query tile that sees the key tile: S^T = K Q^T and dP^T = V dO^T; P^T and dS^T (from the
+//     stored statistics) are written to tensor memory in bf16 and feed dV += P^T dO and
+//     dK += dS^T Q. dV is complete per head; dK is a partial per head group, stored in fp32.
+//  3. dk = scale * (sum of the groups' partials), summed in group order (deterministic).
+// In launches 1 and 2 each 128-column score tile is split into two halves of 64 columns, one
+// per softmax warpgroup, each with its own MMAs and barriers: one half's exponentials run
+// while the tensor core works on the other half. Warp roles (320 threads):
+//   warps 0-3 / 4-7  softmax warpgroups of column halves 0 / 1 (thread = TMEM lane = tile row)
+//   warp 8           TMA producer
+//   warp 9           TMEM allocator and the single MMA-issuing thread
+// Operands are staged by TMA in 128-byte-swizzled boxes; the P and dS operands of the
+// gradient MMAs are read from tensor memory (the A operand of a TS-form MMA). Every wait is
+// bounded; a timeout makes all roles stop, drain their copies and MMAs, and raise a flag.
+#include <cuda.h>
+#include <math.h>
+
+#include "common.cuh"
+#include "kernels.h"
+#include "tc.cuh"
+
+namespace rod {
+namespace {
+
+__device__ unsigned int g_ska_bwd_tc_timeout = 0;
+
+constexpr int TILE = 128;                   // queries or keys per tile
+constexpr int HD = 128;                     // head dim (dk = dv)
+constexpr int HALF = 64;                    // score columns per softmax warpgroup
+constexpr int TILE_BYTES = TILE * HD * 2;   // 32 KB: one 128 x 128 bf16 tile
+constexpr int BOX_BYTES = TILE_BYTES / 2;   // one TMA box: 128 rows x 64 columns
+constexpr int HALF_ROWS = HALF * 128;       // byte offset of row 64 inside a box (8 KB)
+constexpr int NTHREADS = 320;
+constexpr float kLog2e = 1.4426950408889634f;
+
+__device__ __forceinline__ bool wait_bar(uint64_t* bar, uint32_t parity, volatile int* abort_flag) {
+    for (uint32_t i = 1;; ++i) {
+        if (mbar_try_wait(bar, parity)) return true;
+        if ((i & 255u) == 0) {
+            if (*abort_flag) return false;
+            if (i >= kWaitLimit) {
+                *abort_flag = 1;
+                atomicExch(&g_ska_bwd_tc_timeout, 1u);
+                return false;
+            }
+        }
+    }
+}
+
+__device__ __forceinline__ unsigned char* align1024(unsigned char* p) {
+    return reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(p) + 1023) & ~uintptr_t(1023));
+}
+
+// Descriptor low words. K-major: K runs along the 128-byte rows (two boxes for K = 128);
+// MN-major: K runs down the rows, N across the two boxes (LBO = one box).
+__device__ __forceinline__ uint32_t lo_kmajor(uint32_t addr) {
+    return tc::desc_lo(tc::sdesc_sw128(addr, 16, 1024));
+}
+__device__ __forceinline__ uint32_t lo_mnmajor(uint32_t addr) {
+    return tc::desc_lo(tc::sdesc_sw128(addr, BOX_BYTES, 1024));
+}
+// offset (16-byte units) of K step k (16 elements) in a K-major tile of K = 128
+__device__ __forceinline__ uint32_t kstep(int k) { return (uint32_t)(((k / 4) * BOX_BYTES + (k % 4) * 32) >> 4); }
+// offset of K step k (16 rows) in an MN-major tile
+__device__ __forceinline__ uint32_t mnstep(int k) { return (uint32_t)((2048 * k) >> 4); }
+
+// two-wide fp32 arithmetic (one instruction for both lanes of the pair)
+__device__ __forceinline__ float2 f2fma(float2 a, float2 b, float2 c) {
+    float2 d;
+    asm("{\n\t.reg .b64 ra, rb, rc, rd;\n\tmov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\t"
+        "mov.b64 rc, {%6, %7};\n\tfma.rn.f32x2 rd, ra, rb, rc;\n\tmov.b64 {%0, %1}, rd;\n\t}"
+        : "=f"(d.x), "=f"(d.y) : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y), "f"(c.x), "f"(c.y));
+    return d;
+}
+__device__ __forceinline__ float2 f2add(float2 a, float2 b) {
+    float2 d;
+    asm("{\n\t.reg .b64 ra, rb, rd;\n\tmov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\t"
+        "add.rn.f32x2 rd, ra, rb;\n\tmov.b64 {%0, %1}, rd;\n\t}"
+        : "=f"(d.x), "=f"(d.y) : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
+    return d;
+}
+__device__ __forceinline__ float2 f2sub(float2 a, float2 b) {
+    float2 d;
+    asm("{\n\t.reg .b64 ra, rb, rd;\n\tmov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\t"
+        "sub.rn.f32x2 rd, ra, rb;\n\tmov.b64 {%0, %1}, rd;\n\t}"
+        : "=f"(d.x), "=f"(d.y) : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
+    return d;
+}
+__device__ __forceinline__ float2 f2mul(float2 a, float2 b) {
+    float2 d;
+    asm("{\n\t.reg .b64 ra, rb, rd;\n\tmov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\t"
+        "mul.rn.f32x2 rd, ra, rb;\n\tmov.b64 {%0, %1}, rd;\n\t}"
+        : "=f"(d.x), "=f"(d.y) : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
+    return d;
+}
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+    float d;
+    asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+    return d;
+}
+__device__ __forceinline__ float2 raw2(const uint32_t* r, int e) {
+    return make_float2(__uint_as_float(r[e]), __uint_as_float(r[e + 1]));
+}
+__device__ __forceinline__ float2 ex2x2(float2 x) { return make_float2(tc::ex2(x.x), tc::ex2(x.y)); }
+
+// scores outside the window [lo, hi] (column indices of this 32-column chunk) -> -inf
+__device__ __forceinline__ void mask_chunk(uint32_t* s, int c, int lo, int hi) {
+#pragma unroll
+    for (int e = 0; e < 32; ++e) {
+        const int col = 32 * c + e;
+        if (col < lo || col > hi) s[e] = 0xff800000u;
+    }
+}
+// maximum of 32 raw scores: four independent chains of three-input maxima
+__device__ __forceinline__ float max32(const uint32_t* s) {
+    float m4[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        float m = fmax3(__uint_as_float(s[i]), __uint_as_float(s[i + 4]), __uint_as_float(s[i + 8]));
+        m = fmax3(m, __uint_as_float(s[i + 12]), __uint_as_float(s[i + 16]));
+        m = fmax3(m, __uint_as_float(s[i + 20]), __uint_as_float(s[i + 24]));
+        m4[i] = fmaxf(m, __uint_as_float(s[i + 28]));
+    }
+    return fmaxf(fmax3(m4[0], m4[1], m4[2]), m4[3]);
+}
+
+// ============================================================================================
+// Launch 1: query tiles (row statistics, then dQ)
+// ============================================================================================
+namespace qa {
+constexpr int NSLOT = 5;                            // ring of K / V tiles
+constexpr int OFF_Q = 0;
+constexpr int OFF_DO = TILE_BYTES;
+constexpr int OFF_RING = 2 * TILE_BYTES;
+constexpr int OFF_BAR = OFF_RING + NSLOT * TILE_BYTES;
+constexpr int NBAR = 2 * NSLOT + 9;  // full, empty, qfull, sfull[2], sfree[2], done, drain, xch[2]
+constexpr int OFF_PART = OFF_BAR + 8 * NBAR;        // float [3][128]: statistics exchange
+constexpr int OFF_MISC = OFF_PART + 3 * TILE * 4;
+constexpr int SMEM = OFF_MISC + 16 + 1024;
+static_assert(SMEM <= 232448, "shared memory");
+}  // namespace qa
+
+__global__ void __launch_bounds__(NTHREADS, 1)
+ska_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_do,
+                  const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
+                  __nv_bfloat16* __restrict__ dq, float* __restrict__ nlse2, float* __restrict__ dbuf,
+                  int T, int Tpad, int H, int W, float scale_log2, float scale, int n_qtiles) {
+    using namespace qa;
+    extern __shared__ unsigned char smem_raw[];
+    unsigned char* smem = align1024(smem_raw);
+    const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+    const int qt = n_qtiles - 1 - (int)blockIdx.x;  // full-window tiles first
+    const int h = blockIdx.y, b = blockIdx.z;
+    const int bh = b * H + h;
+    const int t0 = qt * TILE;
+    const int kt_lo = (t0 - W + 1 > 0 ? t0 - W + 1 : 0) / TILE;
+    const int n_it = qt - kt_lo + 1;  // key tiles of the window
+    const int U = 2 * n_it;           // tiles over both sweeps
+
+    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + OFF_BAR);
+    uint64_t* full = bars;
+    uint64_t* empty = bars + NSLOT;
+    uint64_t* qfull = bars + 2 * NSLOT;
+    uint64_t* sfull = qfull + 1;
+    uint64_t* sfree = sfull + 2;
+    uint64_t* done = sfree + 2;
+    uint64_t* drain = done + 1;
+    uint64_t* xch = drain + 1;  // statistics exchange between the halves (bounded waits)
+    float* part = reinterpret_cast<float*>(smem + OFF_PART);
+    uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + OFF_MISC);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + OFF_MISC + 4);
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < NSLOT; ++s) {
+            mbar_init(&full[s], 1);
+            mbar_init(&empty[s], 1);
+        }
+        mbar_init(qfull, 1);
+        for (int w = 0; w < 2; ++w) {
+            mbar_init(&sfull[w], 1);
+            mbar_init(&sfree[w], 128);
+        }
+        mbar_init(done, 1);
+        mbar_init(drain, 1);
+        mbar_init(&xch[0], 128);
+        mbar_init(&xch[1], 128);
+        *abort_flag = 0;
+        fence_mbar_init();
+    }
+    if (warp == 9) {
+        tc::tmem_alloc(tmem_holder, 512);
+        tc::tmem_relinquish();
+    }
+    tc::fence_before_sync();
+    __syncthreads();
+    tc::fence_after_sync();
+    const uint32_t tmem = *tmem_holder;
+    // TMEM columns: S [0,128) | dP [128,256) | dQ [256,384); half w of S / dP at +64 w
+
+    if (warp == 8) {
+        // ------------------------------- TMA producer -------------------------------
+        if (lane == 0) {
+            tc::tma_prefetch_desc(&tm_q);
+            tc::tma_prefetch_desc(&tm_do);
+            tc::tma_prefetch_desc(&tm_k);
+            tc::tma_prefetch_desc(&tm_v);
+            mbar_arrive_expect_tx(qfull, 2 * TILE_BYTES);
+            for (int half = 0; half < 2; ++half) {
+                tc::tma_load_3d(smem + OFF_Q + half * BOX_BYTES, &tm_q, half * 64, t0, bh, qfull);
+                tc::tma_load_3d(smem + OFF_DO + half * BOX_BYTES, &tm_do, half * 64, t0, bh, qfull);
+            }
+            // load L: tile u = L / 2 of the two sweeps, K when L is even, V when odd
+            int L = 0;
+            for (; L < 2 * U; ++L) {
+                const int slot = L % NSLOT, use = L / NSLOT;
+                if (use > 0 && !wait_bar(&empty[slot], (uint32_t)((use - 1) & 1), abort_flag)) break;
+                const int key0 = (kt_lo + (L / 2) % n_it) * TILE;
+                unsigned char* dst = smem + OFF_RING + slot * TILE_BYTES;
+                mbar_arrive_expect_tx(&full[slot], TILE_BYTES);
+                for (int half = 0; half < 2; ++half) {
+                    if (L % 2 == 0)
+                        tc::tma_load_3d(dst + half * BOX_BYTES, &tm_k, half * 64, key0, b, &full[slot]);
+                    else
+                        tc::tma_load_3d(dst + half * BOX_BYTES, &tm_v, half * 64, key0, bh, &full[slot]);
+                }
+            }
+            // every copy started here has landed before the CTA can leave
+            mbar_wait_bounded(qfull, 0, kWaitLimit);
+            for (int Li = (L > NSLOT ? L - NSLOT : 0); Li < L; ++Li)
+                mbar_wait_bounded(&full[Li % NSLOT], (uint32_t)((Li / NSLOT) & 1), kWaitLimit);
+        }
+    } else if (warp == 9) {
+        // ------------------------------- MMA issuer -------------------------------
+        if (lane == 0) {
+            const uint32_t idesc_s = tc::idesc_bf16_f32(TILE, HALF, 0, 0);  // S half, both K-major
+            const uint32_t idesc_g = tc::idesc_bf16_f32(TILE, HD, 0, 1);    // dQ += dS K, K MN-major
+            const uint32_t d_hi = tc::desc_hi(tc::sdesc_sw128(0, 16, 1024));
+            const uint32_t q_lo = lo_kmajor(smem_u32(smem + OFF_Q));
+            const uint32_t do_lo = lo_kmajor(smem_u32(smem + OFF_DO));
+            auto ring = [&](int L) { return smem_u32(smem + OFF_RING + (L % NSLOT) * TILE_BYTES); };
+            bool ok = true;
+            auto acquire = [&](int L) {
+                ok = ok && wait_bar(&full[L % NSLOT], (uint32_t)((L / NSLOT) & 1), abort_flag);
+                tc::fence_after_sync();
+                return ok;
+            };
+            // S_w = Q K[64w, 64w+64)^T and dP_w = dO V[64w, 64w+64)^T of tile u
+            auto issue_sdp = [&](int w, int u) {
+                const uint32_t k_lo = lo_kmajor(ring(2 * u) + w * HALF_ROWS);
+                const uint32_t v_lo = lo_kmajor(ring(2 * u + 1) + w * HALF_ROWS);
+#pragma unroll
+                for (int k = 0; k < HD / 16; ++k)
+                    tc::mma_ss_lh(tmem + 64u * w, q_lo + kstep(k), d_hi, k_lo + kstep(k), d_hi, idesc_s, k > 0);
+#pragma unroll
+                for (int k = 0; k < HD / 16; ++k)
+                    tc::mma_ss_lh(tmem + 128u + 64u * w, do_lo + kstep(k), d_hi, v_lo + kstep(k), d_hi, idesc_s, k > 0);
+            };
+            // dQ += dS_w K[64w, 64w+64), dS_w packed in the first 32 columns of S half w
+            auto issue_dq = [&](int w, int u, bool first) {
+                const uint32_t k_lo = lo_mnmajor(ring(2 * u) + w * HALF_ROWS);
+#pragma unroll
+                for (int k = 0; k < HALF / 16; ++k)
+                    tc::mma_ts_lh(tmem + 256u, tmem + 64u * w + 8u * k, k_lo + mnstep(k), d_hi, idesc_g,
+                                  (first && k == 0) ? 0u : 1u);
+            };
+            ok = wait_bar(qfull, 0, abort_flag);
+            tc::fence_after_sync();
+            if (ok && acquire(0) && acquire(1)) {
+                issue_sdp(0, 0);
+                tc::mma_commit(&sfull[0]);
+                issue_sdp(1, 0);
+                tc::mma_commit(&sfull[1]);
+                tc::mma_commit(&empty[0]);  // tile 0 belongs to the first sweep: K and V are done
+                tc::mma_commit(&empty[1]);
+                for (int u = 0; u < U && ok; ++u) {
+                    const bool sweep2 = u >= n_it;
+                    for (int w = 0; w < 2; ++w) {
+                        if (!wait_bar(&sfree[w], (uint32_t)(u & 1), abort_flag)) { ok = false; break; }
+                        tc::fence_after_sync();
+                        if (sweep2) {
+                            issue_dq(w, u, u == n_it && w == 0);
+                            if (w == 1) tc::mma_commit(&empty[(2 * u) % NSLOT]);  // K of tile u
+                        }
+                        if (u + 1 < U) {
+                            if (w == 0 && !(acquire(2 * u + 2) && acquire(2 * u + 3))) break;
+                            issue_sdp(w, u + 1);
+                            tc::mma_commit(&sfull[w]);
+                            if (w == 1) {
+                                if (u + 1 < n_it) tc::mma_commit(&empty[(2 * u + 2) % NSLOT]);
+                                tc::mma_commit(&empty[(2 * u + 3) % NSLOT]);  // V of tile u + 1
+                            }
+                        }
+                    }
+                }
+                if (ok) tc::mma_commit(done);
+            }
+            // every MMA this thread issued has completed before TMEM is released
+            tc::mma_commit(drain);
+            mbar_wait_bounded(drain, 0, kWaitLimit);
+        }
+    } else {
+        // ------------------------------- softmax warpgroups -------------------------------
+        const int w = warp / 4;                    // column half
+        const int row = threadIdx.x % 128;         // query row == TMEM lane
+        const uint32_t lane_base = (uint32_t)(32 * (warp % 4)) << 16;
+        const uint32_t tS = tmem + lane_base + 64u * w;
+        const uint32_t tP = tS + 128u;
+        const uint32_t tQ = tmem + lane_base + 256u + 64u * w;
+        const int t = t0 + row;
+        float m = -INFINITY, l = 0.f, Dacc = 0.f;  // first sweep, over this half's keys
+        float L2 = 0.f, Drow = 0.f;                 // the row's statistics for the second sweep
+        bool ok = true;
+        for (int u = 0; u < U; ++u) {
+            if (!wait_bar(&sfull[w], (uint32_t)(u & 1), abort_flag)) { ok = false; break; }
+            tc::fence_after_sync();
+            const int key0 = (kt_lo + u % n_it) * TILE + HALF * w;  // first key of this half
+            const bool full_tile = key0 >= t0 + TILE - W && key0 + HALF - 1 <= t0;
+            const int lo = t - W + 1 - key0, hi = t - key0;           // valid columns [lo, hi]
+            const float2 sl2 = make_float2(scale_log2, scale_log2);
+            if (u < n_it) {
+#pragma unroll
+                for (int c = 0; c < 2; ++c) {
+                    uint32_t s[32], dp[32];
+                    tc::tmem_ld32(tS + 32u * c, s);
+                    tc::tmem_ld32(tP + 32u * c, dp);
+                    tc::tmem_wait_ld();
+                    if (!full_tile) mask_chunk(s, c, lo, hi);
+                    // online update: the running maximum moves to the chunk's maximum if larger
+                    const float mn = fmaxf(m, max32(s) * scale_log2);
+                    const float alpha = mn == -INFINITY ? 1.f : tc::ex2(m - mn);  // 0 when m = -inf
+                    l *= alpha;
+                    Dacc *= alpha;
+                    m = mn;
+                    const float mu = m == -INFINITY ? 0.f : m;  // nothing visible yet: p = 0
+                    const float2 nm2 = make_float2(-mu, -mu);
+                    float2 l4[4] = {{0.f, 0.f}, {0.f, 0.f}, {0.f, 0.f}, {0.f, 0.f}};
+                    float2 d4[4] = {{0.f, 0.f}, {0.f, 0.f}, {0.f, 0.f}, {0.f, 0.f}};
+#pragma unroll
+                    for (int i = 0; i < 16; ++i) {
+                        const float2 p2 = ex2x2(f2fma(raw2(s, 2 * i), sl2, nm2));
+                        l4[i & 3] = f2add(l4[i & 3], p2);
+                        d4[i & 3] = f2fma(p2, raw2(dp, 2 * i), d4[i & 3]);
+                    }
+                    const float2 ls = f2add(f2add(l4[0], l4[1]), f2add(l4[2], l4[3]));
+                    const float2 ds = f2add(f2add(d4[0], d4[1]), f2add(d4[2], d4[3]));
+                    l += ls.x + ls.y;
+                    Dacc += ds.x + ds.y;
+                }
+                tc::fence_before_sync();
+                mbar_arrive(&sfree[w]);
+                if (u == n_it - 1) {
+                    // merge the two halves' statistics: half 1 hands its (m, l, D) to half 0,
+                    // which forms the row's log-sum-exp and D and hands them back
+                    if (w == 1) {
+                        part[row] = m;
+                        part[TILE + row] = l;
+                        part[2 * TILE + row] = Dacc;
+                        mbar_arrive(&xch[0]);
+                        if (!wait_bar(&xch[1], 0, abort_flag)) { ok = false; break; }
+                        L2 = part[row];
+                        Drow = part[TILE + row];
+                    } else {
+                        if (!wait_bar(&xch[0], 0, abort_flag)) { ok = false; break; }
+                        const float m1 = part[row], l1 = part[TILE + row], D1 = part[2 * TILE + row];
+                        const float M = fmaxf(m, m1);
+                        const float a0 = tc::ex2(m - M), a1 = tc::ex2(m1 - M);
+                        const float lt = l * a0 + l1 * a1, Dt = Dacc * a0 + D1 * a1;
+                        if (t < T) {
+                            L2 = M + log2f(lt);
+                            Drow = Dt / lt;
+                        } else {  // past the end: no probability mass, no gradient
+                            L2 = INFINITY;
+                            Drow = 0.f;
+                        }
+                        nlse2[(int64_t)bh * Tpad + t] = -L2;
+                        dbuf[(int64_t)bh * Tpad + t] = Drow;
+                        part[row] = L2;
+                        part[TILE + row] = Drow;
+                        mbar_arrive(&xch[1]);
+                    }
+                }
+            } else {
+                uint32_t pk[32];
+                const float2 nl2 = make_float2(-L2, -L2), d2 = make_float2(Drow, Drow);
+#pragma unroll
+                for (int c = 0; c < 2; ++c) {
+                    uint32_t s[32], dp[32];
+                    tc::tmem_ld32(tS + 32u * c, s);
+                    tc::tmem_ld32(tP + 32u * c, dp);
+                    tc::tmem_wait_ld();
+                    if (!full_tile) mask_chunk(s, c, lo, hi);
+#pragma unroll
+                    for (int i = 0; i < 16; ++i) {
+                        const float2 p2 = ex2x2(f2fma(raw2(s, 2 * i), sl2, nl2));
+                        const float2 ds = f2mul(p2, f2sub(raw2(dp, 2 * i), d2));
+                        pk[16 * c + i] = pack_bf16x2(ds.x, ds.y);
+                    }
+                }
+                tc::tmem_st32(tS, pk);
+                tc::tmem_wait_st();
+                tc::fence_before_sync();
+                mbar_arrive(&sfree[w]);
+            }
+        }
+        // epilogue: dq = scale * dQ -> bf16, this half's 64 channels
+        if (ok && wait_bar(done, 0, abort_flag)) {
+            tc::fence_after_sync();
+            __nv_bfloat16* out = dq + ((int64_t)bh * T + t) * HD + HALF * w;
+#pragma unroll
+            for (int cb = 0; cb < 2; ++cb) {
+                uint32_t r[32];
+                tc::tmem_ld32(tQ + 32u * cb, r);
+                tc::tmem_wait_ld();
+                if (t < T) {
+#pragma unroll
+                    for (int i = 0; i < 32; i += 8) {
+                        float f[8];
+#pragma unroll
+                        for (int e = 0; e < 8; ++e) f[e] = __uint_as_float(r[i + e]) * scale;
+                        store8(out + 32 * cb + i, f);
+                    }
+                }
+            }
+        }
+    }
+
+    tc::fence_before_sync();
+    __syncthreads();
+    tc::fence_after_sync();
+    if (warp == 9) tc::tmem_dealloc(tmem, 512);
+}
+
+// ============================================================================================
+// Launch 2: key tiles (dV per head, dK partial per head group)
+// ============================================================================================
+namespace ka {
+constexpr int OFF_K = 0;
+constexpr int OFF_V = TILE_BYTES;
+constexpr int OFF_RING = 2 * TILE_BYTES;             // 2 slots of (Q tile, dO tile)
+constexpr int UNIT_BYTES = 2 * TILE_BYTES;
+constexpr int OFF_STAT = OFF_RING + 2 * UNIT_BYTES;  // 2 slots of (lse2[128], D[128]) fp32
+constexpr int STAT_BYTES = 2 * TILE * 4;
+constexpr int OFF_BAR = OFF_STAT + 2 * STAT_BYTES;
+// kfull, vfull, vempty, full[2], empty[2], sfull[2], sfree[2], dvdone, dvfree, done, drain
+constexpr int NBAR = 15;
+constexpr int OFF_MISC = OFF_BAR + 8 * NBAR;
+constexpr int SMEM = OFF_MISC + 16 + 1024;
+static_assert(SMEM <= 232448, "shared memory");
+}  // namespace ka
+
+__global__ void __launch_bounds__(NTHREADS, 1)
+ska_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_do,
+                    const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
+                    const float* __restrict__ nlse2, const float* __restrict__ dbuf,
+                    __nv_bfloat16* __restrict__ dv, float* __restrict__ dk_part, int B, int T, int Tpad,
+                    int H, int HG, int W, float scale_log2, int n_qtiles) {
+    using namespace ka;
+    extern __shared__ unsigned char smem_raw[];
+    unsigned char* smem = align1024(smem_raw);
+    const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+    const int kt = blockIdx.x, grp = blockIdx.y, b = blockIdx.z;
+    const int j0 = kt * TILE;
+    const int qt_lo = kt;  // queries t in [j, j + W - 1] see key j
+    const int64_t last_q = (int64_t)j0 + TILE - 1 + W - 1;  // the last query that sees the tile
+    const int qt_hi = last_q / TILE < n_qtiles - 1 ? (int)(last_q / TILE) : n_qtiles - 1;
+    const int n_q = qt_hi - qt_lo + 1;  // query tiles per head
+    const int h0 = grp * HG;
+    const int U = HG * n_q;             // (head, query tile) pairs, head-major
+
+    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + OFF_BAR);
+    uint64_t* kfull = bars;
+    uint64_t* vfull = bars + 1;
+    uint64_t* vempty = bars + 2;
+    uint64_t* full = bars + 3;
+    uint64_t* empty = bars + 5;
+    uint64_t* sfull = bars + 7;
+    uint64_t* sfree = bars + 9;
+    uint64_t* dvdone = bars + 11;
+    uint64_t* dvfree = bars + 12;
+    uint64_t* done = bars + 13;
+    uint64_t* drain = bars + 14;
+    uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + OFF_MISC);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + OFF_MISC + 4);
+
+    if (threadIdx.x == 0) {
+        mbar_init(kfull, 1);
+        mbar_init(vfull, 1);
+        mbar_init(vempty, 1);
+        for (int s = 0; s < 2; ++s) {
+            mbar_init(&full[s], 1);
+            mbar_init(&empty[s], 1);
+            mbar_init(&sfull[s], 1);
+            mbar_init(&sfree[s], 128);
+        }
+        mbar_init(dvdone, 1);
+        mbar_init(dvfree, 256);
+        mbar_init(done, 1);
+        mbar_init(drain, 1);
+        *abort_flag = 0;
+        fence_mbar_init();
+    }
+    if (warp == 9) {
+        tc::tmem_alloc(tmem_holder, 512);
+        tc::tmem_relinquish();
+    }
+    tc::fence_before_sync();
+    __syncthreads();
+    tc::fence_after_sync();
+    const uint32_t tmem = *tmem_holder;
+    // TMEM columns: S^T [0,128) | dP^T [128,256) | dV [256,384) | dK [384,512)
+
+    if (warp == 8) {
+        // ------------------------------- TMA producer -------------------------------
+        if (lane == 0) {
+            tc::tma_prefetch_desc(&tm_q);
+            tc::tma_prefetch_desc(&tm_do);
+            tc::tma_prefetch_desc(&tm_k);
+            tc::tma_prefetch_desc(&tm_v);
+            mbar_arrive_expect_tx(kfull, TILE_BYTES);
+            for (int half = 0; half < 2; ++half)
+                tc::tma_load_3d(smem + OFF_K + half * BOX_BYTES, &tm_k, half * 64, j0, b, kfull);
+            int u = 0, nv = 0;
+            for (; u < U; ++u) {
+                const int hi = u / n_q, qt = qt_lo + u % n_q, bh = b * H + h0 + hi;
+                if (u % n_q == 0) {  // a new head: its V tile (once the previous head's is used)
+                    if (hi > 0 && !wait_bar(vempty, (uint32_t)((hi - 1) & 1), abort_flag)) break;
+                    mbar_arrive_expect_tx(vfull, TILE_BYTES);
+                    for (int half = 0; half < 2; ++half)
+                        tc::tma_load_3d(smem + OFF_V + half * BOX_BYTES, &tm_v, half * 64, j0, bh, vfull);
+                    ++nv;
+                }
+                const int slot = u % 2, use = u / 2;
+                if (use > 0 && !wait_bar(&empty[slot], (uint32_t)((use - 1) & 1), abort_flag)) break;
+                unsigned char* dst = smem + OFF_RING + slot * UNIT_BYTES;
+                unsigned char* st = smem + OFF_STAT + slot * STAT_BYTES;
+                mbar_arrive_expect_tx(&full[slot], 2 * TILE_BYTES + STAT_BYTES);
+                for (int half = 0; half < 2; ++half) {
+                    tc::tma_load_3d(dst + half * BOX_BYTES, &tm_q, half * 64, qt * TILE, bh, &full[slot]);
+                    tc::tma_load_3d(dst + TILE_BYTES + half * BOX_BYTES, &tm_do, half * 64, qt * TILE, bh,
+                                    &full[slot]);
+                }
+                const int64_t srow = (int64_t)bh * Tpad + (int64_t)qt * TILE;
+                bulk_g2s(st, nlse2 + srow, TILE * 4, &full[slot]);
+                bulk_g2s(st + TILE * 4, dbuf + srow, TILE * 4, &full[slot]);
+            }
+            // every copy started here has landed before the CTA can leave (a V or unit load
+            // older than the latest ones was consumed by MMAs that have completed)
+            mbar_wait_bounded(kfull, 0, kWaitLimit);
+            if (nv > 0) mbar_wait_bounded(vfull, (uint32_t)((nv - 1) & 1), kWaitLimit);
+            for (int ui = (u > 2 ? u - 2 : 0); ui < u; ++ui)
+                mbar_wait_bounded(&full[ui % 2], (uint32_t)((ui / 2) & 1), kWaitLimit);
+        }
+    } else if (warp == 9) {
+        // ------------------------------- MMA issuer -------------------------------
+        if (lane == 0) {
+            const uint32_t idesc_s = tc::idesc_bf16_f32(TILE, HALF, 0, 0);  // S^T half, both K-major
+            const uint32_t idesc_g = tc::idesc_bf16_f32(TILE, HD, 0, 1);    // gradients, B MN-major
+            const uint32_t d_hi = tc::desc_hi(tc::sdesc_sw128(0, 16, 1024));
+            const uint32_t k_lo = lo_kmajor(smem_u32(smem + OFF_K));
+            const uint32_t v_lo = lo_kmajor(smem_u32(smem + OFF_V));
+            auto unit = [&](int u) { return smem_u32(smem + OFF_RING + (u % 2) * UNIT_BYTES); };
+            bool ok = true;
+            auto acquire = [&](uint64_t* bar, uint32_t parity) {
+                ok = ok && wait_bar(bar, parity, abort_flag);
+                tc::fence_after_sync();
+                return ok;
+            };
+            // S^T_w = K Q[64w, 64w+64)^T and dP^T_w = V dO[64w, 64w+64)^T of pair u
+            auto issue_sdp = [&](int w, int u) {
+                const uint32_t q_lo = lo_kmajor(unit(u) + w * HALF_ROWS);
+                const uint32_t o_lo = lo_kmajor(unit(u) + TILE_BYTES + w * HALF_ROWS);
+#pragma unroll
+                for (int k = 0; k < HD / 16; ++k)
+                    tc::mma_ss_lh(tmem + 64u * w, k_lo + kstep(k), d_hi, q_lo + kstep(k), d_hi, idesc_s, k > 0);
+#pragma unroll
+                for (int k = 0; k < HD / 16; ++k)
+                    tc::mma_ss_lh(tmem + 128u + 64u * w, v_lo + kstep(k), d_hi, o_lo + kstep(k), d_hi, idesc_s, k > 0);
+            };
+            // dV += P^T_w dO[64w, 64w+64) and dK += dS^T_w Q[64w, 64w+64), with P^T_w and dS^T_w
+            // packed in the first 32 columns of the S^T and dP^T halves
+            auto issue_grad = [&](int w, int u, bool first_dv, bool first_dk) {
+                const uint32_t q_lo = lo_mnmajor(unit(u) + w * HALF_ROWS);
+                const uint32_t o_lo = lo_mnmajor(unit(u) + TILE_BYTES + w * HALF_ROWS);
+#pragma unroll
+                for (int k = 0; k < HALF / 16; ++k)
+                    tc::mma_ts_lh(tmem + 256u, tmem + 64u * w + 8u * k, o_lo + mnstep(k), d_hi, idesc_g,
+                                  (first_dv && k == 0) ? 0u : 1u);
+#pragma unroll
+                for (int k = 0; k < HALF / 16; ++k)
+                    tc::mma_ts_lh(tmem + 384u, tmem + 128u + 64u * w + 8u * k, q_lo + mnstep(k), d_hi, idesc_g,
+                                  (first_dk && k == 0) ? 0u : 1u);
+            };
+            if (acquire(kfull, 0) && acquire(vfull, 0) && acquire(&full[0], 0)) {
+                issue_sdp(0, 0);
+                tc::mma_commit(&sfull[0]);
+                issue_sdp(1, 0);
+                tc::mma_commit(&sfull[1]);
+                if (n_q == 1) tc::mma_commit(vempty);
+                for (int u = 0; u < U && ok; ++u) {
+                    const int hi = u / n_q;
+                    const bool first_of_head = u % n_q == 0, last_of_head = u % n_q == n_q - 1;
+                    for (int w = 0; w < 2; ++w) {
+                        if (!acquire(&sfree[w], (uint32_t)(u & 1))) break;
+                        if (w == 0 && first_of_head && hi > 0 && !acquire(dvfree, (uint32_t)((hi - 1) & 1)))
+                            break;
+                        issue_grad(w, u, first_of_head && w == 0, u == 0 && w == 0);
+                        if (w == 1) {
+                            tc::mma_commit(&empty[u % 2]);
+                            if (last_of_head) tc::mma_commit(dvdone);
+                        }
+                        if (u + 1 < U) {
+                            if (w == 0) {
+                                if (!acquire(&full[(u + 1) % 2], (uint32_t)(((u + 1) / 2) & 1))) break;
+                                if ((u + 1) % n_q == 0 && !acquire(vfull, (uint32_t)(((u + 1) / n_q) & 1))) break;
+                            }
+                            issue_sdp(w, u + 1);
+                            tc::mma_commit(&sfull[w]);
+                            if (w == 1 && (u + 1) % n_q == n_q - 1) tc::mma_commit(vempty);
+                        }
+                    }
+                }
+                if (ok) tc::mma_commit(done);
+            }
+            tc::mma_commit(drain);
+            mbar_wait_bounded(drain, 0, kWaitLimit);
+        }
+    } else {
+        // ------------------------------- softmax warpgroups -------------------------------
+        const int w = warp / 4;                    // column half (queries 64w .. 64w + 63)
+        const int row = threadIdx.x % 128;         // key row == TMEM lane
+        const uint32_t lane_base = (uint32_t)(32 * (warp % 4)) << 16;
+        const uint32_t tS = tmem + lane_base + 64u * w;
+        const uint32_t tP = tS + 128u;
+        const uint32_t tV = tmem + lane_base + 256u + 64u * w;
+        const uint32_t tK = tmem + lane_base + 384u + 64u * w;
+        const int key = j0 + row;
+        bool ok = true;
+        for (int u = 0; u < U; ++u) {
+            const int hi = u / n_q, qt = qt_lo + u % n_q;
+            const int tq0 = qt * TILE + HALF * w;  // first query of this half
+            if (!wait_bar(&sfull[w], (uint32_t)(u & 1), abort_flag)) { ok = false; break; }
+            tc::fence_after_sync();
+            const float* st = reinterpret_cast<const float*>(smem + OFF_STAT + (u % 2) * STAT_BYTES) + HALF * w;
+            const bool full_tile = tq0 >= j0 + TILE - 1 && tq0 + HALF - 1 <= j0 + W - 1;
+            const int lo = key - tq0, hi_e = key + W - 1 - tq0;  // valid columns [lo, hi_e]
+            // P^T and dS^T of each 32-column chunk go, packed, over the first 16 columns of the
+            // chunk's own 32 (already read): chunk c at columns 16 c of the S^T / dP^T half
+            const float2 sl2 = make_float2(scale_log2, scale_log2);
+#pragma unroll
+            for (int c = 0; c < 2; ++c) {
+                uint32_t s[32], dp[32], pp[16], pd[16];
+                tc::tmem_ld32(tS + 32u * c, s);
+                tc::tmem_ld32(tP + 32u * c, dp);
+                tc::tmem_wait_ld();
+                if (!full_tile) mask_chunk(s, c, lo, hi_e);
+#pragma unroll
+                for (int e4 = 0; e4 < 32; e4 += 4) {
+                    const float4 L4 = *reinterpret_cast<const float4*>(st + 32 * c + e4);  // -lse2
+                    const float4 D4 = *reinterpret_cast<const float4*>(st + TILE + 32 * c + e4);
+                    const float2 pa = ex2x2(f2fma(raw2(s, e4), sl2, make_float2(L4.x, L4.y)));
+                    const float2 pb = ex2x2(f2fma(raw2(s, e4 + 2), sl2, make_float2(L4.z, L4.w)));
+                    const float2 da = f2mul(pa, f2sub(raw2(dp, e4), make_float2(D4.x, D4.y)));
+                    const float2 db = f2mul(pb, f2sub(raw2(dp, e4 + 2), make_float2(D4.z, D4.w)));
+                    pp[e4 / 2] = pack_bf16x2(pa.x, pa.y);
+                    pp[e4 / 2 + 1] = pack_bf16x2(pb.x, pb.y);
+                    pd[e4 / 2] = pack_bf16x2(da.x, da.y);
+                    pd[e4 / 2 + 1] = pack_bf16x2(db.x, db.y);
+                }
+                tc::tmem_st16(tS + 16u * c, pp);
+                tc::tmem_st16(tP + 16u * c, pd);
+            }
+            tc::tmem_wait_st();
+            tc::fence_before_sync();
+            mbar_arrive(&sfree[w]);
+            if (u % n_q == n_q - 1) {
+                // the head's dV rows are complete: store them and release the accumulator
+                if (!wait_bar(dvdone, (uint32_t)(hi & 1), abort_flag)) { ok = false; break; }
+                tc::fence_after_sync();
+                __nv_bfloat16* out = dv + (((int64_t)b * H + h0 + hi) * T + key) * HD + HALF * w;
+#pragma unroll
+                for (int cb = 0; cb < 2; ++cb) {
+                    uint32_t r[32];
+                    tc::tmem_ld32(tV + 32u * cb, r);
+                    tc::tmem_wait_ld();
+                    if (key < T) {
+#pragma unroll
+                        for (int i = 0; i < 32; i += 8) {
+                            float f[8];
+#pragma unroll
+                            for (int e = 0; e < 8; ++e) f[e] = __uint_as_float(r[i + e]);
+                            store8(out + 32 * cb + i, f);
+                        }
+                    }
+                }
+                tc::fence_before_sync();
+                mbar_arrive(dvfree);
+            }
+        }
+        // epilogue: this group's dK partial (unscaled fp32), this half's 64 channels
+        if (ok && wait_bar(done, 0, abort_flag)) {
+            tc::fence_after_sync();
+            float* out = dk_part + (((int64_t)grp * B + b) * T + key) * HD + HALF * w;
+#pragma unroll
+            for (int cb = 0; cb < 2; ++cb) {
+                uint32_t r[32];
+                tc::tmem_ld32(tK + 32u * cb, r);
+                tc::tmem_wait_ld();
+                if (key < T) {
+#pragma unroll
+                    for (int i = 0; i < 32; i += 4)
+                        *reinterpret_cast<float4*>(out + 32 * cb + i) =
+                            make_float4(__uint_as_float(r[i]), __uint_as_float(r[i + 1]),
+                                        __uint_as_float(r[i + 2]), __uint_as_float(r[i + 3]));
+                }
+            }
+        }
+    }
+
+    tc::fence_before_sync();
+    __syncthreads();
+    tc::fence_after_sync();
+    if (warp == 9) tc::tmem_dealloc(tmem, 512);
+}
+
+// ============================================================================================
+// Launch 3: dk = scale * sum over head groups of the partials (group order fixed)
+// ============================================================================================
+__global__ void __launch_bounds__(256)
+ska_bwd_dk_reduce(const float* __restrict__ part, __nv_bfloat16* __restrict__ dk, int64_t n4, int G,
+                  float scale) {
+    const float4* p4 = reinterpret_cast<const float4*>(part);
+    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n4;
+         i += (int64_t)gridDim.x * blockDim.x) {
+        float4 a = p4[i];
+        for (int g = 1; g < G; ++g) {
+            const float4 x = p4[(int64_t)g * n4 + i];
+            a.x += x.x;
+            a.y += x.y;
+            a.z += x.z;
+            a.w += x.w;
+        }
+        store4(dk + 4 * i, make_float4(a.x * scale, a.y * scale, a.z * scale, a.w * scale));
+    }
+}
+
+int sm_count() {
+    static int sms = 0;
+    if (sms == 0) {
+        int dev = 0;
+        if (cudaGetDevice(&dev) != cudaSuccess ||
+            cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || sms < 1)
+            sms = 148;
+    }
+    return sms;
+}
+
+}  // namespace
+
+int64_t swska_backward_tc_tpad(int T) { return ((int64_t)T + TILE - 1) / TILE * TILE; }
+
+size_t swska_backward_tc_workspace_size(int B, int H, int T) {
+    // row statistics (padded rows) + one fp32 dK partial per head group (at most H groups)
+    return ((size_t)2 * B * H * swska_backward_tc_tpad(T) + (size_t)H * B * T * HD) * sizeof(float);
+}
+
+bool swska_backward_tc_supported(int H, int T, int dk, int dv) {
+    return dk == HD && dv == HD && H >= 1 && T >= TILE;
+}
+
+int swska_backward_tc_groups(int B, int H, int T) {
+    // the fewest head groups that still give every SM several key-tile CTAs
+    const int64_t nkt = ((int64_t)T + TILE - 1) / TILE;
+    for (int G = 1; G < H; ++G)
+        if (H % G == 0 && (int64_t)B * nkt * G >= 4 * (int64_t)sm_count()) return G;
+    return H;
+}
+
+cudaError_t swska_backward_tc_launch(const SkaBackwardArgs& a, cudaStream_t stream) {
+    const int B = a.B, H = a.H, T = a.T;
+    const int W = a.W < T ? a.W : T;  // a window longer than the sequence is the whole prefix
+    const int64_t Tpad = swska_backward_tc_tpad(T);
+    float* lse2 = static_cast<float*>(a.workspace);
+    float* dbuf = lse2 + (size_t)B * H * Tpad;
+    float* part = dbuf + (size_t)B * H * Tpad;
+    if (B > 65535 || H > 65535) return cudaErrorInvalidConfiguration;
+    CUtensorMap mq, mdo, mk, mv;
+    cudaError_t e;
+    if ((e = make_tmap_bf16_3d(&mq, a.q, HD, (uint64_t)T, (uint64_t)B * H, 64, TILE)) != cudaSuccess) return e;
+    if ((e = make_tmap_bf16_3d(&mdo, a.dO, HD, (uint64_t)T, (uint64_t)B * H, 64, TILE)) != cudaSuccess) return e;
+    if ((e = make_tmap_bf16_3d(&mk, a.k, HD, (uint64_t)T, (uint64_t)B, 64, TILE)) != cudaSuccess) return e;
+    if ((e = make_tmap_bf16_3d(&mv, a.v, HD, (uint64_t)T, (uint64_t)B * H, 64, TILE)) != cudaSuccess) return e;
+    if ((e = cudaFuncSetAttribute(ska_bwd_dq_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, qa::SMEM)) !=
+        cudaSuccess)
+        return e;
+    if ((e = cudaFuncSetAttribute(ska_bwd_dkdv_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, ka::SMEM)) !=
+        cudaSuccess)
+        return e;
+    const int nqt = (int)(Tpad / TILE);
+    const float sl = a.scale * kLog2e;
+    ska_bwd_dq_kernel<<<dim3((unsigned)nqt, (unsigned)H, (unsigned)B), NTHREADS, qa::SMEM, stream>>>(
+        mq, mdo, mk, mv, static_cast<__nv_bfloat16*>(a.dq), lse2, dbuf, T, (int)Tpad, H, W, sl, a.scale, nqt);
+    const int G = swska_backward_tc_groups(B, H, T);
+    ska_bwd_dkdv_kernel<<<dim3((unsigned)nqt, (unsigned)G, (unsigned)B), NTHREADS, ka::SMEM, stream>>>(
+        mq, mdo, mk, mv, lse2, dbuf, static_cast<__nv_bfloat16*>(a.dv), part, B, T, (int)Tpad, H, H / G, W,
+        sl, nqt);
+    const int64_t n4 = (int64_t)B * T * HD / 4;
+    const int64_t want = (n4 + 255) / 256, cap = 8 * (int64_t)sm_count();
+    ska_bwd_dk_reduce<<<(unsigned)(want < cap ? want : cap), 256, 0, stream>>>(
+        part, static_cast<__nv_bfloat16*>(a.dk), n4, G, a.scale);
+    note_launches(3);
+    return cudaGetLastError();
+}
+
+unsigned swska_backward_tc_take_timeout_flag() {
+    unsigned v = 0, zero = 0;
+    if (cudaMemcpyFromSymbol(&v, g_ska_bwd_tc_timeout, sizeof(v)) != cudaSuccess) return 0;
+    cudaMemcpyToSymbol(g_ska_bwd_tc_timeout, &zero, sizeof(zero));
+    return v;
+}
+
+}  // namespace rod

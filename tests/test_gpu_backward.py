@@ -100,3 +100,25 @@ def test_swska_backward_fp32(dk, dv, W):
 @pytest.mark.parametrize("T,W", [(1, 64), (200, 64), (300, 300), (257, 128)])
 def test_swska_backward_bf16(T, W):
     _ska_check(1, 4, T, 128, 128, W, "bf16", seed=T + W)
+
+
+# bf16 with head dim 128 and T >= 128 runs on the tensor cores: one 128-query tile, ragged
+# tails, windows of 1, below, at and above the tile size, a window longer than the sequence,
+# several batches, and head counts that give one or several heads per key-tile group
+@pytest.mark.parametrize("B,H,T,W", [(1, 2, 128, 128), (2, 3, 384, 1), (1, 5, 640, 200),
+                                     (2, 2, 129, 1000), (1, 16, 1024, 256), (1, 3, 1000, 129),
+                                     (3, 1, 700, 64), (1, 4, 2048, 700)])
+def test_swska_backward_bf16_tensor_core(B, H, T, W):
+    _ska_check(B, H, T, 128, 128, W, "bf16", seed=B * 1000 + H * 100 + T + W)
+
+
+@pytest.mark.parametrize("d", [32, 64])
+def test_swska_backward_bf16_small_head_dim(d):
+    """Head dims other than 128 keep the CUDA-core kernels in bf16."""
+    _ska_check(2, 3, 300, d, d, 100, "bf16", seed=d)
+
+
+def test_swska_backward_full_size():
+    """The benchmarked backward workload (B1 H16 T8192 W4096, bf16, head dim 128), every
+    gradient element against the oracle (about ten seconds of fp64 on the host)."""
+    _ska_check(1, 16, 8192, 128, 128, 4096, "bf16", seed=42)
