@@ -41,6 +41,11 @@ bool swska_prefill_tc_supported(int H, int T, int dk, int dv);
 cudaError_t swska_prefill_tc_launch(const void* q, const void* k, const void* v, void* o, int B,
                                     int H, int T, int window, float scale, cudaStream_t stream);
 unsigned swska_prefill_tc_take_timeout_flag();
+// the same kernel with per-row statistics for the backward: negated base-2 log-sum-exp and
+// D = dO . o into row bh * Tpad + t (o may be null: then the output is not stored)
+cudaError_t swska_prefill_tc_stats_launch(const void* q, const void* k, const void* v, void* o,
+                                          const void* dO, float* nlse2, float* dbuf, int64_t Tpad, int B,
+                                          int H, int T, int window, float scale, cudaStream_t stream);
 
 // TMA descriptors for a 3-D tensor [d2][d1][d0] loaded as boxes of box1 x box0 elements
 cudaError_t make_tmap_3d(CUtensorMap* map, const void* base, bool fp32, uint64_t d0, uint64_t d1,

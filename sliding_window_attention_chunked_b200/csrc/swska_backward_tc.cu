@@ -5,30 +5,31 @@
 // per-head V; setup blog §3: a window of the most recent W tokens):
 //   s_tj = scale q_t . k_j for j in [t-W+1, t],  p_t = softmax(s_t),  o_t = sum_j p_tj v_j.
 // For the loss gradient dO of every output row, with dP_tj = dO_t . v_j:
-//   D_t = sum_j p_tj dP_tj (= dO_t . o_t),   dS_tj = p_tj (dP_tj - D_t),
+//   D_t = sum_j p_tj dP_tj = dO_t . o_t,   dS_tj = p_tj (dP_tj - D_t),
 //   dq_t = scale sum_j dS_tj k_j,   dv_j = sum_t p_tj dO_t (per head),
 //   dk_j = scale sum_h sum_t dS_tj q_t   (the shared key gathers every head's share).
 //
-// Three launches:
-//  1. Query tiles: one CTA per 128 queries of one head. A first sweep over the window's key
-//     tiles computes S = Q K^T and dP = dO V^T and keeps, per query row, the running maximum,
-//     the normaliser and D (online, base 2). The row's negated base-2 log-sum-exp and D are
-//     stored for launch 2 (-inf and 0 for rows past the end of the sequence). A second sweep recomputes S
-//     and dP, forms dS in bf16 in tensor memory and accumulates dQ += dS K there.
-//  2. Key tiles: one CTA per 128 keys and group of heads. For every head of the group and every
-//     query tile that sees the key tile: S^T = K Q^T and dP^T = V dO^T; P^T and dS^T (from the
-//     stored statistics) are written to tensor memory in bf16 and feed dV += P^T dO and
-//     dK += dS^T Q. dV is complete per head; dK is a partial per head group, stored in fp32.
-//  3. dk = scale * (sum of the groups' partials), summed in group order (deterministic).
-// In launches 1 and 2 each 128-column score tile is split into two halves of 64 columns, one
-// per softmax warpgroup, each with its own MMAs and barriers: one half's exponentials run
-// while the tensor core works on the other half. Warp roles (320 threads):
+// Four launches:
+//  1. The forward kernel (swska_prefill_tc.cu) in its statistics mode: per row the negated base-2
+//     log-sum-exp and D_t = dO_t . o_t from the fp32 output (nothing else is stored).
+//  2. Query tiles (one CTA per 128 queries of one head): for each key tile of the window,
+//     S = Q K^T and dP = dO V^T, then dS = P (dP - D) in bf16 in tensor memory and
+//     dQ += dS K there.
+//  3. Key tiles (one CTA per 128 keys and group of heads): for every head of the group and every
+//     query tile that sees the key tile, S^T = K Q^T and dP^T = V dO^T; P^T and dS^T go to
+//     tensor memory in bf16 and feed dV += P^T dO and dK += dS^T Q. dV is complete per head;
+//     dK is a partial per head group, stored in fp32.
+//  4. dk = scale * (sum of the groups' partials), summed in group order (deterministic).
+// Every MMA is M = 128, N = 128, K = 16 (an N = 64 MMA costs most of an N = 128 one to issue).
+// The two softmax warpgroups split each tile's 128 columns (64 each) and work in two phases:
+// P from S as soon as S lands, then dS once dP lands; the MMA order lets the tensor core run
+// the next products meanwhile. Warp roles (320 threads):
 //   warps 0-3 / 4-7  softmax warpgroups of column halves 0 / 1 (thread = TMEM lane = tile row)
-//   warp 8           TMA producer
-//   warp 9           TMEM allocator and the single MMA-issuing thread
-// Operands are staged by TMA in 128-byte-swizzled boxes; the P and dS operands of the
-// gradient MMAs are read from tensor memory (the A operand of a TS-form MMA). Every wait is
-// bounded; a timeout makes all roles stop, drain their copies and MMAs, and raise a flag.
+//   warp 8           TMA producer (one lane)
+//   warp 9           TMEM allocator; MMA issue (the whole warp runs the loop, one elected lane
+//                    issues each tcgen05 instruction)
+// Every wait is bounded; a timeout makes all roles stop, drain their copies and MMAs, and
+// raise a flag.
 #include <cuda.h>
 #include <math.h>
 
@@ -46,7 +47,6 @@ constexpr int HD = 128;                     // head dim (dk = dv)
 constexpr int HALF = 64;                    // score columns per softmax warpgroup
 constexpr int TILE_BYTES = TILE * HD * 2;   // 32 KB: one 128 x 128 bf16 tile
 constexpr int BOX_BYTES = TILE_BYTES / 2;   // one TMA box: 128 rows x 64 columns
-constexpr int HALF_ROWS = HALF * 128;       // byte offset of row 64 inside a box (8 KB)
 constexpr int NTHREADS = 320;
 constexpr float kLog2e = 1.4426950408889634f;
 
@@ -55,6 +55,23 @@ __device__ __forceinline__ bool wait_bar(uint64_t* bar, uint32_t parity, volatil
         if (mbar_try_wait(bar, parity)) return true;
         if ((i & 255u) == 0) {
             if (*abort_flag) return false;
+            if (i >= kWaitLimit) {
+                *abort_flag = 1;
+                atomicExch(&g_ska_bwd_tc_timeout, 1u);
+                return false;
+            }
+        }
+    }
+}
+
+// The same wait executed by a whole warp in lockstep: every lane polls, and the warp leaves
+// together (all lanes saw the phase complete, or the abort flag / limit is seen by all), so the
+// warp stays converged for the elected MMA issue that follows.
+__device__ __forceinline__ bool wait_bar_warp(uint64_t* bar, uint32_t parity, volatile int* abort_flag) {
+    for (uint32_t i = 1;; ++i) {
+        if (__all_sync(0xffffffffu, mbar_try_wait(bar, parity))) return true;
+        if ((i & 255u) == 0) {
+            if (__any_sync(0xffffffffu, *abort_flag != 0)) return false;
             if (i >= kWaitLimit) {
                 *abort_flag = 1;
                 atomicExch(&g_ska_bwd_tc_timeout, 1u);
@@ -89,13 +106,6 @@ __device__ __forceinline__ float2 f2fma(float2 a, float2 b, float2 c) {
         : "=f"(d.x), "=f"(d.y) : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y), "f"(c.x), "f"(c.y));
     return d;
 }
-__device__ __forceinline__ float2 f2add(float2 a, float2 b) {
-    float2 d;
-    asm("{\n\t.reg .b64 ra, rb, rd;\n\tmov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\t"
-        "add.rn.f32x2 rd, ra, rb;\n\tmov.b64 {%0, %1}, rd;\n\t}"
-        : "=f"(d.x), "=f"(d.y) : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
-    return d;
-}
 __device__ __forceinline__ float2 f2sub(float2 a, float2 b) {
     float2 d;
     asm("{\n\t.reg .b64 ra, rb, rd;\n\tmov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\t"
@@ -108,11 +118,6 @@ __device__ __forceinline__ float2 f2mul(float2 a, float2 b) {
     asm("{\n\t.reg .b64 ra, rb, rd;\n\tmov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\t"
         "mul.rn.f32x2 rd, ra, rb;\n\tmov.b64 {%0, %1}, rd;\n\t}"
         : "=f"(d.x), "=f"(d.y) : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
-    return d;
-}
-__device__ __forceinline__ float fmax3(float a, float b, float c) {
-    float d;
-    asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
     return d;
 }
 __device__ __forceinline__ float2 raw2(const uint32_t* r, int e) {
@@ -128,40 +133,35 @@ __device__ __forceinline__ void mask_chunk(uint32_t* s, int c, int lo, int hi) {
         if (col < lo || col > hi) s[e] = 0xff800000u;
     }
 }
-// maximum of 32 raw scores: four independent chains of three-input maxima
-__device__ __forceinline__ float max32(const uint32_t* s) {
-    float m4[4];
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-        float m = fmax3(__uint_as_float(s[i]), __uint_as_float(s[i + 4]), __uint_as_float(s[i + 8]));
-        m = fmax3(m, __uint_as_float(s[i + 12]), __uint_as_float(s[i + 16]));
-        m = fmax3(m, __uint_as_float(s[i + 20]), __uint_as_float(s[i + 24]));
-        m4[i] = fmaxf(m, __uint_as_float(s[i + 28]));
-    }
-    return fmaxf(fmax3(m4[0], m4[1], m4[2]), m4[3]);
-}
-
 // ============================================================================================
-// Launch 1: query tiles (row statistics, then dQ)
+// Launch 2: query tiles (dQ)
 // ============================================================================================
 namespace qa {
-constexpr int NSLOT = 5;                            // ring of K / V tiles
+constexpr int KSLOT = 3, VSLOT = 2;                 // rings of K and V tiles
 constexpr int OFF_Q = 0;
 constexpr int OFF_DO = TILE_BYTES;
-constexpr int OFF_RING = 2 * TILE_BYTES;
-constexpr int OFF_BAR = OFF_RING + NSLOT * TILE_BYTES;
-constexpr int NBAR = 2 * NSLOT + 9;  // full, empty, qfull, sfull[2], sfree[2], done, drain, xch[2]
-constexpr int OFF_PART = OFF_BAR + 8 * NBAR;        // float [3][128]: statistics exchange
-constexpr int OFF_MISC = OFF_PART + 3 * TILE * 4;
+constexpr int OFF_K = 2 * TILE_BYTES;
+constexpr int OFF_V = OFF_K + KSLOT * TILE_BYTES;
+constexpr int OFF_BAR = OFF_V + VSLOT * TILE_BYTES;
+// kfull[3], kempty[3], vfull[2], vempty[2], qfull, sfull[2], pfull, dsready, done, drain
+constexpr int NBAR = 2 * KSLOT + 2 * VSLOT + 7;
+constexpr int OFF_MISC = OFF_BAR + 8 * NBAR;
 constexpr int SMEM = OFF_MISC + 16 + 1024;
 static_assert(SMEM <= 232448, "shared memory");
 }  // namespace qa
 
+// TMEM columns: S buffers at 0 and 384 (tile u uses buffer u & 1), dP at 128, dQ at 256.
+__device__ __forceinline__ uint32_t s_col(int u) { return (u & 1) ? 384u : 0u; }
+// A operand of K step k (16 columns of P or dS) packed by the two warpgroups: warpgroup w's 64
+// columns sit, two per 32-bit column, in columns 64 w .. 64 w + 31 of the S buffer
+__device__ __forceinline__ uint32_t packed_col(int k) { return (uint32_t)(8 * k + (k >= 4 ? 32 : 0)); }
+
 __global__ void __launch_bounds__(NTHREADS, 1)
 ska_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_do,
                   const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
-                  __nv_bfloat16* __restrict__ dq, float* __restrict__ nlse2, float* __restrict__ dbuf,
-                  int T, int Tpad, int H, int W, float scale_log2, float scale, int n_qtiles) {
+                  __nv_bfloat16* __restrict__ dq, const float* __restrict__ nlse2,
+                  const float* __restrict__ dbuf, int T, int Tpad, int H, int W, float scale_log2,
+                  float scale, int n_qtiles) {
     using namespace qa;
     extern __shared__ unsigned char smem_raw[];
     unsigned char* smem = align1024(smem_raw);
@@ -172,35 +172,37 @@ ska_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
     const int t0 = qt * TILE;
     const int kt_lo = (t0 - W + 1 > 0 ? t0 - W + 1 : 0) / TILE;
     const int n_it = qt - kt_lo + 1;  // key tiles of the window
-    const int U = 2 * n_it;           // tiles over both sweeps
 
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + OFF_BAR);
-    uint64_t* full = bars;
-    uint64_t* empty = bars + NSLOT;
-    uint64_t* qfull = bars + 2 * NSLOT;
+    uint64_t* kfull = bars;
+    uint64_t* kempty = bars + KSLOT;
+    uint64_t* vfull = bars + 2 * KSLOT;
+    uint64_t* vempty = vfull + VSLOT;
+    uint64_t* qfull = vempty + VSLOT;
     uint64_t* sfull = qfull + 1;
-    uint64_t* sfree = sfull + 2;
-    uint64_t* done = sfree + 2;
+    uint64_t* pfull = sfull + 2;
+    uint64_t* dsready = pfull + 1;
+    uint64_t* done = dsready + 1;
     uint64_t* drain = done + 1;
-    uint64_t* xch = drain + 1;  // statistics exchange between the halves (bounded waits)
-    float* part = reinterpret_cast<float*>(smem + OFF_PART);
     uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + OFF_MISC);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + OFF_MISC + 4);
 
     if (threadIdx.x == 0) {
-        for (int s = 0; s < NSLOT; ++s) {
-            mbar_init(&full[s], 1);
-            mbar_init(&empty[s], 1);
+        for (int i = 0; i < KSLOT; ++i) {
+            mbar_init(&kfull[i], 1);
+            mbar_init(&kempty[i], 1);
+        }
+        for (int i = 0; i < VSLOT; ++i) {
+            mbar_init(&vfull[i], 1);
+            mbar_init(&vempty[i], 1);
         }
         mbar_init(qfull, 1);
-        for (int w = 0; w < 2; ++w) {
-            mbar_init(&sfull[w], 1);
-            mbar_init(&sfree[w], 128);
-        }
+        mbar_init(&sfull[0], 1);
+        mbar_init(&sfull[1], 1);
+        mbar_init(pfull, 1);
+        mbar_init(dsready, 256);
         mbar_init(done, 1);
         mbar_init(drain, 1);
-        mbar_init(&xch[0], 128);
-        mbar_init(&xch[1], 128);
         *abort_flag = 0;
         fence_mbar_init();
     }
@@ -212,7 +214,6 @@ ska_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
     __syncthreads();
     tc::fence_after_sync();
     const uint32_t tmem = *tmem_holder;
-    // TMEM columns: S [0,128) | dP [128,256) | dQ [256,384); half w of S / dP at +64 w
 
     if (warp == 8) {
         // ------------------------------- TMA producer -------------------------------
@@ -226,201 +227,151 @@ ska_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
                 tc::tma_load_3d(smem + OFF_Q + half * BOX_BYTES, &tm_q, half * 64, t0, bh, qfull);
                 tc::tma_load_3d(smem + OFF_DO + half * BOX_BYTES, &tm_do, half * 64, t0, bh, qfull);
             }
-            // load L: tile u = L / 2 of the two sweeps, K when L is even, V when odd
-            int L = 0;
-            for (; L < 2 * U; ++L) {
-                const int slot = L % NSLOT, use = L / NSLOT;
-                if (use > 0 && !wait_bar(&empty[slot], (uint32_t)((use - 1) & 1), abort_flag)) break;
-                const int key0 = (kt_lo + (L / 2) % n_it) * TILE;
-                unsigned char* dst = smem + OFF_RING + slot * TILE_BYTES;
-                mbar_arrive_expect_tx(&full[slot], TILE_BYTES);
-                for (int half = 0; half < 2; ++half) {
-                    if (L % 2 == 0)
-                        tc::tma_load_3d(dst + half * BOX_BYTES, &tm_k, half * 64, key0, b, &full[slot]);
-                    else
-                        tc::tma_load_3d(dst + half * BOX_BYTES, &tm_v, half * 64, key0, bh, &full[slot]);
-                }
+            int nk = 0, nv = 0;  // loads started
+            for (int u = 0; u < n_it; ++u) {  // K(u) then V(u), each into its own ring
+                const int key0 = (kt_lo + u) * TILE;
+                const int ks = u % KSLOT, vs = u % VSLOT;
+                if (u >= KSLOT && !wait_bar(&kempty[ks], (uint32_t)((u / KSLOT - 1) & 1), abort_flag)) break;
+                mbar_arrive_expect_tx(&kfull[ks], TILE_BYTES);
+                for (int half = 0; half < 2; ++half)
+                    tc::tma_load_3d(smem + OFF_K + ks * TILE_BYTES + half * BOX_BYTES, &tm_k, half * 64, key0, b,
+                                    &kfull[ks]);
+                ++nk;
+                if (u >= VSLOT && !wait_bar(&vempty[vs], (uint32_t)((u / VSLOT - 1) & 1), abort_flag)) break;
+                mbar_arrive_expect_tx(&vfull[vs], TILE_BYTES);
+                for (int half = 0; half < 2; ++half)
+                    tc::tma_load_3d(smem + OFF_V + vs * TILE_BYTES + half * BOX_BYTES, &tm_v, half * 64, key0, bh,
+                                    &vfull[vs]);
+                ++nv;
             }
-            // every copy started here has landed before the CTA can leave
+            // every copy started here has landed before the CTA can leave (an older tile of a
+            // ring was consumed by MMAs that completed before its slot was reused)
             mbar_wait_bounded(qfull, 0, kWaitLimit);
-            for (int Li = (L > NSLOT ? L - NSLOT : 0); Li < L; ++Li)
-                mbar_wait_bounded(&full[Li % NSLOT], (uint32_t)((Li / NSLOT) & 1), kWaitLimit);
+            for (int i = (nk > KSLOT ? nk - KSLOT : 0); i < nk; ++i)
+                mbar_wait_bounded(&kfull[i % KSLOT], (uint32_t)((i / KSLOT) & 1), kWaitLimit);
+            for (int i = (nv > VSLOT ? nv - VSLOT : 0); i < nv; ++i)
+                mbar_wait_bounded(&vfull[i % VSLOT], (uint32_t)((i / VSLOT) & 1), kWaitLimit);
         }
     } else if (warp == 9) {
-        // ------------------------------- MMA issuer -------------------------------
-        if (lane == 0) {
-            const uint32_t idesc_s = tc::idesc_bf16_f32(TILE, HALF, 0, 0);  // S half, both K-major
-            const uint32_t idesc_g = tc::idesc_bf16_f32(TILE, HD, 0, 1);    // dQ += dS K, K MN-major
-            const uint32_t d_hi = tc::desc_hi(tc::sdesc_sw128(0, 16, 1024));
-            const uint32_t q_lo = lo_kmajor(smem_u32(smem + OFF_Q));
-            const uint32_t do_lo = lo_kmajor(smem_u32(smem + OFF_DO));
-            auto ring = [&](int L) { return smem_u32(smem + OFF_RING + (L % NSLOT) * TILE_BYTES); };
-            bool ok = true;
-            auto acquire = [&](int L) {
-                ok = ok && wait_bar(&full[L % NSLOT], (uint32_t)((L / NSLOT) & 1), abort_flag);
-                tc::fence_after_sync();
-                return ok;
-            };
-            // S_w = Q K[64w, 64w+64)^T and dP_w = dO V[64w, 64w+64)^T of tile u
-            auto issue_sdp = [&](int w, int u) {
-                const uint32_t k_lo = lo_kmajor(ring(2 * u) + w * HALF_ROWS);
-                const uint32_t v_lo = lo_kmajor(ring(2 * u + 1) + w * HALF_ROWS);
-#pragma unroll
-                for (int k = 0; k < HD / 16; ++k)
-                    tc::mma_ss_lh(tmem + 64u * w, q_lo + kstep(k), d_hi, k_lo + kstep(k), d_hi, idesc_s, k > 0);
-#pragma unroll
-                for (int k = 0; k < HD / 16; ++k)
-                    tc::mma_ss_lh(tmem + 128u + 64u * w, do_lo + kstep(k), d_hi, v_lo + kstep(k), d_hi, idesc_s, k > 0);
-            };
-            // dQ += dS_w K[64w, 64w+64), dS_w packed in the first 32 columns of S half w
-            auto issue_dq = [&](int w, int u, bool first) {
-                const uint32_t k_lo = lo_mnmajor(ring(2 * u) + w * HALF_ROWS);
-#pragma unroll
-                for (int k = 0; k < HALF / 16; ++k)
-                    tc::mma_ts_lh(tmem + 256u, tmem + 64u * w + 8u * k, k_lo + mnstep(k), d_hi, idesc_g,
-                                  (first && k == 0) ? 0u : 1u);
-            };
-            ok = wait_bar(qfull, 0, abort_flag);
+        // ------------------------------- MMA issue (whole warp) -------------------------------
+        const uint32_t idesc = tc::idesc_bf16_f32(TILE, TILE, 0, 0);  // S, dP: both K-major
+        const uint32_t idesc_g = tc::idesc_bf16_f32(TILE, HD, 0, 1);  // dQ += dS K: K MN-major
+        const uint32_t d_hi = tc::desc_hi(tc::sdesc_sw128(0, 16, 1024));
+        const uint32_t q_lo = lo_kmajor(smem_u32(smem + OFF_Q));
+        const uint32_t do_lo = lo_kmajor(smem_u32(smem + OFF_DO));
+        auto kslot = [&](int u) { return smem_u32(smem + OFF_K + (u % KSLOT) * TILE_BYTES); };
+        auto vslot = [&](int u) { return smem_u32(smem + OFF_V + (u % VSLOT) * TILE_BYTES); };
+        bool ok = true;
+        auto acq_k = [&](int u) {
+            ok = ok && wait_bar_warp(&kfull[u % KSLOT], (uint32_t)((u / KSLOT) & 1), abort_flag);
             tc::fence_after_sync();
-            if (ok && acquire(0) && acquire(1)) {
-                issue_sdp(0, 0);
-                tc::mma_commit(&sfull[0]);
-                issue_sdp(1, 0);
-                tc::mma_commit(&sfull[1]);
-                tc::mma_commit(&empty[0]);  // tile 0 belongs to the first sweep: K and V are done
-                tc::mma_commit(&empty[1]);
-                for (int u = 0; u < U && ok; ++u) {
-                    const bool sweep2 = u >= n_it;
-                    for (int w = 0; w < 2; ++w) {
-                        if (!wait_bar(&sfree[w], (uint32_t)(u & 1), abort_flag)) { ok = false; break; }
-                        tc::fence_after_sync();
-                        if (sweep2) {
-                            issue_dq(w, u, u == n_it && w == 0);
-                            if (w == 1) tc::mma_commit(&empty[(2 * u) % NSLOT]);  // K of tile u
-                        }
-                        if (u + 1 < U) {
-                            if (w == 0 && !(acquire(2 * u + 2) && acquire(2 * u + 3))) break;
-                            issue_sdp(w, u + 1);
-                            tc::mma_commit(&sfull[w]);
-                            if (w == 1) {
-                                if (u + 1 < n_it) tc::mma_commit(&empty[(2 * u + 2) % NSLOT]);
-                                tc::mma_commit(&empty[(2 * u + 3) % NSLOT]);  // V of tile u + 1
-                            }
-                        }
-                    }
+            return ok;
+        };
+        auto acq_v = [&](int u) {
+            ok = ok && wait_bar_warp(&vfull[u % VSLOT], (uint32_t)((u / VSLOT) & 1), abort_flag);
+            tc::fence_after_sync();
+            return ok;
+        };
+        auto issue_s = [&](int u) {  // S(u) = Q K(u)^T
+            const uint32_t k_lo = lo_kmajor(kslot(u));
+#pragma unroll
+            for (int k = 0; k < HD / 16; ++k)
+                tc::mma_ss_lh_warp(tmem + s_col(u), q_lo + kstep(k), d_hi, k_lo + kstep(k), d_hi, idesc, k > 0);
+            tc::mma_commit_warp(&sfull[u & 1]);
+        };
+        auto issue_dp = [&](int u) {  // dP(u) = dO V(u)^T; V(u) is free once it completes
+            const uint32_t v_lo = lo_kmajor(vslot(u));
+#pragma unroll
+            for (int k = 0; k < HD / 16; ++k)
+                tc::mma_ss_lh_warp(tmem + 128u, do_lo + kstep(k), d_hi, v_lo + kstep(k), d_hi, idesc, k > 0);
+            tc::mma_commit_warp(pfull);
+            tc::mma_commit_warp(&vempty[u % VSLOT]);
+        };
+        auto issue_dq = [&](int u) {  // dQ += dS(u) K(u); K(u) is free once it completes
+            const uint32_t k_lo = lo_mnmajor(kslot(u));
+#pragma unroll
+            for (int k = 0; k < TILE / 16; ++k)
+                tc::mma_ts_lh_warp(tmem + 256u, tmem + s_col(u) + packed_col(k), k_lo + mnstep(k), d_hi, idesc_g,
+                                   (u > 0 || k > 0) ? 1u : 0u);
+            tc::mma_commit_warp(&kempty[u % KSLOT]);
+        };
+        ok = wait_bar_warp(qfull, 0, abort_flag);
+        tc::fence_after_sync();
+        if (ok && acq_k(0)) {
+            // order: S(0) dP(0) S(1) | dQ(0) dP(1) S(2) | dQ(1) dP(2) S(3) | ...
+            issue_s(0);
+            if (acq_v(0)) issue_dp(0);
+            if (ok && n_it > 1 && acq_k(1)) issue_s(1);
+            for (int u = 0; u < n_it && ok; ++u) {
+                if (!wait_bar_warp(dsready, (uint32_t)(u & 1), abort_flag)) { ok = false; break; }
+                tc::fence_after_sync();
+                issue_dq(u);
+                if (u + 1 < n_it) {
+                    if (!acq_v(u + 1)) break;
+                    issue_dp(u + 1);
                 }
-                if (ok) tc::mma_commit(done);
+                if (u + 2 < n_it) {
+                    if (!acq_k(u + 2)) break;
+                    issue_s(u + 2);  // into the buffer dQ(u) is reading: the pipe runs in order
+                }
             }
-            // every MMA this thread issued has completed before TMEM is released
-            tc::mma_commit(drain);
-            mbar_wait_bounded(drain, 0, kWaitLimit);
+            if (ok) tc::mma_commit_warp(done);
         }
+        // every MMA this warp issued has completed before TMEM is released
+        tc::mma_commit_warp(drain);
+        mbar_wait_bounded(drain, 0, kWaitLimit);
     } else {
         // ------------------------------- softmax warpgroups -------------------------------
-        const int w = warp / 4;                    // column half
+        const int w = warp / 4;                    // column half (keys 64 w .. 64 w + 63)
         const int row = threadIdx.x % 128;         // query row == TMEM lane
         const uint32_t lane_base = (uint32_t)(32 * (warp % 4)) << 16;
-        const uint32_t tS = tmem + lane_base + 64u * w;
-        const uint32_t tP = tS + 128u;
+        const uint32_t tP = tmem + lane_base + 128u + 64u * w;
         const uint32_t tQ = tmem + lane_base + 256u + 64u * w;
         const int t = t0 + row;
-        float m = -INFINITY, l = 0.f, Dacc = 0.f;  // first sweep, over this half's keys
-        float L2 = 0.f, Drow = 0.f;                 // the row's statistics for the second sweep
+        const float nL = nlse2[(int64_t)bh * Tpad + t];  // -inf past the end: p = 0
+        const float Dr = dbuf[(int64_t)bh * Tpad + t];
+        const float2 sl2 = make_float2(scale_log2, scale_log2), nl2 = make_float2(nL, nL);
+        const float2 d2 = make_float2(Dr, Dr);
         bool ok = true;
-        for (int u = 0; u < U; ++u) {
-            if (!wait_bar(&sfull[w], (uint32_t)(u & 1), abort_flag)) { ok = false; break; }
-            tc::fence_after_sync();
-            const int key0 = (kt_lo + u % n_it) * TILE + HALF * w;  // first key of this half
+        for (int u = 0; u < n_it; ++u) {
+            const uint32_t tS = tmem + lane_base + s_col(u) + 64u * w;
+            const int key0 = (kt_lo + u) * TILE + HALF * w;  // first key of this half
             const bool full_tile = key0 >= t0 + TILE - W && key0 + HALF - 1 <= t0;
-            const int lo = t - W + 1 - key0, hi = t - key0;           // valid columns [lo, hi]
-            const float2 sl2 = make_float2(scale_log2, scale_log2);
-            if (u < n_it) {
+            const int lo = t - W + 1 - key0, hi = t - key0;   // valid columns [lo, hi]
+            // phase 1: P from S
+            if (!wait_bar_warp(&sfull[u & 1], (uint32_t)((u >> 1) & 1), abort_flag)) { ok = false; break; }
+            tc::fence_after_sync();
+            float2 p2[32];
 #pragma unroll
-                for (int c = 0; c < 2; ++c) {
-                    uint32_t s[32], dp[32];
-                    tc::tmem_ld32(tS + 32u * c, s);
-                    tc::tmem_ld32(tP + 32u * c, dp);
-                    tc::tmem_wait_ld();
-                    if (!full_tile) mask_chunk(s, c, lo, hi);
-                    // online update: the running maximum moves to the chunk's maximum if larger
-                    const float mn = fmaxf(m, max32(s) * scale_log2);
-                    const float alpha = mn == -INFINITY ? 1.f : tc::ex2(m - mn);  // 0 when m = -inf
-                    l *= alpha;
-                    Dacc *= alpha;
-                    m = mn;
-                    const float mu = m == -INFINITY ? 0.f : m;  // nothing visible yet: p = 0
-                    const float2 nm2 = make_float2(-mu, -mu);
-                    float2 l4[4] = {{0.f, 0.f}, {0.f, 0.f}, {0.f, 0.f}, {0.f, 0.f}};
-                    float2 d4[4] = {{0.f, 0.f}, {0.f, 0.f}, {0.f, 0.f}, {0.f, 0.f}};
+            for (int c = 0; c < 2; ++c) {
+                uint32_t s[32];
+                tc::tmem_ld32(tS + 32u * c, s);
+                tc::tmem_wait_ld();
+                if (!full_tile) mask_chunk(s, c, lo, hi);
 #pragma unroll
-                    for (int i = 0; i < 16; ++i) {
-                        const float2 p2 = ex2x2(f2fma(raw2(s, 2 * i), sl2, nm2));
-                        l4[i & 3] = f2add(l4[i & 3], p2);
-                        d4[i & 3] = f2fma(p2, raw2(dp, 2 * i), d4[i & 3]);
-                    }
-                    const float2 ls = f2add(f2add(l4[0], l4[1]), f2add(l4[2], l4[3]));
-                    const float2 ds = f2add(f2add(d4[0], d4[1]), f2add(d4[2], d4[3]));
-                    l += ls.x + ls.y;
-                    Dacc += ds.x + ds.y;
-                }
-                tc::fence_before_sync();
-                mbar_arrive(&sfree[w]);
-                if (u == n_it - 1) {
-                    // merge the two halves' statistics: half 1 hands its (m, l, D) to half 0,
-                    // which forms the row's log-sum-exp and D and hands them back
-                    if (w == 1) {
-                        part[row] = m;
-                        part[TILE + row] = l;
-                        part[2 * TILE + row] = Dacc;
-                        mbar_arrive(&xch[0]);
-                        if (!wait_bar(&xch[1], 0, abort_flag)) { ok = false; break; }
-                        L2 = part[row];
-                        Drow = part[TILE + row];
-                    } else {
-                        if (!wait_bar(&xch[0], 0, abort_flag)) { ok = false; break; }
-                        const float m1 = part[row], l1 = part[TILE + row], D1 = part[2 * TILE + row];
-                        const float M = fmaxf(m, m1);
-                        const float a0 = tc::ex2(m - M), a1 = tc::ex2(m1 - M);
-                        const float lt = l * a0 + l1 * a1, Dt = Dacc * a0 + D1 * a1;
-                        if (t < T) {
-                            L2 = M + log2f(lt);
-                            Drow = Dt / lt;
-                        } else {  // past the end: no probability mass, no gradient
-                            L2 = INFINITY;
-                            Drow = 0.f;
-                        }
-                        nlse2[(int64_t)bh * Tpad + t] = -L2;
-                        dbuf[(int64_t)bh * Tpad + t] = Drow;
-                        part[row] = L2;
-                        part[TILE + row] = Drow;
-                        mbar_arrive(&xch[1]);
-                    }
-                }
-            } else {
-                uint32_t pk[32];
-                const float2 nl2 = make_float2(-L2, -L2), d2 = make_float2(Drow, Drow);
-#pragma unroll
-                for (int c = 0; c < 2; ++c) {
-                    uint32_t s[32], dp[32];
-                    tc::tmem_ld32(tS + 32u * c, s);
-                    tc::tmem_ld32(tP + 32u * c, dp);
-                    tc::tmem_wait_ld();
-                    if (!full_tile) mask_chunk(s, c, lo, hi);
-#pragma unroll
-                    for (int i = 0; i < 16; ++i) {
-                        const float2 p2 = ex2x2(f2fma(raw2(s, 2 * i), sl2, nl2));
-                        const float2 ds = f2mul(p2, f2sub(raw2(dp, 2 * i), d2));
-                        pk[16 * c + i] = pack_bf16x2(ds.x, ds.y);
-                    }
-                }
-                tc::tmem_st32(tS, pk);
-                tc::tmem_wait_st();
-                tc::fence_before_sync();
-                mbar_arrive(&sfree[w]);
+                for (int i = 0; i < 16; ++i) p2[16 * c + i] = ex2x2(f2fma(raw2(s, 2 * i), sl2, nl2));
             }
+            // phase 2: dS = P (dP - D), packed over this half's first 32 columns of the S buffer
+            if (!wait_bar_warp(pfull, (uint32_t)(u & 1), abort_flag)) { ok = false; break; }
+            tc::fence_after_sync();
+#pragma unroll
+            for (int c = 0; c < 2; ++c) {
+                uint32_t dp[32], pk[16];
+                tc::tmem_ld32(tP + 32u * c, dp);
+                tc::tmem_wait_ld();
+#pragma unroll
+                for (int i = 0; i < 16; ++i) {
+                    const float2 ds = f2mul(p2[16 * c + i], f2sub(raw2(dp, 2 * i), d2));
+                    pk[i] = pack_bf16x2(ds.x, ds.y);
+                }
+                tc::tmem_st16(tS + 16u * c, pk);
+            }
+            tc::tmem_wait_st();
+            tc::fence_before_sync();
+            mbar_arrive(dsready);
         }
         // epilogue: dq = scale * dQ -> bf16, this half's 64 channels
-        if (ok && wait_bar(done, 0, abort_flag)) {
+        if (ok && wait_bar_warp(done, 0, abort_flag)) {
             tc::fence_after_sync();
             __nv_bfloat16* out = dq + ((int64_t)bh * T + t) * HD + HALF * w;
 #pragma unroll
@@ -448,23 +399,25 @@ ska_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
 }
 
 // ============================================================================================
-// Launch 2: key tiles (dV per head, dK partial per head group)
+// Launch 3: key tiles (dV per head, dK partial per head group)
 // ============================================================================================
 namespace ka {
 constexpr int OFF_K = 0;
 constexpr int OFF_V = TILE_BYTES;
 constexpr int OFF_RING = 2 * TILE_BYTES;             // 2 slots of (Q tile, dO tile)
 constexpr int UNIT_BYTES = 2 * TILE_BYTES;
-constexpr int OFF_STAT = OFF_RING + 2 * UNIT_BYTES;  // 2 slots of (lse2[128], D[128]) fp32
+constexpr int OFF_STAT = OFF_RING + 2 * UNIT_BYTES;  // 2 slots of (-lse2[128], D[128]) fp32
 constexpr int STAT_BYTES = 2 * TILE * 4;
 constexpr int OFF_BAR = OFF_STAT + 2 * STAT_BYTES;
-// kfull, vfull, vempty, full[2], empty[2], sfull[2], sfree[2], dvdone, dvfree, done, drain
+// kfull, vfull, vempty, full[2], empty[2], sfull, pfull, pready, dsready, dvdone, dvfree, done, drain
 constexpr int NBAR = 15;
 constexpr int OFF_MISC = OFF_BAR + 8 * NBAR;
 constexpr int SMEM = OFF_MISC + 16 + 1024;
 static_assert(SMEM <= 232448, "shared memory");
 }  // namespace ka
 
+// TMEM columns: S^T [0,128) | dP^T [128,256) | dV [256,384) | dK [384,512). P^T and dS^T are
+// packed over the first 32 columns of each warpgroup's half of S^T and dP^T (packed_col).
 __global__ void __launch_bounds__(NTHREADS, 1)
 ska_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_do,
                     const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
@@ -491,7 +444,9 @@ ska_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
     uint64_t* full = bars + 3;
     uint64_t* empty = bars + 5;
     uint64_t* sfull = bars + 7;
-    uint64_t* sfree = bars + 9;
+    uint64_t* pfull = bars + 8;
+    uint64_t* pready = bars + 9;
+    uint64_t* dsready = bars + 10;
     uint64_t* dvdone = bars + 11;
     uint64_t* dvfree = bars + 12;
     uint64_t* done = bars + 13;
@@ -503,12 +458,14 @@ ska_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
         mbar_init(kfull, 1);
         mbar_init(vfull, 1);
         mbar_init(vempty, 1);
-        for (int s = 0; s < 2; ++s) {
-            mbar_init(&full[s], 1);
-            mbar_init(&empty[s], 1);
-            mbar_init(&sfull[s], 1);
-            mbar_init(&sfree[s], 128);
+        for (int s2 = 0; s2 < 2; ++s2) {
+            mbar_init(&full[s2], 1);
+            mbar_init(&empty[s2], 1);
         }
+        mbar_init(sfull, 1);
+        mbar_init(pfull, 1);
+        mbar_init(pready, 256);
+        mbar_init(dsready, 256);
         mbar_init(dvdone, 1);
         mbar_init(dvfree, 256);
         mbar_init(done, 1);
@@ -524,7 +481,6 @@ ska_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
     __syncthreads();
     tc::fence_after_sync();
     const uint32_t tmem = *tmem_holder;
-    // TMEM columns: S^T [0,128) | dP^T [128,256) | dV [256,384) | dK [384,512)
 
     if (warp == 8) {
         // ------------------------------- TMA producer -------------------------------
@@ -568,82 +524,78 @@ ska_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                 mbar_wait_bounded(&full[ui % 2], (uint32_t)((ui / 2) & 1), kWaitLimit);
         }
     } else if (warp == 9) {
-        // ------------------------------- MMA issuer -------------------------------
-        if (lane == 0) {
-            const uint32_t idesc_s = tc::idesc_bf16_f32(TILE, HALF, 0, 0);  // S^T half, both K-major
-            const uint32_t idesc_g = tc::idesc_bf16_f32(TILE, HD, 0, 1);    // gradients, B MN-major
-            const uint32_t d_hi = tc::desc_hi(tc::sdesc_sw128(0, 16, 1024));
-            const uint32_t k_lo = lo_kmajor(smem_u32(smem + OFF_K));
-            const uint32_t v_lo = lo_kmajor(smem_u32(smem + OFF_V));
-            auto unit = [&](int u) { return smem_u32(smem + OFF_RING + (u % 2) * UNIT_BYTES); };
-            bool ok = true;
-            auto acquire = [&](uint64_t* bar, uint32_t parity) {
-                ok = ok && wait_bar(bar, parity, abort_flag);
-                tc::fence_after_sync();
-                return ok;
-            };
-            // S^T_w = K Q[64w, 64w+64)^T and dP^T_w = V dO[64w, 64w+64)^T of pair u
-            auto issue_sdp = [&](int w, int u) {
-                const uint32_t q_lo = lo_kmajor(unit(u) + w * HALF_ROWS);
-                const uint32_t o_lo = lo_kmajor(unit(u) + TILE_BYTES + w * HALF_ROWS);
+        // ------------------------------- MMA issue (whole warp) -------------------------------
+        const uint32_t idesc = tc::idesc_bf16_f32(TILE, TILE, 0, 0);  // S^T, dP^T: both K-major
+        const uint32_t idesc_g = tc::idesc_bf16_f32(TILE, HD, 0, 1);  // dV, dK: B MN-major
+        const uint32_t d_hi = tc::desc_hi(tc::sdesc_sw128(0, 16, 1024));
+        const uint32_t k_lo = lo_kmajor(smem_u32(smem + OFF_K));
+        const uint32_t v_lo = lo_kmajor(smem_u32(smem + OFF_V));
+        auto unit = [&](int u) { return smem_u32(smem + OFF_RING + (u % 2) * UNIT_BYTES); };
+        bool ok = true;
+        auto acquire = [&](uint64_t* bar, uint32_t parity) {
+            ok = ok && wait_bar_warp(bar, parity, abort_flag);
+            tc::fence_after_sync();
+            return ok;
+        };
+        auto issue_st = [&](int u) {  // S^T(u) = K Q(u)^T
+            const uint32_t q_lo = lo_kmajor(unit(u));
 #pragma unroll
-                for (int k = 0; k < HD / 16; ++k)
-                    tc::mma_ss_lh(tmem + 64u * w, k_lo + kstep(k), d_hi, q_lo + kstep(k), d_hi, idesc_s, k > 0);
+            for (int k = 0; k < HD / 16; ++k)
+                tc::mma_ss_lh_warp(tmem, k_lo + kstep(k), d_hi, q_lo + kstep(k), d_hi, idesc, k > 0);
+            tc::mma_commit_warp(sfull);
+        };
+        auto issue_dpt = [&](int u) {  // dP^T(u) = V dO(u)^T
+            const uint32_t o_lo = lo_kmajor(unit(u) + TILE_BYTES);
 #pragma unroll
-                for (int k = 0; k < HD / 16; ++k)
-                    tc::mma_ss_lh(tmem + 128u + 64u * w, v_lo + kstep(k), d_hi, o_lo + kstep(k), d_hi, idesc_s, k > 0);
-            };
-            // dV += P^T_w dO[64w, 64w+64) and dK += dS^T_w Q[64w, 64w+64), with P^T_w and dS^T_w
-            // packed in the first 32 columns of the S^T and dP^T halves
-            auto issue_grad = [&](int w, int u, bool first_dv, bool first_dk) {
-                const uint32_t q_lo = lo_mnmajor(unit(u) + w * HALF_ROWS);
-                const uint32_t o_lo = lo_mnmajor(unit(u) + TILE_BYTES + w * HALF_ROWS);
+            for (int k = 0; k < HD / 16; ++k)
+                tc::mma_ss_lh_warp(tmem + 128u, v_lo + kstep(k), d_hi, o_lo + kstep(k), d_hi, idesc, k > 0);
+            tc::mma_commit_warp(pfull);
+            if (u % n_q == n_q - 1) tc::mma_commit_warp(vempty);  // the head's last use of V
+        };
+        auto issue_dv = [&](int u, bool first) {  // dV += P^T(u) dO(u)
+            const uint32_t o_lo = lo_mnmajor(unit(u) + TILE_BYTES);
 #pragma unroll
-                for (int k = 0; k < HALF / 16; ++k)
-                    tc::mma_ts_lh(tmem + 256u, tmem + 64u * w + 8u * k, o_lo + mnstep(k), d_hi, idesc_g,
-                                  (first_dv && k == 0) ? 0u : 1u);
+            for (int k = 0; k < TILE / 16; ++k)
+                tc::mma_ts_lh_warp(tmem + 256u, tmem + packed_col(k), o_lo + mnstep(k), d_hi, idesc_g,
+                                   (first && k == 0) ? 0u : 1u);
+        };
+        auto issue_dk = [&](int u) {  // dK += dS^T(u) Q(u); the unit's slot is free afterwards
+            const uint32_t q_lo = lo_mnmajor(unit(u));
 #pragma unroll
-                for (int k = 0; k < HALF / 16; ++k)
-                    tc::mma_ts_lh(tmem + 384u, tmem + 128u + 64u * w + 8u * k, q_lo + mnstep(k), d_hi, idesc_g,
-                                  (first_dk && k == 0) ? 0u : 1u);
-            };
-            if (acquire(kfull, 0) && acquire(vfull, 0) && acquire(&full[0], 0)) {
-                issue_sdp(0, 0);
-                tc::mma_commit(&sfull[0]);
-                issue_sdp(1, 0);
-                tc::mma_commit(&sfull[1]);
-                if (n_q == 1) tc::mma_commit(vempty);
-                for (int u = 0; u < U && ok; ++u) {
-                    const int hi = u / n_q;
-                    const bool first_of_head = u % n_q == 0, last_of_head = u % n_q == n_q - 1;
-                    for (int w = 0; w < 2; ++w) {
-                        if (!acquire(&sfree[w], (uint32_t)(u & 1))) break;
-                        if (w == 0 && first_of_head && hi > 0 && !acquire(dvfree, (uint32_t)((hi - 1) & 1)))
-                            break;
-                        issue_grad(w, u, first_of_head && w == 0, u == 0 && w == 0);
-                        if (w == 1) {
-                            tc::mma_commit(&empty[u % 2]);
-                            if (last_of_head) tc::mma_commit(dvdone);
-                        }
-                        if (u + 1 < U) {
-                            if (w == 0) {
-                                if (!acquire(&full[(u + 1) % 2], (uint32_t)(((u + 1) / 2) & 1))) break;
-                                if ((u + 1) % n_q == 0 && !acquire(vfull, (uint32_t)(((u + 1) / n_q) & 1))) break;
-                            }
-                            issue_sdp(w, u + 1);
-                            tc::mma_commit(&sfull[w]);
-                            if (w == 1 && (u + 1) % n_q == n_q - 1) tc::mma_commit(vempty);
-                        }
-                    }
+            for (int k = 0; k < TILE / 16; ++k)
+                tc::mma_ts_lh_warp(tmem + 384u, tmem + 128u + packed_col(k), q_lo + mnstep(k), d_hi, idesc_g,
+                                   (u > 0 || k > 0) ? 1u : 0u);
+            tc::mma_commit_warp(&empty[u % 2]);
+        };
+        if (acquire(kfull, 0) && acquire(vfull, 0) && acquire(&full[0], 0)) {
+            // order: S^T(0) dP^T(0) | dV(0) S^T(1) dK(0) dP^T(1) | dV(1) S^T(2) dK(1) dP^T(2) | ...
+            issue_st(0);
+            issue_dpt(0);
+            for (int u = 0; u < U && ok; ++u) {
+                const int hi = u / n_q;
+                const bool first = u % n_q == 0, last = u % n_q == n_q - 1;
+                if (!acquire(pready, (uint32_t)(u & 1))) break;
+                if (first && hi > 0 && !acquire(dvfree, (uint32_t)((hi - 1) & 1))) break;
+                issue_dv(u, first);
+                if (last) tc::mma_commit_warp(dvdone);
+                if (u + 1 < U) {
+                    if (!acquire(&full[(u + 1) % 2], (uint32_t)(((u + 1) / 2) & 1))) break;
+                    issue_st(u + 1);  // over P^T(u), which dV(u) reads first: the pipe runs in order
                 }
-                if (ok) tc::mma_commit(done);
+                if (!acquire(dsready, (uint32_t)(u & 1))) break;
+                issue_dk(u);
+                if (u + 1 < U) {
+                    if ((u + 1) % n_q == 0 && !acquire(vfull, (uint32_t)(((u + 1) / n_q) & 1))) break;
+                    issue_dpt(u + 1);
+                }
             }
-            tc::mma_commit(drain);
-            mbar_wait_bounded(drain, 0, kWaitLimit);
+            if (ok) tc::mma_commit_warp(done);
         }
+        tc::mma_commit_warp(drain);
+        mbar_wait_bounded(drain, 0, kWaitLimit);
     } else {
         // ------------------------------- softmax warpgroups -------------------------------
-        const int w = warp / 4;                    // column half (queries 64w .. 64w + 63)
+        const int w = warp / 4;                    // column half (queries 64 w .. 64 w + 63)
         const int row = threadIdx.x % 128;         // key row == TMEM lane
         const uint32_t lane_base = (uint32_t)(32 * (warp % 4)) << 16;
         const uint32_t tS = tmem + lane_base + 64u * w;
@@ -651,47 +603,63 @@ ska_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
         const uint32_t tV = tmem + lane_base + 256u + 64u * w;
         const uint32_t tK = tmem + lane_base + 384u + 64u * w;
         const int key = j0 + row;
+        const float2 sl2 = make_float2(scale_log2, scale_log2);
         bool ok = true;
         for (int u = 0; u < U; ++u) {
             const int hi = u / n_q, qt = qt_lo + u % n_q;
             const int tq0 = qt * TILE + HALF * w;  // first query of this half
-            if (!wait_bar(&sfull[w], (uint32_t)(u & 1), abort_flag)) { ok = false; break; }
-            tc::fence_after_sync();
             const float* st = reinterpret_cast<const float*>(smem + OFF_STAT + (u % 2) * STAT_BYTES) + HALF * w;
             const bool full_tile = tq0 >= j0 + TILE - 1 && tq0 + HALF - 1 <= j0 + W - 1;
             const int lo = key - tq0, hi_e = key + W - 1 - tq0;  // valid columns [lo, hi_e]
-            // P^T and dS^T of each 32-column chunk go, packed, over the first 16 columns of the
-            // chunk's own 32 (already read): chunk c at columns 16 c of the S^T / dP^T half
-            const float2 sl2 = make_float2(scale_log2, scale_log2);
+            // phase 1: P^T from S^T (the unit's statistics landed with its tiles)
+            if (!wait_bar_warp(sfull, (uint32_t)(u & 1), abort_flag)) { ok = false; break; }
+            tc::fence_after_sync();
+            float2 p2[32];
 #pragma unroll
             for (int c = 0; c < 2; ++c) {
-                uint32_t s[32], dp[32], pp[16], pd[16];
+                uint32_t s[32], pk[16];
                 tc::tmem_ld32(tS + 32u * c, s);
-                tc::tmem_ld32(tP + 32u * c, dp);
                 tc::tmem_wait_ld();
                 if (!full_tile) mask_chunk(s, c, lo, hi_e);
 #pragma unroll
                 for (int e4 = 0; e4 < 32; e4 += 4) {
                     const float4 L4 = *reinterpret_cast<const float4*>(st + 32 * c + e4);  // -lse2
-                    const float4 D4 = *reinterpret_cast<const float4*>(st + TILE + 32 * c + e4);
                     const float2 pa = ex2x2(f2fma(raw2(s, e4), sl2, make_float2(L4.x, L4.y)));
                     const float2 pb = ex2x2(f2fma(raw2(s, e4 + 2), sl2, make_float2(L4.z, L4.w)));
-                    const float2 da = f2mul(pa, f2sub(raw2(dp, e4), make_float2(D4.x, D4.y)));
-                    const float2 db = f2mul(pb, f2sub(raw2(dp, e4 + 2), make_float2(D4.z, D4.w)));
-                    pp[e4 / 2] = pack_bf16x2(pa.x, pa.y);
-                    pp[e4 / 2 + 1] = pack_bf16x2(pb.x, pb.y);
-                    pd[e4 / 2] = pack_bf16x2(da.x, da.y);
-                    pd[e4 / 2 + 1] = pack_bf16x2(db.x, db.y);
+                    p2[16 * c + e4 / 2] = pa;
+                    p2[16 * c + e4 / 2 + 1] = pb;
+                    pk[e4 / 2] = pack_bf16x2(pa.x, pa.y);
+                    pk[e4 / 2 + 1] = pack_bf16x2(pb.x, pb.y);
                 }
-                tc::tmem_st16(tS + 16u * c, pp);
-                tc::tmem_st16(tP + 16u * c, pd);
+                tc::tmem_st16(tS + 16u * c, pk);
             }
             tc::tmem_wait_st();
             tc::fence_before_sync();
-            mbar_arrive(&sfree[w]);
+            mbar_arrive(pready);
+            // phase 2: dS^T = P^T (dP^T - D)
+            if (!wait_bar_warp(pfull, (uint32_t)(u & 1), abort_flag)) { ok = false; break; }
+            tc::fence_after_sync();
+#pragma unroll
+            for (int c = 0; c < 2; ++c) {
+                uint32_t dp[32], pk[16];
+                tc::tmem_ld32(tP + 32u * c, dp);
+                tc::tmem_wait_ld();
+#pragma unroll
+                for (int e4 = 0; e4 < 32; e4 += 4) {
+                    const float4 D4 = *reinterpret_cast<const float4*>(st + TILE + 32 * c + e4);
+                    const float2 da = f2mul(p2[16 * c + e4 / 2], f2sub(raw2(dp, e4), make_float2(D4.x, D4.y)));
+                    const float2 db = f2mul(p2[16 * c + e4 / 2 + 1], f2sub(raw2(dp, e4 + 2), make_float2(D4.z, D4.w)));
+                    pk[e4 / 2] = pack_bf16x2(da.x, da.y);
+                    pk[e4 / 2 + 1] = pack_bf16x2(db.x, db.y);
+                }
+                tc::tmem_st16(tP + 16u * c, pk);
+            }
+            tc::tmem_wait_st();
+            tc::fence_before_sync();
+            mbar_arrive(dsready);
             if (u % n_q == n_q - 1) {
                 // the head's dV rows are complete: store them and release the accumulator
-                if (!wait_bar(dvdone, (uint32_t)(hi & 1), abort_flag)) { ok = false; break; }
+                if (!wait_bar_warp(dvdone, (uint32_t)(hi & 1), abort_flag)) { ok = false; break; }
                 tc::fence_after_sync();
                 __nv_bfloat16* out = dv + (((int64_t)b * H + h0 + hi) * T + key) * HD + HALF * w;
 #pragma unroll
@@ -714,7 +682,7 @@ ska_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
             }
         }
         // epilogue: this group's dK partial (unscaled fp32), this half's 64 channels
-        if (ok && wait_bar(done, 0, abort_flag)) {
+        if (ok && wait_bar_warp(done, 0, abort_flag)) {
             tc::fence_after_sync();
             float* out = dk_part + (((int64_t)grp * B + b) * T + key) * HD + HALF * w;
 #pragma unroll
@@ -740,7 +708,7 @@ ska_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
 }
 
 // ============================================================================================
-// Launch 3: dk = scale * sum over head groups of the partials (group order fixed)
+// Launch 4: dk = scale * sum over head groups of the partials (group order fixed)
 // ============================================================================================
 __global__ void __launch_bounds__(256)
 ska_bwd_dk_reduce(const float* __restrict__ part, __nv_bfloat16* __restrict__ dk, int64_t n4, int G,
@@ -796,12 +764,15 @@ cudaError_t swska_backward_tc_launch(const SkaBackwardArgs& a, cudaStream_t stre
     const int B = a.B, H = a.H, T = a.T;
     const int W = a.W < T ? a.W : T;  // a window longer than the sequence is the whole prefix
     const int64_t Tpad = swska_backward_tc_tpad(T);
-    float* lse2 = static_cast<float*>(a.workspace);
-    float* dbuf = lse2 + (size_t)B * H * Tpad;
+    float* nlse2 = static_cast<float*>(a.workspace);
+    float* dbuf = nlse2 + (size_t)B * H * Tpad;
     float* part = dbuf + (size_t)B * H * Tpad;
     if (B > 65535 || H > 65535) return cudaErrorInvalidConfiguration;
+    // launch 1: the forward in statistics mode (row log-sum-exp and D, no output stored)
+    cudaError_t e = swska_prefill_tc_stats_launch(a.q, a.k, a.v, nullptr, a.dO, nlse2, dbuf, Tpad, B, H, T, W,
+                                                  a.scale, stream);
+    if (e != cudaSuccess) return e;
     CUtensorMap mq, mdo, mk, mv;
-    cudaError_t e;
     if ((e = make_tmap_bf16_3d(&mq, a.q, HD, (uint64_t)T, (uint64_t)B * H, 64, TILE)) != cudaSuccess) return e;
     if ((e = make_tmap_bf16_3d(&mdo, a.dO, HD, (uint64_t)T, (uint64_t)B * H, 64, TILE)) != cudaSuccess) return e;
     if ((e = make_tmap_bf16_3d(&mk, a.k, HD, (uint64_t)T, (uint64_t)B, 64, TILE)) != cudaSuccess) return e;
@@ -815,10 +786,10 @@ cudaError_t swska_backward_tc_launch(const SkaBackwardArgs& a, cudaStream_t stre
     const int nqt = (int)(Tpad / TILE);
     const float sl = a.scale * kLog2e;
     ska_bwd_dq_kernel<<<dim3((unsigned)nqt, (unsigned)H, (unsigned)B), NTHREADS, qa::SMEM, stream>>>(
-        mq, mdo, mk, mv, static_cast<__nv_bfloat16*>(a.dq), lse2, dbuf, T, (int)Tpad, H, W, sl, a.scale, nqt);
+        mq, mdo, mk, mv, static_cast<__nv_bfloat16*>(a.dq), nlse2, dbuf, T, (int)Tpad, H, W, sl, a.scale, nqt);
     const int G = swska_backward_tc_groups(B, H, T);
     ska_bwd_dkdv_kernel<<<dim3((unsigned)nqt, (unsigned)G, (unsigned)B), NTHREADS, ka::SMEM, stream>>>(
-        mq, mdo, mk, mv, lse2, dbuf, static_cast<__nv_bfloat16*>(a.dv), part, B, T, (int)Tpad, H, H / G, W,
+        mq, mdo, mk, mv, nlse2, dbuf, static_cast<__nv_bfloat16*>(a.dv), part, B, T, (int)Tpad, H, H / G, W,
         sl, nqt);
     const int64_t n4 = (int64_t)B * T * HD / 4;
     const int64_t want = (n4 + 255) / 256, cap = 8 * (int64_t)sm_count();

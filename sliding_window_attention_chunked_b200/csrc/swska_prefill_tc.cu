@@ -97,10 +97,14 @@ __device__ __forceinline__ float2 fadd2(float2 a, float2 b) {
     return d;
 }
 
+// STATS: the backward's statistics mode (row log-sum-exp and D = dO . o, output optional); a
+// separate instantiation so the plain forward carries none of its registers
+template <bool STATS>
 __global__ void __launch_bounds__(NTHREADS, 1)
 swska_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                 const __grid_constant__ CUtensorMap tm_v, __nv_bfloat16* __restrict__ o, int T,
-                int H, int W, float scale_log2, int n_qtiles) {
+                int H, int W, float scale_log2, int n_qtiles, const __nv_bfloat16* __restrict__ dO,
+                float* __restrict__ nlse2, float* __restrict__ dbuf, int Tpad) {
     extern __shared__ unsigned char smem_raw[];
     unsigned char* smem = reinterpret_cast<unsigned char*>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -347,17 +351,21 @@ swska_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             tc::fence_before_sync();
             mbar_arrive(&pfull[h]);
         }
-        // epilogue: O / l -> bf16 rows
+        // epilogue: O / l -> bf16 rows. With statistics requested (the backward's first step), each
+        // row also gets its negated base-2 log-sum-exp and D = dO . o from the fp32 O in TMEM
+        // (-inf and 0 for rows past the end of the sequence), and O itself is stored only if asked.
         if (ok && wait_bar(&odone[h], 0, abort_flag)) {
             tc::fence_after_sync();
             const float inv = 1.f / l_run;
-            __nv_bfloat16* orow = o + ((int64_t)(b * H + 2 * hp + h) * T + t) * HD;
+            const bool live = t < T && 2 * hp + h < H;  // an odd H's last pair computes one head twice
+            const int64_t orow_i = ((int64_t)(b * H + 2 * hp + h) * T + t) * HD;
+            float dacc = 0.f;
 #pragma unroll
             for (int cb = 0; cb < HD; cb += 32) {
                 uint32_t r[32];
                 tc::tmem_ld32(tO + cb, r);
                 tc::tmem_wait_ld();
-                if (t < T && 2 * hp + h < H) {  // an odd H's last pair computes one head twice
+                if (live && (!STATS || o != nullptr)) {
 #pragma unroll
                     for (int i = 0; i < 32; i += 8) {
                         uint4 u;
@@ -365,9 +373,23 @@ swska_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                         u.y = pack_bf16x2(__uint_as_float(r[i + 2]) * inv, __uint_as_float(r[i + 3]) * inv);
                         u.z = pack_bf16x2(__uint_as_float(r[i + 4]) * inv, __uint_as_float(r[i + 5]) * inv);
                         u.w = pack_bf16x2(__uint_as_float(r[i + 6]) * inv, __uint_as_float(r[i + 7]) * inv);
-                        *reinterpret_cast<uint4*>(orow + cb + i) = u;
+                        *reinterpret_cast<uint4*>(o + orow_i + cb + i) = u;
                     }
                 }
+                if (STATS && live) {
+#pragma unroll
+                    for (int i = 0; i < 32; i += 8) {
+                        float g[8];
+                        load8(dO + orow_i + cb + i, g);
+#pragma unroll
+                        for (int e = 0; e < 8; ++e) dacc = fmaf(g[e], __uint_as_float(r[i + e]) * inv, dacc);
+                    }
+                }
+            }
+            if (STATS && 2 * hp + h < H) {
+                const int64_t srow = (int64_t)(b * H + 2 * hp + h) * Tpad + t;
+                nlse2[srow] = live ? -(m_run + log2f(l_run)) : -INFINITY;
+                dbuf[srow] = live ? dacc : 0.f;
             }
         }
     }
@@ -386,19 +408,29 @@ bool swska_prefill_tc_supported(int H, int T, int dk, int dv) {
 
 cudaError_t swska_prefill_tc_launch(const void* q, const void* k, const void* v, void* o, int B,
                                     int H, int T, int window, float scale, cudaStream_t stream) {
+    return swska_prefill_tc_stats_launch(q, k, v, o, nullptr, nullptr, nullptr, 0, B, H, T, window, scale,
+                                         stream);
+}
+
+cudaError_t swska_prefill_tc_stats_launch(const void* q, const void* k, const void* v, void* o,
+                                          const void* dO, float* nlse2, float* dbuf, int64_t Tpad, int B,
+                                          int H, int T, int window, float scale, cudaStream_t stream) {
     CUtensorMap mq, mk, mv;
     cudaError_t e;
     if ((e = make_tmap_bf16_3d(&mq, q, HD, (uint64_t)T, (uint64_t)B * H, 64, BM)) != cudaSuccess) return e;
     if ((e = make_tmap_bf16_3d(&mk, k, HD, (uint64_t)T, (uint64_t)B, 64, BN)) != cudaSuccess) return e;
     if ((e = make_tmap_bf16_3d(&mv, v, HD, (uint64_t)T, (uint64_t)B * H, 64, BN)) != cudaSuccess) return e;
-    e = cudaFuncSetAttribute(swska_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
+    const bool stats = nlse2 != nullptr;
+    e = stats ? cudaFuncSetAttribute(swska_tc_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES)
+              : cudaFuncSetAttribute(swska_tc_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
     if (e != cudaSuccess) return e;
     const int n_qtiles = (T + BM - 1) / BM;
     if (B > 65535 || (H + 1) / 2 > 65535) return cudaErrorInvalidConfiguration;
     dim3 grid((unsigned)n_qtiles, (unsigned)((H + 1) / 2), (unsigned)B);
-    swska_tc_kernel<<<grid, NTHREADS, SMEM_BYTES, stream>>>(
+    auto* kern = stats ? swska_tc_kernel<true> : swska_tc_kernel<false>;
+    kern<<<grid, NTHREADS, SMEM_BYTES, stream>>>(
         mq, mk, mv, static_cast<__nv_bfloat16*>(o), T, H, window, scale * 1.4426950408889634f,
-        n_qtiles);
+        n_qtiles, static_cast<const __nv_bfloat16*>(dO), nlse2, dbuf, (int)Tpad);
     note_launches(1);
     return cudaGetLastError();
 }
