@@ -23,11 +23,13 @@
 // Every MMA is M = 128, N = 128, K = 16 (an N = 64 MMA costs most of an N = 128 one to issue).
 // The two softmax warpgroups split each tile's 128 columns (64 each) and work in two phases:
 // P from S as soon as S lands, then dS once dP lands; the MMA order lets the tensor core run
-// the next products meanwhile. Warp roles (320 threads):
+// the next products meanwhile. Warp roles (320 threads; 384 in the key-tile kernel):
 //   warps 0-3 / 4-7  softmax warpgroups of column halves 0 / 1 (thread = TMEM lane = tile row)
 //   warp 8           TMA producer (one lane)
 //   warp 9           TMEM allocator; MMA issue (the whole warp runs the loop, one elected lane
 //                    issues each tcgen05 instruction)
+//   warps 10-11      (key-tile kernel only) idle: they complete the third warpgroup, which gives
+//                    its registers to the softmax warpgroups
 // Every wait is bounded; a timeout makes all roles stop, drain their copies and MMAs, and
 // raise a flag.
 #include <cuda.h>
@@ -48,6 +50,15 @@ constexpr int HALF = 64;                    // score columns per softmax warpgro
 constexpr int TILE_BYTES = TILE * HD * 2;   // 32 KB: one 128 x 128 bf16 tile
 constexpr int BOX_BYTES = TILE_BYTES / 2;   // one TMA box: 128 rows x 64 columns
 constexpr int NTHREADS = 320;
+// The key-tile kernel runs three full warpgroups (warps 10-11 idle) so that it can move registers
+// to the softmax warpgroups with setmaxnreg: the register file is split among the SM's four
+// sub-partitions and each holds one warp of every warpgroup, so per sub-partition the launch
+// provides 3 x 168 = 504 registers per lane, and the split below uses 216 + 216 + 72 = 504.
+constexpr int NTHREADS_KEY = 384;
+constexpr int kLaunchRegs = 168;
+constexpr int kSoftmaxRegs = 216;
+constexpr int kControlRegs = 72;
+static_assert(2 * kSoftmaxRegs + kControlRegs <= 3 * kLaunchRegs, "register split exceeds launch");
 constexpr float kLog2e = 1.4426950408889634f;
 
 __device__ __forceinline__ bool wait_bar(uint64_t* bar, uint32_t parity, volatile int* abort_flag) {
@@ -106,6 +117,13 @@ __device__ __forceinline__ float2 f2fma(float2 a, float2 b, float2 c) {
         : "=f"(d.x), "=f"(d.y) : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y), "f"(c.x), "f"(c.y));
     return d;
 }
+__device__ __forceinline__ float2 f2add(float2 a, float2 b) {
+    float2 d;
+    asm("{\n\t.reg .b64 ra, rb, rd;\n\tmov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\t"
+        "add.rn.f32x2 rd, ra, rb;\n\tmov.b64 {%0, %1}, rd;\n\t}"
+        : "=f"(d.x), "=f"(d.y) : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
+    return d;
+}
 __device__ __forceinline__ float2 f2sub(float2 a, float2 b) {
     float2 d;
     asm("{\n\t.reg .b64 ra, rb, rd;\n\tmov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\t"
@@ -124,6 +142,35 @@ __device__ __forceinline__ float2 raw2(const uint32_t* r, int e) {
     return make_float2(__uint_as_float(r[e]), __uint_as_float(r[e + 1]));
 }
 __device__ __forceinline__ float2 ex2x2(float2 x) { return make_float2(tc::ex2(x.x), tc::ex2(x.y)); }
+
+// 2^x on the FMA pipe, two lanes per instruction, for part of the exponentials (the SFU that
+// serves ex2 retires 16 per clock per SM and is the softmax's bound). Range reduction: adding
+// 1.5 * 2^23 rounds x to the nearest integer n (held in the low mantissa bits of the sum), and
+// f = x - n lies in [-1/2, 1/2]. 2^f is a cubic whose coefficients were fitted for this kernel
+// (least squares on the relative error over [-1/2, 1/2], reweighted toward equal ripple: at most
+// 7.5e-5 relative, below the bf16 rounding the result gets). 2^n is added into the exponent field.
+// Inputs are clamped at -125 so the exponent stays normal: masked (-inf) scores give 2^-125.
+constexpr float kExpC0 = 0.9999281764030457f;
+constexpr float kExpC1 = 0.6932609677314758f;
+constexpr float kExpC2 = 0.24260969460010529f;
+constexpr float kExpC3 = 0.055170830339193344f;
+__device__ __forceinline__ float2 ex2x2_fma(float2 x) {
+    x = make_float2(fmaxf(x.x, -125.f), fmaxf(x.y, -125.f));
+    const float2 shifter = make_float2(12582912.f, 12582912.f);
+    const float2 j = f2add(x, shifter);
+    const float2 fr = f2sub(x, f2sub(j, shifter));
+    float2 q = f2fma(make_float2(kExpC3, kExpC3), fr, make_float2(kExpC2, kExpC2));
+    q = f2fma(q, fr, make_float2(kExpC1, kExpC1));
+    q = f2fma(q, fr, make_float2(kExpC0, kExpC0));
+    return make_float2(__uint_as_float(__float_as_uint(q.x) + (__float_as_uint(j.x) << 23)),
+                       __uint_as_float(__float_as_uint(q.y) + (__float_as_uint(j.y) << 23)));
+}
+// Which groups of four exponentials in a 32-column chunk go to the FMA pipe (bit g: columns
+// 4 g .. 4 g + 3); the rest use the SFU.
+#ifndef ROD_BWD_POLY_GROUPS
+#define ROD_BWD_POLY_GROUPS 0xAAu
+#endif
+constexpr unsigned kPolyGroups = ROD_BWD_POLY_GROUPS;
 
 // scores outside the window [lo, hi] (column indices of this 32-column chunk) -> -inf
 __device__ __forceinline__ void mask_chunk(uint32_t* s, int c, int lo, int hi) {
@@ -349,7 +396,15 @@ ska_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
                 tc::tmem_wait_ld();
                 if (!full_tile) mask_chunk(s, c, lo, hi);
 #pragma unroll
-                for (int i = 0; i < 16; ++i) p2[16 * c + i] = ex2x2(f2fma(raw2(s, 2 * i), sl2, nl2));
+                for (int g = 0; g < 8; ++g) {
+                    if ((kPolyGroups >> g) & 1u) {
+                        p2[16 * c + 2 * g] = ex2x2_fma(f2fma(raw2(s, 4 * g), sl2, nl2));
+                        p2[16 * c + 2 * g + 1] = ex2x2_fma(f2fma(raw2(s, 4 * g + 2), sl2, nl2));
+                    } else {
+                        p2[16 * c + 2 * g] = ex2x2(f2fma(raw2(s, 4 * g), sl2, nl2));
+                        p2[16 * c + 2 * g + 1] = ex2x2(f2fma(raw2(s, 4 * g + 2), sl2, nl2));
+                    }
+                }
             }
             // phase 2: dS = P (dP - D), packed over this half's first 32 columns of the S buffer
             if (!wait_bar_warp(pfull, (uint32_t)(u & 1), abort_flag)) { ok = false; break; }
@@ -409,16 +464,19 @@ constexpr int UNIT_BYTES = 2 * TILE_BYTES;
 constexpr int OFF_STAT = OFF_RING + 2 * UNIT_BYTES;  // 2 slots of (-lse2[128], D[128]) fp32
 constexpr int STAT_BYTES = 2 * TILE * 4;
 constexpr int OFF_BAR = OFF_STAT + 2 * STAT_BYTES;
-// kfull, vfull, vempty, full[2], empty[2], sfull, pfull, pready, dsready, dvdone, dvfree, done, drain
-constexpr int NBAR = 15;
+// kfull, vfull, vempty, full[2], empty[2], sfull, pfull, sread, pwritten, dsready, dvdone, dvfree,
+// done, drain
+constexpr int NBAR = 16;
 constexpr int OFF_MISC = OFF_BAR + 8 * NBAR;
 constexpr int SMEM = OFF_MISC + 16 + 1024;
 static_assert(SMEM <= 232448, "shared memory");
 }  // namespace ka
 
-// TMEM columns: S^T [0,128) | dP^T [128,256) | dV [256,384) | dK [384,512). P^T and dS^T are
-// packed over the first 32 columns of each warpgroup's half of S^T and dP^T (packed_col).
-__global__ void __launch_bounds__(NTHREADS, 1)
+// TMEM columns: S^T [0,128) | dP^T [128,256) | dV [256,384) | dK [384,512). Once a warpgroup has
+// read its half of dP^T, that half holds its P^T (packed, first 32 columns) and dS^T (packed,
+// last 32 columns), so the S^T region is free as soon as it has been read: the next S^T is
+// computed while this pair's gradients are formed.
+__global__ void __launch_bounds__(NTHREADS_KEY, 1)
 ska_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_do,
                     const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
                     const float* __restrict__ nlse2, const float* __restrict__ dbuf,
@@ -445,12 +503,13 @@ ska_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
     uint64_t* empty = bars + 5;
     uint64_t* sfull = bars + 7;
     uint64_t* pfull = bars + 8;
-    uint64_t* pready = bars + 9;
-    uint64_t* dsready = bars + 10;
-    uint64_t* dvdone = bars + 11;
-    uint64_t* dvfree = bars + 12;
-    uint64_t* done = bars + 13;
-    uint64_t* drain = bars + 14;
+    uint64_t* sread = bars + 9;      // S^T read by both warpgroups: the region is free
+    uint64_t* pwritten = bars + 10;  // P^T written (dP^T read)
+    uint64_t* dsready = bars + 11;   // dS^T written
+    uint64_t* dvdone = bars + 12;
+    uint64_t* dvfree = bars + 13;
+    uint64_t* done = bars + 14;
+    uint64_t* drain = bars + 15;
     uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + OFF_MISC);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + OFF_MISC + 4);
 
@@ -464,7 +523,8 @@ ska_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
         }
         mbar_init(sfull, 1);
         mbar_init(pfull, 1);
-        mbar_init(pready, 256);
+        mbar_init(sread, 256);
+        mbar_init(pwritten, 256);
         mbar_init(dsready, 256);
         mbar_init(dvdone, 1);
         mbar_init(dvfree, 256);
@@ -482,6 +542,7 @@ ska_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
     tc::fence_after_sync();
     const uint32_t tmem = *tmem_holder;
 
+    if (warp >= 8) asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kControlRegs));
     if (warp == 8) {
         // ------------------------------- TMA producer -------------------------------
         if (lane == 0) {
@@ -556,35 +617,36 @@ ska_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
             const uint32_t o_lo = lo_mnmajor(unit(u) + TILE_BYTES);
 #pragma unroll
             for (int k = 0; k < TILE / 16; ++k)
-                tc::mma_ts_lh_warp(tmem + 256u, tmem + packed_col(k), o_lo + mnstep(k), d_hi, idesc_g,
+                tc::mma_ts_lh_warp(tmem + 256u, tmem + 128u + packed_col(k), o_lo + mnstep(k), d_hi, idesc_g,
                                    (first && k == 0) ? 0u : 1u);
         };
         auto issue_dk = [&](int u) {  // dK += dS^T(u) Q(u); the unit's slot is free afterwards
             const uint32_t q_lo = lo_mnmajor(unit(u));
 #pragma unroll
             for (int k = 0; k < TILE / 16; ++k)
-                tc::mma_ts_lh_warp(tmem + 384u, tmem + 128u + packed_col(k), q_lo + mnstep(k), d_hi, idesc_g,
+                tc::mma_ts_lh_warp(tmem + 384u, tmem + 160u + packed_col(k), q_lo + mnstep(k), d_hi, idesc_g,
                                    (u > 0 || k > 0) ? 1u : 0u);
             tc::mma_commit_warp(&empty[u % 2]);
         };
         if (acquire(kfull, 0) && acquire(vfull, 0) && acquire(&full[0], 0)) {
-            // order: S^T(0) dP^T(0) | dV(0) S^T(1) dK(0) dP^T(1) | dV(1) S^T(2) dK(1) dP^T(2) | ...
+            // order: S^T(0) dP^T(0) | S^T(1) dV(0) dK(0) dP^T(1) | S^T(2) dV(1) dK(1) dP^T(2) | ...
             issue_st(0);
             issue_dpt(0);
             for (int u = 0; u < U && ok; ++u) {
                 const int hi = u / n_q;
                 const bool first = u % n_q == 0, last = u % n_q == n_q - 1;
-                if (!acquire(pready, (uint32_t)(u & 1))) break;
+                if (u + 1 < U) {  // the next S^T as soon as this one has been read
+                    if (!acquire(sread, (uint32_t)(u & 1))) break;
+                    if (!acquire(&full[(u + 1) % 2], (uint32_t)(((u + 1) / 2) & 1))) break;
+                    issue_st(u + 1);
+                }
+                if (!acquire(pwritten, (uint32_t)(u & 1))) break;
                 if (first && hi > 0 && !acquire(dvfree, (uint32_t)((hi - 1) & 1))) break;
                 issue_dv(u, first);
                 if (last) tc::mma_commit_warp(dvdone);
-                if (u + 1 < U) {
-                    if (!acquire(&full[(u + 1) % 2], (uint32_t)(((u + 1) / 2) & 1))) break;
-                    issue_st(u + 1);  // over P^T(u), which dV(u) reads first: the pipe runs in order
-                }
                 if (!acquire(dsready, (uint32_t)(u & 1))) break;
                 issue_dk(u);
-                if (u + 1 < U) {
+                if (u + 1 < U) {  // over P^T(u) and dS^T(u), which dV(u) and dK(u) read first
                     if ((u + 1) % n_q == 0 && !acquire(vfull, (uint32_t)(((u + 1) / n_q) & 1))) break;
                     issue_dpt(u + 1);
                 }
@@ -593,8 +655,9 @@ ska_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
         }
         tc::mma_commit_warp(drain);
         mbar_wait_bounded(drain, 0, kWaitLimit);
-    } else {
+    } else if (warp < 8) {
         // ------------------------------- softmax warpgroups -------------------------------
+        asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kSoftmaxRegs));
         const int w = warp / 4;                    // column half (queries 64 w .. 64 w + 63)
         const int row = threadIdx.x % 128;         // key row == TMEM lane
         const uint32_t lane_base = (uint32_t)(32 * (warp % 4)) << 16;
@@ -611,52 +674,60 @@ ska_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
             const float* st = reinterpret_cast<const float*>(smem + OFF_STAT + (u % 2) * STAT_BYTES) + HALF * w;
             const bool full_tile = tq0 >= j0 + TILE - 1 && tq0 + HALF - 1 <= j0 + W - 1;
             const int lo = key - tq0, hi_e = key + W - 1 - tq0;  // valid columns [lo, hi_e]
-            // phase 1: P^T from S^T (the unit's statistics landed with its tiles)
+            // P^T from S^T (the unit's statistics landed with its tiles); S^T is released as soon
+            // as it has been read
             if (!wait_bar_warp(sfull, (uint32_t)(u & 1), abort_flag)) { ok = false; break; }
             tc::fence_after_sync();
             float2 p2[32];
 #pragma unroll
             for (int c = 0; c < 2; ++c) {
-                uint32_t s[32], pk[16];
+                uint32_t s[32];
                 tc::tmem_ld32(tS + 32u * c, s);
                 tc::tmem_wait_ld();
+                if (c == 1) {
+                    tc::fence_before_sync();
+                    mbar_arrive(sread);
+                }
                 if (!full_tile) mask_chunk(s, c, lo, hi_e);
 #pragma unroll
                 for (int e4 = 0; e4 < 32; e4 += 4) {
                     const float4 L4 = *reinterpret_cast<const float4*>(st + 32 * c + e4);  // -lse2
-                    const float2 pa = ex2x2(f2fma(raw2(s, e4), sl2, make_float2(L4.x, L4.y)));
-                    const float2 pb = ex2x2(f2fma(raw2(s, e4 + 2), sl2, make_float2(L4.z, L4.w)));
-                    p2[16 * c + e4 / 2] = pa;
-                    p2[16 * c + e4 / 2 + 1] = pb;
-                    pk[e4 / 2] = pack_bf16x2(pa.x, pa.y);
-                    pk[e4 / 2 + 1] = pack_bf16x2(pb.x, pb.y);
+                    const bool fma_pipe = (kPolyGroups >> (e4 / 4)) & 1u;
+                    const float2 xa = f2fma(raw2(s, e4), sl2, make_float2(L4.x, L4.y));
+                    const float2 xb = f2fma(raw2(s, e4 + 2), sl2, make_float2(L4.z, L4.w));
+                    p2[16 * c + e4 / 2] = fma_pipe ? ex2x2_fma(xa) : ex2x2(xa);
+                    p2[16 * c + e4 / 2 + 1] = fma_pipe ? ex2x2_fma(xb) : ex2x2(xb);
                 }
-                tc::tmem_st16(tS + 16u * c, pk);
             }
-            tc::tmem_wait_st();
-            tc::fence_before_sync();
-            mbar_arrive(pready);
-            // phase 2: dS^T = P^T (dP^T - D)
+            // dP^T read; P^T packed over the first 32 columns of this half of it as soon as those
+            // have been read (dV may start), then dS^T = P^T (dP^T - D) over the last 32
             if (!wait_bar_warp(pfull, (uint32_t)(u & 1), abort_flag)) { ok = false; break; }
             tc::fence_after_sync();
-#pragma unroll
-            for (int c = 0; c < 2; ++c) {
-                uint32_t dp[32], pk[16];
-                tc::tmem_ld32(tP + 32u * c, dp);
+            {
+                uint32_t dp[64], pk[32];
+                tc::tmem_ld32(tP, dp);
                 tc::tmem_wait_ld();
 #pragma unroll
-                for (int e4 = 0; e4 < 32; e4 += 4) {
-                    const float4 D4 = *reinterpret_cast<const float4*>(st + TILE + 32 * c + e4);
-                    const float2 da = f2mul(p2[16 * c + e4 / 2], f2sub(raw2(dp, e4), make_float2(D4.x, D4.y)));
-                    const float2 db = f2mul(p2[16 * c + e4 / 2 + 1], f2sub(raw2(dp, e4 + 2), make_float2(D4.z, D4.w)));
+                for (int i = 0; i < 32; ++i) pk[i] = pack_bf16x2(p2[i].x, p2[i].y);
+                tc::tmem_st32(tP, pk);
+                tc::tmem_wait_st();
+                tc::fence_before_sync();
+                mbar_arrive(pwritten);
+                tc::tmem_ld32(tP + 32u, dp + 32);
+                tc::tmem_wait_ld();
+#pragma unroll
+                for (int e4 = 0; e4 < 64; e4 += 4) {
+                    const float4 D4 = *reinterpret_cast<const float4*>(st + TILE + e4);
+                    const float2 da = f2mul(p2[e4 / 2], f2sub(raw2(dp, e4), make_float2(D4.x, D4.y)));
+                    const float2 db = f2mul(p2[e4 / 2 + 1], f2sub(raw2(dp, e4 + 2), make_float2(D4.z, D4.w)));
                     pk[e4 / 2] = pack_bf16x2(da.x, da.y);
                     pk[e4 / 2 + 1] = pack_bf16x2(db.x, db.y);
                 }
-                tc::tmem_st16(tP + 16u * c, pk);
+                tc::tmem_st32(tP + 32u, pk);
+                tc::tmem_wait_st();
+                tc::fence_before_sync();
+                mbar_arrive(dsready);
             }
-            tc::tmem_wait_st();
-            tc::fence_before_sync();
-            mbar_arrive(dsready);
             if (u % n_q == n_q - 1) {
                 // the head's dV rows are complete: store them and release the accumulator
                 if (!wait_bar_warp(dvdone, (uint32_t)(hi & 1), abort_flag)) { ok = false; break; }
@@ -788,7 +859,7 @@ cudaError_t swska_backward_tc_launch(const SkaBackwardArgs& a, cudaStream_t stre
     ska_bwd_dq_kernel<<<dim3((unsigned)nqt, (unsigned)H, (unsigned)B), NTHREADS, qa::SMEM, stream>>>(
         mq, mdo, mk, mv, static_cast<__nv_bfloat16*>(a.dq), nlse2, dbuf, T, (int)Tpad, H, W, sl, a.scale, nqt);
     const int G = swska_backward_tc_groups(B, H, T);
-    ska_bwd_dkdv_kernel<<<dim3((unsigned)nqt, (unsigned)G, (unsigned)B), NTHREADS, ka::SMEM, stream>>>(
+    ska_bwd_dkdv_kernel<<<dim3((unsigned)nqt, (unsigned)G, (unsigned)B), NTHREADS_KEY, ka::SMEM, stream>>>(
         mq, mdo, mk, mv, nlse2, dbuf, static_cast<__nv_bfloat16*>(a.dv), part, B, T, (int)Tpad, H, H / G, W,
         sl, nqt);
     const int64_t n4 = (int64_t)B * T * HD / 4;
