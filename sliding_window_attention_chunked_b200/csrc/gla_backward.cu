@@ -7,82 +7,123 @@
 //   dS_t    = q_t^T dO_t + diag(g_{t+1}) dS_{t+1}            (reverse in time, from dS_T)
 //   dk_t[c] = sum_j dS_t[c][j] v_t[j],   dv_t[j] = sum_c dS_t[c][j] k_t[c]
 //   dg_t[c] = sum_j dS_t[c][j] S_{t-1}[c][j],   d(initial state) = diag(g_1) dS_1.
-// Three sweeps per (batch, head), each keeping a state in registers for the whole sequence:
-//   1. forward, thread c = state row c: dq, checkpoints of S every 16 steps (stored transposed,
-//      element (j, c) at stride 1 in c, so the threads' accesses coalesce);
-//   2. reverse, thread c = gradient-state row c: per block of 16 steps the states S_{t-1} are
-//      recomputed from the block's checkpoint into a scratch (the forward rows live in padded
-//      shared memory meanwhile), then the block is walked backwards for dk, dg and the
-//      propagation of dS; the last dS is the initial-state gradient;
-//   3. reverse, thread j = gradient-state column j: dv.
-// This is the correctness-first form of the training path: O(T d^2) FMAs per (batch, head) in
-// sequence, every product in fp32.
+// Both state recurrences act on each column j (S, dS) independently, and on each row c for the
+// dv sweep: only the sums over j (dq, dk, dg) and over c (dv) couple them. So each (batch, head)
+// is a thread-block cluster of CTAs, each owning CG = 8 state columns (rows in the dv sweep)
+// with one thread per state row (column): 16x the CTAs of one CTA per (batch, head) at d = 128,
+// and a thread's step is 8 FMAs per product instead of 128. Each CTA writes its partial sums of
+// a block of BLK steps to its shared memory; after a cluster barrier every CTA adds up one slice
+// of rows over the cluster's CTAs, in rank order (deterministic), reading them through
+// distributed shared memory. The partial buffers alternate between blocks, so one barrier per
+// block suffices (a CTA writes buffer b % 2 only after every peer has passed the barrier that
+// ends the reads of block b - 2).
+// Three sweeps:
+//   1. forward, rows: dq, and a checkpoint of S before every block of BLK steps;
+//   2. reverse, rows: per block, the states S_{t-1} are recomputed from the block's checkpoint
+//      into registers (BLK x CG per thread), then the block is walked backwards for dk, dg and
+//      the propagation of dS; the last dS is the initial-state gradient;
+//   3. reverse, columns: dv.
+// Every product is fp32.
+#include <cooperative_groups.h>
+
 #include "common.cuh"
 #include "kernels.h"
+
+namespace cg = cooperative_groups;
 
 namespace rod {
 namespace {
 
-// Steps between checkpoints. The reverse sweep writes and reads back the BLK states of the
-// block it walks (BLK x 64 KB per (batch, head) at d = 128): 16 keeps that scratch in L2 for
-// 64 concurrent (batch, head) pairs (with 64 steps it spilled to DRAM: 31 GB of traffic at
-// B4 H16 T4096 and 37 ms of the 49 ms backward).
-constexpr int BLK = 16;
-constexpr int TT = 16;   // tokens staged per shared-memory tile
+constexpr int BLK = 16;  // steps per block: checkpoint spacing and reduction period
+constexpr int CG = 8;    // state columns (rows, in the dv sweep) per CTA
 
-// workspace per (batch, head): checkpoints [nblk][DV][DK] (state before each block's first
-// step), then the block scratch [BLK][DV][DK] (states S_{t-1} of the block being walked)
+// workspace per (batch, head): checkpoints [nblk][DV][DK], the state before each block's first
+// step, element (j, c) at j * DK + c (the threads' accesses coalesce)
 __host__ __device__ inline size_t ckpt_floats(int T, int dk, int dv) {
     return (size_t)((T + BLK - 1) / BLK) * dk * dv;
 }
-__host__ __device__ inline size_t per_bh_floats(int T, int dk, int dv) {
-    return ckpt_floats(T, dk, dv) + (size_t)BLK * dk * dv;
-}
 
-// ---- sweep 1: forward, rows --------------------------------------------------------------
-template <typename T, int DK, int DV>
-__global__ void __launch_bounds__(128)
-gla_bwd_fwd_rows(const T* __restrict__ q, const T* __restrict__ k, const T* __restrict__ v,
-                 const float* __restrict__ g, const float* __restrict__ state0, const T* __restrict__ dO,
-                 T* __restrict__ dq, float* __restrict__ ws, int T_len) {
-    __shared__ __align__(16) float s_v[TT][DV], s_do[TT][DV];
-    const int64_t bh = blockIdx.x;
-    const int c = threadIdx.x;
-    const bool live = c < DK;
-    float* ckpt = ws + bh * per_bh_floats(T_len, DK, DV);
-    float S[DV];
+// sum of a partial buffer over the cluster's NC CTAs for this CTA's slice of the N columns (rows
+// of the state), written through `store(t_in_block, index, value)` for steps below nt; the NC
+// remote loads of an element are issued together, then added in rank order
+template <int N, int NC, typename Store>
+__device__ __forceinline__ void cluster_reduce(cg::cluster_group& cl, const float* part, int nt, Store store) {
+    constexpr int per = (N + NC - 1) / NC;
+    const int rank = (int)cl.block_rank();
+    for (int i = threadIdx.x; i < BLK * per; i += blockDim.x) {
+        const int tt = i / per, n = rank * per + i % per;
+        if (tt < nt && n < N) {
+            float x[NC];
 #pragma unroll
-    for (int j = 0; j < DV; ++j) S[j] = live ? state0[(bh * DK + c) * DV + j] : 0.f;
-    for (int t0 = 0; t0 < T_len; t0 += TT) {
-        const int nt = T_len - t0 < TT ? T_len - t0 : TT;
-        __syncthreads();
-        for (int i = threadIdx.x; i < nt * DV; i += blockDim.x) {
-            const int tt = i / DV, j = i % DV;
-            const int64_t idx = (bh * T_len + t0 + tt) * DV + j;
-            s_v[tt][j] = to_f32(v[idx]);
-            s_do[tt][j] = to_f32(dO[idx]);
-        }
-        __syncthreads();
-        for (int tt = 0; tt < nt; ++tt) {
-            const int t = t0 + tt;
-            if (t % BLK == 0 && live) {
-                float* dst = ckpt + (size_t)(t / BLK) * DV * DK;
+            for (int r = 0; r < NC; ++r) x[r] = cl.map_shared_rank(part, r)[tt * N + n];
+            float acc = 0.f;
 #pragma unroll
-                for (int j = 0; j < DV; ++j) dst[j * DK + c] = S[j];
-            }
-            const int64_t tk = (bh * T_len + t) * DK + c;
-            const float gc = live ? g[tk] : 0.f, kc = live ? to_f32(k[tk]) : 0.f;
-            float a0 = 0.f, a1 = 0.f;
-#pragma unroll
-            for (int j = 0; j < DV; j += 2) {
-                S[j] = fmaf(gc, S[j], kc * s_v[tt][j]);
-                S[j + 1] = fmaf(gc, S[j + 1], kc * s_v[tt][j + 1]);
-                a0 = fmaf(S[j], s_do[tt][j], a0);
-                a1 = fmaf(S[j + 1], s_do[tt][j + 1], a1);
-            }
-            if (live) dq[tk] = from_f32<T>(a0 + a1);
+            for (int r = 0; r < NC; ++r) acc += x[r];
+            store(tt, n, acc);
         }
     }
+}
+
+// ---- sweep 1: forward, rows (dq, checkpoints) ------------------------------------------------
+template <typename T, int DK, int DV>
+__global__ void __launch_bounds__(128)
+gla_bwd_fwd_rows(const T* __restrict__ k, const T* __restrict__ v, const float* __restrict__ g,
+                 const float* __restrict__ state0, const T* __restrict__ dO, T* __restrict__ dq,
+                 float* __restrict__ ws, int T_len) {
+    constexpr int NG = DV / CG;
+    __shared__ __align__(16) float s_v[BLK][CG], s_do[BLK][CG], s_g[BLK][DK], s_k[BLK][DK];
+    __shared__ __align__(16) float part[2][BLK * DK];
+    cg::cluster_group cl = cg::this_cluster();
+    const int j0 = (int)cl.block_rank() * CG;
+    const int64_t bh = blockIdx.x / NG;
+    const int c = threadIdx.x;
+    const bool live = c < DK;
+    float* ckpt = ws + bh * ckpt_floats(T_len, DK, DV);
+    float S[CG];
+#pragma unroll
+    for (int j = 0; j < CG; ++j) S[j] = live ? state0[(bh * DK + c) * DV + j0 + j] : 0.f;
+    const int nblk = (T_len + BLK - 1) / BLK;
+    for (int b = 0; b < nblk; ++b) {
+        const int t0 = b * BLK, nt = T_len - t0 < BLK ? T_len - t0 : BLK;
+        __syncthreads();
+        for (int i = threadIdx.x; i < BLK * CG; i += blockDim.x) {
+            const int tt = i / CG, j = i % CG;
+            const int64_t idx = (bh * T_len + t0 + tt) * DV + j0 + j;
+            s_v[tt][j] = tt < nt ? to_f32(v[idx]) : 0.f;
+            s_do[tt][j] = tt < nt ? to_f32(dO[idx]) : 0.f;
+        }
+        for (int i = threadIdx.x; i < BLK * DK; i += blockDim.x) {
+            const int tt = i / DK, r = i % DK;
+            const int64_t idx = (bh * T_len + t0 + tt) * DK + r;
+            s_g[tt][r] = tt < nt ? g[idx] : 0.f;
+            s_k[tt][r] = tt < nt ? to_f32(k[idx]) : 0.f;
+        }
+        __syncthreads();
+        if (live) {
+            float* dst = ckpt + (size_t)b * DV * DK;
+#pragma unroll
+            for (int j = 0; j < CG; ++j) dst[(j0 + j) * DK + c] = S[j];
+        }
+        float* pb = part[b & 1];
+#pragma unroll
+        for (int tt = 0; tt < BLK; ++tt) {
+            float acc = 0.f;
+            if (tt < nt) {
+                const float gc = live ? s_g[tt][c] : 0.f, kc = live ? s_k[tt][c] : 0.f;
+#pragma unroll
+                for (int j = 0; j < CG; ++j) {
+                    S[j] = fmaf(gc, S[j], kc * s_v[tt][j]);
+                    acc = fmaf(S[j], s_do[tt][j], acc);
+                }
+            }
+            if (live) pb[tt * DK + c] = acc;
+        }
+        cl.sync();
+        cluster_reduce<DK, NG>(cl, pb, nt, [&](int tt, int n, float x) {
+            dq[(bh * T_len + t0 + tt) * DK + n] = from_f32<T>(x);
+        });
+    }
+    cl.sync();  // every peer has read this CTA's partials
 }
 
 // ---- sweep 2: reverse, rows (dk, dg, initial-state gradient) --------------------------------
@@ -91,78 +132,89 @@ __global__ void __launch_bounds__(128)
 gla_bwd_rev_rows(const T* __restrict__ q, const T* __restrict__ k, const T* __restrict__ v,
                  const float* __restrict__ g, const T* __restrict__ dO, const float* __restrict__ dSf,
                  T* __restrict__ dk, float* __restrict__ dg, float* __restrict__ dstate0,
-                 float* __restrict__ ws, int T_len) {
+                 const float* __restrict__ ws, int T_len) {
+    constexpr int NG = DV / CG;
+    // dynamic shared memory (57 KB at dk = 128): staged rows of the block, then the partial sums
     extern __shared__ __align__(16) float sm[];
-    float* s_rows = sm;                    // [DK][DV + 1] forward rows during the recompute
-    float* s_v = s_rows + DK * (DV + 1);   // [BLK][DV]
-    float* s_do = s_v + BLK * DV;          // [BLK][DV]
-    const int64_t bh = blockIdx.x;
+    float(*s_v)[CG] = reinterpret_cast<float(*)[CG]>(sm);
+    float(*s_do)[CG] = reinterpret_cast<float(*)[CG]>(sm + BLK * CG);
+    float(*s_q)[DK] = reinterpret_cast<float(*)[DK]>(sm + 2 * BLK * CG);
+    float(*s_k)[DK] = reinterpret_cast<float(*)[DK]>(sm + 2 * BLK * CG + BLK * DK);
+    float(*s_g)[DK] = reinterpret_cast<float(*)[DK]>(sm + 2 * BLK * CG + 2 * BLK * DK);
+    float* part_k[2] = {sm + 2 * BLK * CG + 3 * BLK * DK, sm + 2 * BLK * CG + 4 * BLK * DK};
+    float* part_g[2] = {sm + 2 * BLK * CG + 5 * BLK * DK, sm + 2 * BLK * CG + 6 * BLK * DK};
+    cg::cluster_group cl = cg::this_cluster();
+    const int j0 = (int)cl.block_rank() * CG;
+    const int64_t bh = blockIdx.x / NG;
     const int c = threadIdx.x;
     const bool live = c < DK;
-    float* ckpt = ws + bh * per_bh_floats(T_len, DK, DV);
-    float* scratch = ckpt + ckpt_floats(T_len, DK, DV);
-    float dS[DV];
+    const float* ckpt = ws + bh * ckpt_floats(T_len, DK, DV);
+    float dS[CG];
 #pragma unroll
-    for (int j = 0; j < DV; ++j) dS[j] = (live && dSf) ? dSf[(bh * DK + c) * DV + j] : 0.f;
+    for (int j = 0; j < CG; ++j) dS[j] = (live && dSf) ? dSf[(bh * DK + c) * DV + j0 + j] : 0.f;
     const int nblk = (T_len + BLK - 1) / BLK;
-    for (int blk = nblk - 1; blk >= 0; --blk) {
-        const int t0 = blk * BLK, t1 = t0 + BLK < T_len ? t0 + BLK : T_len, nt = t1 - t0;
-        __syncthreads();  // the previous block's staged tokens are no longer read
-        for (int i = threadIdx.x; i < nt * DV; i += blockDim.x) {
-            const int tt = i / DV, j = i % DV;
-            const int64_t idx = (bh * T_len + t0 + tt) * DV + j;
-            s_v[tt * DV + j] = to_f32(v[idx]);
-            s_do[tt * DV + j] = to_f32(dO[idx]);
+    for (int b = nblk - 1; b >= 0; --b) {
+        const int t0 = b * BLK, nt = T_len - t0 < BLK ? T_len - t0 : BLK;
+        __syncthreads();
+        for (int i = threadIdx.x; i < BLK * CG; i += blockDim.x) {
+            const int tt = i / CG, j = i % CG;
+            const int64_t idx = (bh * T_len + t0 + tt) * DV + j0 + j;
+            s_v[tt][j] = tt < nt ? to_f32(v[idx]) : 0.f;
+            s_do[tt][j] = tt < nt ? to_f32(dO[idx]) : 0.f;
         }
-        // recompute S_{t-1} for t in the block from its checkpoint (row c in shared memory)
-        if (live) {
-            const float* src = ckpt + (size_t)blk * DV * DK;
-#pragma unroll 4
-            for (int j = 0; j < DV; ++j) s_rows[c * (DV + 1) + j] = src[j * DK + c];
+        for (int i = threadIdx.x; i < BLK * DK; i += blockDim.x) {
+            const int tt = i / DK, r = i % DK;
+            const int64_t idx = (bh * T_len + t0 + tt) * DK + r;
+            s_q[tt][r] = tt < nt ? to_f32(q[idx]) : 0.f;
+            s_k[tt][r] = tt < nt ? to_f32(k[idx]) : 0.f;
+            s_g[tt][r] = tt < nt ? g[idx] : 0.f;
         }
         __syncthreads();
-        for (int tt = 0; tt < nt; ++tt) {
-            const int64_t tk = (bh * T_len + t0 + tt) * DK + c;
-            const float gc = live ? g[tk] : 0.f, kc = live ? to_f32(k[tk]) : 0.f;
-            if (live) {
-                float* row = s_rows + c * (DV + 1);
-                float* dst = scratch + (size_t)tt * DV * DK;
-#pragma unroll 16
-                for (int j = 0; j < DV; ++j) {
-                    dst[j * DK + c] = row[j];  // S_{t-1}
-                    row[j] = fmaf(gc, row[j], kc * s_v[tt * DV + j]);
-                }
-            }
-        }
-        __syncthreads();  // (each thread reads back only what it wrote; kept for clarity)
-        for (int tt = nt - 1; tt >= 0; --tt) {
-            const int64_t tk = (bh * T_len + t0 + tt) * DK + c;
-            const float gc = live ? g[tk] : 0.f, qc = live ? to_f32(q[tk]) : 0.f;
-            const float* sp = scratch + (size_t)tt * DV * DK;
-            float ak0 = 0.f, ak1 = 0.f, ag0 = 0.f, ag1 = 0.f;
+        // the block's states S_{t0 + tt - 1}, recomputed from its checkpoint
+        float Sp[BLK][CG];
 #pragma unroll
-            for (int j = 0; j < DV; j += 2) {
-                dS[j] = fmaf(qc, s_do[tt * DV + j], dS[j]);
-                dS[j + 1] = fmaf(qc, s_do[tt * DV + j + 1], dS[j + 1]);
-                ak0 = fmaf(dS[j], s_v[tt * DV + j], ak0);
-                ak1 = fmaf(dS[j + 1], s_v[tt * DV + j + 1], ak1);
-                if (live) {
-                    ag0 = fmaf(dS[j], sp[j * DK + c], ag0);
-                    ag1 = fmaf(dS[j + 1], sp[(j + 1) * DK + c], ag1);
+        for (int j = 0; j < CG; ++j) Sp[0][j] = live ? ckpt[(size_t)b * DV * DK + (j0 + j) * DK + c] : 0.f;
+#pragma unroll
+        for (int tt = 1; tt < BLK; ++tt) {
+            // (past the block's last step the staged g, k, v are 0 and these states are unused)
+            const float gc = live ? s_g[tt - 1][c] : 0.f, kc = live ? s_k[tt - 1][c] : 0.f;
+#pragma unroll
+            for (int j = 0; j < CG; ++j) Sp[tt][j] = fmaf(gc, Sp[tt - 1][j], kc * s_v[tt - 1][j]);
+        }
+        float* pk = part_k[b & 1];
+        float* pg = part_g[b & 1];
+#pragma unroll
+        for (int tt = BLK - 1; tt >= 0; --tt) {
+            float ak = 0.f, ag = 0.f;
+            if (tt < nt) {
+                const float gc = live ? s_g[tt][c] : 0.f, qc = live ? s_q[tt][c] : 0.f;
+#pragma unroll
+                for (int j = 0; j < CG; ++j) {
+                    dS[j] = fmaf(qc, s_do[tt][j], dS[j]);
+                    ak = fmaf(dS[j], s_v[tt][j], ak);
+                    ag = fmaf(dS[j], Sp[tt][j], ag);
                 }
+#pragma unroll
+                for (int j = 0; j < CG; ++j) dS[j] *= gc;
             }
             if (live) {
-                dk[tk] = from_f32<T>(ak0 + ak1);
-                dg[tk] = ag0 + ag1;
+                pk[tt * DK + c] = ak;
+                pg[tt * DK + c] = ag;
             }
-#pragma unroll
-            for (int j = 0; j < DV; ++j) dS[j] *= gc;
         }
+        cl.sync();
+        cluster_reduce<DK, NG>(cl, pk, nt, [&](int tt, int n, float x) {
+            dk[(bh * T_len + t0 + tt) * DK + n] = from_f32<T>(x);
+        });
+        cluster_reduce<DK, NG>(cl, pg, nt, [&](int tt, int n, float x) {
+            dg[(bh * T_len + t0 + tt) * DK + n] = x;
+        });
     }
     if (live) {
 #pragma unroll
-        for (int j = 0; j < DV; ++j) dstate0[(bh * DK + c) * DV + j] = dS[j];
+        for (int j = 0; j < CG; ++j) dstate0[(bh * DK + c) * DV + j0 + j] = dS[j];
     }
+    cl.sync();
 }
 
 // ---- sweep 3: reverse, columns (dv) --------------------------------------------------------
@@ -171,62 +223,102 @@ __global__ void __launch_bounds__(128)
 gla_bwd_rev_cols(const T* __restrict__ q, const T* __restrict__ k, const float* __restrict__ g,
                  const T* __restrict__ dO, const float* __restrict__ dSf, T* __restrict__ dv,
                  int T_len) {
-    __shared__ __align__(16) float s_q[TT][DK], s_k[TT][DK], s_g[TT][DK];
-    const int64_t bh = blockIdx.x;
+    constexpr int NG = DK / CG;
+    __shared__ __align__(16) float s_q[BLK][CG], s_k[BLK][CG], s_g[BLK][CG], s_do[BLK][DV];
+    __shared__ __align__(16) float part[2][BLK * DV];
+    cg::cluster_group cl = cg::this_cluster();
+    const int c0 = (int)cl.block_rank() * CG;
+    const int64_t bh = blockIdx.x / NG;
     const int j = threadIdx.x;
     const bool live = j < DV;
-    float dS[DK];
+    float dS[CG];  // column j of the gradient state, rows c0 .. c0 + CG - 1
 #pragma unroll
-    for (int c = 0; c < DK; ++c) dS[c] = (live && dSf) ? dSf[(bh * DK + c) * DV + j] : 0.f;
-    for (int t1 = T_len; t1 > 0; t1 -= TT) {
-        const int t0 = t1 - TT > 0 ? t1 - TT : 0, nt = t1 - t0;
+    for (int i = 0; i < CG; ++i) dS[i] = (live && dSf) ? dSf[(bh * DK + c0 + i) * DV + j] : 0.f;
+    const int nblk = (T_len + BLK - 1) / BLK;
+    for (int b = nblk - 1; b >= 0; --b) {
+        const int t0 = b * BLK, nt = T_len - t0 < BLK ? T_len - t0 : BLK;
         __syncthreads();
-        for (int i = threadIdx.x; i < nt * DK; i += blockDim.x) {
-            const int tt = i / DK, c = i % DK;
-            const int64_t idx = (bh * T_len + t0 + tt) * DK + c;
-            s_q[tt][c] = to_f32(q[idx]);
-            s_k[tt][c] = to_f32(k[idx]);
-            s_g[tt][c] = g[idx];
+        for (int i = threadIdx.x; i < BLK * CG; i += blockDim.x) {
+            const int tt = i / CG, r = i % CG;
+            const int64_t idx = (bh * T_len + t0 + tt) * DK + c0 + r;
+            s_q[tt][r] = tt < nt ? to_f32(q[idx]) : 0.f;
+            s_k[tt][r] = tt < nt ? to_f32(k[idx]) : 0.f;
+            s_g[tt][r] = tt < nt ? g[idx] : 0.f;
+        }
+        for (int i = threadIdx.x; i < BLK * DV; i += blockDim.x) {
+            const int tt = i / DV, n = i % DV;
+            s_do[tt][n] = tt < nt ? to_f32(dO[(bh * T_len + t0 + tt) * DV + n]) : 0.f;
         }
         __syncthreads();
-        for (int tt = nt - 1; tt >= 0; --tt) {
-            const int64_t tv = (bh * T_len + t0 + tt) * DV + j;
-            const float doj = live ? to_f32(dO[tv]) : 0.f;
-            float a0 = 0.f, a1 = 0.f;
+        float* pb = part[b & 1];
 #pragma unroll
-            for (int c = 0; c < DK; c += 2) {
-                dS[c] = fmaf(s_q[tt][c], doj, dS[c]);
-                dS[c + 1] = fmaf(s_q[tt][c + 1], doj, dS[c + 1]);
-                a0 = fmaf(s_k[tt][c], dS[c], a0);
-                a1 = fmaf(s_k[tt][c + 1], dS[c + 1], a1);
-                dS[c] *= s_g[tt][c];
-                dS[c + 1] *= s_g[tt][c + 1];
+        for (int tt = BLK - 1; tt >= 0; --tt) {
+            float a = 0.f;
+            if (tt < nt) {
+                const float doj = live ? s_do[tt][j] : 0.f;
+#pragma unroll
+                for (int i = 0; i < CG; ++i) {
+                    dS[i] = fmaf(s_q[tt][i], doj, dS[i]);
+                    a = fmaf(s_k[tt][i], dS[i], a);
+                    dS[i] *= s_g[tt][i];
+                }
             }
-            if (live) dv[tv] = from_f32<T>(a0 + a1);
+            if (live) pb[tt * DV + j] = a;
         }
+        cl.sync();
+        cluster_reduce<DV, NG>(cl, pb, nt, [&](int tt, int n, float x) {
+            dv[(bh * T_len + t0 + tt) * DV + n] = from_f32<T>(x);
+        });
     }
+    cl.sync();
+}
+
+template <int DK>
+constexpr size_t rev_rows_smem() { return sizeof(float) * (2 * BLK * CG + 7 * BLK * DK); }
+
+template <typename K, typename... Args>
+cudaError_t launch_cluster(K kernel, int64_t clusters, int csize, int threads, size_t smem, cudaStream_t s,
+                           Args... args) {
+    cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+    if (e == cudaSuccess && smem > 0)
+        e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    if (clusters * csize > 0x7fffffff) return cudaErrorInvalidConfiguration;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)(clusters * csize), 1, 1);
+    cfg.blockDim = dim3((unsigned)threads, 1, 1);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = (unsigned)csize;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kernel, args...);
 }
 
 template <typename T, int DK, int DV>
 cudaError_t launch_t(const GlaBackwardArgs& a, cudaStream_t s) {
-    const unsigned grid = (unsigned)((int64_t)a.B * a.H);
+    static_assert(DK % CG == 0 && DV % CG == 0, "state dims are multiples of the column group");
+    const int64_t bhs = (int64_t)a.B * a.H;
     const int rows = DK < 32 ? 32 : DK, cols = DV < 32 ? 32 : DV;
     float* ws = static_cast<float*>(a.workspace);
-    gla_bwd_fwd_rows<T, DK, DV><<<grid, rows, 0, s>>>(
-        static_cast<const T*>(a.q), static_cast<const T*>(a.k), static_cast<const T*>(a.v), a.g, a.state0,
-        static_cast<const T*>(a.dO), static_cast<T*>(a.dq), ws, a.T);
-    const size_t smem = sizeof(float) * ((size_t)DK * (DV + 1) + 2 * (size_t)BLK * DV);
-    cudaError_t e = cudaFuncSetAttribute(gla_bwd_rev_rows<T, DK, DV>,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    cudaError_t e = launch_cluster(gla_bwd_fwd_rows<T, DK, DV>, bhs, DV / CG, rows, 0, s,
+                                   static_cast<const T*>(a.k), static_cast<const T*>(a.v), a.g, a.state0,
+                                   static_cast<const T*>(a.dO), static_cast<T*>(a.dq), ws, a.T);
     if (e != cudaSuccess) return e;
-    gla_bwd_rev_rows<T, DK, DV><<<grid, rows, smem, s>>>(
-        static_cast<const T*>(a.q), static_cast<const T*>(a.k), static_cast<const T*>(a.v), a.g,
-        static_cast<const T*>(a.dO), a.dstate_final, static_cast<T*>(a.dk), a.dg, a.dstate0, ws, a.T);
-    gla_bwd_rev_cols<T, DK, DV><<<grid, cols, 0, s>>>(
-        static_cast<const T*>(a.q), static_cast<const T*>(a.k), a.g, static_cast<const T*>(a.dO),
-        a.dstate_final, static_cast<T*>(a.dv), a.T);
+    e = launch_cluster(gla_bwd_rev_rows<T, DK, DV>, bhs, DV / CG, rows, rev_rows_smem<DK>(), s,
+                       static_cast<const T*>(a.q),
+                       static_cast<const T*>(a.k), static_cast<const T*>(a.v), a.g, static_cast<const T*>(a.dO),
+                       a.dstate_final, static_cast<T*>(a.dk), a.dg, a.dstate0, static_cast<const float*>(ws), a.T);
+    if (e != cudaSuccess) return e;
+    e = launch_cluster(gla_bwd_rev_cols<T, DK, DV>, bhs, DK / CG, cols, 0, s, static_cast<const T*>(a.q),
+                       static_cast<const T*>(a.k), a.g, static_cast<const T*>(a.dO), a.dstate_final,
+                       static_cast<T*>(a.dv), a.T);
     note_launches(3);
-    return cudaGetLastError();
+    return e;
 }
 
 template <typename T, int DK>
@@ -254,7 +346,7 @@ cudaError_t launch_dk(const GlaBackwardArgs& a, cudaStream_t s) {
 }  // namespace
 
 size_t gla_backward_workspace_size(int B, int H, int T, int dk, int dv) {
-    return (size_t)B * H * per_bh_floats(T, dk, dv) * sizeof(float);
+    return (size_t)B * H * ckpt_floats(T, dk, dv) * sizeof(float);
 }
 
 cudaError_t gla_backward_launch(const GlaBackwardArgs& a, bool bf16, cudaStream_t stream) {
