@@ -127,8 +127,9 @@ gla_bwd_fwd_rows(const T* __restrict__ k, const T* __restrict__ v, const float* 
 }
 
 // ---- sweep 2: reverse, rows (dk, dg, initial-state gradient) --------------------------------
+// three CTAs per SM (167 registers, no spills; the block's states take 128 of them)
 template <typename T, int DK, int DV>
-__global__ void __launch_bounds__(128)
+__global__ void __launch_bounds__(128, 3)
 gla_bwd_rev_rows(const T* __restrict__ q, const T* __restrict__ k, const T* __restrict__ v,
                  const float* __restrict__ g, const T* __restrict__ dO, const float* __restrict__ dSf,
                  T* __restrict__ dk, float* __restrict__ dg, float* __restrict__ dstate0,
