@@ -36,6 +36,7 @@
 #include <math.h>
 
 #include "common.cuh"
+#include "exp2x2.cuh"
 #include "kernels.h"
 #include "tc.cuh"
 
@@ -109,68 +110,15 @@ __device__ __forceinline__ uint32_t kstep(int k) { return (uint32_t)(((k / 4) * 
 // offset of K step k (16 rows) in an MN-major tile
 __device__ __forceinline__ uint32_t mnstep(int k) { return (uint32_t)((2048 * k) >> 4); }
 
-// two-wide fp32 arithmetic (one instruction for both lanes of the pair)
-__device__ __forceinline__ float2 f2fma(float2 a, float2 b, float2 c) {
-    float2 d;
-    asm("{\n\t.reg .b64 ra, rb, rc, rd;\n\tmov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\t"
-        "mov.b64 rc, {%6, %7};\n\tfma.rn.f32x2 rd, ra, rb, rc;\n\tmov.b64 {%0, %1}, rd;\n\t}"
-        : "=f"(d.x), "=f"(d.y) : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y), "f"(c.x), "f"(c.y));
-    return d;
-}
-__device__ __forceinline__ float2 f2add(float2 a, float2 b) {
-    float2 d;
-    asm("{\n\t.reg .b64 ra, rb, rd;\n\tmov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\t"
-        "add.rn.f32x2 rd, ra, rb;\n\tmov.b64 {%0, %1}, rd;\n\t}"
-        : "=f"(d.x), "=f"(d.y) : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
-    return d;
-}
-__device__ __forceinline__ float2 f2sub(float2 a, float2 b) {
-    float2 d;
-    asm("{\n\t.reg .b64 ra, rb, rd;\n\tmov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\t"
-        "sub.rn.f32x2 rd, ra, rb;\n\tmov.b64 {%0, %1}, rd;\n\t}"
-        : "=f"(d.x), "=f"(d.y) : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
-    return d;
-}
-__device__ __forceinline__ float2 f2mul(float2 a, float2 b) {
-    float2 d;
-    asm("{\n\t.reg .b64 ra, rb, rd;\n\tmov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\t"
-        "mul.rn.f32x2 rd, ra, rb;\n\tmov.b64 {%0, %1}, rd;\n\t}"
-        : "=f"(d.x), "=f"(d.y) : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
-    return d;
-}
+using fx::ex2x2_fma;
+using fx::f2add;
+using fx::f2fma;
+using fx::f2mul;
+using fx::f2sub;
 __device__ __forceinline__ float2 raw2(const uint32_t* r, int e) {
     return make_float2(__uint_as_float(r[e]), __uint_as_float(r[e + 1]));
 }
-__device__ __forceinline__ float2 ex2x2(float2 x) { return make_float2(tc::ex2(x.x), tc::ex2(x.y)); }
-
-// 2^x on the FMA pipe, two lanes per instruction, for part of the exponentials (the SFU that
-// serves ex2 retires 16 per clock per SM and is the softmax's bound). Range reduction: adding
-// 1.5 * 2^23 rounds x to the nearest integer n (held in the low mantissa bits of the sum), and
-// f = x - n lies in [-1/2, 1/2]. 2^f is a cubic whose coefficients were fitted for this kernel
-// (least squares on the relative error over [-1/2, 1/2], reweighted toward equal ripple: at most
-// 7.5e-5 relative, below the bf16 rounding the result gets). 2^n is added into the exponent field.
-// Inputs are clamped at -125 so the exponent stays normal: masked (-inf) scores give 2^-125.
-constexpr float kExpC0 = 0.9999281764030457f;
-constexpr float kExpC1 = 0.6932609677314758f;
-constexpr float kExpC2 = 0.24260969460010529f;
-constexpr float kExpC3 = 0.055170830339193344f;
-__device__ __forceinline__ float2 ex2x2_fma(float2 x) {
-    x = make_float2(fmaxf(x.x, -125.f), fmaxf(x.y, -125.f));
-    const float2 shifter = make_float2(12582912.f, 12582912.f);
-    const float2 j = f2add(x, shifter);
-    const float2 fr = f2sub(x, f2sub(j, shifter));
-    float2 q = f2fma(make_float2(kExpC3, kExpC3), fr, make_float2(kExpC2, kExpC2));
-    q = f2fma(q, fr, make_float2(kExpC1, kExpC1));
-    q = f2fma(q, fr, make_float2(kExpC0, kExpC0));
-    return make_float2(__uint_as_float(__float_as_uint(q.x) + (__float_as_uint(j.x) << 23)),
-                       __uint_as_float(__float_as_uint(q.y) + (__float_as_uint(j.y) << 23)));
-}
-// Which groups of four exponentials in a 32-column chunk go to the FMA pipe (bit g: columns
-// 4 g .. 4 g + 3); the rest use the SFU.
-#ifndef ROD_BWD_POLY_GROUPS
-#define ROD_BWD_POLY_GROUPS 0xAAu
-#endif
-constexpr unsigned kPolyGroups = ROD_BWD_POLY_GROUPS;
+__device__ __forceinline__ float2 ex2x2(float2 x) { return fx::ex2x2_sfu(x); }
 
 // scores outside the window [lo, hi] (column indices of this 32-column chunk) -> -inf
 __device__ __forceinline__ void mask_chunk(uint32_t* s, int c, int lo, int hi) {
@@ -180,6 +128,10 @@ __device__ __forceinline__ void mask_chunk(uint32_t* s, int c, int lo, int hi) {
         if (col < lo || col > hi) s[e] = 0xff800000u;
     }
 }
+// Which groups of four exponentials in a 32-column chunk go to the FMA pipe (bit g: columns
+// 4 g .. 4 g + 3); the rest use the SFU.
+constexpr unsigned kPolyGroups = 0xAAu;
+
 // ============================================================================================
 // Launch 2: query tiles (dQ)
 // ============================================================================================
