@@ -51,9 +51,19 @@ class OracleLib:
                                               i64, i64, i64, i64, ctypes.c_double, ctypes.c_int]
         lib.rodref_gla_backward.argtypes = [f32p, f32p, f32p, f32p, f64p, f32p, f32p, f64p, f64p,
                                             f64p, f64p, f64p, i64, i64, i64, i64, i64, ctypes.c_int]
+        u8p = ctypes.POINTER(ctypes.c_uint8)
+        lib.rodref_e4m3_encode_array.argtypes = [f32p, u8p, i64, ctypes.c_float]
+        lib.rodref_e4m3_decode_array.argtypes = [u8p, f64p, i64]
+        lib.rodref_swska_decode_fp8.argtypes = [f32p, f32p, f32p, u8p, u8p, i64p, f64p, i64, i64, i64,
+                                                i64, i64, ctypes.c_double, ctypes.c_double,
+                                                ctypes.c_double, ctypes.c_int]
+        lib.rodref_swska_cache_fill_fp8.argtypes = [f32p, f32p, u8p, u8p, i64, i64, i64, i64, i64, i64,
+                                                    ctypes.c_float, ctypes.c_float]
         for name in ("rodref_gla_backward", "rodref_swska_backward", "rodref_gla_prefill", "rodref_gla_decode_step",
                      "rodref_swska_prefill",
-                     "rodref_swska_decode", "rodref_swska_cache_fill", "rodref_swska_decode_paged"):
+                     "rodref_swska_decode", "rodref_swska_cache_fill", "rodref_swska_decode_paged",
+                     "rodref_e4m3_encode_array", "rodref_e4m3_decode_array", "rodref_swska_decode_fp8",
+                     "rodref_swska_cache_fill_fp8"):
             getattr(lib, name).restype = ctypes.c_int
         self.lib = lib
         self.path = path
@@ -123,6 +133,16 @@ def _p64(a):
 
 def _pi64(a):
     return a.ctypes.data_as(ctypes.POINTER(ctypes.c_int64))
+
+
+def _pu8(a):
+    return a.ctypes.data_as(ctypes.POINTER(ctypes.c_uint8))
+
+
+def _u8(x) -> np.ndarray:
+    if hasattr(x, "detach"):
+        x = x.detach().to("cpu").contiguous().view(__import__("torch").uint8).numpy()
+    return np.ascontiguousarray(np.asarray(x, dtype=np.uint8))
 
 
 def _check(rc, name):
@@ -283,3 +303,60 @@ def swska_backward(q, k, v, dO, window, scale=None, nthreads=None):
                                     nthreads or default_threads())
     _check(rc, "swska_backward")
     return dq, dk_, dv_
+
+
+# ------------------------------------------------------------------------------------------
+# FP8 (E4M3) window cache (SALA blog §4.3; format and rounding as read in rodref.c's header)
+# ------------------------------------------------------------------------------------------
+
+
+def e4m3_encode(x, scale=1.0):
+    """E4M3 codes (uint8) of x / scale: the quotient in fp32, the nearest code, ties to the even
+    code, magnitudes past 448 saturated."""
+    x = _f32(x)
+    out = np.empty(x.shape, dtype=np.uint8)
+    rc = _L().rodref_e4m3_encode_array(_p32(x), _pu8(out), x.size, float(np.float32(scale)))
+    _check(rc, "e4m3_encode")
+    return out
+
+
+def e4m3_decode(codes):
+    """Values (float64) of E4M3 codes."""
+    c = _u8(codes)
+    out = np.empty(c.shape, dtype=np.float64)
+    rc = _L().rodref_e4m3_decode_array(_pu8(c), _p64(out), c.size)
+    _check(rc, "e4m3_decode")
+    return out
+
+
+def swska_decode_fp8(q, k_new, v_new, k_cache, v_cache, pos, window, scale=None, k_scale=1.0,
+                     v_scale=1.0, nthreads=None):
+    """Decode over FP8 rings (codes k_cache [N,W,dk], v_cache [N,H,W,dv]). Returns
+    (o [N,H,dv] float64, k_cache', v_cache') with the new token's codes written."""
+    q, k_new, v_new = _f32(q), _f32(k_new), _f32(v_new)
+    kc, vc = _u8(k_cache).copy(), _u8(v_cache).copy()
+    pos = np.ascontiguousarray(np.asarray(pos.cpu() if hasattr(pos, "cpu") else pos, dtype=np.int64))
+    N, H, dk = q.shape
+    dv = v_new.shape[-1]
+    if scale is None or scale <= 0:
+        scale = 1.0 / np.sqrt(dk)
+    o = np.empty((N, H, dv))
+    rc = _L().rodref_swska_decode_fp8(_p32(q), _p32(k_new), _p32(v_new), _pu8(kc), _pu8(vc), _pi64(pos),
+                                      _p64(o), N, H, dk, dv, int(window), float(scale),
+                                      float(np.float32(k_scale)), float(np.float32(v_scale)),
+                                      nthreads or default_threads())
+    _check(rc, "swska_decode_fp8")
+    return o, kc, vc
+
+
+def swska_cache_fill_fp8(k, v, k_cache, v_cache, window, k_scale=1.0, v_scale=1.0):
+    """Hand-off into FP8 rings: positions [max(0,T-W), T) of k [B,T,dk], v [B,H,T,dv] to slot
+    p mod W as E4M3 codes of x / scale. Returns the updated (k_cache, v_cache) copies (uint8)."""
+    k, v = _f32(k), _f32(v)
+    kc, vc = _u8(k_cache).copy(), _u8(v_cache).copy()
+    B, T, dk = k.shape
+    H, dv = v.shape[1], v.shape[-1]
+    rc = _L().rodref_swska_cache_fill_fp8(_p32(k), _p32(v), _pu8(kc), _pu8(vc), B, H, T, dk, dv,
+                                          int(window), float(np.float32(k_scale)), float(np.float32(v_scale)))
+    _check(rc, "swska_cache_fill_fp8")
+    return kc, vc

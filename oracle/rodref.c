@@ -24,7 +24,9 @@
  *  [SALA]      sparse + linear attention blog: §2.1 sliding-window attention (each query looks
  *              only at recent keys), §2.2 linear attention state O_i = phi(q_i) * sum_j phi(k_j)^T v_j
  *              with a d x d state, §3.3 ring-buffer window cache and in-place state update at
- *              decode, §4.3 third tip (a decay factor makes old state weights fall exponentially).
+ *              decode, §4.3 first tip (store the KV cache in FP8: half the memory, a faster
+ *              decode, at some loss of detail), §4.3 third tip (a decay factor makes old state
+ *              weights fall exponentially).
  *
  * Readings taken where the pages are silent or garbled (the DDTS gate equation in [CodeFuse]
  * is stripped from the extracted text):
@@ -34,6 +36,13 @@
  *  - the window of query t holds W keys including t itself: j in [t-W+1, t], clipped at 0.
  *    W = 1 then gives o_t = v_t and W >= T gives full causal attention.
  *  - softmax attention uses o = sum_j p_j v_j / sum_j p_j with p_j = exp(s_j - max s).
+ *  - FP8 window cache ([SALA] §4.3 names FP8 and nothing more): the OCP E4M3 format (1 sign
+ *    bit, 4 exponent bits with bias 7, 3 mantissa bits, no infinities, S.1111.111 is NaN, the
+ *    largest finite value 448), one fp32 scale per cache, stored code = e4m3(x / scale) with x
+ *    and the quotient in fp32 (the precision the kernel decides in), rounded to the nearest
+ *    code with ties to the even code and saturated at +-448; the attention reads
+ *    value(code) * scale. The new token is written to the cache first and read back like the
+ *    other window entries.
  */
 #include <math.h>
 #include <pthread.h>
@@ -537,6 +546,143 @@ int rodref_swska_cache_fill(const float* k, const float* v, float* k_cache, floa
             for (int64_t h = 0; h < H; ++h)
                 memcpy(v_cache + ((b * H + h) * W + slot) * dv, v + ((b * H + h) * T + p) * dv,
                        (size_t)dv * sizeof(float));
+        }
+    return 0;
+}
+
+/* ---- FP8 (E4M3) window cache ([SALA] §4.3; format and rounding: the reading in the header) --- */
+
+/* value of an E4M3 code, from the format's definition: exponent field 0 is subnormal
+ * (mantissa/8 * 2^-6), otherwise (1 + mantissa/8) * 2^(exponent - 7); S.1111.111 is NaN */
+double rodref_e4m3_decode(uint8_t code) {
+    const int sign = code >> 7, e = (code >> 3) & 15, m = code & 7;
+    double v;
+    if (e == 15 && m == 7) return NAN;
+    if (e == 0)
+        v = ldexp((double)m / 8.0, -6);
+    else
+        v = ldexp(1.0 + (double)m / 8.0, e - 7);
+    return sign ? -v : v;
+}
+
+/* nearest E4M3 code to the fp32 value x: every non-negative finite code (0x00 .. 0x7E) is a
+ * candidate for |x|, the closest wins, a tie goes to the even code; magnitudes beyond 448 take
+ * 448 (saturation); the sign bit is x's; NaN gives 0x7F */
+uint8_t rodref_e4m3_encode(float x) {
+    if (isnan(x)) return 0x7F;
+    const double a = fabs((double)x);
+    int best = 0;
+    double best_d = INFINITY;
+    for (int c = 0; c <= 0x7E; ++c) {
+        const double d = fabs(rodref_e4m3_decode((uint8_t)c) - a);
+        if (d < best_d || (d == best_d && (c & 1) == 0 && (best & 1) == 1)) {
+            best = c;
+            best_d = d;
+        }
+    }
+    if (a > 448.0) best = 0x7E;
+    return (uint8_t)(best | (signbit(x) ? 0x80 : 0));
+}
+
+int rodref_e4m3_encode_array(const float* x, uint8_t* out, int64_t n, float scale) {
+    if (!x || !out || n < 0 || !(scale > 0.f)) return RODREF_EINVAL;
+    for (int64_t i = 0; i < n; ++i) out[i] = rodref_e4m3_encode(x[i] / scale);
+    return 0;
+}
+
+int rodref_e4m3_decode_array(const uint8_t* c, double* out, int64_t n) {
+    if (!c || !out || n < 0) return RODREF_EINVAL;
+    for (int64_t i = 0; i < n; ++i) out[i] = rodref_e4m3_decode(c[i]);
+    return 0;
+}
+
+/* Decode with FP8 ring caches: k_cache [N,W,dk] and v_cache [N,H,W,dv] hold E4M3 codes. For
+ * each sequence n with P = pos[n] >= 0: the new token's codes e4m3(k_new / k_scale) and
+ * e4m3(v_new[h] / v_scale) go to slot P mod W, then o[n,h] is the softmax attention of q[n,h]
+ * over positions max(0, P-W+1) .. P read back from their slots as value(code) * scale.
+ * pos < 0: o = NaN and the caches are left untouched. */
+typedef struct {
+    const float *q, *k_new, *v_new;
+    uint8_t *kc, *vc;
+    const int64_t* pos;
+    double* o;
+    int64_t H, dk, dv, W;
+    double scale, k_scale, v_scale;
+} ska_dec8_args_t;
+
+static void ska_dec8_unit(const void* p, int64_t n) {
+    const ska_dec8_args_t* a = (const ska_dec8_args_t*)p;
+    const int64_t H = a->H, dk = a->dk, dv = a->dv, W = a->W, P = a->pos[n];
+    if (P < 0) {
+        for (int64_t i = 0; i < H * dv; ++i) a->o[n * H * dv + i] = NAN;
+        return;
+    }
+    const int64_t slot = P % W;
+    for (int64_t c = 0; c < dk; ++c)
+        a->kc[(n * W + slot) * dk + c] = rodref_e4m3_encode(a->k_new[n * dk + c] / (float)a->k_scale);
+    for (int64_t h = 0; h < H; ++h)
+        for (int64_t c = 0; c < dv; ++c)
+            a->vc[((n * H + h) * W + slot) * dv + c] =
+                rodref_e4m3_encode(a->v_new[(n * H + h) * dv + c] / (float)a->v_scale);
+    const int64_t p0 = P - W + 1 > 0 ? P - W + 1 : 0, cnt = P - p0 + 1;
+    double* s = malloc((size_t)cnt * sizeof(double));
+    if (!s) return;
+    for (int64_t h = 0; h < H; ++h) {
+        const float* qv = a->q + (n * H + h) * dk;
+        double m = -INFINITY;
+        for (int64_t i = 0; i < cnt; ++i) {
+            const int64_t sl = (p0 + i) % W;
+            double acc = 0.0;
+            for (int64_t c = 0; c < dk; ++c)
+                acc += (double)qv[c] * rodref_e4m3_decode(a->kc[(n * W + sl) * dk + c]) * a->k_scale;
+            s[i] = a->scale * acc;
+            if (s[i] > m) m = s[i];
+        }
+        double l = 0.0;
+        for (int64_t i = 0; i < cnt; ++i) {
+            s[i] = exp(s[i] - m);
+            l += s[i];
+        }
+        double* on = a->o + (n * H + h) * dv;
+        for (int64_t c = 0; c < dv; ++c) on[c] = 0.0;
+        for (int64_t i = 0; i < cnt; ++i) {
+            const int64_t sl = (p0 + i) % W;
+            for (int64_t c = 0; c < dv; ++c)
+                on[c] += s[i] * rodref_e4m3_decode(a->vc[((n * H + h) * W + sl) * dv + c]) * a->v_scale;
+        }
+        for (int64_t c = 0; c < dv; ++c) on[c] /= l;
+    }
+    free(s);
+}
+
+int rodref_swska_decode_fp8(const float* q, const float* k_new, const float* v_new, uint8_t* k_cache,
+                            uint8_t* v_cache, const int64_t* pos, double* o, int64_t N, int64_t H,
+                            int64_t dk, int64_t dv, int64_t W, double scale, double k_scale,
+                            double v_scale, int nthreads) {
+    if (!q || !k_new || !v_new || !k_cache || !v_cache || !pos || !o) return RODREF_EINVAL;
+    if (N < 0 || H < 1 || dk < 1 || dv < 1 || W < 1 || !(k_scale > 0) || !(v_scale > 0)) return RODREF_EINVAL;
+    ska_dec8_args_t a = {q, k_new, v_new, k_cache, v_cache, pos, o, H, dk, dv, W, scale, k_scale, v_scale};
+    return run_units(ska_dec8_unit, &a, N, nthreads);
+}
+
+/* Prefill -> decode hand-off into FP8 rings: positions [max(0, T-W), T) of k [B,T,dk] and
+ * v [B,H,T,dv] go to slot p mod W as e4m3(x / scale); other slots are untouched. */
+int rodref_swska_cache_fill_fp8(const float* k, const float* v, uint8_t* k_cache, uint8_t* v_cache,
+                                int64_t B, int64_t H, int64_t T, int64_t dk, int64_t dv, int64_t W,
+                                float k_scale, float v_scale) {
+    if (!k || !v || !k_cache || !v_cache) return RODREF_EINVAL;
+    if (B < 0 || H < 1 || T < 0 || dk < 1 || dv < 1 || W < 1 || !(k_scale > 0.f) || !(v_scale > 0.f))
+        return RODREF_EINVAL;
+    const int64_t p0 = T > W ? T - W : 0;
+    for (int64_t b = 0; b < B; ++b)
+        for (int64_t p = p0; p < T; ++p) {
+            const int64_t slot = p % W;
+            for (int64_t c = 0; c < dk; ++c)
+                k_cache[(b * W + slot) * dk + c] = rodref_e4m3_encode(k[(b * T + p) * dk + c] / k_scale);
+            for (int64_t h = 0; h < H; ++h)
+                for (int64_t c = 0; c < dv; ++c)
+                    v_cache[((b * H + h) * W + slot) * dv + c] =
+                        rodref_e4m3_encode(v[((b * H + h) * T + p) * dv + c] / v_scale);
         }
     return 0;
 }

@@ -6,7 +6,9 @@ term, the readout using k, an off-by-one window, a dropped scale or normaliser, 
 ring-buffer slot, a hand-off that drops a token or numbers slots from the window start, a paged cache read
 without its table or written at the wrong row, a backward that weights the gate gradient
 with the updated state or decays the gradient state on the wrong channel, an attention backward
-without the softmax row term or with the shared key's gradient from one head), builds the copy with gcc and runs every pin against it. Each planted
+without the softmax row term or with the shared key's gradient from one head, an E4M3 encoder
+that breaks ties to the odd code, misplaces the subnormals or does not saturate, an FP8 decode
+that forgets the value scale, an FP8 fill that multiplies by the scale), builds the copy with gcc and runs every pin against it. Each planted
 mistake must make at least one pin fail; otherwise the pins are too weak to trust.
 """
 import inspect
@@ -52,6 +54,14 @@ MUTATIONS = {
                                     "for (int64_t h = 0; h < 1; ++h) acc += dkp[(b * H + h) * T * dk + i];"),
     "paged_write_wrong_row": ("t = table[n * pps + s / page], r = s % page;\n            memcpy(k_pool",
                               "t = table[n * pps + s / page], r = (s + 1) % page;\n            memcpy(k_pool"),
+    "e4m3_ties_to_odd": ("(d == best_d && (c & 1) == 0 && (best & 1) == 1)",
+                         "(d == best_d && (c & 1) == 1 && (best & 1) == 0)"),
+    "e4m3_subnormal_exponent": ("v = ldexp((double)m / 8.0, -6);", "v = ldexp((double)m / 8.0, -7);"),
+    "e4m3_no_saturation": ("if (a > 448.0) best = 0x7E;", "if (a > 464.0) best = 0x7F;"),
+    "fp8_decode_v_unscaled": ("on[c] += s[i] * rodref_e4m3_decode(a->vc[((n * H + h) * W + sl) * dv + c]) * a->v_scale;",
+                              "on[c] += s[i] * rodref_e4m3_decode(a->vc[((n * H + h) * W + sl) * dv + c]);"),
+    "fp8_fill_scale_multiplies": ("k_cache[(b * W + slot) * dk + c] = rodref_e4m3_encode(k[(b * T + p) * dk + c] / k_scale);",
+                                  "k_cache[(b * W + slot) * dk + c] = rodref_e4m3_encode(k[(b * T + p) * dk + c] * k_scale);"),
 }
 
 

@@ -499,3 +499,96 @@ def test_swska_backward_matches_torch_autograd(W):
     np.testing.assert_allclose(dq, tq.grad.numpy(), rtol=1e-10, atol=1e-12)
     np.testing.assert_allclose(dk_, tk.grad.numpy(), rtol=1e-10, atol=1e-12)
     np.testing.assert_allclose(dv_, tv.grad.numpy(), rtol=1e-10, atol=1e-12)
+
+
+# ------------------------------------------------------------------------------------------
+# FP8 (E4M3) window cache (SALA blog §4.3: the KV cache stored in FP8)
+# ------------------------------------------------------------------------------------------
+
+
+def test_e4m3_codebook_closed_forms():
+    """Values fixed by the E4M3 definition (1 sign, 4 exponent bits with bias 7, 3 mantissa bits,
+    exponent field 0 subnormal, S.1111.111 NaN): zero, the subnormal step 2^-9, the smallest
+    normal 2^-6, one, the largest finite 448, the sign bit."""
+    d = oracle.e4m3_decode(np.arange(256, dtype=np.uint8))
+    assert d[0x00] == 0.0 and math.copysign(1.0, d[0x80]) == -1.0
+    assert d[0x01] == 2.0 ** -9 and d[0x07] == 7 * 2.0 ** -9
+    assert d[0x08] == 2.0 ** -6 and d[0x38] == 1.0 and d[0x39] == 1.125
+    assert d[0x77] == 1.875 * 2 ** 7 and d[0x7E] == 448.0 and d[0xFE] == -448.0
+    assert np.isnan(d[0x7F]) and np.isnan(d[0xFF])
+    finite = d[np.isfinite(d)]
+    assert finite.size == 254  # every code but the two NaNs
+    pos = d[:0x7F]
+    assert (np.diff(pos) > 0).all()  # non-negative codes in increasing order
+
+
+def test_e4m3_encode_round_trip_ties_and_saturation():
+    codes = np.array([c for c in range(256) if c not in (0x7F, 0xFF)], dtype=np.uint8)
+    vals = oracle.e4m3_decode(codes).astype(np.float32)
+    np.testing.assert_array_equal(oracle.e4m3_encode(vals), codes)  # exact values round-trip
+    # midpoints between neighbouring codes go to the even code
+    lo = oracle.e4m3_decode(np.arange(0, 0x7E, dtype=np.uint8))
+    hi = oracle.e4m3_decode(np.arange(1, 0x7F, dtype=np.uint8))
+    mid = ((lo + hi) / 2).astype(np.float32)
+    assert np.array_equal(mid.astype(np.float64), (lo + hi) / 2)  # the midpoints are exact in fp32
+    enc = oracle.e4m3_encode(mid).astype(int)
+    expect = np.where(np.arange(0, 0x7E) % 2 == 0, np.arange(0, 0x7E), np.arange(1, 0x7F))
+    np.testing.assert_array_equal(enc, expect)
+    # saturation at +-448, NaN stays NaN
+    np.testing.assert_array_equal(oracle.e4m3_encode(np.array([449, 464, 1e9, np.inf, -500, -np.inf], np.float32)),
+                                  np.array([0x7E, 0x7E, 0x7E, 0x7E, 0xFE, 0xFE], np.uint8))
+    assert oracle.e4m3_encode(np.array([np.nan], np.float32))[0] & 0x7F == 0x7F
+    # the scale divides in fp32 before rounding
+    np.testing.assert_array_equal(oracle.e4m3_encode(np.array([3.0], np.float32), scale=2.0),
+                                  oracle.e4m3_encode(np.array([1.5], np.float32)))
+
+
+def test_e4m3_encode_matches_torch_float8_in_range():
+    """PyTorch's float8_e4m3fn conversion (a library routine, round to nearest even) agrees code
+    for code on values inside the finite range (PyTorch does not saturate beyond it)."""
+    r = _rng(7).normal(0, 40, 200000).astype(np.float32)
+    r = np.concatenate([r[np.abs(r) <= 448], _rng(8).uniform(-2 ** -5, 2 ** -5, 20000).astype(np.float32)])
+    t = torch.from_numpy(r).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+    np.testing.assert_array_equal(oracle.e4m3_encode(r), t)
+
+
+@pytest.mark.parametrize("W,T,steps,ks,vs", [(8, 5, 6, 1.0, 1.0), (5, 23, 7, 0.25, 2.0), (1, 4, 3, 1.0, 0.5)])
+def test_swska_fp8_cache_fill_then_decode_equals_prefill_of_dequantized_kv(W, T, steps, ks, vs):
+    """With FP8 rings, decode reads value(code) * scale: filling the rings from a T-token prefill
+    and decoding positions T .. T+steps-1 reproduces the (pinned) fp64 prefill of the whole
+    sequence run on the dequantized keys and values, e4m3(x / scale) * scale."""
+    H, dk, dv, B = 3, 6, 5, 2
+    total = T + steps
+    q, k, v = _ska_case(B=B, H=H, T=total, dk=dk, dv=dv, seed=21)
+    kq = (oracle.e4m3_decode(oracle.e4m3_encode(k, ks)) * np.float32(ks)).astype(np.float32)
+    vq = (oracle.e4m3_decode(oracle.e4m3_encode(v, vs)) * np.float32(vs)).astype(np.float32)
+    o_pre = oracle.swska_prefill(q, kq, vq, W)
+    kc = np.full((B, W, dk), 0x55, np.uint8)
+    vc = np.full((B, H, W, dv), 0x55, np.uint8)
+    kc, vc = oracle.swska_cache_fill_fp8(k[:, :T], v[:, :, :T], kc, vc, W, ks, vs)
+    if T < W:
+        assert (kc[:, T:] == 0x55).all() and (vc[:, :, T:] == 0x55).all()
+    for P in range(T, total):
+        o, kc, vc = oracle.swska_decode_fp8(q[:, :, P], k[:, P], v[:, :, P], kc, vc,
+                                            np.full(B, P, np.int64), W, k_scale=ks, v_scale=vs)
+        _close(o, o_pre[:, :, P], 1e-13)
+
+
+def test_swska_fp8_decode_writes_codes_and_rejects_negative_position():
+    H, dk, dv, N, W = 2, 4, 3, 3, 6
+    r = _rng(23)
+    q = r.standard_normal((N, H, dk)).astype(np.float32)
+    kn = r.standard_normal((N, dk)).astype(np.float32)
+    vn = r.standard_normal((N, H, dv)).astype(np.float32)
+    kc = oracle.e4m3_encode(r.standard_normal((N, W, dk)).astype(np.float32))
+    vc = oracle.e4m3_encode(r.standard_normal((N, H, W, dv)).astype(np.float32))
+    pos = np.array([9, 2, -1], np.int64)
+    o, kc2, vc2 = oracle.swska_decode_fp8(q, kn, vn, kc, vc, pos, W, k_scale=0.5, v_scale=0.5)
+    np.testing.assert_array_equal(kc2[0, 9 % W], oracle.e4m3_encode(kn[0], 0.5))
+    np.testing.assert_array_equal(vc2[1, :, 2], oracle.e4m3_encode(vn[1], 0.5))
+    np.testing.assert_array_equal(kc2[2], kc[2])  # the rejected sequence's cache is untouched
+    np.testing.assert_array_equal(vc2[2], vc[2])
+    assert np.isnan(o[2]).all() and np.isfinite(o[:2]).all()
+    # only the new slot changed for the accepted sequences
+    changed = (kc2 != kc).any(axis=-1)
+    assert not changed[0, [s for s in range(W) if s != 9 % W]].any()
