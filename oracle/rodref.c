@@ -673,15 +673,15 @@ int rodref_swska_cache_fill_fp8(const float* k, const float* v, uint8_t* k_cache
     if (!k || !v || !k_cache || !v_cache) return RODREF_EINVAL;
     if (B < 0 || H < 1 || T < 0 || dk < 1 || dv < 1 || W < 1 || !(k_scale > 0.f) || !(v_scale > 0.f))
         return RODREF_EINVAL;
-    const int64_t p0 = T > W ? T - W : 0;
+    const int64_t first = T > W ? T - W : 0;  /* the oldest position still in the window */
     for (int64_t b = 0; b < B; ++b)
-        for (int64_t p = p0; p < T; ++p) {
-            const int64_t slot = p % W;
+        for (int64_t p = first; p < T; ++p) {
+            const int64_t ring_slot = p % W;
             for (int64_t c = 0; c < dk; ++c)
-                k_cache[(b * W + slot) * dk + c] = rodref_e4m3_encode(k[(b * T + p) * dk + c] / k_scale);
+                k_cache[(b * W + ring_slot) * dk + c] = rodref_e4m3_encode(k[(b * T + p) * dk + c] / k_scale);
             for (int64_t h = 0; h < H; ++h)
                 for (int64_t c = 0; c < dv; ++c)
-                    v_cache[((b * H + h) * W + slot) * dv + c] =
+                    v_cache[((b * H + h) * W + ring_slot) * dv + c] =
                         rodref_e4m3_encode(v[((b * H + h) * T + p) * dv + c] / v_scale);
         }
     return 0;

@@ -60,8 +60,8 @@ MUTATIONS = {
     "e4m3_no_saturation": ("if (a > 448.0) best = 0x7E;", "if (a > 464.0) best = 0x7F;"),
     "fp8_decode_v_unscaled": ("on[c] += s[i] * rodref_e4m3_decode(a->vc[((n * H + h) * W + sl) * dv + c]) * a->v_scale;",
                               "on[c] += s[i] * rodref_e4m3_decode(a->vc[((n * H + h) * W + sl) * dv + c]);"),
-    "fp8_fill_scale_multiplies": ("k_cache[(b * W + slot) * dk + c] = rodref_e4m3_encode(k[(b * T + p) * dk + c] / k_scale);",
-                                  "k_cache[(b * W + slot) * dk + c] = rodref_e4m3_encode(k[(b * T + p) * dk + c] * k_scale);"),
+    "fp8_fill_scale_multiplies": ("k_cache[(b * W + ring_slot) * dk + c] = rodref_e4m3_encode(k[(b * T + p) * dk + c] / k_scale);",
+                                  "k_cache[(b * W + ring_slot) * dk + c] = rodref_e4m3_encode(k[(b * T + p) * dk + c] * k_scale);"),
 }
 
 
