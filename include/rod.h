@@ -267,6 +267,33 @@ ROD_API int rod_swska_decode_paged(const void* q, const void* k_new, const void*
 ROD_API int rod_swska_cache_fill(const void* k, const void* v, void* k_cache, void* v_cache, int B,
                                  int H, int T, int dk, int dv, int window, int dtype, void* stream);
 
+/* ---- SW-SKA: FP8 (E4M3) window cache ------------------------------------------------------- */
+/*
+ * The ring-buffer decode and the hand-off with the window cache stored in FP8 (SALA blog §4.3:
+ * the KV cache in FP8 halves its memory and speeds decode). The pages name FP8 only; this
+ * library reads it as the OCP E4M3 format (1 sign bit, 4 exponent bits with bias 7, 3 mantissa
+ * bits, no infinities, largest finite value 448) with one fp32 scale per cache:
+ *   code = the E4M3 value nearest to x / scale (quotient in fp32, ties to the even code,
+ *          magnitudes past 448 saturated),   value read = value(code) * scale.
+ *
+ * rod_swska_decode_fp8: as rod_swska_decode, with k_cache [N,W,dk] and v_cache [N,H,W,dv] of
+ * E4M3 codes (one byte each). The new token's k_new / v_new (bf16) are written to slot
+ * pos[n] mod W as codes first; attention then reads every window entry, the new one included,
+ * from the cache. q, k_new, v_new, o: bf16 in the layouts of rod_swska_decode; k_scale,
+ * v_scale > 0 (finite). Only dk = dv = 128 and 1 <= H <= 16.
+ * rod_swska_cache_fill_fp8: as rod_swska_cache_fill into E4M3 rings (k, v bf16).
+ * A negative pos[n] leaves that sequence's caches untouched and its output NaN.
+ * Errors: ROD_ERR_NULL, ROD_ERR_SHAPE (dims or H unsupported, window < 1, a scale not positive
+ * and finite), ROD_ERR_ALIGN, ROD_ERR_CUDA. N = 0 (B = 0, T = 0) is a no-op.
+ */
+ROD_API int rod_swska_decode_fp8(const void* q, const void* k_new, const void* v_new, void* k_cache,
+                                 void* v_cache, const int64_t* pos, void* o, int N, int H, int dk,
+                                 int dv, int window, float scale, float k_scale, float v_scale,
+                                 void* stream);
+ROD_API int rod_swska_cache_fill_fp8(const void* k, const void* v, void* k_cache, void* v_cache, int B,
+                                     int H, int T, int dk, int dv, int window, float k_scale,
+                                     float v_scale, void* stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -565,22 +565,36 @@ double rodref_e4m3_decode(uint8_t code) {
     return sign ? -v : v;
 }
 
-/* nearest E4M3 code to the fp32 value x: every non-negative finite code (0x00 .. 0x7E) is a
- * candidate for |x|, the closest wins, a tie goes to the even code; magnitudes beyond 448 take
- * 448 (saturation); the sign bit is x's; NaN gives 0x7F */
+/* The 256 code values, evaluated from rodref_e4m3_decode once before any worker thread starts
+ * (every entry point below fills it first; filling twice writes the same numbers). */
+static double e4m3_table[256];
+static int e4m3_table_ready = 0;
+static void e4m3_fill_table(void) {
+    if (e4m3_table_ready) return;
+    for (int c = 0; c < 256; ++c) e4m3_table[c] = rodref_e4m3_decode((uint8_t)c);
+    e4m3_table_ready = 1;
+}
+
+/* nearest E4M3 code to the fp32 value x: the non-negative finite codes 0x00 .. 0x7E have
+ * increasing values, so bisection finds the last code whose value is <= |x|; of it and the next
+ * code the closer one wins, a tie goes to the even code; magnitudes beyond 448 take 448
+ * (saturation); the sign bit is x's; NaN gives 0x7F */
 uint8_t rodref_e4m3_encode(float x) {
+    e4m3_fill_table();
     if (isnan(x)) return 0x7F;
     const double a = fabs((double)x);
-    int best = 0;
-    double best_d = INFINITY;
-    for (int c = 0; c <= 0x7E; ++c) {
-        const double d = fabs(rodref_e4m3_decode((uint8_t)c) - a);
-        if (d < best_d || (d == best_d && (c & 1) == 0 && (best & 1) == 1)) {
-            best = c;
-            best_d = d;
+    int best;
+    if (a >= 448.0) {
+        best = 0x7E;
+    } else {
+        int lo = 0, hi = 0x7E;  /* value(lo) <= a < value(hi) */
+        while (hi - lo > 1) {
+            const int mid = (lo + hi) / 2;
+            if (e4m3_table[mid] <= a) lo = mid; else hi = mid;
         }
+        const double dl = a - e4m3_table[lo], dh = e4m3_table[hi] - a;
+        best = dl < dh ? lo : (dh < dl ? hi : ((lo & 1) == 0 ? lo : hi));
     }
-    if (a > 448.0) best = 0x7E;
     return (uint8_t)(best | (signbit(x) ? 0x80 : 0));
 }
 
@@ -592,7 +606,8 @@ int rodref_e4m3_encode_array(const float* x, uint8_t* out, int64_t n, float scal
 
 int rodref_e4m3_decode_array(const uint8_t* c, double* out, int64_t n) {
     if (!c || !out || n < 0) return RODREF_EINVAL;
-    for (int64_t i = 0; i < n; ++i) out[i] = rodref_e4m3_decode(c[i]);
+    e4m3_fill_table();
+    for (int64_t i = 0; i < n; ++i) out[i] = e4m3_table[c[i]];
     return 0;
 }
 
@@ -634,7 +649,7 @@ static void ska_dec8_unit(const void* p, int64_t n) {
             const int64_t sl = (p0 + i) % W;
             double acc = 0.0;
             for (int64_t c = 0; c < dk; ++c)
-                acc += (double)qv[c] * rodref_e4m3_decode(a->kc[(n * W + sl) * dk + c]) * a->k_scale;
+                acc += (double)qv[c] * e4m3_table[a->kc[(n * W + sl) * dk + c]] * a->k_scale;
             s[i] = a->scale * acc;
             if (s[i] > m) m = s[i];
         }
@@ -648,7 +663,7 @@ static void ska_dec8_unit(const void* p, int64_t n) {
         for (int64_t i = 0; i < cnt; ++i) {
             const int64_t sl = (p0 + i) % W;
             for (int64_t c = 0; c < dv; ++c)
-                on[c] += s[i] * rodref_e4m3_decode(a->vc[((n * H + h) * W + sl) * dv + c]) * a->v_scale;
+                on[c] += s[i] * e4m3_table[a->vc[((n * H + h) * W + sl) * dv + c]] * a->v_scale;
         }
         for (int64_t c = 0; c < dv; ++c) on[c] /= l;
     }
@@ -661,6 +676,7 @@ int rodref_swska_decode_fp8(const float* q, const float* k_new, const float* v_n
                             double v_scale, int nthreads) {
     if (!q || !k_new || !v_new || !k_cache || !v_cache || !pos || !o) return RODREF_EINVAL;
     if (N < 0 || H < 1 || dk < 1 || dv < 1 || W < 1 || !(k_scale > 0) || !(v_scale > 0)) return RODREF_EINVAL;
+    e4m3_fill_table();
     ska_dec8_args_t a = {q, k_new, v_new, k_cache, v_cache, pos, o, H, dk, dv, W, scale, k_scale, v_scale};
     return run_units(ska_dec8_unit, &a, N, nthreads);
 }

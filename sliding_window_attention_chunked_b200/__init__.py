@@ -14,6 +14,10 @@ the calls raise.
     swska_cache_fill(k, v, k_cache, v_cache, window)   prefill -> decode ring-buffer hand-off
     swska_decode_paged(q, k_new, v_new, k_pool, v_pool, block_table, page_size, pos, window)
                                                     decode over a paged window cache
+    swska_decode_fp8(q, k_new, v_new, k_cache, v_cache, pos, window, k_scale=1, v_scale=1)
+                                                    decode over an FP8 (E4M3) window cache
+    swska_cache_fill_fp8(k, v, k_cache, v_cache, window, k_scale=1, v_scale=1)
+                                                    hand-off into FP8 rings
 """
 from ._binding import (  # noqa: F401
     ROD_BF16,
@@ -31,7 +35,9 @@ from ._binding import (  # noqa: F401
     load_library,
     swska_backward,
     swska_cache_fill,
+    swska_cache_fill_fp8,
     swska_decode,
+    swska_decode_fp8,
     swska_decode_paged,
     swska_prefill,
 )

@@ -78,6 +78,10 @@ def load_library() -> ctypes.CDLL:
     lib.rod_swska_backward.argtypes = [vp] * 7 + [i] * 6 + [f, i, vp, sz, vp]
     lib.rod_swska_backward.restype = i
     lib.rod_swska_cache_fill.restype = i
+    lib.rod_swska_decode_fp8.argtypes = [vp, vp, vp, vp, vp, vp, vp, i, i, i, i, i, f, f, f, vp]
+    lib.rod_swska_decode_fp8.restype = i
+    lib.rod_swska_cache_fill_fp8.argtypes = [vp, vp, vp, vp, i, i, i, i, i, i, f, f, vp]
+    lib.rod_swska_cache_fill_fp8.restype = i
     _lib = lib
     return lib
 
@@ -355,3 +359,63 @@ def swska_backward(q, k, v, dO, window, scale=None, workspace=None, stream=None)
                                 _ptr(workspace), workspace.numel(), _stream(stream))
     _raise_on("rod_swska_backward", st)
     return dq, dk_, dv_
+
+
+def _need_codes(t, name, ndim):
+    """An FP8 cache: a CUDA tensor of one-byte E4M3 codes (uint8 or float8_e4m3fn), contiguous."""
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a torch.Tensor")
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be on a CUDA device")
+    if t.dtype not in (torch.uint8, torch.float8_e4m3fn):
+        raise ValueError(f"{name} must hold E4M3 codes (uint8 or float8_e4m3fn), got {t.dtype}")
+    if t.dim() != ndim or not t.is_contiguous():
+        raise ValueError(f"{name} must be a contiguous {ndim}-d tensor")
+
+
+def swska_decode_fp8(q, k_new, v_new, k_cache, v_cache, pos, window, scale=None, k_scale=1.0,
+                     v_scale=1.0, o=None, stream=None):
+    """Ring-buffer decode over FP8 caches (SALA blog §4.3): k_cache [N,W,dk] and v_cache
+    [N,H,W,dv] hold E4M3 codes (value = code * scale) and are updated in place at slot pos mod W
+    with the quantized new token. q [N,H,dk], k_new [N,dk], v_new [N,H,dv] bf16, pos [N] int64.
+    Returns o [N,H,dv] bf16."""
+    _need(q, "q", torch.bfloat16, 3)
+    _need(k_new, "k_new", torch.bfloat16, 2)
+    _need(v_new, "v_new", torch.bfloat16, 3)
+    _need_codes(k_cache, "k_cache", 3)
+    _need_codes(v_cache, "v_cache", 4)
+    _need(pos, "pos", torch.int64, 1)
+    N, H, dk = q.shape
+    dv = v_new.shape[-1]
+    W = int(window)
+    if (tuple(k_new.shape) != (N, dk) or tuple(k_cache.shape) != (N, W, dk)
+            or tuple(v_cache.shape) != (N, H, W, dv) or pos.shape[0] != N):
+        raise ValueError("shape mismatch")
+    if o is None:
+        o = torch.empty((N, H, dv), dtype=q.dtype, device=q.device)
+    _need(o, "o", q.dtype, 3)
+    st = load_library().rod_swska_decode_fp8(_ptr(q), _ptr(k_new), _ptr(v_new), _ptr(k_cache),
+                                             _ptr(v_cache), _ptr(pos), _ptr(o), N, H, dk, dv, W,
+                                             float(scale or 0.0), float(k_scale), float(v_scale),
+                                             _stream(stream))
+    _raise_on("rod_swska_decode_fp8", st)
+    return o
+
+
+def swska_cache_fill_fp8(k, v, k_cache, v_cache, window, k_scale=1.0, v_scale=1.0, stream=None):
+    """Prefill -> decode hand-off into FP8 rings: k [B,T,dk], v [B,H,T,dv] (bf16) quantized into
+    k_cache [B,W,dk], v_cache [B,H,W,dv] (E4M3 codes of x / scale at slot p mod W)."""
+    _need(k, "k", torch.bfloat16, 3)
+    _need(v, "v", torch.bfloat16, 4)
+    _need_codes(k_cache, "k_cache", 3)
+    _need_codes(v_cache, "v_cache", 4)
+    B, T, dk = k.shape
+    H, dv = v.shape[1], v.shape[-1]
+    W = int(window)
+    if (tuple(v.shape) != (B, H, T, dv) or tuple(k_cache.shape) != (B, W, dk)
+            or tuple(v_cache.shape) != (B, H, W, dv)):
+        raise ValueError("shape mismatch")
+    st = load_library().rod_swska_cache_fill_fp8(_ptr(k), _ptr(v), _ptr(k_cache), _ptr(v_cache), B, H, T,
+                                                 dk, dv, W, float(k_scale), float(v_scale), _stream(stream))
+    _raise_on("rod_swska_cache_fill_fp8", st)
+    return k_cache, v_cache

@@ -105,6 +105,16 @@ cudaError_t swska_backward_tc_launch(const SkaBackwardArgs& a, cudaStream_t stre
 unsigned swska_backward_tc_take_timeout_flag();
 cudaError_t gla_backward_launch(const GlaBackwardArgs& a, bool bf16, cudaStream_t stream);
 
+// SW-SKA decode with FP8 (E4M3) ring caches: k_cache [N,W,128], v_cache [N,H,W,128] codes,
+// value = code * scale; q, k_new, v_new, o bf16
+cudaError_t swska_decode_fp8_launch(const void* q, const void* k_new, const void* v_new, void* k_cache,
+                                    void* v_cache, const int64_t* pos, void* o, int N, int H, int window,
+                                    float scale, float k_scale, float v_scale, cudaStream_t stream);
+// hand-off into FP8 rings (bf16 prefill rows quantized as e4m3(x / scale))
+cudaError_t swska_cache_fill_fp8_launch(const void* k, const void* v, void* k_cache, void* v_cache, int B,
+                                        int H, int T, int dk, int dv, int window, float k_scale, float v_scale,
+                                        cudaStream_t stream);
+
 // SW-SKA prefill -> decode hand-off: the last W tokens' K / V rows into the ring buffers
 cudaError_t swska_cache_fill_launch(const void* k, const void* v, void* k_cache, void* v_cache, int B,
                                     int H, int T, int dk, int dv, int window, size_t elem_bytes,

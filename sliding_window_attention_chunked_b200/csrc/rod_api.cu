@@ -242,4 +242,32 @@ int rod_swska_cache_fill(const void* k, const void* v, void* k_cache, void* v_ca
                                                   static_cast<cudaStream_t>(stream)));
 }
 
+static bool scale_ok(float s) { return s > 0.f && !isinf(s) && s == s; }
+
+int rod_swska_decode_fp8(const void* q, const void* k_new, const void* v_new, void* k_cache, void* v_cache,
+                         const int64_t* pos, void* o, int N, int H, int dk, int dv, int window, float scale,
+                         float k_scale, float v_scale, void* stream) {
+    if (N < 0 || !rod::swska_decode_warp_supported(H, dk, dv) || window < 1) return ROD_ERR_SHAPE;
+    if (!(scale == scale) || isinf(scale) || !scale_ok(k_scale) || !scale_ok(v_scale)) return ROD_ERR_SHAPE;
+    if (N == 0) return ROD_OK;
+    if (!q || !k_new || !v_new || !k_cache || !v_cache || !pos || !o) return ROD_ERR_NULL;
+    if (!aligned16(q) || !aligned16(k_new) || !aligned16(v_new) || !aligned16(k_cache) ||
+        !aligned16(v_cache) || !aligned16(pos) || !aligned16(o))
+        return ROD_ERR_ALIGN;
+    return from_cuda(rod::swska_decode_fp8_launch(q, k_new, v_new, k_cache, v_cache, pos, o, N, H, window,
+                                                  resolve_scale(scale, dk), k_scale, v_scale,
+                                                  static_cast<cudaStream_t>(stream)));
+}
+
+int rod_swska_cache_fill_fp8(const void* k, const void* v, void* k_cache, void* v_cache, int B, int H, int T,
+                             int dk, int dv, int window, float k_scale, float v_scale, void* stream) {
+    if (B < 0 || T < 0 || window < 1 || !rod::swska_decode_warp_supported(H, dk, dv)) return ROD_ERR_SHAPE;
+    if (!scale_ok(k_scale) || !scale_ok(v_scale)) return ROD_ERR_SHAPE;
+    if (B == 0 || T == 0) return ROD_OK;
+    if (!k || !v || !k_cache || !v_cache) return ROD_ERR_NULL;
+    if (!aligned16(k) || !aligned16(v) || !aligned16(k_cache) || !aligned16(v_cache)) return ROD_ERR_ALIGN;
+    return from_cuda(rod::swska_cache_fill_fp8_launch(k, v, k_cache, v_cache, B, H, T, dk, dv, window, k_scale,
+                                                      v_scale, static_cast<cudaStream_t>(stream)));
+}
+
 }  // extern "C"

@@ -30,16 +30,26 @@
 //    all HG head warps have read the stage.
 //  * The SP partial (max, sum, accumulator) triples meet in distributed shared memory; CTA r
 //    finalises the heads h with h mod SP == r.
+//  * FP8 instance (SALA blog §4.3: the window cache stored in FP8): the rings hold OCP E4M3 codes
+//    with one fp32 scale per cache, so a row is 128 bytes and a stage half the bytes. A lane's 4
+//    channels are one 32-bit word, converted to f16 (exactly: every E4M3 value is an f16) and
+//    multiplied with q (held in f16) by f16 x f16 -> fp32 FMAs; p is rounded to f16 for V. The
+//    K scale folds into the score scale and the V scale into the final normalisation. The new
+//    token is quantized by the producer: x / scale in fp32, then the nearest E4M3 code (ties to
+//    even, saturated at +-448), into the stage and the cache.
 // Every wait is bounded. On expiry the waiting warp raises the CTA's abort flag, every role stops
 // at its next wait, the producer waits (bounded) for the copies it issued, the timeout flag is
 // raised, the affected outputs are NaN, and all threads still meet at the cluster barriers.
 #include <cooperative_groups.h>
+#include <cuda_fp16.h>
+#include <cuda_fp8.h>
 
 #include <math.h>
 
 #include <mutex>
 
 #include "common.cuh"
+#include "fp8.cuh"
 #include "kernels.h"
 
 namespace cg = cooperative_groups;
@@ -53,19 +63,21 @@ constexpr int KT = 8;            // slots per stage
 constexpr int MAX_STAGES = 16;   // ring depth limit (the depth is a launch parameter)
 constexpr int DH = 128;          // d_k = d_v
 constexpr int ROW = DH * 2;      // bytes of one bf16 row
+constexpr int ROW8 = DH;         // bytes of one E4M3 row
 constexpr int MAX_H = 16;        // heads per CTA (one warp each)
+template <bool FP8> constexpr int row_bytes() { return FP8 ? ROW8 : ROW; }
 constexpr int OFF_FLAG = 256;    // after full[MAX_STAGES] and empty[MAX_STAGES]
 constexpr int OFF_PM = 320;      // per-head max   [MAX_H] f32
 constexpr int OFF_PL = 384;      // per-head sum   [MAX_H] f32
 constexpr int OFF_PACC = 512;    // per-head accumulator [HG][128] f32
 
-// HG: heads served by one CTA (warps 0 .. HG-1) next to the producer warp HG
-__host__ __device__ constexpr uint32_t stage_bytes(int HG) { return (uint32_t)(KT * ROW * (1 + HG)); }
+// HG: heads served by one CTA (warps 0 .. HG-1) next to the producer warp HG; row: bytes per row
+__host__ __device__ constexpr uint32_t stage_bytes(int HG, int row = ROW) { return (uint32_t)(KT * row * (1 + HG)); }
 __host__ __device__ constexpr uint32_t ring_offset(int HG) { return (uint32_t)(OFF_PACC + HG * DH * 4); }
 // a CTA's slice of a paged block table: at most pages_per_seq + 1 entries (ROD_MAX_PAGES_PER_SEQ)
 constexpr uint32_t kPageSlice = 520;
-__host__ __device__ constexpr uint32_t smem_total(int HG, int stages) {
-    return ring_offset(HG) + (uint32_t)stages * stage_bytes(HG) + 4u * kPageSlice;
+__host__ __device__ constexpr uint32_t smem_total(int HG, int stages, int row = ROW) {
+    return ring_offset(HG) + (uint32_t)stages * stage_bytes(HG, row) + 4u * kPageSlice;
 }
 
 __device__ __forceinline__ bool wait_stage(uint64_t* bar, uint32_t parity, volatile int* abort_flag) {
@@ -105,23 +117,44 @@ __device__ __forceinline__ void axpy4_bf16(uint32_t pw, uint2 w, float* acc) {
         : "+f"(acc[0]), "+f"(acc[1]), "+f"(acc[2]), "+f"(acc[3]) : "r"(pw), "r"(w.x), "r"(w.y));
 }
 
+// c + a.lo * b.lo + a.hi * b.hi for two packed f16 pairs: f16 operands, fp32 products and sum
+__device__ __forceinline__ float dot2_f16(uint32_t a, uint32_t b, float c) {
+    asm("{\n\t.reg .b16 al, ah, bl, bh;\n\tmov.b32 {al, ah}, %1;\n\tmov.b32 {bl, bh}, %2;\n\t"
+        "fma.rn.f32.f16 %0, al, bl, %0;\n\tfma.rn.f32.f16 %0, ah, bh, %0;\n\t}"
+        : "+f"(c) : "r"(a), "r"(b));
+    return c;
+}
+// acc[i] += p * v[i] for the 4 f16 in (w0, w1), p an f16 in the low half of pw; fp32 accumulation
+__device__ __forceinline__ void axpy4_f16(uint32_t pw, uint32_t w0, uint32_t w1, float* acc) {
+    asm("{\n\t.reg .b16 p, ph, v0, v1, v2, v3;\n\tmov.b32 {p, ph}, %4;\n\tmov.b32 {v0, v1}, %5;\n\t"
+        "mov.b32 {v2, v3}, %6;\n\tfma.rn.f32.f16 %0, p, v0, %0;\n\tfma.rn.f32.f16 %1, p, v1, %1;\n\t"
+        "fma.rn.f32.f16 %2, p, v2, %2;\n\tfma.rn.f32.f16 %3, p, v3, %3;\n\t}"
+        : "+f"(acc[0]), "+f"(acc[1]), "+f"(acc[2]), "+f"(acc[3]) : "r"(pw), "r"(w0), "r"(w1));
+}
 struct HeadState {
     float acc[4] = {0.f, 0.f, 0.f, 0.f};  // output columns 4 lane .. 4 lane + 3, unnormalised
     float m_run = -INFINITY;               // running max of the base-2 scores (warp-uniform)
     float l_part = 0.f;                    // this lane's share of the running sum
 };
 
-// One stage of KT slots for one head. kb / vb point at this lane's 8 bytes of the stage's first
-// K row and first V row of the head (rows ROW bytes apart). FULL: all KT rows are valid.
-template <bool FULL>
+// One stage of KT slots for one head. kb / vb point at this lane's 4 channels of the stage's first
+// K row and first V row of the head (8 bytes of bf16 or 4 of E4M3; rows row_bytes apart); qw is
+// the lane's 4 channels of q (bf16, or f16 for the FP8 instance). FULL: all KT rows are valid.
+template <bool FULL, bool FP8>
 __device__ __forceinline__ void head_stage(const unsigned char* kb, const unsigned char* vb, uint2 qw,
                                            float scale_log2, int rows, int lane, HeadState& hs) {
+    constexpr int RB = row_bytes<FP8>();
     // partial dots over this lane's 4 channels, one per slot
     float part[KT];
 #pragma unroll
     for (int j = 0; j < KT; ++j) {
-        const uint2 kw = *reinterpret_cast<const uint2*>(kb + j * ROW);
-        part[j] = dot2_bf16(kw.y, qw.y, dot2_bf16(kw.x, qw.x, 0.f));
+        if (FP8) {
+            const uint32_t kw = *reinterpret_cast<const uint32_t*>(kb + j * RB);
+            part[j] = dot2_f16(e4m3x2_to_f16x2(kw >> 16), qw.y, dot2_f16(e4m3x2_to_f16x2(kw), qw.x, 0.f));
+        } else {
+            const uint2 kw = *reinterpret_cast<const uint2*>(kb + j * RB);
+            part[j] = dot2_bf16(kw.y, qw.y, dot2_bf16(kw.x, qw.x, 0.f));
+        }
     }
     // reduce-scatter over the warp: halves of the slot set cross lane bit 4, then bit 3, then
     // bit 2; bits 1 and 0 finish the sums. Lane l ends with the score of slot (l >> 2) & 7.
@@ -158,16 +191,28 @@ __device__ __forceinline__ void head_stage(const unsigned char* kb, const unsign
         for (int i = 0; i < 4; ++i) hs.acc[i] *= alpha;
         hs.m_run = mx;
     }
-    // p in bf16 (as the weights of V); the sum takes the same rounded value
-    const __nv_bfloat16 pb = __float2bfloat16_rn(ex2_approx(s - hs.m_run));  // past the end: 0
-    if ((lane & 3) == 0) hs.l_part += __bfloat162float(pb);
-    const uint32_t pw = (uint32_t)__bfloat16_as_ushort(pb);
+    // p in bf16 (f16 for the FP8 instance) as the weights of V; the sum takes the same rounded value
+    uint32_t pw;
+    if (FP8) {
+        const __half ph = __float2half_rn(ex2_approx(s - hs.m_run));  // past the end: 0
+        if ((lane & 3) == 0) hs.l_part += __half2float(ph);
+        pw = (uint32_t)__half_as_ushort(ph);
+    } else {
+        const __nv_bfloat16 pb = __float2bfloat16_rn(ex2_approx(s - hs.m_run));
+        if ((lane & 3) == 0) hs.l_part += __bfloat162float(pb);
+        pw = (uint32_t)__bfloat16_as_ushort(pb);
+    }
 #pragma unroll
     for (int j = 0; j < KT; ++j) {
         const uint32_t pj = __shfl_sync(0xffffffffu, pw, 4 * j);
         if (FULL || j < rows) {  // rows past the end hold stale bytes
-            const uint2 vw = *reinterpret_cast<const uint2*>(vb + j * ROW);
-            axpy4_bf16(pj, vw, hs.acc);
+            if (FP8) {
+                const uint32_t vw = *reinterpret_cast<const uint32_t*>(vb + j * RB);
+                axpy4_f16(pj, e4m3x2_to_f16x2(vw), e4m3x2_to_f16x2(vw >> 16), hs.acc);
+            } else {
+                const uint2 vw = *reinterpret_cast<const uint2*>(vb + j * RB);
+                axpy4_bf16(pj, vw, hs.acc);
+            }
         }
     }
 }
@@ -177,10 +222,11 @@ __device__ __forceinline__ void head_stage(const unsigned char* kb, const unsign
 // window): the ring's slots are cut into pages of `page` slots; logical page i of sequence n is
 // physical page table[n * pps + i] of the pools k [pages][page][DH] and v [pages][H][page][DH].
 struct CacheRef {
-    __nv_bfloat16* k;
-    __nv_bfloat16* v;
+    unsigned char* k;      // rows of row_bytes (bf16 or E4M3)
+    unsigned char* v;
     const int32_t* table;  // paged only
     int page, pps;         // slots per page, pages per sequence (paged only)
+    float k_scale, v_scale;  // FP8 only: value = code * scale
 };
 // Paged lookups read the CTA's slice of the block table, staged in shared memory at kernel start
 // (pages[i] = table entry of logical page pg0 + i).
@@ -197,7 +243,7 @@ __device__ __forceinline__ int64_t v_row(const CacheRef& c, int64_t n, int H, in
     return ((int64_t)pages[slot / c.page - pg0] * H + h) * c.page + slot % c.page;
 }
 
-template <bool PAGED>
+template <bool PAGED, bool FP8>
 __global__ void __launch_bounds__(32 * (MAX_H + 1), 2)
 swska_decode_warp_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ k_new,
                          const __nv_bfloat16* __restrict__ v_new, CacheRef cache,
@@ -210,7 +256,8 @@ swska_decode_warp_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat1
     const int64_t n = blockIdx.x / SP;
     const int hg0 = (int)blockIdx.y * HG;  // this CTA serves heads hg0 .. hg0 + HG - 1
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const uint32_t SB = stage_bytes(HG);
+    constexpr int RB = row_bytes<FP8>();
+    const uint32_t SB = stage_bytes(HG, RB);
     uint64_t* full = reinterpret_cast<uint64_t*>(smem);
     uint64_t* empty = full + MAX_STAGES;
     volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + OFF_FLAG);
@@ -266,18 +313,20 @@ swska_decode_warp_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat1
                 // the evicted slot takes the new token: into the stage and into the cache (its
                 // old content lies outside the window, so it is never copied in); the shared K
                 // row goes to the cache from head group 0 only
-                for (int i = lane; i < (1 + HG) * (ROW / 16); i += 32) {
-                    const int row = i / (ROW / 16), c16 = i % (ROW / 16);
+                for (int i = lane; i < (1 + HG) * (RB / 16); i += 32) {
+                    const int row = i / (RB / 16), c16 = i % (RB / 16);
                     const int64_t hv = n * H + hg0 + (row - 1);  // (sequence, head) of a V row
                     const uint4* src = row == 0 ? reinterpret_cast<const uint4*>(k_new + n * DH)
                                                 : reinterpret_cast<const uint4*>(v_new + hv * DH);
-                    const uint4 val = src[c16];
-                    reinterpret_cast<uint4*>(dst + (size_t)row * KT * ROW + (size_t)r_new * ROW)[c16] = val;
+                    // FP8: 16 codes from 16 bf16 of the row, quantized with the cache's scale
+                    const uint4 val = FP8 ? quantize16(src[2 * c16], src[2 * c16 + 1], row == 0 ? cache.k_scale : cache.v_scale)
+                                          : src[c16];
+                    reinterpret_cast<uint4*>(dst + (size_t)row * KT * RB + (size_t)r_new * RB)[c16] = val;
                     if (row == 0) {
                         if (blockIdx.y == 0)
-                            reinterpret_cast<uint4*>(cache.k + k_row<PAGED>(cache, n, W, s_new, pages, pg0) * DH)[c16] = val;
+                            reinterpret_cast<uint4*>(cache.k + k_row<PAGED>(cache, n, W, s_new, pages, pg0) * RB)[c16] = val;
                     } else {
-                        reinterpret_cast<uint4*>(cache.v + v_row<PAGED>(cache, n, H, W, hg0 + row - 1, s_new, pages, pg0) * DH)[c16] = val;
+                        reinterpret_cast<uint4*>(cache.v + v_row<PAGED>(cache, n, H, W, hg0 + row - 1, s_new, pages, pg0) * RB)[c16] = val;
                     }
                 }
                 // the generic stores precede later bulk copies into the same bytes
@@ -285,10 +334,10 @@ swska_decode_warp_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat1
             }
             __syncwarp();
             const int copied = rows - (r_new >= 0 ? 1 : 0);
-            if (lane == 0) mbar_arrive_expect_tx(&full[buf], (uint32_t)(copied * ROW * (1 + HG)));
+            if (lane == 0) mbar_arrive_expect_tx(&full[buf], (uint32_t)(copied * RB * (1 + HG)));
             __syncwarp();
             if (lane <= HG) {  // lane 0: the K rows; lane 1 + h: head hg0 + h's V rows
-                unsigned char* d = dst + (size_t)lane * KT * ROW;
+                unsigned char* d = dst + (size_t)lane * KT * RB;
                 // rows s0 .. s0 + rows - 1 are contiguous (one page holds a whole stage)
                 int64_t row0;
                 if (PAGED) {
@@ -297,11 +346,11 @@ swska_decode_warp_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat1
                 } else {
                     row0 = lane == 0 ? n * W + s0 : (n * H + hg0 + lane - 1) * W + s0;
                 }
-                const __nv_bfloat16* src = (lane == 0 ? cache.k : cache.v) + row0 * DH;
+                const unsigned char* src = (lane == 0 ? cache.k : cache.v) + row0 * RB;
                 const int a0 = 0, a1 = r_new >= 0 ? r_new : rows;   // rows [a0, a1)
                 const int b0 = r_new >= 0 ? r_new + 1 : rows, b1 = rows;  // rows [b0, b1)
-                if (a1 > a0) bulk_g2s(d + (size_t)a0 * ROW, src + (int64_t)a0 * DH, (uint32_t)((a1 - a0) * ROW), &full[buf]);
-                if (b1 > b0) bulk_g2s(d + (size_t)b0 * ROW, src + (int64_t)b0 * DH, (uint32_t)((b1 - b0) * ROW), &full[buf]);
+                if (a1 > a0) bulk_g2s(d + (size_t)a0 * RB, src + (int64_t)a0 * RB, (uint32_t)((a1 - a0) * RB), &full[buf]);
+                if (b1 > b0) bulk_g2s(d + (size_t)b0 * RB, src + (int64_t)b0 * RB, (uint32_t)((b1 - b0) * RB), &full[buf]);
             }
             ++issued;
             if (++buf == stages) { buf = 0; par ^= 1u; }
@@ -319,7 +368,12 @@ swska_decode_warp_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat1
     else {
         // -------------------------- head warp h: head hg0 + h --------------------------
         const int h = warp;
-        const uint2 qw = *reinterpret_cast<const uint2*>(q + (n * H + hg0 + h) * (int64_t)DH + 4 * lane);
+        uint2 qw = *reinterpret_cast<const uint2*>(q + (n * H + hg0 + h) * (int64_t)DH + 4 * lane);
+        if (FP8) {  // q in f16 for the f16 x f16 products with the E4M3 rows
+            const __half2 a = __floats2half2_rn(bf16lo(qw.x), bf16hi(qw.x));
+            const __half2 b = __floats2half2_rn(bf16lo(qw.y), bf16hi(qw.y));
+            qw = make_uint2(*reinterpret_cast<const uint32_t*>(&a), *reinterpret_cast<const uint32_t*>(&b));
+        }
         HeadState hs;
         bool ok = true;
         int buf = 0;
@@ -331,10 +385,10 @@ swska_decode_warp_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat1
             }
             const int s0 = s_begin + st * KT;
             const int rows = s_end - s0 < KT ? s_end - s0 : KT;
-            const unsigned char* kb = ring + (size_t)buf * SB + 8 * lane;
-            const unsigned char* vb = kb + (size_t)(1 + h) * KT * ROW;
-            if (rows == KT) head_stage<true>(kb, vb, qw, scale_log2, KT, lane, hs);
-            else head_stage<false>(kb, vb, qw, scale_log2, rows, lane, hs);
+            const unsigned char* kb = ring + (size_t)buf * SB + (RB / 32) * lane;
+            const unsigned char* vb = kb + (size_t)(1 + h) * KT * RB;
+            if (rows == KT) head_stage<true, FP8>(kb, vb, qw, scale_log2, KT, lane, hs);
+            else head_stage<false, FP8>(kb, vb, qw, scale_log2, rows, lane, hs);
             __syncwarp();
             if (lane == 0) mbar_arrive(&empty[buf]);
             if (++buf == stages) { buf = 0; par ^= 1u; }
@@ -368,7 +422,7 @@ swska_decode_warp_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat1
                 a[0] = fmaf(w, pa.x, a[0]); a[1] = fmaf(w, pa.y, a[1]);
                 a[2] = fmaf(w, pa.z, a[2]); a[3] = fmaf(w, pa.w, a[3]);
             }
-            const float inv = 1.f / L;
+            const float inv = (FP8 ? cache.v_scale : 1.f) / L;
 #pragma unroll
             for (int i = 0; i < 4; ++i) out[i] = a[i] * inv;
         }
@@ -385,26 +439,26 @@ struct DecodeConfig {
 };
 
 // ring depth: about 64 KB of copies in flight per CTA, at least 3 stages
-int stages_for(int HG) {
-    int st = (int)(65536u / stage_bytes(HG));
+int stages_for(int HG, int row = ROW) {
+    int st = (int)(65536u / stage_bytes(HG, row));
     return st < 3 ? 3 : (st > MAX_STAGES ? MAX_STAGES : st);
 }
 
-template <bool PAGED>
+template <bool PAGED, bool FP8>
 cudaError_t set_attributes(size_t smem) {
-    cudaError_t e = cudaFuncSetAttribute(swska_decode_warp_kernel<PAGED>,
+    cudaError_t e = cudaFuncSetAttribute(swska_decode_warp_kernel<PAGED, FP8>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e == cudaSuccess)
-        e = cudaFuncSetAttribute(swska_decode_warp_kernel<PAGED>,
+        e = cudaFuncSetAttribute(swska_decode_warp_kernel<PAGED, FP8>,
                                  cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
     return e;
 }
 
-// Clusters of the given shape that the GPU holds at once (queried once per device and shape;
-// 0 if the shape cannot be launched).
-int clusters_that_fit(int HG, int sp) {
+// Clusters of the given shape that the GPU holds at once (queried once per device, shape and
+// cache format; 0 if the shape cannot be launched).
+int clusters_that_fit(int HG, int sp, bool fp8) {
     static std::mutex mu;
-    static int cache[64][MAX_H + 1][5];
+    static int cache[64][MAX_H + 1][5][2];
     static bool init = false;
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 0;
@@ -414,14 +468,16 @@ int clusters_that_fit(int HG, int sp) {
     if (!init) {
         for (auto& a : cache)
             for (auto& b : a)
-                for (int& c : b) c = -1;
+                for (auto& c : b)
+                    for (int& d : c) d = -1;
         init = true;
     }
-    int& slot = cache[dev][HG][si];
+    int& slot = cache[dev][HG][si][fp8 ? 1 : 0];
     if (slot < 0) {
-        const size_t smem = smem_total(HG, stages_for(HG));
+        const int row = fp8 ? ROW8 : ROW;
+        const size_t smem = smem_total(HG, stages_for(HG, row), row);
         int num = 0;
-        if (set_attributes<false>(smem) == cudaSuccess) {
+        if ((fp8 ? set_attributes<false, true>(smem) : set_attributes<false, false>(smem)) == cudaSuccess) {
             cudaLaunchConfig_t cfg = {};
             cfg.gridDim = dim3((unsigned)sp, 1, 1);
             cfg.blockDim = dim3((unsigned)(32 * (HG + 1)), 1, 1);
@@ -433,8 +489,10 @@ int clusters_that_fit(int HG, int sp) {
             attr[0].val.clusterDim.z = 1;
             cfg.attrs = attr;
             cfg.numAttrs = 1;
-            // the paged instance has the same resources
-            if (cudaOccupancyMaxActiveClusters(&num, swska_decode_warp_kernel<false>, &cfg) != cudaSuccess) num = 0;
+            // the paged instance has the same resources as the ring one
+            const cudaError_t q = fp8 ? cudaOccupancyMaxActiveClusters(&num, swska_decode_warp_kernel<false, true>, &cfg)
+                                      : cudaOccupancyMaxActiveClusters(&num, swska_decode_warp_kernel<false, false>, &cfg);
+            if (q != cudaSuccess) num = 0;
         }
         cudaGetLastError();
         slot = num;
@@ -449,18 +507,20 @@ int clusters_that_fit(int HG, int sp) {
 // where one CTA streams about 1/200 of the GPU's bandwidth (measured: ~31 GB/s against
 // 6.4 TB/s with 16 heads per CTA). Splitting the heads (fewer per CTA) and the window (bigger
 // clusters, up to 16) multiplies the CTAs for small batches at the price of reading K once per
-// head group. Among equal estimates the smaller split wins.
+// head group. Among equal estimates the smaller split wins. (Rows are the unit: the FP8 rows'
+// halved bytes scale both terms alike.)
 constexpr double kCtasToSaturate = 200.0;
 
-DecodeConfig pick_config(int N, int H, int W) {
-    DecodeConfig best{1, H, stages_for(H)};
+DecodeConfig pick_config(int N, int H, int W, bool fp8) {
+    const int row = fp8 ? ROW8 : ROW;
+    DecodeConfig best{1, H, stages_for(H, row)};
     double best_cost = -1.0;
     for (int HG = H; HG >= 1; --HG) {
         if (H % HG) continue;
         const int groups = H / HG;
         const double bytes = (double)N * W * (double)(groups + H);
         for (int sp = 1; sp <= 16; sp *= 2) {
-            const int64_t cap = (int64_t)clusters_that_fit(HG, sp) * sp;  // CTAs resident at once
+            const int64_t cap = (int64_t)clusters_that_fit(HG, sp, fp8) * sp;  // CTAs resident at once
             if (cap <= 0) continue;
             const int64_t ctas = (int64_t)N * sp * groups;
             const double waves = (double)((ctas + cap - 1) / cap);
@@ -469,7 +529,7 @@ DecodeConfig pick_config(int N, int H, int W) {
             const double cost = t > bytes ? t : bytes;
             if (best_cost < 0.0 || cost < best_cost * 0.98) {
                 best_cost = cost;
-                best = DecodeConfig{sp, HG, stages_for(HG)};
+                best = DecodeConfig{sp, HG, stages_for(HG, row)};
             }
         }
     }
@@ -484,13 +544,14 @@ bool swska_decode_warp_supported(int H, int dk, int dv) {
 
 namespace {
 
-template <bool PAGED>
+template <bool PAGED, bool FP8>
 cudaError_t launch(const void* q, const void* k_new, const void* v_new, CacheRef cache, const int64_t* pos,
                    void* o, int N, int H, int window, float scale, cudaStream_t stream) {
     if (N == 0) return cudaSuccess;
-    const DecodeConfig c = pick_config(N, H, window);
-    const size_t smem = smem_total(c.HG, c.stages);
-    cudaError_t e = set_attributes<PAGED>(smem);
+    constexpr int RB = row_bytes<FP8>();
+    const DecodeConfig c = pick_config(N, H, window, FP8);
+    const size_t smem = smem_total(c.HG, c.stages, RB);
+    cudaError_t e = set_attributes<PAGED, FP8>(smem);
     if (e != cudaSuccess) return e;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3((unsigned)((int64_t)N * c.SP), (unsigned)(H / c.HG), 1);
@@ -504,9 +565,10 @@ cudaError_t launch(const void* q, const void* k_new, const void* v_new, CacheRef
     attr[0].val.clusterDim.z = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    const float scale_log2 = scale * 1.4426950408889634f;
+    // the K scale multiplies every score: folded into the base-2 score scale
+    const float scale_log2 = scale * 1.4426950408889634f * (FP8 ? cache.k_scale : 1.f);
     note_launches(1);
-    return cudaLaunchKernelEx(&cfg, swska_decode_warp_kernel<PAGED>,
+    return cudaLaunchKernelEx(&cfg, swska_decode_warp_kernel<PAGED, FP8>,
                               static_cast<const __nv_bfloat16*>(q), static_cast<const __nv_bfloat16*>(k_new),
                               static_cast<const __nv_bfloat16*>(v_new), cache, pos,
                               static_cast<__nv_bfloat16*>(o), H, c.HG, window, c.stages, scale_log2);
@@ -517,17 +579,26 @@ cudaError_t launch(const void* q, const void* k_new, const void* v_new, CacheRef
 cudaError_t swska_decode_warp_launch(const void* q, const void* k_new, const void* v_new,
                                      void* k_cache, void* v_cache, const int64_t* pos, void* o,
                                      int N, int H, int window, float scale, cudaStream_t stream) {
-    const CacheRef c{static_cast<__nv_bfloat16*>(k_cache), static_cast<__nv_bfloat16*>(v_cache), nullptr, 0, 0};
-    return launch<false>(q, k_new, v_new, c, pos, o, N, H, window, scale, stream);
+    const CacheRef c{static_cast<unsigned char*>(k_cache), static_cast<unsigned char*>(v_cache), nullptr, 0, 0,
+                     1.f, 1.f};
+    return launch<false, false>(q, k_new, v_new, c, pos, o, N, H, window, scale, stream);
 }
 
 cudaError_t swska_decode_paged_launch(const void* q, const void* k_new, const void* v_new, void* k_pool,
                                       void* v_pool, const int32_t* block_table, int page_size,
                                       int pages_per_seq, const int64_t* pos, void* o, int N, int H,
                                       int window, float scale, cudaStream_t stream) {
-    const CacheRef c{static_cast<__nv_bfloat16*>(k_pool), static_cast<__nv_bfloat16*>(v_pool), block_table,
-                     page_size, pages_per_seq};
-    return launch<true>(q, k_new, v_new, c, pos, o, N, H, window, scale, stream);
+    const CacheRef c{static_cast<unsigned char*>(k_pool), static_cast<unsigned char*>(v_pool), block_table,
+                     page_size, pages_per_seq, 1.f, 1.f};
+    return launch<true, false>(q, k_new, v_new, c, pos, o, N, H, window, scale, stream);
+}
+
+cudaError_t swska_decode_fp8_launch(const void* q, const void* k_new, const void* v_new, void* k_cache,
+                                    void* v_cache, const int64_t* pos, void* o, int N, int H, int window,
+                                    float scale, float k_scale, float v_scale, cudaStream_t stream) {
+    const CacheRef c{static_cast<unsigned char*>(k_cache), static_cast<unsigned char*>(v_cache), nullptr, 0, 0,
+                     k_scale, v_scale};
+    return launch<false, true>(q, k_new, v_new, c, pos, o, N, H, window, scale, stream);
 }
 
 unsigned swska_decode_warp_take_timeout_flag() {

@@ -154,6 +154,16 @@ def decode_inputs(N, H, dk, dv, W, *, seed=0, dtype="bf16", device="cpu", full=T
                 pos=decode_positions(N, W, full=full, device=device))
 
 
+def fp8_codes(shape, *, seed=0, device="cpu"):
+    """Random E4M3 cache contents as codes (uint8): sign uniform, exponent field uniform in
+    4 .. 9 (magnitudes 2^-3 .. 7.5), mantissa field uniform. Bit assembly only."""
+    gen = _gen(seed, device)
+    sign = torch.randint(0, 2, shape, generator=gen, device=device, dtype=torch.uint8)
+    expo = torch.randint(4, 10, shape, generator=gen, device=device, dtype=torch.uint8)
+    mant = torch.randint(0, 8, shape, generator=gen, device=device, dtype=torch.uint8)
+    return (sign << 7) | (expo << 3) | mant
+
+
 # ------------------------------------------------------------------------------------------
 # long-context stack: layer l even = recurrence, odd = SW-SKA; per-layer seed = l
 # ------------------------------------------------------------------------------------------

@@ -147,6 +147,30 @@ def test_swska_cache_fill_validation(lib):
     assert f(None, None, None, None, 1, 2, 0, 16, 32, 4, 2, None) == OK   # T = 0
 
 
+def test_swska_fp8_validation(lib):
+    """FP8 cache entry points: argument checks before any launch (no GPU needed)."""
+    d = lib.rod_swska_decode_fp8
+    args = lambda N=2, H=4, dk=128, dv=128, W=64, s=0.0, ks=1.0, vs=1.0, q=P, kc=P: (
+        q, P, P, kc, P, P, P, N, H, dk, dv, W, s, ks, vs, None)
+    assert d(*args(W=0)) == SHAPE
+    assert d(*args(dk=64, dv=64)) == SHAPE             # only 128-wide heads
+    assert d(*args(H=17)) == SHAPE
+    assert d(*args(ks=0.0)) == SHAPE                   # scales positive and finite
+    assert d(*args(vs=-1.0)) == SHAPE
+    assert d(*args(ks=float("inf"))) == SHAPE
+    assert d(*args(vs=float("nan"))) == SHAPE
+    assert d(*args(q=None)) == NULL
+    assert d(*args(kc=MIS)) == ALIGN
+    assert d(*args(N=0, q=None, kc=None)) == OK
+    f = lib.rod_swska_cache_fill_fp8
+    assert f(P, P, P, P, 1, 2, 8, 128, 128, 0, 1.0, 1.0, None) == SHAPE   # window < 1
+    assert f(P, P, P, P, 1, 2, 8, 64, 64, 4, 1.0, 1.0, None) == SHAPE     # only 128-wide heads
+    assert f(P, P, P, P, 1, 2, 8, 128, 128, 4, 0.0, 1.0, None) == SHAPE
+    assert f(P, None, P, P, 1, 2, 8, 128, 128, 4, 1.0, 1.0, None) == NULL
+    assert f(P, P, MIS, P, 1, 2, 8, 128, 128, 4, 1.0, 1.0, None) == ALIGN
+    assert f(None, None, None, None, 1, 2, 0, 128, 128, 4, 1.0, 1.0, None) == OK   # T = 0
+
+
 def test_binding_refuses_cpu_tensors():
     import torch
     q = torch.zeros(1, 2, 8, 16)

@@ -54,12 +54,12 @@ MUTATIONS = {
                                     "for (int64_t h = 0; h < 1; ++h) acc += dkp[(b * H + h) * T * dk + i];"),
     "paged_write_wrong_row": ("t = table[n * pps + s / page], r = s % page;\n            memcpy(k_pool",
                               "t = table[n * pps + s / page], r = (s + 1) % page;\n            memcpy(k_pool"),
-    "e4m3_ties_to_odd": ("(d == best_d && (c & 1) == 0 && (best & 1) == 1)",
-                         "(d == best_d && (c & 1) == 1 && (best & 1) == 0)"),
+    "e4m3_ties_to_odd": ("best = dl < dh ? lo : (dh < dl ? hi : ((lo & 1) == 0 ? lo : hi));",
+                         "best = dl < dh ? lo : (dh < dl ? hi : ((lo & 1) == 1 ? lo : hi));"),
     "e4m3_subnormal_exponent": ("v = ldexp((double)m / 8.0, -6);", "v = ldexp((double)m / 8.0, -7);"),
-    "e4m3_no_saturation": ("if (a > 448.0) best = 0x7E;", "if (a > 464.0) best = 0x7F;"),
-    "fp8_decode_v_unscaled": ("on[c] += s[i] * rodref_e4m3_decode(a->vc[((n * H + h) * W + sl) * dv + c]) * a->v_scale;",
-                              "on[c] += s[i] * rodref_e4m3_decode(a->vc[((n * H + h) * W + sl) * dv + c]);"),
+    "e4m3_no_saturation": ("    if (a >= 448.0) {\n        best = 0x7E;", "    if (a >= 464.0) {\n        best = 0x7F;"),
+    "fp8_decode_v_unscaled": ("on[c] += s[i] * e4m3_table[a->vc[((n * H + h) * W + sl) * dv + c]] * a->v_scale;",
+                              "on[c] += s[i] * e4m3_table[a->vc[((n * H + h) * W + sl) * dv + c]];"),
     "fp8_fill_scale_multiplies": ("k_cache[(b * W + ring_slot) * dk + c] = rodref_e4m3_encode(k[(b * T + p) * dk + c] / k_scale);",
                                   "k_cache[(b * W + ring_slot) * dk + c] = rodref_e4m3_encode(k[(b * T + p) * dk + c] * k_scale);"),
 }
