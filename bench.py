@@ -365,6 +365,24 @@ def run_gpu(args):
     rod.check()
     paged_ms = ranks_max(pe0.elapsed_time(pe1) / dsteps)
     del v_pool, k_pool, table
+
+    # the same SW-SKA decode over FP8 (E4M3) rings (SALA blog §4.3): one byte per cached element
+    kc8 = wl.fp8_codes((N, Wd, dk), seed=seed_base + 81, device=dev)
+    vc8 = wl.fp8_codes((N, H, Wd, dv), seed=seed_base + 82, device=dev)
+    for _ in range(3):
+        rod.swska_decode_fp8(dd["sq"], dd["k_new"], dd["v_new"], kc8, vc8, dd["pos"], Wd, o=o2)
+    rod.check()
+    fe0, fe1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier()
+    fe0.record(stream)
+    for _ in range(dsteps):
+        rod.swska_decode_fp8(dd["sq"], dd["k_new"], dd["v_new"], kc8, vc8, dd["pos"], Wd, o=o2)
+    fe1.record(stream)
+    barrier()
+    rod.check()
+    fp8_ms = ranks_max(fe0.elapsed_time(fe1) / dsteps)
+    ska_fp8_bytes = 1.0 * N * Wd * dk + N * H * Wd * dv + N * H * (dk + dv + dv) * 2 + N * dk * 2
+    del kc8, vc8
     decode = {
         "workload": "decode_n256 (N=256 sequences x 1 token, H=16, 128x128 fp32 state, "
                     "SW-SKA ring window 4096)",
@@ -393,6 +411,14 @@ def run_gpu(args):
                                        "frac": round(ska_dec_bytes / (paged_ms / 1e3) / 1e9 / hbm, 4),
                                        "note": "not in the step: the same decode over 64-slot pages "
                                                "through a shuffled block table"},
+            "rod_swska_decode_fp8": {"bound": "hbm", "avg_launch_ms": round(fp8_ms, 4),
+                                     "algorithmic_bytes": ska_fp8_bytes,
+                                     "achieved": round(ska_fp8_bytes / (fp8_ms / 1e3) / 1e9, 1),
+                                     "peak": hbm, "unit": "GB/s",
+                                     "frac": round(ska_fp8_bytes / (fp8_ms / 1e3) / 1e9 / hbm, 4),
+                                     "speedup_vs_bf16_cache": round(ska_dec_ms / fp8_ms, 3),
+                                     "note": "not in the step: the same decode over E4M3 rings (one "
+                                             "byte per cached element, fp32 scales)"},
         },
     }
 
@@ -691,6 +717,10 @@ def run_profile_case(args):
         if case == "ska_decode":
             fn = lambda: rod.swska_decode(dd["sq"], dd["k_new"], dd["v_new"], dd["k_cache"],
                                           dd["v_cache"], dd["pos"], Wd, o=o)
+        elif case == "ska_decode_fp8":  # E4M3 rings
+            kc8 = wl.fp8_codes((N, Wd, dk), seed=81, device=dev)
+            vc8 = wl.fp8_codes((N, H, Wd, dv), seed=82, device=dev)
+            fn = lambda: rod.swska_decode_fp8(dd["sq"], dd["k_new"], dd["v_new"], kc8, vc8, dd["pos"], Wd, o=o)
         elif case == "ska_decode_paged":  # pages of 64 slots, shuffled table
             page, pps = 64, Wd // 64
             k_pool = dd["k_cache"].reshape(N * pps, page, dk)
@@ -729,7 +759,8 @@ def main():
     ap.add_argument("--no-generate", action="store_true")
     ap.add_argument("--no-backward", action="store_true")
     ap.add_argument("--profile-case", choices=["ska_prefill", "gla_prefill", "ska_decode", "gla_decode",
-                                               "ska_decode_paged", "gla_backward", "ska_backward"],
+                                               "ska_decode_paged", "ska_decode_fp8", "gla_backward",
+                                               "ska_backward"],
                     help="run one kernel family alone (for ncu captures) and exit")
     ap.add_argument("--profile-n", type=int, default=128, help="sequences for the decode cases")
     args = ap.parse_args()
