@@ -14,13 +14,15 @@
 //   warps 0-3   softmax warpgroup of head 0 (thread i owns query row i = TMEM lane i)
 //   warps 4-7   softmax warpgroup of head 1
 //   warp  8     TMA producer: Q once, then K_j, V0_j, V1_j into a ring of 32 KB slots
-//   warp  9     TMEM allocator and the single MMA-issuing thread
+//   warp  9     TMEM allocator and MMA issuer
 //   warps 10-11 idle (they complete the third warpgroup, which gives its registers away)
 // TMEM (512 columns): S0 | O0 | S1 | O1, 128 columns each. S_h = Q_h K_j^T is read by the
 // softmax warps, which write P_h (bf16, packed two per column) over the first 64 columns of
 // S_h; O_h += P_h V_h,j then reads P_h straight from TMEM (A operand in TMEM). The issue order
 //   S0(0) S1(0) | PV0(j) S0(j+1) PV1(j) S1(j+1) | ...
-// lets each head's softmax run while the tensor core works on the other head. Softmax is in
+// lets each head's softmax run while the tensor core works on the other head, and each P_h is
+// handed over in two halves of 64 keys, so the first half's P V runs while the softmax forms
+// the second. The issuing warp runs in lockstep with one elected lane issuing. Softmax is in
 // base 2 on scores pre-scaled by scale*log2(e), with lazy rescaling: the running maximum used
 // for the exponent only moves when a row's maximum grows by more than 8 (so P <= 256), and
 // then the O row is rescaled in TMEM by its owning thread. The row maximum runs as eight
@@ -58,7 +60,7 @@ constexpr float kRescaleThreshold = 8.0f;  // log2 units
 constexpr int OFF_Q = 0;
 constexpr int OFF_RING = 2 * TILE_BYTES;
 constexpr int OFF_BAR = OFF_RING + NSLOT * TILE_BYTES;
-constexpr int NBAR = 2 * NSLOT + 8;        // full, empty, qfull, sfull[2], pfull[2], odone[2], drain
+constexpr int NBAR = 2 * NSLOT + 10;       // full, empty, qfull, sfull[2], pfull[2], phalf[2], odone[2], drain
 constexpr int OFF_MISC = OFF_BAR + 8 * NBAR;
 constexpr int SMEM_BYTES = OFF_MISC + 16 + 1024;  // + slack for 1024-byte alignment
 
@@ -67,6 +69,21 @@ __device__ __forceinline__ bool wait_bar(uint64_t* bar, uint32_t parity, volatil
         if (mbar_try_wait(bar, parity)) return true;
         if ((i & 255u) == 0) {
             if (*abort_flag) return false;
+            if (i >= kWaitLimit) {
+                *abort_flag = 1;
+                atomicExch(&g_swska_tc_timeout, 1u);
+                return false;
+            }
+        }
+    }
+}
+
+// warp-wide form: every lane of the warp probes together and all leave with the same result
+__device__ __forceinline__ bool wait_bar_warp(uint64_t* bar, uint32_t parity, volatile int* abort_flag) {
+    for (uint32_t i = 1;; ++i) {
+        if (__all_sync(0xffffffffu, mbar_try_wait(bar, parity))) return true;
+        if ((i & 255u) == 0) {
+            if (__any_sync(0xffffffffu, *abort_flag != 0)) return false;
             if (i >= kWaitLimit) {
                 *abort_flag = 1;
                 atomicExch(&g_swska_tc_timeout, 1u);
@@ -122,8 +139,9 @@ swska_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     uint64_t* empty = bars + NSLOT;
     uint64_t* qfull = bars + 2 * NSLOT;
     uint64_t* sfull = qfull + 1;
-    uint64_t* pfull = sfull + 2;
-    uint64_t* odone = pfull + 2;
+    uint64_t* pfull = sfull + 2;  // all of P_h stored (and O_h rescaled)
+    uint64_t* phalf = pfull + 2;  // the first 64 keys' P_h stored (and O_h rescaled)
+    uint64_t* odone = phalf + 2;
     uint64_t* drain = odone + 2;
     uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + OFF_MISC);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + OFF_MISC + 4);
@@ -137,6 +155,7 @@ swska_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         for (int h = 0; h < 2; ++h) {
             mbar_init(&sfull[h], 1);
             mbar_init(&pfull[h], 128);
+            mbar_init(&phalf[h], 128);
             mbar_init(&odone[h], 1);
         }
         mbar_init(drain, 1);
@@ -189,84 +208,96 @@ swska_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         }
     } else if (warp == 9) {
         // ------------------------------- MMA issuer -------------------------------
-        if (lane == 0) {
-            const uint32_t idesc_s = tc::idesc_bf16_f32(BM, BN, 0, 0);  // Q K^T, both K-major
-            const uint32_t idesc_o = tc::idesc_bf16_f32(BM, HD, 0, 1);  // P V, V is MN-major
-            const uint32_t q_base = smem_u32(smem + OFF_Q);
-            // TMEM columns: S_h at 256 h, O_h at 256 h + 128; Q_h at q_base + h * TILE_BYTES
-            auto ring = [&](int L) { return smem_u32(smem + OFF_RING + (L % NSLOT) * TILE_BYTES); };
-            auto acquire = [&](int L) {
-                const bool ok = wait_bar(&full[L % NSLOT], (uint32_t)((L / NSLOT) & 1), abort_flag);
-                tc::fence_after_sync();
-                return ok;
-            };
-            // descriptors built once; a K step adds its offset (bytes >> 4) to the low word
-            const uint64_t dq0 = tc::sdesc_sw128(q_base, 16, 1024);
-            const uint64_t dq1 = tc::sdesc_sw128(q_base + TILE_BYTES, 16, 1024);
-            const uint32_t dk_hi = tc::desc_hi(tc::sdesc_sw128(q_base, 16, 1024));  // LBO 16, SBO 1024
-            const uint32_t dv_hi = tc::desc_hi(tc::sdesc_sw128(q_base, HALF_BYTES, 1024));
-            auto issue_s = [&](int h, int L) {
-                const uint32_t a_lo = tc::desc_lo(h ? dq1 : dq0), a_hi = tc::desc_hi(h ? dq1 : dq0);
-                const uint32_t b_lo = tc::desc_lo(tc::sdesc_sw128(ring(L), 16, 1024));
-#pragma unroll
-                for (int k = 0; k < HD / 16; ++k) {
-                    const uint32_t koff = (uint32_t)(((k / 4) * HALF_BYTES + (k % 4) * 32) >> 4);
-                    tc::mma_ss_lh(tmem + 256u * h, a_lo + koff, a_hi, b_lo + koff, dk_hi, idesc_s, k > 0);
-                }
-            };
-            auto issue_pv = [&](int h, int L, bool acc) {
-                const uint32_t b_lo = tc::desc_lo(tc::sdesc_sw128(ring(L), HALF_BYTES, 1024));
-#pragma unroll
-                for (int k = 0; k < BN / 16; ++k)
-                    tc::mma_ts_lh(tmem + 256u * h + 128u, tmem + 256u * h + 8u * k, b_lo + (uint32_t)((2048 * k) >> 4),
-                                  dv_hi, idesc_o, (acc || k > 0) ? 1u : 0u);
-            };
-            bool ok = wait_bar(qfull, 0, abort_flag);
+        // The whole warp runs the issue loop in lockstep and one lane, elected inside each
+        // instruction sequence, issues: the descriptors then stay in uniform registers and no
+        // lane waits for another at a branch.
+        const uint32_t idesc_s = tc::idesc_bf16_f32(BM, BN, 0, 0);  // Q K^T, both K-major
+        const uint32_t idesc_o = tc::idesc_bf16_f32(BM, HD, 0, 1);  // P V, V is MN-major
+        const uint32_t q_base = smem_u32(smem + OFF_Q);
+        // TMEM columns: S_h at 256 h, O_h at 256 h + 128; Q_h at q_base + h * TILE_BYTES
+        auto ring = [&](int L) { return smem_u32(smem + OFF_RING + (L % NSLOT) * TILE_BYTES); };
+        auto acquire = [&](int L) {
+            const bool ok = wait_bar_warp(&full[L % NSLOT], (uint32_t)((L / NSLOT) & 1), abort_flag);
             tc::fence_after_sync();
-            if (ok && acquire(0)) {
-                issue_s(0, 0);
-                tc::mma_commit(&sfull[0]);
-                issue_s(1, 0);
-                tc::mma_commit(&sfull[1]);
-                tc::mma_commit(&empty[0]);
-                for (int j = 0; j < n_it; ++j) {
-                    const bool more = j + 1 < n_it;
-                    // V0_j first (it landed long ago), then the softmax hand-off; the next key
-                    // tile is only tested, so PV0 is never delayed by it, and when it is there
-                    // PV0 and S0 go to the tensor core back to back (an empty issue queue costs
-                    // the pipe's start latency again)
-                    if (!acquire(3 * j + 1)) break;
-                    if (!wait_bar(&pfull[0], (uint32_t)(j & 1), abort_flag)) break;
-                    const bool k_ready =
-                        more && mbar_test_wait(&full[(3 * j + 3) % NSLOT], (uint32_t)(((3 * j + 3) / NSLOT) & 1));
-                    tc::fence_after_sync();
-                    issue_pv(0, 3 * j + 1, j > 0);
-                    tc::mma_commit(&empty[(3 * j + 1) % NSLOT]);
-                    if (more) {
-                        if (!k_ready && !acquire(3 * j + 3)) break;
-                        issue_s(0, 3 * j + 3);
-                        tc::mma_commit(&sfull[0]);
-                    } else {
-                        tc::mma_commit(&odone[0]);
-                    }
-                    if (!acquire(3 * j + 2)) break;
-                    if (!wait_bar(&pfull[1], (uint32_t)(j & 1), abort_flag)) break;
-                    tc::fence_after_sync();
-                    issue_pv(1, 3 * j + 2, j > 0);
-                    tc::mma_commit(&empty[(3 * j + 2) % NSLOT]);
-                    if (more) {
-                        issue_s(1, 3 * j + 3);
-                        tc::mma_commit(&sfull[1]);
-                        tc::mma_commit(&empty[(3 * j + 3) % NSLOT]);
-                    } else {
-                        tc::mma_commit(&odone[1]);
-                    }
+            return ok;
+        };
+        auto handoff = [&](uint64_t* bar, int j) {
+            const bool ok = wait_bar_warp(bar, (uint32_t)(j & 1), abort_flag);
+            tc::fence_after_sync();
+            return ok;
+        };
+        // descriptors built once; a K step adds its offset (bytes >> 4) to the low word
+        const uint64_t dq0 = tc::sdesc_sw128(q_base, 16, 1024);
+        const uint64_t dq1 = tc::sdesc_sw128(q_base + TILE_BYTES, 16, 1024);
+        const uint32_t dk_hi = tc::desc_hi(tc::sdesc_sw128(q_base, 16, 1024));  // LBO 16, SBO 1024
+        const uint32_t dv_hi = tc::desc_hi(tc::sdesc_sw128(q_base, HALF_BYTES, 1024));
+        auto issue_s = [&](int h, int L) {
+            const uint32_t a_lo = tc::desc_lo(h ? dq1 : dq0), a_hi = tc::desc_hi(h ? dq1 : dq0);
+            const uint32_t b_lo = tc::desc_lo(tc::sdesc_sw128(ring(L), 16, 1024));
+#pragma unroll
+            for (int k = 0; k < HD / 16; ++k) {
+                const uint32_t koff = (uint32_t)(((k / 4) * HALF_BYTES + (k % 4) * 32) >> 4);
+                tc::mma_ss_lh_warp(tmem + 256u * h, a_lo + koff, a_hi, b_lo + koff, dk_hi, idesc_s, k > 0);
+            }
+        };
+        // O_h += P_h V over the keys 64 * half .. 64 * half + 63 (P_h packed in TMEM columns
+        // 32 * half .. 32 * half + 31 of S_h)
+        auto issue_pv = [&](int h, int L, bool acc, int half) {
+            const uint32_t b_lo = tc::desc_lo(tc::sdesc_sw128(ring(L), HALF_BYTES, 1024));
+#pragma unroll
+            for (int k = 4 * half; k < 4 * half + 4; ++k)
+                tc::mma_ts_lh_warp(tmem + 256u * h + 128u, tmem + 256u * h + 8u * k,
+                                   b_lo + (uint32_t)((2048 * k) >> 4), dv_hi, idesc_o, (acc || k > 0) ? 1u : 0u);
+        };
+        bool ok = wait_bar_warp(qfull, 0, abort_flag);
+        tc::fence_after_sync();
+        if (ok && acquire(0)) {
+            issue_s(0, 0);
+            tc::mma_commit_warp(&sfull[0]);
+            issue_s(1, 0);
+            tc::mma_commit_warp(&sfull[1]);
+            tc::mma_commit_warp(&empty[0]);
+            for (int j = 0; j < n_it; ++j) {
+                const bool more = j + 1 < n_it;
+                // V0_j first (it landed long ago), then the softmax hand-off in two halves: the
+                // first 64 keys' P V runs while the softmax still forms the rest of P. The next
+                // key tile is only tested, so PV0 is never delayed by it, and when it is there
+                // PV0 and S0 go to the tensor core back to back.
+                if (!acquire(3 * j + 1)) break;
+                if (!handoff(&phalf[0], j)) break;
+                issue_pv(0, 3 * j + 1, j > 0, 0);
+                if (!handoff(&pfull[0], j)) break;
+                const bool k_ready =
+                    more && __all_sync(0xffffffffu, mbar_test_wait(&full[(3 * j + 3) % NSLOT],
+                                                                   (uint32_t)(((3 * j + 3) / NSLOT) & 1)));
+                tc::fence_after_sync();
+                issue_pv(0, 3 * j + 1, j > 0, 1);
+                tc::mma_commit_warp(&empty[(3 * j + 1) % NSLOT]);
+                if (more) {
+                    if (!k_ready && !acquire(3 * j + 3)) break;
+                    issue_s(0, 3 * j + 3);
+                    tc::mma_commit_warp(&sfull[0]);
+                } else {
+                    tc::mma_commit_warp(&odone[0]);
+                }
+                if (!acquire(3 * j + 2)) break;
+                if (!handoff(&phalf[1], j)) break;
+                issue_pv(1, 3 * j + 2, j > 0, 0);
+                if (!handoff(&pfull[1], j)) break;
+                issue_pv(1, 3 * j + 2, j > 0, 1);
+                tc::mma_commit_warp(&empty[(3 * j + 2) % NSLOT]);
+                if (more) {
+                    issue_s(1, 3 * j + 3);
+                    tc::mma_commit_warp(&sfull[1]);
+                    tc::mma_commit_warp(&empty[(3 * j + 3) % NSLOT]);
+                } else {
+                    tc::mma_commit_warp(&odone[1]);
                 }
             }
-            // every MMA this thread issued has completed before TMEM is released
-            tc::mma_commit(drain);
-            mbar_wait_bounded(drain, 0, kWaitLimit);
         }
+        // every MMA this warp issued has completed before TMEM is released
+        tc::mma_commit_warp(drain);
+        mbar_wait_bounded(drain, 0, kWaitLimit);
     } else if (warp < 8) {
         // ------------------------------- softmax warpgroups -------------------------------
         asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kSoftmaxRegs));
@@ -312,6 +343,20 @@ swska_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             l_run *= alpha;
             if (need) m_run = m_tile;
             const float m_use = m_run == -INFINITY ? 0.f : m_run;
+            // a row whose maximum moved rescales its O row first (PV of the previous tile is done:
+            // this tile's S was committed after it), so that the first half of P can be handed
+            // over as soon as it is stored
+            if (j > 0 && __any_sync(0xffffffffu, need)) {
+#pragma unroll
+                for (int cb = 0; cb < HD; cb += 32) {
+                    uint32_t r[32];
+                    tc::tmem_ld32(tO + cb, r);
+                    tc::tmem_wait_ld();
+#pragma unroll
+                    for (int i = 0; i < 32; ++i) r[i] = __float_as_uint(__uint_as_float(r[i]) * alpha);
+                    tc::tmem_st32(tO + cb, r);
+                }
+            }
             // P = 2^(s * scale * log2 e - m) as bf16 pairs over the first 64 columns of S; the
             // exponent arguments and the row sum use packed two-wide fp32 arithmetic, the sum in
             // four independent accumulators
@@ -329,27 +374,14 @@ swska_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                     pk[i] = pack_bf16x2(p.x, p.y);
                 }
                 tc::tmem_st32(tS + 32u * half, pk);
+                tc::tmem_wait_st();
+                tc::fence_before_sync();
+                mbar_arrive(half == 0 ? &phalf[h] : &pfull[h]);
             }
             {
                 const float2 a = fadd2(l4[0], l4[1]), b2 = fadd2(l4[2], l4[3]), t2 = fadd2(a, b2);
                 l_run += t2.x + t2.y;
             }
-            // a row whose maximum moved rescales its O row (PV of the previous tile is done:
-            // this tile's S was committed after it)
-            if (j > 0 && __any_sync(0xffffffffu, need)) {
-#pragma unroll
-                for (int cb = 0; cb < HD; cb += 32) {
-                    uint32_t r[32];
-                    tc::tmem_ld32(tO + cb, r);
-                    tc::tmem_wait_ld();
-#pragma unroll
-                    for (int i = 0; i < 32; ++i) r[i] = __float_as_uint(__uint_as_float(r[i]) * alpha);
-                    tc::tmem_st32(tO + cb, r);
-                }
-            }
-            tc::tmem_wait_st();
-            tc::fence_before_sync();
-            mbar_arrive(&pfull[h]);
         }
         // epilogue: O / l -> bf16 rows. With statistics requested (the backward's first step), each
         // row also gets its negated base-2 log-sum-exp and D = dO . o from the fp32 O in TMEM
