@@ -269,12 +269,33 @@ def test_swska_decode_bf16_small_windows(W):
 
 
 @pytest.mark.parametrize("N,H,W", [(1, 16, 4096), (2, 16, 4096), (3, 12, 1000), (1, 3, 4096),
-                                   (5, 16, 2048), (12, 16, 4096)])
+                                   (5, 16, 2048), (12, 16, 4096), (16, 16, 4096), (32, 16, 4096)])
 def test_swska_decode_bf16_small_batches(N, H, W):
     """Small batches split the heads over CTAs (K read once per head group) and the window over
     clusters of up to 16 CTAs: full and partially filled windows against the oracle."""
     _ska_decode_check(N, H, 128, 128, W, "bf16", full=True, seed=80 + N + H)
     _ska_decode_check(N, H, 128, 128, W, "bf16", full=False, seed=90 + N + H)
+
+
+@pytest.mark.parametrize("N", [1, 4, 16, 48])
+def test_swska_decode_repeatable(N):
+    """Thirty identical calls give bit-identical outputs. For a fixed launch shape the decode is
+    deterministic, so a stage read before its copies landed (a broken ring hand-off between the
+    consumer warps that share a head) would show as a mismatch; the first call is also checked
+    against the oracle."""
+    H, W = 16, 4096
+    dd = wl.decode_inputs(N, H, 128, 128, W, seed=300 + N, dtype="bf16", full=True)
+    o_ref, _, _ = oracle.swska_decode(dd["sq"], dd["k_new"], dd["v_new"], dd["k_cache"], dd["v_cache"],
+                                      dd["pos"], W)
+    sq, kn, vn, kc, vc, p = _cuda(dd["sq"], dd["k_new"], dd["v_new"], dd["k_cache"], dd["v_cache"],
+                                  dd["pos"])
+    first = rod.swska_decode(sq, kn, vn, kc, vc, p, W)
+    rod.check()
+    compare(first, o_ref, "bf16", f"swska_decode N{N}")
+    for _ in range(30):
+        o = rod.swska_decode(sq, kn, vn, kc, vc, p, W)
+        assert torch.equal(o, first)
+    rod.check()
 
 
 def test_swska_decode_full_workload_sampled():
