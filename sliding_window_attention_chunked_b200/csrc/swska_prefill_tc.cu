@@ -7,13 +7,15 @@
 // and §3.2: block-wise windowed attention, each query block visiting only the key blocks of its
 // window -- here with a per-element causal/window mask on the two edge blocks.)
 //
-// One CTA computes a 128-query tile for a PAIR of heads of one sequence (with an odd head
-// count the last pair computes its single head twice and stores it once). Each shared key tile
+// A work item is a 128-query tile for a PAIR of heads of one sequence (with an odd head count
+// the last pair computes its single head twice and stores it once). The kernel is persistent:
+// one CTA per SM takes items in turn, so the next item's Q load and first score MMAs overlap
+// the current item's last tile and output rows. Each shared key tile
 // is brought into shared memory once by TMA and feeds both heads' score MMAs (the pair's
 // remaining reuse of K across the other heads goes through L2). Warp roles (384 threads):
 //   warps 0-3   softmax warpgroup of head 0 (thread i owns query row i = TMEM lane i)
 //   warps 4-7   softmax warpgroup of head 1
-//   warp  8     TMA producer: Q once, then K_j, V0_j, V1_j into a ring of 32 KB slots
+//   warp  8     TMA producer: per item Q, then K_j, V0_j, V1_j into a ring of 32 KB slots
 //   warp  9     TMEM allocator and MMA issuer
 //   warps 10-11 idle (they complete the third warpgroup, which gives its registers away)
 // TMEM (512 columns): S0 | O0 | S1 | O1, 128 columns each. S_h = Q_h K_j^T is read by the
@@ -60,7 +62,7 @@ constexpr float kRescaleThreshold = 8.0f;  // log2 units
 constexpr int OFF_Q = 0;
 constexpr int OFF_RING = 2 * TILE_BYTES;
 constexpr int OFF_BAR = OFF_RING + NSLOT * TILE_BYTES;
-constexpr int NBAR = 2 * NSLOT + 10;       // full, empty, qfull, sfull[2], pfull[2], phalf[2], odone[2], drain
+constexpr int NBAR = 2 * NSLOT + 11;       // full, empty, qfull, qempty, sfull[2], pfull[2], phalf[2], odone[2], drain
 constexpr int OFF_MISC = OFF_BAR + 8 * NBAR;
 constexpr int SMEM_BYTES = OFF_MISC + 16 + 1024;  // + slack for 1024-byte alignment
 
@@ -114,31 +116,45 @@ __device__ __forceinline__ float2 fadd2(float2 a, float2 b) {
     return d;
 }
 
+// One work item: a 128-query tile of a head pair of one sequence, with the key tiles it visits.
+// Items are numbered with the query tile fastest, full-window tiles first and short ones last.
+struct Item {
+    int t0, kt_lo, n_it, hp, b;
+};
+__device__ __forceinline__ Item item_at(int i, int n_qtiles, int HP, int W) {
+    Item it;
+    const int qt = n_qtiles - 1 - i % n_qtiles;
+    const int rest = i / n_qtiles;
+    it.hp = rest % HP;
+    it.b = rest / HP;
+    it.t0 = qt * BM;
+    it.kt_lo = (it.t0 - W + 1 > 0 ? it.t0 - W + 1 : 0) / BN;
+    it.n_it = it.t0 / BN - it.kt_lo + 1;
+    return it;
+}
+
 // STATS: the backward's statistics mode (row log-sum-exp and D = dO . o, output optional); a
 // separate instantiation so the plain forward carries none of its registers
 template <bool STATS>
 __global__ void __launch_bounds__(NTHREADS, 1)
 swska_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                 const __grid_constant__ CUtensorMap tm_v, __nv_bfloat16* __restrict__ o, int T,
-                int H, int W, float scale_log2, int n_qtiles, const __nv_bfloat16* __restrict__ dO,
+                int H, int W, float scale_log2, int n_qtiles, int n_items, const __nv_bfloat16* __restrict__ dO,
                 float* __restrict__ nlse2, float* __restrict__ dbuf, int Tpad) {
     extern __shared__ unsigned char smem_raw[];
     unsigned char* smem = reinterpret_cast<unsigned char*>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
-    const int qt = n_qtiles - 1 - (int)blockIdx.x;  // full-window tiles first, short ones last
-    const int hp = blockIdx.y;
-    const int b = blockIdx.z;
-    const int t0 = qt * BM;
-    const int kt_lo = (t0 - W + 1 > 0 ? t0 - W + 1 : 0) / BN;
-    const int kt_hi = t0 / BN;
-    const int n_it = kt_hi - kt_lo + 1;
+    const int HP = (H + 1) / 2;
+    // persistent: this CTA takes the items blockIdx.x, blockIdx.x + gridDim.x, ... in turn, and
+    // every role walks the same sequence
 
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + OFF_BAR);
     uint64_t* full = bars;
     uint64_t* empty = bars + NSLOT;
     uint64_t* qfull = bars + 2 * NSLOT;
-    uint64_t* sfull = qfull + 1;
+    uint64_t* qempty = qfull + 1;  // the item's last S has read Q: the next item's Q may land
+    uint64_t* sfull = qempty + 1;
     uint64_t* pfull = sfull + 2;  // all of P_h stored (and O_h rescaled)
     uint64_t* phalf = pfull + 2;  // the first 64 keys' P_h stored (and O_h rescaled)
     uint64_t* odone = phalf + 2;
@@ -152,6 +168,7 @@ swska_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             mbar_init(&empty[s], 1);
         }
         mbar_init(qfull, 1);
+        mbar_init(qempty, 1);
         for (int h = 0; h < 2; ++h) {
             mbar_init(&sfull[h], 1);
             mbar_init(&pfull[h], 128);
@@ -180,29 +197,40 @@ swska_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             tc::tma_prefetch_desc(&tm_q);
             tc::tma_prefetch_desc(&tm_k);
             tc::tma_prefetch_desc(&tm_v);
-            mbar_arrive_expect_tx(qfull, 2 * TILE_BYTES);
-            for (int h = 0; h < 2; ++h)
-                for (int half = 0; half < 2; ++half)
-                    tc::tma_load_3d(smem + OFF_Q + h * TILE_BYTES + half * HALF_BYTES, &tm_q,
-                                    half * 64, t0, b * H + min(2 * hp + h, H - 1), qfull);
-            int L = 0;
-            for (; L < 3 * n_it; ++L) {
-                const int slot = L % NSLOT, use = L / NSLOT;
-                if (use > 0 && !wait_bar(&empty[slot], (uint32_t)((use - 1) & 1), abort_flag)) break;
-                const int j = L / 3, which = L % 3, key0 = (kt_lo + j) * BN;
-                unsigned char* dst = smem + OFF_RING + slot * TILE_BYTES;
-                mbar_arrive_expect_tx(&full[slot], TILE_BYTES);
-                for (int half = 0; half < 2; ++half) {
-                    if (which == 0)
-                        tc::tma_load_3d(dst + half * HALF_BYTES, &tm_k, half * 64, key0, b, &full[slot]);
-                    else
-                        tc::tma_load_3d(dst + half * HALF_BYTES, &tm_v, half * 64, key0,
-                                        b * H + min(2 * hp + which - 1, H - 1), &full[slot]);
+            int L = 0, nq = 0;  // ring loads and Q loads issued so far
+            bool ok = true;
+            for (int item = blockIdx.x; ok && item < n_items; item += gridDim.x) {
+                const Item it = item_at(item, n_qtiles, HP, W);
+                // the previous item's last S has read its Q
+                if (nq > 0 && !wait_bar(qempty, (uint32_t)((nq - 1) & 1), abort_flag)) break;
+                mbar_arrive_expect_tx(qfull, 2 * TILE_BYTES);
+                for (int h = 0; h < 2; ++h)
+                    for (int half = 0; half < 2; ++half)
+                        tc::tma_load_3d(smem + OFF_Q + h * TILE_BYTES + half * HALF_BYTES, &tm_q,
+                                        half * 64, it.t0, it.b * H + min(2 * it.hp + h, H - 1), qfull);
+                ++nq;
+                // K_j, V0_j, V1_j for the key tiles j of the item, through the ring
+                for (int l = 0; l < 3 * it.n_it; ++l, ++L) {
+                    const int slot = L % NSLOT, use = L / NSLOT;
+                    if (use > 0 && !wait_bar(&empty[slot], (uint32_t)((use - 1) & 1), abort_flag)) {
+                        ok = false;
+                        break;
+                    }
+                    const int j = l / 3, which = l % 3, key0 = (it.kt_lo + j) * BN;
+                    unsigned char* dst = smem + OFF_RING + slot * TILE_BYTES;
+                    mbar_arrive_expect_tx(&full[slot], TILE_BYTES);
+                    for (int half = 0; half < 2; ++half) {
+                        if (which == 0)
+                            tc::tma_load_3d(dst + half * HALF_BYTES, &tm_k, half * 64, key0, it.b, &full[slot]);
+                        else
+                            tc::tma_load_3d(dst + half * HALF_BYTES, &tm_v, half * 64, key0,
+                                            it.b * H + min(2 * it.hp + which - 1, H - 1), &full[slot]);
+                    }
                 }
             }
-            // every copy this thread started (loads 0 .. L-1) has landed before the CTA can
-            // leave: the last NSLOT of them are the latest phase of each slot
-            mbar_wait_bounded(qfull, 0, kWaitLimit);
+            // every copy this thread started has landed before the CTA can leave: the last Q
+            // load, and the last NSLOT ring loads (the latest phase of each slot)
+            if (nq > 0) mbar_wait_bounded(qfull, (uint32_t)((nq - 1) & 1), kWaitLimit);
             for (int Li = (L > NSLOT ? L - NSLOT : 0); Li < L; ++Li)
                 mbar_wait_bounded(&full[Li % NSLOT], (uint32_t)((Li / NSLOT) & 1), kWaitLimit);
         }
@@ -249,51 +277,62 @@ swska_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                 tc::mma_ts_lh_warp(tmem + 256u * h + 128u, tmem + 256u * h + 8u * k,
                                    b_lo + (uint32_t)((2048 * k) >> 4), dv_hi, idesc_o, (acc || k > 0) ? 1u : 0u);
         };
-        bool ok = wait_bar_warp(qfull, 0, abort_flag);
-        tc::fence_after_sync();
-        if (ok && acquire(0)) {
-            issue_s(0, 0);
+        // Per item: S0(0) S1(0) | PV0(j) S0(j+1) PV1(j) S1(j+1) | ... The ring position Lb, the
+        // tile count tb (phases of sfull / phalf / pfull) and the item count (phases of qfull /
+        // odone / qempty) run on across items. The next item's first S follows the last P V
+        // at once: it only needs its Q and K, and its first P V waits for the softmax warps,
+        // which finish the previous item's output rows before they hand over that P.
+        int Lb = 0, tb = 0, items = 0;
+        bool ok = true;
+        for (int item = blockIdx.x; ok && item < n_items; item += gridDim.x) {
+            const int n_it = item_at(item, n_qtiles, HP, W).n_it;
+            if (!handoff(qfull, items) || !acquire(Lb)) break;
+            issue_s(0, Lb);
             tc::mma_commit_warp(&sfull[0]);
-            issue_s(1, 0);
+            issue_s(1, Lb);
             tc::mma_commit_warp(&sfull[1]);
-            tc::mma_commit_warp(&empty[0]);
+            tc::mma_commit_warp(&empty[Lb % NSLOT]);
+            if (n_it == 1) tc::mma_commit_warp(qempty);
             for (int j = 0; j < n_it; ++j) {
                 const bool more = j + 1 < n_it;
+                const int Lj = Lb + 3 * j, tj = tb + j;
                 // V0_j first (it landed long ago), then the softmax hand-off in two halves: the
                 // first 64 keys' P V runs while the softmax still forms the rest of P. The next
                 // key tile is only tested, so PV0 is never delayed by it, and when it is there
                 // PV0 and S0 go to the tensor core back to back.
-                if (!acquire(3 * j + 1)) break;
-                if (!handoff(&phalf[0], j)) break;
-                issue_pv(0, 3 * j + 1, j > 0, 0);
-                if (!handoff(&pfull[0], j)) break;
+                if (!acquire(Lj + 1) || !handoff(&phalf[0], tj)) { ok = false; break; }
+                issue_pv(0, Lj + 1, j > 0, 0);
+                if (!handoff(&pfull[0], tj)) { ok = false; break; }
                 const bool k_ready =
-                    more && __all_sync(0xffffffffu, mbar_test_wait(&full[(3 * j + 3) % NSLOT],
-                                                                   (uint32_t)(((3 * j + 3) / NSLOT) & 1)));
+                    more && __all_sync(0xffffffffu, mbar_test_wait(&full[(Lj + 3) % NSLOT],
+                                                                   (uint32_t)(((Lj + 3) / NSLOT) & 1)));
                 tc::fence_after_sync();
-                issue_pv(0, 3 * j + 1, j > 0, 1);
-                tc::mma_commit_warp(&empty[(3 * j + 1) % NSLOT]);
+                issue_pv(0, Lj + 1, j > 0, 1);
+                tc::mma_commit_warp(&empty[(Lj + 1) % NSLOT]);
                 if (more) {
-                    if (!k_ready && !acquire(3 * j + 3)) break;
-                    issue_s(0, 3 * j + 3);
+                    if (!k_ready && !acquire(Lj + 3)) { ok = false; break; }
+                    issue_s(0, Lj + 3);
                     tc::mma_commit_warp(&sfull[0]);
                 } else {
                     tc::mma_commit_warp(&odone[0]);
                 }
-                if (!acquire(3 * j + 2)) break;
-                if (!handoff(&phalf[1], j)) break;
-                issue_pv(1, 3 * j + 2, j > 0, 0);
-                if (!handoff(&pfull[1], j)) break;
-                issue_pv(1, 3 * j + 2, j > 0, 1);
-                tc::mma_commit_warp(&empty[(3 * j + 2) % NSLOT]);
+                if (!acquire(Lj + 2) || !handoff(&phalf[1], tj)) { ok = false; break; }
+                issue_pv(1, Lj + 2, j > 0, 0);
+                if (!handoff(&pfull[1], tj)) { ok = false; break; }
+                issue_pv(1, Lj + 2, j > 0, 1);
+                tc::mma_commit_warp(&empty[(Lj + 2) % NSLOT]);
                 if (more) {
-                    issue_s(1, 3 * j + 3);
+                    issue_s(1, Lj + 3);
                     tc::mma_commit_warp(&sfull[1]);
-                    tc::mma_commit_warp(&empty[(3 * j + 3) % NSLOT]);
+                    tc::mma_commit_warp(&empty[(Lj + 3) % NSLOT]);
+                    if (j + 2 == n_it) tc::mma_commit_warp(qempty);  // the item's last S
                 } else {
                     tc::mma_commit_warp(&odone[1]);
                 }
             }
+            Lb += 3 * n_it;
+            tb += n_it;
+            ++items;
         }
         // every MMA this warp issued has completed before TMEM is released
         tc::mma_commit_warp(drain);
@@ -306,87 +345,94 @@ swska_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         const uint32_t lane_base = (uint32_t)(32 * (warp % 4)) << 16;
         const uint32_t tS = tmem + 256u * h + lane_base;
         const uint32_t tO = tS + 128u;
-        const int t = t0 + row;
-        float m_run = -INFINITY, l_run = 0.f;
+        int tb = 0, items = 0;  // tiles and items done: the phases of sfull and odone
         bool ok = true;
-        for (int j = 0; j < n_it; ++j) {
-            if (!wait_bar(&sfull[h], (uint32_t)(j & 1), abort_flag)) { ok = false; break; }
-            tc::fence_after_sync();
-            uint32_t s[BN];  // raw fp32 bits of the score row
-            tc::tmem_ld32(tS + 0, s);
-            tc::tmem_ld32(tS + 32, s + 32);
-            tc::tmem_ld32(tS + 64, s + 64);
-            tc::tmem_ld32(tS + 96, s + 96);
-            tc::tmem_wait_ld();
-            const int key0 = (kt_lo + j) * BN;
-            const bool full_tile = key0 >= t0 + BM - W && key0 + BN - 1 <= t0;
-            if (!full_tile) {
-                const int lo = t - W + 1 - key0, hi = t - key0;  // valid key columns [lo, hi]
+        for (int item = blockIdx.x; ok && item < n_items; item += gridDim.x) {
+            const Item it = item_at(item, n_qtiles, HP, W);
+            const int t0 = it.t0, kt_lo = it.kt_lo, n_it = it.n_it, hp = it.hp, b = it.b;
+            const int t = t0 + row;
+            float m_run = -INFINITY, l_run = 0.f;
+            for (int j = 0; j < n_it; ++j) {
+                if (!wait_bar(&sfull[h], (uint32_t)((tb + j) & 1), abort_flag)) { ok = false; break; }
+                tc::fence_after_sync();
+                uint32_t s[BN];  // raw fp32 bits of the score row
+                tc::tmem_ld32(tS + 0, s);
+                tc::tmem_ld32(tS + 32, s + 32);
+                tc::tmem_ld32(tS + 64, s + 64);
+                tc::tmem_ld32(tS + 96, s + 96);
+                tc::tmem_wait_ld();
+                const int key0 = (kt_lo + j) * BN;
+                const bool full_tile = key0 >= t0 + BM - W && key0 + BN - 1 <= t0;
+                if (!full_tile) {
+                    const int lo = t - W + 1 - key0, hi = t - key0;  // valid key columns [lo, hi]
 #pragma unroll
-                for (int c = 0; c < BN; ++c)
-                    if (c < lo || c > hi) s[c] = 0xff800000u;  // -inf
-            }
-            // row maximum: 8 independent chains of 3-input maxima over the columns c = 8k + i
-            float m8[8];
+                    for (int c = 0; c < BN; ++c)
+                        if (c < lo || c > hi) s[c] = 0xff800000u;  // -inf
+                }
+                // row maximum: 8 independent chains of 3-input maxima over the columns c = 8k + i
+                float m8[8];
 #pragma unroll
-            for (int i = 0; i < 8; ++i) {
-                float m = __uint_as_float(s[i]);
+                for (int i = 0; i < 8; ++i) {
+                    float m = __uint_as_float(s[i]);
 #pragma unroll
-                for (int k = 1; k < 15; k += 2)
-                    m = fmax3(m, __uint_as_float(s[8 * k + i]), __uint_as_float(s[8 * k + 8 + i]));
-                m8[i] = fmaxf(m, __uint_as_float(s[120 + i]));
-            }
-            const float mx = fmax3(fmax3(m8[0], m8[1], m8[2]), fmax3(m8[3], m8[4], m8[5]), fmaxf(m8[6], m8[7]));
-            const float m_tile = mx * scale_log2;
-            const bool need = m_tile > m_run + kRescaleThreshold;
-            const float alpha = need ? tc::ex2(m_run - m_tile) : 1.f;  // 0 when m_run = -inf
-            l_run *= alpha;
-            if (need) m_run = m_tile;
-            const float m_use = m_run == -INFINITY ? 0.f : m_run;
-            // a row whose maximum moved rescales its O row first (PV of the previous tile is done:
-            // this tile's S was committed after it), so that the first half of P can be handed
-            // over as soon as it is stored
-            if (j > 0 && __any_sync(0xffffffffu, need)) {
+                    for (int k = 1; k < 15; k += 2)
+                        m = fmax3(m, __uint_as_float(s[8 * k + i]), __uint_as_float(s[8 * k + 8 + i]));
+                    m8[i] = fmaxf(m, __uint_as_float(s[120 + i]));
+                }
+                const float mx = fmax3(fmax3(m8[0], m8[1], m8[2]), fmax3(m8[3], m8[4], m8[5]), fmaxf(m8[6], m8[7]));
+                const float m_tile = mx * scale_log2;
+                const bool need = m_tile > m_run + kRescaleThreshold;
+                const float alpha = need ? tc::ex2(m_run - m_tile) : 1.f;  // 0 when m_run = -inf
+                l_run *= alpha;
+                if (need) m_run = m_tile;
+                const float m_use = m_run == -INFINITY ? 0.f : m_run;
+                // a row whose maximum moved rescales its O row first (PV of the previous tile is done:
+                // this tile's S was committed after it), so that the first half of P can be handed
+                // over as soon as it is stored
+                if (j > 0 && __any_sync(0xffffffffu, need)) {
 #pragma unroll
-                for (int cb = 0; cb < HD; cb += 32) {
-                    uint32_t r[32];
-                    tc::tmem_ld32(tO + cb, r);
-                    tc::tmem_wait_ld();
+                    for (int cb = 0; cb < HD; cb += 32) {
+                        uint32_t r[32];
+                        tc::tmem_ld32(tO + cb, r);
+                        tc::tmem_wait_ld();
 #pragma unroll
-                    for (int i = 0; i < 32; ++i) r[i] = __float_as_uint(__uint_as_float(r[i]) * alpha);
-                    tc::tmem_st32(tO + cb, r);
+                        for (int i = 0; i < 32; ++i) r[i] = __float_as_uint(__uint_as_float(r[i]) * alpha);
+                        tc::tmem_st32(tO + cb, r);
+                    }
+                }
+                // P = 2^(s * scale * log2 e - m) as bf16 pairs over the first 64 columns of S; the
+                // exponent arguments and the row sum use packed two-wide fp32 arithmetic, the sum in
+                // four independent accumulators
+                const float2 sc2 = make_float2(scale_log2, scale_log2), nm2 = make_float2(-m_use, -m_use);
+                float2 l4[4] = {{0.f, 0.f}, {0.f, 0.f}, {0.f, 0.f}, {0.f, 0.f}};
+#pragma unroll
+                for (int half = 0; half < 2; ++half) {
+                    uint32_t pk[32];
+#pragma unroll
+                    for (int i = 0; i < 32; ++i) {
+                        const int c = 64 * half + 2 * i;
+                        const float2 x = ffma2(make_float2(__uint_as_float(s[c]), __uint_as_float(s[c + 1])), sc2, nm2);
+                        const float2 p = make_float2(tc::ex2(x.x), tc::ex2(x.y));
+                        l4[i & 3] = fadd2(l4[i & 3], p);
+                        pk[i] = pack_bf16x2(p.x, p.y);
+                    }
+                    tc::tmem_st32(tS + 32u * half, pk);
+                    tc::tmem_wait_st();
+                    tc::fence_before_sync();
+                    mbar_arrive(half == 0 ? &phalf[h] : &pfull[h]);
+                }
+                {
+                    const float2 a = fadd2(l4[0], l4[1]), b2 = fadd2(l4[2], l4[3]), t2 = fadd2(a, b2);
+                    l_run += t2.x + t2.y;
                 }
             }
-            // P = 2^(s * scale * log2 e - m) as bf16 pairs over the first 64 columns of S; the
-            // exponent arguments and the row sum use packed two-wide fp32 arithmetic, the sum in
-            // four independent accumulators
-            const float2 sc2 = make_float2(scale_log2, scale_log2), nm2 = make_float2(-m_use, -m_use);
-            float2 l4[4] = {{0.f, 0.f}, {0.f, 0.f}, {0.f, 0.f}, {0.f, 0.f}};
-#pragma unroll
-            for (int half = 0; half < 2; ++half) {
-                uint32_t pk[32];
-#pragma unroll
-                for (int i = 0; i < 32; ++i) {
-                    const int c = 64 * half + 2 * i;
-                    const float2 x = ffma2(make_float2(__uint_as_float(s[c]), __uint_as_float(s[c + 1])), sc2, nm2);
-                    const float2 p = make_float2(tc::ex2(x.x), tc::ex2(x.y));
-                    l4[i & 3] = fadd2(l4[i & 3], p);
-                    pk[i] = pack_bf16x2(p.x, p.y);
-                }
-                tc::tmem_st32(tS + 32u * half, pk);
-                tc::tmem_wait_st();
-                tc::fence_before_sync();
-                mbar_arrive(half == 0 ? &phalf[h] : &pfull[h]);
+            // epilogue: O / l -> bf16 rows. With statistics requested (the backward's first step), each
+            // row also gets its negated base-2 log-sum-exp and D = dO . o from the fp32 O in TMEM
+            // (-inf and 0 for rows past the end of the sequence), and O itself is stored only if asked.
+            if (!ok || !wait_bar(&odone[h], (uint32_t)(items & 1), abort_flag)) {
+                ok = false;
+                break;
             }
-            {
-                const float2 a = fadd2(l4[0], l4[1]), b2 = fadd2(l4[2], l4[3]), t2 = fadd2(a, b2);
-                l_run += t2.x + t2.y;
-            }
-        }
-        // epilogue: O / l -> bf16 rows. With statistics requested (the backward's first step), each
-        // row also gets its negated base-2 log-sum-exp and D = dO . o from the fp32 O in TMEM
-        // (-inf and 0 for rows past the end of the sequence), and O itself is stored only if asked.
-        if (ok && wait_bar(&odone[h], 0, abort_flag)) {
             tc::fence_after_sync();
             const float inv = 1.f / l_run;
             const bool live = t < T && 2 * hp + h < H;  // an odd H's last pair computes one head twice
@@ -423,6 +469,8 @@ swska_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                 nlse2[srow] = live ? -(m_run + log2f(l_run)) : -INFINITY;
                 dbuf[srow] = live ? dacc : 0.f;
             }
+            tb += n_it;
+            ++items;
         }
     }
 
@@ -430,6 +478,19 @@ swska_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     __syncthreads();
     tc::fence_after_sync();
     if (warp == 9) tc::tmem_dealloc(tmem, 512);
+}
+
+// streaming multiprocessors of the current device (queried once per device)
+int sm_count() {
+    static int cache[64] = {0};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 148;
+    if (cache[dev] == 0) {
+        int sms = 0;
+        if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || sms < 1) sms = 148;
+        cache[dev] = sms;
+    }
+    return cache[dev];
 }
 
 }  // namespace
@@ -457,12 +518,15 @@ cudaError_t swska_prefill_tc_stats_launch(const void* q, const void* k, const vo
               : cudaFuncSetAttribute(swska_tc_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
     if (e != cudaSuccess) return e;
     const int n_qtiles = (T + BM - 1) / BM;
-    if (B > 65535 || (H + 1) / 2 > 65535) return cudaErrorInvalidConfiguration;
-    dim3 grid((unsigned)n_qtiles, (unsigned)((H + 1) / 2), (unsigned)B);
+    const int64_t n_items = (int64_t)n_qtiles * ((H + 1) / 2) * B;
+    if (n_items > INT32_MAX) return cudaErrorInvalidConfiguration;
+    // persistent: one CTA per SM (the shared memory allows no second), each taking items in turn
+    const int sms = sm_count();
+    const unsigned grid = (unsigned)(n_items < sms ? n_items : sms);
     auto* kern = stats ? swska_tc_kernel<true> : swska_tc_kernel<false>;
     kern<<<grid, NTHREADS, SMEM_BYTES, stream>>>(
         mq, mk, mv, static_cast<__nv_bfloat16*>(o), T, H, window, scale * 1.4426950408889634f,
-        n_qtiles, static_cast<const __nv_bfloat16*>(dO), nlse2, dbuf, (int)Tpad);
+        n_qtiles, (int)n_items, static_cast<const __nv_bfloat16*>(dO), nlse2, dbuf, (int)Tpad);
     note_launches(1);
     return cudaGetLastError();
 }
