@@ -117,14 +117,27 @@ __device__ __forceinline__ float2 fadd2(float2 a, float2 b) {
 }
 
 // One work item: a 128-query tile of a head pair of one sequence, with the key tiles it visits.
-// Items are numbered with the query tile fastest, full-window tiles first and short ones last.
+// Two numberings, both with full-window tiles first and short ones last:
+//  - qt_slow: all (head pair, sequence) items of a query tile together. With the rounds dealt
+//    out boustrophedon (CTA c takes item c of even rounds and G-1-c of odd ones) the CTAs' loads
+//    come out within a few percent of each other even over a few rounds, and while HP x B is
+//    small every head pair still has several neighbouring query tiles in flight, sharing K and
+//    V tiles in L2;
+//  - otherwise the query tile fastest, dealt out in plain stride: neighbouring query tiles of
+//    a head pair run side by side whatever HP x B is, and over many rounds the loads even out.
 struct Item {
     int t0, kt_lo, n_it, hp, b;
 };
-__device__ __forceinline__ Item item_at(int i, int n_qtiles, int HP, int W) {
+__device__ __forceinline__ Item item_at(int i, int n_qtiles, int HP, int NHB, int W, bool qt_slow) {
     Item it;
-    const int qt = n_qtiles - 1 - i % n_qtiles;
-    const int rest = i / n_qtiles;
+    int qt, rest;
+    if (qt_slow) {
+        qt = n_qtiles - 1 - i / NHB;
+        rest = i % NHB;
+    } else {
+        qt = n_qtiles - 1 - i % n_qtiles;
+        rest = i / n_qtiles;
+    }
     it.hp = rest % HP;
     it.b = rest / HP;
     it.t0 = qt * BM;
@@ -132,22 +145,30 @@ __device__ __forceinline__ Item item_at(int i, int n_qtiles, int HP, int W) {
     it.n_it = it.t0 / BN - it.kt_lo + 1;
     return it;
 }
+// the k-th item of this CTA (round k of gridDim.x items), or -1 past the last
+__device__ __forceinline__ int cta_item(int k, int n_items, bool snake) {
+    const int G = (int)gridDim.x, base = k * G;
+    if (base >= n_items) return -1;
+    const int i = base + ((snake && (k & 1)) ? G - 1 - (int)blockIdx.x : (int)blockIdx.x);
+    return i < n_items ? i : -1;
+}
 
 // STATS: the backward's statistics mode (row log-sum-exp and D = dO . o, output optional); a
 // separate instantiation so the plain forward carries none of its registers
-template <bool STATS>
+template <bool STATS, bool QT_SLOW>
 __global__ void __launch_bounds__(NTHREADS, 1)
 swska_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                 const __grid_constant__ CUtensorMap tm_v, __nv_bfloat16* __restrict__ o, int T,
-                int H, int W, float scale_log2, int n_qtiles, int n_items, const __nv_bfloat16* __restrict__ dO,
+                int H, int W, float scale_log2, int n_qtiles, int n_items,
+                const __nv_bfloat16* __restrict__ dO,
                 float* __restrict__ nlse2, float* __restrict__ dbuf, int Tpad) {
     extern __shared__ unsigned char smem_raw[];
     unsigned char* smem = reinterpret_cast<unsigned char*>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
-    const int HP = (H + 1) / 2;
-    // persistent: this CTA takes the items blockIdx.x, blockIdx.x + gridDim.x, ... in turn, and
-    // every role walks the same sequence
+    const int HP = (H + 1) / 2, NHB = n_items / n_qtiles;  // NHB: head pairs x sequences
+    // persistent: this CTA takes one item per round (cta_item), and every role walks the same
+    // sequence
 
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + OFF_BAR);
     uint64_t* full = bars;
@@ -199,8 +220,10 @@ swska_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             tc::tma_prefetch_desc(&tm_v);
             int L = 0, nq = 0;  // ring loads and Q loads issued so far
             bool ok = true;
-            for (int item = blockIdx.x; ok && item < n_items; item += gridDim.x) {
-                const Item it = item_at(item, n_qtiles, HP, W);
+            for (int k_item = 0; ok; ++k_item) {
+                const int item = cta_item(k_item, n_items, QT_SLOW);
+                if (item < 0) break;
+                const Item it = item_at(item, n_qtiles, HP, NHB, W, QT_SLOW);
                 // the previous item's last S has read its Q
                 if (nq > 0 && !wait_bar(qempty, (uint32_t)((nq - 1) & 1), abort_flag)) break;
                 mbar_arrive_expect_tx(qfull, 2 * TILE_BYTES);
@@ -284,8 +307,10 @@ swska_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         // which finish the previous item's output rows before they hand over that P.
         int Lb = 0, tb = 0, items = 0;
         bool ok = true;
-        for (int item = blockIdx.x; ok && item < n_items; item += gridDim.x) {
-            const int n_it = item_at(item, n_qtiles, HP, W).n_it;
+        for (int k_item = 0; ok; ++k_item) {
+            const int item = cta_item(k_item, n_items, QT_SLOW);
+            if (item < 0) break;
+            const int n_it = item_at(item, n_qtiles, HP, NHB, W, QT_SLOW).n_it;
             if (!handoff(qfull, items) || !acquire(Lb)) break;
             issue_s(0, Lb);
             tc::mma_commit_warp(&sfull[0]);
@@ -347,8 +372,10 @@ swska_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         const uint32_t tO = tS + 128u;
         int tb = 0, items = 0;  // tiles and items done: the phases of sfull and odone
         bool ok = true;
-        for (int item = blockIdx.x; ok && item < n_items; item += gridDim.x) {
-            const Item it = item_at(item, n_qtiles, HP, W);
+        for (int k_item = 0; ok; ++k_item) {
+            const int item = cta_item(k_item, n_items, QT_SLOW);
+            if (item < 0) break;
+            const Item it = item_at(item, n_qtiles, HP, NHB, W, QT_SLOW);
             const int t0 = it.t0, kt_lo = it.kt_lo, n_it = it.n_it, hp = it.hp, b = it.b;
             const int t = t0 + row;
             float m_run = -INFINITY, l_run = 0.f;
@@ -514,16 +541,22 @@ cudaError_t swska_prefill_tc_stats_launch(const void* q, const void* k, const vo
     if ((e = make_tmap_bf16_3d(&mk, k, HD, (uint64_t)T, (uint64_t)B, 64, BN)) != cudaSuccess) return e;
     if ((e = make_tmap_bf16_3d(&mv, v, HD, (uint64_t)T, (uint64_t)B * H, 64, BN)) != cudaSuccess) return e;
     const bool stats = nlse2 != nullptr;
-    e = stats ? cudaFuncSetAttribute(swska_tc_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES)
-              : cudaFuncSetAttribute(swska_tc_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
-    if (e != cudaSuccess) return e;
     const int n_qtiles = (T + BM - 1) / BM;
     const int64_t n_items = (int64_t)n_qtiles * ((H + 1) / 2) * B;
     if (n_items > INT32_MAX) return cudaErrorInvalidConfiguration;
-    // persistent: one CTA per SM (the shared memory allows no second), each taking items in turn
+    // persistent: one CTA per SM (the shared memory allows no second), each taking items in turn.
+    // With few rounds of items a plain stride leaves the CTAs' loads uneven (at T 8192, W 4096,
+    // 8 head pairs: 3.5 rounds, the busiest CTA 1.39x the mean): there the query-tile-slowest
+    // numbering dealt out boustrophedon, while the head pairs x sequences are few enough to keep
+    // neighbouring query tiles of each in flight together. With many rounds the stride is within
+    // a few percent and keeps the tighter L2 reuse (measured: T 131072 3.4% faster with it).
     const int sms = sm_count();
     const unsigned grid = (unsigned)(n_items < sms ? n_items : sms);
-    auto* kern = stats ? swska_tc_kernel<true> : swska_tc_kernel<false>;
+    const bool qt_slow = (int64_t)((H + 1) / 2) * B <= 32 && n_items < 16 * (int64_t)sms;
+    auto* kern = stats ? (qt_slow ? swska_tc_kernel<true, true> : swska_tc_kernel<true, false>)
+                       : (qt_slow ? swska_tc_kernel<false, true> : swska_tc_kernel<false, false>);
+    if ((e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES)) != cudaSuccess)
+        return e;
     kern<<<grid, NTHREADS, SMEM_BYTES, stream>>>(
         mq, mk, mv, static_cast<__nv_bfloat16*>(o), T, H, window, scale * 1.4426950408889634f,
         n_qtiles, (int)n_items, static_cast<const __nv_bfloat16*>(dO), nlse2, dbuf, (int)Tpad);
