@@ -496,7 +496,8 @@ gla_chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
             asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
             tc::fence_before_sync();
             grp_sync(1);
-            if (tid == 0) {
+            if (warp == 0) {
+                // the whole warp issues in lockstep, one lane elected inside each instruction
                 tc::fence_after_sync();
                 if (MODE == PASS_C && fast) {
                     // descriptors built once; a K step adds its offset (bytes >> 4) to the low word
@@ -506,15 +507,15 @@ gla_chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
 #pragma unroll
                     for (int k = 0; k < D / 16; ++k) {
                         const uint32_t koff = (uint32_t)(((k / 4) * BOX_BYTES + (k % 4) * 32) >> 4);
-                        tc::mma_ss_lh(tmem + TM_A + 64u * st, q_lo + koff, hi, k_lo + koff, hi, idesc_A, k > 0);
+                        tc::mma_ss_lh_warp(tmem + TM_A + 64u * st, q_lo + koff, hi, k_lo + koff, hi, idesc_A, k > 0);
                     }
-                    tc::mma_commit(&barA[st]);
+                    tc::mma_commit_warp(&barA[st]);
                 }
-                mbar_arrive(&ops[st]);
+                if (lane == 0) mbar_arrive(&ops[st]);
             }
         }
-        if (tid == 0) {  // every MMA this thread issued has completed before TMEM is released
-            tc::mma_commit(drain0);
+        if (warp == 0) {  // every MMA this warp issued has completed before TMEM is released
+            tc::mma_commit_warp(drain0);
             mbar_wait_bounded(drain0, 0, kWaitLimit);
         }
     } else if (warp < 8) {
@@ -632,7 +633,7 @@ gla_chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
             asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
             tc::fence_before_sync();
             grp_sync(2);
-            if (tid == 128) {
+            if (warp == 4) {  // the whole warp issues in lockstep, one lane elected inside each instruction
                 tc::fence_after_sync();
                 // R += k^'^T V (pass A starts from an empty R: the first MMA overwrites)
                 // descriptors built once (all share the high word: SBO 1024, SW128); a K step adds
@@ -642,22 +643,22 @@ gla_chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                 const uint32_t va_lo = tc::desc_lo(tc::sdesc_sw128(smem_u32(base + ST_V), BOX_BYTES, 1024));
 #pragma unroll
                 for (int k = 0; k < C / 16; ++k)
-                    tc::mma_ss_lh(tmem + TM_S, kh_lo + 128u * k, hi, va_lo + 128u * k, hi, idesc_U,
-                                  (MODE == PASS_A && n == 0 && k == 0) ? 0u : 1u);
+                    tc::mma_ss_lh_warp(tmem + TM_S, kh_lo + 128u * k, hi, va_lo + 128u * k, hi, idesc_U,
+                                       (MODE == PASS_A && n == 0 && k == 0) ? 0u : 1u);
                 if (MODE == PASS_C) {  // O = P V + q~' R_bf16
                     const uint32_t pa_lo = tc::desc_lo(tc::sdesc_sw128(smem_u32(base + ST_P), 16, 1024));
                     const uint32_t qa_lo = tc::desc_lo(tc::sdesc_sw128(smem_u32(base + ST_Q), 16, 1024));
                     const uint32_t sb_lo = tc::desc_lo(tc::sdesc_sw128(smem_u32(smem + OFF_SBF), D * 128, 1024));
 #pragma unroll
                     for (int k = 0; k < C / 16; ++k)
-                        tc::mma_ss_lh(tmem + TM_O, pa_lo + 2u * k, hi, va_lo + 128u * k, hi, idesc_O, k > 0);
+                        tc::mma_ss_lh_warp(tmem + TM_O, pa_lo + 2u * k, hi, va_lo + 128u * k, hi, idesc_O, k > 0);
 #pragma unroll
                     for (int k = 0; k < D / 16; ++k)
-                        tc::mma_ss_lh(tmem + TM_O, qa_lo + (uint32_t)(((k / 4) * BOX_BYTES + (k % 4) * 32) >> 4), hi,
-                                      sb_lo + 128u * k, hi, idesc_O, 1u);
+                        tc::mma_ss_lh_warp(tmem + TM_O, qa_lo + (uint32_t)(((k / 4) * BOX_BYTES + (k % 4) * 32) >> 4),
+                                           hi, sb_lo + 128u * k, hi, idesc_O, 1u);
                 }
-                tc::mma_commit(barO);
-                tc::mma_commit(&empty[st]);
+                tc::mma_commit_warp(barO);
+                tc::mma_commit_warp(&empty[st]);
             }
         }
 
@@ -685,8 +686,8 @@ gla_chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                 }
             }
         }
-        if (tid == 128) {  // every MMA this thread issued has completed before TMEM is released
-            tc::mma_commit(drain1);
+        if (warp == 4) {  // every MMA this warp issued has completed before TMEM is released
+            tc::mma_commit_warp(drain1);
             mbar_wait_bounded(drain1, 0, kWaitLimit);
         }
     }
