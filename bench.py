@@ -402,7 +402,7 @@ def run_gpu(args):
                                  "peak": hbm, "unit": "GB/s",
                                  "frac": round(ska_dec_bytes / (ska_dec_ms / 1e3) / 1e9 / hbm, 4),
                                  "traffic": recorded_traffic("swska_decode_n256",
-                                                             ["swska_decode_warp.cu", "common.cuh"])},
+                                                             ["swska_decode_warp.cu", "common.cuh", "fp8.cuh"])},
             "rod_swska_decode_paged": {"bound": "hbm", "page_slots": page,
                                        "avg_launch_ms": round(paged_ms, 4),
                                        "algorithmic_bytes": ska_dec_bytes,
