@@ -15,6 +15,7 @@ baseline, an end-to-end number through host buffers, clocks and the launch count
 from __future__ import annotations
 
 import argparse
+import datetime
 import hashlib
 import json
 import math
@@ -56,27 +57,46 @@ def swska_pairs(T, W):
 
 
 class ClockSampler:
-    """nvidia-smi sampled every 200 ms while the timed region runs."""
+    """nvidia-smi sampled every 100 ms. Started before the warm-up steps, so that the tool is
+    already sampling when the timed region begins; mark() brackets the timed region, and the
+    summary keeps the samples whose timestamps fall inside it (all samples if the timestamps
+    cannot be read)."""
 
-    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+    FIELDS = ("timestamp,index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
 
-    def __init__(self, gpu_index):
+    def __init__(self, gpu_index, interval_ms=100):
         self.gpu = gpu_index
+        self.interval_ms = interval_ms
         self.proc = None
         self.file = None
+        self.window = None  # (start, end) of the timed region, host epoch seconds
 
     def __enter__(self):
         try:
             self.file = tempfile.NamedTemporaryFile("w+", suffix=".csv", delete=False)
             self.proc = subprocess.Popen(
                 ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}",
-                 "--format=csv,noheader,nounits", "-lms", "200"],
+                 "--format=csv,noheader,nounits", "-lms", str(self.interval_ms)],
                 stdout=self.file, stderr=subprocess.DEVNULL)
         except Exception:
             self.proc = None
         return self
+
+    def wait_started(self, timeout_s=5.0):
+        """Return once the first sample is written (or after timeout_s)."""
+        t0 = time.time()
+        while self.proc is not None and time.time() - t0 < timeout_s:
+            try:
+                if os.path.getsize(self.file.name) > 0:
+                    return
+            except OSError:
+                return
+            time.sleep(0.05)
+
+    def mark(self, start, end):
+        self.window = (start, end)
 
     def __exit__(self, *exc):
         if self.proc is not None:
@@ -87,28 +107,53 @@ class ClockSampler:
                 self.proc.kill()
         return False
 
+    @staticmethod
+    def _epoch(stamp):
+        for fmt in ("%Y/%m/%d %H:%M:%S.%f", "%Y/%m/%d %H:%M:%S"):
+            try:
+                return datetime.datetime.strptime(stamp.strip(), fmt).timestamp()
+            except ValueError:
+                continue
+        return None
+
     def summary(self):
         if self.proc is None or self.file is None:
             return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
         self.file.flush()
         with open(self.file.name) as f:
-            rows = [r.strip().split(", ") for r in f if r.strip()]
+            lines = [line for line in f if line.strip()]
         os.unlink(self.file.name)
-        sm, mx, reasons, power = [], None, set(), []
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        for r in rows:
-            if len(r) < 9:
+        return self.summarise(lines, self.window)
+
+    @classmethod
+    def summarise(cls, lines, window=None):
+        """Median SM clock under load, the maximum clock and the throttle reasons seen, from
+        nvidia-smi rows (the FIELDS above), restricted to the timed window when it can be."""
+        rows = []
+        for line in lines:
+            r = [x.strip() for x in line.strip().split(",")]
+            if len(r) < 10:
                 continue
             try:
-                sm.append(float(r[1]))
-                mx = float(r[2])
-                power.append(float(r[3]))
+                rows.append((cls._epoch(r[0]), float(r[2]), float(r[3]), float(r[4]), r[6:10]))
             except ValueError:
                 continue
-            for n, val in zip(names, r[5:9]):
-                if val.strip().lower() == "active":
+        in_window = rows
+        if window is not None and rows and all(t is not None for t, *_ in rows):
+            lo, hi = window[0] - 0.05, window[1] + 0.15
+            inside = [x for x in rows if lo <= x[0] <= hi]
+            if inside:
+                in_window = inside
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        sm = [x[1] for x in in_window]
+        power = [x[3] for x in in_window]
+        mx = in_window[-1][2] if in_window else None
+        reasons = set()
+        for x in in_window:
+            for n, val in zip(names, x[4]):
+                if val.lower() == "active":
                     reasons.add(n)
-        loaded = [s for s, p in zip(sm, power) if p > 300] or sm
+        loaded = [c for c, p in zip(sm, power) if p > 300] or sm
         return {"sm_mhz": statistics.median(loaded) if loaded else None, "sm_max_mhz": mx,
                 "reasons": sorted(reasons), "samples": len(sm)}
 
@@ -217,7 +262,6 @@ def run_gpu(args):
     rank = int(os.environ.get("RANK", "0"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
     if world > 1:
-        import datetime
         torch.cuda.set_device(local)
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
                                 device_id=torch.device("cuda", local))
@@ -268,20 +312,23 @@ def run_gpu(args):
                     e1.record(stream)
                     ska_events.append((e0, e1))
 
-    for _ in range(args.warmup):
-        step()
-    rod.check()
-    barrier()
-    n0 = rod.launch_count()
     with ClockSampler(dev.index) as clk:
+        clk.wait_started()
+        for _ in range(args.warmup):
+            step()
+        rod.check()
+        barrier()
+        n0 = rod.launch_count()
         ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         barrier()
+        t_start = time.time()
         ev0.record(stream)
         for _ in range(args.steps):
             step(record=True)
         ev1.record(stream)
         barrier()
-    launches = rod.launch_count() - n0
+        clk.mark(t_start, time.time())
+        launches = rod.launch_count() - n0
     rod.check()
     ms_local = ev0.elapsed_time(ev1)
     ms = ranks_max(ms_local)
@@ -781,7 +828,7 @@ def run_profile_case(args):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=5)
+    ap.add_argument("--steps", type=int, default=10)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", default="rod", choices=["rod", "reference"])
     ap.add_argument("--e2e-steps", type=int, default=1)
