@@ -119,3 +119,29 @@ def test_oracle_backward_equals_chunk_form(T, C, final):
                                  dSf[b, h].astype(np.float64) if final else None, C)
             for name, a, r in zip(("dq", "dk", "dv", "dg", "dstate0"), got, ref):
                 np.testing.assert_allclose(a, r[b, h], rtol=1e-9, atol=1e-9, err_msg=name)
+
+
+def test_query_key_term_of_the_gate_gradient_by_recurrence():
+    """The fourth term of dg_t, sum over s < t <= r of P(t+1, r) P(s+1, t-1) q_r k_s (dO_r . v_s),
+    computed as a kernel would: K_{t+1}[r] = g_t K_t[r] + (dO_r . v_t) k_t over the chunk, then
+    sum_{r>=t} P(t+1, r) q_r K_t[r]. It equals the direct double sum, gates of 0 included."""
+    rng = np.random.default_rng(7)
+    C, dk, dv = 12, 4, 3
+    q, k = rng.standard_normal((C, dk)), rng.standard_normal((C, dk))
+    v, dO = rng.standard_normal((C, dv)), rng.standard_normal((C, dv))
+    g = rng.uniform(0.2, 1.0, (C, dk))
+    g[3, 1] = g[7, 2] = 0.0
+    P = range_products(g)
+    A2 = dO @ v.T  # A2[r, s] = dO_r . v_s
+    direct = np.zeros((C, dk))
+    for t in range(C):
+        for r in range(t, C):
+            for s in range(t):
+                direct[t] += P[t + 1, r] * P[s + 1, t - 1] * q[r] * k[s] * A2[r, s]
+    K = np.zeros((C, dk))  # K_t[r], t = 0: empty sum
+    rec = np.zeros((C, dk))
+    for t in range(C):
+        for r in range(t, C):
+            rec[t] += P[t + 1, r] * q[r] * K[r]
+        K = g[t] * K + A2[:, t:t + 1] * k[t]
+    np.testing.assert_allclose(rec, direct, rtol=1e-12, atol=1e-12)
