@@ -145,3 +145,97 @@ def test_query_key_term_of_the_gate_gradient_by_recurrence():
             rec[t] += P[t + 1, r] * q[r] * K[r]
         K = g[t] * K + A2[:, t:t + 1] * k[t]
     np.testing.assert_allclose(rec, direct, rtol=1e-12, atol=1e-12)
+
+
+def chunk_backward_products(q, k, v, g, dO, S0, dSf, C, fast_min=2.0 ** -60):
+    """The chunk backward in the shape a tensor-core kernel computes it, for one (batch, head):
+    per chunk, matrix products with the prefix products G (fast route: q~ = q.G, k~ = k/G,
+    k^ = k.(a/G)) when every channel's chunk decay a is at least fast_min, else range products
+    (exact route); the gate gradient from two decayed scans and the query-key recurrence.
+    Returns dq, dk, dv, dg, dstate0 and the number of chunks that took the exact route."""
+    T, dk = q.shape
+    bounds = [(c0, min(c0 + C, T)) for c0 in range(0, T, C)]
+    S_in, S = [], S0.copy()
+    for c0, c1 in bounds:  # forward: incoming states
+        S_in.append(S)
+        G = np.cumprod(g[c0:c1], axis=0)
+        P = range_products(g[c0:c1])
+        n = c1 - c0
+        S = G[-1][:, None] * S + (k[c0:c1] * P[1:n + 1, n - 1]).T @ v[c0:c1]
+    out = [np.zeros_like(q), np.zeros_like(k), np.zeros_like(v), np.zeros_like(q)]
+    dq, dkk, dvv, dg = out
+    dS_out = np.zeros((dk, v.shape[1])) if dSf is None else dSf.copy()
+    exact_chunks = 0
+    for ci in range(len(bounds) - 1, -1, -1):
+        c0, c1 = bounds[ci]
+        n = c1 - c0
+        qc, kc, vc, oc, gc = q[c0:c1], k[c0:c1], v[c0:c1], dO[c0:c1], g[c0:c1]
+        Sin = S_in[ci]
+        G = np.cumprod(gc, axis=0)
+        a = G[-1]
+        A2 = oc @ vc.T                                   # A2[t, s] = dO_t . v_s
+        M = np.tril(np.ones((n, n)))
+        if a.min() >= fast_min:
+            qt, kt, kh = qc * G, kc / G, kc * (a / G)
+            dq[c0:c1] = (oc @ Sin.T + (M * A2) @ kt) * G
+            dkk[c0:c1] = ((M * A2).T @ qt) / G + (vc @ dS_out.T) * (a / G)
+            dvv[c0:c1] = (M * (qt @ kt.T)).T @ oc + kh @ dS_out
+            F = a / G                                    # P(t+1, n-1)
+        else:
+            exact_chunks += 1
+            P = range_products(gc)
+            for t in range(n):
+                dq[c0 + t] = (Sin @ oc[t]) * P[0, t] + sum(A2[t, s] * kc[s] * P[s + 1, t] for s in range(t + 1))
+            for s in range(n):
+                dkk[c0 + s] = (dS_out @ vc[s]) * P[s + 1, n - 1] + sum(
+                    A2[t, s] * qc[t] * P[s + 1, t] for t in range(s, n))
+                dvv[c0 + s] = (kc[s] * P[s + 1, n - 1]) @ dS_out + sum(
+                    ((qc[t] * P[s + 1, t]) @ kc[s]) * oc[t] for t in range(s, n))
+            F = P[1:n + 1, n - 1]
+        Gprev = np.vstack([np.ones((1, dk)), G[:-1]])    # P(0, t-1)
+        # the four terms of dg_t = sum_j D_t[:, j] S_{t-1}[:, j]
+        BE = F * Gprev * np.sum(dS_out * Sin, axis=1)
+        Y, X = kc * (vc @ dS_out.T), qc * (oc @ Sin.T)
+        Z, BF = np.zeros(dk), np.zeros((n, dk))
+        for t in range(n):                               # Z_t = sum_{s<t} P(s+1, t-1) Y_s
+            BF[t] = F[t] * Z
+            Z = gc[t] * Z + Y[t]
+        W, AE = np.zeros(dk), np.zeros((n, dk))
+        for t in range(n - 1, -1, -1):                   # W_t = sum_{r>=t} P(t+1, r) X_r
+            W = X[t] + (gc[t + 1] * W if t + 1 < n else 0.0)
+            AE[t] = Gprev[t] * W
+        K, AF = np.zeros((n, dk)), np.zeros((n, dk))
+        for t in range(n):                               # K_t[r] = sum_{s<t} P(s+1, t-1) A2[r, s] k_s
+            acc, dec = np.zeros(dk), np.ones(dk)
+            for r in range(t, n):                        # sum_{r>=t} P(t+1, r) q_r K_t[r]
+                if r > t:
+                    dec = dec * gc[r]
+                acc = acc + dec * qc[r] * K[r]
+            AF[t] = acc
+            K = gc[t] * K + A2[:, t:t + 1] * kc[t]
+        dg[c0:c1] = BE + BF + AE + AF
+        dS_out = a[:, None] * dS_out + (qc * G).T @ oc
+    return dq, dkk, dvv, dg, dS_out, exact_chunks
+
+
+@pytest.mark.parametrize("gates,T,C", [("slow", 70, 16), ("resets", 70, 16), ("slow", 9, 16)])
+def test_product_shaped_chunk_backward_equals_oracle(gates, T, C):
+    """Both routes of the product-shaped chunk backward against the oracle: gates in [0.9, 1]
+    keep every chunk on the fast route, gates with zeros send chunks to the exact route."""
+    rng = np.random.default_rng(11 + T)
+    B, H, dk, dv = 1, 1, 6, 4
+    q = rng.standard_normal((B, H, T, dk)).astype(np.float32)
+    k = rng.standard_normal((B, H, T, dk)).astype(np.float32)
+    v = rng.standard_normal((B, H, T, dv)).astype(np.float32)
+    g = rng.uniform(0.9, 1.0, (B, H, T, dk)).astype(np.float32)
+    if gates == "resets":
+        g[0, 0, 5, 2] = g[0, 0, 40, 0] = 0.0
+    dO = rng.standard_normal((B, H, T, dv)).astype(np.float32)
+    S0 = rng.standard_normal((B, H, dk, dv))
+    dSf = rng.standard_normal((B, H, dk, dv)).astype(np.float32)
+    ref = oracle.gla_backward(q, k, v, g, dO, state0=S0, dS_final=dSf)
+    *got, exact = chunk_backward_products(*(x[0, 0].astype(np.float64) for x in (q, k, v, g, dO)),
+                                         S0[0, 0], dSf[0, 0].astype(np.float64), C)
+    assert (exact > 0) == (gates == "resets")
+    for name, a, r in zip(("dq", "dk", "dv", "dg", "dstate0"), got, ref):
+        np.testing.assert_allclose(a, r[0, 0], rtol=1e-8, atol=1e-8, err_msg=name)
