@@ -1,5 +1,6 @@
-"""A randomized model of the hand-off protocol of the tensor-core SW-SKA backward's key-tile
-kernel (csrc/swska_backward_tc.cu, ska_bwd_dkdv_kernel), checked on the CPU.
+"""Randomized models of the hand-off protocols of the tensor-core SW-SKA backward
+(csrc/swska_backward_tc.cu), checked on the CPU: the key-tile kernel (ska_bwd_dkdv_kernel) here,
+the query-tile kernel (ska_bwd_dq_kernel) further down.
 
 One CTA owns a key tile and walks U = HG x n_q (head, query tile) units:
 - the producer loads K once, the V tile of each head, and each unit's Q, dO and row
@@ -27,35 +28,10 @@ import random
 
 import pytest
 
-
-class Bar:
-    def __init__(self, count):
-        self.count, self.pending, self.tx, self.phase = count, count, 0, 0
-
-    def arrive(self, n=1):
-        self.pending -= n
-        assert self.pending >= 0, "more arrivals than the barrier's count"
-        self._complete()
-
-    def expect_tx(self, nbytes):
-        self.tx += nbytes
-        self.arrive()
-
-    def complete_tx(self, nbytes):
-        self.tx -= nbytes
-        self._complete()
-
-    def _complete(self):
-        if self.pending == 0 and self.tx == 0:
-            self.phase += 1
-            self.pending = self.count
-
-    def passed(self, parity):
-        return (self.phase & 1) != parity
+from .barrier_model import Bar, simulate
 
 
 def run(HG, n_q, seed, mistake=None):
-    rnd = random.Random(seed)
     U = HG * n_q
     kfull, vfull, vempty = Bar(1), Bar(1), Bar(1)
     full, empty = [Bar(1), Bar(1)], [Bar(1), Bar(1)]
@@ -179,40 +155,21 @@ def run(HG, n_q, seed, mistake=None):
             m["dK"] += 1
             m["slot_readers"][u % 2].add("DK")
 
-    actors = {"producer": producer(), "issuer": issuer(), "half0": softmax(0), "half1": softmax(1)}
-    waiting = dict.fromkeys(actors)
-    finished = set()
-    for _ in range(2_000_000):
-        ready = [a for a in actors if a not in finished
-                 and (waiting[a] is None or waiting[a][0].passed(waiting[a][1]))]
-        ready += ["pipe"] * bool(pipe) + ["copy"] * bool(copies)
-        if not ready:
-            assert len(finished) == len(actors), f"deadlock, waiting: {waiting}"
-            return
-        a = rnd.choice(ready)
-        if a == "pipe":
-            execute(pipe.pop(0))
-        elif a == "copy":
-            kind, s, what, bar = copies.pop(rnd.randrange(len(copies)))
-            if kind == "K":
-                m["K"] = what
-            elif kind == "V":
-                m["V"] = what
-            else:
-                prev = m["slot"][s]
-                assert prev is None or m["slot_readers"][s] == {"ST", "DPT", "DV", "DK"}, \
-                    f"slot {s} reloaded while unit {prev} is in use"
-                m["slot"][s], m["slot_readers"][s] = what, set()
-            bar.complete_tx(1)
+    def land(copy):
+        kind, s, what, bar = copy
+        if kind == "K":
+            m["K"] = what
+        elif kind == "V":
+            m["V"] = what
         else:
-            waiting[a] = None
-            try:
-                r = next(actors[a])
-                if r[0] == "wait":
-                    waiting[a] = (r[1], r[2])
-            except StopIteration:
-                finished.add(a)
-    raise AssertionError("no progress")
+            prev = m["slot"][s]
+            assert prev is None or m["slot_readers"][s] == {"ST", "DPT", "DV", "DK"}, \
+                f"slot {s} reloaded while unit {prev} is in use"
+            m["slot"][s], m["slot_readers"][s] = what, set()
+        bar.complete_tx(1)
+
+    actors = {"producer": producer(), "issuer": issuer(), "half0": softmax(0), "half1": softmax(1)}
+    simulate(seed, actors, pipe, copies, execute, land)
 
 
 def _shape(seed):
@@ -239,6 +196,133 @@ def test_model_catches_planted_protocol_mistakes(mistake):
         HG, n_q = _shape(seed)
         try:
             run(max(HG, 2), max(n_q, 2), seed, mistake)
+        except AssertionError:
+            caught += 1
+    assert caught >= 50, f"{mistake}: caught in {caught} of 100 runs"
+
+
+# ---- launch 2: query tiles (ska_bwd_dq_kernel) -------------------------------------------------
+# One CTA owns a query tile and walks its n key tiles: K(u) through a three-slot ring, V(u)
+# through a two-slot ring; S(u) = Q K(u)^T into TMEM buffer u mod 2, dP(u) = dO V(u)^T into one
+# region; the two softmax warpgroups (one per half of the keys) form P from S, then
+# dS = P (dP - D) over the first columns of the same S buffer; dQ += dS(u) K(u). The issue
+# order S(0) dP(0) S(1) | dQ(0) dP(1) S(2) | dQ(1) dP(2) S(3) | ... puts S(u+2) into the buffer
+# dQ(u) reads, which the in-order pipe allows.
+
+
+def run_dq(n, seed, mistake=None):
+    KS, VS = 3, 2
+    kfull, kempty = [Bar(1) for _ in range(KS)], [Bar(1) for _ in range(KS)]
+    vfull, vempty = [Bar(1) for _ in range(VS)], [Bar(1) for _ in range(VS)]
+    qfull, pfull, done = Bar(1), Bar(1), Bar(1)
+    sfull, dsready = [Bar(1), Bar(1)], Bar(256)
+    m = {"q": False, "k": [None] * KS, "k_readers": [set() for _ in range(KS)],
+         "v": [None] * VS, "v_readers": [set() for _ in range(VS)],
+         "S": [None, None], "dS": [set(), set()], "dP": None, "dP_readers": set(), "dQ": 0}
+    pipe, copies = [], []
+
+    def producer():
+        qfull.expect_tx(1)
+        copies.append(("q", None, None, qfull))
+        for u in range(n):
+            if u >= KS and mistake != "k_slot_reloaded_early":
+                yield ("wait", kempty[u % KS], (u // KS - 1) & 1)
+            kfull[u % KS].expect_tx(1)
+            copies.append(("k", u % KS, u, kfull[u % KS]))
+            if u >= VS:
+                yield ("wait", vempty[u % VS], (u // VS - 1) & 1)
+            vfull[u % VS].expect_tx(1)
+            copies.append(("v", u % VS, u, vfull[u % VS]))
+            yield ("step",)
+
+    def issuer():
+        yield ("wait", qfull, 0)
+        yield ("wait", kfull[0], 0)
+        pipe.extend([("S", 0), ("C", sfull[0])])
+        yield ("wait", vfull[0], 0)
+        pipe.extend([("DP", 0), ("C", pfull), ("C", vempty[0])])
+        if n > 1:
+            yield ("wait", kfull[1], 0)
+            pipe.extend([("S", 1), ("C", sfull[1])])
+        for u in range(n):
+            if mistake == "s_before_dsready" and u + 2 < n:
+                yield ("wait", kfull[(u + 2) % KS], ((u + 2) // KS) & 1)
+                pipe.extend([("S", u + 2), ("C", sfull[(u + 2) & 1])])
+            yield ("wait", dsready, u & 1)
+            pipe.extend([("DQ", u), ("C", kempty[u % KS])])
+            if u + 1 < n:
+                yield ("wait", vfull[(u + 1) % VS], ((u + 1) // VS) & 1)
+                pipe.extend([("DP", u + 1), ("C", pfull), ("C", vempty[(u + 1) % VS])])
+            if u + 2 < n and mistake != "s_before_dsready":
+                yield ("wait", kfull[(u + 2) % KS], ((u + 2) // KS) & 1)
+                pipe.extend([("S", u + 2), ("C", sfull[(u + 2) & 1])])
+        pipe.append(("C", done))
+
+    def softmax(w):
+        for u in range(n):
+            yield ("wait", sfull[u & 1], (u >> 1) & 1)
+            assert m["S"][u & 1] == u, f"half {w} read S {m['S'][u & 1]} for {u}"
+            yield ("step",)
+            assert m["S"][u & 1] == u, "S overwritten while being read"
+            yield ("wait", pfull, u & 1)
+            assert m["dP"] == u, f"half {w} read dP {m['dP']} for {u}"
+            m["dS"][u & 1].add(w)
+            m["dP_readers"].add(w)
+            dsready.arrive(128)
+        yield ("wait", done, 0)
+        assert m["dQ"] == n
+
+    def execute(op):
+        kind = op[0]
+        if kind == "C":
+            op[1].arrive()
+        elif kind == "S":
+            u = op[1]
+            assert m["q"] and m["k"][u % KS] == u
+            b = u & 1
+            assert m["S"][b] is None or m["dQ"] > m["S"][b], "S buffer overwritten before dQ read its dS"
+            m["S"][b], m["dS"][b] = u, set()
+            m["k_readers"][u % KS].add("S")
+        elif kind == "DP":
+            u = op[1]
+            assert m["v"][u % VS] == u
+            assert m["dP"] is None or m["dP_readers"] == {0, 1}, "dP overwritten while in use"
+            m["dP"], m["dP_readers"] = u, set()
+            m["v_readers"][u % VS].add("DP")
+        else:
+            u = op[1]
+            assert m["S"][u & 1] == u and m["dS"][u & 1] == {0, 1}, f"dQ({u}) read an unfinished dS"
+            assert m["k"][u % KS] == u and m["dQ"] == u
+            m["dQ"] += 1
+            m["k_readers"][u % KS].add("DQ")
+
+    def land(copy):
+        kind, s, u, bar = copy
+        if kind == "q":
+            m["q"] = True
+        elif kind == "k":
+            assert m["k"][s] is None or m["k_readers"][s] == {"S", "DQ"}, f"K slot {s} reloaded early"
+            m["k"][s], m["k_readers"][s] = u, set()
+        else:
+            assert m["v"][s] is None or m["v_readers"][s] == {"DP"}, f"V slot {s} reloaded early"
+            m["v"][s], m["v_readers"][s] = u, set()
+        bar.complete_tx(1)
+
+    actors = {"producer": producer(), "issuer": issuer(), "half0": softmax(0), "half1": softmax(1)}
+    simulate(seed, actors, pipe, copies, execute, land)
+
+
+def test_query_tile_protocol_holds():
+    for seed in range(300):
+        run_dq(random.Random(seed).choice([1, 2, 3, 4, 7, 33]), seed)
+
+
+@pytest.mark.parametrize("mistake", ["s_before_dsready", "k_slot_reloaded_early"])
+def test_query_tile_model_catches_planted_mistakes(mistake):
+    caught = 0
+    for seed in range(100):
+        try:
+            run_dq(random.Random(seed).choice([4, 7, 33]), seed, mistake)
         except AssertionError:
             caught += 1
     assert caught >= 50, f"{mistake}: caught in {caught} of 100 runs"

@@ -24,42 +24,14 @@ import random
 
 import pytest
 
+from .barrier_model import Bar, simulate
+
 NSLOT = 4
-
-
-class Bar:
-    """mbarrier: `count` arrivals plus the expected transaction bytes complete a phase."""
-
-    def __init__(self, count):
-        self.count, self.pending, self.tx, self.phase = count, count, 0, 0
-
-    def arrive(self, n=1):
-        self.pending -= n
-        assert self.pending >= 0, "more arrivals than the barrier's count"
-        self._complete()
-
-    def expect_tx(self, nbytes):
-        self.tx += nbytes
-        self.arrive()
-
-    def complete_tx(self, nbytes):
-        self.tx -= nbytes
-        self._complete()
-
-    def _complete(self):
-        if self.pending == 0 and self.tx == 0:
-            self.phase += 1
-            self.pending = self.count
-
-    def passed(self, parity):
-        # a parity wait succeeds unless the barrier's current phase has that parity
-        return (self.phase & 1) != parity
 
 
 def run(items, seed, mistake=None):
     """items: key tiles per work item of one CTA, in order. Raises AssertionError on a
     protocol violation or a deadlock."""
-    rnd = random.Random(seed)
     full = [Bar(1) for _ in range(NSLOT)]
     empty = [Bar(1) for _ in range(NSLOT)]
     qfull, qempty = Bar(1), Bar(1)
@@ -173,39 +145,19 @@ def run(items, seed, mistake=None):
             O[h] = (it, 2 * j + half + 1)
         slot_reads[s] += 1
 
-    actors = {"producer": producer(), "issuer": issuer(), "softmax0": softmax(0), "softmax1": softmax(1)}
-    waiting = dict.fromkeys(actors)
-    finished = set()
-    for _ in range(2_000_000):
-        ready = [a for a in actors if a not in finished
-                 and (waiting[a] is None or waiting[a][0].passed(waiting[a][1]))]
-        ready += ["pipe"] * bool(pipe) + ["copy"] * bool(copies)
-        if not ready:
-            assert len(finished) == len(actors), f"deadlock, waiting: {waiting}"
-            break
-        a = rnd.choice(ready)
-        if a == "pipe":
-            execute(pipe.pop(0))
-        elif a == "copy":
-            kind, s, tile, bar, nbytes = copies.pop(rnd.randrange(len(copies)))
-            if kind == "q":
-                prev = items[tile - 1] if tile > 0 else 0
-                assert st["q_reads"] == 2 * prev, "Q overwritten before its score MMAs ran"
-                st["q"], st["q_reads"] = tile, 0
-            else:
-                assert slot[s] is None or slot_reads[s] == 2, f"slot {s} overwritten: {slot[s]}"
-                slot[s], slot_reads[s] = tile, 0
-            bar.complete_tx(nbytes)
+    def land(copy):
+        kind, s, tile, bar, nbytes = copy
+        if kind == "q":
+            prev = items[tile - 1] if tile > 0 else 0
+            assert st["q_reads"] == 2 * prev, "Q overwritten before its score MMAs ran"
+            st["q"], st["q_reads"] = tile, 0
         else:
-            waiting[a] = None
-            try:
-                r = next(actors[a])
-                if r[0] == "wait":
-                    waiting[a] = (r[1], r[2])
-            except StopIteration:
-                finished.add(a)
-    else:
-        raise AssertionError("no progress")
+            assert slot[s] is None or slot_reads[s] == 2, f"slot {s} overwritten: {slot[s]}"
+            slot[s], slot_reads[s] = tile, 0
+        bar.complete_tx(nbytes)
+
+    actors = {"producer": producer(), "issuer": issuer(), "softmax0": softmax(0), "softmax1": softmax(1)}
+    simulate(seed, actors, pipe, copies, execute, land)
     if mistake != "next_item_before_epilogue":
         assert all(len(epilogue_done[h]) == len(items) for h in (0, 1))
 
