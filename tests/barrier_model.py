@@ -3,9 +3,9 @@
 - `Bar` follows mbarrier semantics. A phase completes when its arrival count is reached and the
   transaction bytes it expects have landed. A parity wait succeeds unless the current phase has
   that parity, so a waiter two phases ahead passes at once, as on the GPU.
-- `simulate` runs the kernel's roles as coroutines under a random scheduler, beside an in-order
-  MMA pipe (a commit arrives once everything issued before it has executed) and copies that
-  land at random times.
+- `simulate` runs the kernel's roles as coroutines under a random scheduler, beside in-order MMA
+  pipes, one per issuing warp (a commit arrives once everything its warp issued before it has
+  executed), and copies that land at random times.
 """
 import random
 
@@ -36,23 +36,24 @@ class Bar:
         return (self.phase & 1) != parity
 
 
-def simulate(seed, actors, pipe, copies, execute, land, max_steps=2_000_000):
-    """actors: name -> generator yielding ("wait", bar, parity) or ("step",). pipe: list of
-    issued ops, executed in order by execute(op). copies: pending copies, each landed by
-    land(copy) in random order. Raises AssertionError on a deadlock or no progress."""
+def simulate(seed, actors, pipes, copies, execute, land, max_steps=2_000_000):
+    """actors: name -> generator yielding ("wait", bar, parity) or ("step",). pipes: one list of
+    issued ops per issuing warp, each executed in order by execute(op), with no order between
+    pipes. copies: pending copies, each landed by land(copy) in random order. Raises
+    AssertionError on a deadlock or no progress."""
     rnd = random.Random(seed)
     waiting = dict.fromkeys(actors)
     finished = set()
     for _ in range(max_steps):
         ready = [a for a in actors if a not in finished
                  and (waiting[a] is None or waiting[a][0].passed(waiting[a][1]))]
-        ready += ["pipe"] * bool(pipe) + ["copy"] * bool(copies)
+        ready += [("pipe", i) for i, p in enumerate(pipes) if p] + ["copy"] * bool(copies)
         if not ready:
             assert len(finished) == len(actors), f"deadlock, waiting: {waiting}"
             return
         a = rnd.choice(ready)
-        if a == "pipe":
-            execute(pipe.pop(0))
+        if isinstance(a, tuple):
+            execute(pipes[a[1]].pop(0))
         elif a == "copy":
             land(copies.pop(rnd.randrange(len(copies))))
         else:

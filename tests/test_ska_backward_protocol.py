@@ -169,7 +169,7 @@ def run(HG, n_q, seed, mistake=None):
         bar.complete_tx(1)
 
     actors = {"producer": producer(), "issuer": issuer(), "half0": softmax(0), "half1": softmax(1)}
-    simulate(seed, actors, pipe, copies, execute, land)
+    simulate(seed, actors, [pipe], copies, execute, land)
 
 
 def _shape(seed):
@@ -309,7 +309,7 @@ def run_dq(n, seed, mistake=None):
         bar.complete_tx(1)
 
     actors = {"producer": producer(), "issuer": issuer(), "half0": softmax(0), "half1": softmax(1)}
-    simulate(seed, actors, pipe, copies, execute, land)
+    simulate(seed, actors, [pipe], copies, execute, land)
 
 
 def test_query_tile_protocol_holds():

@@ -157,7 +157,7 @@ def run(items, seed, mistake=None):
         bar.complete_tx(nbytes)
 
     actors = {"producer": producer(), "issuer": issuer(), "softmax0": softmax(0), "softmax1": softmax(1)}
-    simulate(seed, actors, pipe, copies, execute, land)
+    simulate(seed, actors, [pipe], copies, execute, land)
     if mistake != "next_item_before_epilogue":
         assert all(len(epilogue_done[h]) == len(items) for h in (0, 1))
 
