@@ -37,10 +37,10 @@ class Bar:
 
 
 def simulate(seed, actors, pipes, copies, execute, land, max_steps=2_000_000):
-    """actors: name -> generator yielding ("wait", bar, parity) or ("step",). pipes: one list of
-    issued ops per issuing warp, each executed in order by execute(op), with no order between
-    pipes. copies: pending copies, each landed by land(copy) in random order. Raises
-    AssertionError on a deadlock or no progress."""
+    """actors: name (a string) -> generator yielding ("wait", bar, parity) or ("step",).
+    pipes: one list of issued ops per issuing warp, each executed in order by execute(op), with
+    no order between pipes. copies: pending copies, each landed by land(copy) in random order.
+    Raises AssertionError on a deadlock or no progress."""
     rnd = random.Random(seed)
     waiting = dict.fromkeys(actors)
     finished = set()
