@@ -585,8 +585,10 @@ gla_chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                 }
             }
             // pass C needs the previous chunk's MMAs done every chunk (its outputs, S_bf reuse);
-            // pass A only when R is rescaled (S = diag(D) R takes new terms without touching R)
-            const bool need_prev = n > 0 && (MODE == PASS_C || rmw);
+            // pass A when R is rescaled (S = diag(D) R takes new terms without touching R), and
+            // before its last chunk: the tail then waits for the last phase of barO with every
+            // earlier phase known complete (a parity wait must not be two phases ahead)
+            const bool need_prev = n > 0 && (MODE == PASS_C || rmw || n == n_ch - 1);
             if (need_prev) {
                 if (!grp_all(2, wait_bar(barO, (uint32_t)((n - 1) & 1), abort_flag))) { ok = false; break; }
                 tc::fence_after_sync();

@@ -144,3 +144,96 @@ def test_model_catches_planted_protocol_mistakes(mistake):
         except AssertionError:
             caught += 1
     assert caught >= 50, f"{mistake}: caught in {caught} of 100 runs"
+
+
+def run_pass_a(rescales, seed, mistake=None):
+    """Pass A (the segment's state contribution only): no A, P or O; warp 4 issues R += k^^T V
+    per chunk. Warpgroup 1 waits for the previous chunk's MMAs only when R is rescaled in place
+    (a read-modify-write of R in TMEM by its threads), which must not overlap an R update."""
+    N = len(rescales)
+    full, empty, ops = [Bar(1), Bar(1)], [Bar(1), Bar(1)], [Bar(1), Bar(1)]
+    barO = Bar(1)
+    m = {"stage": [None, None], "operands": [None, None], "readers": [set(), set()],
+         "R": 0, "R_rescaled": set()}
+    pipe4, copies = [], []
+
+    def producer():
+        for n in range(N):
+            st = n & 1
+            if n >= 2:
+                yield ("wait", empty[st], ((n >> 1) - 1) & 1)
+            full[st].expect_tx(1)
+            copies.append((st, n, full[st]))
+            yield ("step",)
+
+    def operands():
+        for n in range(N):
+            st = n & 1
+            yield ("wait", full[st], (n >> 1) & 1)
+            assert m["stage"][st] == n
+            yield ("step",)
+            m["operands"][st] = n
+            m["readers"][st].add("wg0")
+            ops[st].arrive()
+
+    def state():
+        for n in range(N):
+            st = n & 1
+            yield ("wait", ops[st], (n >> 1) & 1)
+            # the previous chunk's MMAs are awaited before a rescale, and before the last chunk
+            # (so that the final wait below cannot alias an earlier phase)
+            last = n == N - 1 and mistake != "no_wait_before_last_chunk"
+            if (rescales[n] or last) and n > 0 and mistake != "rescale_without_barO":
+                yield ("wait", barO, (n - 1) & 1)
+            if rescales[n] and n > 0:
+                assert m["R"] == n, f"R rescaled for chunk {n} while {n - m['R']} updates are pending"
+                yield ("step",)
+                assert m["R"] == n, "R updated during its in-place rescale"
+                m["R_rescaled"].add(n)
+            pipe4.extend([("R", n, st), ("C", barO), ("C", empty[st])])
+        yield ("wait", barO, (N - 1) & 1)
+        assert m["R"] == N
+
+    def execute(op):
+        if op[0] == "C":
+            op[1].arrive()
+            return
+        _, n, st = op
+        assert m["operands"][st] == n and m["R"] == n
+        assert not rescales[n] or n == 0 or n in m["R_rescaled"], "R updated before its rescale"
+        m["R"] = n + 1
+        m["readers"][st].add("R")
+
+    def land(copy):
+        st, n, bar = copy
+        if m["stage"][st] is not None:
+            assert m["readers"][st] >= {"wg0", "R"}, f"stage {st} reloaded while in use"
+        m["stage"][st], m["readers"][st], m["operands"][st] = n, set(), None
+        bar.complete_tx(1)
+
+    simulate(seed, {"producer": producer(), "operands": operands(), "state": state()},
+             [pipe4], copies, execute, land)
+
+
+def test_pass_a_protocol_holds():
+    for seed in range(300):
+        rnd = random.Random(seed)
+        run_pass_a([rnd.random() < 0.3 for _ in range(rnd.randint(1, 12))], seed)
+
+
+@pytest.mark.parametrize("mistake", ["rescale_without_barO", "no_wait_before_last_chunk"])
+def test_pass_a_model_catches_planted_mistakes(mistake):
+    """The second is the pass's earlier form: without the wait before the last chunk, the final
+    wait for phase N-1 could pass while phase N-2 was still pending (a parity wait two phases
+    ahead), and the segment's state would be read before its last updates."""
+    caught = 0
+    for seed in range(300):
+        rnd = random.Random(seed)
+        rescales = [rnd.random() < 0.5 for _ in range(rnd.randint(4, 12))]
+        if mistake == "no_wait_before_last_chunk":
+            rescales[-1] = False
+        try:
+            run_pass_a(rescales, seed, mistake)
+        except AssertionError:
+            caught += 1
+    assert caught >= 15, f"{mistake}: caught in {caught} of 300 runs"
