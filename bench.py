@@ -349,19 +349,30 @@ def run_gpu(args):
                 "traffic": recorded_traffic("swska_prefill_stack", ["swska_prefill_tc.cu", "tc.cuh", "common.cuh"])}
 
     # ---- batched decode step (recurrence + SW-SKA), 256 sequences ----
+    # Timed over rotating input sets so that no iteration finds its state or cache in L2 from
+    # the one before: 4 recurrence sets (state 537 MB each, 2.1 GB in all) and 2 SW-SKA sets
+    # (4.6 GB of cache each), each set visited once per rotation.
     dd_dims = wl.WORKLOADS["decode_n256"].dims
     N, Wd = dd_dims["N"], dd_dims["window"]
-    dd = wl.decode_inputs(N, H, dk, dv, Wd, seed=seed_base + 77, device=dev)
+    n_gla_sets, n_ska_sets = 4, 2
+    gsets = [wl.decode_inputs(N, H, dk, dv, Wd, seed=seed_base + 77 + i, device=dev)
+             for i in range(max(n_gla_sets, n_ska_sets))]
+    for i, sset in enumerate(gsets):  # keep the recurrence part of every set, caches of the first two
+        if i >= n_ska_sets:
+            del sset["k_cache"], sset["v_cache"]
+    torch.cuda.empty_cache()
+    dd = gsets[0]
     o1 = torch.empty(N, H, dv, dtype=torch.bfloat16, device=dev)
     o2 = torch.empty_like(o1)
 
-    def dec_step():
-        rod.gla_decode_step(dd["q"], dd["k"], dd["v"], dd["g"], dd["state"], o=o1)
-        rod.swska_decode(dd["sq"], dd["k_new"], dd["v_new"], dd["k_cache"], dd["v_cache"],
-                         dd["pos"], Wd, o=o2)
+    def dec_step(i):
+        a, b = gsets[i % n_gla_sets], gsets[i % n_ska_sets]
+        rod.gla_decode_step(a["q"], a["k"], a["v"], a["g"], a["state"], o=o1)
+        rod.swska_decode(b["sq"], b["k_new"], b["v_new"], b["k_cache"], b["v_cache"],
+                         b["pos"], Wd, o=o2)
 
-    for _ in range(max(3, args.warmup)):
-        dec_step()
+    for i in range(max(4, args.warmup)):
+        dec_step(i)
     rod.check()
     dsteps = max(20, args.steps * 4)
     ge = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(dsteps)]
@@ -371,12 +382,13 @@ def run_gpu(args):
     e1 = torch.cuda.Event(enable_timing=True)
     e0.record(stream)
     for i in range(dsteps):
+        a, b = gsets[i % n_gla_sets], gsets[i % n_ska_sets]
         ge[i][0].record(stream)
-        rod.gla_decode_step(dd["q"], dd["k"], dd["v"], dd["g"], dd["state"], o=o1)
+        rod.gla_decode_step(a["q"], a["k"], a["v"], a["g"], a["state"], o=o1)
         ge[i][1].record(stream)
         se[i][0].record(stream)
-        rod.swska_decode(dd["sq"], dd["k_new"], dd["v_new"], dd["k_cache"], dd["v_cache"],
-                         dd["pos"], Wd, o=o2)
+        rod.swska_decode(b["sq"], b["k_new"], b["v_new"], b["k_cache"], b["v_cache"],
+                         b["pos"], Wd, o=o2)
         se[i][1].record(stream)
     e1.record(stream)
     barrier()
@@ -433,6 +445,8 @@ def run_gpu(args):
     decode = {
         "workload": "decode_n256 (N=256 sequences x 1 token, H=16, 128x128 fp32 state, "
                     "SW-SKA ring window 4096)",
+        "l2": f"rotating input sets: {n_gla_sets} recurrence sets (537 MB of state each), "
+              f"{n_ska_sets} SW-SKA sets (4.6 GB of cache each)",
         "value": round(N * world / (dec_ms / 1e3), 1), "unit": "tokens/s",
         "ms_per_step": round(dec_ms, 4),
         "kernels": {
@@ -488,7 +502,7 @@ def run_gpu(args):
     if not args.no_e2e:
         e2e = run_e2e(args, rod, torch, layers, d, ws, stream, barrier, ranks_max, world)
 
-    del layers, dd
+    del layers, dd, gsets
     torch.cuda.empty_cache()
 
     # ---- generation loop: one token through all 24 layers' decode kernels, eager vs graph ----
@@ -499,6 +513,10 @@ def run_gpu(args):
     backward = None
     if not args.no_backward:
         backward = run_backward(rod, torch, wl, dev, H, dk, W, seed_base, barrier, ranks_max, world)
+    configs = None
+    if not args.no_configs:
+        configs = run_configs(rod, torch, wl, dev, seed_base, barrier, ranks_max, world, rank,
+                              with_oracle=(rank == 0 and world == 1 and not args.no_cpu_baseline))
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         cpu = oracle_stack_sample(d)
@@ -517,7 +535,7 @@ def run_gpu(args):
                    "l2": "inputs > L2 (55 GB per step), no flush needed"},
         "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": launches,
         "clocks": clocks, "decode": decode, "generate": generate, "backward": backward,
-        "kernels": kernels,
+        "kernels": kernels, "configs": configs,
     }
     if rank == 0:
         print(json.dumps(line), flush=True)
@@ -585,6 +603,148 @@ def run_backward(rod, torch, wl, dev, H, d, W, seed_base, barrier, reduce_max, w
                              "peak_source": f"{peaks_src} bf16_tflops (burst: timed alone)",
                              "executed_flop_per_pair": 18 * d}
     del q, k, v, dO
+    torch.cuda.empty_cache()
+    return out
+
+
+def run_configs(rod, torch, wl, dev, seed_base, barrier, reduce_max, world, rank, with_oracle):
+    """The three single-mixer workloads beside the stack, each with its own throughput, its
+    roofline fraction and the oracle timed on the host cores (rank 0, one GPU only):
+      tiny_fp32                 both mixers, B1 T256 H2 dk16 dv32 (latency-bound: no fraction)
+      gla_prefill_b4_t4096      recurrence prefill, HBM-bound
+      swska_prefill_b2_t32768   SW-SKA prefill, tensor-bound (burst bf16 peak: timed alone)
+    Launches of the two large ones are timed one by one with CUDA events, with a read of a
+    512 MB buffer between them (outside the events) so that every launch starts with its
+    inputs out of L2 and with no dirty lines of the previous launch left to write back."""
+    import numpy as np
+
+    import oracle
+
+    peaks, peaks_src = load_peaks()
+    hbm, tc_peak = peaks.get("hbm_gbs"), peaks.get("bf16_tflops")
+    flush = torch.empty(512 << 20, dtype=torch.uint8, device=dev)
+    out = {}
+
+    def timed_flushed(fn, iters):
+        fn()
+        barrier()
+        ts = []
+        for _ in range(iters):
+            flush.sum(dtype=torch.int64)
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            fn()
+            e1.record()
+            torch.cuda.synchronize()
+            ts.append(e0.elapsed_time(e1))
+        rod.check()
+        return reduce_max(statistics.median(ts))
+
+    def timed_loop(fn, iters):
+        fn()
+        barrier()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for _ in range(iters):
+            fn()
+        e1.record()
+        barrier()
+        rod.check()
+        return reduce_max(e0.elapsed_time(e1) / iters)
+
+    def oracle_timed(fn):
+        t0 = time.perf_counter()
+        fn()
+        return time.perf_counter() - t0
+
+    cores = oracle.default_threads()
+    # ---- tiny fp32: both mixers, every product an fp32 FMA (CUDA cores) ----
+    d = wl.WORKLOADS["tiny_fp32"].dims
+    B, T, H, dk, dv, C, W = d["B"], d["T"], d["H"], d["dk"], d["dv"], d["chunk"], d["window"]
+    q, k, v, g = wl.gla_inputs(B, H, T, dk, dv, dist="tiny", seed=seed_base, dtype="fp32")
+    sq, sk, sv = wl.swska_inputs(B, H, T, dk, dv, dist="tiny", seed=seed_base + 1, dtype="fp32")
+    gq, gk, gv, gg = [t.to(dev) for t in (q, k, v, g)]
+    dq_, dk_, dv_ = [t.to(dev) for t in (sq, sk, sv)]
+    st = torch.zeros(B, H, dk, dv, device=dev)
+    o1 = torch.empty(B, H, T, dv, device=dev)
+    o2 = torch.empty(B, H, T, dv, device=dev)
+    gla_ms = timed_loop(lambda: rod.gla_prefill(gq, gk, gv, gg, st.zero_(), o=o1, chunk=C), 200)
+    ska_ms = timed_loop(lambda: rod.swska_prefill(dq_, dk_, dv_, W, o=o2), 200)
+    ent = {"workload": "tiny_fp32: recurrence + SW-SKA, B1 T256 H2 dk16 dv32 chunk 32 window 64, fp32",
+           "bound": "latency", "frac": None,
+           "gla_prefill_us": round(gla_ms * 1e3, 2), "swska_prefill_us": round(ska_ms * 1e3, 2),
+           "value": round(B * T * world / ((gla_ms + ska_ms) / 1e3), 1),
+           "unit": "tokens/s (both mixers)"}
+    if with_oracle:
+        reps = 20
+        sec = oracle_timed(lambda: [(oracle.gla_prefill(q, k, v, g), oracle.swska_prefill(sq, sk, sv, W))
+                                    for _ in range(reps)]) / reps
+        ent["cpu_baseline"] = {"value": round(B * T / sec, 1), "unit": "tokens/s (both mixers)",
+                               "cores": cores, "kind": "oracle", "sample": "the whole workload"}
+    out["tiny_fp32"] = ent
+    del gq, gk, gv, gg, dq_, dk_, dv_, st, o1, o2
+
+    # ---- recurrence prefill B4 T4096 H16 d128 chunk 64 (HBM-bound) ----
+    d = wl.WORKLOADS["gla_prefill_b4_t4096"].dims
+    B, T, H, dk, dv, C = d["B"], d["T"], d["H"], d["dk"], d["dv"], d["chunk"]
+    q, k, v, g = wl.gla_inputs(B, H, T, dk, dv, dist="l2", seed=seed_base + 2, device=dev)
+    st = torch.zeros(B, H, dk, dv, device=dev)
+    o = torch.empty(B, H, T, dv, dtype=torch.bfloat16, device=dev)
+    ws = torch.empty(max(rod.gla_prefill_workspace_size(B, H, T, dk, dv, C), 16), dtype=torch.uint8, device=dev)
+    ms = timed_flushed(lambda: rod.gla_prefill(q, k, v, g, st.zero_(), o=o, chunk=C, workspace=ws), 20)
+    nbytes = B * H * T * (3 * dk * 2 + dk * 4 + dv * 2) + B * H * dk * dv * 4 * 2
+    flop = B * H * T * (2 * dk * (C + 1) / 2 * 2 + 4 * dk * dv)  # intra QK + AV, readout, state
+    ent = {"workload": "gla_prefill_b4_t4096: recurrence prefill, B4 T4096 H16 d128 chunk 64, bf16 in, "
+                       "fp32 gates and state",
+           "ms": round(ms, 4), "value": round(B * T * world / (ms / 1e3), 1), "unit": "tokens/s",
+           "bound": "hbm", "algorithmic_bytes": nbytes,
+           "achieved": round(nbytes / (ms / 1e3) / 1e9, 1), "peak": hbm, "peak_unit": "GB/s",
+           "frac": round(nbytes / (ms / 1e3) / 1e9 / hbm, 4),
+           "tflops_algorithmic": round(flop / (ms / 1e3) / 1e12, 2),
+           "traffic": recorded_traffic("gla_prefill_b4_t4096", ["gla_prefill_tc.cu", "tc.cuh", "common.cuh"])}
+    del q, k, v, g, st, o, ws
+    if with_oracle:
+        qh, kh, vh, gh = wl.gla_inputs(B, H, T, dk, dv, dist="l2", seed=seed_base + 2)
+        sec = oracle_timed(lambda: oracle.gla_prefill(qh, kh, vh, gh))
+        ent["cpu_baseline"] = {"value": round(B * T / sec, 1), "unit": "tokens/s", "cores": cores,
+                               "kind": "oracle", "sample": f"the whole workload ({sec:.2f} s)"}
+        del qh, kh, vh, gh
+    out["gla_prefill_b4_t4096"] = ent
+
+    # ---- SW-SKA prefill B2 T32768 H16 d128 window 4096 (tensor-bound) ----
+    d = wl.WORKLOADS["swska_prefill_b2_t32768"].dims
+    B, T, H, dk, dv, W = d["B"], d["T"], d["H"], d["dk"], d["dv"], d["window"]
+    q, k, v = wl.swska_inputs(B, H, T, dk, dv, seed=seed_base + 3, device=dev)
+    o = torch.empty(B, H, T, dv, dtype=torch.bfloat16, device=dev)
+    ms = timed_flushed(lambda: rod.swska_prefill(q, k, v, W, o=o), 10)
+    flop = 2.0 * (dk + dv) * swska_pairs(T, W) * B * H
+    nbytes = B * H * T * (dk + 2 * dv) * 2 + B * T * dk * 2
+    ent = {"workload": "swska_prefill_b2_t32768: SW-SKA prefill, B2 T32768 H16 d128 window 4096, bf16",
+           "ms": round(ms, 4), "value": round(B * T * world / (ms / 1e3), 1), "unit": "tokens/s",
+           "bound": "tensor", "flop": flop, "achieved": round(flop / (ms / 1e3) / 1e12, 1),
+           "peak": tc_peak, "peak_unit": "TFLOP/s",
+           "peak_source": f"{peaks_src} bf16_tflops (burst: timed alone)",
+           "frac": round(flop / (ms / 1e3) / 1e12 / tc_peak, 4),
+           "achieved_gbs": round(nbytes / (ms / 1e3) / 1e9, 1)}
+    del q, k, v, o
+    if with_oracle:
+        qh, kh, vh = wl.swska_inputs(B, H, T, dk, dv, seed=seed_base + 3)
+        n_rows = 8192
+        rng = np.random.default_rng(3)
+        rows = rng.integers(0, B * H * T, n_rows)
+        # the cost of a row is its window length: scale by the workload's mean window length
+        tt = rows % T
+        mean_w_sample = float(np.mean(np.minimum(tt + 1, W)))
+        mean_w_all = swska_pairs(T, W) / T
+        sec = oracle_timed(lambda: oracle.swska_prefill(qh, kh, vh, W, rows=rows))
+        sec_all = sec / n_rows * (B * H * T) * mean_w_all / mean_w_sample
+        ent["cpu_baseline"] = {"value": round(B * T / sec_all, 2), "unit": "tokens/s", "cores": cores,
+                               "kind": "oracle",
+                               "sample": f"{n_rows} random output rows ({sec:.2f} s), scaled to the whole "
+                                         "workload by window length"}
+        del qh, kh, vh
+    out["swska_prefill_b2_t32768"] = ent
+    del flush
     torch.cuda.empty_cache()
     return out
 
@@ -831,11 +991,12 @@ def main():
     ap.add_argument("--steps", type=int, default=10)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", default="rod", choices=["rod", "reference"])
-    ap.add_argument("--e2e-steps", type=int, default=1)
+    ap.add_argument("--e2e-steps", type=int, default=3)
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-generate", action="store_true")
     ap.add_argument("--no-backward", action="store_true")
+    ap.add_argument("--no-configs", action="store_true")
     ap.add_argument("--profile-case", choices=["ska_prefill", "gla_prefill", "ska_decode", "gla_decode",
                                                "ska_decode_paged", "ska_decode_fp8", "gla_backward",
                                                "ska_backward"],

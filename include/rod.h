@@ -78,6 +78,17 @@ ROD_API int rod_abi_version(void);
  * counts each kernel it enqueues; host-side counter, no synchronisation). */
 ROD_API uint64_t rod_launch_count(void);
 
+/* Diagnostics for the failure-detection path (no counterpart in the source pages). Arms the
+ * NEXT rod_gla_prefill call that runs the tensor-core kernels (bf16, dk = dv = 128, chunk 64):
+ * its TMA producers issue no copies and every bounded device wait in its kernels gives up
+ * after `probes` probes instead of the default 2^22, so the call's consumers find their first
+ * input barrier never completes, abort, drain and return. rod_check() then reports
+ * ROD_ERR_TIMEOUT; that call's outputs and final state are unspecified, and later calls run
+ * normally (the arming is consumed by the one call). Nothing faults, traps or hangs.
+ * probes = 0 disarms. Always returns ROD_OK. Not thread-safe against concurrent prefill calls
+ * from other host threads (they may consume the arming). */
+ROD_API int rod_test_expire_waits(uint32_t probes);
+
 /* ---- gated linear recurrence: chunkwise prefill ------------------------------------------ */
 /*
  * Bytes of device workspace rod_gla_prefill needs for these sizes (0 if none). The caller
@@ -97,7 +108,11 @@ ROD_API size_t rod_gla_prefill_workspace_size(int B, int H, int T, int dk, int d
  *   o     [B,H,T,dv]   dtype          outputs o_t = q_t S_t (no scale, no normaliser)
  *   chunk              tokens per chunk: a multiple of 16 in [16, 128]. It changes rounding
  *                      only, never the mathematical result; a T that is not a multiple of
- *                      chunk is handled by masking the tail chunk.
+ *                      chunk is handled by masking the tail chunk. Only dtype ROD_BF16 with
+ *                      dk = dv = 128 and chunk = 64 runs the chunkwise tensor-core kernels;
+ *                      every other combination (all of ROD_FP32, other chunk sizes or head
+ *                      dims) runs a sequential-in-time CUDA-core kernel with exact fp32 FMAs,
+ *                      one thread per state column: correct, but far slower at long T.
  *   workspace, ws_bytes  at least rod_gla_prefill_workspace_size(...) bytes (may be NULL
  *                      when that size is 0).
  * Calling it twice, on tokens [0,T1) and then [T1,T) with the returned state, equals one
@@ -196,7 +211,11 @@ ROD_API int rod_swska_prefill(const void* q, const void* k, const void* v, void*
  *   q [B,H,T,dk], k [B,T,dk], v [B,H,T,dv], dO [B,H,T,dv]: dtype;  outputs dq, dk, dv in the
  *   layouts of q, k, v and dtype;  workspace of rod_swska_backward_workspace_size bytes
  *   (the row log-sum-exp and D_t, recomputed here from the inputs).
- * Runs on CUDA cores with fp32 dot products (one warp per query row, then one per key).
+ * Two routes, chosen by dtype and shape: ROD_BF16 with dk = dv = 128 and T >= 128 runs four
+ * tcgen05 tensor-core launches (the forward in a statistics mode for the row log-sum-exp and
+ * D_t, then query tiles for dq, key tiles for dv and per-group dk partials, and a fixed-order
+ * reduction of dk, so the result is deterministic); every other case runs on CUDA cores with
+ * fp32 dot products (one warp per query row, then one per key).
  * Errors: ROD_ERR_NULL, ROD_ERR_SHAPE (window < 1, dims unsupported, H > 64), ROD_ERR_ALIGN,
  * ROD_ERR_DTYPE, ROD_ERR_WORKSPACE, ROD_ERR_CUDA. T = 0 or B*H = 0 is a no-op.
  */

@@ -40,4 +40,5 @@ from ._binding import (  # noqa: F401
     swska_decode_fp8,
     swska_decode_paged,
     swska_prefill,
+    test_expire_waits,
 )

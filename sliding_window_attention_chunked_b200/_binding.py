@@ -53,6 +53,8 @@ def load_library() -> ctypes.CDLL:
     lib.rod_abi_version.restype = i
     lib.rod_launch_count.argtypes = []
     lib.rod_launch_count.restype = ctypes.c_uint64
+    lib.rod_test_expire_waits.argtypes = [ctypes.c_uint32]
+    lib.rod_test_expire_waits.restype = i
     lib.rod_gla_prefill_workspace_size.argtypes = [i, i, i, i, i, i, i]
     lib.rod_gla_prefill_workspace_size.restype = sz
     lib.rod_gla_prefill.argtypes = [vp, vp, vp, vp, vp, vp, i, i, i, i, i, i, i, vp, sz, vp]
@@ -129,6 +131,13 @@ def abi_version() -> int:
 def launch_count() -> int:
     """Kernels launched by librod.so in this process so far."""
     return int(load_library().rod_launch_count())
+
+
+def test_expire_waits(probes: int) -> None:
+    """Diagnostics (rod_test_expire_waits): arm the next tensor-core recurrence prefill call so
+    that its producers issue no copies and its bounded waits give up after `probes` probes;
+    check() then raises RodError with status ROD_ERR_TIMEOUT (-7). 0 disarms."""
+    _raise_on("rod_test_expire_waits", load_library().rod_test_expire_waits(int(probes)))
 
 
 def check(stream=None) -> None:

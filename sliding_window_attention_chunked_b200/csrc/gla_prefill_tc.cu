@@ -47,6 +47,8 @@
 #include <cuda.h>
 #include <math.h>
 
+#include <atomic>
+
 #include "common.cuh"
 #include "kernels.h"
 #include "tc.cuh"
@@ -103,6 +105,8 @@ struct GlaArgs {
     const __nv_bfloat16 *q, *k, *v;  // the inputs again, for L2 prefetches ahead of TMA
     const float* g;
     int T, L_seg, n_seg;
+    uint32_t wait_limit;    // probes before a wait gives up (kWaitLimit; smaller only in tests)
+    int copies_off;         // nonzero only in the wait-expiry test: the producer issues no copies
 };
 
 // byte offset of the 16-byte chunk holding columns [col, col + 8) of row `row` in a K-major
@@ -133,12 +137,13 @@ __device__ __forceinline__ uint64_t mul2(uint64_t a, uint64_t b) {
     return d;
 }
 
-__device__ __forceinline__ bool wait_bar(uint64_t* bar, uint32_t parity, volatile int* abort_flag) {
+__device__ __forceinline__ bool wait_bar(uint64_t* bar, uint32_t parity, volatile int* abort_flag,
+                                         uint32_t limit) {
     for (uint32_t i = 1;; ++i) {
         if (mbar_try_wait(bar, parity)) return true;
         if ((i & 255u) == 0) {
             if (*abort_flag) return false;
-            if (i >= kWaitLimit) {
+            if (i >= limit) {
                 *abort_flag = 1;
                 atomicExch(&g_gla_tc_timeout, 1u);
                 return false;
@@ -244,6 +249,7 @@ gla_chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
     __syncthreads();
     tc::fence_after_sync();
     const uint32_t tmem = *tmem_holder;
+    const uint32_t wlim = args.wait_limit;
     bool ok = true;
 
     if (warp >= 8) {
@@ -253,9 +259,9 @@ gla_chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
         // ------------------------------- TMA producer -------------------------------
         if (lane == 0) {
             int n = 0;
-            for (; n < n_ch; ++n) {
+            for (; n < n_ch && !args.copies_off; ++n) {
                 const int st = n & 1, use = n >> 1;
-                if (use > 0 && !wait_bar(&empty[st], (uint32_t)((use - 1) & 1), abort_flag)) break;
+                if (use > 0 && !wait_bar(&empty[st], (uint32_t)((use - 1) & 1), abort_flag, wlim)) break;
                 unsigned char* base = smem + st * STAGE_BYTES;
                 const int y = t_begin + n * C;
                 mbar_arrive_expect_tx(&full[st], kStageTx);
@@ -301,7 +307,7 @@ gla_chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
             unsigned char* base = smem + st * STAGE_BYTES;
             float* gsm = reinterpret_cast<float*>(base + ST_G);
             const int nvalid = min(C, t_end - (t_begin + n * C));
-            if (!grp_all(1, wait_bar(&full[st], (uint32_t)((n >> 1) & 1), abort_flag))) { ok = false; break; }
+            if (!grp_all(1, wait_bar(&full[st], (uint32_t)((n >> 1) & 1), abort_flag, wlim))) { ok = false; break; }
 
             auto load_gates = [&](int i, float* g8) {  // gates of row r0+i, my 8 channels
                 const float4* p = reinterpret_cast<const float4*>(gsm + (r0 + i) * D + c0);
@@ -555,7 +561,7 @@ gla_chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
         for (int n = 0; n < n_ch; ++n) {
             const int st = n & 1;
             unsigned char* base = smem + st * STAGE_BYTES;
-            if (!grp_all(2, wait_bar(&ops[st], (uint32_t)((n >> 1) & 1), abort_flag))) { ok = false; break; }
+            if (!grp_all(2, wait_bar(&ops[st], (uint32_t)((n >> 1) & 1), abort_flag, wlim))) { ok = false; break; }
             tc::fence_after_sync();
             const int fl = flag[st];
             const bool exact = (fl & kFlagExact) != 0, rmw = (fl & kFlagRescale) != 0;
@@ -566,7 +572,7 @@ gla_chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                 // exact route, was stored into TMEM by warpgroup 0 before the operands signal)
                 if (!exact) {
                     const uint32_t ph = st == 0 ? nA0 : nA1;
-                    if (!grp_all(2, wait_bar(&barA[st], ph & 1, abort_flag))) { ok = false; break; }
+                    if (!grp_all(2, wait_bar(&barA[st], ph & 1, abort_flag, wlim))) { ok = false; break; }
                     if (st == 0) ++nA0; else ++nA1;
                     tc::fence_after_sync();
                 }
@@ -590,7 +596,7 @@ gla_chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
             // earlier phase known complete (a parity wait must not be two phases ahead)
             const bool need_prev = n > 0 && (MODE == PASS_C || rmw || n == n_ch - 1);
             if (need_prev) {
-                if (!grp_all(2, wait_bar(barO, (uint32_t)((n - 1) & 1), abort_flag))) { ok = false; break; }
+                if (!grp_all(2, wait_bar(barO, (uint32_t)((n - 1) & 1), abort_flag, wlim))) { ok = false; break; }
                 tc::fence_after_sync();
                 if (MODE == PASS_C) epilogue(n - 1);
             }
@@ -665,7 +671,7 @@ gla_chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
         }
 
         // ---- tail: last chunk's outputs and the segment's state S = diag(D) R
-        if (ok && n_ch > 0 && grp_all(2, wait_bar(barO, (uint32_t)((n_ch - 1) & 1), abort_flag))) {
+        if (ok && n_ch > 0 && grp_all(2, wait_bar(barO, (uint32_t)((n_ch - 1) & 1), abort_flag, wlim))) {
             tc::fence_after_sync();
             if (MODE == PASS_C) epilogue(n_ch - 1);
             float* dst = nullptr;
@@ -732,6 +738,10 @@ struct Plan {
     int L_seg, n_seg;
 };
 
+// one-shot test arming (rod_test_expire_waits): the next launch runs with this wait limit and
+// with its producers issuing no copies, so that every consumer's first wait gives up
+std::atomic<uint32_t> g_expire_probes{0};
+
 // Segments per (b, h): one wave of the output pass (one CTA per SM), i.e. floor(SMs / (B H)),
 // at least 1. Measured on B200 (recurrence layer, d = 128): at B4 H16 T4096 two segments per
 // head take 240 us against 271 us for a single segment (the sequential schedule) and 284 us for
@@ -783,6 +793,9 @@ cudaError_t gla_prefill_tc_launch(const void* q, const void* k, const void* v, c
         if (e != cudaSuccess) return e;
     }
     GlaArgs a{};
+    const uint32_t expire = g_expire_probes.exchange(0u);
+    a.wait_limit = expire ? expire : kWaitLimit;
+    a.copies_off = expire ? 1 : 0;
     a.q = static_cast<const __nv_bfloat16*>(q);
     a.k = static_cast<const __nv_bfloat16*>(k);
     a.v = static_cast<const __nv_bfloat16*>(v);
@@ -815,6 +828,8 @@ cudaError_t gla_prefill_tc_launch(const void* q, const void* k, const void* v, c
     note_launches(1);
     return cudaGetLastError();
 }
+
+void gla_prefill_tc_arm_wait_expiry(uint32_t probes) { g_expire_probes.store(probes); }
 
 unsigned gla_prefill_tc_take_timeout_flag() {
     unsigned v = 0, zero = 0;

@@ -30,6 +30,9 @@ cudaError_t gla_prefill_tc_launch(const void* q, const void* k, const void* v, c
                                   float* state, void* o, int B, int H, int T, void* workspace,
                                   cudaStream_t stream);
 unsigned gla_prefill_tc_take_timeout_flag();
+// test only: the next gla_prefill_tc_launch runs with `probes` as its wait limit and issues no
+// copies, so that its bounded waits expire (probes = 0 disarms)
+void gla_prefill_tc_arm_wait_expiry(uint32_t probes);
 
 // SW-SKA prefill on CUDA cores (fp32 FMA, online softmax)
 cudaError_t swska_prefill_simt_launch(const void* q, const void* k, const void* v, void* o,

@@ -51,6 +51,11 @@ int rod_last_cuda_error(void) { return t_last_cuda_error; }
 
 int rod_abi_version(void) { return 1; }
 
+int rod_test_expire_waits(uint32_t probes) {
+    rod::gla_prefill_tc_arm_wait_expiry(probes);
+    return ROD_OK;
+}
+
 uint64_t rod_launch_count(void) { return rod::g_launches.load(std::memory_order_relaxed); }
 
 int rod_check(void* stream) {

@@ -55,6 +55,12 @@ def test_status_strings_and_version(lib):
     assert lib.rod_abi_version() == 1
 
 
+def test_wait_expiry_arming_is_host_only(lib):
+    # arming and disarming the wait-expiry diagnostic touches no device state
+    assert lib.rod_test_expire_waits(4096) == OK
+    assert lib.rod_test_expire_waits(0) == OK
+
+
 P = ctypes.c_void_p(0x10000)   # aligned, never dereferenced (every call below fails first)
 MIS = ctypes.c_void_p(0x10008)  # 8-byte aligned only
 

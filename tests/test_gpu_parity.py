@@ -64,7 +64,9 @@ def test_gla_prefill_bf16_short(T):
 
 
 @pytest.mark.parametrize("chunk", [16, 32, 128])
-def test_gla_prefill_bf16_chunk_sizes(chunk):
+def test_gla_prefill_bf16_chunk_sizes_cuda_core_kernel(chunk):
+    """Chunk sizes other than 64 run the sequential CUDA-core kernel (only bf16, d = 128,
+    chunk 64 takes the tensor-core path): the chunk size must not change the result."""
     _gla_check(1, 2, 300, 128, 128, chunk, "bf16", "l2", seed=chunk)
 
 
@@ -98,6 +100,33 @@ def test_gla_prefill_mixed_strong_and_mild_decay():
 def test_gla_prefill_many_segments(B, H, T):
     """Small B*H spreads the sequence over many segments (segment pass + state scan)."""
     _gla_check(B, H, T, 128, 128, 64, "bf16", "l2", seed=T, state0_scale=0.2)
+
+
+@pytest.mark.parametrize("gates", ["one", "one_minus_2^-10", "sigmoid(N(8,1))"])
+def test_gla_prefill_long_sequence_gates_near_one(gates):
+    """Gates at or near 1 over a long sequence (g = 1 is linear attention, SALA blog §2.2): the
+    state sums thousands of k^T v terms and grows with T, the regime where the readout's bf16
+    copy of the state would be most likely to lose accuracy. B1 H2 T16384 cuts each head into
+    many segments, so the segment pass, the scan and the output pass all run. v is scaled by
+    sqrt(128 / T) so that outputs and states stay O(1) and the absolute bound keeps its
+    meaning; relative accuracy, which is what the long state tests, does not depend on it."""
+    B, H, T, d = 1, 2, 16384, 128
+    q, k, v, g = wl.gla_inputs(B, H, T, d, d, dist="l2", seed=61)
+    v = (v.float() * (128.0 / T) ** 0.5).to(v.dtype)
+    if gates == "one":
+        g = torch.ones_like(g)
+    elif gates == "one_minus_2^-10":
+        g = torch.full_like(g, 1.0 - 2.0 ** -10)
+    else:
+        gen = torch.Generator().manual_seed(62)
+        g = torch.sigmoid(torch.randn(g.shape, generator=gen) + 8.0)
+    assert rod.gla_prefill_workspace_size(B, H, T, d, d, 64) > 0  # several segments
+    o_ref, S_ref = oracle.gla_prefill(q, k, v, g)
+    S = torch.zeros(B, H, d, d, device=DEV)
+    o = rod.gla_prefill(q.to(DEV), k.to(DEV), v.to(DEV), g.to(DEV), S, chunk=64)
+    rod.check()
+    compare(o, o_ref, "bf16", f"o ({gates})")
+    compare(S, S_ref, "bf16", f"state ({gates})")
 
 
 def test_gla_prefill_deterministic():
