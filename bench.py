@@ -449,6 +449,10 @@ def run_gpu(args):
               f"{n_ska_sets} SW-SKA sets (4.6 GB of cache each)",
         "value": round(N * world / (dec_ms / 1e3), 1), "unit": "tokens/s",
         "ms_per_step": round(dec_ms, 4),
+        # the step as a whole: a kernel's dirty lines can still sit in L2 when it ends and be
+        # written back under the next kernel, so the pair's bytes over the pair's time is the
+        # fraction free of that shift
+        "step_frac_hbm": round((gla_dec_bytes + ska_dec_bytes) / (dec_ms / 1e3) / 1e9 / hbm, 4),
         "kernels": {
             "rod_gla_decode_step": {"bound": "hbm", "avg_launch_ms": round(gla_dec_ms, 4),
                                     "algorithmic_bytes": gla_dec_bytes,

@@ -130,6 +130,29 @@ __device__ __forceinline__ void mma_ts_lh_warp(uint32_t d_tmem, uint32_t a_tmem,
         "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], db, %4, p;\n\t}"
         ::"r"(d_tmem), "r"(a_tmem), "r"(b_lo), "r"(b_hi), "r"(idesc), "r"(accumulate) : "memory");
 }
+// tf32 MMA with A read from tensor memory (32-bit elements, row i of A in lane i, one K element
+// per column, so a K step of 8 moves the A address by 8 columns): every lane of the issuing warp
+// executes it with the same operands and one elected lane issues. The accumulator of an earlier
+// fp32 MMA can serve directly as A: the tensor core reads the top 19 bits of each element.
+__device__ __forceinline__ void mma_tf32_ts_lh_warp(uint32_t d_tmem, uint32_t a_tmem, uint32_t b_lo,
+                                                    uint32_t b_hi, uint32_t idesc, uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p, e;\n\t.reg .b64 db;\n\tsetp.ne.b32 p, %5, 0;\n\t"
+        "mov.b64 db, {%2, %3};\n\t"
+        "elect.sync _|e, 0xffffffff;\n\t"
+        "@e tcgen05.mma.cta_group::1.kind::tf32 [%0], [%1], db, %4, p;\n\t}"
+        ::"r"(d_tmem), "r"(a_tmem), "r"(b_lo), "r"(b_hi), "r"(idesc), "r"(accumulate) : "memory");
+}
+// Instruction descriptor for kind::tf32 (A and B tf32, fp32 accumulator).
+__host__ __device__ constexpr uint32_t idesc_tf32_f32(int M, int N, int a_mn, int b_mn) {
+    return (1u << 4)                      // D format: f32
+         | (2u << 7)                      // A format: tf32
+         | (2u << 10)                     // B format: tf32
+         | ((uint32_t)a_mn << 15)
+         | ((uint32_t)b_mn << 16)
+         | ((uint32_t)(N >> 3) << 17)
+         | ((uint32_t)(M >> 4) << 24);
+}
 __device__ __forceinline__ uint32_t desc_lo(uint64_t d) { return (uint32_t)d; }
 __device__ __forceinline__ uint32_t desc_hi(uint64_t d) { return (uint32_t)(d >> 32); }
 
@@ -194,6 +217,22 @@ __device__ __forceinline__ void tma_load_3d(void* dst_smem, const CUtensorMap* m
         ::"r"(smem_u32(dst_smem)), "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(z),
           "r"(smem_u32(bar))
         : "memory");
+}
+// tiled shared -> global store of one box (rows outside the tensor are not written); the
+// source must stay untouched until bulk_wait_read() of the issuing thread returns
+__device__ __forceinline__ void tma_store_3d(const CUtensorMap* map, const void* src_smem, int x, int y, int z) {
+    asm volatile(
+        "cp.async.bulk.tensor.3d.global.shared::cta.tile.bulk_group [%0, {%2, %3, %4}], [%1];"
+        ::"l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(src_smem)), "r"(x), "r"(y), "r"(z)
+        : "memory");
+}
+__device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+// the issuing thread's committed bulk stores have finished reading shared memory
+__device__ __forceinline__ void bulk_wait_read() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
+// the issuing thread's committed bulk stores are complete
+__device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
+__device__ __forceinline__ void fence_proxy_async() {
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
 // bring `bytes` of global memory into L2 ahead of use (16-byte aligned address and size)
 __device__ __forceinline__ void prefetch_l2(const void* gmem, uint32_t bytes) {
