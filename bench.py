@@ -930,6 +930,8 @@ def run_profile_case(args):
     d = wl.WORKLOADS[WORKLOAD].dims
     B, H, T, dk, dv, W, C = d["B"], d["H"], d["T"], d["dk"], d["dv"], d["window"], d["chunk"]
     case = args.profile_case
+    if args.profile_t:
+        T = args.profile_t
     if case in ("ska_prefill", "gla_prefill"):
         layer = 1 if case == "ska_prefill" else 0
         ins = wl.stack_layer_inputs(layer, B, H, T, dk, dv, device=dev)
@@ -1006,6 +1008,8 @@ def main():
                                                "ska_backward"],
                     help="run one kernel family alone (for ncu captures) and exit")
     ap.add_argument("--profile-n", type=int, default=128, help="sequences for the decode cases")
+    ap.add_argument("--profile-t", type=int, default=0,
+                    help="tokens per sequence for the prefill cases (default: the stack's 131072)")
     args = ap.parse_args()
     args.warmup = max(3, args.warmup)  # timing rule: at least 3 untimed warm-up steps
     if args.profile_case:

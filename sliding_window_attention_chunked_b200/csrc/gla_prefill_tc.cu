@@ -29,10 +29,10 @@
 // tensor cores would have put them; q.G becomes q.2^L and a/G becomes 2^(L_last - L).
 //
 // Parallelism over the sequence: the T tokens are cut into segments of L_seg tokens. Pass A
-// (per segment but the last) computes the segment's state contribution U and decay a_seg from
-// k, v, g; a scan kernel chains S_in(m+1) = diag(a_seg,m) S_in(m) + U_m per (b, h); pass C
-// recomputes every segment from its S_in and writes o (and the final state). One segment means
-// pass C alone.
+// (per segment but the last, each cut into `sub` pieces when that fills more SMs) computes each
+// piece's state contribution U and decay a from k, v, g; a scan kernel chains
+// S(j+1) = diag(a_j) S(j) + U_j per (b, h) over the pieces; pass C recomputes every segment from
+// its S_in and writes o (and the final state). One segment means pass C alone.
 //
 // CTA: 512 threads = 4 warpgroups, setmaxnreg 56 / 152 / 152 / 152, a pipeline over the chunks
 // of a segment through two 96 KB stages:
@@ -97,7 +97,7 @@ constexpr float kFastMin = 8.673617e-19f;          // 2^-60: chunk decay for q~ 
 constexpr float kRescaleMin = 5.421011e-20f;       // 2^-64: smallest running decay D
 constexpr int kFlagExact = 1, kFlagRescale = 2;
 constexpr float kLog2Floor = -126.0f;              // log2 of the smallest gate used
-constexpr int kPrefetchChunks = 3;                 // L2 prefetch distance in chunks
+constexpr int kPrefetchChunks = 1;                 // L2 prefetch distance in chunks (measured best of 0-4)
 
 // TMEM columns
 constexpr uint32_t TM_R = 0, TM_O = 128, TM_A = 256;
@@ -108,11 +108,13 @@ struct GlaArgs {
     const float* s_in;      // PASS_C: [BH][s_in_slots][D][D] incoming states (slot = segment)
     int s_in_slots;         // 1: every (b,h) reads slot 0 of s_in (initial state, single segment)
     float* state_out;       // PASS_C: [BH][D][D] final state, written by the last segment
-    float* u_out;           // PASS_A: [BH][n_seg][D][D] (segment m writes slot m+1)
-    float* a_out;           // PASS_A: [BH][n_seg][D]    (segment m writes slot m)
+    float* u_out;           // PASS_A: [BH][n_slots][D][D] (sub-segment j writes slot j+1)
+    float* a_out;           // PASS_A: [BH][n_slots][D]    (sub-segment j writes slot j)
     const __nv_bfloat16 *q, *k, *v;  // the inputs again, for L2 prefetches ahead of TMA
     const float* g;
-    int T, L_seg, n_seg;
+    int T, L_seg, n_seg;    // tokens per CTA (a pass A CTA covers a sub-segment); CTAs per (b,h)
+    int n_slots;            // workspace slots per (b,h): sub-segments of pass A + 1
+    int sub;                // pass C: segment m starts at sub-segment boundary m * sub
     uint32_t wait_limit;    // probes before a wait gives up (kWaitLimit; smaller only in tests)
     int copies_off;         // nonzero only in the wait-expiry test: the producer issues no copies
 };
@@ -592,7 +594,7 @@ gla_chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
             }
         }
         if (MODE == PASS_A && ok && qr == 0)
-            *reinterpret_cast<uint64_t*>(args.a_out + ((int64_t)bh * args.n_seg + seg) * D + c0) = aseg;
+            *reinterpret_cast<uint64_t*>(args.a_out + ((int64_t)bh * args.n_slots + seg) * D + c0) = aseg;
     } else {
         asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kStRegs));
         // ------------------- state warps: P, output rows, initial / final state -------------------
@@ -642,7 +644,7 @@ gla_chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
 
             // R^T <- S_in^T with D = 1
             {
-                const int slot = args.s_in_slots == 1 ? 0 : seg;
+                const int slot = args.s_in_slots == 1 ? 0 : seg * args.sub;
                 const float* src = args.s_in + ((int64_t)bh * args.s_in_slots + slot) * D * D;
 #pragma unroll
                 for (int cb = 0; cb < D; cb += 32) {
@@ -688,7 +690,7 @@ gla_chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
         } else {
             if (all2(wait_bar(fin, 0, abort_flag, wlim))) {
                 tc::fence_after_sync();
-                store_state(args.u_out + ((int64_t)bh * args.n_seg + seg + 1) * D * D,
+                store_state(args.u_out + ((int64_t)bh * args.n_slots + seg + 1) * D * D,
                             abuf + ((n_ch - 1) & 1) * 3 * D + 2 * D);
             }
         }
@@ -729,7 +731,9 @@ gla_segment_scan_kernel(const float* __restrict__ state, float* __restrict__ s_s
 }
 
 struct Plan {
-    int L_seg, n_seg;
+    int L_seg, n_seg;   // output pass: segments of L_seg tokens, n_seg per (b, h)
+    int sub;            // segment pass: each of the first n_seg - 1 segments in `sub` pieces
+    int slots() const { return n_seg > 1 ? (n_seg - 1) * sub + 1 : 0; }
 };
 
 // one-shot test arming (rod_test_expire_waits): the next launch runs with this wait limit and
@@ -738,7 +742,10 @@ std::atomic<uint32_t> g_expire_probes{0};
 
 // Segments per (b, h): one wave of the output pass (one CTA per SM), i.e. floor(SMs / (B H)),
 // at least 1. Fewer segments mean fewer k, v, g bytes read twice (segment pass and output pass);
-// more than one wave adds segment-pass traffic and a tail.
+// more than one wave adds segment-pass traffic and a tail. The segment pass has one segment
+// fewer per (b, h), so with few segments it would leave SMs idle (B4 H16: 64 CTAs): there each
+// segment is split into `sub` equal pieces of whole chunks, as many as still fit one wave, and
+// the scan chains the pieces.
 Plan plan(int B, int H, int T) {
     const int64_t BH = (int64_t)B * H;
     const int chunks = (T + C - 1) / C;
@@ -755,6 +762,11 @@ Plan plan(int B, int H, int T) {
     Plan p;
     p.L_seg = per * C;
     p.n_seg = (T + p.L_seg - 1) / p.L_seg;
+    p.sub = 1;
+    if (p.n_seg > 1) {
+        for (int k = per; k > 1; --k)  // the largest divisor of the segment's chunk count that fits
+            if (per % k == 0 && BH * (p.n_seg - 1) * k <= sms) { p.sub = k; break; }
+    }
     return p;
 }
 
@@ -765,7 +777,7 @@ bool gla_prefill_tc_supported(int dk, int dv, int chunk) { return dk == D && dv 
 size_t gla_prefill_tc_workspace_size(int B, int H, int T) {
     const Plan p = plan(B, H, T);
     if (p.n_seg <= 1) return 0;
-    return (size_t)B * H * p.n_seg * ((size_t)D * D + D) * sizeof(float);
+    return (size_t)B * H * p.slots() * ((size_t)D * D + D) * sizeof(float);
 }
 
 cudaError_t gla_prefill_tc_launch(const void* q, const void* k, const void* v, const float* g,
@@ -794,27 +806,31 @@ cudaError_t gla_prefill_tc_launch(const void* q, const void* k, const void* v, c
     a.v = static_cast<const __nv_bfloat16*>(v);
     a.g = g;
     a.T = T;
-    a.L_seg = p.L_seg;
     a.n_seg = p.n_seg;
+    a.sub = p.sub;
+    a.n_slots = p.slots();
     a.state_out = state;
     if (p.n_seg == 1) {
         a.s_in = state;
         a.s_in_slots = 1;
     } else {
         float* slots = static_cast<float*>(workspace);
-        float* aseg = slots + (size_t)BH * p.n_seg * D * D;
+        float* aseg = slots + (size_t)BH * a.n_slots * D * D;
         a.u_out = slots;
         a.a_out = aseg;
-        gla_chunk_kernel<PASS_A><<<dim3((unsigned)(p.n_seg - 1), (unsigned)BH), NTHREADS, SMEM_BYTES, stream>>>(
+        const int n_sub = (p.n_seg - 1) * p.sub;
+        a.L_seg = p.L_seg / p.sub;  // a segment-pass CTA covers one piece
+        gla_chunk_kernel<PASS_A><<<dim3((unsigned)n_sub, (unsigned)BH), NTHREADS, SMEM_BYTES, stream>>>(
             mq, mk, mv, mg, mo, a);
         if ((e = cudaGetLastError()) != cudaSuccess) return e;
         gla_segment_scan_kernel<<<dim3((D * D / 4 + 255) / 256, (unsigned)BH), 256, 0, stream>>>(
-            state, slots, aseg, p.n_seg);
+            state, slots, aseg, a.n_slots);
         if ((e = cudaGetLastError()) != cudaSuccess) return e;
         note_launches(2);
         a.s_in = slots;
-        a.s_in_slots = p.n_seg;
+        a.s_in_slots = a.n_slots;
     }
+    a.L_seg = p.L_seg;
     gla_chunk_kernel<PASS_C><<<dim3((unsigned)p.n_seg, (unsigned)BH), NTHREADS, SMEM_BYTES, stream>>>(
         mq, mk, mv, mg, mo, a);
     note_launches(1);

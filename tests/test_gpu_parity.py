@@ -96,9 +96,10 @@ def test_gla_prefill_mixed_strong_and_mild_decay():
     compare(S, S_ref, "bf16", "state")
 
 
-@pytest.mark.parametrize("B,H,T", [(1, 2, 5000), (1, 1, 64 * 40 + 3), (3, 5, 777)])
+@pytest.mark.parametrize("B,H,T", [(1, 2, 5000), (1, 1, 64 * 40 + 3), (3, 5, 777), (5, 14, 700)])
 def test_gla_prefill_many_segments(B, H, T):
-    """Small B*H spreads the sequence over many segments (segment pass + state scan)."""
+    """Small B*H spreads the sequence over many segments (segment pass + state scan); at B5 H14
+    the segment pass cuts each segment into two pieces and the scan chains the pieces."""
     _gla_check(B, H, T, 128, 128, 64, "bf16", "l2", seed=T, state0_scale=0.2)
 
 
