@@ -163,8 +163,13 @@ ROD_API int rod_gla_prefill_noalloc(const void* q, const void* k, const void* v,
  *   dstate_final [B,H,dk,dv] fp32, or NULL for no loss on the final state;
  *   outputs dq, dk [B,H,T,dk] and dv [B,H,T,dv] in dtype; dg [B,H,T,dk] and dstate0
  *   [B,H,dk,dv] fp32; workspace of rod_gla_backward_workspace_size bytes (caller-owned).
- * Runs on CUDA cores with every product an fp32 FMA (three sweeps over the sequence per
- * (batch, head), states in registers).
+ * Two routes, chosen by dtype and shape. ROD_BF16 with dk = dv = 128 runs the chunkwise form
+ * on the tensor cores in three launches: each chunk's contributions to the state and to its
+ * gradient, a scan over chunks (incoming states forward, state gradients backward, both kept in
+ * bf16 in the workspace), and one CTA per chunk for dq, dk, dv, dg (bf16 operands, fp32
+ * accumulation). Every other case runs on CUDA cores with every product an fp32 FMA (three
+ * sweeps over the sequence per (batch, head), states in registers).
+ * rod_gla_backward_workspace_size does not depend on dtype: it returns enough for either route.
  * Errors: ROD_ERR_NULL, ROD_ERR_SHAPE, ROD_ERR_ALIGN, ROD_ERR_DTYPE, ROD_ERR_WORKSPACE,
  * ROD_ERR_CUDA. B*H = 0 is a no-op.
  */

@@ -89,6 +89,11 @@ struct GlaBackwardArgs {
     void* workspace;
 };
 size_t gla_backward_workspace_size(int B, int H, int T, int dk, int dv);
+// the chunkwise tensor-core backward (bf16, d_k = d_v = 128): contributions, scans, gradients
+bool gla_backward_tc_supported(int dk, int dv);
+size_t gla_backward_tc_workspace_size(int B, int H, int T);
+cudaError_t gla_backward_tc_launch(const GlaBackwardArgs& a, cudaStream_t stream);
+unsigned gla_backward_tc_take_timeout_flag();
 
 // backward of SW-SKA prefill: gradients of q, the shared k, and v (tensor cores for bf16 with
 // head dim 128 and T >= 128, CUDA cores otherwise)

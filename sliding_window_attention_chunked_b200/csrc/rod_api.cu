@@ -65,6 +65,7 @@ int rod_check(void* stream) {
                            rod::swska_decode_warp_take_timeout_flag() |
                            rod::swska_prefill_tc_take_timeout_flag() |
                            rod::gla_prefill_tc_take_timeout_flag() |
+                           rod::gla_backward_tc_take_timeout_flag() |
                            rod::swska_backward_tc_take_timeout_flag();
     if (flags) return ROD_ERR_TIMEOUT;
     return from_cuda(cudaGetLastError());
@@ -154,7 +155,14 @@ int rod_swska_decode(const void* q, const void* k_new, const void* v_new, void* 
 
 size_t rod_gla_backward_workspace_size(int B, int H, int T, int dk, int dv) {
     if (B < 0 || H < 0 || T < 0 || !dim_ok(dk) || !dim_ok(dv)) return 0;
-    return rod::gla_backward_workspace_size(B, H, T, dk, dv);
+    // the size does not depend on dtype: enough for either route (tensor cores for bf16 at
+    // d = 128, CUDA cores otherwise)
+    size_t need = rod::gla_backward_workspace_size(B, H, T, dk, dv);
+    if (rod::gla_backward_tc_supported(dk, dv)) {
+        const size_t tc = rod::gla_backward_tc_workspace_size(B, H, T);
+        if (tc > need) need = tc;
+    }
+    return need;
 }
 
 int rod_gla_backward(const void* q, const void* k, const void* v, const float* g, const float* state0,
@@ -178,11 +186,16 @@ int rod_gla_backward(const void* q, const void* k, const void* v, const float* g
     if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(g) || !aligned16(dO) ||
         !aligned16(dq) || !aligned16(dk) || !aligned16(dv) || !aligned16(dg))
         return ROD_ERR_ALIGN;
-    const size_t need = rod::gla_backward_workspace_size(B, H, T, dk_dim, dv_dim);
+    const bool tc = dtype == ROD_BF16 && rod::gla_backward_tc_supported(dk_dim, dv_dim);
+    const size_t need = tc ? rod::gla_backward_tc_workspace_size(B, H, T)
+                           : rod::gla_backward_workspace_size(B, H, T, dk_dim, dv_dim);
     if (!workspace || ws_bytes < need) return ROD_ERR_WORKSPACE;
     if (!aligned16(workspace)) return ROD_ERR_ALIGN;
     rod::GlaBackwardArgs a{q, k, v, g, state0, dO, dstate_final, dq, dk, dv, dg, dstate0,
                            B, H, T, dk_dim, dv_dim, workspace};
+    // bf16 with 128-wide heads runs the chunkwise tensor-core backward; fp32 (exact FMA) and
+    // the other head dims run the step-by-step CUDA-core sweeps
+    if (tc) return from_cuda(rod::gla_backward_tc_launch(a, s));
     return from_cuda(rod::gla_backward_launch(a, dtype == ROD_BF16, s));
 }
 
