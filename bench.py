@@ -594,6 +594,8 @@ def run_backward(rod, torch, wl, dev, H, d, W, seed_base, barrier, reduce_max, w
                            "frac": round(nbytes / (ms / 1e3) / 1e9 / hbm, 4),
                            "tflops_algorithmic": round(flop / (ms / 1e3) / 1e12, 2),
                            "peak_source": f"{peaks_src} hbm_gbs",
+                           "traffic": recorded_traffic("gla_backward_b4_t4096",
+                                                       ["gla_backward_tc.cu", "tc.cuh", "common.cuh"]),
                            "note": "chunkwise tensor-core backward (contributions, scans, gradients); "
                                    "its workspace traffic (per-chunk states and contributions) is "
                                    "about 3.7x the algorithmic bytes"}
