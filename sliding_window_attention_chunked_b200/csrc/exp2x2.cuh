@@ -46,14 +46,14 @@ __device__ __forceinline__ float2 ex2x2_sfu(float2 x) { return make_float2(tc::e
 
 // 2^x for both lanes on the FMA pipe, for x <= 0. Range reduction: adding 1.5 * 2^23 rounds x
 // to the nearest integer n (held in the low mantissa bits of the sum), and f = x - n lies in
-// [-1/2, 1/2]. 2^f is a cubic whose coefficients were fitted for these kernels (least squares on
-// the relative error over [-1/2, 1/2], reweighted toward equal ripple: at most 7.5e-5 relative,
-// below the bf16 rounding the probabilities get). 2^n is added into the exponent field. Inputs
-// are clamped at -125 so the exponent stays normal: masked (-inf) scores give 2^-125.
-constexpr float kExpC0 = 0.9999281764030457f;
+// [-1/2, 1/2]. 2^f is the minimax cubic for relative error on that interval (Lawson's algorithm,
+// fit_exp2_cubic.py beside this file prints these constants): at most 7.5e-5 relative, below the
+// bf16 rounding the probabilities get. 2^n is added into the exponent field. Inputs are clamped
+// at -125 so the exponent stays normal: masked (-inf) scores give 2^-125.
+constexpr float kExpC0 = 0.9999280571937561f;
 constexpr float kExpC1 = 0.6932609677314758f;
-constexpr float kExpC2 = 0.24260969460010529f;
-constexpr float kExpC3 = 0.055170830339193344f;
+constexpr float kExpC2 = 0.24261116981506348f;
+constexpr float kExpC3 = 0.0551716648042202f;
 __device__ __forceinline__ float2 ex2x2_fma(float2 x) {
     x = make_float2(fmaxf(x.x, -125.f), fmaxf(x.y, -125.f));
     const float2 shifter = make_float2(12582912.f, 12582912.f);
