@@ -943,6 +943,8 @@ def run_profile_case(args):
     case = args.profile_case
     if args.profile_t:
         T = args.profile_t
+    if args.profile_b:
+        B = args.profile_b
     if case in ("ska_prefill", "gla_prefill"):
         layer = 1 if case == "ska_prefill" else 0
         ins = wl.stack_layer_inputs(layer, B, H, T, dk, dv, device=dev)
@@ -1021,6 +1023,8 @@ def main():
     ap.add_argument("--profile-n", type=int, default=128, help="sequences for the decode cases")
     ap.add_argument("--profile-t", type=int, default=0,
                     help="tokens per sequence for the prefill cases (default: the stack's 131072)")
+    ap.add_argument("--profile-b", type=int, default=0,
+                    help="sequences for the prefill cases (default: the stack's 1)")
     args = ap.parse_args()
     args.warmup = max(3, args.warmup)  # timing rule: at least 3 untimed warm-up steps
     if args.profile_case:
