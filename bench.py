@@ -617,7 +617,18 @@ def run_backward(rod, torch, wl, dev, H, d, W, seed_base, barrier, reduce_max, w
                              "frac": round(flop / (ms / 1e3) / 1e12 / tc_peak, 4),
                              "peak_source": f"{peaks_src} bf16_tflops (burst: timed alone)",
                              "executed_flop_per_pair": 18 * d}
-    del q, k, v, dO
+    # the same gradients from the forward's saved output and log-sum-exp (what a training step
+    # keeps from its forward): the statistics pass becomes one read of o, dO and lse, and the
+    # kernels execute 14 d FLOP per pair
+    o, lse = rod.swska_prefill_lse(q, k, v, W)
+    ms_s = timed(lambda: rod.swska_backward_lse(q, k, v, o, lse, dO, W, workspace=ws), 10)
+    out["swska_backward_saved_statistics"] = {
+        "workload": f"B{B} H{H} T{T} d{d} window {W} bf16, from swska_prefill_lse's o and lse",
+        "ms": round(ms_s, 3), "tokens_per_s": round(B * T * world / (ms_s / 1e3), 1),
+        "bound": "tensor", "achieved": round(flop / (ms_s / 1e3) / 1e12, 1), "peak": tc_peak,
+        "unit": "TFLOP/s", "frac": round(flop / (ms_s / 1e3) / 1e12 / tc_peak, 4),
+        "peak_source": f"{peaks_src} bf16_tflops (burst: timed alone)", "executed_flop_per_pair": 14 * d}
+    del q, k, v, dO, o, lse
     torch.cuda.empty_cache()
     return out
 

@@ -207,6 +207,19 @@ ROD_API int rod_gla_decode_step(const void* q, const void* k, const void* v, con
 ROD_API int rod_swska_prefill(const void* q, const void* k, const void* v, void* o, int B, int H,
                       int T, int dk, int dv, int window, float scale, int dtype, void* stream);
 
+/* ---- SW-SKA: prefill that also keeps each row's log-sum-exp (for the backward) ------------- */
+/*
+ * rod_swska_prefill (same inputs, output, routes, window and scale rules) that also writes
+ *   lse[b,h,t] = log sum_{j in the window of t} exp(scale * q[b,h,t] . k[b,j])   (natural log),
+ * lse [B,H,T] fp32, 4-byte aligned, caller-owned. Together with o it is what
+ * rod_swska_backward_lse needs, so a training step need not run the forward twice (the
+ * statistics the backward uses are the scores' log-sum-exp and D_t = dO_t . o_t).
+ * Errors: those of rod_swska_prefill; ROD_ERR_NULL also for a null lse.
+ */
+ROD_API int rod_swska_prefill_lse(const void* q, const void* k, const void* v, void* o, float* lse,
+                                  int B, int H, int T, int dk, int dv, int window, float scale,
+                                  int dtype, void* stream);
+
 /* ---- SW-SKA: backward (training path) -------------------------------------------------------- */
 /*
  * Gradients of rod_swska_prefill for the loss gradient dO of every output row (same window
@@ -229,6 +242,22 @@ ROD_API int rod_swska_backward(const void* q, const void* k, const void* v, cons
                                void* dq, void* dk, void* dv, int B, int H, int T, int dk_dim,
                                int dv_dim, int window, float scale, int dtype, void* workspace,
                                size_t ws_bytes, void* stream);
+/*
+ * rod_swska_backward given the forward's output o [B,H,T,dv] (dtype) and lse [B,H,T] fp32 from
+ * rod_swska_prefill_lse with the same inputs, window and scale. On the tensor-core route the
+ * first launch then reads o, dO and lse (one warp per row: D_t = dO_t . o_t, and the log-sum-exp
+ * in the kernels' base-2 form) instead of running the forward again; the other launches, the
+ * workspace (rod_swska_backward_workspace_size) and the outputs are those of rod_swska_backward.
+ * D_t is taken from the stored (rounded) o, as the pages' plain definition reads it. The
+ * CUDA-core route recomputes its statistics and ignores o and lse. An o or lse that does not
+ * come from these inputs gives wrong gradients (it is not checked).
+ * Errors: those of rod_swska_backward; ROD_ERR_NULL also for a null o or lse.
+ */
+ROD_API int rod_swska_backward_lse(const void* q, const void* k, const void* v, const void* o,
+                                   const float* lse, const void* dO, void* dq, void* dk, void* dv,
+                                   int B, int H, int T, int dk_dim, int dv_dim, int window,
+                                   float scale, int dtype, void* workspace, size_t ws_bytes,
+                                   void* stream);
 
 /* ---- SW-SKA: decode with a ring-buffer window cache --------------------------------------- */
 /*

@@ -38,6 +38,8 @@ class OracleLib:
                                                i64, i64, i64, i64, ctypes.c_int]
         lib.rodref_swska_prefill.argtypes = [f32p, f32p, f32p, f64p, i64, i64, i64, i64, i64,
                                              i64, ctypes.c_double, i64p, i64, ctypes.c_int]
+        lib.rodref_swska_prefill_lse.argtypes = [f32p, f32p, f32p, f64p, f64p, i64, i64, i64, i64, i64,
+                                                 i64, ctypes.c_double, i64p, i64, ctypes.c_int]
         lib.rodref_swska_decode.argtypes = [f32p, f32p, f32p, f32p, f32p, i64p, f64p,
                                             i64, i64, i64, i64, i64, ctypes.c_double,
                                             ctypes.c_int]
@@ -60,7 +62,7 @@ class OracleLib:
         lib.rodref_swska_cache_fill_fp8.argtypes = [f32p, f32p, u8p, u8p, i64, i64, i64, i64, i64, i64,
                                                     ctypes.c_float, ctypes.c_float]
         for name in ("rodref_gla_backward", "rodref_swska_backward", "rodref_gla_prefill", "rodref_gla_decode_step",
-                     "rodref_swska_prefill",
+                     "rodref_swska_prefill", "rodref_swska_prefill_lse",
                      "rodref_swska_decode", "rodref_swska_cache_fill", "rodref_swska_decode_paged",
                      "rodref_e4m3_encode_array", "rodref_e4m3_decode_array", "rodref_swska_decode_fp8",
                      "rodref_swska_cache_fill_fp8"):
@@ -203,6 +205,29 @@ def swska_prefill(q, k, v, window, scale=None, rows=None, nthreads=None):
                                    nthreads or default_threads())
     _check(rc, "swska_prefill")
     return o
+
+
+def swska_prefill_lse(q, k, v, window, scale=None, rows=None, nthreads=None):
+    """swska_prefill and each output row's natural log-sum-exp of its scaled scores
+    (rodref_swska_prefill_lse). Returns (o, lse): [B,H,T,dv] and [B,H,T], or [len(rows), dv]
+    and [len(rows)] for the given flat rows. float64."""
+    q, k, v = _f32(q), _f32(k), _f32(v)
+    B, H, T, dk = q.shape
+    dv = v.shape[-1]
+    assert k.shape == (B, T, dk) and v.shape == (B, H, T, dv)
+    if scale is None or scale <= 0:
+        scale = 1.0 / np.sqrt(dk)
+    if rows is None:
+        o, lse = np.empty((B, H, T, dv)), np.empty((B, H, T))
+        rp, n = None, 0
+    else:
+        rows = np.ascontiguousarray(np.asarray(rows, dtype=np.int64))
+        o, lse = np.empty((rows.shape[0], dv)), np.empty(rows.shape[0])
+        rp, n = _pi64(rows), rows.shape[0]
+    rc = _L().rodref_swska_prefill_lse(_p32(q), _p32(k), _p32(v), _p64(o), _p64(lse), B, H, T, dk, dv,
+                                       int(window), float(scale), rp, n, nthreads or default_threads())
+    _check(rc, "swska_prefill_lse")
+    return o, lse
 
 
 def swska_decode(q, k_new, v_new, k_cache, v_cache, pos, window, scale=None, nthreads=None):

@@ -269,8 +269,10 @@ int rodref_gla_decode_step(const float* q, const float* k, const float* v, const
  *     s_j = scale * sum_c q[b,h,t,c] * k[b,j,c]
  *     p_j = exp(s_j - max_{j' in J_t} s_j')
  *     o[b,h,t,:] = sum_j p_j v[b,h,j,:] / sum_j p_j
+ * and the row's log-sum-exp  lse = log sum_j exp(s_j) = max_j s_j + log sum_j p_j  (natural log),
+ * the statistic a backward pass keeps from the forward.
  * ---------------------------------------------------------------------------------------- */
-static void softmax_row(const float* qrow, const float* kbase, const float* vbase,
+static double softmax_row(const float* qrow, const float* kbase, const float* vbase,
                         int64_t j0, int64_t j1, int64_t dk, int64_t dv, double scale,
                         double* s, double* out) {
     /* kbase row j is kbase + j*dk; vbase row j is vbase + j*dv; keys j0..j1 inclusive */
@@ -291,6 +293,7 @@ static void softmax_row(const float* qrow, const float* kbase, const float* vbas
         for (int64_t i = 0; i < dv; ++i) out[i] += p * (double)vr[i];
     }
     for (int64_t i = 0; i < dv; ++i) out[i] /= l;
+    return m + log(l);
 }
 
 typedef struct {
@@ -299,6 +302,7 @@ typedef struct {
     int64_t B, H, T, dk, dv, W;
     double scale;
     const int64_t* rows;
+    double* lse; /* optional: one per output row */
 } ska_args_t;
 
 static void ska_unit(const void* p, int64_t r) {
@@ -310,20 +314,25 @@ static void ska_unit(const void* p, int64_t r) {
     int64_t j0 = t - a->W + 1;
     if (j0 < 0) j0 = 0;
     double* s = (double*)malloc((size_t)(t - j0 + 1) * sizeof(double));
-    if (!s) { for (int64_t i = 0; i < a->dv; ++i) a->o[r * a->dv + i] = NAN; return; }
-    softmax_row(a->q + flat * a->dk, a->k + b * a->T * a->dk, a->v + bh * a->T * a->dv,
-                j0, t, a->dk, a->dv, a->scale, s, a->o + r * a->dv);
+    if (!s) {
+        for (int64_t i = 0; i < a->dv; ++i) a->o[r * a->dv + i] = NAN;
+        if (a->lse) a->lse[r] = NAN;
+        return;
+    }
+    const double lse = softmax_row(a->q + flat * a->dk, a->k + b * a->T * a->dk, a->v + bh * a->T * a->dv,
+                                   j0, t, a->dk, a->dv, a->scale, s, a->o + r * a->dv);
+    if (a->lse) a->lse[r] = lse;
     free(s);
 }
 
 /*
  * q: [B,H,T,dk]; k: [B,T,dk] (shared by the H heads); v: [B,H,T,dv].
- * rows == NULL: o is [B,H,T,dv] (every output row).
- * rows != NULL: o is [n_rows, dv]; row r is output row rows[r] = (b*H + h)*T + t.
+ * rows == NULL: o is [B,H,T,dv] (every output row), lse (if not NULL) [B,H,T].
+ * rows != NULL: o is [n_rows, dv] and lse [n_rows]; row r is output row rows[r] = (b*H + h)*T + t.
  */
-int rodref_swska_prefill(const float* q, const float* k, const float* v, double* o,
-                         int64_t B, int64_t H, int64_t T, int64_t dk, int64_t dv, int64_t W,
-                         double scale, const int64_t* rows, int64_t n_rows, int nthreads) {
+int rodref_swska_prefill_lse(const float* q, const float* k, const float* v, double* o, double* lse,
+                             int64_t B, int64_t H, int64_t T, int64_t dk, int64_t dv, int64_t W,
+                             double scale, const int64_t* rows, int64_t n_rows, int nthreads) {
     if (!q || !k || !v || !o) return RODREF_EINVAL;
     if (B < 0 || H < 0 || T < 0 || dk < 1 || dv < 1 || W < 1) return RODREF_EINVAL;
     const int64_t total = B * H * T;
@@ -333,8 +342,15 @@ int rodref_swska_prefill(const float* q, const float* k, const float* v, double*
     } else {
         n_rows = total;
     }
-    ska_args_t a = {q, k, v, o, B, H, T, dk, dv, W, scale, rows};
+    ska_args_t a = {q, k, v, o, B, H, T, dk, dv, W, scale, rows, lse};
     return run_units(ska_unit, &a, n_rows, nthreads);
+}
+
+/* the same without the log-sum-exp */
+int rodref_swska_prefill(const float* q, const float* k, const float* v, double* o,
+                         int64_t B, int64_t H, int64_t T, int64_t dk, int64_t dv, int64_t W,
+                         double scale, const int64_t* rows, int64_t n_rows, int nthreads) {
+    return rodref_swska_prefill_lse(q, k, v, o, NULL, B, H, T, dk, dv, W, scale, rows, n_rows, nthreads);
 }
 
 /*

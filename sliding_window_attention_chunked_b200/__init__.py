@@ -10,6 +10,8 @@ the calls raise.
     gla_backward(q, k, v, g, dO, state0, dstate_final)   gradients of the recurrence
     swska_prefill(q, k, v, window, scale=None)      sliding-window shared-key attention
     swska_backward(q, k, v, dO, window)             gradients of the attention
+    swska_prefill_lse(q, k, v, window)              the attention and each row's log-sum-exp
+    swska_backward_lse(q, k, v, o, lse, dO, window) gradients from the forward's o and lse
     swska_decode(q, k_new, v_new, k_cache, v_cache, pos, window)   ring-buffer decode
     swska_cache_fill(k, v, k_cache, v_cache, window)   prefill -> decode ring-buffer hand-off
     swska_decode_paged(q, k_new, v_new, k_pool, v_pool, block_table, page_size, pos, window)
@@ -34,11 +36,13 @@ from ._binding import (  # noqa: F401
     library_path,
     load_library,
     swska_backward,
+    swska_backward_lse,
     swska_cache_fill,
     swska_cache_fill_fp8,
     swska_decode,
     swska_decode_fp8,
     swska_decode_paged,
     swska_prefill,
+    swska_prefill_lse,
     test_expire_waits,
 )

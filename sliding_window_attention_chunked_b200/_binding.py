@@ -79,6 +79,10 @@ def load_library() -> ctypes.CDLL:
     lib.rod_swska_backward_workspace_size.restype = sz
     lib.rod_swska_backward.argtypes = [vp] * 7 + [i] * 6 + [f, i, vp, sz, vp]
     lib.rod_swska_backward.restype = i
+    lib.rod_swska_prefill_lse.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, i, i, f, i, vp]
+    lib.rod_swska_prefill_lse.restype = i
+    lib.rod_swska_backward_lse.argtypes = [vp] * 9 + [i] * 6 + [f, i, vp, sz, vp]
+    lib.rod_swska_backward_lse.restype = i
     lib.rod_swska_cache_fill.restype = i
     lib.rod_swska_decode_fp8.argtypes = [vp, vp, vp, vp, vp, vp, vp, i, i, i, i, i, f, f, f, vp]
     lib.rod_swska_decode_fp8.restype = i
@@ -243,6 +247,30 @@ def swska_prefill(q, k, v, window, scale=None, o=None, stream=None):
     return o
 
 
+def swska_prefill_lse(q, k, v, window, scale=None, o=None, lse=None, stream=None):
+    """swska_prefill that also returns each row's natural log-sum-exp of the scaled scores.
+    Returns (o [B,H,T,dv], lse [B,H,T] fp32), the pair swska_backward_lse takes."""
+    _need(q, "q", None, 4)
+    _need(k, "k", q.dtype, 3)
+    _need(v, "v", q.dtype, 4)
+    B, H, T, dk = q.shape
+    dv = v.shape[-1]
+    if tuple(k.shape) != (B, T, dk) or tuple(v.shape[:3]) != (B, H, T):
+        raise ValueError("k must be [B,T,dk] and v [B,H,T,dv]")
+    if o is None:
+        o = torch.empty((B, H, T, dv), dtype=q.dtype, device=q.device)
+    if lse is None:
+        lse = torch.empty((B, H, T), dtype=torch.float32, device=q.device)
+    _need(o, "o", q.dtype, 4)
+    _need(lse, "lse", torch.float32, 3)
+    if tuple(o.shape) != (B, H, T, dv) or tuple(lse.shape) != (B, H, T):
+        raise ValueError("o must be [B,H,T,dv] and lse [B,H,T]")
+    st = load_library().rod_swska_prefill_lse(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), B, H, T, dk, dv,
+                                              int(window), float(scale or 0.0), _dtype_code(q), _stream(stream))
+    _raise_on("rod_swska_prefill_lse", st)
+    return o, lse
+
+
 def swska_decode(q, k_new, v_new, k_cache, v_cache, pos, window, scale=None, o=None,
                  stream=None):
     """Ring-buffer decode. q [N,H,dk], k_new [N,dk], v_new [N,H,dv], k_cache [N,W,dk] and
@@ -367,6 +395,33 @@ def swska_backward(q, k, v, dO, window, scale=None, workspace=None, stream=None)
                                 B, H, T, dk, dv, int(window), float(scale or 0.0), _dtype_code(q),
                                 _ptr(workspace), workspace.numel(), _stream(stream))
     _raise_on("rod_swska_backward", st)
+    return dq, dk_, dv_
+
+
+def swska_backward_lse(q, k, v, o, lse, dO, window, scale=None, workspace=None, stream=None):
+    """swska_backward given the forward's o and lse (from swska_prefill_lse with the same q, k, v,
+    window and scale): the tensor-core route reads them instead of recomputing the forward.
+    Returns (dq, dk, dv)."""
+    _need(q, "q", None, 4)
+    _need(k, "k", q.dtype, 3)
+    _need(v, "v", q.dtype, 4)
+    _need(o, "o", q.dtype, 4)
+    _need(lse, "lse", torch.float32, 3)
+    _need(dO, "dO", q.dtype, 4)
+    B, H, T, dk = q.shape
+    dv = v.shape[-1]
+    if (tuple(k.shape) != (B, T, dk) or tuple(v.shape[:3]) != (B, H, T) or tuple(dO.shape) != tuple(v.shape)
+            or tuple(o.shape) != tuple(v.shape) or tuple(lse.shape) != (B, H, T)):
+        raise ValueError("shape mismatch")
+    lib = load_library()
+    need = lib.rod_swska_backward_workspace_size(B, H, T)
+    if workspace is None:
+        workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=q.device)
+    dq, dk_, dv_ = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    st = lib.rod_swska_backward_lse(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), _ptr(dO), _ptr(dq), _ptr(dk_),
+                                    _ptr(dv_), B, H, T, dk, dv, int(window), float(scale or 0.0), _dtype_code(q),
+                                    _ptr(workspace), workspace.numel(), _stream(stream))
+    _raise_on("rod_swska_backward_lse", st)
     return dq, dk_, dv_
 
 

@@ -34,21 +34,26 @@ unsigned gla_prefill_tc_take_timeout_flag();
 // copies, so that its bounded waits expire (probes = 0 disarms)
 void gla_prefill_tc_arm_wait_expiry(uint32_t probes);
 
-// SW-SKA prefill on CUDA cores (fp32 FMA, online softmax)
+// SW-SKA prefill on CUDA cores (fp32 FMA, online softmax); lse (optional, [B,H,T] fp32): the
+// natural log-sum-exp of each row's scaled scores
 cudaError_t swska_prefill_simt_launch(const void* q, const void* k, const void* v, void* o,
                                       int B, int H, int T, int dk, int dv, int window,
-                                      float scale, bool bf16, cudaStream_t stream);
+                                      float scale, bool bf16, cudaStream_t stream, float* lse = nullptr);
 
 // SW-SKA prefill on tcgen05 tensor cores (bf16, dk = dv = 128, T >= 128)
 bool swska_prefill_tc_supported(int H, int T, int dk, int dv);
 cudaError_t swska_prefill_tc_launch(const void* q, const void* k, const void* v, void* o, int B,
                                     int H, int T, int window, float scale, cudaStream_t stream);
 unsigned swska_prefill_tc_take_timeout_flag();
-// the same kernel with per-row statistics for the backward: negated base-2 log-sum-exp and
-// D = dO . o into row bh * Tpad + t (o may be null: then the output is not stored)
+// the same kernel with per-row statistics: lse_mul * (base-2 log-sum-exp) into row bh * Tpad + t
+// of `lse` (-1 gives the backward's negated base-2 form, ln 2 the natural log-sum-exp; rows past
+// T, up to Tpad, get -inf) and, with dO given, D = dO . o into the same row of dbuf. o may be
+// null (the output is then not stored), and so may dO and dbuf.
 cudaError_t swska_prefill_tc_stats_launch(const void* q, const void* k, const void* v, void* o,
-                                          const void* dO, float* nlse2, float* dbuf, int64_t Tpad, int B,
-                                          int H, int T, int window, float scale, cudaStream_t stream);
+                                          const void* dO, float* lse, float* dbuf, int64_t Tpad, int B,
+                                          int H, int T, int window, float scale, cudaStream_t stream,
+                                          float lse_mul = -1.f);
+
 
 // TMA descriptors for a 3-D tensor [d2][d1][d0] loaded as boxes of box1 x box0 elements
 cudaError_t make_tmap_3d(CUtensorMap* map, const void* base, bool fp32, uint64_t d0, uint64_t d1,
@@ -103,6 +108,9 @@ struct SkaBackwardArgs {
     int B, H, T, d_k, d_v, W;
     float scale;                 // resolved (> 0)
     void* workspace;             // swska_backward_workspace_size bytes, 16-byte aligned
+    const void* o = nullptr;     // optional: the forward's output [B,H,T,dv] ...
+    const float* lse = nullptr;  // ... and natural log-sum-exp [B,H,T]: the row statistics are then
+                                 // taken from them instead of recomputing the forward
 };
 size_t swska_backward_workspace_size(int B, int H, int T);
 cudaError_t swska_backward_launch(const SkaBackwardArgs& a, bool bf16, cudaStream_t stream);

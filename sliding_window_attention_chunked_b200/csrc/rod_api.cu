@@ -135,6 +135,26 @@ int rod_swska_prefill(const void* q, const void* k, const void* v, void* o, int 
                                                     resolve_scale(scale, dk), dtype == ROD_BF16, s));
 }
 
+int rod_swska_prefill_lse(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H,
+                          int T, int dk, int dv, int window, float scale, int dtype, void* stream) {
+    if (!dtype_ok(dtype)) return ROD_ERR_DTYPE;
+    if (B < 0 || H < 0 || T < 0 || H > 64 || window < 1 || !dim_ok(dk) || !dim_ok(dv))
+        return ROD_ERR_SHAPE;
+    if (!(scale == scale) || isinf(scale)) return ROD_ERR_SHAPE;
+    if ((int64_t)B * H == 0 || T == 0) return ROD_OK;
+    if (!q || !k || !v || !o || !lse) return ROD_ERR_NULL;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || reinterpret_cast<uintptr_t>(lse) % 4)
+        return ROD_ERR_ALIGN;
+    const cudaStream_t s = static_cast<cudaStream_t>(stream);
+    // the routes of rod_swska_prefill; the tensor-core kernel runs its statistics instantiation,
+    // which stores the output and each row's log-sum-exp (times ln 2: natural log)
+    if (dtype == ROD_BF16 && rod::swska_prefill_tc_supported(H, T, dk, dv))
+        return from_cuda(rod::swska_prefill_tc_stats_launch(q, k, v, o, nullptr, lse, nullptr, T, B, H, T, window,
+                                                            resolve_scale(scale, dk), s, 0.6931471805599453f));
+    return from_cuda(rod::swska_prefill_simt_launch(q, k, v, o, B, H, T, dk, dv, window,
+                                                    resolve_scale(scale, dk), dtype == ROD_BF16, s, lse));
+}
+
 int rod_swska_decode(const void* q, const void* k_new, const void* v_new, void* k_cache,
                      void* v_cache, const int64_t* pos, void* o, int N, int H, int dk, int dv,
                      int window, float scale, int dtype, void* stream) {
@@ -220,6 +240,26 @@ int rod_swska_backward(const void* q, const void* k, const void* v, const void* 
     if (!aligned16(workspace)) return ROD_ERR_ALIGN;
     rod::SkaBackwardArgs a{q, k, v, dO, dq, dk, dv, B, H, T, dk_dim, dv_dim, window,
                            resolve_scale(scale, dk_dim), workspace};
+    return from_cuda(rod::swska_backward_launch(a, dtype == ROD_BF16, static_cast<cudaStream_t>(stream)));
+}
+
+int rod_swska_backward_lse(const void* q, const void* k, const void* v, const void* o, const float* lse,
+                           const void* dO, void* dq, void* dk, void* dv, int B, int H, int T, int dk_dim,
+                           int dv_dim, int window, float scale, int dtype, void* workspace, size_t ws_bytes,
+                           void* stream) {
+    if (!dtype_ok(dtype)) return ROD_ERR_DTYPE;
+    if (B < 0 || H < 0 || T < 0 || H > 64 || window < 1 || !dim_ok(dk_dim) || !dim_ok(dv_dim))
+        return ROD_ERR_SHAPE;
+    if (!(scale == scale) || isinf(scale)) return ROD_ERR_SHAPE;
+    if ((int64_t)B * H == 0 || T == 0) return ROD_OK;
+    if (!q || !k || !v || !o || !lse || !dO || !dq || !dk || !dv) return ROD_ERR_NULL;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || reinterpret_cast<uintptr_t>(lse) % 4 ||
+        !aligned16(dO) || !aligned16(dq) || !aligned16(dk) || !aligned16(dv))
+        return ROD_ERR_ALIGN;
+    if (!workspace || ws_bytes < rod::swska_backward_workspace_size(B, H, T)) return ROD_ERR_WORKSPACE;
+    if (!aligned16(workspace)) return ROD_ERR_ALIGN;
+    rod::SkaBackwardArgs a{q, k, v, dO, dq, dk, dv, B, H, T, dk_dim, dv_dim, window,
+                           resolve_scale(scale, dk_dim), workspace, o, lse};
     return from_cuda(rod::swska_backward_launch(a, dtype == ROD_BF16, static_cast<cudaStream_t>(stream)));
 }
 

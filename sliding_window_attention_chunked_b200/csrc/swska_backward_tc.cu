@@ -731,6 +731,40 @@ ska_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
 }
 
 // ============================================================================================
+// Launch 1 when the forward's output and log-sum-exp were kept: one warp per (padded) row,
+// lane l holding channels 4l .. 4l + 3, D = dO . o in fp32 and nlse2 = -lse * log2(e); rows
+// past T get -inf and 0, as the statistics pass gives them.
+__global__ void __launch_bounds__(256)
+ska_rowstats_kernel(const __nv_bfloat16* __restrict__ o, const __nv_bfloat16* __restrict__ dO,
+                    const float* __restrict__ lse, float* __restrict__ nlse2, float* __restrict__ dbuf, int T,
+                    int Tpad, int64_t rows) {
+    const int64_t r = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+    const int lane = threadIdx.x & 31;
+    if (r >= rows) return;
+    const int64_t bh = r / Tpad;
+    const int t = (int)(r - bh * Tpad);
+    if (t >= T) {
+        if (lane == 0) {
+            nlse2[r] = -INFINITY;
+            dbuf[r] = 0.f;
+        }
+        return;
+    }
+    const int64_t off = (bh * T + t) * HD + 4 * lane;
+    const uint2 ow = *reinterpret_cast<const uint2*>(o + off);
+    const uint2 gw = *reinterpret_cast<const uint2*>(dO + off);
+    float d = bf16lo(ow.x) * bf16lo(gw.x);
+    d = fmaf(bf16hi(ow.x), bf16hi(gw.x), d);
+    d = fmaf(bf16lo(ow.y), bf16lo(gw.y), d);
+    d = fmaf(bf16hi(ow.y), bf16hi(gw.y), d);
+#pragma unroll
+    for (int sh = 16; sh > 0; sh >>= 1) d += __shfl_xor_sync(0xffffffffu, d, sh);
+    if (lane == 0) {
+        dbuf[r] = d;
+        nlse2[r] = -lse[bh * T + t] * kLog2e;
+    }
+}
+
 // Launch 4: dk = scale * sum over head groups of the partials (group order fixed)
 // ============================================================================================
 __global__ void __launch_bounds__(256)
@@ -791,10 +825,21 @@ cudaError_t swska_backward_tc_launch(const SkaBackwardArgs& a, cudaStream_t stre
     float* dbuf = nlse2 + (size_t)B * H * Tpad;
     float* part = dbuf + (size_t)B * H * Tpad;
     if (B > 65535 || H > 65535) return cudaErrorInvalidConfiguration;
-    // launch 1: the forward in statistics mode (row log-sum-exp and D, no output stored)
-    cudaError_t e = swska_prefill_tc_stats_launch(a.q, a.k, a.v, nullptr, a.dO, nlse2, dbuf, Tpad, B, H, T, W,
-                                                  a.scale, stream);
-    if (e != cudaSuccess) return e;
+    // launch 1: the row statistics, from the forward's saved output and log-sum-exp when given,
+    // else from the forward in statistics mode (row log-sum-exp and D, no output stored)
+    cudaError_t e;
+    if (a.o != nullptr && a.lse != nullptr) {
+        const int64_t rows = (int64_t)B * H * Tpad;
+        ska_rowstats_kernel<<<(unsigned)((rows * 32 + 255) / 256), 256, 0, stream>>>(
+            static_cast<const __nv_bfloat16*>(a.o), static_cast<const __nv_bfloat16*>(a.dO), a.lse, nlse2, dbuf,
+            T, (int)Tpad, rows);
+        note_launches(1);
+        if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    } else {
+        e = swska_prefill_tc_stats_launch(a.q, a.k, a.v, nullptr, a.dO, nlse2, dbuf, Tpad, B, H, T, W, a.scale,
+                                          stream);
+        if (e != cudaSuccess) return e;
+    }
     CUtensorMap mq, mdo, mk, mv;
     if ((e = make_tmap_bf16_3d(&mq, a.q, HD, (uint64_t)T, (uint64_t)B * H, 64, TILE)) != cudaSuccess) return e;
     if ((e = make_tmap_bf16_3d(&mdo, a.dO, HD, (uint64_t)T, (uint64_t)B * H, 64, TILE)) != cudaSuccess) return e;

@@ -24,8 +24,8 @@ constexpr int BK = 32;
 template <typename T, int DK, int DV>
 __global__ void __launch_bounds__(256)
 swska_prefill_simt_kernel(const T* __restrict__ q, const T* __restrict__ k,
-                          const T* __restrict__ v, T* __restrict__ o, int H, int T_len, int W,
-                          float scale_log2) {
+                          const T* __restrict__ v, T* __restrict__ o, float* __restrict__ lse, int H,
+                          int T_len, int W, float scale_log2) {
     constexpr int QP = DK / 4, VP = DV / 4;  // per-thread quarter of q and of the output
     __shared__ __align__(16) float sK[BK][DK];
     __shared__ __align__(16) float sV[BK][DV];
@@ -100,42 +100,44 @@ swska_prefill_simt_kernel(const T* __restrict__ q, const T* __restrict__ k,
         const float inv = 1.f / l_run;
 #pragma unroll
         for (int i = 0; i < VP; ++i) op[i] = from_f32<T>(acc[i] * inv);
+        // natural log-sum-exp of the row's scaled scores: the base-2 one times ln 2
+        if (lse != nullptr && part == 0) lse[bh * T_len + t] = (m_run + log2f(l_run)) * 0.6931471805599453f;
     }
 }
 
 template <typename T, int DK, int DV>
-cudaError_t launch_t(const void* q, const void* k, const void* v, void* o, int B, int H, int T_len,
-                     int W, float scale, cudaStream_t s) {
+cudaError_t launch_t(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H,
+                     int T_len, int W, float scale, cudaStream_t s) {
     const int64_t qtiles = (T_len + BQ - 1) / BQ;
     const int64_t grid = qtiles * B * H;
     if (grid > 0x7fffffffLL) return cudaErrorInvalidConfiguration;
     swska_prefill_simt_kernel<T, DK, DV><<<(unsigned)grid, 256, 0, s>>>(
         static_cast<const T*>(q), static_cast<const T*>(k), static_cast<const T*>(v),
-        static_cast<T*>(o), H, T_len, W, scale * 1.4426950408889634f);
+        static_cast<T*>(o), lse, H, T_len, W, scale * 1.4426950408889634f);
     note_launches(1);
     return cudaGetLastError();
 }
 
 template <typename T, int DK>
-cudaError_t launch_dv(int dv, const void* q, const void* k, const void* v, void* o, int B, int H,
+cudaError_t launch_dv(int dv, const void* q, const void* k, const void* v, void* o, float* lse, int B, int H,
                       int T_len, int W, float scale, cudaStream_t s) {
     switch (dv) {
-        case 16: return launch_t<T, DK, 16>(q, k, v, o, B, H, T_len, W, scale, s);
-        case 32: return launch_t<T, DK, 32>(q, k, v, o, B, H, T_len, W, scale, s);
-        case 64: return launch_t<T, DK, 64>(q, k, v, o, B, H, T_len, W, scale, s);
-        case 128: return launch_t<T, DK, 128>(q, k, v, o, B, H, T_len, W, scale, s);
+        case 16: return launch_t<T, DK, 16>(q, k, v, o, lse, B, H, T_len, W, scale, s);
+        case 32: return launch_t<T, DK, 32>(q, k, v, o, lse, B, H, T_len, W, scale, s);
+        case 64: return launch_t<T, DK, 64>(q, k, v, o, lse, B, H, T_len, W, scale, s);
+        case 128: return launch_t<T, DK, 128>(q, k, v, o, lse, B, H, T_len, W, scale, s);
     }
     return cudaErrorInvalidValue;
 }
 
 template <typename T>
-cudaError_t launch_dk(int dk, int dv, const void* q, const void* k, const void* v, void* o, int B,
+cudaError_t launch_dk(int dk, int dv, const void* q, const void* k, const void* v, void* o, float* lse, int B,
                       int H, int T_len, int W, float scale, cudaStream_t s) {
     switch (dk) {
-        case 16: return launch_dv<T, 16>(dv, q, k, v, o, B, H, T_len, W, scale, s);
-        case 32: return launch_dv<T, 32>(dv, q, k, v, o, B, H, T_len, W, scale, s);
-        case 64: return launch_dv<T, 64>(dv, q, k, v, o, B, H, T_len, W, scale, s);
-        case 128: return launch_dv<T, 128>(dv, q, k, v, o, B, H, T_len, W, scale, s);
+        case 16: return launch_dv<T, 16>(dv, q, k, v, o, lse, B, H, T_len, W, scale, s);
+        case 32: return launch_dv<T, 32>(dv, q, k, v, o, lse, B, H, T_len, W, scale, s);
+        case 64: return launch_dv<T, 64>(dv, q, k, v, o, lse, B, H, T_len, W, scale, s);
+        case 128: return launch_dv<T, 128>(dv, q, k, v, o, lse, B, H, T_len, W, scale, s);
     }
     return cudaErrorInvalidValue;
 }
@@ -144,10 +146,10 @@ cudaError_t launch_dk(int dk, int dv, const void* q, const void* k, const void* 
 
 cudaError_t swska_prefill_simt_launch(const void* q, const void* k, const void* v, void* o,
                                       int B, int H, int T, int dk, int dv, int window,
-                                      float scale, bool bf16, cudaStream_t stream) {
+                                      float scale, bool bf16, cudaStream_t stream, float* lse) {
     if ((int64_t)B * H == 0 || T == 0) return cudaSuccess;
-    return bf16 ? launch_dk<__nv_bfloat16>(dk, dv, q, k, v, o, B, H, T, window, scale, stream)
-                : launch_dk<float>(dk, dv, q, k, v, o, B, H, T, window, scale, stream);
+    return bf16 ? launch_dk<__nv_bfloat16>(dk, dv, q, k, v, o, lse, B, H, T, window, scale, stream)
+                : launch_dk<float>(dk, dv, q, k, v, o, lse, B, H, T, window, scale, stream);
 }
 
 }  // namespace rod

@@ -153,15 +153,15 @@ __device__ __forceinline__ int cta_item(int k, int n_items, bool snake) {
     return i < n_items ? i : -1;
 }
 
-// STATS: the backward's statistics mode (row log-sum-exp and D = dO . o, output optional); a
-// separate instantiation so the plain forward carries none of its registers
+// STATS: the statistics mode (each row's log-sum-exp times lse_mul, D = dO . o when dO is given,
+// output optional); a separate instantiation so the plain forward carries none of its registers
 template <bool STATS, bool QT_SLOW>
 __global__ void __launch_bounds__(NTHREADS, 1)
 swska_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                 const __grid_constant__ CUtensorMap tm_v, __nv_bfloat16* __restrict__ o, int T,
                 int H, int W, float scale_log2, int n_qtiles, int n_items,
                 const __nv_bfloat16* __restrict__ dO,
-                float* __restrict__ nlse2, float* __restrict__ dbuf, int Tpad) {
+                float* __restrict__ lse, float* __restrict__ dbuf, int Tpad, float lse_mul) {
     extern __shared__ unsigned char smem_raw[];
     unsigned char* smem = reinterpret_cast<unsigned char*>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -481,7 +481,7 @@ swska_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                         *reinterpret_cast<uint4*>(o + orow_i + cb + i) = u;
                     }
                 }
-                if (STATS && live) {
+                if (STATS && live && dO != nullptr) {
 #pragma unroll
                     for (int i = 0; i < 32; i += 8) {
                         float g[8];
@@ -491,10 +491,11 @@ swska_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                     }
                 }
             }
-            if (STATS && 2 * hp + h < H) {
+            // rows past T only where the statistics rows are padded (t < Tpad)
+            if (STATS && 2 * hp + h < H && t < Tpad) {
                 const int64_t srow = (int64_t)(b * H + 2 * hp + h) * Tpad + t;
-                nlse2[srow] = live ? -(m_run + log2f(l_run)) : -INFINITY;
-                dbuf[srow] = live ? dacc : 0.f;
+                lse[srow] = live ? lse_mul * (m_run + log2f(l_run)) : -INFINITY;
+                if (dbuf != nullptr) dbuf[srow] = live ? dacc : 0.f;
             }
             tb += n_it;
             ++items;
@@ -529,18 +530,19 @@ bool swska_prefill_tc_supported(int H, int T, int dk, int dv) {
 cudaError_t swska_prefill_tc_launch(const void* q, const void* k, const void* v, void* o, int B,
                                     int H, int T, int window, float scale, cudaStream_t stream) {
     return swska_prefill_tc_stats_launch(q, k, v, o, nullptr, nullptr, nullptr, 0, B, H, T, window, scale,
-                                         stream);
+                                         stream, -1.f);
 }
 
 cudaError_t swska_prefill_tc_stats_launch(const void* q, const void* k, const void* v, void* o,
-                                          const void* dO, float* nlse2, float* dbuf, int64_t Tpad, int B,
-                                          int H, int T, int window, float scale, cudaStream_t stream) {
+                                          const void* dO, float* lse, float* dbuf, int64_t Tpad, int B,
+                                          int H, int T, int window, float scale, cudaStream_t stream,
+                                          float lse_mul) {
     CUtensorMap mq, mk, mv;
     cudaError_t e;
     if ((e = make_tmap_bf16_3d(&mq, q, HD, (uint64_t)T, (uint64_t)B * H, 64, BM)) != cudaSuccess) return e;
     if ((e = make_tmap_bf16_3d(&mk, k, HD, (uint64_t)T, (uint64_t)B, 64, BN)) != cudaSuccess) return e;
     if ((e = make_tmap_bf16_3d(&mv, v, HD, (uint64_t)T, (uint64_t)B * H, 64, BN)) != cudaSuccess) return e;
-    const bool stats = nlse2 != nullptr;
+    const bool stats = lse != nullptr;
     const int n_qtiles = (T + BM - 1) / BM;
     const int64_t n_items = (int64_t)n_qtiles * ((H + 1) / 2) * B;
     if (n_items > INT32_MAX) return cudaErrorInvalidConfiguration;
@@ -559,7 +561,7 @@ cudaError_t swska_prefill_tc_stats_launch(const void* q, const void* k, const vo
         return e;
     kern<<<grid, NTHREADS, SMEM_BYTES, stream>>>(
         mq, mk, mv, static_cast<__nv_bfloat16*>(o), T, H, window, scale * 1.4426950408889634f,
-        n_qtiles, (int)n_items, static_cast<const __nv_bfloat16*>(dO), nlse2, dbuf, (int)Tpad);
+        n_qtiles, (int)n_items, static_cast<const __nv_bfloat16*>(dO), lse, dbuf, (int)Tpad, lse_mul);
     note_launches(1);
     return cudaGetLastError();
 }

@@ -167,3 +167,55 @@ def test_swska_backward_full_size():
     """The benchmarked backward workload (B1 H16 T8192 W4096, bf16, head dim 128), every
     gradient element against the oracle (about ten seconds of fp64 on the host)."""
     _ska_check(1, 16, 8192, 128, 128, 4096, "bf16", seed=42)
+
+
+# SW-SKA with the forward's saved statistics
+# ------------------------------------------------------------------------------------------
+
+
+def _ska_lse_check(B, H, T, dk, dv, W, dtype, seed):
+    """swska_prefill_lse (output and natural log-sum-exp per row) and swska_backward_lse (the
+    gradients from that output and log-sum-exp) against the oracle. The output must equal
+    swska_prefill's bit for bit (the same arithmetic); the log-sum-exp is a sum of fp32
+    exponentials of fp32 scores on both routes, held to 1e-4 relative (its terms carry the SFU's
+    2^-22 and the scores' fp32 rounding); the gradients to the backward's tolerances."""
+    q, k, v = wl.swska_inputs(B, H, T, dk, dv, seed=seed, dtype=dtype)
+    dO = (torch.randn(B, H, T, dv, generator=torch.Generator().manual_seed(seed + 5)) * 0.5).to(q.dtype)
+    o_ref, lse_ref = oracle.swska_prefill_lse(q, k, v, W)
+    qd, kd, vd, dOd = q.to(DEV), k.to(DEV), v.to(DEV), dO.to(DEV)
+    o, lse = rod.swska_prefill_lse(qd, kd, vd, W)
+    o_plain = rod.swska_prefill(qd, kd, vd, W)
+    rod.check()
+    what = f"B{B} H{H} T{T} dk{dk} dv{dv} W{W} {dtype}"
+    assert torch.equal(o, o_plain), f"o of swska_prefill_lse differs from swska_prefill ({what})"
+    compare(o, o_ref, dtype, f"o {what}")
+    lse_err = np.abs(lse.double().cpu().numpy() - lse_ref)
+    lim = 1e-4 * np.maximum(1.0, np.abs(lse_ref))
+    assert np.all(lse_err <= lim), f"lse {what}: max error {lse_err.max():.3e}"
+    ref = oracle.swska_backward(q, k, v, dO, W)
+    got = rod.swska_backward_lse(qd, kd, vd, o, lse, dOd, W)
+    rod.check()
+    for name, a, b in zip(("dq", "dk", "dv"), got, ref):
+        compare(a, b, dtype, f"{name} from saved statistics, {what}")
+
+
+# tensor-core route (bf16, head dim 128, T >= 128): one tile, ragged tails, windows of 1 and
+# beyond the sequence, several heads and batches
+@pytest.mark.parametrize("B,H,T,W", [(1, 2, 128, 128), (2, 3, 300, 1), (1, 4, 1000, 4096),
+                                     (1, 16, 1024, 256), (3, 1, 700, 64)])
+def test_swska_saved_statistics_tensor_core(B, H, T, W):
+    _ska_lse_check(B, H, T, 128, 128, W, "bf16", seed=7 * B + 11 * H + T + W)
+
+
+# CUDA-core route (fp32, other head dims, or T < 128): the prefill writes the log-sum-exp, the
+# backward recomputes its statistics
+@pytest.mark.parametrize("B,H,T,d,W,dtype", [(2, 3, 150, 32, 7, "fp32"), (2, 3, 300, 64, 100, "bf16"),
+                                             (1, 2, 100, 128, 40, "bf16")])
+def test_swska_saved_statistics_cuda_cores(B, H, T, d, W, dtype):
+    _ska_lse_check(B, H, T, d, d, W, dtype, seed=T + d + W)
+
+
+def test_swska_saved_statistics_full_size():
+    """The benchmarked backward workload (B1 H16 T8192 W4096, bf16) through the saved-statistics
+    path, every element against the oracle."""
+    _ska_lse_check(1, 16, 8192, 128, 128, 4096, "bf16", seed=43)

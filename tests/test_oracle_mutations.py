@@ -6,7 +6,8 @@ term, the readout using k, an off-by-one window, a dropped scale or normaliser, 
 ring-buffer slot, a hand-off that drops a token or numbers slots from the window start, a paged cache read
 without its table or written at the wrong row, a backward that weights the gate gradient
 with the updated state or decays the gradient state on the wrong channel, an attention backward
-without the softmax row term or with the shared key's gradient from one head, an E4M3 encoder
+without the softmax row term or with the shared key's gradient from one head, a row log-sum-exp
+without its maximum, an E4M3 encoder
 that breaks ties to the odd code, misplaces the subnormals or does not saturate, an FP8 decode
 that forgets the value scale, an FP8 fill that multiplies by the scale), builds the copy with gcc and runs every pin against it. Each planted
 mistake must make at least one pin fail; otherwise the pins are too weak to trust.
@@ -22,6 +23,7 @@ import oracle
 from oracle import build as obuild
 
 from . import test_oracle_pins as pins
+from . import test_oracle_swska_lse as lse_pins
 
 MUTATIONS = {
     "gate_on_wrong_channel": ("const double gc = (double)g[c];",
@@ -32,8 +34,9 @@ MUTATIONS = {
                          "acc += (double)k[c] * S[c * dv + j];"),
     "window_one_too_wide": ("int64_t j0 = t - a->W + 1;", "int64_t j0 = t - a->W;"),
     "scale_dropped": ("s[j - j0] = scale * acc;", "s[j - j0] = acc;"),
-    "normaliser_dropped": ("for (int64_t i = 0; i < dv; ++i) out[i] /= l;\n}",
-                           "for (int64_t i = 0; i < dv; ++i) out[i] /= 1.0;\n}"),
+    "normaliser_dropped": ("for (int64_t i = 0; i < dv; ++i) out[i] /= l;\n    return m + log(l);\n}",
+                           "for (int64_t i = 0; i < dv; ++i) out[i] /= 1.0;\n    return m + log(l);\n}"),
+    "lse_without_max": ("    return m + log(l);\n}", "    return log(l);\n}"),
     "ring_slot_off_by_one": ("const int64_t slot = pos[n] % W;",
                              "const int64_t slot = (pos[n] + 1) % W;"),
     "decode_window_too_wide": ("const int64_t p0 = P - a->W + 1 > 0 ? P - a->W + 1 : 0;",
@@ -68,7 +71,7 @@ MUTATIONS = {
 def _pin_calls():
     """Every pin test with each of its parametrizations, as zero-argument callables."""
     calls = []
-    for name, fn in inspect.getmembers(pins, inspect.isfunction):
+    for name, fn in [m for mod in (pins, lse_pins) for m in inspect.getmembers(mod, inspect.isfunction)]:
         if not name.startswith("test_"):
             continue
         marks = getattr(fn, "pytestmark", [])
