@@ -71,13 +71,19 @@ constexpr int OFF_PM = 320;      // per-head max   [MAX_H] f32
 constexpr int OFF_PL = 384;      // per-head sum   [MAX_H] f32
 constexpr int OFF_PACC = 512;    // per-head accumulator [HG][128] f32
 
-// HG: heads served by one CTA (warps 0 .. HG-1) next to the producer warp HG; row: bytes per row
+// HG: heads served by one CTA; C: head warps per head, each taking every C-th stage from a ring
+// of its own (warps 0 .. HG C - 1, head w / C, ring w mod C) next to the producer warp HG C;
+// D: stages per ring; row: bytes per row
 __host__ __device__ constexpr uint32_t stage_bytes(int HG, int row = ROW) { return (uint32_t)(KT * row * (1 + HG)); }
 __host__ __device__ constexpr uint32_t ring_offset(int HG) { return (uint32_t)(OFF_PACC + HG * DH * 4); }
 // a CTA's slice of a paged block table: at most pages_per_seq + 1 entries (ROD_MAX_PAGES_PER_SEQ)
 constexpr uint32_t kPageSlice = 520;
-__host__ __device__ constexpr uint32_t smem_total(int HG, int stages, int row = ROW) {
-    return ring_offset(HG) + (uint32_t)stages * stage_bytes(HG, row) + 4u * kPageSlice;
+// with C > 1, each head warp's partial for the in-CTA merge: 128 accumulator columns, then the
+// max and the sum, padded so that every partial starts on a 16-byte boundary (float4 accesses)
+constexpr int PART = DH + 4;
+__host__ __device__ constexpr uint32_t part_bytes(int HG, int C) { return C > 1 ? (uint32_t)(HG * C * PART * 4) : 0u; }
+__host__ __device__ constexpr uint32_t smem_total(int HG, int C, int D, int row = ROW) {
+    return ring_offset(HG) + (uint32_t)(C * D) * stage_bytes(HG, row) + 4u * kPageSlice + part_bytes(HG, C);
 }
 
 __device__ __forceinline__ bool wait_stage(uint64_t* bar, uint32_t parity, volatile int* abort_flag) {
@@ -243,12 +249,14 @@ __device__ __forceinline__ int64_t v_row(const CacheRef& c, int64_t n, int H, in
     return ((int64_t)pages[slot / c.page - pg0] * H + h) * c.page + slot % c.page;
 }
 
-template <bool PAGED, bool FP8>
+// MULTI: several head warps per head (C > 1); the C = 1 instantiation keeps the single-ring code
+template <bool PAGED, bool FP8, bool MULTI>
 __global__ void __launch_bounds__(32 * (MAX_H + 1), 2)
 swska_decode_warp_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ k_new,
                          const __nv_bfloat16* __restrict__ v_new, CacheRef cache,
                          const int64_t* __restrict__ pos, __nv_bfloat16* __restrict__ o, int H, int HG,
-                         int W, int stages, float scale_log2) {
+                         int W, int C_arg, int D, float scale_log2) {
+    const int C = MULTI ? C_arg : 1;
     extern __shared__ __align__(128) unsigned char smem[];
     cg::cluster_group cluster = cg::this_cluster();
     const int SP = (int)cluster.num_blocks();
@@ -277,8 +285,9 @@ swska_decode_warp_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat1
     const int s_end = s_begin + per < cnt ? s_begin + per : cnt;
     const int nst = (int)((s_end - s_begin + KT - 1) / KT);
 
+    // stage st lives in ring st mod C, buffer (st / C) mod D of it: buffer index (st mod C) D + that
     if (threadIdx.x == 0) {
-        for (int s = 0; s < stages; ++s) {
+        for (int s = 0; s < C * D; ++s) {
             mbar_init(&full[s], 1);
             mbar_init(&empty[s], (uint32_t)HG);
         }
@@ -287,87 +296,178 @@ swska_decode_warp_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat1
     }
     __syncthreads();
 
-    if (warp == HG) {
+    if (warp == HG * C) {
         // ---------------------------------- producer warp ----------------------------------
-        int32_t* pages = reinterpret_cast<int32_t*>(ring + (size_t)stages * SB);
+        int32_t* pages = reinterpret_cast<int32_t*>(ring + (size_t)(C * D) * SB);
         const int pg0 = PAGED ? s_begin / cache.page : 0;
         if (PAGED) {
             const int npg = s_end > s_begin ? (s_end - 1) / cache.page - pg0 + 1 : 0;
             for (int i = lane; i < npg; i += 32) pages[i] = cache.table[n * cache.pps + pg0 + i];
             __syncwarp();
         }
-        int issued = 0;
-        int buf = 0;
-        uint32_t par = 0;  // parity of this use of buffer buf (uses counted from 0)
-        int pi = 0, off = PAGED ? (int)(s_begin % cache.page) : 0;  // page slot of s0 (paged)
-        for (int st = 0; st < nst; ++st) {
-            if (st >= stages) {
-                const bool ok = wait_stage(&empty[buf], par ^ 1u, abort_flag);
-                if (!__all_sync(0xffffffffu, ok)) break;
-            }
-            const int s0 = s_begin + st * KT;
-            const int rows = s_end - s0 < KT ? s_end - s0 : KT;
-            unsigned char* dst = ring + (size_t)buf * SB;
-            const int r_new = (s_new >= s0 && s_new < s0 + rows) ? (int)(s_new - s0) : -1;
-            if (r_new >= 0) {
-                // the evicted slot takes the new token: into the stage and into the cache (its
-                // old content lies outside the window, so it is never copied in); the shared K
-                // row goes to the cache from head group 0 only
-                for (int i = lane; i < (1 + HG) * (RB / 16); i += 32) {
-                    const int row = i / (RB / 16), c16 = i % (RB / 16);
-                    const int64_t hv = n * H + hg0 + (row - 1);  // (sequence, head) of a V row
-                    const uint4* src = row == 0 ? reinterpret_cast<const uint4*>(k_new + n * DH)
-                                                : reinterpret_cast<const uint4*>(v_new + hv * DH);
-                    // FP8: 16 codes from 16 bf16 of the row, quantized with the cache's scale
-                    const uint4 val = FP8 ? quantize16(src[2 * c16], src[2 * c16 + 1], row == 0 ? cache.k_scale : cache.v_scale)
-                                          : src[c16];
-                    reinterpret_cast<uint4*>(dst + (size_t)row * KT * RB + (size_t)r_new * RB)[c16] = val;
-                    if (row == 0) {
-                        if (blockIdx.y == 0)
-                            reinterpret_cast<uint4*>(cache.k + k_row<PAGED>(cache, n, W, s_new, pages, pg0) * RB)[c16] = val;
-                    } else {
-                        reinterpret_cast<uint4*>(cache.v + v_row<PAGED>(cache, n, H, W, hg0 + row - 1, s_new, pages, pg0) * RB)[c16] = val;
+        if (!MULTI) {
+            // one ring, one stage per instruction (lanes 0 .. HG: the K rows and each head's V rows)
+            int issued = 0;
+            int buf = 0;
+            uint32_t par = 0;  // parity of this use of buffer buf (uses counted from 0)
+            int pi = 0, off = PAGED ? (int)(s_begin % cache.page) : 0;  // page slot of s0 (paged)
+            for (int st = 0; st < nst; ++st) {
+                if (st >= D) {
+                    const bool ok = wait_stage(&empty[buf], par ^ 1u, abort_flag);
+                    if (!__all_sync(0xffffffffu, ok)) break;
+                }
+                const int s0 = s_begin + st * KT;
+                const int rows = s_end - s0 < KT ? s_end - s0 : KT;
+                unsigned char* dst = ring + (size_t)buf * SB;
+                const int r_new = (s_new >= s0 && s_new < s0 + rows) ? (int)(s_new - s0) : -1;
+                if (r_new >= 0) {
+                    // the evicted slot takes the new token: into the stage and into the cache (its
+                    // old content lies outside the window, so it is never copied in); the shared K
+                    // row goes to the cache from head group 0 only
+                    for (int i = lane; i < (1 + HG) * (RB / 16); i += 32) {
+                        const int row = i / (RB / 16), c16 = i % (RB / 16);
+                        const int64_t hv = n * H + hg0 + (row - 1);  // (sequence, head) of a V row
+                        const uint4* src = row == 0 ? reinterpret_cast<const uint4*>(k_new + n * DH)
+                                                    : reinterpret_cast<const uint4*>(v_new + hv * DH);
+                        // FP8: 16 codes from 16 bf16 of the row, quantized with the cache's scale
+                        const uint4 val = FP8 ? quantize16(src[2 * c16], src[2 * c16 + 1], row == 0 ? cache.k_scale : cache.v_scale)
+                                              : src[c16];
+                        reinterpret_cast<uint4*>(dst + (size_t)row * KT * RB + (size_t)r_new * RB)[c16] = val;
+                        if (row == 0) {
+                            if (blockIdx.y == 0)
+                                reinterpret_cast<uint4*>(cache.k + k_row<PAGED>(cache, n, W, s_new, pages, pg0) * RB)[c16] = val;
+                        } else {
+                            reinterpret_cast<uint4*>(cache.v + v_row<PAGED>(cache, n, H, W, hg0 + row - 1, s_new, pages, pg0) * RB)[c16] = val;
+                        }
                     }
+                    // the generic stores precede later bulk copies into the same bytes
+                    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
                 }
-                // the generic stores precede later bulk copies into the same bytes
-                asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+                __syncwarp();
+                const int copied = rows - (r_new >= 0 ? 1 : 0);
+                if (lane == 0) mbar_arrive_expect_tx(&full[buf], (uint32_t)(copied * RB * (1 + HG)));
+                __syncwarp();
+                if (lane <= HG) {  // lane 0: the K rows; lane 1 + h: head hg0 + h's V rows
+                    unsigned char* d = dst + (size_t)lane * KT * RB;
+                    // rows s0 .. s0 + rows - 1 are contiguous (one page holds a whole stage)
+                    int64_t row0;
+                    if (PAGED) {
+                        const int64_t t = pages[pi];
+                        row0 = lane == 0 ? t * cache.page + off : (t * H + hg0 + lane - 1) * cache.page + off;
+                    } else {
+                        row0 = lane == 0 ? n * W + s0 : (n * H + hg0 + lane - 1) * W + s0;
+                    }
+                    const unsigned char* src = (lane == 0 ? cache.k : cache.v) + row0 * RB;
+                    const int a0 = 0, a1 = r_new >= 0 ? r_new : rows;   // rows [a0, a1)
+                    const int b0 = r_new >= 0 ? r_new + 1 : rows, b1 = rows;  // rows [b0, b1)
+                    if (a1 > a0) bulk_g2s(d + (size_t)a0 * RB, src + (int64_t)a0 * RB, (uint32_t)((a1 - a0) * RB), &full[buf]);
+                    if (b1 > b0) bulk_g2s(d + (size_t)b0 * RB, src + (int64_t)b0 * RB, (uint32_t)((b1 - b0) * RB), &full[buf]);
+                }
+                ++issued;
+                if (++buf == D) { buf = 0; par ^= 1u; }
+                if (PAGED && (off += KT) == cache.page) { off = 0; ++pi; }
+            }
+            // every copy issued has landed before the CTA's shared memory can go away (in the normal
+            // course the head warps waited for these phases already)
+            if (lane == 0) {
+                for (int s2 = issued > D ? issued - D : 0; s2 < issued; ++s2)
+                    if (!mbar_wait_bounded(&full[s2 % D], (uint32_t)((s2 / D) & 1), kWaitLimit))
+                        atomicExch(&g_swska_decode_warp_timeout, 1u);
             }
             __syncwarp();
-            const int copied = rows - (r_new >= 0 ? 1 : 0);
-            if (lane == 0) mbar_arrive_expect_tx(&full[buf], (uint32_t)(copied * RB * (1 + HG)));
-            __syncwarp();
-            if (lane <= HG) {  // lane 0: the K rows; lane 1 + h: head hg0 + h's V rows
-                unsigned char* d = dst + (size_t)lane * KT * RB;
-                // rows s0 .. s0 + rows - 1 are contiguous (one page holds a whole stage)
-                int64_t row0;
-                if (PAGED) {
-                    const int64_t t = pages[pi];
-                    row0 = lane == 0 ? t * cache.page + off : (t * H + hg0 + lane - 1) * cache.page + off;
-                } else {
-                    row0 = lane == 0 ? n * W + s0 : (n * H + hg0 + lane - 1) * W + s0;
-                }
-                const unsigned char* src = (lane == 0 ? cache.k : cache.v) + row0 * RB;
-                const int a0 = 0, a1 = r_new >= 0 ? r_new : rows;   // rows [a0, a1)
-                const int b0 = r_new >= 0 ? r_new + 1 : rows, b1 = rows;  // rows [b0, b1)
-                if (a1 > a0) bulk_g2s(d + (size_t)a0 * RB, src + (int64_t)a0 * RB, (uint32_t)((a1 - a0) * RB), &full[buf]);
-                if (b1 > b0) bulk_g2s(d + (size_t)b0 * RB, src + (int64_t)b0 * RB, (uint32_t)((b1 - b0) * RB), &full[buf]);
+        } else {
+            // Stages go out C at a time, one per ring (batch u holds stages u C .. u C + C - 1, each in
+            // buffer u mod D of its ring). One instruction carries a batch's copies: lane l takes row
+            // group l mod RG (0: the K rows, 1 + h: head hg0 + h's V rows) of the batch's stage l / RG.
+            // (One thread's copies go out a few hundred clocks apart; different lanes' together.)
+            const int RG = 1 + HG;
+            const int lst = lane / RG, lrg = lane - lst * RG;  // this lane's stage in a batch, row group
+            int ub = 0;                                        // u mod D
+            uint32_t par = 0;                                  // parity of use u / D of the buffers
+            int pi = 0, poff = 0;  // paged: page (index into pages) and slot of this lane's stage
+            if (PAGED) {
+                const int rel = s_begin - pg0 * cache.page + lst * KT;
+                pi = rel / cache.page;
+                poff = rel - pi * cache.page;
             }
-            ++issued;
-            if (++buf == stages) { buf = 0; par ^= 1u; }
-            if (PAGED && (off += KT) == cache.page) { off = 0; ++pi; }
+            const int st_new = (s_new >= s_begin && s_new < s_end) ? (s_new - s_begin) / KT : -1;
+            int issued_batches = 0;
+            for (int st0 = 0; st0 < nst; st0 += C) {
+                const int nb = nst - st0 < C ? nst - st0 : C;  // stages in this batch
+                // the batch's buffers are free once their previous uses are released
+                const bool need = lane < nb && st0 >= C * D;
+                if (!__all_sync(0xffffffffu, !need || wait_stage(&empty[lane * D + ub], par ^ 1u, abort_flag))) break;
+                if (st_new >= st0 && st_new < st0 + nb) {
+                    // the evicted slot takes the new token: into the stage and into the cache (its
+                    // old content lies outside the window, so it is never copied in); the shared K
+                    // row goes to the cache from head group 0 only
+                    const int r_new = s_new - (s_begin + st_new * KT);
+                    unsigned char* dst = ring + (size_t)((st_new - st0) * D + ub) * SB;
+                    for (int i = lane; i < RG * (RB / 16); i += 32) {
+                        const int row = i / (RB / 16), c16 = i % (RB / 16);
+                        const int64_t hv = n * H + hg0 + (row - 1);  // (sequence, head) of a V row
+                        const uint4* src = row == 0 ? reinterpret_cast<const uint4*>(k_new + n * DH)
+                                                    : reinterpret_cast<const uint4*>(v_new + hv * DH);
+                        // FP8: 16 codes from 16 bf16 of the row, quantized with the cache's scale
+                        const uint4 val = FP8 ? quantize16(src[2 * c16], src[2 * c16 + 1], row == 0 ? cache.k_scale : cache.v_scale)
+                                              : src[c16];
+                        reinterpret_cast<uint4*>(dst + (size_t)row * KT * RB + (size_t)r_new * RB)[c16] = val;
+                        if (row == 0) {
+                            if (blockIdx.y == 0)
+                                reinterpret_cast<uint4*>(cache.k + k_row<PAGED>(cache, n, W, s_new, pages, pg0) * RB)[c16] = val;
+                        } else {
+                            reinterpret_cast<uint4*>(cache.v + v_row<PAGED>(cache, n, H, W, hg0 + row - 1, s_new, pages, pg0) * RB)[c16] = val;
+                        }
+                    }
+                    // the generic stores precede later bulk copies into the same bytes
+                    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+                }
+                __syncwarp();
+                // each stage's full barrier expects its bytes before any of its copies can land
+                if (lane < nb) {
+                    const int st = st0 + lane, s0 = s_begin + st * KT;
+                    const int rows = s_end - s0 < KT ? s_end - s0 : KT;
+                    mbar_arrive_expect_tx(&full[lane * D + ub], (uint32_t)((rows - (st == st_new ? 1 : 0)) * RB * RG));
+                }
+                __syncwarp();
+                if (lst < nb) {
+                    const int st = st0 + lst, s0 = s_begin + st * KT;
+                    const int rows = s_end - s0 < KT ? s_end - s0 : KT;
+                    const int r_new = st == st_new ? s_new - s0 : -1;
+                    uint64_t* fb = &full[lst * D + ub];
+                    unsigned char* d = ring + (size_t)(lst * D + ub) * SB + (size_t)lrg * KT * RB;
+                    // rows s0 .. s0 + rows - 1 are contiguous (one page holds a whole stage)
+                    int64_t row0;
+                    if (PAGED) {
+                        const int64_t t = pages[pi];
+                        row0 = lrg == 0 ? t * cache.page + poff : (t * H + hg0 + lrg - 1) * cache.page + poff;
+                    } else {
+                        row0 = lrg == 0 ? n * W + s0 : (n * H + hg0 + lrg - 1) * W + s0;
+                    }
+                    const unsigned char* src = (lrg == 0 ? cache.k : cache.v) + row0 * RB;
+                    const int a0 = 0, a1 = r_new >= 0 ? r_new : rows;         // rows [a0, a1)
+                    const int b0 = r_new >= 0 ? r_new + 1 : rows, b1 = rows;  // rows [b0, b1)
+                    if (a1 > a0) bulk_g2s(d + (size_t)a0 * RB, src + (int64_t)a0 * RB, (uint32_t)((a1 - a0) * RB), fb);
+                    if (b1 > b0) bulk_g2s(d + (size_t)b0 * RB, src + (int64_t)b0 * RB, (uint32_t)((b1 - b0) * RB), fb);
+                }
+                ++issued_batches;
+                if (++ub == D) { ub = 0; par ^= 1u; }
+                if (PAGED)
+                    for (poff += C * KT; poff >= cache.page; poff -= cache.page) ++pi;
+            }
+            // every copy issued has landed before the CTA's shared memory can go away (in the normal
+            // course the head warps waited for these phases already): the last D batches of each ring
+            if (lane < C) {
+                for (int u = issued_batches > D ? issued_batches - D : 0; u < issued_batches; ++u)
+                    if (u * C + lane < nst &&
+                        !mbar_wait_bounded(&full[lane * D + u % D], (uint32_t)((u / D) & 1), kWaitLimit))
+                        atomicExch(&g_swska_decode_warp_timeout, 1u);
+            }
+            __syncwarp();
         }
-        // every copy issued has landed before the CTA's shared memory can go away (in the normal
-        // course the head warps waited for these phases already)
-        if (lane == 0) {
-            for (int s2 = issued > stages ? issued - stages : 0; s2 < issued; ++s2)
-                if (!mbar_wait_bounded(&full[s2 % stages], (uint32_t)((s2 / stages) & 1), kWaitLimit))
-                    atomicExch(&g_swska_decode_warp_timeout, 1u);
-        }
-        __syncwarp();
-    }
-    else {
-        // -------------------------- head warp h: head hg0 + h --------------------------
-        const int h = warp;
+    } else if (warp < HG * C) {
+        // -------------------- head warp: head hg0 + h, stages c, c + C, ... --------------------
+        const int h = warp / C, c = warp - h * C;
         uint2 qw = *reinterpret_cast<const uint2*>(q + (n * H + hg0 + h) * (int64_t)DH + 4 * lane);
         if (FP8) {  // q in f16 for the f16 x f16 products with the E4M3 rows
             const __half2 a = __floats2half2_rn(bf16lo(qw.x), bf16hi(qw.x));
@@ -376,29 +476,65 @@ swska_decode_warp_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat1
         }
         HeadState hs;
         bool ok = true;
-        int buf = 0;
+        int ub = 0;
         uint32_t par = 0;
-        for (int st = 0; st < nst; ++st) {
-            if (!__all_sync(0xffffffffu, wait_stage(&full[buf], par, abort_flag))) {
+        for (int st = c; st < nst; st += C) {
+            const int bi = c * D + ub;
+            if (!__all_sync(0xffffffffu, wait_stage(&full[bi], par, abort_flag))) {
                 ok = false;
                 break;
             }
             const int s0 = s_begin + st * KT;
             const int rows = s_end - s0 < KT ? s_end - s0 : KT;
-            const unsigned char* kb = ring + (size_t)buf * SB + (RB / 32) * lane;
+            const unsigned char* kb = ring + (size_t)bi * SB + (RB / 32) * lane;
             const unsigned char* vb = kb + (size_t)(1 + h) * KT * RB;
             if (rows == KT) head_stage<true, FP8>(kb, vb, qw, scale_log2, KT, lane, hs);
             else head_stage<false, FP8>(kb, vb, qw, scale_log2, rows, lane, hs);
             __syncwarp();
-            if (lane == 0) mbar_arrive(&empty[buf]);
-            if (++buf == stages) { buf = 0; par ^= 1u; }
+            if (lane == 0) mbar_arrive(&empty[bi]);
+            if (++ub == D) { ub = 0; par ^= 1u; }
         }
         float l = hs.l_part;
 #pragma unroll
         for (int off = 16; off > 0; off >>= 1) l += __shfl_xor_sync(0xffffffffu, l, off);
-        if (lane == 0) { s_pm[h] = ok ? hs.m_run : NAN; s_pl[h] = l; }
-        *reinterpret_cast<float4*>(s_pacc + h * DH + 4 * lane) =
-            make_float4(hs.acc[0], hs.acc[1], hs.acc[2], hs.acc[3]);
+        if (!MULTI) {
+            if (lane == 0) { s_pm[h] = ok ? hs.m_run : NAN; s_pl[h] = l; }
+            *reinterpret_cast<float4*>(s_pacc + h * DH + 4 * lane) =
+                make_float4(hs.acc[0], hs.acc[1], hs.acc[2], hs.acc[3]);
+        } else {
+            float* part = reinterpret_cast<float*>(ring + (size_t)(C * D) * SB + 4u * kPageSlice) +
+                          (size_t)warp * PART;
+            if (lane == 0) { part[DH] = ok ? hs.m_run : NAN; part[DH + 1] = l; }
+            *reinterpret_cast<float4*>(part + 4 * lane) = make_float4(hs.acc[0], hs.acc[1], hs.acc[2], hs.acc[3]);
+        }
+    }
+    if (MULTI) {
+        // merge each head's C partials, in ring order (deterministic), into the head's triple
+        __syncthreads();
+        if (warp < HG * C && warp % C == 0) {
+            const int h = warp / C;
+            const float* part = reinterpret_cast<const float*>(ring + (size_t)(C * D) * SB + 4u * kPageSlice) +
+                                (size_t)warp * PART;
+            float M = -INFINITY;
+            bool nan = false;
+            for (int cc = 0; cc < C; ++cc) {
+                const float m = part[cc * PART + DH];
+                nan |= isnan(m);
+                M = fmaxf(M, m);
+            }
+            float L = 0.f, a[4] = {0.f, 0.f, 0.f, 0.f};
+            for (int cc = 0; cc < C; ++cc) {
+                const float* pc = part + cc * PART;
+                if (!(pc[DH] > -INFINITY)) continue;  // a head warp without slots (or one that gave up)
+                const float w = ex2_approx(pc[DH] - M);
+                L = fmaf(w, pc[DH + 1], L);
+                const float4 pa = *reinterpret_cast<const float4*>(pc + 4 * lane);
+                a[0] = fmaf(w, pa.x, a[0]); a[1] = fmaf(w, pa.y, a[1]);
+                a[2] = fmaf(w, pa.z, a[2]); a[3] = fmaf(w, pa.w, a[3]);
+            }
+            if (lane == 0) { s_pm[h] = nan ? NAN : M; s_pl[h] = L; }
+            *reinterpret_cast<float4*>(s_pacc + h * DH + 4 * lane) = make_float4(a[0], a[1], a[2], a[3]);
+        }
     }
     cluster.sync();
     // ---- combine: CTA `rank` finalises the heads h with h mod SP == rank (warp h, 4 columns a lane)
@@ -435,7 +571,8 @@ swska_decode_warp_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat1
 struct DecodeConfig {
     int SP;      // CTAs per cluster: the window split
     int HG;      // heads per CTA
-    int stages;  // ring depth
+    int stages;  // ring depth (per ring)
+    int C = 1;   // head warps per head, one ring each
 };
 
 // ring depth: about 64 KB of copies in flight per CTA, at least 3 stages
@@ -444,12 +581,12 @@ int stages_for(int HG, int row = ROW) {
     return st < 3 ? 3 : (st > MAX_STAGES ? MAX_STAGES : st);
 }
 
-template <bool PAGED, bool FP8>
+template <bool PAGED, bool FP8, bool MULTI = false>
 cudaError_t set_attributes(size_t smem) {
-    cudaError_t e = cudaFuncSetAttribute(swska_decode_warp_kernel<PAGED, FP8>,
+    cudaError_t e = cudaFuncSetAttribute(swska_decode_warp_kernel<PAGED, FP8, MULTI>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e == cudaSuccess)
-        e = cudaFuncSetAttribute(swska_decode_warp_kernel<PAGED, FP8>,
+        e = cudaFuncSetAttribute(swska_decode_warp_kernel<PAGED, FP8, MULTI>,
                                  cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
     return e;
 }
@@ -475,7 +612,7 @@ int clusters_that_fit(int HG, int sp, bool fp8) {
     int& slot = cache[dev][HG][si][fp8 ? 1 : 0];
     if (slot < 0) {
         const int row = fp8 ? ROW8 : ROW;
-        const size_t smem = smem_total(HG, stages_for(HG, row), row);
+        const size_t smem = smem_total(HG, 1, stages_for(HG, row), row);
         int num = 0;
         if ((fp8 ? set_attributes<false, true>(smem) : set_attributes<false, false>(smem)) == cudaSuccess) {
             cudaLaunchConfig_t cfg = {};
@@ -490,8 +627,8 @@ int clusters_that_fit(int HG, int sp, bool fp8) {
             cfg.attrs = attr;
             cfg.numAttrs = 1;
             // the paged instance has the same resources as the ring one
-            const cudaError_t q = fp8 ? cudaOccupancyMaxActiveClusters(&num, swska_decode_warp_kernel<false, true>, &cfg)
-                                      : cudaOccupancyMaxActiveClusters(&num, swska_decode_warp_kernel<false, false>, &cfg);
+            const cudaError_t q = fp8 ? cudaOccupancyMaxActiveClusters(&num, swska_decode_warp_kernel<false, true, false>, &cfg)
+                                      : cudaOccupancyMaxActiveClusters(&num, swska_decode_warp_kernel<false, false, false>, &cfg);
             if (q != cudaSuccess) num = 0;
         }
         cudaGetLastError();
@@ -513,6 +650,26 @@ constexpr double kCtasToSaturate = 200.0;
 
 DecodeConfig pick_config(int N, int H, int W, bool fp8) {
     const int row = fp8 ? ROW8 : ROW;
+    // Small batches (N H <= 64): with one head warp per head, each CTA walks its 8-slot stages one
+    // after the other at about 900 clocks each, and the time follows the stages per CTA, not the
+    // bytes (measured at N 1: 5 us + 3.4 us per 1024 slots for any head count). There, about 256
+    // CTAs of one or two heads each, a 16-CTA cluster at most splitting a window, and each head
+    // spread over C = 8 head warps (each taking every C-th stage from a ring of its own, the
+    // producer sending C stages per instruction): measured at H 16, W 4096, in CUDA graphs,
+    // N 1: 11.9 against 20.8 us, N 4: 20.1 against 24.5 us; at N 16 it no longer pays.
+    if ((int64_t)N * H <= 64) {
+        const int HG = ((int64_t)N * H * 16 <= 256 || H % 2) ? 1 : 2;
+        int sp = 16;
+        while (sp > 1 && (int64_t)N * sp * (H / HG) > 256) sp /= 2;
+        const int stages_per_cta = ((W + sp - 1) / sp + KT - 1) / KT;
+        int C = 1;
+        while (2 * C <= 8 && 2 * C * (1 + HG) <= 32 && 2 * C * HG <= 16 && 8 * C <= stages_per_cta) C *= 2;
+        if (C > 1 && clusters_that_fit(HG, sp, fp8) > 0) {
+            const int by_bytes = (int)(65536u / ((uint32_t)C * stage_bytes(HG, row)));
+            const int D = 16 / C < by_bytes ? 16 / C : by_bytes;
+            return DecodeConfig{sp, HG, D < 2 ? 2 : D, C};
+        }
+    }
     DecodeConfig best{1, H, stages_for(H, row)};
     double best_cost = -1.0;
     for (int HG = H; HG >= 1; --HG) {
@@ -550,12 +707,12 @@ cudaError_t launch(const void* q, const void* k_new, const void* v_new, CacheRef
     if (N == 0) return cudaSuccess;
     constexpr int RB = row_bytes<FP8>();
     const DecodeConfig c = pick_config(N, H, window, FP8);
-    const size_t smem = smem_total(c.HG, c.stages, RB);
-    cudaError_t e = set_attributes<PAGED, FP8>(smem);
+    const size_t smem = smem_total(c.HG, c.C, c.stages, RB);
+    cudaError_t e = c.C > 1 ? set_attributes<PAGED, FP8, true>(smem) : set_attributes<PAGED, FP8, false>(smem);
     if (e != cudaSuccess) return e;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3((unsigned)((int64_t)N * c.SP), (unsigned)(H / c.HG), 1);
-    cfg.blockDim = dim3((unsigned)(32 * (c.HG + 1)), 1, 1);
+    cfg.blockDim = dim3((unsigned)(32 * (c.HG * c.C + 1)), 1, 1);
     cfg.dynamicSmemBytes = smem;
     cfg.stream = stream;
     cudaLaunchAttribute attr[1];
@@ -568,10 +725,11 @@ cudaError_t launch(const void* q, const void* k_new, const void* v_new, CacheRef
     // the K scale multiplies every score: folded into the base-2 score scale
     const float scale_log2 = scale * 1.4426950408889634f * (FP8 ? cache.k_scale : 1.f);
     note_launches(1);
-    return cudaLaunchKernelEx(&cfg, swska_decode_warp_kernel<PAGED, FP8>,
+    auto* kern = c.C > 1 ? swska_decode_warp_kernel<PAGED, FP8, true> : swska_decode_warp_kernel<PAGED, FP8, false>;
+    return cudaLaunchKernelEx(&cfg, kern,
                               static_cast<const __nv_bfloat16*>(q), static_cast<const __nv_bfloat16*>(k_new),
                               static_cast<const __nv_bfloat16*>(v_new), cache, pos,
-                              static_cast<__nv_bfloat16*>(o), H, c.HG, window, c.stages, scale_log2);
+                              static_cast<__nv_bfloat16*>(o), H, c.HG, window, c.C, c.stages, scale_log2);
 }
 
 }  // namespace
