@@ -10,7 +10,9 @@
 // owns float4 column group cg of rows rg, rg+RG, ...; a warp touches whole contiguous rows,
 // so every access is a coalesced 128-bit load or store. All row loads are issued before any
 // arithmetic so that each thread keeps DK/RG independent 16-byte loads in flight. The column
-// sums of q * S_new are reduced across the RG row groups through shared memory.
+// sums of q * S_new are reduced across the RG row groups through shared memory. With few
+// (n, h) pairs the columns are split over SPLIT CTAs (each column of o needs only its own column
+// of S), so that more CTAs share the latency of the state's round trip.
 #include "common.cuh"
 #include "kernels.h"
 
@@ -18,7 +20,7 @@ namespace rod {
 namespace {
 
 template <typename T, int DK, int DV>
-struct DecodeShape {
+struct DecodeShape {                                    // DV: the columns one CTA handles
     static constexpr int TPC = DV / 4;                  // threads across the columns
     static constexpr int RG0 = 256 / TPC;
     static constexpr int RG = RG0 < DK ? RG0 : DK;      // row groups
@@ -26,11 +28,12 @@ struct DecodeShape {
     static constexpr int THREADS = TPC * RG;
 };
 
-template <typename T, int DK, int DV>
+// DV: the state's columns; DVC: the columns of this CTA (blockIdx.y selects which)
+template <typename T, int DK, int DV, int DVC>
 __global__ void __launch_bounds__(256)
 gla_decode_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* __restrict__ v,
                   const float* __restrict__ g, float* __restrict__ state, T* __restrict__ o) {
-    using Sh = DecodeShape<T, DK, DV>;
+    using Sh = DecodeShape<T, DK, DVC>;
     constexpr int TPC = Sh::TPC, RG = Sh::RG, RPT = Sh::RPT;
     __shared__ float s_q[DK], s_k[DK], s_g[DK];
     __shared__ float4 s_red[RG][TPC];
@@ -38,7 +41,8 @@ gla_decode_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* __r
     const int64_t nh = blockIdx.x;
     const int tid = threadIdx.x;
     const int cg = tid % TPC, rg = tid / TPC;
-    float* S = state + nh * (int64_t)(DK * DV);
+    const int col0 = (int)blockIdx.y * DVC;
+    float* S = state + nh * (int64_t)(DK * DV) + col0;
 
     float4 s4[RPT];
 #pragma unroll
@@ -50,7 +54,7 @@ gla_decode_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* __r
         s_k[c] = to_f32(k[nh * DK + c]);
         s_g[c] = g[nh * DK + c];
     }
-    const float4 v4 = load4(v + nh * DV + 4 * cg);
+    const float4 v4 = load4(v + nh * DV + col0 + 4 * cg);
     __syncthreads();
 
     float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
@@ -78,15 +82,15 @@ gla_decode_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* __r
             const float4 p = s_red[r][cg];
             tot.x += p.x; tot.y += p.y; tot.z += p.z; tot.w += p.w;
         }
-        store4(o + nh * DV + 4 * cg, tot);
+        store4(o + nh * DV + col0 + 4 * cg, tot);
     }
 }
 
-template <typename T, int DK, int DV>
+template <typename T, int DK, int DV, int DVC = DV>
 cudaError_t launch_t(const void* q, const void* k, const void* v, const float* g, float* state,
                      void* o, int64_t NH, cudaStream_t stream) {
-    using Sh = DecodeShape<T, DK, DV>;
-    gla_decode_kernel<T, DK, DV><<<(unsigned)NH, Sh::THREADS, 0, stream>>>(
+    using Sh = DecodeShape<T, DK, DVC>;
+    gla_decode_kernel<T, DK, DV, DVC><<<dim3((unsigned)NH, DV / DVC), Sh::THREADS, 0, stream>>>(
         static_cast<const T*>(q), static_cast<const T*>(k), static_cast<const T*>(v), g, state,
         static_cast<T*>(o));
     note_launches(1);
@@ -100,7 +104,12 @@ cudaError_t launch_dv(int dv, const void* q, const void* k, const void* v, const
         case 16: return launch_t<T, DK, 16>(q, k, v, g, state, o, NH, s);
         case 32: return launch_t<T, DK, 32>(q, k, v, g, state, o, NH, s);
         case 64: return launch_t<T, DK, 64>(q, k, v, g, state, o, NH, s);
-        case 128: return launch_t<T, DK, 128>(q, k, v, g, state, o, NH, s);
+        case 128:
+            // few (n, h) pairs: the columns split over 4 or 2 CTAs (N 1, H 16, in CUDA graphs:
+            // 2.79 -> 1.86 us; N 4: 2.85 -> 2.31 us)
+            if (NH <= 64) return launch_t<T, DK, 128, 32>(q, k, v, g, state, o, NH, s);
+            if (NH <= 128) return launch_t<T, DK, 128, 64>(q, k, v, g, state, o, NH, s);
+            return launch_t<T, DK, 128>(q, k, v, g, state, o, NH, s);
     }
     return cudaErrorInvalidValue;
 }

@@ -166,8 +166,10 @@ def test_gla_prefill_full_workload():
 # ------------------------------------------------------------------------------------------
 
 
+# dv = 128 with few (n, h) pairs splits the columns over 4 (N H <= 64) or 2 (<= 128) CTAs
 @pytest.mark.parametrize("dtype,N,H,dk,dv", [("fp32", 3, 2, 16, 32), ("fp32", 5, 3, 128, 64),
-                                             ("bf16", 256, 16, 128, 128)])
+                                             ("bf16", 256, 16, 128, 128), ("bf16", 1, 16, 128, 128),
+                                             ("fp32", 2, 3, 64, 128), ("bf16", 5, 20, 128, 128)])
 def test_gla_decode_step(dtype, N, H, dk, dv):
     dd = wl.decode_inputs(N, H, dk, dv, 8, seed=N + dk, dtype=dtype)
     o_ref, S_ref = oracle.gla_decode_step(dd["q"], dd["k"], dd["v"], dd["g"], dd["state"])
