@@ -218,11 +218,14 @@ constexpr int CA_SCAN = 12 * BOX;
 constexpr int CA_BAR = CA_SCAN + 4 * D * 4;
 constexpr int CA_MISC = CA_BAR + 32;
 constexpr int CA_SMEM = CA_MISC + 32 + 1024;
+constexpr int CA_STAGE = 32 * 32 * 4;   // one 32 x 32 fp32 tile of U or U' on its way out
+static_assert(8 * 2 * CA_STAGE <= CA_G - CA_Q, "two staging tiles per warp fit over q, k, v, dO");
 
 __global__ void __launch_bounds__(256, 2)
 gla_bwd_contrib_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                        const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
-                       const __grid_constant__ CUtensorMap tm_g, BwdArgs args) {
+                       const __grid_constant__ CUtensorMap tm_g, const __grid_constant__ CUtensorMap tm_u,
+                       const __grid_constant__ CUtensorMap tm_u2, BwdArgs args) {
     extern __shared__ unsigned char smem_raw[];
     unsigned char* smem = reinterpret_cast<unsigned char*>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -321,20 +324,38 @@ gla_bwd_contrib_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_co
     }
     if (ok && __syncthreads_and(wait_bar(mma, 0, abort_flag))) {
         tc::fence_after_sync();
-        // warps 0-3: U rows, warps 4-7: U' rows (row c = TMEM lane)
-        const int c = 32 * (warp & 3) + lane;
+        // warps 0-3: U rows, warps 4-7: U' rows (row c = TMEM lane). A warp moves 32 rows x 32
+        // columns at a time through shared memory (the operand tiles are free once the MMAs are
+        // done): each thread writes its row with the 128-byte swizzle, so the eight 16-byte pieces
+        // of a quarter-warp land in distinct banks, and one lane stores the tile with TMA. Direct
+        // row-per-thread global stores would touch 32 lines per instruction and back up the
+        // load/store queue.
+        const int rw = 32 * (warp & 3);
         const uint32_t col0 = warp < 4 ? 0u : 128u;
-        float* dst = (warp < 4 ? args.U : args.U2) + (((int64_t)bh * args.NC + n) * D + c) * D;
+        const CUtensorMap* tm = warp < 4 ? &tm_u : &tm_u2;
+        unsigned char* stage = smem + CA_Q + warp * (2 * CA_STAGE);
+        const int z = bh * args.NC + n;
 #pragma unroll
         for (int cb = 0; cb < D; cb += 32) {
+            unsigned char* buf = stage + ((cb / 32) & 1) * CA_STAGE;
             uint32_t r[32];
-            tc::tmem_ld32(tmem + col0 + cb + ((uint32_t)(32 * (warp & 3)) << 16), r);
+            tc::tmem_ld32(tmem + col0 + cb + ((uint32_t)rw << 16), r);
+            if (cb >= 64 && lane == 0) tc::bulk_wait_read_1();  // the store two tiles back has read buf
+            __syncwarp();
             tc::tmem_wait_ld();
 #pragma unroll
-            for (int i = 0; i < 32; i += 4)
-                *reinterpret_cast<float4*>(dst + cb + i) = make_float4(__uint_as_float(r[i]), __uint_as_float(r[i + 1]),
-                                                                       __uint_as_float(r[i + 2]), __uint_as_float(r[i + 3]));
+            for (int j = 0; j < 8; ++j)
+                *reinterpret_cast<uint4*>(buf + lane * 128 + ((j ^ (lane & 7)) << 4)) =
+                    make_uint4(r[4 * j], r[4 * j + 1], r[4 * j + 2], r[4 * j + 3]);
+            tc::fence_proxy_async();
+            __syncwarp();
+            if (lane == 0) {
+                tc::tma_store_3d(tm, buf, cb, rw, z);
+                tc::bulk_commit();
+            }
         }
+        if (lane == 0) tc::bulk_wait_all();
+        __syncwarp();
     } else if (ok && warp == 0) {
         // the MMAs were issued but did not complete in time: wait once more before TMEM is freed
         mbar_wait_bounded(mma, 0, kWaitLimit);
@@ -899,7 +920,7 @@ cudaError_t gla_backward_tc_launch(const GlaBackwardArgs& g, cudaStream_t stream
     a.dstate0 = g.dstate0;
     const int NC = a.NC;
     if ((int64_t)NC * BH > 0x7fffffff) return cudaErrorInvalidConfiguration;
-    CUtensorMap mq, mk, mv, mdo, mg, msin, me, mdq, mdk, mdv, mdg;
+    CUtensorMap mq, mk, mv, mdo, mg, msin, me, mdq, mdk, mdv, mdg, mu, mu2;
     cudaError_t e;
     const uint64_t Tu = (uint64_t)T, BHu = (uint64_t)BH;
     if ((e = make_tmap_3d(&mq, g.q, false, D, Tu, BHu, 64, C, true)) != cudaSuccess) return e;
@@ -913,13 +934,15 @@ cudaError_t gla_backward_tc_launch(const GlaBackwardArgs& g, cudaStream_t stream
     if ((e = make_tmap_3d(&mdk, g.dk, false, D, Tu, BHu, D, C, false)) != cudaSuccess) return e;
     if ((e = make_tmap_3d(&mdv, g.dv, false, D, Tu, BHu, D, C, false)) != cudaSuccess) return e;
     if ((e = make_tmap_3d(&mdg, g.dg, true, D, Tu, BHu, D, C, false)) != cudaSuccess) return e;
+    if ((e = make_tmap_3d(&mu, a.U, true, D, D, BHu * NC, 32, 32, true)) != cudaSuccess) return e;
+    if ((e = make_tmap_3d(&mu2, a.U2, true, D, D, BHu * NC, 32, 32, true)) != cudaSuccess) return e;
     if ((e = cudaFuncSetAttribute(gla_bwd_contrib_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, CA_SMEM)) !=
         cudaSuccess)
         return e;
     if ((e = cudaFuncSetAttribute(gla_bwd_grad_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, GB_SMEM)) !=
         cudaSuccess)
         return e;
-    gla_bwd_contrib_kernel<<<dim3((unsigned)NC, (unsigned)BH), 256, CA_SMEM, stream>>>(mq, mk, mv, mdo, mg, a);
+    gla_bwd_contrib_kernel<<<dim3((unsigned)NC, (unsigned)BH), 256, CA_SMEM, stream>>>(mq, mk, mv, mdo, mg, mu, mu2, a);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     gla_bwd_scan_kernel<<<dim3((D * D / 4 + 255) / 256, (unsigned)BH), 256, 0, stream>>>(a);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
