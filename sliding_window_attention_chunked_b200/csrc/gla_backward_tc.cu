@@ -70,6 +70,10 @@ struct BwdArgs {
     const float* state0;        // [BH][D][D]
     const float* dstate_final;  // [BH][D][D] or null
     float* dstate0;             // [BH][D][D]
+    // the gradient kernel's inputs, for its L2 prefetch of the chunk one wave ahead
+    const __nv_bfloat16 *q, *k, *v, *dO;
+    const float* g;
+    int wave;                   // CTAs resident at once (0: no prefetch)
 };
 
 // ---- small helpers ---------------------------------------------------------------------------
@@ -354,7 +358,7 @@ gla_bwd_contrib_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_co
                 tc::bulk_commit();
             }
         }
-        if (lane == 0) tc::bulk_wait_all();
+        if (lane == 0) tc::bulk_wait_read();
         __syncwarp();
     } else if (ok && warp == 0) {
         // the MMAs were issued but did not complete in time: wait once more before TMEM is freed
@@ -497,6 +501,23 @@ gla_bwd_grad_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                 tc::tma_load_3d(smem + GB_E + h * BOX128, &tm_e, h * 64, 0, zc, full);
             }
             tc::tma_load_3d(smem + GB_G, &tm_g, 0, t0, bh, full);
+            // CTAs start in linear order, one per SM: the chunk one wave later streams into L2
+            // while this one computes, so its copies come from L2 instead of waiting on HBM
+            const int64_t nxt = (int64_t)blockIdx.y * gridDim.x + blockIdx.x + args.wave;
+            if (args.wave > 0 && nxt < (int64_t)gridDim.x * gridDim.y) {
+                const int n2 = (int)(nxt % gridDim.x), bh2 = (int)(nxt / gridDim.x);
+                const int t2 = n2 * C;
+                const uint32_t rows = (uint32_t)min(C, args.T - t2);
+                const int64_t row0 = (int64_t)bh2 * args.T + t2;
+                const int64_t z2 = (int64_t)bh2 * args.NC + n2;
+                tc::prefetch_l2(args.q + row0 * D, rows * D * 2);
+                tc::prefetch_l2(args.k + row0 * D, rows * D * 2);
+                tc::prefetch_l2(args.v + row0 * D, rows * D * 2);
+                tc::prefetch_l2(args.dO + row0 * D, rows * D * 2);
+                tc::prefetch_l2(args.g + row0 * D, rows * D * 4);
+                tc::prefetch_l2(args.SIN + z2 * D * D, D * D * 2);
+                tc::prefetch_l2(args.EE + z2 * D * D, D * D * 2);
+            }
             mbar_wait_bounded(full, 0, kWaitLimit);  // copies land before the CTA can leave
         } else if (warp == 1) {
             // ------------------------------ MMA issuer ------------------------------
@@ -795,7 +816,7 @@ gla_bwd_grad_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
             tc::tma_store_3d(&tm_dk, smem + GB_DO, 0, t0, bh);
             tc::tma_store_3d(&tm_dg, smem + GB_Q, 0, t0, bh);
             tc::bulk_commit();
-            tc::bulk_wait_all();
+            tc::bulk_wait_read();  // shared memory stays valid until the stores have read it
         }
     } else {
         asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(152));
@@ -866,7 +887,7 @@ gla_bwd_grad_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
         if (ok && stid == 0) {
             tc::tma_store_3d(&tm_dv, smem + GB_K, 0, t0, bh);
             tc::bulk_commit();
-            tc::bulk_wait_all();
+            tc::bulk_wait_read();
         }
     }
     tc::fence_before_sync();
@@ -899,6 +920,17 @@ size_t layout(int B, int H, int T, BwdArgs* a, void* ws) {
     return off;
 }
 
+int sm_count() {
+    static int sms = 0;
+    if (sms == 0) {
+        int dev = 0;
+        if (cudaGetDevice(&dev) != cudaSuccess ||
+            cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || sms < 1)
+            sms = 148;
+    }
+    return sms;
+}
+
 }  // namespace
 
 bool gla_backward_tc_supported(int dk, int dv) { return dk == D && dv == D; }
@@ -918,6 +950,12 @@ cudaError_t gla_backward_tc_launch(const GlaBackwardArgs& g, cudaStream_t stream
     a.state0 = g.state0;
     a.dstate_final = g.dstate_final;
     a.dstate0 = g.dstate0;
+    a.q = static_cast<const __nv_bfloat16*>(g.q);
+    a.k = static_cast<const __nv_bfloat16*>(g.k);
+    a.v = static_cast<const __nv_bfloat16*>(g.v);
+    a.dO = static_cast<const __nv_bfloat16*>(g.dO);
+    a.g = g.g;
+    a.wave = sm_count();
     const int NC = a.NC;
     if ((int64_t)NC * BH > 0x7fffffff) return cudaErrorInvalidConfiguration;
     CUtensorMap mq, mk, mv, mdo, mg, msin, me, mdq, mdk, mdv, mdg, mu, mu2;
