@@ -598,7 +598,7 @@ def run_backward(rod, torch, wl, dev, H, d, W, seed_base, barrier, reduce_max, w
                                                        ["gla_backward_tc.cu", "tc.cuh", "common.cuh"]),
                            "note": "chunkwise tensor-core backward (contributions, scans, gradients); "
                                    "its workspace traffic (per-chunk states and contributions) is "
-                                   "about 3.7x the algorithmic bytes"}
+                                   "about 3.5x the algorithmic bytes"}
     del q, k, v, g, dO, S0, dSf, ws
     # SW-SKA: B1 H16 T8192, window W, d 128; algorithmic work 10 d FLOP per (query, key, head)
     # pair inside the window: the five products S = Q K^T, dP = dO V^T, dV = P^T dO,
