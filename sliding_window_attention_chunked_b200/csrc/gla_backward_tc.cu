@@ -700,22 +700,33 @@ gla_bwd_grad_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                     tc::tmem_ld32(xa + 32u * hh, ra_);
                     tc::tmem_ld32(xb + 32u * hh, rb_);
                     tc::tmem_wait_ld();
+                    // eight tokens' operands and gates are loaded ahead of their arithmetic: the
+                    // compiler cannot move a shared-memory load above the previous token's
+                    // shared-memory stores, so a load per token would pay its latency every token
 #pragma unroll
-                    for (int i = 31; i >= 0; --i) {
-                        const int t = 32 * hh + i;
-                        const float x_a = __uint_as_float(ra_[i]), x_b = __uint_as_float(rb_[i]);
-                        if (half == 0) {
-                            const float qt = ldbf(smem + GB_Q + sw_off_elem(t, c, C));
-                            stq[t * D + c] = __float2bfloat16_rn((x_a + x_b) * (ac * rcp(F)));
-                            acc1 = fmaf(qt, x_a + x_b, acc1);
-                            T1[t * D + c] = acc1;
-                        } else {
-                            const float kt = ldbf(smem + GB_KT + sw_off_elem(t, c, C));
-                            stk[t * D + c] = __float2bfloat16_rn(fmaf(ac, x_b, x_a) * (F * ra));
-                            acc3 = fmaf(kt, x_a, acc3);
-                            T2[t * D + c] = -acc3;
+                    for (int i0 = 24; i0 >= 0; i0 -= 8) {
+                        float opv[8], gv[8];
+#pragma unroll
+                        for (int j = 0; j < 8; ++j) {
+                            const int t = 32 * hh + i0 + j;
+                            opv[j] = ldbf(smem + (half == 0 ? GB_Q : GB_KT) + sw_off_elem(t, c, C));
+                            gv[j] = t < nvalid ? gcol[t * D] : 1.f;
                         }
-                        F *= t < nvalid ? gcol[t * D] : 1.f;
+#pragma unroll
+                        for (int j = 7; j >= 0; --j) {
+                            const int i = i0 + j, t = 32 * hh + i;
+                            const float x_a = __uint_as_float(ra_[i]), x_b = __uint_as_float(rb_[i]);
+                            if (half == 0) {
+                                stq[t * D + c] = __float2bfloat16_rn((x_a + x_b) * (ac * rcp(F)));
+                                acc1 = fmaf(opv[j], x_a + x_b, acc1);
+                                T1[t * D + c] = acc1;
+                            } else {
+                                stk[t * D + c] = __float2bfloat16_rn(fmaf(ac, x_b, x_a) * (F * ra));
+                                acc3 = fmaf(opv[j], x_a, acc3);
+                                T2[t * D + c] = -acc3;
+                            }
+                            F *= gv[j];
+                        }
                     }
                 }
                 if (half == 1) {
@@ -726,10 +737,20 @@ gla_bwd_grad_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                         tc::tmem_ld32(xb + 32u * hh, rb_);
                         tc::tmem_wait_ld();
 #pragma unroll
-                        for (int i = 0; i < 32; ++i) {
-                            const int t = 32 * hh + i;
-                            T2[t * D + c] = fmaf(ac, ex, T2[t * D + c]);
-                            ex = fmaf(ldbf(smem + GB_KT + sw_off_elem(t, c, C)), __uint_as_float(rb_[i]), ex);
+                        for (int i0 = 0; i0 < 32; i0 += 8) {
+                            float t2v[8], kv[8];
+#pragma unroll
+                            for (int j = 0; j < 8; ++j) {
+                                const int t = 32 * hh + i0 + j;
+                                t2v[j] = T2[t * D + c];
+                                kv[j] = ldbf(smem + GB_KT + sw_off_elem(t, c, C));
+                            }
+#pragma unroll
+                            for (int j = 0; j < 8; ++j) {
+                                const int t = 32 * hh + i0 + j;
+                                T2[t * D + c] = fmaf(ac, ex, t2v[j]);
+                                ex = fmaf(kv[j], __uint_as_float(rb_[i0 + j]), ex);
+                            }
                         }
                     }
                 }
@@ -802,11 +823,22 @@ gla_bwd_grad_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
             // dg[t][c] = (T1 + T2 + a rho) / g_t on the product route, T1 + T2 on the exact one;
             // the 256 threads split the tokens: WG1 rows 0-31, WG2 rows 32-63
             float* dgst = reinterpret_cast<float*>(smem + GB_Q);
-            for (int i = 0; i < 32; ++i) {
-                const int t = 32 * half + i;
-                float v = T1[t * D + c] + T2[t * D + c];
-                if (fast) v = (v + ac * rho[c]) * (t < nvalid ? rcp(gcol[t * D]) : 1.f);
-                dgst[t * D + c] = v;
+            const float rhoc = rho[c];
+            for (int i0 = 0; i0 < 32; i0 += 8) {
+                float sv[8], gv[8];
+#pragma unroll
+                for (int j = 0; j < 8; ++j) {
+                    const int t = 32 * half + i0 + j;
+                    sv[j] = T1[t * D + c] + T2[t * D + c];
+                    gv[j] = gcol[t * D];
+                }
+#pragma unroll
+                for (int j = 0; j < 8; ++j) {
+                    const int t = 32 * half + i0 + j;
+                    float v = sv[j];
+                    if (fast) v = (v + ac * rhoc) * (t < nvalid ? rcp(gv[j]) : 1.f);
+                    dgst[t * D + c] = v;
+                }
             }
         }
         tc::fence_proxy_async();
