@@ -231,3 +231,83 @@ def test_planted_mistakes_are_caught(mistake):
         except AssertionError:
             caught += 1
     assert caught > 0, f"{mistake} never caught in 300 schedules"
+
+
+# ------------------------------------------------------------------------------------------------
+# The contributions kernel (gla_bwd_contrib_kernel): each warp moves its 32 TMEM rows of U or U'
+# out in four 32 x 32 fp32 tiles through two shared-memory buffers laid over the spent operand
+# tiles. Before it writes a buffer the third time or later, the lane that issues the stores waits
+# until all but its most recent bulk store have read shared memory (wait_group.read 1); before
+# the CTA leaves, until all have (wait_group.read 0).
+# ------------------------------------------------------------------------------------------------
+def run_contrib(seed, mistake=None, warps=8, tiles=4):
+    mma = Bar(1)
+    tile_read = [[Bar(1) for _ in range(tiles)] for _ in range(warps)]
+    end = Bar(warps + 1)
+    operands = {"read_by_mma": False}
+    buf = {}         # (warp, buffer) -> (tile staged there, read by its store yet)
+    out = set()
+    pipe, copies = [], []
+
+    def execute(op):
+        if op[0] == "C":
+            op[1].arrive()
+        else:
+            operands["read_by_mma"] = True
+
+    def land(copy):
+        w, t, b = copy
+        staged, _ = buf[(w, b)]
+        assert staged == t, f"warp {w}: store of tile {t} read buffer {b} holding tile {staged}"
+        buf[(w, b)] = (t, True)
+        out.add((w, t))
+        tile_read[w][t].arrive()
+
+    def issuer():
+        pipe.extend([("M", "U"), ("M", "U2"), ("C", mma)])
+        yield ("step",)
+        parity = end.phase & 1
+        end.arrive()
+        yield ("wait", end, parity)
+
+    def warp(w):
+        yield ("wait", mma, 0)
+        for t in range(tiles):
+            b = t % 2
+            if t >= 2 and mistake != "no_read_wait":
+                # wait_group.read 1: every store but the newest has read shared memory
+                for u in range(t - 1):
+                    yield ("wait", tile_read[w][u], 0)
+            assert operands["read_by_mma"], "staging written over operands the MMAs still read"
+            if (w, b) in buf:
+                assert buf[(w, b)][1], f"warp {w}: buffer {b} rewritten before its store read it"
+            buf[(w, b)] = (t, False)
+            yield ("step",)
+            copies.append((w, t, b))
+        for u in range(tiles):  # wait_group.read 0 before the CTA leaves
+            yield ("wait", tile_read[w][u], 0)
+        assert all(buf[(w, b)][1] for b in range(2)), "CTA left before its stores read"
+        parity = end.phase & 1
+        end.arrive()
+        yield ("wait", end, parity)
+
+    actors = {"issuer": issuer()}
+    actors.update({f"w{w}": warp(w) for w in range(warps)})
+    simulate(seed, actors, [pipe], copies, execute, land)
+    assert out == {(w, t) for w in range(warps) for t in range(tiles)}, "a tile was never stored"
+
+
+@pytest.mark.parametrize("seed", range(200))
+def test_contributions_staging_protocol_holds(seed):
+    run_contrib(seed)
+
+
+def test_contributions_staging_mistake_is_caught():
+    # with no wait before a buffer's reuse, some schedule rewrites it before its store read it
+    caught = 0
+    for seed in range(200):
+        try:
+            run_contrib(seed, "no_read_wait")
+        except AssertionError:
+            caught += 1
+    assert caught > 0
